@@ -1,0 +1,287 @@
+"""CPU oracle for the quantized-KV-cache hot path (test infrastructure).
+
+TEST INFRASTRUCTURE ONLY.  The test-suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are the only callers allowed; the product
+library never imports, links or runs anything here, and this package never
+imports the product library.  The arithmetic lives in ``kvq_oracle.c`` (plain
+C, built with ``-ffp-contract=off`` and no fast-math); this module only
+marshals numpy arrays and loops over (sequence, KV head) pairs.
+
+Every function cites the page passage it follows; the readings taken where
+the pages are silent are listed at the top of ``kvq_oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvq_oracle.c")
+_LIB = os.path.join(_HERE, "libkvq_oracle.so")
+
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+          "-fexcess-precision=standard", "-fPIC", "-shared"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``kvq_oracle.c`` into ``libkvq_oracle.so`` with gcc."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, u64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_double
+        lib.kvqo_f32_to_f16.argtypes = [ctypes.c_float]
+        lib.kvqo_f32_to_f16.restype = ctypes.c_uint16
+        lib.kvqo_f16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.kvqo_f16_to_f32.restype = ctypes.c_float
+        lib.kvqo_f32_to_f16_up.argtypes = [ctypes.c_float]
+        lib.kvqo_f32_to_f16_up.restype = ctypes.c_uint16
+        lib.kvqo_f32_to_f16_array.argtypes = [P, i64, P]
+        lib.kvqo_f16_to_f32_array.argtypes = [P, i64, P]
+        lib.kvqo_quantize_group.argtypes = [P, i32, i32, P, P, P]
+        lib.kvqo_quantize_rows.argtypes = [P, i64, i32, i32, i32, P, P]
+        lib.kvqo_dequantize_rows.argtypes = [P, P, i64, i32, i32, i32, P]
+        lib.kvqo_attention.argtypes = [P, i32, P, P, i64, i32, f64, P, P]
+        lib.kvqo_attention_blocks.argtypes = [P, i32, P, P, i32, f64, P, i32, P, P]
+        lib.kvqo_attention_packed.argtypes = [P, i32, i32, P, P, i32, P, P, i32, i32,
+                                              i64, i32, f64, P, P]
+        lib.kvqo_chunk_assign.argtypes = [P, P, i32, i32, f64, f64, P, P]
+        lib.kvqo_chunk_partition.argtypes = [P, i32, P, P]
+        lib.kvqo_kv_elements.argtypes = [u64, u64, u64, u64, u64]
+        lib.kvqo_kv_elements.restype = u64
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def _c(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# --------------------------------------------------------------------------
+# binary16 codec (IEEE 754 binary16, round to nearest even)
+# --------------------------------------------------------------------------
+
+def f32_to_f16_bits(x) -> np.ndarray:
+    """fp32 values -> binary16 bit patterns (uint16), ties to even."""
+    lib = _load()
+    x = _c(x, np.float32)
+    out = np.zeros(x.shape, np.uint16)
+    lib.kvqo_f32_to_f16_array(_p(x), x.size, _p(out))
+    return out
+
+
+def f32_to_f16_bits_up(x) -> np.ndarray:
+    """positive fp32 values -> smallest binary16 value not below them."""
+    lib = _load()
+    x = _c(x, np.float32).ravel()
+    return np.array([lib.kvqo_f32_to_f16_up(float(v)) for v in x], np.uint16)
+
+
+def f16_bits_to_f32(h) -> np.ndarray:
+    lib = _load()
+    h = _c(h, np.uint16)
+    out = np.zeros(h.shape, np.float32)
+    lib.kvqo_f16_to_f32_array(_p(h), h.size, _p(out))
+    return out
+
+
+# --------------------------------------------------------------------------
+# group quantization (Cocktail page 3.2.2; static-quantization page 2.1)
+# --------------------------------------------------------------------------
+
+def quantize_group(x16, bits: int):
+    """One group of fp16 bit patterns -> (codes uint8[G], s16, z16)."""
+    lib = _load()
+    x16 = _c(x16, np.uint16)
+    G = x16.size
+    code = np.zeros(G, np.uint8)
+    s = np.zeros(1, np.uint16)
+    z = np.zeros(1, np.uint16)
+    lib.kvqo_quantize_group(_p(x16), G, bits, _p(code), _p(s), _p(z))
+    return code, int(s[0]), int(z[0])
+
+
+def quantize_rows(x16, group: int, bits: int):
+    """Token rows [N, D] of fp16 bit patterns -> (codes [N, D*bits/8] uint8,
+    meta [N, D/G, 2] uint16 holding the (scale, zero) fp16 patterns)."""
+    lib = _load()
+    x16 = _c(x16, np.uint16)
+    N, D = x16.shape
+    codes = np.zeros((N, D * bits // 8), np.uint8)
+    ng = D // group if bits != 16 else 1
+    meta = np.zeros((N, ng, 2), np.uint16)
+    lib.kvqo_quantize_rows(_p(x16), N, D, group, bits, _p(codes), _p(meta))
+    return codes, meta
+
+
+def dequantize_rows(codes, meta, D: int, group: int, bits: int) -> np.ndarray:
+    """Packed rows -> fp64 [N, D], x_hat = (c - z) * s (exact in fp64)."""
+    lib = _load()
+    codes = _c(codes, np.uint8)
+    N = codes.shape[0]
+    meta = _c(meta if meta is not None else np.zeros((N, 1, 2), np.uint16), np.uint16)
+    out = np.zeros((N, D), np.float64)
+    lib.kvqo_dequantize_rows(_p(codes), _p(meta), N, D, group if bits != 16 else D, bits,
+                             _p(out))
+    return out
+
+
+# --------------------------------------------------------------------------
+# fp64 attention (score definition: KVO-LLM page 3.2; chunked + merge:
+# Cocktail page 3.2.3)
+# --------------------------------------------------------------------------
+
+def attention(q, K, V, scale: float):
+    """q [g, D], K/V [L, D] fp64 -> (o [g, D], lse [g]) in fp64."""
+    lib = _load()
+    q = _c(q, np.float64)
+    K = _c(K, np.float64)
+    V = _c(V, np.float64)
+    g, D = q.shape
+    L = K.shape[0]
+    o = np.zeros((g, D), np.float64)
+    lse = np.zeros(g, np.float64)
+    lib.kvqo_attention(_p(q), g, _p(K), _p(V), L, D, float(scale), _p(o), _p(lse))
+    return o, lse
+
+
+def attention_blocks(q, K, V, scale: float, bounds: Sequence[int]):
+    """Block-wise attention merged by log-sum-exp; bounds = [0, ..., L]."""
+    lib = _load()
+    q = _c(q, np.float64)
+    K = _c(K, np.float64)
+    V = _c(V, np.float64)
+    g, D = q.shape
+    b = _c(bounds, np.int64)
+    o = np.zeros((g, D), np.float64)
+    lse = np.zeros(g, np.float64)
+    lib.kvqo_attention_blocks(_p(q), g, _p(K), _p(V), D, float(scale), _p(b), b.size - 1,
+                              _p(o), _p(lse))
+    return o, lse
+
+
+def attention_packed(q16, q_is_bf16: bool, k_codes, k_meta, k_bits: int, v_codes, v_meta,
+                     v_bits: int, group: int, L: int, scale: float):
+    """Attention of g query heads over one packed (sequence, KV head) cache."""
+    lib = _load()
+    q16 = _c(q16, np.uint16)
+    g, D = q16.shape
+    kc = _c(k_codes, np.uint8)
+    vc = _c(v_codes, np.uint8)
+    km = _c(k_meta, np.uint16) if k_bits != 16 else np.zeros(1, np.uint16)
+    vm = _c(v_meta, np.uint16) if v_bits != 16 else np.zeros(1, np.uint16)
+    o = np.zeros((g, D), np.float64)
+    lse = np.zeros(g, np.float64)
+    lib.kvqo_attention_packed(_p(q16), int(bool(q_is_bf16)), g, _p(kc), _p(km), k_bits,
+                              _p(vc), _p(vm), v_bits, group, L, D, float(scale), _p(o),
+                              _p(lse))
+    return o, lse
+
+
+# --------------------------------------------------------------------------
+# Cocktail chunk search and reorder (Cocktail page 3.1.1, 3.1.2)
+# --------------------------------------------------------------------------
+
+def chunk_assign(emb, qemb, alpha: float, beta: float):
+    """emb [n, E] fp32, qemb [E] fp32 -> (sim fp64 [n], class uint8 [n])."""
+    lib = _load()
+    emb = _c(emb, np.float32)
+    qemb = _c(qemb, np.float32)
+    n, E = emb.shape
+    sim = np.zeros(n, np.float64)
+    bits = np.zeros(n, np.uint8)
+    lib.kvqo_chunk_assign(_p(emb), _p(qemb), n, E, float(alpha), float(beta), _p(sim),
+                          _p(bits))
+    return sim, bits
+
+
+def chunk_partition(bits):
+    """class per chunk -> (perm int32 [n], counts int32 [3] for FP16/INT4/INT2)."""
+    lib = _load()
+    bits = _c(bits, np.uint8)
+    perm = np.zeros(bits.size, np.int32)
+    counts = np.zeros(3, np.int32)
+    lib.kvqo_chunk_partition(_p(bits), bits.size, _p(perm), _p(counts))
+    return perm, counts
+
+
+def kv_elements(layers: int, kv_heads: int, head_dim: int, seq_len: int, batch: int) -> int:
+    """2 * layers * kv_heads * head_dim * seq_len * batch (KV-cache size page)."""
+    return int(_load().kvqo_kv_elements(layers, kv_heads, head_dim, seq_len, batch))
+
+
+# --------------------------------------------------------------------------
+# Whole-cache helpers built from the functions above
+# --------------------------------------------------------------------------
+
+def quantize_cache(x16, group: int, bits: int):
+    """x16 [..., T, D] fp16 patterns -> codes [..., T, D*bits/8], meta [..., T, D/G, 2]."""
+    x16 = _c(x16, np.uint16)
+    lead = x16.shape[:-1]
+    D = x16.shape[-1]
+    codes, meta = quantize_rows(x16.reshape(-1, D), group, bits)
+    return codes.reshape(*lead, -1), meta.reshape(*lead, meta.shape[-2], 2)
+
+
+def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: float,
+                     pairs=None):
+    """Decode attention of every query head over one or more packed segments.
+
+    q16: [B, Hq, D] fp16/bf16 patterns.  segments: list of dicts with numpy
+    arrays ``k_codes``/``v_codes`` [B, Hkv, T, row_bytes], ``k_meta``/``v_meta``
+    [B, Hkv, T, D/G, 2] (None for bits 16), ``bits``, ``group``.
+    seq_lens_per_seg: list of int arrays [B].  The segments of a sequence are
+    concatenated in token order (attention does not depend on the order).
+    pairs: optional list of (b, kv_head) to evaluate; others stay NaN.
+    Returns (o [B, Hq, D] fp64, lse [B, Hq] fp64).
+    """
+    q16 = _c(q16, np.uint16)
+    B, Hq, D = q16.shape
+    Hkv = segments[0]["k_codes"].shape[1]
+    g = Hq // Hkv
+    o = np.full((B, Hq, D), np.nan)
+    lse = np.full((B, Hq), np.nan)
+    if pairs is None:
+        pairs = [(b, h) for b in range(B) for h in range(Hkv)]
+    for b, h in pairs:
+        Ks, Vs = [], []
+        for seg, lens in zip(segments, seq_lens_per_seg):
+            L = int(lens[b])
+            bits, G = seg["bits"], seg["group"]
+            km = seg["k_meta"][b, h, :L] if bits != 16 else None
+            vm = seg["v_meta"][b, h, :L] if bits != 16 else None
+            Ks.append(dequantize_rows(seg["k_codes"][b, h, :L], km, D, G, bits))
+            Vs.append(dequantize_rows(seg["v_codes"][b, h, :L], vm, D, G, bits))
+        K = np.concatenate(Ks, 0)
+        V = np.concatenate(Vs, 0)
+        qh = q16[b, h * g:(h + 1) * g]
+        qd = (bf16_bits_to_f64(qh) if q_is_bf16 else f16_bits_to_f32(qh).astype(np.float64)
+              ).reshape(g, D)
+        ob, lb = attention(qd, K, V, scale)
+        o[b, h * g:(h + 1) * g] = ob
+        lse[b, h * g:(h + 1) * g] = lb
+    return o, lse
+
+
+def bf16_bits_to_f64(h) -> np.ndarray:
+    """bfloat16 bit patterns -> fp64 (exact: the pattern is the top half of fp32)."""
+    h = _c(h, np.uint16)
+    return (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

@@ -1,0 +1,492 @@
+/*
+ * kvq_oracle.c -- plain CPU oracle for the quantized-KV-cache hot path.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test-suite, the smoke
+ * check and the CPU-baseline leg of the benchmark may load this file's
+ * library.  It shares no code, header, table or constant generator with the
+ * CUDA library; it is written straight from the pages it cites, in their
+ * notation, with no blocking, fusion or reordering.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC
+ * (no FMA contraction, no fast-math: every fp32 operation below is one IEEE
+ * operation rounded to nearest-even, in the order written).
+ *
+ * Sources (page title, section):
+ *   [P1] "大模型KV缓存量化技术：原理、优化与实践", section 2.1 (static global
+ *        quantization: scale = (max - min) / (2^bits - 1)).
+ *   [P2] "大模型推理加速之KV Cache量化压缩原理与工程实现": the KV-cache size
+ *        formula (2 * layers * kv_heads * head_dim * seq_len * batch * bytes);
+ *        "常见问题排查" (scale clamped to at least 1e-5); INT4 asymmetric
+ *        group quantization with group_size 128 or 64.
+ *   [P3] "长上下文LLM推理中的KV Cache优化技术解析", section 3.2
+ *        (score = q . k^T / sqrt(dim)).
+ *   [P4] Cocktail page (peacm.com news 1099647): 3.1.1 (chunk search: cosine
+ *        similarity, T_low / T_high from alpha and beta, FP16 / INT4 / INT2);
+ *        3.1.2 (reorder chunks so equal bit-widths are contiguous);
+ *        3.2.2 (group quantization quant(x) = round(x/s) + z);
+ *        3.2.3 (chunked attention, merged, equal to unchunked attention).
+ *   [P5] TurboQuant page (bhfrc.com news 57821): 1.2 (KV element count
+ *        worked example); 2.3 (per-group scaling, dequantization inside
+ *        the attention matmul).
+ *
+ * Readings taken where the pages are silent (each one also listed in the
+ * design notes):
+ *   R1  "round" is round-half-to-even (rintf in the default rounding mode).
+ *   R2  The 1e-5 scale floor is applied in fp32 before s is stored in fp16,
+ *       and s is stored rounded toward +infinity (the smallest fp16 value
+ *       not below the fp32 scale): then the stored grid still spans
+ *       [min, max] in 2^b - 1 steps and every element keeps |x - x_hat|
+ *       <= s/2.  Rounding s to nearest could shrink it and push the
+ *       group's maximum one code past 2^b - 1.
+ *   R3  Quantization divides by the stored fp16 scale, not the fp32 one.
+ *   R4  z = rint(-min / s), clamped to the fp16 range, stored as fp16, NOT
+ *       clamped to [0, qmax]; a zero-point of -0 is stored as +0.
+ *   R5  quant(x) rounds x/s first and then adds the integer z; the result is
+ *       clamped to [0, qmax].
+ *   R6  Groups run along head_dim within one token row.
+ *   R7  Codes are packed little-endian inside bytes: element j of a row sits
+ *       in byte floor(j*b/8) at bit offset (j*b) mod 8.
+ *   R8  Cocktail's garbled threshold rule reads: sim > T_high -> FP16,
+ *       T_low < sim <= T_high -> INT4, sim <= T_low -> INT2; s_min and s_max
+ *       are taken over the chunks of one sequence; all in fp64.
+ *   R9  Reorder order: FP16 chunks, then INT4, then INT2, each class in
+ *       ascending original chunk index.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* IEEE 754 binary16 <-> binary32, written from the format definition.      */
+/* ------------------------------------------------------------------------ */
+
+/* Round an fp32 value to the nearest binary16 value, ties to even. */
+uint16_t kvqo_f32_to_f16(float f)
+{
+    uint32_t x;
+    memcpy(&x, &f, sizeof x);
+    uint32_t sign = (x >> 16) & 0x8000u;
+    uint32_t exp8 = (x >> 23) & 0xffu;
+    uint32_t frac = x & 0x7fffffu;
+
+    if (exp8 == 0xffu) /* infinity or NaN */
+        return (uint16_t)(sign | 0x7c00u | (frac ? 0x0200u : 0u));
+
+    int32_t e = (int32_t)exp8 - 127; /* unbiased exponent */
+    if (e >= 16)                     /* |f| >= 2^16: beyond the largest finite */
+        return (uint16_t)(sign | 0x7c00u);
+
+    if (e >= -14) {
+        /* normal binary16 range: keep 10 fraction bits, round the other 13 */
+        uint32_t h = ((uint32_t)(e + 15) << 10) | (frac >> 13);
+        uint32_t rest = frac & 0x1fffu;
+        if (rest > 0x1000u || (rest == 0x1000u && (h & 1u)))
+            h += 1u; /* a carry into the exponent is the correct result */
+        return (uint16_t)(sign | h);
+    }
+
+    /* subnormal binary16: value = m * 2^-24, m in [0, 1023] */
+    if (exp8 == 0u)
+        return (uint16_t)sign; /* fp32 subnormals are far below 2^-25 */
+    uint32_t full = frac | 0x800000u; /* value = full * 2^(e - 23) */
+    int32_t shift = -e - 1;           /* m = full * 2^(e + 1), i.e. >> (-e-1) */
+    if (shift > 24)
+        return (uint16_t)sign; /* below half of the smallest subnormal */
+    uint32_t m = full >> shift;
+    uint32_t rest = full & ((1u << shift) - 1u);
+    uint32_t half = 1u << (shift - 1);
+    if (rest > half || (rest == half && (m & 1u)))
+        m += 1u;
+    return (uint16_t)(sign | m);
+}
+
+float kvqo_f16_to_f32(uint16_t h);
+
+/* Round a positive finite fp32 value up to the nearest binary16 value
+ * (the smallest binary16 value >= f). */
+uint16_t kvqo_f32_to_f16_up(float f)
+{
+    uint16_t h = kvqo_f32_to_f16(f);
+    if (kvqo_f16_to_f32(h) < f)
+        h = (uint16_t)(h + 1u); /* next binary16 value above */
+    return h;
+}
+
+float kvqo_f16_to_f32(uint16_t h)
+{
+    uint32_t exp5 = (h >> 10) & 0x1fu;
+    uint32_t frac = h & 0x3ffu;
+    float v;
+    if (exp5 == 0u)
+        v = ldexpf((float)frac, -24);
+    else if (exp5 == 31u)
+        v = frac ? NAN : INFINITY;
+    else
+        v = ldexpf((float)(1024u + frac), (int)exp5 - 25);
+    return (h & 0x8000u) ? -v : v;
+}
+
+void kvqo_f32_to_f16_array(const float *x, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = kvqo_f32_to_f16(x[i]);
+}
+
+void kvqo_f16_to_f32_array(const uint16_t *h, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = kvqo_f16_to_f32(h[i]);
+}
+
+float kvqo_bf16_to_f32(uint16_t h)
+{
+    uint32_t x = (uint32_t)h << 16;
+    float v;
+    memcpy(&v, &x, sizeof v);
+    return v;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Group-wise asymmetric quantization ([P4] 3.2.2, [P1] 2.1, [P2], [P5] 2.3) */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Quantize one group x[0..G-1] (binary16 bit patterns) to `bits`-bit codes.
+ * Writes the G unpacked codes, and the fp16 bit patterns of s and z.
+ */
+void kvqo_quantize_group(const uint16_t *x, int G, int bits,
+                         uint8_t *code, uint16_t *s_out, uint16_t *z_out)
+{
+    const float qmax = (float)((1 << bits) - 1);
+
+    /* min and max of the group, in fp32 (exact for fp16 inputs) */
+    float mn = kvqo_f16_to_f32(x[0]);
+    float mx = mn;
+    for (int j = 1; j < G; ++j) {
+        float v = kvqo_f16_to_f32(x[j]);
+        if (v < mn)
+            mn = v;
+        if (v > mx)
+            mx = v;
+    }
+
+    /* scale = (max - min) / (2^bits - 1), floored at 1e-5, stored fp16 (R2) */
+    float s32 = (mx - mn) / qmax;
+    if (s32 < 1e-5f)
+        s32 = 1e-5f;
+    uint16_t s16 = kvqo_f32_to_f16_up(s32);
+    float s = kvqo_f16_to_f32(s16); /* R3: the stored scale is the one used */
+
+    /* zero point z = round(-min / s) (R1, R4) */
+    float zf = rintf(-mn / s) + 0.0f; /* + 0.0f turns -0 into +0 */
+    if (zf > 65504.0f)
+        zf = 65504.0f;
+    if (zf < -65504.0f)
+        zf = -65504.0f;
+    uint16_t z16 = kvqo_f32_to_f16(zf);
+    float z = kvqo_f16_to_f32(z16);
+
+    /* quant(x) = round(x / s) + z, clamped to the code range (R5) */
+    for (int j = 0; j < G; ++j) {
+        float c = rintf(kvqo_f16_to_f32(x[j]) / s) + z;
+        if (c < 0.0f)
+            c = 0.0f;
+        if (c > qmax)
+            c = qmax;
+        code[j] = (uint8_t)c;
+    }
+    *s_out = s16;
+    *z_out = z16;
+}
+
+/*
+ * Quantize n_rows token rows of D fp16 values, groups of G along the row
+ * (R6).  codes: [n_rows][D*bits/8] packed (R7); meta: [n_rows][D/G][2]
+ * binary16 (scale, zero).  bits == 16 stores the fp16 row unchanged and
+ * writes no meta (the FP16 class of [P4] 3.1.1).
+ */
+void kvqo_quantize_rows(const uint16_t *x, int64_t n_rows, int D, int G,
+                        int bits, uint8_t *codes, uint16_t *meta)
+{
+    const int64_t row_bytes = (int64_t)D * bits / 8;
+    uint8_t *tmp = (uint8_t *)malloc((size_t)G);
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint16_t *xr = x + r * D;
+        uint8_t *cr = codes + r * row_bytes;
+        if (bits == 16) {
+            memcpy(cr, xr, (size_t)row_bytes);
+            continue;
+        }
+        memset(cr, 0, (size_t)row_bytes);
+        for (int g = 0; g < D / G; ++g) {
+            uint16_t s16, z16;
+            kvqo_quantize_group(xr + g * G, G, bits, tmp, &s16, &z16);
+            meta[(r * (D / G) + g) * 2 + 0] = s16;
+            meta[(r * (D / G) + g) * 2 + 1] = z16;
+            for (int j = 0; j < G; ++j) {
+                int e = g * G + j; /* element index within the row */
+                int bitpos = e * bits;
+                cr[bitpos / 8] |= (uint8_t)(tmp[j] << (bitpos % 8));
+            }
+        }
+    }
+    free(tmp);
+}
+
+/* Unpack code e of a packed row (R7). */
+static unsigned kvqo_code_at(const uint8_t *row, int e, int bits)
+{
+    int bitpos = e * bits;
+    return (row[bitpos / 8] >> (bitpos % 8)) & ((1u << bits) - 1u);
+}
+
+/*
+ * Dequantize n_rows packed rows: x_hat = (c - z) * s, evaluated in fp64,
+ * where it is exact (|c - z| < 2^17 and s has 11 significant bits).
+ */
+void kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *meta,
+                          int64_t n_rows, int D, int G, int bits, double *out)
+{
+    const int64_t row_bytes = (int64_t)D * bits / 8;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint8_t *cr = codes + r * row_bytes;
+        for (int e = 0; e < D; ++e) {
+            if (bits == 16) {
+                uint16_t h = (uint16_t)(cr[2 * e] | (cr[2 * e + 1] << 8));
+                out[r * D + e] = (double)kvqo_f16_to_f32(h);
+                continue;
+            }
+            int g = e / G;
+            double s = (double)kvqo_f16_to_f32(meta[(r * (D / G) + g) * 2 + 0]);
+            double z = (double)kvqo_f16_to_f32(meta[(r * (D / G) + g) * 2 + 1]);
+            double c = (double)kvqo_code_at(cr, e, bits);
+            out[r * D + e] = (c - z) * s;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention in fp64 ([P3] 3.2 score; [P4] 3.2.3 chunked + merge)    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One KV head serving g query heads.  q: [g][D], K, V: [L][D] (dequantized),
+ * all fp64.  For each head: score_t = scale * sum_j q_j K_tj;
+ * p = softmax(score) with the max subtracted; o = sum_t p_t V_t;
+ * lse = log sum_t exp(score_t).  L == 0 gives o = 0, lse = -inf.
+ */
+void kvqo_attention(const double *q, int g, const double *K, const double *V,
+                    int64_t L, int D, double scale, double *o, double *lse)
+{
+    double *score = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
+    for (int h = 0; h < g; ++h) {
+        const double *qh = q + (int64_t)h * D;
+        double *oh = o + (int64_t)h * D;
+        for (int j = 0; j < D; ++j)
+            oh[j] = 0.0;
+        if (L == 0) {
+            lse[h] = -INFINITY;
+            continue;
+        }
+        double m = -INFINITY;
+        for (int64_t t = 0; t < L; ++t) {
+            double acc = 0.0;
+            for (int j = 0; j < D; ++j)
+                acc += qh[j] * K[t * D + j];
+            score[t] = scale * acc;
+            if (score[t] > m)
+                m = score[t];
+        }
+        double l = 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            double p = exp(score[t] - m);
+            l += p;
+            for (int j = 0; j < D; ++j)
+                oh[j] += p * V[t * D + j];
+        }
+        for (int j = 0; j < D; ++j)
+            oh[j] /= l;
+        lse[h] = m + log(l);
+    }
+    free(score);
+}
+
+/*
+ * The same attention computed block by block and merged by log-sum-exp:
+ * tokens are cut at bounds[0] = 0 < bounds[1] < ... < bounds[n_blocks] = L.
+ * Block b keeps its own max m_b, sum l_b = sum exp(score - m_b) and
+ * unnormalised output u_b = sum exp(score - m_b) V.  The merge takes
+ * M = max m_b, l = sum exp(m_b - M) l_b, o = sum exp(m_b - M) u_b / l,
+ * lse = M + log l.  Empty blocks contribute nothing.
+ */
+void kvqo_attention_blocks(const double *q, int g, const double *K,
+                           const double *V, int D, double scale,
+                           const int64_t *bounds, int n_blocks, double *o,
+                           double *lse)
+{
+    double *mb = (double *)malloc((size_t)n_blocks * sizeof(double));
+    double *lb = (double *)malloc((size_t)n_blocks * sizeof(double));
+    double *ub = (double *)malloc((size_t)n_blocks * D * sizeof(double));
+    for (int h = 0; h < g; ++h) {
+        const double *qh = q + (int64_t)h * D;
+        for (int b = 0; b < n_blocks; ++b) {
+            int64_t t0 = bounds[b], t1 = bounds[b + 1];
+            double m = -INFINITY;
+            for (int64_t t = t0; t < t1; ++t) {
+                double acc = 0.0;
+                for (int j = 0; j < D; ++j)
+                    acc += qh[j] * K[t * D + j];
+                if (scale * acc > m)
+                    m = scale * acc;
+            }
+            double l = 0.0;
+            for (int j = 0; j < D; ++j)
+                ub[b * D + j] = 0.0;
+            for (int64_t t = t0; t < t1; ++t) {
+                double acc = 0.0;
+                for (int j = 0; j < D; ++j)
+                    acc += qh[j] * K[t * D + j];
+                double p = exp(scale * acc - m);
+                l += p;
+                for (int j = 0; j < D; ++j)
+                    ub[b * D + j] += p * V[t * D + j];
+            }
+            mb[b] = m;
+            lb[b] = l;
+        }
+        double M = -INFINITY;
+        for (int b = 0; b < n_blocks; ++b)
+            if (lb[b] > 0.0 && mb[b] > M)
+                M = mb[b];
+        double l = 0.0;
+        double *oh = o + (int64_t)h * D;
+        for (int j = 0; j < D; ++j)
+            oh[j] = 0.0;
+        for (int b = 0; b < n_blocks; ++b) {
+            if (lb[b] == 0.0)
+                continue;
+            double w = exp(mb[b] - M);
+            l += w * lb[b];
+            for (int j = 0; j < D; ++j)
+                oh[j] += w * ub[b * D + j];
+        }
+        if (l == 0.0) {
+            lse[h] = -INFINITY;
+            continue;
+        }
+        for (int j = 0; j < D; ++j)
+            oh[j] /= l;
+        lse[h] = M + log(l);
+    }
+    free(mb);
+    free(lb);
+    free(ub);
+}
+
+/*
+ * Decode attention straight from a packed cache of one (sequence, KV head):
+ * each token row is dequantized ((c - z) * s in fp64) as it is read, then
+ * the fp64 attention above is applied.  q16: [g][D] binary16 or bfloat16
+ * bit patterns (q_is_bf16).
+ */
+void kvqo_attention_packed(const uint16_t *q16, int q_is_bf16, int g,
+                           const uint8_t *k_codes, const uint16_t *k_meta,
+                           int k_bits, const uint8_t *v_codes,
+                           const uint16_t *v_meta, int v_bits, int G,
+                           int64_t L, int D, double scale, double *o,
+                           double *lse)
+{
+    double *q = (double *)malloc((size_t)g * D * sizeof(double));
+    for (int64_t i = 0; i < (int64_t)g * D; ++i)
+        q[i] = q_is_bf16 ? (double)kvqo_bf16_to_f32(q16[i])
+                         : (double)kvqo_f16_to_f32(q16[i]);
+    double *K = (double *)malloc((size_t)(L > 0 ? L : 1) * D * sizeof(double));
+    double *V = (double *)malloc((size_t)(L > 0 ? L : 1) * D * sizeof(double));
+    int Gk = (k_bits == 16) ? D : G;
+    int Gv = (v_bits == 16) ? D : G;
+    kvqo_dequantize_rows(k_codes, k_meta, L, D, Gk, k_bits, K);
+    kvqo_dequantize_rows(v_codes, v_meta, L, D, Gv, v_bits, V);
+    kvqo_attention(q, g, K, V, L, D, scale, o, lse);
+    free(q);
+    free(K);
+    free(V);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Cocktail chunk-level bit-width search and reorder ([P4] 3.1.1, 3.1.2)   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * sim(q, c_i) = (q . c_i) / (||q|| * ||c_i||) in fp64, every sum taken in
+ * index order with separate multiply and add.  T_low = s_min + (s_max -
+ * s_min) * alpha, T_high = s_max - (s_max - s_min) * beta.  Class (R8):
+ * 16 (FP16) if sim > T_high, 4 (INT4) if T_low < sim <= T_high, else 2.
+ */
+void kvqo_chunk_assign(const float *emb, const float *qemb, int n_chunks,
+                       int dim, double alpha, double beta, double *sim,
+                       uint8_t *bits_out)
+{
+    double qq = 0.0;
+    for (int d = 0; d < dim; ++d)
+        qq += (double)qemb[d] * (double)qemb[d];
+    double nq = sqrt(qq);
+    double s_min = INFINITY, s_max = -INFINITY;
+    for (int i = 0; i < n_chunks; ++i) {
+        const float *c = emb + (int64_t)i * dim;
+        double dot = 0.0, cc = 0.0;
+        for (int d = 0; d < dim; ++d) {
+            dot += (double)qemb[d] * (double)c[d];
+            cc += (double)c[d] * (double)c[d];
+        }
+        sim[i] = dot / (nq * sqrt(cc));
+        if (sim[i] < s_min)
+            s_min = sim[i];
+        if (sim[i] > s_max)
+            s_max = sim[i];
+    }
+    double span = s_max - s_min;
+    double t_low = s_min + span * alpha;
+    double t_high = s_max - span * beta;
+    for (int i = 0; i < n_chunks; ++i) {
+        if (sim[i] > t_high)
+            bits_out[i] = 16;
+        else if (sim[i] > t_low)
+            bits_out[i] = 4;
+        else
+            bits_out[i] = 2;
+    }
+}
+
+/*
+ * Stable partition of chunk indices by class (R9).  perm[k] is the original
+ * index of the chunk at position k of the reordered cache; counts[0..2] are
+ * the numbers of FP16, INT4 and INT2 chunks.
+ */
+void kvqo_chunk_partition(const uint8_t *bits, int n_chunks, int32_t *perm,
+                          int32_t *counts)
+{
+    static const uint8_t order[3] = {16, 4, 2};
+    int k = 0;
+    for (int c = 0; c < 3; ++c) {
+        counts[c] = 0;
+        for (int i = 0; i < n_chunks; ++i) {
+            if (bits[i] == order[c]) {
+                perm[k++] = i;
+                counts[c] += 1;
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* KV-cache size ([P2] formula; [P5] 1.2 worked example)                    */
+/* ------------------------------------------------------------------------ */
+
+/* Number of cached K and V elements: 2 * layers * kv_heads * head_dim *
+ * seq_len * batch. */
+uint64_t kvqo_kv_elements(uint64_t layers, uint64_t kv_heads,
+                          uint64_t head_dim, uint64_t seq_len, uint64_t batch)
+{
+    return 2u * layers * kv_heads * head_dim * seq_len * batch;
+}

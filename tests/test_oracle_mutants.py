@@ -1,0 +1,151 @@
+"""Mutation check of the oracle's pins.
+
+Each case plants one plausible mistake in a temporary copy of the oracle's C
+source (never in the oracle itself), rebuilds the copy, and asserts that at
+least one pin -- a hand-derived fixture, a library routine or a closed form
+-- now fails.  A mutant that survives would mean the pins cannot tell that
+mistake from the real thing."""
+import importlib.util
+import json
+import math
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ORACLE_DIR = os.path.join(ROOT, "oracle")
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+# (name, original text, mutated text)
+MUTANTS = [
+    ("round half away from zero", "float c = rintf(kvqo_f16_to_f32(x[j]) / s) + z;",
+     "float c = roundf(kvqo_f16_to_f32(x[j]) / s) + z;"),
+    ("scale rounded to nearest", "uint16_t s16 = kvqo_f32_to_f16_up(s32);",
+     "uint16_t s16 = kvqo_f32_to_f16(s32);"),
+    ("zero point clamped to code range", "    uint16_t z16 = kvqo_f32_to_f16(zf);",
+     "    if (zf < 0.0f) zf = 0.0f; if (zf > qmax) zf = qmax;\n    uint16_t z16 = kvqo_f32_to_f16(zf);"),
+    ("no scale floor", "    if (s32 < 1e-5f)\n        s32 = 1e-5f;", ""),
+    ("zero point sign flipped", "float zf = rintf(-mn / s) + 0.0f;", "float zf = rintf(mn / s) + 0.0f;"),
+    ("negative zero kept", "float zf = rintf(-mn / s) + 0.0f;", "float zf = rintf(-mn / s);"),
+    ("2^bits levels", "const float qmax = (float)((1 << bits) - 1);",
+     "const float qmax = (float)(1 << bits);"),
+    ("high nibble first", "cr[bitpos / 8] |= (uint8_t)(tmp[j] << (bitpos % 8));",
+     "cr[bitpos / 8] |= (uint8_t)(tmp[j] << (8 - bits - bitpos % 8));"),
+    ("dequant adds zero point", "out[r * D + e] = (c - z) * s;", "out[r * D + e] = (c + z) * s;"),
+    ("score not scaled", "score[t] = scale * acc;", "score[t] = acc;"),
+    ("lse in log2", "lse[h] = m + log(l);\n    }\n    free(score);",
+     "lse[h] = m + log2(l);\n    }\n    free(score);"),
+    ("merge drops block weights", "l += w * lb[b];", "l += lb[b];"),
+    ("FP16 threshold inclusive", "if (sim[i] > t_high)", "if (sim[i] >= t_high)"),
+    ("query norm missing", "sim[i] = dot / (nq * sqrt(cc));", "sim[i] = dot / sqrt(cc);"),
+    ("INT2 before INT4", "static const uint8_t order[3] = {16, 4, 2};",
+     "static const uint8_t order[3] = {16, 2, 4};"),
+    ("f16 rounding truncates", "if (rest > 0x1000u || (rest == 0x1000u && (h & 1u)))",
+     "if (rest > 0x1000u)"),
+]
+
+
+def _build_mutant(tmp_path, orig, new):
+    src = open(os.path.join(ORACLE_DIR, "kvq_oracle.c")).read()
+    assert orig in src, orig
+    d = tmp_path / "oracle_mutant"
+    d.mkdir()
+    (d / "kvq_oracle.c").write_text(src.replace(orig, new, 1))
+    shutil.copy(os.path.join(ORACLE_DIR, "__init__.py"), d / "__init__.py")
+    spec = importlib.util.spec_from_file_location("oracle_mutant_" + str(abs(hash(new))),
+                                                  str(d / "__init__.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build(force=True)
+    return mod
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _pins(o):
+    """Yield (pin name, passed) for a compact set of the oracle's pins."""
+    ex = _golden("quant_worked_examples.json")
+    ok = True
+    for g in ex["groups"]:
+        with np.errstate(all="ignore"):
+            code, s16, z16 = o.quantize_group(np.asarray(g["x"], np.float16).view(np.uint16),
+                                              g["bits"])
+        ok &= (list(code) == g["codes"] and s16 == int(g["s16"], 16)
+               and z16 == int(g["z16"], 16))
+    yield "quant worked examples", ok
+
+    j = np.arange(128)
+    x = np.where(j < 64, j % 16, -((j - 64) % 16)).astype(np.float16).view(np.uint16)[None]
+    codes, _ = o.quantize_rows(x, 64, 4)
+    yield "packing example", codes[0].tobytes().hex() == ex["rows"][0]["codes_hex"]
+
+    rng = np.random.default_rng(0)
+    G, bits = 64, 4
+    xs = np.concatenate([rng.standard_normal((200, G)), rng.uniform(1, 9, (200, G))]).astype(np.float16)
+    with np.errstate(all="ignore"):
+        c, m = o.quantize_rows(xs.view(np.uint16), G, bits)
+        xh = o.dequantize_rows(c, m, G, G, bits)
+    s = m[:, 0, 0].view(np.float16).astype(np.float64)
+    err = np.abs(xs.astype(np.float64) - xh)
+    yield "half-step bound", bool(np.all(err <= s[:, None] / 2 * (1 + 2.0**-12) + 1e-12))
+
+    h = np.arange(0, 0x7c00, dtype=np.uint32).astype(np.uint16)
+    lo = h[:-1].view(np.float16).astype(np.float64)
+    hi = h[1:].view(np.float16).astype(np.float64)
+    mid = ((lo + hi) / 2).astype(np.float32)
+    yield "fp16 ties vs numpy", bool(np.array_equal(o.f32_to_f16_bits(mid),
+                                                    mid.astype(np.float16).view(np.uint16)))
+
+    a = _golden("attention_two_tokens.json")
+    oo, ll = o.attention(np.array(a["q"]), np.array(a["K"]), np.array(a["V"]), a["scale"])
+    yield "two-token expansion", bool(np.allclose(oo, a["o"], atol=1e-14)
+                                      and np.allclose(ll, a["lse"], atol=1e-14))
+
+    q = rng.standard_normal((4, 32))
+    K = rng.standard_normal((50, 32))
+    V = rng.standard_normal((50, 32))
+    oo, ll = o.attention(q, K, V, 0.2)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, :, None], torch.from_numpy(K)[None, None].expand(1, 4, 50, 32),
+        torch.from_numpy(V)[None, None].expand(1, 4, 50, 32), scale=0.2)[0, :, 0].numpy()
+    lref = np.log(np.exp(0.2 * q @ K.T).sum(1))
+    yield "torch sdpa", bool(np.allclose(oo, ref, atol=1e-12) and np.allclose(ll, lref, atol=1e-12))
+    ob, lb = o.attention_blocks(q, K * 3, V, 0.2, [0, 7, 7, 30, 50])
+    od, ld = o.attention(q, K * 3, V, 0.2)
+    yield "blocks equal direct", bool(np.allclose(ob, od, atol=1e-12) and np.allclose(lb, ld, atol=1e-12))
+
+    t = _golden("chunk_threshold_toy.json")
+    sim, cls = o.chunk_assign(np.array(t["chunks"], np.float32), np.array(t["query"], np.float32),
+                              t["alpha"], t["beta"])
+    perm, _ = o.chunk_partition(cls)
+    yield "threshold toy", (sim.tolist() == t["sims"] and cls.tolist() == t["classes"]
+                            and perm.tolist() == t["perm"])
+
+    emb = rng.standard_normal((64, 24)).astype(np.float32)
+    qe = (3 * rng.standard_normal(24)).astype(np.float32)
+    sim, _ = o.chunk_assign(emb, qe, 0.6, 0.1)
+    e64, q64 = emb.astype(np.float64), qe.astype(np.float64)
+    ref = e64 @ q64 / (np.linalg.norm(e64, axis=1) * np.linalg.norm(q64))
+    yield "cosine vs numpy", bool(np.allclose(sim, ref, rtol=1e-12, atol=1e-15))
+
+
+def test_real_oracle_passes_compact_pins():
+    import oracle
+    failed = [name for name, ok in _pins(oracle) if not ok]
+    assert failed == []
+
+
+@pytest.mark.parametrize("name,orig,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, orig, new):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc missing")
+    mod = _build_mutant(tmp_path, orig, new)
+    results = dict(_pins(mod))
+    assert not all(results.values()), f"mutant '{name}' passed every pin: {results}"
