@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the quantized KV cache on B200.
+
+One step = quantize-on-write of one new token per sequence
+(kvq_quantize_append) + decode attention of one query per sequence over the
+whole packed cache (kvq_decode_partials + kvq_decode_merge, i.e.
+kvq_decode_attention).  Default workload: the Llama-2-7B-shaped MHA layer
+(batch 16, 32 heads, head_dim 128, context 4096, INT8 group 128, bf16
+queries); the cache length runs through the workload's 100-step episode
+(4097 .. 4196 tokens) and restarts, so any --steps keeps the same shape.
+
+Prints one JSON line (rank 0): tokens/s over all ranks (device-timed, max
+over ranks), the roofline of the split-K attention kernel against the
+measured HBM copy bandwidth, end-to-end tokens/s through the public API with
+host buffers, the oracle's CPU throughput, and clocks sampled during the
+timed region.  `--impl reference` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-KV decode attention tokens/s; KV-read GB/s as % of B200 HBM peak"
+DTYPE = {2: "u2", 4: "u4", 8: "u8", 16: "f16"}
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
+    p.add_argument("--workload", default="llama2_7b_mha_int8")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def bytes_per_head_token(bits: int, group: int, head_dim: int = 128) -> int:
+    """K plus V bytes of one (sequence, KV head, token): codes + (s, z) pairs."""
+    meta = 0 if bits == 16 else (head_dim // group) * 4
+    return 2 * (head_dim * bits // 8 + meta)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("kvq_decode.cu", "kvq_device.cuh"):
+        with open(os.path.join(ROOT, "quantized_kv_cache_12_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per split-kernel launch from the committed ncu summary, or
+    None when the kernel source changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(workload)
+    except Exception:
+        return None
+    if not rec or rec.get("kernel_sha") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons (every 100 ms)."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 6:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        inside = [s for t, s in self.samples if t0 <= t <= t1]
+        window = "timed region"
+        if not inside:
+            inside = [s for _, s in self.samples]
+            window = "whole run (timed region shorter than the 100 ms sampling period)"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in inside for i in range(4)
+                          if s[2 + i].lower().startswith("active")})
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(s[0]) for s in inside if num(s[0]) is not None]
+        mx = [num(s[1]) for s in inside if num(s[1]) is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(inside), "window": window}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, wl):
+    """The CPU oracle as it stands, on this host's cores: each step attends
+    one (sequence, KV head) of the workload after appending one token."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import workloads
+    sub = wl.scaled(batch=1, kv_heads=min(wl.kv_heads, 4),
+                    q_heads=min(wl.kv_heads, 4) * wl.group_ratio)
+    L = wl.context
+    k, v = workloads.kv_tokens(sub, L, "cpu")
+    kn, vn = workloads.kv_tokens(sub, 1, "cpu", stream_extra=1)
+    q = workloads.queries(sub, "cpu")
+    g = wl.group_ratio
+    prepared = []
+    for h in range(sub.kv_heads):
+        kc, km = oracle.quantize_rows(k[0, h].numpy().view(np.uint16), wl.group, wl.bits)
+        vc, vm = oracle.quantize_rows(v[0, h].numpy().view(np.uint16), wl.group, wl.bits)
+        qh = q[0, h * g:(h + 1) * g].contiguous().view(torch.int16).numpy().view(np.uint16)
+        prepared.append((kc, km, vc, vm, qh, kn[0, h].numpy().view(np.uint16),
+                         vn[0, h].numpy().view(np.uint16)))
+
+    def step(i):
+        kc, km, vc, vm, qh, knew, vnew = prepared[i % len(prepared)]
+        ck, mk = oracle.quantize_rows(knew, wl.group, wl.bits)
+        cv, mv = oracle.quantize_rows(vnew, wl.group, wl.bits)
+        kc2 = np.concatenate([kc, ck])
+        km2 = np.concatenate([km, mk])
+        vc2 = np.concatenate([vc, cv])
+        vm2 = np.concatenate([vm, mv])
+        oracle.attention_packed(qh, wl.q_dtype == "bf16", kc2, km2, wl.bits, vc2, vm2, wl.bits,
+                                wl.group, L + 1, 128 ** -0.5)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    value = args.steps / wl.kv_heads / el
+    sample = (f"each step: one (sequence, KV head) of {wl.name} at {L + 1} tokens "
+              f"(append 1 token + attention of {g} query heads); tokens/s = steps / kv_heads "
+              f"({wl.kv_heads}) / seconds")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": DTYPE[wl.bits], "data": "synthetic",
+        "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, extra=None):
+    cfg = {"workload": wl.name, "batch_per_gpu": wl.batch, "q_heads": wl.q_heads,
+           "kv_heads": wl.kv_heads, "head_dim": wl.head_dim, "context": wl.context,
+           "bits": wl.bits, "group": wl.group, "q_dtype": wl.q_dtype,
+           "episode_steps": wl.steps if wl.append else 0}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ---------------------------------------------------------------- CPU baseline
+
+def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
+    """The oracle (single-threaded C, fp64 attention) on a bounded sample of
+    the same inputs: (sequence, KV head) pairs, each one append + attention."""
+    import numpy as np
+    import torch
+
+    import oracle
+    g = wl.group_ratio
+    pairs = [(b, h) for b in range(min(wl.batch, 2)) for h in range(min(wl.kv_heads, 4))]
+    prepared = []
+    for b, h in pairs:
+        kk = k[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        vv = v[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        kc, km = oracle.quantize_rows(kk, wl.group, wl.bits)
+        vc, vm = oracle.quantize_rows(vv, wl.group, wl.bits)
+        qh = q[b, h * g:(h + 1) * g].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        knew = kn[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        vnew = vn[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        prepared.append((kc, km, vc, vm, qh, knew, vnew))
+    L = k.shape[2]
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        kc, km, vc, vm, qh, knew, vnew = prepared[n % len(prepared)]
+        ck, mk = oracle.quantize_rows(knew, wl.group, wl.bits)
+        cv, mv = oracle.quantize_rows(vnew, wl.group, wl.bits)
+        oracle.attention_packed(qh, wl.q_dtype == "bf16", np.concatenate([kc, ck]),
+                                np.concatenate([km, mk]), wl.bits, np.concatenate([vc, cv]),
+                                np.concatenate([vm, mv]), wl.bits, wl.group, L + 1,
+                                128 ** -0.5)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and n >= 2:
+            break
+    return {"value": n / wl.kv_heads / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} (sequence, KV head) decode steps of {wl.name} at {L + 1} tokens "
+                      f"cycling over {len(prepared)} pairs, {el:.1f} s on one host thread; "
+                      f"tokens/s = pairs / kv_heads / seconds"}
+
+
+# ---------------------------------------------------------------- kvq arm
+
+def run_kvq(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import workloads
+    from quantized_kv_cache_12_b200 import kvq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if wl.chunk_tokens:
+        raise SystemExit("bench: the chunk-level mixed-precision workload is a parity case here")
+    B, H, Hq, D = wl.batch, wl.kv_heads, wl.q_heads, wl.head_dim
+    ctx = wl.context
+    episode = wl.steps if wl.append else 1
+    max_tokens = workloads.round_up(ctx + episode + 1, 64)
+    wlr = wl.scaled(seed=wl.seed + 1000 * rank)  # each rank its own sequences
+
+    # ---- resident inputs (untimed set-up)
+    k, v = workloads.kv_tokens(wlr, ctx, dev)
+    cache = kvq.QuantizedKVCache.allocate(B, H, D, max_tokens, wl.bits, wl.group, dev)
+    cache.seq_lens.zero_()
+    kvq.kvq_quantize_append(cache, k, v, ctx, advance_seq_lens=True)
+    base_lens = cache.seq_lens.clone()
+    kn = torch.stack([torch.stack(workloads.kv_tokens(wlr, 1, dev, stream_extra=1 + e))
+                      for e in range(episode)])           # [E, 2, B, H, 1, D]
+    qs = torch.stack([workloads.queries(wlr, dev, step=e) for e in range(episode)])
+    hint = ctx + episode
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    ws = kvq.alloc_workspace(cache, Hq, hint, device=dev)
+    ws_bytes = kvq.kvq_decode_workspace_bytes(cache, Hq, hint)
+    bh = B * Hq
+    parts = next(p for p in range(1, 1 << 16)
+                 if 256 + (bh * p * 8 + 255) // 256 * 256 + bh * p * D * 4 == ws_bytes)
+    launches_per_step = (1 if wl.append else 0) + 1 + (1 if parts > 1 else 0)
+    stream = torch.cuda.current_stream()
+
+    def step(s, ev=None):
+        e = s % episode
+        if wl.append:
+            if e == 0:
+                cache.seq_lens.copy_(base_lens, non_blocking=True)
+            kvq.kvq_quantize_append(cache, kn[e, 0], kn[e, 1], 1, advance_seq_lens=True)
+        if ev is not None:
+            ev[0].record(stream)
+        kvq.kvq_decode_partials(cache, qs[e], out, lse, ws, max_len_hint=hint)
+        if ev is not None:
+            ev[1].record(stream)
+        kvq.kvq_decode_merge(cache, qs[e], out, lse, ws, max_len_hint=hint)
+
+    def lens_at(s):
+        return ctx + (s % episode) + 1 if wl.append else ctx
+
+    # ---- warm-up
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    h0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    h1 = time.time()
+    ms = t_start.elapsed_time(t_end)
+    split_ms = sum(a.elapsed_time(b) for a, b in evs)
+    assert kvq.workspace_error_word(ws) == 0, "device wait gave up (error word set)"
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clocks = sampler.summary(h0, h1) if sampler else None
+    if sampler:
+        sampler.stop()
+
+    bpt = bytes_per_head_token(wl.bits, wl.group, D)
+    kv_bytes = [B * H * lens_at(args.warmup + i) * bpt for i in range(args.steps)]
+    q_bytes = B * Hq * D * 2
+    alg_bytes = sum(kv_bytes) + args.steps * q_bytes
+    tokens = B * args.steps * world
+    value = tokens / (ms / 1e3)
+
+    # ---- end to end through the public call with pinned host buffers
+    kn_h = kn.cpu().pin_memory()
+    qs_h = qs.cpu().pin_memory()
+    k_d = torch.empty_like(kn[0, 0])
+    v_d = torch.empty_like(kn[0, 1])
+    q_d = torch.empty_like(qs[0])
+    out_h = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
+    lse_h = torch.empty((B, Hq), dtype=torch.float32).pin_memory()
+    cache.seq_lens.copy_(base_lens)
+
+    def e2e_step(s):
+        e = s % episode
+        if wl.append:
+            if e == 0:
+                cache.seq_lens.copy_(base_lens, non_blocking=True)
+            k_d.copy_(kn_h[e, 0], non_blocking=True)
+            v_d.copy_(kn_h[e, 1], non_blocking=True)
+        q_d.copy_(qs_h[e], non_blocking=True)
+        if wl.append:
+            kvq.kvq_quantize_append(cache, k_d, v_d, 1, advance_seq_lens=True)
+        kvq.kvq_decode_attention(cache, q_d, out, lse, ws, max_len_hint=hint)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    for s in range(args.warmup):
+        e2e_step(s)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(args.warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    h2d = (kn[0].numel() * 2 if wl.append else 0) + qs[0].numel() * 2
+    d2h = out.numel() * 4 + lse.numel() * 4
+
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peak()
+    achieved = alg_bytes / (split_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": DTYPE[wl.bits], "data": "synthetic",
+        "config": workload_config(wl, {
+            "global_batch": B * world, "parallelism": f"dp{world} (sequences sharded)",
+            "cache_tokens_per_step": f"{ctx + 1}..{ctx + episode}" if wl.append else ctx,
+            "l2": f"inputs larger than L2: {sum(kv_bytes) / args.steps / 1e6:.0f} MB of packed "
+                  f"K/V read per step per GPU (L2 126 MB)",
+            "step": "quantize-append 1 token/seq + split-K decode attention + LSE merge"}),
+        "kv_read_gbs": sum(kv_bytes) / (ms / 1e3) / 1e9 * world,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                     "traffic": recorded_traffic(wl.name), "kernel": "decode_split_kernel",
+                     "alg_bytes_per_launch": alg_bytes / args.steps,
+                     "avg_launch_us": split_ms / args.steps * 1e3},
+        "e2e": {"value": B * args.steps * world / (e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, k, v, kn[0, 0], kn[0, 1], qs[0],
+                                            args.cpu_seconds)
+    return line
+
+
+def main():
+    args = parse_args()
+    import workloads
+    wl = workloads.WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_kvq(args, wl, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,260 @@
+/*
+ * kvq.h -- C ABI of libkvq: a group-quantized KV cache and decode attention
+ * that reads it, for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (pages cited by title and section):
+ *  - Group-wise asymmetric quantization of K and V as they are written:
+ *    quant(x) = round(x/s) + z with one scale s and zero point z per group
+ *    (Cocktail page, peacm.com news 1099647, section 3.2.2; the TurboQuant
+ *    page, bhfrc.com news 57821, section 2.3, "one scale per group";
+ *    s = (max - min) / (2^bits - 1), "大模型KV缓存量化技术" page section 2.1;
+ *    s floored at 1e-5, "大模型推理加速之KV Cache量化压缩原理与工程实现" page,
+ *    troubleshooting).
+ *  - Single-query decode attention straight over the packed codes, the
+ *    dequantization folded into the QK^T and PV products instead of a
+ *    separate pass (TurboQuant page 2.3, last paragraph), split over the
+ *    token axis and merged by log-sum-exp (Cocktail page 3.2.3: block-wise
+ *    attention merged is equal to the unchunked computation).
+ *  - Cocktail's chunk-level mixed precision: per-chunk FP16/INT4/INT2 class
+ *    from the cosine similarity of chunk and query embeddings with
+ *    T_low = s_min + (s_max - s_min) * alpha and
+ *    T_high = s_max - (s_max - s_min) * beta (Cocktail page 3.1.1), and the
+ *    reorder that makes equal bit-widths contiguous (3.1.2).
+ *
+ * Numerics (fixed so that codes, scales and zero points are reproducible
+ * bit for bit): per group of G fp16 values, in fp32 with IEEE operations:
+ *   mn, mx = min, max;  s32 = max((mx - mn) / qmax, 1e-5), qmax = 2^bits - 1;
+ *   s = fp16 value of s32 rounded toward +infinity (stored);
+ *   z = rint(-mn / s) (+0 for a zero result), clamped to +-65504, stored fp16;
+ *   code = clamp(rint(x / s) + z, 0, qmax), rint = round half to even.
+ * Dequantized value: (code - z) * s.
+ *
+ * Conventions for every entry point:
+ *  - Ownership: the caller owns every buffer.  The library never allocates,
+ *    frees or synchronizes; work is enqueued on the given stream and the
+ *    call returns as soon as it is enqueued.  Pointers marked "device" must
+ *    be device (or managed) memory of the current device.
+ *  - Errors: arguments are validated on the host before anything is
+ *    enqueued; a non-OK status means nothing was enqueued (except
+ *    KVQ_ERR_CUDA, returned when a launch failed).  No entry point reads
+ *    device memory on the host, so values held only on the device (the
+ *    sequence lengths) are bounds-checked by the kernels themselves: they
+ *    never read or write outside the buffers described here.
+ *  - Thread safety: calls on different streams may run concurrently; calls
+ *    that share a cache or workspace must be ordered by the caller.
+ *  - Streams: `stream` is a cudaStream_t passed as void*; NULL is the
+ *    legacy default stream.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvq_status {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned buffer   */
+    KVQ_ERR_UNSUPPORTED = 2, /* valid but not built: (bits, G, head_dim, g) */
+    KVQ_ERR_CAPACITY = 3,    /* a host-known size exceeds the cache         */
+    KVQ_ERR_WORKSPACE = 4,   /* workspace missing or too small              */
+    KVQ_ERR_CUDA = 5         /* a CUDA launch or runtime call failed        */
+} kvq_status;
+
+typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
+
+/*
+ * One K or V plane of a cache (one bit-width).
+ *   bits 2, 4, 8: codes  u8  [batch][kv_heads][max_tokens][head_dim*bits/8],
+ *                 element j of a token row in byte j*bits/8 at bit offset
+ *                 (j*bits) mod 8 (low bits first);
+ *                 meta  f16 [batch][kv_heads][max_tokens][head_dim/G][2],
+ *                 the pair (scale, zero point) of each group, groups of G
+ *                 consecutive head_dim elements of one token row.
+ *   bits 16:      codes f16 [batch][kv_heads][max_tokens][head_dim] raw
+ *                 values (Cocktail's FP16 class); meta unused (may be NULL).
+ * Both buffers 16-byte aligned.
+ */
+typedef struct kvq_plane {
+    int32_t bits;       /* 2, 4, 8 or 16                                    */
+    int32_t group_size; /* G: 32, 64 or 128, dividing head_dim (bits < 16)  */
+    void *codes;        /* device                                           */
+    void *meta;         /* device; NULL when bits == 16                     */
+} kvq_plane;
+
+/*
+ * A cache (or one bit-width segment of a mixed-precision cache).
+ * seq_lens[b] is the number of valid tokens of sequence b (tokens
+ * [0, seq_lens[b]) of every KV head).  max_tokens must be a multiple of 64.
+ */
+typedef struct kvq_cache {
+    int32_t batch;
+    int32_t kv_heads;
+    int32_t head_dim;   /* 128 in this build                                */
+    int32_t max_tokens; /* token capacity per (sequence, KV head)           */
+    kvq_plane k;
+    kvq_plane v;
+    int32_t *seq_lens;  /* device, [batch]                                  */
+} kvq_cache;
+
+/* Human-readable name of a status. Never NULL. */
+const char *kvq_status_string(kvq_status status);
+
+/* Library version string, e.g. "kvq 0.1 sm_100a". */
+const char *kvq_version(void);
+
+/*
+ * Bytes of the codes and meta buffers of one plane (host-only, no CUDA).
+ * Source: the KV-cache size formula of the "大模型推理加速之KV Cache量化压缩
+ * 原理与工程实现" page (2 * layers * kv_heads * head_dim * seq_len * batch *
+ * bytes per element), per plane and layer, with bits/8 bytes per element
+ * plus 4 bytes of (scale, zero) per group.
+ * Returns KVQ_ERR_INVALID_ARG on non-positive sizes or null outputs,
+ * KVQ_ERR_UNSUPPORTED on a (bits, G, head_dim) this build does not pack.
+ */
+kvq_status kvq_plane_bytes(int32_t batch, int32_t kv_heads, int32_t head_dim,
+                           int32_t max_tokens, int32_t bits, int32_t group_size,
+                           size_t *codes_bytes, size_t *meta_bytes);
+
+/*
+ * Number of K and V elements of a model's cache, 2 * layers * kv_heads *
+ * head_dim * seq_len * batch (same page's formula; the TurboQuant page's
+ * section 1.2 worked example, 32 layers x 32 heads x 128 x 131072 tokens,
+ * gives 34,359,738,368).  Host-only.  Returns 0 on overflow.
+ */
+uint64_t kvq_kv_elements(uint64_t layers, uint64_t kv_heads, uint64_t head_dim,
+                         uint64_t seq_len, uint64_t batch);
+
+/*
+ * Quantize n_new tokens per sequence and write them at positions
+ * seq_lens[b] .. seq_lens[b] + n_new - 1 of each sequence's K and V planes
+ * (quantize-on-write: Cocktail page 3.2.2 formula; Oaken's write pipeline,
+ * jsqmd.com news 825302 section 3.2.3, quantizes inside the memory write).
+ *   k_new, v_new: device fp16 [batch][kv_heads][n_new][head_dim], 16-byte
+ *                 aligned.  n_new = 1 is the decode-step append; n_new = the
+ *                 prompt length is the bulk prefill (with seq_lens = 0).
+ *   advance_seq_lens: nonzero adds n_new to seq_lens[b] after the write
+ *                 (capped at max_tokens), in stream order.
+ * Tokens whose position would reach max_tokens are not written (the
+ * kernel checks on the device).  Both planes must have bits 2, 4 or 8 and
+ * the same group size.  Errors: KVQ_ERR_INVALID_ARG (nulls, n_new < 1,
+ * misalignment), KVQ_ERR_CAPACITY (n_new > max_tokens),
+ * KVQ_ERR_UNSUPPORTED, KVQ_ERR_CUDA.
+ */
+kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k_new,
+                               const void *v_new, int32_t n_new,
+                               int32_t advance_seq_lens, void *stream);
+
+/*
+ * Workspace bytes that kvq_decode_attention needs for these segments and
+ * arguments (host-only).  The workspace holds the per-split partial
+ * results (m, l, o) merged by log-sum-exp and a 256-byte header whose
+ * first 32-bit word is a sticky device error flag (nonzero after a kernel
+ * gave up a bounded wait; the library never clears it).
+ */
+kvq_status kvq_decode_workspace_bytes(const kvq_cache *segs, int32_t n_segs,
+                                      int32_t q_heads, int32_t max_len_hint,
+                                      size_t *bytes);
+
+/*
+ * Decode attention of one query token per sequence over the packed cache:
+ *   out[b][h] = sum_t p_t * V_hat[b][h/g][t],  p = softmax_t(softmax_scale *
+ *   q[b][h] . K_hat[b][h/g][t]),  lse[b][h] = log sum_t exp(score_t),
+ * over the tokens [0, seq_lens[b]) of every segment (the union, Cocktail
+ * page 3.2.3), with g = q_heads / kv_heads (GQA: query head h reads KV head
+ * h / g).  K_hat, V_hat are dequantized inside the QK^T and PV products
+ * (TurboQuant page 2.3); scores follow the KVO-LLM page, section 3.2
+ * (q . k^T / sqrt(dim)); pass softmax_scale = 1/sqrt(head_dim) for it.
+ *   segs: 1 segment, or several segments of one mixed-precision cache (same
+ *         batch, kv_heads, head_dim; each its own bits, planes, seq_lens).
+ *   q: device [batch][q_heads][head_dim] fp16 or bf16 (q_dtype); bf16 values
+ *      are used as fp16 (exact for magnitudes in [2^-14, 65504]).
+ *   out: device fp32 [batch][q_heads][head_dim]; lse: device fp32
+ *        [batch][q_heads] natural log, or NULL.
+ *   max_len_hint: an upper bound of the seq_lens used to pick the split
+ *        count (<= 0: max_tokens); results are correct for any seq_lens.
+ *   workspace: device, >= kvq_decode_workspace_bytes(same arguments),
+ *        256-byte aligned.
+ * A sequence with no tokens gives out = 0 and lse = -inf.
+ * Supported: head_dim 128; g in 1..8; bits 2/4/8 with G 32/64/128, and bits
+ * 16 with fp16 q.  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED,
+ * KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA.
+ */
+kvq_status kvq_decode_attention(const kvq_cache *segs, int32_t n_segs,
+                                const void *q, kvq_dtype q_dtype,
+                                int32_t q_heads, float softmax_scale,
+                                float *out, float *lse, int32_t max_len_hint,
+                                void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/*
+ * The two halves of kvq_decode_attention, for callers that time or overlap
+ * them separately (same arguments, checks and errors as
+ * kvq_decode_attention; call both, in this order, on the same stream).
+ * kvq_decode_partials launches the split-K kernels: each split writes its
+ * partial result -- running max m (log2 units), sum l = sum 2^(x - m) and
+ * the unnormalised output -- into the workspace, or, when the plan has a
+ * single partial, the final out/lse directly.  kvq_decode_merge combines
+ * the partials by log-sum-exp (Cocktail page 3.2.3) into out/lse; it
+ * enqueues nothing when there is a single partial.
+ */
+kvq_status kvq_decode_partials(const kvq_cache *segs, int32_t n_segs,
+                               const void *q, kvq_dtype q_dtype,
+                               int32_t q_heads, float softmax_scale,
+                               float *out, float *lse, int32_t max_len_hint,
+                               void *workspace, size_t workspace_bytes,
+                               void *stream);
+kvq_status kvq_decode_merge(const kvq_cache *segs, int32_t n_segs,
+                            const void *q, kvq_dtype q_dtype, int32_t q_heads,
+                            float softmax_scale, float *out, float *lse,
+                            int32_t max_len_hint, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
+ * Cocktail chunk-level bit-width search (Cocktail page 3.1.1): for each
+ * sequence b and chunk i, sim = (q . c_i) / (||q|| * ||c_i||) in fp64 (sums
+ * in index order); T_low and T_high from that sequence's s_min, s_max and
+ * alpha, beta; class 16 if sim > T_high, 4 if T_low < sim <= T_high, else 2.
+ *   chunk_emb: device fp32 [batch][n_chunks][emb_dim]
+ *   query_emb: device fp32 [batch][emb_dim]
+ *   sim_out:   device fp64 [batch][n_chunks], or NULL
+ *   chunk_bits_out: device u8 [batch][n_chunks] (16, 4 or 2)
+ * n_chunks <= 4096.  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_CUDA.
+ */
+kvq_status kvq_chunk_assign(const float *chunk_emb, const float *query_emb,
+                            int32_t batch, int32_t n_chunks, int32_t emb_dim,
+                            double alpha, double beta, double *sim_out,
+                            uint8_t *chunk_bits_out, void *stream);
+
+/*
+ * Reorder a prompt's fp16 K/V into three segments by chunk class and
+ * quantize them (Cocktail page 3.1.2: reorder so equal bit-widths are
+ * contiguous, then quantize, then compute).
+ *   segs[0]: the FP16 segment (bits 16), segs[1]: the INT4 segment (bits 4),
+ *   segs[2]: the INT2 segment (bits 2); same batch, kv_heads, head_dim; each
+ *   with max_tokens >= context_len.  Their seq_lens are overwritten with the
+ *   number of tokens of each class.
+ *   k_src, v_src: device fp16 [batch][kv_heads][context_len][head_dim]
+ *   chunk_bits: device u8 [batch][n_chunks], n_chunks = context_len /
+ *               chunk_tokens (as written by kvq_chunk_assign); a value other
+ *               than 16 or 4 is treated as 2
+ *   perm_out: device int32 [batch][n_chunks]: perm_out[b][k] is the original
+ *             index of the k-th chunk of the reordered sequence; FP16 chunks
+ *             first, then INT4, then INT2, each in ascending original index.
+ * chunk_tokens must be a multiple of 16 and divide context_len; n_chunks <=
+ * 4096.  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY,
+ * KVQ_ERR_CUDA.
+ */
+kvq_status kvq_chunk_reorder(const kvq_cache *segs, const void *k_src,
+                             const void *v_src, int32_t context_len,
+                             int32_t chunk_tokens, const uint8_t *chunk_bits,
+                             int32_t *perm_out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -238,7 +238,8 @@ def quantize_cache(x16, group: int, bits: int):
     lead = x16.shape[:-1]
     D = x16.shape[-1]
     codes, meta = quantize_rows(x16.reshape(-1, D), group, bits)
-    return codes.reshape(*lead, -1), meta.reshape(*lead, meta.shape[-2], 2)
+    return (codes.reshape(*lead, D * bits // 8),
+            meta.reshape(*lead, meta.shape[-2], 2))
 
 
 def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: float,

@@ -1,0 +1,327 @@
+// kvq_abi.cu -- the C ABI of libkvq (declared in include/kvq.h): argument
+// validation, launch configuration and dispatch.  Every check that can be
+// made on the host runs before any CUDA call, so a non-OK status means
+// nothing was enqueued.  No allocation, no synchronization.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "kvq.h"
+#include "kvq_internal.h"
+
+namespace {
+
+constexpr int kD = 128;
+constexpr size_t kHeaderBytes = 256;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_group(int g) { return g == 32 || g == 64 || g == 128; }
+
+kvq_status check_plane(const kvq_plane& p, int head_dim, bool allow16) {
+  if (p.codes == nullptr || !aligned16(p.codes)) return KVQ_ERR_INVALID_ARG;
+  if (p.bits == 16) {
+    if (!allow16) return KVQ_ERR_UNSUPPORTED;
+    return KVQ_OK;
+  }
+  if (!(p.bits == 2 || p.bits == 4 || p.bits == 8)) return KVQ_ERR_UNSUPPORTED;
+  if (!valid_group(p.group_size) || head_dim % p.group_size != 0) return KVQ_ERR_UNSUPPORTED;
+  if (p.meta == nullptr || !aligned16(p.meta)) return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
+kvq_status check_cache(const kvq_cache* c, bool allow16) {
+  if (c == nullptr) return KVQ_ERR_INVALID_ARG;
+  if (c->batch <= 0 || c->kv_heads <= 0 || c->max_tokens <= 0 || c->head_dim <= 0)
+    return KVQ_ERR_INVALID_ARG;
+  if (c->head_dim != kD) return KVQ_ERR_UNSUPPORTED;
+  if (c->max_tokens % 64 != 0) return KVQ_ERR_INVALID_ARG;
+  if (c->seq_lens == nullptr) return KVQ_ERR_INVALID_ARG;
+  kvq_status s = check_plane(c->k, c->head_dim, allow16);
+  if (s != KVQ_OK) return s;
+  s = check_plane(c->v, c->head_dim, allow16);
+  if (s != KVQ_OK) return s;
+  if (c->k.bits != c->v.bits) return KVQ_ERR_UNSUPPORTED;
+  if (c->k.bits != 16 && c->k.group_size != c->v.group_size) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+// Split count of one segment: enough CTAs for several waves over 148 SMs,
+// but at least 256 tokens per CTA.
+int choose_splits(const kvq_cache& c, int max_len_hint) {
+  const long long pairs = (long long)c.batch * c.kv_heads;
+  int len = c.max_tokens;
+  if (max_len_hint > 0 && max_len_hint < len) len = max_len_hint;
+  const long long target = 148LL * 2 * 6;  // ~6 waves of 2 CTAs per SM
+  long long n = (target + pairs - 1) / pairs;
+  const long long cap = (len + 255) / 256;
+  if (n > cap) n = cap;
+  if (n < 1) n = 1;
+  return (int)n;
+}
+
+struct SplitPlan {
+  int n_split[16];
+  int parts;
+};
+
+kvq_status plan_splits(const kvq_cache* segs, int n_segs, int max_len_hint, SplitPlan* plan) {
+  plan->parts = 0;
+  for (int i = 0; i < n_segs; ++i) {
+    plan->n_split[i] = choose_splits(segs[i], max_len_hint);
+    plan->parts += plan->n_split[i];
+  }
+  return KVQ_OK;
+}
+
+kvq_status check_segments(const kvq_cache* segs, int n_segs, int q_heads) {
+  if (segs == nullptr || n_segs < 1 || n_segs > 16) return KVQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n_segs; ++i) {
+    kvq_status s = check_cache(&segs[i], true);
+    if (s != KVQ_OK) return s;
+    if (segs[i].batch != segs[0].batch || segs[i].kv_heads != segs[0].kv_heads ||
+        segs[i].head_dim != segs[0].head_dim)
+      return KVQ_ERR_INVALID_ARG;
+  }
+  if (q_heads <= 0 || q_heads % segs[0].kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+  const int g = q_heads / segs[0].kv_heads;
+  for (int i = 0; i < n_segs; ++i) {
+    const int bits = segs[i].k.bits;
+    if (!kvq::decode_supported(bits, bits == 16 ? kD : segs[i].k.group_size, g))
+      return KVQ_ERR_UNSUPPORTED;
+  }
+  return KVQ_OK;
+}
+
+size_t workspace_for(const kvq_cache* segs, int q_heads, int parts) {
+  const size_t bh = (size_t)segs[0].batch * q_heads;
+  const size_t ml = bh * parts * 2 * sizeof(float);
+  const size_t o = bh * parts * kD * sizeof(float);
+  return kHeaderBytes + ((ml + 255) / 256) * 256 + o;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "cache capacity exceeded";
+    case KVQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case KVQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* kvq_version(void) { return "kvq 0.1 sm_100a"; }
+
+kvq_status kvq_plane_bytes(int32_t batch, int32_t kv_heads, int32_t head_dim, int32_t max_tokens,
+                           int32_t bits, int32_t group_size, size_t* codes_bytes,
+                           size_t* meta_bytes) {
+  if (codes_bytes == nullptr || meta_bytes == nullptr) return KVQ_ERR_INVALID_ARG;
+  if (batch <= 0 || kv_heads <= 0 || head_dim <= 0 || max_tokens <= 0) return KVQ_ERR_INVALID_ARG;
+  if (!(bits == 2 || bits == 4 || bits == 8 || bits == 16)) return KVQ_ERR_UNSUPPORTED;
+  if (bits != 16 && (!valid_group(group_size) || head_dim % group_size != 0))
+    return KVQ_ERR_UNSUPPORTED;
+  if ((head_dim * bits) % 8 != 0) return KVQ_ERR_UNSUPPORTED;
+  const size_t rows = (size_t)batch * kv_heads * max_tokens;
+  *codes_bytes = rows * (size_t)head_dim * bits / 8;
+  *meta_bytes = (bits == 16) ? 0 : rows * (size_t)(head_dim / group_size) * 4;
+  return KVQ_OK;
+}
+
+uint64_t kvq_kv_elements(uint64_t layers, uint64_t kv_heads, uint64_t head_dim,
+                         uint64_t seq_len, uint64_t batch) {
+  uint64_t f[5] = {layers, kv_heads, head_dim, seq_len, batch};
+  uint64_t n = 2;
+  for (int i = 0; i < 5; ++i) {
+    if (f[i] != 0 && n > UINT64_MAX / f[i]) return 0;
+    n *= f[i];
+  }
+  return n;
+}
+
+kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const void* v_new,
+                               int32_t n_new, int32_t advance_seq_lens, void* stream) {
+  kvq_status st = check_cache(cache, false);
+  if (st != KVQ_OK) return st;
+  if (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new))
+    return KVQ_ERR_INVALID_ARG;
+  if (n_new < 1) return KVQ_ERR_INVALID_ARG;
+  if (n_new > cache->max_tokens) return KVQ_ERR_CAPACITY;
+  kvq::QuantArgs a;
+  a.k_new = static_cast<const __half*>(k_new);
+  a.v_new = static_cast<const __half*>(v_new);
+  a.k_codes = static_cast<uint8_t*>(cache->k.codes);
+  a.v_codes = static_cast<uint8_t*>(cache->v.codes);
+  a.k_meta = static_cast<uint8_t*>(cache->k.meta);
+  a.v_meta = static_cast<uint8_t*>(cache->v.meta);
+  a.seq_lens = cache->seq_lens;
+  a.batch = cache->batch;
+  a.kv_heads = cache->kv_heads;
+  a.max_tokens = cache->max_tokens;
+  a.n_new = n_new;
+  a.advance = advance_seq_lens != 0;
+  cudaError_t e = kvq::launch_quantize(a, cache->k.bits, cache->k.group_size,
+                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_decode_workspace_bytes(const kvq_cache* segs, int32_t n_segs, int32_t q_heads,
+                                      int32_t max_len_hint, size_t* bytes) {
+  if (bytes == nullptr) return KVQ_ERR_INVALID_ARG;
+  kvq_status st = check_segments(segs, n_segs, q_heads);
+  if (st != KVQ_OK) return st;
+  SplitPlan plan;
+  plan_splits(segs, n_segs, max_len_hint, &plan);
+  *bytes = workspace_for(segs, q_heads, plan.parts);
+  return KVQ_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+enum DecodeStage { kPartials = 1, kMerge = 2, kBoth = 3 };
+
+kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
+                         kvq_dtype q_dtype, int32_t q_heads, float softmax_scale, float* out,
+                         float* lse, int32_t max_len_hint, void* workspace,
+                         size_t workspace_bytes, void* stream, int stages) {
+  kvq_status st = check_segments(segs, n_segs, q_heads);
+  if (st != KVQ_OK) return st;
+  if (q == nullptr || out == nullptr) return KVQ_ERR_INVALID_ARG;
+  if (q_dtype != KVQ_F16 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n_segs; ++i)
+    if (segs[i].k.bits == 16 && q_dtype == KVQ_BF16) return KVQ_ERR_UNSUPPORTED;
+  SplitPlan plan;
+  plan_splits(segs, n_segs, max_len_hint, &plan);
+  const size_t need = workspace_for(segs, q_heads, plan.parts);
+  if (workspace == nullptr || workspace_bytes < need) return KVQ_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KVQ_ERR_INVALID_ARG;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t bh = (size_t)segs[0].batch * q_heads;
+  const size_t ml_bytes = ((bh * plan.parts * 2 * sizeof(float) + 255) / 256) * 256;
+  kvq::DecodeArgs a;
+  a.batch = segs[0].batch;
+  a.kv_heads = segs[0].kv_heads;
+  a.q_heads = q_heads;
+  a.group_ratio = q_heads / segs[0].kv_heads;
+  a.q = q;
+  a.q_is_bf16 = q_dtype == KVQ_BF16;
+  a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
+  a.parts = plan.parts;
+  a.err = reinterpret_cast<uint32_t*>(ws);
+  a.part_ml = reinterpret_cast<float*>(ws + kHeaderBytes);
+  a.part_o = reinterpret_cast<float*>(ws + kHeaderBytes + ml_bytes);
+  a.out = out;
+  a.lse = lse;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int base = 0;
+  for (int i = 0; i < n_segs; ++i) {
+    kvq::SegView v;
+    v.k_codes = static_cast<const uint8_t*>(segs[i].k.codes);
+    v.v_codes = static_cast<const uint8_t*>(segs[i].v.codes);
+    v.k_meta = static_cast<const uint8_t*>(segs[i].k.meta);
+    v.v_meta = static_cast<const uint8_t*>(segs[i].v.meta);
+    v.seq_lens = segs[i].seq_lens;
+    v.bits = segs[i].k.bits;
+    v.group = segs[i].k.bits == 16 ? kD : segs[i].k.group_size;
+    v.max_tokens = segs[i].max_tokens;
+    v.n_split = plan.n_split[i];
+    v.part_base = base;
+    base += plan.n_split[i];
+    if ((stages & kPartials) && kvq::launch_decode_segment(a, v, s) != cudaSuccess)
+      return KVQ_ERR_CUDA;
+  }
+  if ((stages & kMerge) && plan.parts > 1 && kvq::launch_decode_merge(a, s) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_attention(const kvq_cache* segs, int32_t n_segs, const void* q,
+                                kvq_dtype q_dtype, int32_t q_heads, float softmax_scale,
+                                float* out, float* lse, int32_t max_len_hint, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  return decode_stages(segs, n_segs, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
+                       workspace, workspace_bytes, stream, kBoth);
+}
+
+kvq_status kvq_decode_partials(const kvq_cache* segs, int32_t n_segs, const void* q,
+                               kvq_dtype q_dtype, int32_t q_heads, float softmax_scale,
+                               float* out, float* lse, int32_t max_len_hint, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return decode_stages(segs, n_segs, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
+                       workspace, workspace_bytes, stream, kPartials);
+}
+
+kvq_status kvq_decode_merge(const kvq_cache* segs, int32_t n_segs, const void* q,
+                            kvq_dtype q_dtype, int32_t q_heads, float softmax_scale, float* out,
+                            float* lse, int32_t max_len_hint, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return decode_stages(segs, n_segs, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
+                       workspace, workspace_bytes, stream, kMerge);
+}
+
+kvq_status kvq_chunk_assign(const float* chunk_emb, const float* query_emb, int32_t batch,
+                            int32_t n_chunks, int32_t emb_dim, double alpha, double beta,
+                            double* sim_out, uint8_t* chunk_bits_out, void* stream) {
+  if (chunk_emb == nullptr || query_emb == nullptr || chunk_bits_out == nullptr)
+    return KVQ_ERR_INVALID_ARG;
+  if (batch <= 0 || n_chunks <= 0 || n_chunks > 4096 || emb_dim <= 0) return KVQ_ERR_INVALID_ARG;
+  if (!isfinite(alpha) || !isfinite(beta)) return KVQ_ERR_INVALID_ARG;
+  cudaError_t e = kvq::launch_chunk_assign(chunk_emb, query_emb, batch, n_chunks, emb_dim, alpha,
+                                           beta, sim_out, chunk_bits_out,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+kvq_status kvq_chunk_reorder(const kvq_cache* segs, const void* k_src, const void* v_src,
+                             int32_t context_len, int32_t chunk_tokens, const uint8_t* chunk_bits,
+                             int32_t* perm_out, void* stream) {
+  if (segs == nullptr || k_src == nullptr || v_src == nullptr || chunk_bits == nullptr ||
+      perm_out == nullptr)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_src) || !aligned16(v_src)) return KVQ_ERR_INVALID_ARG;
+  const int want_bits[3] = {16, 4, 2};
+  for (int i = 0; i < 3; ++i) {
+    kvq_status st = check_cache(&segs[i], true);
+    if (st != KVQ_OK) return st;
+    if (segs[i].k.bits != want_bits[i]) return KVQ_ERR_INVALID_ARG;
+    if (segs[i].batch != segs[0].batch || segs[i].kv_heads != segs[0].kv_heads)
+      return KVQ_ERR_INVALID_ARG;
+  }
+  if (segs[1].k.group_size != segs[2].k.group_size) return KVQ_ERR_UNSUPPORTED;
+  if (chunk_tokens <= 0 || chunk_tokens % 16 != 0 || context_len <= 0 ||
+      context_len % chunk_tokens != 0)
+    return KVQ_ERR_INVALID_ARG;
+  const int n_chunks = context_len / chunk_tokens;
+  if (n_chunks > 4096) return KVQ_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (segs[i].max_tokens < context_len) return KVQ_ERR_CAPACITY;
+  kvq::ReorderArgs r;
+  r.k_src = static_cast<const __half*>(k_src);
+  r.v_src = static_cast<const __half*>(v_src);
+  r.chunk_bits = chunk_bits;
+  r.perm = perm_out;
+  for (int i = 0; i < 3; ++i) r.seg[i] = segs[i];
+  r.batch = segs[0].batch;
+  r.kv_heads = segs[0].kv_heads;
+  r.context_len = context_len;
+  r.chunk_tokens = chunk_tokens;
+  r.n_chunks = n_chunks;
+  cudaError_t e = kvq::launch_chunk_reorder(r, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// kvq_internal.h -- launch interfaces between the C ABI (kvq_abi.cu) and the
+// kernels.  Host-visible structs only; no device code here.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+// One K/V plane pair of one cache segment, as the kernels see it.
+struct SegView {
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const uint8_t* k_meta;  // (scale, zero) fp16 pairs; null for bits 16
+  const uint8_t* v_meta;
+  const int32_t* seq_lens;
+  int32_t bits;
+  int32_t group;
+  int32_t max_tokens;
+  int32_t n_split;       // CTAs per (sequence, KV head) for this segment
+  int32_t part_base;     // index of this segment's first partial
+};
+
+struct DecodeArgs {
+  int32_t batch, kv_heads, q_heads, group_ratio;
+  const void* q;
+  int32_t q_is_bf16;
+  float scale_log2;      // softmax_scale * log2(e)
+  int32_t parts;         // partial results per (sequence, query head)
+  float* part_ml;        // [batch][q_heads][parts][2] (max in log2 units, sum)
+  float* part_o;         // [batch][q_heads][parts][head_dim], unnormalised
+  float* out;            // [batch][q_heads][head_dim]
+  float* lse;            // [batch][q_heads] or null
+  uint32_t* err;         // sticky device error word
+};
+
+struct QuantArgs {
+  const __half* k_new;
+  const __half* v_new;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  uint8_t* k_meta;
+  uint8_t* v_meta;
+  int32_t* seq_lens;
+  int32_t batch, kv_heads, max_tokens, n_new;
+  int32_t advance;
+};
+
+// Per-bit-width launchers (kvq_quantize.cu, kvq_decode.cu, kvq_chunk.cu).
+cudaError_t launch_quantize(const QuantArgs& a, int bits, int group, cudaStream_t s);
+bool decode_supported(int bits, int group, int group_ratio);
+int decode_smem_bytes(int bits, int group);
+cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
+cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_chunk_assign(const float* emb, const float* qemb, int batch, int n_chunks,
+                                int emb_dim, double alpha, double beta, double* sim,
+                                uint8_t* bits, cudaStream_t s);
+struct ReorderArgs {
+  const __half* k_src;
+  const __half* v_src;
+  const uint8_t* chunk_bits;
+  int32_t* perm;
+  kvq_cache seg[3];
+  int32_t batch, kv_heads, context_len, chunk_tokens, n_chunks;
+};
+cudaError_t launch_chunk_reorder(const ReorderArgs& a, cudaStream_t s);
+
+}  // namespace kvq

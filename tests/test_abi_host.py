@@ -1,0 +1,187 @@
+"""Host-only checks of the C ABI (no GPU needed): the library loads, exports
+every entry point declared in include/kvq.h, sizes its buffers by the
+pages' KV-size formula, and rejects bad arguments before touching CUDA."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from quantized_kv_cache_12_b200 import build
+    build.build()
+    from quantized_kv_cache_12_b200 import kvq as m
+    return m
+
+
+def declared_functions():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_header_declares_the_north_star_entry_points():
+    names = declared_functions()
+    for n in ("kvq_quantize_append", "kvq_decode_attention", "kvq_chunk_reorder"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(kvq):
+    lib = ctypes.CDLL(kvq.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert missing == []
+
+
+def test_binding_has_a_function_per_entry_point(kvq):
+    for n in declared_functions():
+        assert callable(getattr(kvq, n)), n
+
+
+def test_version_and_status_strings(kvq):
+    assert "sm_100a" in kvq.kvq_version()
+    assert kvq.kvq_status_string(0) == "ok"
+    assert "workspace" in kvq.kvq_status_string(4)
+
+
+def test_kv_elements_matches_worked_example(kvq):
+    ex = json.load(open(os.path.join(ROOT, "tests", "golden", "kv_size_worked_example.json")))
+    n = kvq.kvq_kv_elements(ex["layers"], ex["kv_heads"], ex["head_dim"], ex["seq_len"],
+                            ex["batch"])
+    assert n == ex["elements"]
+    assert kvq.kvq_kv_elements(2**40, 2**40, 1, 1, 1) == 0  # overflow reported as 0
+
+
+def test_plane_bytes(kvq):
+    # per plane: rows * head_dim * bits/8 code bytes + rows * (head_dim/G) * 4 meta bytes
+    assert kvq.kvq_plane_bytes(16, 32, 128, 4224, 8, 128) == (16 * 32 * 4224 * 128,
+                                                             16 * 32 * 4224 * 4)
+    assert kvq.kvq_plane_bytes(1, 8, 128, 131072, 4, 64) == (8 * 131072 * 64, 8 * 131072 * 8)
+    assert kvq.kvq_plane_bytes(2, 3, 128, 64, 2, 32) == (2 * 3 * 64 * 32, 2 * 3 * 64 * 16)
+    assert kvq.kvq_plane_bytes(1, 1, 128, 64, 16, 0) == (64 * 256, 0)
+    # per (sequence, head, token), K plus V: 144 bytes for INT4 G64, 264 for INT8 G128
+    c, m = kvq.kvq_plane_bytes(1, 1, 128, 1, 4, 64)
+    assert 2 * (c + m) == 144
+    c, m = kvq.kvq_plane_bytes(1, 1, 128, 1, 8, 128)
+    assert 2 * (c + m) == 264
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_plane_bytes(1, 1, 128, 64, 3, 64)
+    assert e.value.status == kvq.KVQ_ERR_UNSUPPORTED
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_plane_bytes(0, 1, 128, 64, 4, 64)
+    assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
+
+
+def _fake_cache(kvq, bits=4, group=64, max_tokens=256, batch=2, kv_heads=2, head_dim=128):
+    c = kvq.kvq_cache()
+    c.batch, c.kv_heads, c.head_dim, c.max_tokens = batch, kv_heads, head_dim, max_tokens
+    # fake, never-dereferenced 256-aligned addresses: validation must reject
+    # or accept without touching memory
+    c.k = kvq.kvq_plane(bits, group, 0x10000, 0x20000)
+    c.v = kvq.kvq_plane(bits, group, 0x30000, 0x40000)
+    c.seq_lens = 0x50000
+    return c
+
+
+def _status(fn, *args):
+    try:
+        fn(*args)
+    except Exception as e:  # KvqError
+        return getattr(e, "status", None)
+    return 0
+
+
+def test_quantize_append_rejects_bad_arguments(kvq):
+    S = kvq.kvq_quantize_append
+    ok_ptr = 0x60000
+
+    class T:  # minimal tensor stand-in: only data_ptr() is used
+        def __init__(self, p):
+            self.p = p
+
+        def data_ptr(self):
+            return self.p
+
+    c = _fake_cache(kvq)
+    assert _status(S, c, T(0), T(ok_ptr), 1) == kvq.KVQ_ERR_INVALID_ARG       # null k_new
+    assert _status(S, c, T(ok_ptr + 4), T(ok_ptr), 1) == kvq.KVQ_ERR_INVALID_ARG  # misaligned
+    assert _status(S, c, T(ok_ptr), T(ok_ptr), 0) == kvq.KVQ_ERR_INVALID_ARG  # n_new < 1
+    assert _status(S, c, T(ok_ptr), T(ok_ptr), 257) == kvq.KVQ_ERR_CAPACITY
+    assert _status(S, _fake_cache(kvq, bits=3), T(ok_ptr), T(ok_ptr), 1) == kvq.KVQ_ERR_UNSUPPORTED
+    assert _status(S, _fake_cache(kvq, group=48), T(ok_ptr), T(ok_ptr), 1) == \
+        kvq.KVQ_ERR_UNSUPPORTED
+    assert _status(S, _fake_cache(kvq, head_dim=64), T(ok_ptr), T(ok_ptr), 1) == \
+        kvq.KVQ_ERR_UNSUPPORTED
+    assert _status(S, _fake_cache(kvq, max_tokens=100), T(ok_ptr), T(ok_ptr), 1) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    assert _status(S, _fake_cache(kvq, bits=16), T(ok_ptr), T(ok_ptr), 1) == \
+        kvq.KVQ_ERR_UNSUPPORTED  # FP16 planes are written by the reorder, not quantized
+    c2 = _fake_cache(kvq)
+    c2.v.group_size = 32
+    assert _status(S, c2, T(ok_ptr), T(ok_ptr), 1) == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_decode_workspace_and_argument_checks(kvq):
+    c = _fake_cache(kvq, batch=4, kv_heads=8, max_tokens=8192)
+    n1 = kvq.kvq_decode_workspace_bytes(c, 32)
+    n2 = kvq.kvq_decode_workspace_bytes(c, 32, max_len_hint=300)
+    assert n1 > n2 > 256
+    assert (n1 - 256) % 4 == 0
+    # q_heads not a multiple of kv_heads; unsupported group ratio; too many rows
+    assert _status(kvq.kvq_decode_workspace_bytes, c, 12) == kvq.KVQ_ERR_INVALID_ARG
+    assert _status(kvq.kvq_decode_workspace_bytes, c, 24) == kvq.KVQ_ERR_UNSUPPORTED
+    c32 = _fake_cache(kvq, group=32, kv_heads=4)
+    assert _status(kvq.kvq_decode_workspace_bytes, c32, 32) == kvq.KVQ_ERR_UNSUPPORTED
+    assert kvq.kvq_decode_workspace_bytes(c32, 16) > 0
+
+    lib = kvq.lib
+    arr = (kvq.kvq_cache * 1)(c)
+    fake = ctypes.c_void_p(0x70000)
+    st = lib.kvq_decode_attention(arr, 1, fake, 0, 32, ctypes.c_float(0.088), fake, None, 0,
+                                  ctypes.c_void_p(0x80000), 16, None)
+    assert st == kvq.KVQ_ERR_WORKSPACE
+    st = lib.kvq_decode_attention(arr, 1, None, 0, 32, ctypes.c_float(0.088), fake, None, 0,
+                                  ctypes.c_void_p(0x80000), n1, None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+    st = lib.kvq_decode_attention(arr, 1, fake, 0, 32, ctypes.c_float(-1.0), fake, None, 0,
+                                  ctypes.c_void_p(0x80000), n1, None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+    st = lib.kvq_decode_attention(arr, 1, fake, 0, 32, ctypes.c_float(0.088), fake, None, 0,
+                                  ctypes.c_void_p(0x80010), n1, None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG  # workspace not 256-byte aligned
+    c16 = _fake_cache(kvq, bits=16, batch=4, kv_heads=8, max_tokens=8192)
+    arr16 = (kvq.kvq_cache * 1)(c16)
+    n16 = kvq.kvq_decode_workspace_bytes(c16, 32)
+    st = lib.kvq_decode_attention(arr16, 1, fake, kvq.KVQ_BF16, 32, ctypes.c_float(0.088), fake,
+                                  None, 0, ctypes.c_void_p(0x80000), n16, None)
+    assert st == kvq.KVQ_ERR_UNSUPPORTED  # bf16 queries with raw fp16 keys
+
+
+def test_chunk_entry_points_reject_bad_arguments(kvq):
+    lib = kvq.lib
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.kvq_chunk_assign(None, fake, 8, 1024, 768, 0.6, 0.1, None, fake, None) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_chunk_assign(fake, fake, 8, 5000, 768, 0.6, 0.1, None, fake, None) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    segs = (kvq.kvq_cache * 3)(_fake_cache(kvq, bits=16, max_tokens=1024),
+                               _fake_cache(kvq, bits=4, group=32, max_tokens=1024),
+                               _fake_cache(kvq, bits=2, group=32, max_tokens=1024))
+    # chunk size not a multiple of 16; context not a multiple of the chunk size
+    assert lib.kvq_chunk_reorder(segs, fake, fake, 1024, 24, fake, fake, None) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_chunk_reorder(segs, fake, fake, 1000, 32, fake, fake, None) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_chunk_reorder(segs, fake, fake, 2048, 32, fake, fake, None) == \
+        kvq.KVQ_ERR_CAPACITY
+    wrong = (kvq.kvq_cache * 3)(segs[1], segs[0], segs[2])
+    assert lib.kvq_chunk_reorder(wrong, fake, fake, 1024, 32, fake, fake, None) == \
+        kvq.KVQ_ERR_INVALID_ARG

@@ -1,0 +1,220 @@
+"""GPU parity of kvq_decode_attention against the fp64 oracle on the same
+seeded fp16 inputs: max-abs <= 2e-3 and relative L2 <= 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_util import assert_close, f16_bits, fill_cache, fill_fp16_segment, oracle_segment, q_bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    from quantized_kv_cache_12_b200 import kvq as m
+    return m
+
+
+def _poison(c):
+    c.k_codes.fill_(0x77)
+    c.v_codes.fill_(0x88)
+    if c.k_meta is not None:
+        c.k_meta.view(torch.int16).fill_(-1)  # NaN patterns in unused slots
+        c.v_meta.view(torch.int16).fill_(-1)
+
+
+def _run(kvq, segs, q, max_len_hint=0):
+    B, Hq, D = q.shape
+    out = torch.full((B, Hq, D), float("nan"), device=DEV)
+    lse = torch.full((B, Hq), float("nan"), device=DEV)
+    ws = kvq.alloc_workspace(segs, Hq, max_len_hint, device=DEV)
+    kvq.kvq_decode_attention(segs, q, out, lse, ws, max_len_hint=max_len_hint)
+    torch.cuda.synchronize()
+    assert kvq.workspace_error_word(ws) == 0
+    return out, lse
+
+
+def _case(kvq, wl, lens, max_tokens, max_len_hint=0, T=None):
+    B = len(lens)
+    T = T or max(lens)
+    k, v = workloads.kv_tokens(wl, T, DEV, batch=B)
+    q = workloads.queries(wl, DEV, batch=B)
+    c = kvq.QuantizedKVCache.allocate(B, wl.kv_heads, 128, max_tokens, wl.bits, wl.group, DEV)
+    _poison(c)
+    fill_cache(kvq, c, k, v, lens)
+    out, lse = _run(kvq, c, q, max_len_hint)
+    seg = oracle_segment(k, v, wl.bits, wl.group)
+    ref, lref = oracle.decode_attention(q_bits(q), q.dtype == torch.bfloat16, [seg], [lens],
+                                        128 ** -0.5)
+    return out, lse, ref, lref
+
+
+BASES = {
+    "int4_g64_gqa8": workloads.WORKLOADS["llama3_8b_gqa_int4"],
+    "int8_g128_mha_bf16": workloads.WORKLOADS["llama2_7b_mha_int8"],
+    "int4_g64_mha_tiny": workloads.WORKLOADS["tiny"],
+    "int4_g64_long": workloads.WORKLOADS["long_gqa_int4"],
+}
+
+
+@pytest.mark.parametrize("name", list(BASES))
+def test_workload_shapes_small(kvq, name):
+    base = BASES[name]
+    g = base.group_ratio
+    wl = base.scaled(kv_heads=2, q_heads=2 * g)
+    lens = [37, 300, 16]
+    out, lse, ref, lref = _case(kvq, wl, lens, 320)
+    assert_close(out, ref, lse, lref, what=name)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("G", [32, 64, 128])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_bits_groups_ratios(kvq, bits, G, g):
+    if (128 // G) * g > 16:
+        pytest.skip("unsupported combination (more than 16 group x head rows)")
+    wl = workloads.WORKLOADS["long_gqa_int4"].scaled(kv_heads=2, q_heads=2 * g, bits=bits,
+                                                     group=G)
+    lens = [129, 250]
+    out, lse, ref, lref = _case(kvq, wl, lens, 256)
+    assert_close(out, ref, lse, lref, what=f"bits{bits} G{G} g{g}")
+
+
+@pytest.mark.parametrize("hint", [0, 64, 100000])
+def test_split_counts_do_not_change_results(kvq, hint):
+    wl = workloads.WORKLOADS["llama3_8b_gqa_int4"].scaled(kv_heads=1, q_heads=8)
+    lens = [1000, 777]
+    out, lse, ref, lref = _case(kvq, wl, lens, 1024, max_len_hint=hint)
+    assert_close(out, ref, lse, lref, what=f"hint {hint}")
+
+
+def test_edge_lengths(kvq):
+    """Empty sequence (out 0, lse -inf), one token, exact tile multiples, the
+    full capacity, and a tail of one token past a tile."""
+    wl = workloads.WORKLOADS["tiny"].scaled(kv_heads=2, q_heads=4)
+    lens = [0, 1, 16, 64, 17, 128]
+    out, lse, ref, lref = _case(kvq, wl, lens, 128)
+    o = out.cpu().numpy()
+    assert np.all(o[0] == 0.0)
+    assert np.all(np.isneginf(lse.cpu().numpy()[0]))
+    mask = np.ones(len(lens), bool)
+    mask[0] = False
+    assert_close(out, ref, lse, lref, mask=mask, what="edge lengths")
+    # one token: the output is that token's dequantized value
+    seg = oracle_segment(*workloads.kv_tokens(wl, 128, DEV, batch=len(lens)), wl.bits, wl.group)
+    v1 = oracle.dequantize_rows(seg["v_codes"][1, 0, :1], seg["v_meta"][1, 0, :1], 128, 64, 4)
+    np.testing.assert_allclose(o[1, 0], v1[0], atol=1e-5)
+
+
+def test_fp16_segment(kvq):
+    """Raw fp16 rows (Cocktail's FP16 class), ragged lengths, NaN bytes past
+    the valid length."""
+    wl = workloads.WORKLOADS["cocktail_mixed"].scaled(kv_heads=3, q_heads=3)
+    lens = [45, 100]
+    B = len(lens)
+    k, v = workloads.kv_tokens(wl, 100, DEV, batch=B)
+    q = workloads.queries(wl, DEV, batch=B)
+    c = kvq.QuantizedKVCache.allocate(B, 3, 128, 128, 16, 128, DEV)
+    c.k_codes.fill_(0xFF)
+    c.v_codes.fill_(0xFF)  # NaN fp16 everywhere first
+    fill_fp16_segment(c, k, v, lens)
+    c.k_codes[0, :, 45:].fill_(0xFF)
+    c.v_codes[0, :, 45:].fill_(0xFF)
+    out, lse = _run(kvq, c, q)
+    seg = oracle_segment(k, v, 16, 128)
+    ref, lref = oracle.decode_attention(q_bits(q), False, [seg], [lens], 128 ** -0.5)
+    assert_close(out, ref, lse, lref, what="fp16 segment")
+
+
+def test_mixed_segments_equal_unchunked(kvq):
+    """Three segments (FP16, INT4, INT2) of one sequence merged by log-sum-exp
+    equal attention over all their tokens (Cocktail page 3.2.3)."""
+    B, H = 2, 3
+    wl = workloads.WORKLOADS["cocktail_mixed"].scaled(kv_heads=H, q_heads=H)
+    q = workloads.queries(wl, DEV, batch=B)
+    lens = [[32, 64], [96, 0], [500, 320]]
+    segs, osegs = [], []
+    for i, (bits, G) in enumerate(((16, 128), (4, 32), (2, 32))):
+        k, v = workloads.kv_tokens(wl, max(lens[i]), DEV, stream_extra=10 + i, batch=B)
+        c = kvq.QuantizedKVCache.allocate(B, H, 128, 512, bits, G, DEV)
+        _poison(c)
+        if bits == 16:
+            fill_fp16_segment(c, k, v, lens[i])
+        else:
+            fill_cache(kvq, c, k, v, lens[i])
+        segs.append(c)
+        osegs.append(oracle_segment(k, v, bits, G))
+    out, lse = _run(kvq, segs, q)
+    ref, lref = oracle.decode_attention(q_bits(q), False, osegs, lens, 128 ** -0.5)
+    assert_close(out, ref, lse, lref, what="mixed segments")
+
+
+def test_decode_steps_with_append(kvq):
+    """Append one token per sequence, attend, repeat (the decode loop)."""
+    wl = workloads.WORKLOADS["llama3_8b_gqa_int4"].scaled(batch=2, kv_heads=2, q_heads=16)
+    B, ctx = 2, 200
+    k, v = workloads.kv_tokens(wl, ctx, DEV)
+    c = kvq.QuantizedKVCache.allocate(B, 2, 128, 256, 4, 64, DEV)
+    _poison(c)
+    fill_cache(kvq, c, k, v, [ctx, ctx])
+    ks, vs = [k], [v]
+    for step in range(5):
+        kn, vn = workloads.kv_tokens(wl, 1, DEV, stream_extra=1 + step)
+        kvq.kvq_quantize_append(c, kn, vn, 1, advance_seq_lens=True)
+        ks.append(kn)
+        vs.append(vn)
+        q = workloads.queries(wl, DEV, step=step)
+        out, lse = _run(kvq, c, q)
+        seg = oracle_segment(torch.cat(ks, 2), torch.cat(vs, 2), 4, 64)
+        n = ctx + step + 1
+        ref, lref = oracle.decode_attention(q_bits(q), False, [seg], [[n, n]], 128 ** -0.5)
+        assert_close(out, ref, lse, lref, what=f"step {step}")
+    assert c.seq_lens.tolist() == [ctx + 5] * 2
+
+
+def _full_size(kvq, name, pairs, steps=1):
+    """Full-size workload in the benchmark's launch configuration, the oracle
+    evaluated on sampled (sequence, KV head) pairs."""
+    wl = workloads.WORKLOADS[name]
+    B, H, L = wl.batch, wl.kv_heads, wl.context
+    max_tokens = workloads.round_up(L + 64, 64)
+    k, v = workloads.kv_tokens(wl, L, DEV)
+    c = kvq.QuantizedKVCache.allocate(B, H, 128, max_tokens, wl.bits, wl.group, DEV)
+    c.seq_lens.zero_()
+    kvq.kvq_quantize_append(c, k, v, L, advance_seq_lens=True)
+    kn, vn = workloads.kv_tokens(wl, 1, DEV, stream_extra=1)
+    kvq.kvq_quantize_append(c, kn, vn, 1, advance_seq_lens=True)
+    q = workloads.queries(wl, DEV)
+    out, lse = _run(kvq, c, q, max_len_hint=L + 1)
+    g = wl.group_ratio
+    ref = np.full((B, wl.q_heads, 128), np.nan)
+    lref = np.full((B, wl.q_heads), np.nan)
+    mask = np.zeros((B, wl.q_heads), bool)
+    for b, h in pairs:
+        kk = torch.cat([k[b:b + 1, h:h + 1], kn[b:b + 1, h:h + 1]], 2)
+        vv = torch.cat([v[b:b + 1, h:h + 1], vn[b:b + 1, h:h + 1]], 2)
+        seg = oracle_segment(kk, vv, wl.bits, wl.group)
+        qq = q[b:b + 1, h * g:(h + 1) * g]
+        r, lr = oracle.decode_attention(q_bits(qq), q.dtype == torch.bfloat16, [seg], [[L + 1]],
+                                        128 ** -0.5)
+        ref[b, h * g:(h + 1) * g] = r[0]
+        lref[b, h * g:(h + 1) * g] = lr[0]
+        mask[b, h * g:(h + 1) * g] = True
+    assert_close(out, ref, lse, lref, mask=mask, what=name)
+
+
+def test_full_size_llama2_mha_int8_sampled(kvq):
+    _full_size(kvq, "llama2_7b_mha_int8", [(0, 0), (3, 17), (15, 31), (7, 5)])
+
+
+def test_full_size_llama3_gqa_int4_sampled(kvq):
+    _full_size(kvq, "llama3_8b_gqa_int4", [(0, 0), (31, 7), (12, 3)])
+
+
+def test_full_size_long_context_sampled(kvq):
+    _full_size(kvq, "long_gqa_int4", [(0, 0), (0, 5)])
