@@ -44,6 +44,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     p.add_argument("--workload", default="llama2_7b_mha_int8")
+    p.add_argument("--batch", type=int, default=0,
+                   help="override the workload's batch (smaller cases for profiling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     return p.parse_args()
@@ -432,6 +434,8 @@ def main():
     args = parse_args()
     import workloads
     wl = workloads.WORKLOADS[args.workload]
+    if args.batch > 0:
+        wl = wl.scaled(batch=args.batch)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
