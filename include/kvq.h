@@ -214,6 +214,41 @@ kvq_status kvq_decode_merge(const kvq_cache *segs, int32_t n_segs,
                             size_t workspace_bytes, void *stream);
 
 /*
+ * Size of the library-owned scratch array used by
+ * kvq_decode_attention_noalloc (8 MiB on every device that loads the
+ * library, held until the process exits).
+ */
+#define KVQ_STATIC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * kvq_decode_attention for callers that cannot allocate device memory.
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot call cudaMalloc -- a plugin inside a host program that owns and
+ * budgets all device memory, a language binding with no device allocator,
+ * or a latency-critical loop that cannot afford cudaMalloc's implicit
+ * device synchronization.  Same arguments and results as
+ * kvq_decode_attention, minus the workspace: the scratch (split partials
+ * and error word) lives in a fixed array of KVQ_STATIC_SCRATCH_BYTES inside
+ * the library.  The caller still owns q, out, lse and the cache.
+ *  - Returns KVQ_ERR_WORKSPACE, enqueuing nothing, when the request needs
+ *    more scratch than KVQ_STATIC_SCRATCH_BYTES (kvq_decode_workspace_bytes
+ *    with the same arguments tells how much it needs).
+ *  - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *    call.  The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current and caches it; make
+ *    that first call before any stream capture.
+ *  - Every call shares the one array, which keeps the last call's contents
+ *    (the error word is cleared at the start of each call).  Calls whose
+ *    work overlaps on the GPU -- on different streams, or from different
+ *    threads -- race on it; order them.
+ */
+kvq_status kvq_decode_attention_noalloc(const kvq_cache *segs, int32_t n_segs,
+                                        const void *q, kvq_dtype q_dtype,
+                                        int32_t q_heads, float softmax_scale,
+                                        float *out, float *lse,
+                                        int32_t max_len_hint, void *stream);
+
+/*
  * Cocktail chunk-level bit-width search (Cocktail page 3.1.1): for each
  * sequence b and chunk i, sim = (q . c_i) / (||q|| * ||c_i||) in fp64 (sums
  * in index order); T_low and T_high from that sequence's s_min, s_max and

@@ -9,7 +9,7 @@ built libkvq.so raises ImportError (there is no fallback path).
 _BINDING_NAMES = (
     "QuantizedKVCache", "KvqError", "alloc_workspace", "workspace_error_word",
     "kvq_chunk_assign", "kvq_chunk_reorder", "kvq_decode_attention", "kvq_decode_partials",
-    "kvq_decode_merge",
+    "kvq_decode_merge", "kvq_decode_attention_noalloc",
     "kvq_decode_workspace_bytes", "kvq_kv_elements", "kvq_plane_bytes",
     "kvq_quantize_append", "kvq_status_string", "kvq_version",
 )

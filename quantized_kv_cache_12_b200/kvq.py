@@ -63,6 +63,9 @@ def _load():
     lib.kvq_decode_workspace_bytes.argtypes = [cp, i32, i32, i32, ctypes.POINTER(sz)]
     for name in ("kvq_decode_attention", "kvq_decode_partials", "kvq_decode_merge"):
         getattr(lib, name).argtypes = [cp, i32, P, ctypes.c_int, i32, f32, P, P, i32, P, sz, P]
+    lib.kvq_decode_attention_noalloc.argtypes = [cp, i32, P, ctypes.c_int, i32, f32, P, P,
+                                                 i32, P]
+    lib.kvq_decode_attention_noalloc.restype = ctypes.c_int
     lib.kvq_chunk_assign.argtypes = [P, P, i32, i32, i32, f64, f64, P, P, P]
     lib.kvq_chunk_reorder.argtypes = [cp, P, P, i32, i32, P, P, P]
     for name in ("kvq_plane_bytes", "kvq_quantize_append", "kvq_decode_workspace_bytes",
@@ -171,6 +174,20 @@ def kvq_decode_merge(segs, q: torch.Tensor, out: torch.Tensor, lse: Optional[tor
                      max_len_hint: int = 0, stream=None):
     _decode_call(lib.kvq_decode_merge, "kvq_decode_merge", segs, q, out, lse, workspace,
                  softmax_scale, max_len_hint, stream)
+
+
+def kvq_decode_attention_noalloc(segs, q: torch.Tensor, out: torch.Tensor,
+                                 lse: Optional[torch.Tensor], softmax_scale: Optional[float] = None,
+                                 max_len_hint: int = 0, stream=None):
+    """kvq_decode_attention with the library's own fixed scratch array instead
+    of a caller workspace (for callers that cannot allocate device memory)."""
+    arr = _caches(segs)
+    dt = KVQ_BF16 if q.dtype == torch.bfloat16 else KVQ_F16
+    scale = softmax_scale if softmax_scale is not None else q.shape[2] ** -0.5
+    _check(lib.kvq_decode_attention_noalloc(arr, len(arr), _ptr(q), dt, int(q.shape[1]),
+                                            float(scale), _ptr(out), _ptr(lse),
+                                            int(max_len_hint), _stream(stream)),
+           "kvq_decode_attention_noalloc")
 
 
 def kvq_chunk_assign(chunk_emb: torch.Tensor, query_emb: torch.Tensor, alpha: float,
