@@ -170,8 +170,9 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache *segs, int32_t n_segs,
  * (q . k^T / sqrt(dim)); pass softmax_scale = 1/sqrt(head_dim) for it.
  *   segs: 1 segment, or several segments of one mixed-precision cache (same
  *         batch, kv_heads, head_dim; each its own bits, planes, seq_lens).
- *   q: device [batch][q_heads][head_dim] fp16 or bf16 (q_dtype); bf16 values
- *      are used as fp16 (exact for magnitudes in [2^-14, 65504]).
+ *   q: device [batch][q_heads][head_dim] fp16 or bf16 (q_dtype), 16-byte
+ *      aligned; bf16 values are used as fp16 (exact for magnitudes in
+ *      [2^-14, 65504]).
  *   out: device fp32 [batch][q_heads][head_dim]; lse: device fp32
  *        [batch][q_heads] natural log, or NULL.
  *   max_len_hint: an upper bound of the seq_lens used to pick the split

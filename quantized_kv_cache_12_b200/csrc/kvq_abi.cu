@@ -47,18 +47,37 @@ kvq_status check_cache(const kvq_cache* c, bool allow16) {
   return KVQ_OK;
 }
 
-// Split count of one segment: enough CTAs for several waves over 148 SMs,
-// but at least 256 tokens per CTA.
+// Split count of one segment.  A split is one CTA; the decode kernel keeps
+// three CTAs on each of the 148 SMs, so the CTAs run in waves of 444.  The
+// count minimises (waves) x (tokens per CTA + a fixed per-CTA cost of about
+// 96 tokens' worth of work), tokens per CTA being rounded up to the
+// kernel's 128-token granularity, with at least 128 tokens per CTA.  The
+// result depends only on (sequences x KV heads, length), so it is cached
+// per thread.
 int choose_splits(const kvq_cache& c, int max_len_hint) {
   const long long pairs = (long long)c.batch * c.kv_heads;
-  int len = c.max_tokens;
+  long long len = c.max_tokens;
   if (max_len_hint > 0 && max_len_hint < len) len = max_len_hint;
-  const long long target = 148LL * 2 * 6;  // ~6 waves of 2 CTAs per SM
-  long long n = (target + pairs - 1) / pairs;
-  const long long cap = (len + 255) / 256;
-  if (n > cap) n = cap;
-  if (n < 1) n = 1;
-  return (int)n;
+  if (len <= 0 || pairs <= 0) return 1;
+  thread_local long long cached_pairs = -1, cached_len = -1;
+  thread_local int cached_n = 1;
+  if (pairs == cached_pairs && len == cached_len) return cached_n;
+  constexpr long long kSlots = 148LL * 3, kOverhead = 96, kGran = 128;
+  const long long cap = (len + kGran - 1) / kGran;
+  long long best_n = 1, best_cost = -1;
+  for (long long n = 1; n <= cap && n <= 2048; ++n) {
+    const long long chunk = ((len + n - 1) / n + kGran - 1) / kGran * kGran;
+    const long long waves = (pairs * n + kSlots - 1) / kSlots;
+    const long long cost = waves * (chunk + kOverhead);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_n = n;
+    }
+  }
+  cached_pairs = pairs;
+  cached_len = len;
+  cached_n = (int)best_n;
+  return cached_n;
 }
 
 struct SplitPlan {
@@ -194,7 +213,7 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
                          size_t workspace_bytes, void* stream, int stages) {
   kvq_status st = check_segments(segs, n_segs, q_heads);
   if (st != KVQ_OK) return st;
-  if (q == nullptr || out == nullptr) return KVQ_ERR_INVALID_ARG;
+  if (q == nullptr || out == nullptr || !aligned16(q)) return KVQ_ERR_INVALID_ARG;
   if (q_dtype != KVQ_F16 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
   for (int i = 0; i < n_segs; ++i)

@@ -24,6 +24,9 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <atomic>
+#include <type_traits>
+
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
@@ -42,13 +45,31 @@ struct Cfg {
   static constexpr int VC = (GE / 8) * BITS / 8;       // V bytes per lane per group
   static constexpr int VW = VC >= 4 ? VC / 4 : 1;      // V words per lane per group
   static constexpr int NTG = GE / 8;                   // PV n-tiles per group
-  static constexpr int STAGE = 2 * kTile * RB + 2 * kTile * MB;
-  static constexpr int STAGES_RAW = 20480 / STAGE;
+  static constexpr int SUB = (BITS == 16) ? 1 : 2;          // 16-token sub-tiles per stage
+  static constexpr int STOK = SUB * kTile;                   // tokens per stage
+  static constexpr int STAGE = 2 * STOK * RB + 2 * STOK * MB;
+  static constexpr int MF_FLOATS = 2 * kTile * NG * 2;       // fp32 (s, z) of a sub-tile
+  // header: mbarriers (<= 512 B), q rows as fp16 (<= 8 x 128), group sums,
+  // the A fragments of all 32 lane positions (8 x 32 x 16 B)
+  static constexpr int HDR_BARS = 0, HDR_Q = 512, HDR_QS = 512 + 8 * kHeadDim * 2;
+  static constexpr int HDR_QF = HDR_QS + 128;
+  static constexpr int HDR_MF = HDR_QF + 8 * 32 * 16;        // per-warp fp32 meta
+  static constexpr int HDR_BYTES = HDR_MF + kWarps * MF_FLOATS * 4;
+  // as many stages as fit in a budget that keeps three CTAs on an SM
+  // (3 x (74 KB + 1 KB reserved) <= 228 KB)
+  static constexpr int SMEM_BUDGET = 74 * 1024;
+  static constexpr int STAGES_RAW = (SMEM_BUDGET - HDR_BYTES) / (kWarps * STAGE);
   static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 16 ? 16 : STAGES_RAW);
-  static constexpr int BAR_BYTES = 1024;
-  static constexpr int SMEM = BAR_BYTES + kWarps * STAGES * STAGE;
+  static constexpr int SMEM = HDR_BYTES + kWarps * STAGES * STAGE;
   static constexpr int CROSS = (BITS == 16) ? 2 : (BITS == 8 ? 4 : (BITS == 4 ? 8 : 16));
+  static constexpr int PER_W = (NTG < CROSS) ? NTG : CROSS;  // V n-tiles per word
+  static constexpr int EMAX = WordPairs<BITS>::kEmax;
 };
+
+// 2^n as an exact float constant (|n| <= 60).
+__host__ __device__ constexpr float pow2f(int n) {
+  return n >= 0 ? float(1ull << (n > 60 ? 60 : n)) : 1.0f / float(1ull << (-n > 60 ? 60 : -n));
+}
 
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return h2_as_u32(__floats2half2_rn(a, b));
@@ -80,10 +101,20 @@ struct SplitParams {
   SegView seg;
 };
 
-template <int BITS, int GE>
+// Token order inside an 8-token n-tile: MMA column n reads token row
+// rho(n) = n ^ ((n >> 1) & 1) = 0 1 3 2 4 5 7 6.  Softmax and attention do
+// not depend on token order; this order keeps the 16-byte K loads free of
+// shared-memory bank conflicts and halves those of the V loads (the four
+// rows a V load instruction touches alternate between the two 64-byte
+// halves of a bank window).
+__device__ __forceinline__ int rho(int n) { return n ^ ((n >> 1) & 1); }
+
+template <int BITS, int GE, int GR>
 __global__ void __launch_bounds__(kWarps * 32)
 decode_split_kernel(const __grid_constant__ SplitParams P) {
   using C = Cfg<BITS, GE>;
+  using WP = WordPairs<BITS>;
+  using XP = CrossPairs<BITS>;
   constexpr int D = C::D;
   const DecodeArgs& a = P.a;
   const SegView& seg = P.seg;
@@ -93,91 +124,140 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   const int lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int g = a.group_ratio;
-  const int R = C::NG * g;  // valid MMA rows (group, head)
+  constexpr int g = GR;                  // query heads per KV head: 1, 2, 4 or 8
+  constexpr int lg = GR == 1 ? 0 : (GR == 2 ? 1 : (GR == 4 ? 2 : 3));
+  constexpr int R = C::NG * g;           // valid MMA rows (group, head)
+  static_assert(R <= 16, "at most 16 (group, head) rows");
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem) + warp * C::STAGES;
-  uint8_t* stages = smem + C::BAR_BYTES + warp * C::STAGES * C::STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::HDR_BARS) + warp * C::STAGES;
+  __half* q_sm = reinterpret_cast<__half*>(smem + C::HDR_Q);      // [g][D]
+  float* qs_sm = reinterpret_cast<float*>(smem + C::HDR_QS);      // [R]
+  uint4* qf_sm = reinterpret_cast<uint4*>(smem + C::HDR_QF);      // [8][32 lanes]
+  float2* mf = reinterpret_cast<float2*>(smem + C::HDR_MF) + warp * (C::MF_FLOATS / 2);
+  uint8_t* stages = smem + C::HDR_BYTES + warp * C::STAGES * C::STAGE;
 
-  // ---- token range of this warp
+  // ---- token range of this warp (a multiple of the stage size, so a
+  // stage's copy never runs past round_up(seq_len, 32) <= max_tokens)
   int L = seg.seq_lens[b];
   L = max(0, min(L, seg.max_tokens));
   const int per_split = (L + seg.n_split - 1) / seg.n_split;
-  const int chunk = ((per_split + 63) / 64) * 64;
+  const int chunk = ((per_split + 127) / 128) * 128;
   const int c0 = split * chunk;
   const int c1 = min(c0 + chunk, L);
   const int wq = chunk / kWarps;
   const int w0 = c0 + warp * wq;
   const int w1 = min(w0 + wq, c1);
-  const int n_tiles = (w1 > w0) ? (w1 - w0 + kTile - 1) / kTile : 0;
-  const long long row0 = ((long long)b * a.kv_heads + kvh) * seg.max_tokens;
+  const int n_tiles = (w1 > w0) ? (w1 - w0 + C::STOK - 1) / C::STOK : 0;
 
   const uint64_t policy = l2_evict_first_policy();
-  auto issue = [&](int i) {
-    const int st = i % C::STAGES;
+  const uint8_t* kc_src = seg.k_codes + (((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0) * C::RB;
+  const uint8_t* vc_src = seg.v_codes + (((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0) * C::RB;
+  const uint8_t* km_src = seg.k_meta + (((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0) * C::MB;
+  const uint8_t* vm_src = seg.v_meta + (((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0) * C::MB;
+  // copy tile `i` into stage `st` (lane 0 only)
+  auto issue = [&](int i, int st) {
     uint8_t* dst = stages + st * C::STAGE;
-    const long long row = row0 + w0 + (long long)i * kTile;
     mbar_arrive_expect_tx(&bars[st], C::STAGE);
-    bulk_load(dst, seg.k_codes + row * C::RB, kTile * C::RB, &bars[st], policy);
-    bulk_load(dst + kTile * C::RB, seg.v_codes + row * C::RB, kTile * C::RB, &bars[st], policy);
+    bulk_load(dst, kc_src + (size_t)i * (C::STOK * C::RB), C::STOK * C::RB, &bars[st], policy);
+    bulk_load(dst + C::STOK * C::RB, vc_src + (size_t)i * (C::STOK * C::RB), C::STOK * C::RB,
+              &bars[st], policy);
     if constexpr (C::MB > 0) {
-      bulk_load(dst + 2 * kTile * C::RB, seg.k_meta + row * C::MB, kTile * C::MB, &bars[st],
-                policy);
-      bulk_load(dst + 2 * kTile * C::RB + kTile * C::MB, seg.v_meta + row * C::MB,
-                kTile * C::MB, &bars[st], policy);
+      bulk_load(dst + 2 * C::STOK * C::RB, km_src + (size_t)i * (C::STOK * C::MB),
+                C::STOK * C::MB, &bars[st], policy);
+      bulk_load(dst + 2 * C::STOK * C::RB + C::STOK * C::MB,
+                vm_src + (size_t)i * (C::STOK * C::MB), C::STOK * C::MB, &bars[st], policy);
     }
   };
 
   if (lane == 0) {
     for (int s = 0; s < C::STAGES; ++s) mbar_init(&bars[s], 1);
     fence_barrier_init();
-  }
-  __syncwarp();
-  if (lane == 0) {
     const int pre = min(n_tiles, C::STAGES);
-    for (int i = 0; i < pre; ++i) issue(i);
+    for (int i = 0; i < pre; ++i) issue(i, i);
   }
 
-  // ---- query fragments: row r = gr * g + h holds q_h masked to group gr
-  const __half* qh16 = reinterpret_cast<const __half*>(a.q);
-  const __nv_bfloat16* qb16 = reinterpret_cast<const __nv_bfloat16*>(a.q);
-  const long long qbase = ((long long)b * a.q_heads + (long long)kvh * g) * D;
-  auto qval = [&](int r, int d) -> float {
-    if (r >= R || d / GE != r / g) return 0.0f;
-    const long long i = qbase + (long long)(r % g) * D + d;
-    // bf16 queries are used through fp16 (exact for |q| in [2^-14, 65504])
-    return a.q_is_bf16 ? __half2float(__float2half_rn(__bfloat162float(qb16[i])))
-                       : __half2float(qh16[i]);
-  };
-  using WP = WordPairs<BITS>;
-  auto kdim = [&](int p, int e) -> int {
-    return 32 * tig + (p / WP::kPairs) * WP::kDims + WP::dim(p % WP::kPairs, e);
-  };
+  // ---- the g query rows of this KV head, once per CTA, as fp16 in smem
+  // (bf16 queries are used through fp16: exact for |q| in [2^-14, 65504])
+  const int t = threadIdx.x;
+  {
+    const long long qbase = ((long long)b * a.q_heads + (long long)kvh * g) * D;
+    if (t < g * (D / 8)) {
+      const uint4 raw = reinterpret_cast<const uint4*>(
+          static_cast<const uint16_t*>(a.q) + qbase)[t];
+      uint4 h16 = raw;
+      if (a.q_is_bf16) {
+        const __nv_bfloat162* bb = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        __half2* hh = reinterpret_cast<__half2*>(&h16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) hh[i] = __float22half2_rn(__bfloat1622float2(bb[i]));
+      }
+      reinterpret_cast<uint4*>(q_sm)[t] = h16;
+    }
+  }
+  __syncthreads();
+  // sum of q over each (group, head) row, in the MMA's units (the QK MMA
+  // returns 2^(EMAX - 24) * sum(q * c))
+  if constexpr (BITS != 16) {
+    const int r = t >> 3, part = t & 7;
+    float acc = 0.f;
+    if (r < R) {
+      const __half* qr = q_sm + (r & (g - 1)) * D + (r >> lg) * GE + part * (GE / 8);
+#pragma unroll 4
+      for (int i = 0; i < GE / 8; ++i) acc += __half2float(qr[i]);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if (r < R && part == 0) qs_sm[r] = acc * pow2f(C::EMAX - 24);
+  }
+  // A fragments, built once per CTA for every lane position: row r =
+  // gr * g + h holds q_h masked to group gr, each element scaled by
+  // 2^(EMAX - e) for the subnormal exponent e of the code it meets.
+  // Thread t builds 8 of the 32 registers of lane position t / 4.
+  {
+    const int fl = t >> 2;                 // lane position
+    const int fg = fl >> 2, ft = fl & 3;   // its gid, tig
+    auto qx = [&](int r, int d, int e) -> float {
+      if (r >= R || d / GE != (r >> lg)) return 0.0f;
+      return __half2float(q_sm[(r & (g - 1)) * D + d]) * pow2f(C::EMAX - e);
+    };
+    auto kdim = [&](int pidx, int e) -> int {
+      return 32 * ft + (pidx / WP::kPairs) * WP::kDims + WP::dim(pidx % WP::kPairs, e);
+    };
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {          // this thread: k-steps 2 * (t & 3) + u
+      const int ks = 2 * (t & 3) + u;
+      const int pA = 2 * ks, pB = 2 * ks + 1;
+      const int eA = WP::exp(pA % WP::kPairs), eB = WP::exp(pB % WP::kPairs);
+      uint4 v;
+      v.x = pack_h2(qx(fg, kdim(pA, 0), eA), qx(fg, kdim(pA, 1), eA));
+      v.y = pack_h2(qx(fg + 8, kdim(pA, 0), eA), qx(fg + 8, kdim(pA, 1), eA));
+      v.z = pack_h2(qx(fg, kdim(pB, 0), eB), qx(fg, kdim(pB, 1), eB));
+      v.w = pack_h2(qx(fg + 8, kdim(pB, 0), eB), qx(fg + 8, kdim(pB, 1), eB));
+      qf_sm[ks * 32 + fl] = v;
+    }
+  }
+  __syncthreads();
   uint32_t qf[8][4];
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
-    const int pA = 2 * ks, pB = 2 * ks + 1;
-    qf[ks][0] = pack_h2(qval(gid, kdim(pA, 0)), qval(gid, kdim(pA, 1)));
-    qf[ks][1] = pack_h2(qval(gid + 8, kdim(pA, 0)), qval(gid + 8, kdim(pA, 1)));
-    qf[ks][2] = pack_h2(qval(gid, kdim(pB, 0)), qval(gid, kdim(pB, 1)));
-    qf[ks][3] = pack_h2(qval(gid + 8, kdim(pB, 0)), qval(gid + 8, kdim(pB, 1)));
+    const uint4 v = qf_sm[ks * 32 + lane];
+    qf[ks][0] = v.x; qf[ks][1] = v.y; qf[ks][2] = v.z; qf[ks][3] = v.w;
   }
-  // sum of q over the row's group (for the zero-point term)
-  float qs0 = 0.f, qs1 = 0.f;
-  if constexpr (BITS != 16) {
-    if (gid < R) {
-      const int gr = gid / g;
-      for (int d = gr * GE; d < (gr + 1) * GE; ++d) qs0 += qval(gid, d);
-    }
-    if (gid + 8 < R) {
-      const int gr = (gid + 8) / g;
-      for (int d = gr * GE; d < (gr + 1) * GE; ++d) qs1 += qval(gid + 8, d);
-    }
-  }
-  const int gr0 = (gid < R) ? gid / g : 0;
-  const int gr1 = (gid + 8 < R) ? (gid + 8) / g : 0;
   const bool row0_ok = gid < R, row1_ok = gid + 8 < R;
+  const float qs0 = (BITS != 16 && row0_ok) ? qs_sm[gid] : 0.f;
+  const float qs1 = (BITS != 16 && row1_ok) ? qs_sm[gid + 8] : 0.f;
+  const int gr0 = row0_ok ? (gid >> lg) : 0;
+  const int gr1 = row1_ok ? ((gid + 8) >> lg) : 0;
   const bool head_ok = gid < g;  // this lane's PV rows are a real head
+  // log2-domain softmax scale including the MMA's 2^(24 - EMAX)
+  const float score_scale = a.scale_log2 * pow2f(24 - C::EMAX);
+  // this lane's token rows within a tile: MMA columns 2*tig, 2*tig+1 of the
+  // two n-tiles, in the rho order
+  const int tokA = rho(2 * tig), tokB = rho(2 * tig + 1);
+  const int tokC = 8 + tokA, tokD = 8 + tokB;
+  const int tok4[4] = {tokA, tokB, tokC, tokD};
+  const int krow = rho(gid);  // K row this lane feeds into MMA column gid
 
   // ---- running state (head = gid)
   float o_acc[16][4];
@@ -186,29 +266,44 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   float corr[C::NG];
 #pragma unroll
   for (int i = 0; i < C::NG; ++i) corr[i] = 0.f;
+  // m_run is a reference point, not the exact max: p = 2^(x - m_run) may
+  // reach 2^kLazy before the accumulators are rescaled
+  constexpr float kLazy = 4.0f;
   float m_run = -INFINITY, l_part = 0.f;
   int failed_at = -1;
+  int st = 0;
+  uint32_t phase = 0;
 
-  for (int i = 0; i < n_tiles; ++i) {
-    const int st = i % C::STAGES;
-    if (!mbar_wait_bounded(&bars[st], (i / C::STAGES) & 1, 1u << 22)) {
-      failed_at = i;
-      break;
+  // one 16-token sub-tile: QK^T, online softmax, PV.  FULL = all 16 tokens
+  // valid (no masking work).
+  auto sub_tile = [&](auto full_tag, const uint8_t* sK, const uint8_t* sV, const uint8_t* sKm,
+                      const uint8_t* sVm, int n_valid) {
+    constexpr bool FULL = decltype(full_tag)::value;
+    auto valid = [&](int tok) { return FULL || tok < n_valid; };
+
+    // (s, z) of the sub-tile's K and V rows to fp32, once per warp: each
+    // lane converts NG pairs, every lane then reads the ones it needs
+    if constexpr (BITS != 16) {
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < C::NG; ++j) {
+        const int idx = lane * C::NG + j;  // 0 .. 32 * NG - 1
+        const int plane = idx >= kTile * C::NG;
+        const __half2* src = reinterpret_cast<const __half2*>(plane ? sVm : sKm);
+        mf[idx] = __half22float2(src[idx - plane * kTile * C::NG]);
+      }
+      __syncwarp();
     }
-    const uint8_t* sK = stages + st * C::STAGE;
-    const uint8_t* sV = sK + kTile * C::RB;
-    const uint8_t* sKm = sK + 2 * kTile * C::RB;
-    const uint8_t* sVm = sKm + kTile * C::MB;
-    const int t0 = w0 + i * kTile;
-    const int n_valid = min(kTile, w1 - t0);
 
-    // ---- S = Qx * K^T for the two 8-token n-tiles
-    float s_acc[2][4];
+    // ---- S = Qx * K^T for the two 8-token n-tiles (two MMA chains each)
+    float s_acc[2][2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      s_acc[nt][0] = s_acc[nt][1] = s_acc[nt][2] = s_acc[nt][3] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        s_acc[nt][c][0] = s_acc[nt][c][1] = s_acc[nt][c][2] = s_acc[nt][c][3] = 0.f;
       uint32_t kw[C::KW];
-      load_chunk<C::KC, C::KW>(sK + (nt * 8 + gid) * C::RB + tig * C::KC, kw);
+      load_chunk<C::KC, C::KW>(sK + (nt * 8 + krow) * C::RB + tig * C::KC, kw);
       uint32_t pr[16];
 #pragma unroll
       for (int w = 0; w < C::KW; ++w) {
@@ -219,33 +314,24 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
       }
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        mma_f16(s_acc[nt], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], pr[2 * ks],
+        mma_f16(s_acc[nt][ks & 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], pr[2 * ks],
                 pr[2 * ks + 1]);
     }
 
-    // ---- scores of head (gid mod g) for tokens nt*8 + 2*tig + e
+    // ---- scores of head (gid mod g) for this lane's four tokens.  Rows
+    // past R hold zero queries (S = 0, qs = 0), so they add nothing.
     float sc[4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int tok = nt * 8 + 2 * tig + e;
-        float c;
-        if constexpr (BITS == 16) {
-          c = row0_ok ? s_acc[nt][e] : 0.f;
-        } else {
-          const __half2* m = reinterpret_cast<const __half2*>(sKm + tok * C::MB);
-          c = 0.f;
-          if (row0_ok) {
-            const float2 sz = __half22float2(m[gr0]);
-            c = sz.x * (s_acc[nt][e] - sz.y * qs0);
-          }
-          if (row1_ok) {
-            const float2 sz = __half22float2(m[gr1]);
-            c += sz.x * (s_acc[nt][2 + e] - sz.y * qs1);
-          }
-        }
-        sc[nt * 2 + e] = c;
+    for (int k = 0; k < 4; ++k) {
+      const int nt = k >> 1, e = k & 1;
+      const float S0 = s_acc[nt][0][e] + s_acc[nt][1][e];
+      if constexpr (BITS == 16) {
+        sc[k] = S0;
+      } else {
+        const float S1 = s_acc[nt][0][2 + e] + s_acc[nt][1][2 + e];
+        const float2 sz0 = mf[tok4[k] * C::NG + gr0];
+        const float2 sz1 = mf[tok4[k] * C::NG + gr1];
+        sc[k] = fmaf(sz1.x, fmaf(-sz1.y, qs1, S1), sz0.x * fmaf(-sz0.y, qs0, S0));
       }
     }
     // sum the group rows of each head: lanes gid and gid ^ m (m >= g)
@@ -259,14 +345,15 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
     float tmax = -INFINITY;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const int tok = (k >> 1) * 8 + 2 * tig + (k & 1);
-      sc[k] = (tok < n_valid) ? sc[k] * a.scale_log2 : -INFINITY;
+      sc[k] = valid(tok4[k]) ? sc[k] * score_scale : -INFINITY;
       tmax = fmaxf(tmax, sc[k]);
     }
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-    if (tmax > m_run) {  // new running max: rescale what was accumulated
-      const float alpha = exp2f(m_run - tmax);  // 0 when m_run = -inf
+    if (m_run == -INFINITY) {
+      m_run = tmax;  // nothing accumulated yet: no rescale needed
+    } else if (tmax > m_run + kLazy) {
+      const float alpha = fast_exp2(m_run - tmax);
 #pragma unroll
       for (int n = 0; n < 16; ++n)
 #pragma unroll
@@ -279,13 +366,11 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
     float p[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      p[k] = (m_run == -INFINITY) ? 0.f : exp2f(sc[k] - m_run);
-      if (!head_ok) p[k] = 0.f;
+      p[k] = head_ok ? fast_exp2(sc[k] - m_run) : 0.f;  // 0 for masked tokens
       l_part += p[k];
     }
 
     // ---- O += P' * V per group (hi rows gid, lo rows gid + 8)
-    const int tokA = 2 * tig, tokB = 2 * tig + 1, tokC = 8 + 2 * tig, tokD = 9 + 2 * tig;
 #pragma unroll
     for (int gr = 0; gr < C::NG; ++gr) {
       float pp[4];
@@ -293,29 +378,23 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) pp[k] = p[k];
       } else {
-        const int toks[4] = {tokA, tokB, tokC, tokD};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           // slots past the valid length may hold any bytes (NaN scales):
           // select, never multiply by a zero weight
-          const bool valid = toks[k] < n_valid;
-          const float2 sz =
-              __half22float2(reinterpret_cast<const __half2*>(sVm + toks[k] * C::MB)[gr]);
-          pp[k] = valid ? p[k] * sz.x : 0.f;
-          corr[gr] += valid ? pp[k] * sz.y : 0.f;
+          const float2 sz = mf[kTile * C::NG + tok4[k] * C::NG + gr];
+          pp[k] = valid(tok4[k]) ? p[k] * sz.x : 0.f;
+          corr[gr] = valid(tok4[k]) ? fmaf(pp[k], sz.y, corr[gr]) : corr[gr];
         }
       }
-      __half hi[4];
-      float lo[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        hi[k] = __float2half_rn(pp[k]);
-        lo[k] = pp[k] - __half2float(hi[k]);
-      }
-      const uint32_t a0 = h2_as_u32(__halves2half2(hi[0], hi[1]));
-      const uint32_t a1 = pack_h2(lo[0], lo[1]);
-      const uint32_t a2 = h2_as_u32(__halves2half2(hi[2], hi[3]));
-      const uint32_t a3 = pack_h2(lo[2], lo[3]);
+      const __half2 h01 = __floats2half2_rn(pp[0], pp[1]);
+      const __half2 h23 = __floats2half2_rn(pp[2], pp[3]);
+      const float2 f01 = __half22float2(h01);
+      const float2 f23 = __half22float2(h23);
+      const uint32_t a0 = h2_as_u32(h01);
+      const uint32_t a1 = pack_h2(pp[0] - f01.x, pp[1] - f01.y);
+      const uint32_t a2 = h2_as_u32(h23);
+      const uint32_t a3 = pack_h2(pp[2] - f23.x, pp[3] - f23.y);
 
       const uint8_t* vbase = sV + gr * (GE * BITS / 8) + gid * C::VC;
       uint32_t wA[C::VW], wB[C::VW], wC[C::VW], wD[C::VW];
@@ -323,31 +402,57 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
       load_chunk<C::VC, C::VW>(vbase + tokB * C::RB, wB);
       load_chunk<C::VC, C::VW>(vbase + tokC * C::RB, wC);
       load_chunk<C::VC, C::VW>(vbase + tokD * C::RB, wD);
-      if constexpr (BITS == 16) {
+      if constexpr (BITS == 16 && !FULL) {
         // raw fp16 rows past the valid length may hold anything: zero them
-        if (n_valid < kTile) {
 #pragma unroll
-          for (int w = 0; w < C::VW; ++w) {
-            if (tokA >= n_valid) wA[w] = 0u;
-            if (tokB >= n_valid) wB[w] = 0u;
-            if (tokC >= n_valid) wC[w] = 0u;
-            if (tokD >= n_valid) wD[w] = 0u;
-          }
+        for (int w = 0; w < C::VW; ++w) {
+          wA[w] = valid(tokA) ? wA[w] : 0u;
+          wB[w] = valid(tokB) ? wB[w] : 0u;
+          wC[w] = valid(tokC) ? wC[w] : 0u;
+          wD[w] = valid(tokD) ? wD[w] : 0u;
         }
       }
 #pragma unroll
       for (int w = 0; w < C::VW; ++w) {
         uint32_t x[C::CROSS], y[C::CROSS];
-        CrossPairs<BITS>::run(wA[w], wB[w], x);
-        CrossPairs<BITS>::run(wC[w], wD[w], y);
-        constexpr int PER_W = (C::NTG < C::CROSS) ? C::NTG : C::CROSS;
+        XP::run(wA[w], wB[w], x);
+        XP::run(wC[w], wD[w], y);
 #pragma unroll
-        for (int j = 0; j < PER_W; ++j)
-          mma_f16(o_acc[gr * C::NTG + w * PER_W + j], a0, a1, a2, a3, x[j], y[j]);
+        for (int j = 0; j < C::PER_W; ++j)
+          mma_f16(o_acc[gr * C::NTG + w * C::PER_W + j], a0, a1, a2, a3, x[j], y[j]);
       }
     }
+  };
+
+  for (int i = 0; i < n_tiles; ++i) {
+    if (!mbar_wait_bounded(&bars[st], phase, 1u << 22)) {
+      failed_at = i;
+      break;
+    }
+    const uint8_t* sK = stages + st * C::STAGE;
+    const uint8_t* sV = sK + C::STOK * C::RB;
+    const uint8_t* sKm = sK + 2 * C::STOK * C::RB;
+    const uint8_t* sVm = sKm + C::STOK * C::MB;
+    const int n_stage = min(C::STOK, w1 - (w0 + i * C::STOK));
+#pragma unroll
+    for (int sub = 0; sub < C::SUB; ++sub) {
+      const int nv = n_stage - sub * kTile;
+      if (nv <= 0) break;
+      const uint8_t* k_sub = sK + sub * kTile * C::RB;
+      const uint8_t* v_sub = sV + sub * kTile * C::RB;
+      const uint8_t* km_sub = sKm + sub * kTile * C::MB;
+      const uint8_t* vm_sub = sVm + sub * kTile * C::MB;
+      if (nv >= kTile)
+        sub_tile(std::integral_constant<bool, true>(), k_sub, v_sub, km_sub, vm_sub, kTile);
+      else
+        sub_tile(std::integral_constant<bool, false>(), k_sub, v_sub, km_sub, vm_sub, nv);
+    }
     __syncwarp();
-    if (lane == 0 && i + C::STAGES < n_tiles) issue(i + C::STAGES);
+    if (lane == 0 && i + C::STAGES < n_tiles) issue(i + C::STAGES, st);
+    if (++st == C::STAGES) {
+      st = 0;
+      phase ^= 1u;
+    }
   }
 
   if (failed_at >= 0) {
@@ -369,7 +474,7 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
 
   // ---- merge the 4 warps in shared memory (reusing the stage buffers)
   __syncthreads();
-  float* ms = reinterpret_cast<float*>(smem + C::BAR_BYTES);  // [kWarps][8]
+  float* ms = reinterpret_cast<float*>(smem + C::HDR_BYTES);  // [kWarps][8]
   float* ls = ms + kWarps * 8;                                 // [kWarps][8]
   float* os = ls + kWarps * 8;                                 // [kWarps][8][D]
   if (head_ok) {
@@ -383,12 +488,13 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
       const int gr = nt / C::NTG, jj = nt % C::NTG;
       const int d0 = gr * GE + (2 * tig) * C::NTG + jj;
       const int d1 = d0 + C::NTG;
-      oh[d0] = o_acc[nt][0] + o_acc[nt][2] - corr[gr];
-      oh[d1] = o_acc[nt][1] + o_acc[nt][3] - corr[gr];
+      // undo the subnormal code scale 2^(e - 24) of this column
+      const float f = pow2f(24 - XP::exp(jj));
+      oh[d0] = fmaf(o_acc[nt][0] + o_acc[nt][2], f, -corr[gr]);
+      oh[d1] = fmaf(o_acc[nt][1] + o_acc[nt][3], f, -corr[gr]);
     }
   }
   __syncthreads();
-  const int t = threadIdx.x;  // one output dim per thread
   const int part = seg.part_base + split;
   for (int h = 0; h < g; ++h) {
     float M = -INFINITY;
@@ -423,44 +529,87 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
 }
 
 // Merge the partial (m, l, o) of every split and segment (log-sum-exp).
+// One CTA per (sequence, query head); the 128 threads first reduce the max
+// and the weights over the partials together, then each thread sums one
+// output dim over the partials.
 __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs a) {
+  extern __shared__ float w_sm[];  // [parts] weights 2^(m_p - M)
+  __shared__ float red[kHeadDim / 32];
   const long long bh = blockIdx.x;
-  const int t = threadIdx.x;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const float* ml = a.part_ml + bh * a.parts * 2;
   const float* po = a.part_o + bh * a.parts * kHeadDim;
-  float M = -INFINITY;
-  for (int p = 0; p < a.parts; ++p)
-    if (ml[2 * p + 1] > 0.f) M = fmaxf(M, ml[2 * p]);
-  float L = 0.f, O = 0.f;
-  if (M != -INFINITY) {
-    for (int p = 0; p < a.parts; ++p) {
-      const float l = ml[2 * p + 1];
-      if (l > 0.f) {
-        const float w = exp2f(ml[2 * p] - M);
-        L += w * l;
-        O += w * po[(long long)p * kHeadDim + t];
-      }
-    }
+  float m = -INFINITY;
+  for (int p = t; p < a.parts; p += kHeadDim)
+    if (ml[2 * p + 1] > 0.f) m = fmaxf(m, ml[2 * p]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  float l = 0.f;
+  for (int p = t; p < a.parts; p += kHeadDim) {
+    const float lp = ml[2 * p + 1];
+    const float w = (lp > 0.f && M != -INFINITY) ? exp2f(ml[2 * p] - M) : 0.f;
+    w_sm[p] = w;
+    l += w * lp;
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (lane == 0) red[warp] = l;
+  __syncthreads();
+  const float L = red[0] + red[1] + red[2] + red[3];
+  float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
+  int p = 0;
+  for (; p + 4 <= a.parts; p += 4) {
+    O0 = fmaf(w_sm[p], po[(long long)p * kHeadDim + t], O0);
+    O1 = fmaf(w_sm[p + 1], po[(long long)(p + 1) * kHeadDim + t], O1);
+    O2 = fmaf(w_sm[p + 2], po[(long long)(p + 2) * kHeadDim + t], O2);
+    O3 = fmaf(w_sm[p + 3], po[(long long)(p + 3) * kHeadDim + t], O3);
+  }
+  for (; p < a.parts; ++p) O0 = fmaf(w_sm[p], po[(long long)p * kHeadDim + t], O0);
+  const float O = (O0 + O1) + (O2 + O3);
   a.out[bh * kHeadDim + t] = (L > 0.f) ? O / L : 0.f;
   if (a.lse != nullptr && t == 0)
     a.lse[bh] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
-template <int BITS, int GE>
-cudaError_t launch_split(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
+template <int BITS, int GE, int GR>
+cudaError_t launch_split_g(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   using C = Cfg<BITS, GE>;
-  static bool attr_set = false;  // per process; harmless to repeat
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<BITS, GE>,
+  // the shared-memory opt-in is a per-device function attribute: set it once
+  // per device (bit i of the mask = device i)
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set.load() & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<BITS, GE, GR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set.fetch_or(bit);
   }
   SplitParams P{a, seg};
   dim3 grid(seg.n_split, a.kv_heads, a.batch);
-  decode_split_kernel<BITS, GE><<<grid, kWarps * 32, C::SMEM, s>>>(P);
+  decode_split_kernel<BITS, GE, GR><<<grid, kWarps * 32, C::SMEM, s>>>(P);
   return cudaGetLastError();
+}
+
+template <int BITS, int GE>
+cudaError_t launch_split(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
+  constexpr int NG = kHeadDim / GE;
+  switch (a.group_ratio) {
+    case 1: return launch_split_g<BITS, GE, 1>(a, seg, s);
+    case 2: return launch_split_g<BITS, GE, 2>(a, seg, s);
+    case 4:
+      if constexpr (NG * 4 <= 16) return launch_split_g<BITS, GE, 4>(a, seg, s);
+      break;
+    case 8:
+      if constexpr (NG * 8 <= 16) return launch_split_g<BITS, GE, 8>(a, seg, s);
+      break;
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -498,7 +647,13 @@ cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaS
 }
 
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s) {
-  decode_merge_kernel<<<(unsigned)((long long)a.batch * a.q_heads), kHeadDim, 0, s>>>(a);
+  const size_t smem = (size_t)a.parts * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(decode_merge_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  decode_merge_kernel<<<(unsigned)((long long)a.batch * a.q_heads), kHeadDim, smem, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -99,84 +99,77 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
   return r;
 }
-// (x & mask) | base in one LOP3.
-__device__ __forceinline__ uint32_t and_or(uint32_t x, uint32_t mask, uint32_t base) {
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(mask), "r"(base));
-  return r;
-}
-// Exact fp16 subtraction of the conversion offset (both halves).
-__device__ __forceinline__ uint32_t hsub_u32(uint32_t x, uint32_t off) {
-  return h2_as_u32(__hsub2(u32_as_h2(x), u32_as_h2(off)));
-}
-
 // ---------------------------------------------------------------- code -> fp16
-// Integer codes become exact fp16 values by writing them into the mantissa
-// of a power of two whose unit in the last place is 1 for that bit field
-// (bits 0-1 of a half: 1024 = 0x6400; bits 2-3: 256 = 0x5C00; bits 4-5:
-// 64 = 0x5400; bits 6-7: 16 = 0x4C00), then subtracting the power of two,
-// which is exact.
+// A b-bit code masked in place into mantissa bits 0..9 of a half is already
+// an exact fp16 value: the subnormal code * 2^(e - 24), where e is the bit
+// offset of the field (a code at bits 4..7 is code * 2^-20).  The tensor
+// cores multiply fp16 subnormals exactly, so the conversion is one AND per
+// pair of codes; the power-of-two factors are folded into the (exact,
+// power-of-two scaled) query operand and into the output scale.
 //
 // Pairs of one token (K side): a 32-bit word of packed codes of consecutive
-// dims yields half2 pairs; the pair -> dim order is fixed by
-//   INT4 word (dims 0..7):  pair j (0..3) = dims (j, j + 4)
-//   INT2 word (dims 0..15): pair j (0..7) = dims (j, j + 8)
-//   INT8 word (dims 0..3):  pair j (0..1) = dims (2j, 2j + 1)
-//   FP16 word (dims 0..1):  the word itself
+// dims yields half2 pairs (kPairs of them, covering kDims dims):
+//   INT4 word (dims 0..7):  pair j (0..3) = dims (j, j + 4), e = 4 * (j & 1)
+//   INT2 word (dims 0..15): pair j (0..7) = dims (j, j + 8), e = 2 * (j & 3)
+//   INT8 word (dims 0..3):  pair j (0..1) = dims (j, j + 2), e = 0
+//   FP16 word (dims 0..1):  the word itself, e = 24 (factor 1)
 template <int BITS>
 struct WordPairs;
 
 template <>
 struct WordPairs<4> {
-  static constexpr int kPairs = 4, kDims = 8;
+  static constexpr int kPairs = 4, kDims = 8, kEmax = 4;
   __device__ __forceinline__ static void run(uint32_t w, uint32_t (&p)[4]) {
     const uint32_t w8 = w >> 8;
-    p[0] = hsub_u32(and_or(w, 0x000F000Fu, 0x64006400u), 0x64006400u);
-    p[1] = hsub_u32(and_or(w, 0x00F000F0u, 0x54005400u), 0x54005400u);
-    p[2] = hsub_u32(and_or(w8, 0x000F000Fu, 0x64006400u), 0x64006400u);
-    p[3] = hsub_u32(and_or(w8, 0x00F000F0u, 0x54005400u), 0x54005400u);
+    p[0] = w & 0x000F000Fu;
+    p[1] = w & 0x00F000F0u;
+    p[2] = w8 & 0x000F000Fu;
+    p[3] = w8 & 0x00F000F0u;
   }
-  __device__ __forceinline__ static int dim(int j, int e) { return j + 4 * e; }
+  __host__ __device__ static constexpr int dim(int j, int e) { return j + 4 * e; }
+  __host__ __device__ static constexpr int exp(int j) { return 4 * (j & 1); }
 };
 
 template <>
 struct WordPairs<2> {
-  static constexpr int kPairs = 8, kDims = 16;
+  static constexpr int kPairs = 8, kDims = 16, kEmax = 6;
   __device__ __forceinline__ static void run(uint32_t w, uint32_t (&p)[8]) {
     const uint32_t w8 = w >> 8;
-    p[0] = hsub_u32(and_or(w, 0x00030003u, 0x64006400u), 0x64006400u);
-    p[1] = hsub_u32(and_or(w, 0x000C000Cu, 0x5C005C00u), 0x5C005C00u);
-    p[2] = hsub_u32(and_or(w, 0x00300030u, 0x54005400u), 0x54005400u);
-    p[3] = hsub_u32(and_or(w, 0x00C000C0u, 0x4C004C00u), 0x4C004C00u);
-    p[4] = hsub_u32(and_or(w8, 0x00030003u, 0x64006400u), 0x64006400u);
-    p[5] = hsub_u32(and_or(w8, 0x000C000Cu, 0x5C005C00u), 0x5C005C00u);
-    p[6] = hsub_u32(and_or(w8, 0x00300030u, 0x54005400u), 0x54005400u);
-    p[7] = hsub_u32(and_or(w8, 0x00C000C0u, 0x4C004C00u), 0x4C004C00u);
+    p[0] = w & 0x00030003u;
+    p[1] = w & 0x000C000Cu;
+    p[2] = w & 0x00300030u;
+    p[3] = w & 0x00C000C0u;
+    p[4] = w8 & 0x00030003u;
+    p[5] = w8 & 0x000C000Cu;
+    p[6] = w8 & 0x00300030u;
+    p[7] = w8 & 0x00C000C0u;
   }
-  __device__ __forceinline__ static int dim(int j, int e) { return j + 8 * e; }
+  __host__ __device__ static constexpr int dim(int j, int e) { return j + 8 * e; }
+  __host__ __device__ static constexpr int exp(int j) { return 2 * (j & 3); }
 };
 
 template <>
 struct WordPairs<8> {
-  static constexpr int kPairs = 2, kDims = 4;
+  static constexpr int kPairs = 2, kDims = 4, kEmax = 0;
   __device__ __forceinline__ static void run(uint32_t w, uint32_t (&p)[2]) {
-    p[0] = hsub_u32(prmt(w, 0x64646464u, 0x4140u), 0x64006400u);
-    p[1] = hsub_u32(prmt(w, 0x64646464u, 0x4342u), 0x64006400u);
+    p[0] = w & 0x00FF00FFu;
+    p[1] = (w >> 8) & 0x00FF00FFu;
   }
-  __device__ __forceinline__ static int dim(int j, int e) { return 2 * j + e; }
+  __host__ __device__ static constexpr int dim(int j, int e) { return j + 2 * e; }
+  __host__ __device__ static constexpr int exp(int) { return 0; }
 };
 
 template <>
 struct WordPairs<16> {
-  static constexpr int kPairs = 1, kDims = 2;
+  static constexpr int kPairs = 1, kDims = 2, kEmax = 24;
   __device__ __forceinline__ static void run(uint32_t w, uint32_t (&p)[1]) { p[0] = w; }
-  __device__ __forceinline__ static int dim(int j, int e) { return e; }
+  __host__ __device__ static constexpr int dim(int, int e) { return e; }
+  __host__ __device__ static constexpr int exp(int) { return 24; }
 };
 
 // Pairs across two tokens (V side): words a (token A) and b (token B) hold
 // the same dims; out[i] = half2(code_A[dim i], code_B[dim i]) for the dims of
-// the low 16 bits (INT4: 4 dims, INT2: 8 dims, INT8: 2 dims, FP16: 1 dim)
-// and of the high 16 bits (the same count again), in dim order.
+// the word in order, with the subnormal exponent exp(i).
 template <int BITS>
 struct CrossPairs;
 
@@ -184,48 +177,51 @@ template <>
 struct CrossPairs<4> {
   static constexpr int kOut = 8;  // dims per 32-bit word
   __device__ __forceinline__ static void run(uint32_t a, uint32_t b, uint32_t (&o)[8]) {
-    uint32_t x = prmt(a, b, 0x5410u);  // [a.b0 a.b1 b.b0 b.b1]
-    uint32_t y = prmt(a, b, 0x7632u);  // [a.b2 a.b3 b.b2 b.b3]
-    uint32_t x8 = x >> 8, y8 = y >> 8;
-    o[0] = hsub_u32(and_or(x, 0x000F000Fu, 0x64006400u), 0x64006400u);
-    o[1] = hsub_u32(and_or(x, 0x00F000F0u, 0x54005400u), 0x54005400u);
-    o[2] = hsub_u32(and_or(x8, 0x000F000Fu, 0x64006400u), 0x64006400u);
-    o[3] = hsub_u32(and_or(x8, 0x00F000F0u, 0x54005400u), 0x54005400u);
-    o[4] = hsub_u32(and_or(y, 0x000F000Fu, 0x64006400u), 0x64006400u);
-    o[5] = hsub_u32(and_or(y, 0x00F000F0u, 0x54005400u), 0x54005400u);
-    o[6] = hsub_u32(and_or(y8, 0x000F000Fu, 0x64006400u), 0x64006400u);
-    o[7] = hsub_u32(and_or(y8, 0x00F000F0u, 0x54005400u), 0x54005400u);
+    const uint32_t x = prmt(a, b, 0x5410u);  // [a.b0 a.b1 b.b0 b.b1]
+    const uint32_t y = prmt(a, b, 0x7632u);  // [a.b2 a.b3 b.b2 b.b3]
+    const uint32_t x8 = x >> 8, y8 = y >> 8;
+    o[0] = x & 0x000F000Fu;
+    o[1] = x & 0x00F000F0u;
+    o[2] = x8 & 0x000F000Fu;
+    o[3] = x8 & 0x00F000F0u;
+    o[4] = y & 0x000F000Fu;
+    o[5] = y & 0x00F000F0u;
+    o[6] = y8 & 0x000F000Fu;
+    o[7] = y8 & 0x00F000F0u;
   }
+  __host__ __device__ static constexpr int exp(int i) { return 4 * (i & 1); }
 };
 
 template <>
 struct CrossPairs<2> {
   static constexpr int kOut = 16;
   __device__ __forceinline__ static void run(uint32_t a, uint32_t b, uint32_t (&o)[16]) {
-    uint32_t x = prmt(a, b, 0x5410u);
-    uint32_t y = prmt(a, b, 0x7632u);
-    uint32_t v[4] = {x, x >> 8, y, y >> 8};
+    const uint32_t x = prmt(a, b, 0x5410u);
+    const uint32_t y = prmt(a, b, 0x7632u);
+    const uint32_t v[4] = {x, x >> 8, y, y >> 8};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      o[4 * i + 0] = hsub_u32(and_or(v[i], 0x00030003u, 0x64006400u), 0x64006400u);
-      o[4 * i + 1] = hsub_u32(and_or(v[i], 0x000C000Cu, 0x5C005C00u), 0x5C005C00u);
-      o[4 * i + 2] = hsub_u32(and_or(v[i], 0x00300030u, 0x54005400u), 0x54005400u);
-      o[4 * i + 3] = hsub_u32(and_or(v[i], 0x00C000C0u, 0x4C004C00u), 0x4C004C00u);
+      o[4 * i + 0] = v[i] & 0x00030003u;
+      o[4 * i + 1] = v[i] & 0x000C000Cu;
+      o[4 * i + 2] = v[i] & 0x00300030u;
+      o[4 * i + 3] = v[i] & 0x00C000C0u;
     }
   }
+  __host__ __device__ static constexpr int exp(int i) { return 2 * (i & 3); }
 };
 
 template <>
 struct CrossPairs<8> {
   static constexpr int kOut = 4;
   __device__ __forceinline__ static void run(uint32_t a, uint32_t b, uint32_t (&o)[4]) {
-    uint32_t lo = prmt(a, b, 0x5140u);  // [a.b0 b.b0 a.b1 b.b1]
-    uint32_t hi = prmt(a, b, 0x7362u);  // [a.b2 b.b2 a.b3 b.b3]
-    o[0] = hsub_u32(prmt(lo, 0x64646464u, 0x4140u), 0x64006400u);
-    o[1] = hsub_u32(prmt(lo, 0x64646464u, 0x4342u), 0x64006400u);
-    o[2] = hsub_u32(prmt(hi, 0x64646464u, 0x4140u), 0x64006400u);
-    o[3] = hsub_u32(prmt(hi, 0x64646464u, 0x4342u), 0x64006400u);
+    const uint32_t x = prmt(a, b, 0x5410u);  // [a.b0 a.b1 b.b0 b.b1]
+    const uint32_t y = prmt(a, b, 0x7632u);  // [a.b2 a.b3 b.b2 b.b3]
+    o[0] = x & 0x00FF00FFu;
+    o[1] = (x >> 8) & 0x00FF00FFu;
+    o[2] = y & 0x00FF00FFu;
+    o[3] = (y >> 8) & 0x00FF00FFu;
   }
+  __host__ __device__ static constexpr int exp(int) { return 0; }
 };
 
 template <>
@@ -235,6 +231,14 @@ struct CrossPairs<16> {
     o[0] = prmt(a, b, 0x5410u);
     o[1] = prmt(a, b, 0x7632u);
   }
+  __host__ __device__ static constexpr int exp(int) { return 24; }
 };
+
+// 2^x for the softmax (hardware approximation, relative error ~2^-22).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 }  // namespace kvq

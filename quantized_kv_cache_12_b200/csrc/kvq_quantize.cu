@@ -47,7 +47,7 @@ __device__ __forceinline__ RowRef locate_row(const QuantArgs& a, long long r, in
 // advances seq_lens[b] itself (every thread has read the old value before
 // the barrier, so the update cannot race with the writes).
 template <int BITS, int G>
-__global__ void __launch_bounds__(256) quantize_append_kernel(const QuantArgs a) {
+__global__ void __launch_bounds__(1024) quantize_append_kernel(const QuantArgs a) {
   const int b = blockIdx.x;
   const int base = a.seq_lens[b];
   const int rows_per_side = a.kv_heads * a.n_new;
@@ -101,7 +101,10 @@ template <int BITS, int G>
 cudaError_t launch_q(const QuantArgs& a, cudaStream_t s) {
   const int rows_per_seq = 2 * a.kv_heads * a.n_new;
   if (rows_per_seq <= 512) {
-    quantize_append_kernel<BITS, G><<<a.batch, 256, 0, s>>>(a);
+    // one pass over the sequence's rows when they fit in one CTA
+    int threads = ((rows_per_seq * 16 + 63) / 64) * 64;
+    if (threads > 1024) threads = 1024;
+    quantize_append_kernel<BITS, G><<<a.batch, threads, 0, s>>>(a);
     return cudaGetLastError();
   }
   const long long rows = (long long)a.batch * rows_per_seq;
