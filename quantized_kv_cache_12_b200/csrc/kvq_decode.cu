@@ -45,10 +45,12 @@ struct Cfg {
   static constexpr int VC = (GE / 8) * BITS / 8;       // V bytes per lane per group
   static constexpr int VW = VC >= 4 ? VC / 4 : 1;      // V words per lane per group
   static constexpr int NTG = GE / 8;                   // PV n-tiles per group
-  static constexpr int SUB = (BITS == 16) ? 1 : 2;          // 16-token sub-tiles per stage
+  // 16-token sub-tiles per stage: two side by side, except where the
+  // registers of two would not fit three CTAs per SM (fp16 rows, 4 groups)
+  static constexpr int SUB = (BITS == 16 || NG == 4) ? 1 : 2;
   static constexpr int STOK = SUB * kTile;                   // tokens per stage
   static constexpr int STAGE = 2 * STOK * RB + 2 * STOK * MB;
-  static constexpr int MF_FLOATS = 2 * kTile * NG * 2;       // fp32 (s, z) of a sub-tile
+  static constexpr int MF_FLOATS = 2 * STOK * NG * 2;        // fp32 (s, z) of a stage
   // header: mbarriers (<= 512 B), q rows as fp16 (<= 8 x 128), group sums,
   // the A fragments of all 32 lane positions (8 x 32 x 16 B)
   static constexpr int HDR_BARS = 0, HDR_Q = 512, HDR_QS = 512 + 8 * kHeadDim * 2;
@@ -110,7 +112,7 @@ struct SplitParams {
 __device__ __forceinline__ int rho(int n) { return n ^ ((n >> 1) & 1); }
 
 template <int BITS, int GE, int GR>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, 3)
 decode_split_kernel(const __grid_constant__ SplitParams P) {
   using C = Cfg<BITS, GE>;
   using WP = WordPairs<BITS>;
@@ -274,64 +276,72 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   int st = 0;
   uint32_t phase = 0;
 
-  // one 16-token sub-tile: QK^T, online softmax, PV.  FULL = all 16 tokens
-  // valid (no masking work).
-  auto sub_tile = [&](auto full_tag, const uint8_t* sK, const uint8_t* sV, const uint8_t* sKm,
-                      const uint8_t* sVm, int n_valid) {
+  // One stage (SUB sub-tiles of 16 tokens): QK^T of every sub-tile, one
+  // online-softmax update, then PV of every sub-tile.  Working on the
+  // sub-tiles side by side gives the scheduler independent MMA chains and
+  // conversions to interleave.  FULL = all STOK tokens valid (no masking).
+  auto stage_body = [&](auto full_tag, const uint8_t* sK, const uint8_t* sV, const uint8_t* sKm,
+                        const uint8_t* sVm, int n_valid) {
     constexpr bool FULL = decltype(full_tag)::value;
-    auto valid = [&](int tok) { return FULL || tok < n_valid; };
+    constexpr int NS = C::SUB;
+    auto valid = [&](int tok) { return FULL || tok < n_valid; };  // tok: 0 .. STOK-1
 
-    // (s, z) of the sub-tile's K and V rows to fp32, once per warp: each
-    // lane converts NG pairs, every lane then reads the ones it needs
+    // (s, z) of the stage's K and V rows to fp32, once per warp: each lane
+    // converts SUB * NG pairs, every lane then reads the ones it needs
     if constexpr (BITS != 16) {
       __syncwarp();
 #pragma unroll
-      for (int j = 0; j < C::NG; ++j) {
-        const int idx = lane * C::NG + j;  // 0 .. 32 * NG - 1
-        const int plane = idx >= kTile * C::NG;
+      for (int j = 0; j < NS * C::NG; ++j) {
+        const int idx = lane * (NS * C::NG) + j;  // 0 .. 2 * STOK * NG - 1
+        const int plane = idx >= C::STOK * C::NG;
         const __half2* src = reinterpret_cast<const __half2*>(plane ? sVm : sKm);
-        mf[idx] = __half22float2(src[idx - plane * kTile * C::NG]);
+        mf[idx] = __half22float2(src[idx - plane * C::STOK * C::NG]);
       }
       __syncwarp();
     }
 
-    // ---- S = Qx * K^T for the two 8-token n-tiles (two MMA chains each)
-    float s_acc[2][2][4];
+    // ---- S = Qx * K^T for every 8-token n-tile of the stage
+    float s_acc[NS][2][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int sub = 0; sub < NS; ++sub) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
-        s_acc[nt][c][0] = s_acc[nt][c][1] = s_acc[nt][c][2] = s_acc[nt][c][3] = 0.f;
-      uint32_t kw[C::KW];
-      load_chunk<C::KC, C::KW>(sK + (nt * 8 + krow) * C::RB + tig * C::KC, kw);
-      uint32_t pr[16];
+      for (int nt = 0; nt < 2; ++nt) {
+        s_acc[sub][nt][0] = s_acc[sub][nt][1] = s_acc[sub][nt][2] = s_acc[sub][nt][3] = 0.f;
+        uint32_t kw[C::KW];
+        load_chunk<C::KC, C::KW>(sK + ((sub * 2 + nt) * 8 + krow) * C::RB + tig * C::KC, kw);
+        uint32_t pr[16];
 #pragma unroll
-      for (int w = 0; w < C::KW; ++w) {
-        uint32_t tmp[WP::kPairs];
-        WP::run(kw[w], tmp);
+        for (int w = 0; w < C::KW; ++w) {
+          uint32_t tmp[WP::kPairs];
+          WP::run(kw[w], tmp);
 #pragma unroll
-        for (int j = 0; j < WP::kPairs; ++j) pr[w * WP::kPairs + j] = tmp[j];
+          for (int j = 0; j < WP::kPairs; ++j) pr[w * WP::kPairs + j] = tmp[j];
+        }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_f16(s_acc[sub][nt], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], pr[2 * ks],
+                  pr[2 * ks + 1]);
       }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma_f16(s_acc[nt][ks & 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], pr[2 * ks],
-                pr[2 * ks + 1]);
     }
 
-    // ---- scores of head (gid mod g) for this lane's four tokens.  Rows
-    // past R hold zero queries (S = 0, qs = 0), so they add nothing.
-    float sc[4];
+    // ---- scores of head (gid mod g) for this lane's tokens.  Rows past R
+    // hold zero queries (S = 0, qs = 0), so they add nothing.
+    float sc[NS][4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int nt = k >> 1, e = k & 1;
-      const float S0 = s_acc[nt][0][e] + s_acc[nt][1][e];
-      if constexpr (BITS == 16) {
-        sc[k] = S0;
-      } else {
-        const float S1 = s_acc[nt][0][2 + e] + s_acc[nt][1][2 + e];
-        const float2 sz0 = mf[tok4[k] * C::NG + gr0];
-        const float2 sz1 = mf[tok4[k] * C::NG + gr1];
-        sc[k] = fmaf(sz1.x, fmaf(-sz1.y, qs1, S1), sz0.x * fmaf(-sz0.y, qs0, S0));
+    for (int sub = 0; sub < NS; ++sub) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int nt = k >> 1, e = k & 1;
+        const float S0 = s_acc[sub][nt][e];
+        if constexpr (BITS == 16) {
+          sc[sub][k] = S0;
+        } else {
+          const float S1 = s_acc[sub][nt][2 + e];
+          const float2* m = mf + (sub * kTile + tok4[k]) * C::NG;
+          const float2 sz0 = m[gr0];
+          const float2 sz1 = m[gr1];
+          sc[sub][k] = fmaf(sz1.x, fmaf(-sz1.y, qs1, S1), sz0.x * fmaf(-sz0.y, qs0, S0));
+        }
       }
     }
     // sum the group rows of each head: lanes gid and gid ^ m (m >= g)
@@ -339,15 +349,20 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
     for (int m = 1; m < 8; m <<= 1) {
       if (m >= g) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) sc[k] += __shfl_xor_sync(0xffffffffu, sc[k], 4 * m);
+        for (int sub = 0; sub < NS; ++sub)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            sc[sub][k] += __shfl_xor_sync(0xffffffffu, sc[sub][k], 4 * m);
       }
     }
     float tmax = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      sc[k] = valid(tok4[k]) ? sc[k] * score_scale : -INFINITY;
-      tmax = fmaxf(tmax, sc[k]);
-    }
+    for (int sub = 0; sub < NS; ++sub)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        sc[sub][k] = valid(sub * kTile + tok4[k]) ? sc[sub][k] * score_scale : -INFINITY;
+        tmax = fmaxf(tmax, sc[sub][k]);
+      }
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
     if (m_run == -INFINITY) {
@@ -363,63 +378,69 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
       l_part *= alpha;
       m_run = tmax;
     }
-    float p[4];
+    float p[NS][4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      p[k] = head_ok ? fast_exp2(sc[k] - m_run) : 0.f;  // 0 for masked tokens
-      l_part += p[k];
-    }
+    for (int sub = 0; sub < NS; ++sub)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        p[sub][k] = head_ok ? fast_exp2(sc[sub][k] - m_run) : 0.f;  // 0 for masked tokens
+        l_part += p[sub][k];
+      }
 
-    // ---- O += P' * V per group (hi rows gid, lo rows gid + 8)
+    // ---- O += P' * V per group and sub-tile (hi rows gid, lo rows gid + 8)
 #pragma unroll
     for (int gr = 0; gr < C::NG; ++gr) {
-      float pp[4];
-      if constexpr (BITS == 16) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) pp[k] = p[k];
-      } else {
+      for (int sub = 0; sub < NS; ++sub) {
+        float pp[4];
+        if constexpr (BITS == 16) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          // slots past the valid length may hold any bytes (NaN scales):
-          // select, never multiply by a zero weight
-          const float2 sz = mf[kTile * C::NG + tok4[k] * C::NG + gr];
-          pp[k] = valid(tok4[k]) ? p[k] * sz.x : 0.f;
-          corr[gr] = valid(tok4[k]) ? fmaf(pp[k], sz.y, corr[gr]) : corr[gr];
+          for (int k = 0; k < 4; ++k) pp[k] = p[sub][k];
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            // slots past the valid length may hold any bytes (NaN scales):
+            // select, never multiply by a zero weight
+            const bool ok = valid(sub * kTile + tok4[k]);
+            const float2 sz = mf[(C::STOK + sub * kTile + tok4[k]) * C::NG + gr];
+            pp[k] = ok ? p[sub][k] * sz.x : 0.f;
+            corr[gr] = ok ? fmaf(pp[k], sz.y, corr[gr]) : corr[gr];
+          }
         }
-      }
-      const __half2 h01 = __floats2half2_rn(pp[0], pp[1]);
-      const __half2 h23 = __floats2half2_rn(pp[2], pp[3]);
-      const float2 f01 = __half22float2(h01);
-      const float2 f23 = __half22float2(h23);
-      const uint32_t a0 = h2_as_u32(h01);
-      const uint32_t a1 = pack_h2(pp[0] - f01.x, pp[1] - f01.y);
-      const uint32_t a2 = h2_as_u32(h23);
-      const uint32_t a3 = pack_h2(pp[2] - f23.x, pp[3] - f23.y);
+        const __half2 h01 = __floats2half2_rn(pp[0], pp[1]);
+        const __half2 h23 = __floats2half2_rn(pp[2], pp[3]);
+        const float2 f01 = __half22float2(h01);
+        const float2 f23 = __half22float2(h23);
+        const uint32_t a0 = h2_as_u32(h01);
+        const uint32_t a1 = pack_h2(pp[0] - f01.x, pp[1] - f01.y);
+        const uint32_t a2 = h2_as_u32(h23);
+        const uint32_t a3 = pack_h2(pp[2] - f23.x, pp[3] - f23.y);
 
-      const uint8_t* vbase = sV + gr * (GE * BITS / 8) + gid * C::VC;
-      uint32_t wA[C::VW], wB[C::VW], wC[C::VW], wD[C::VW];
-      load_chunk<C::VC, C::VW>(vbase + tokA * C::RB, wA);
-      load_chunk<C::VC, C::VW>(vbase + tokB * C::RB, wB);
-      load_chunk<C::VC, C::VW>(vbase + tokC * C::RB, wC);
-      load_chunk<C::VC, C::VW>(vbase + tokD * C::RB, wD);
-      if constexpr (BITS == 16 && !FULL) {
-        // raw fp16 rows past the valid length may hold anything: zero them
+        const uint8_t* vbase = sV + sub * kTile * C::RB + gr * (GE * BITS / 8) + gid * C::VC;
+        uint32_t wA[C::VW], wB[C::VW], wC[C::VW], wD[C::VW];
+        load_chunk<C::VC, C::VW>(vbase + tokA * C::RB, wA);
+        load_chunk<C::VC, C::VW>(vbase + tokB * C::RB, wB);
+        load_chunk<C::VC, C::VW>(vbase + tokC * C::RB, wC);
+        load_chunk<C::VC, C::VW>(vbase + tokD * C::RB, wD);
+        if constexpr (BITS == 16 && !FULL) {
+          // raw fp16 rows past the valid length may hold anything: zero them
+#pragma unroll
+          for (int w = 0; w < C::VW; ++w) {
+            wA[w] = valid(sub * kTile + tokA) ? wA[w] : 0u;
+            wB[w] = valid(sub * kTile + tokB) ? wB[w] : 0u;
+            wC[w] = valid(sub * kTile + tokC) ? wC[w] : 0u;
+            wD[w] = valid(sub * kTile + tokD) ? wD[w] : 0u;
+          }
+        }
 #pragma unroll
         for (int w = 0; w < C::VW; ++w) {
-          wA[w] = valid(tokA) ? wA[w] : 0u;
-          wB[w] = valid(tokB) ? wB[w] : 0u;
-          wC[w] = valid(tokC) ? wC[w] : 0u;
-          wD[w] = valid(tokD) ? wD[w] : 0u;
+          uint32_t x[C::CROSS], y[C::CROSS];
+          XP::run(wA[w], wB[w], x);
+          XP::run(wC[w], wD[w], y);
+#pragma unroll
+          for (int j = 0; j < C::PER_W; ++j)
+            mma_f16(o_acc[gr * C::NTG + w * C::PER_W + j], a0, a1, a2, a3, x[j], y[j]);
         }
-      }
-#pragma unroll
-      for (int w = 0; w < C::VW; ++w) {
-        uint32_t x[C::CROSS], y[C::CROSS];
-        XP::run(wA[w], wB[w], x);
-        XP::run(wC[w], wD[w], y);
-#pragma unroll
-        for (int j = 0; j < C::PER_W; ++j)
-          mma_f16(o_acc[gr * C::NTG + w * C::PER_W + j], a0, a1, a2, a3, x[j], y[j]);
       }
     }
   };
@@ -434,19 +455,10 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
     const uint8_t* sKm = sK + 2 * C::STOK * C::RB;
     const uint8_t* sVm = sKm + C::STOK * C::MB;
     const int n_stage = min(C::STOK, w1 - (w0 + i * C::STOK));
-#pragma unroll
-    for (int sub = 0; sub < C::SUB; ++sub) {
-      const int nv = n_stage - sub * kTile;
-      if (nv <= 0) break;
-      const uint8_t* k_sub = sK + sub * kTile * C::RB;
-      const uint8_t* v_sub = sV + sub * kTile * C::RB;
-      const uint8_t* km_sub = sKm + sub * kTile * C::MB;
-      const uint8_t* vm_sub = sVm + sub * kTile * C::MB;
-      if (nv >= kTile)
-        sub_tile(std::integral_constant<bool, true>(), k_sub, v_sub, km_sub, vm_sub, kTile);
-      else
-        sub_tile(std::integral_constant<bool, false>(), k_sub, v_sub, km_sub, vm_sub, nv);
-    }
+    if (n_stage == C::STOK)
+      stage_body(std::integral_constant<bool, true>(), sK, sV, sKm, sVm, C::STOK);
+    else
+      stage_body(std::integral_constant<bool, false>(), sK, sV, sKm, sVm, n_stage);
     __syncwarp();
     if (lane == 0 && i + C::STAGES < n_tiles) issue(i + C::STAGES, st);
     if (++st == C::STAGES) {
