@@ -153,7 +153,8 @@ kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k_new,
  * arguments (host-only).  The workspace holds the per-split partial
  * results (m, l, o) merged by log-sum-exp and a 256-byte header whose
  * first 32-bit word is a sticky device error flag (nonzero after a kernel
- * gave up a bounded wait; the library never clears it).
+ * gave up a bounded wait; the library never clears it), followed by the
+ * work counters of the persistent decode kernel.
  */
 kvq_status kvq_decode_workspace_bytes(const kvq_cache *segs, int32_t n_segs,
                                       int32_t q_heads, int32_t max_len_hint,
@@ -178,7 +179,9 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache *segs, int32_t n_segs,
  *   max_len_hint: an upper bound of the seq_lens used to pick the split
  *        count (<= 0: max_tokens); results are correct for any seq_lens.
  *   workspace: device, >= kvq_decode_workspace_bytes(same arguments),
- *        256-byte aligned.
+ *        256-byte aligned, zero-filled before its first use (its header
+ *        holds work counters that the kernels return to zero at the end of
+ *        every call, so it stays reusable without clearing).
  * A sequence with no tokens gives out = 0 and lse = -inf.
  * Supported: head_dim 128; g in 1..8; bits 2/4/8 with G 32/64/128, and bits
  * 16 with fp16 q.  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED,

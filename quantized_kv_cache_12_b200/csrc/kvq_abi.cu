@@ -47,13 +47,15 @@ kvq_status check_cache(const kvq_cache* c, bool allow16) {
   return KVQ_OK;
 }
 
-// Split count of one segment.  A split is one CTA; the decode kernel keeps
-// three CTAs on each of the 148 SMs, so the CTAs run in waves of 444.  The
-// count minimises (waves) x (tokens per CTA + a fixed per-CTA cost of about
-// 96 tokens' worth of work), tokens per CTA being rounded up to the
-// kernel's 128-token granularity, with at least 128 tokens per CTA.  The
-// result depends only on (sequences x KV heads, length), so it is cached
-// per thread.
+// Split count of one segment.  A (sequence, KV head, split) is one unit of
+// work; the decode kernel runs one wave of persistent CTAs (three per SM,
+// 444 on a B200) that take units from a counter.  With equal units the
+// kernel takes ceil(units / 444) unit-times, so the count minimises
+// ceil(units / 444) x (tokens per unit + a fixed per-unit cost), tokens per
+// unit being rounded up to the 32-token stage, with at least 128 tokens per
+// unit.  The fixed cost -- the start of a unit waits for its query rows and
+// first copies -- was measured at about 400 tokens' worth of work.  The result depends only on
+// (sequences x KV heads, length), so it is cached per thread.
 int choose_splits(const kvq_cache& c, int max_len_hint) {
   const long long pairs = (long long)c.batch * c.kv_heads;
   long long len = c.max_tokens;
@@ -62,10 +64,10 @@ int choose_splits(const kvq_cache& c, int max_len_hint) {
   thread_local long long cached_pairs = -1, cached_len = -1;
   thread_local int cached_n = 1;
   if (pairs == cached_pairs && len == cached_len) return cached_n;
-  constexpr long long kSlots = 148LL * 3, kOverhead = 96, kGran = 128;
-  const long long cap = (len + kGran - 1) / kGran;
+  constexpr long long kSlots = 148LL * 3, kOverhead = 400, kGran = 32, kMinTokens = 128;
+  const long long cap = (len + kMinTokens - 1) / kMinTokens;
   long long best_n = 1, best_cost = -1;
-  for (long long n = 1; n <= cap && n <= 2048; ++n) {
+  for (long long n = 1; n <= cap && n <= 4096; ++n) {
     const long long chunk = ((len + n - 1) / n + kGran - 1) / kGran * kGran;
     const long long waves = (pairs * n + kSlots - 1) / kSlots;
     const long long cost = waves * (chunk + kOverhead);

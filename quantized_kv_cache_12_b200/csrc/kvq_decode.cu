@@ -45,8 +45,11 @@ struct Cfg {
   static constexpr int VC = (GE / 8) * BITS / 8;       // V bytes per lane per group
   static constexpr int VW = VC >= 4 ? VC / 4 : 1;      // V words per lane per group
   static constexpr int NTG = GE / 8;                   // PV n-tiles per group
+  // CTAs kept on one SM: four for the 2- and 4-bit formats (the query
+  // fragments live in shared memory, not registers), three otherwise
+  static constexpr int MIN_CTAS = 3;
   // 16-token sub-tiles per stage: two side by side, except where the
-  // registers of two would not fit three CTAs per SM (fp16 rows, 4 groups)
+  // registers of two would not fit (fp16 rows, 4 groups)
   static constexpr int SUB = (BITS == 16 || NG == 4) ? 1 : 2;
   static constexpr int STOK = SUB * kTile;                   // tokens per stage
   static constexpr int STAGE = 2 * STOK * RB + 2 * STOK * MB;
@@ -56,10 +59,11 @@ struct Cfg {
   static constexpr int HDR_BARS = 0, HDR_Q = 512, HDR_QS = 512 + 8 * kHeadDim * 2;
   static constexpr int HDR_QF = HDR_QS + 128;
   static constexpr int HDR_MF = HDR_QF + 8 * 32 * 16;        // per-warp fp32 meta
-  static constexpr int HDR_BYTES = HDR_MF + kWarps * MF_FLOATS * 4;
-  // as many stages as fit in a budget that keeps three CTAs on an SM
-  // (3 x (74 KB + 1 KB reserved) <= 228 KB)
-  static constexpr int SMEM_BUDGET = 74 * 1024;
+  static constexpr int HDR_MISC = HDR_MF + kWarps * MF_FLOATS * 4;  // unit id, fail flag
+  static constexpr int HDR_BYTES = HDR_MISC + 128;
+  // as many stages as fit in a budget that keeps MIN_CTAS CTAs on an SM
+  // (3 x (74 KB + 1 KB reserved) and 4 x (56 KB + 1 KB) <= 228 KB)
+  static constexpr int SMEM_BUDGET = (MIN_CTAS == 4 ? 56 : 74) * 1024;
   static constexpr int STAGES_RAW = (SMEM_BUDGET - HDR_BYTES) / (kWarps * STAGE);
   static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 16 ? 16 : STAGES_RAW);
   static constexpr int SMEM = HDR_BYTES + kWarps * STAGES * STAGE;
@@ -112,7 +116,7 @@ struct SplitParams {
 __device__ __forceinline__ int rho(int n) { return n ^ ((n >> 1) & 1); }
 
 template <int BITS, int GE, int GR>
-__global__ void __launch_bounds__(kWarps * 32, 3)
+__global__ void __launch_bounds__(kWarps * 32, Cfg<BITS, GE>::MIN_CTAS)
 decode_split_kernel(const __grid_constant__ SplitParams P) {
   using C = Cfg<BITS, GE>;
   using WP = WordPairs<BITS>;
@@ -125,7 +129,6 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   constexpr int g = GR;                  // query heads per KV head: 1, 2, 4 or 8
   constexpr int lg = GR == 1 ? 0 : (GR == 2 ? 1 : (GR == 4 ? 2 : 3));
   constexpr int R = C::NG * g;           // valid MMA rows (group, head)
@@ -137,21 +140,50 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   uint4* qf_sm = reinterpret_cast<uint4*>(smem + C::HDR_QF);      // [8][32 lanes]
   float2* mf = reinterpret_cast<float2*>(smem + C::HDR_MF) + warp * (C::MF_FLOATS / 2);
   uint8_t* stages = smem + C::HDR_BYTES + warp * C::STAGES * C::STAGE;
+  int* unit_sm = reinterpret_cast<int*>(smem + C::HDR_MISC);
+  int* fail_sm = unit_sm + 1;
+  uint32_t* counters = a.err + 1;  // [0] next unit, [1] CTAs done
+
+  const uint64_t policy = l2_evict_first_policy();
+  // the stage ring (position and mbarrier phase) runs on across units
+  int st = 0;
+  uint32_t phase = 0;
+  if (lane == 0) {
+    for (int s2 = 0; s2 < C::STAGES; ++s2) mbar_init(&bars[s2], 1);
+    fence_barrier_init();
+  }
+  if (threadIdx.x == 0) *fail_sm = 0;
+  __syncwarp();
+  const int t = threadIdx.x;
+  const int units = seg.n_split * a.kv_heads * a.batch;
+
+  // Persistent CTA: take (sequence, KV head, split) units from a counter in
+  // the workspace until none is left.  The barrier after the fetch also
+  // orders the previous unit's reads of the merge scratch before this
+  // unit's copies into the stage buffers.
+  for (;;) {
+  if (t == 0) *unit_sm = (int)atomicAdd(&counters[0], 1u);
+  __syncthreads();
+  const int unit = *unit_sm;
+  if (unit >= units || *fail_sm) break;
+  const int split = unit % seg.n_split;
+  const int kvh = (unit / seg.n_split) % a.kv_heads;
+  const int b = unit / (seg.n_split * a.kv_heads);
 
   // ---- token range of this warp (a multiple of the stage size, so a
   // stage's copy never runs past round_up(seq_len, 32) <= max_tokens)
   int L = seg.seq_lens[b];
   L = max(0, min(L, seg.max_tokens));
+  // a unit is `chunk` tokens (a multiple of the 32-token stage); its stages
+  // go to the four warps round-robin: warp w takes stages w, w + 4, ...
   const int per_split = (L + seg.n_split - 1) / seg.n_split;
-  const int chunk = ((per_split + 127) / 128) * 128;
+  const int chunk = ((per_split + 31) / 32) * 32;
   const int c0 = split * chunk;
   const int c1 = min(c0 + chunk, L);
-  const int wq = chunk / kWarps;
-  const int w0 = c0 + warp * wq;
-  const int w1 = min(w0 + wq, c1);
-  const int n_tiles = (w1 > w0) ? (w1 - w0 + C::STOK - 1) / C::STOK : 0;
+  const int unit_stages = (c1 > c0) ? (c1 - c0 + C::STOK - 1) / C::STOK : 0;
+  const int n_tiles = (unit_stages > warp) ? (unit_stages - warp + kWarps - 1) / kWarps : 0;
+  const int w0 = c0 + warp * C::STOK;  // first token of this warp's first stage
 
-  const uint64_t policy = l2_evict_first_policy();
   const uint8_t* kc_src = seg.k_codes + (((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0) * C::RB;
   const uint8_t* vc_src = seg.v_codes + (((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0) * C::RB;
   const uint8_t* km_src = seg.k_meta + (((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0) * C::MB;
@@ -160,27 +192,24 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   auto issue = [&](int i, int st) {
     uint8_t* dst = stages + st * C::STAGE;
     mbar_arrive_expect_tx(&bars[st], C::STAGE);
-    bulk_load(dst, kc_src + (size_t)i * (C::STOK * C::RB), C::STOK * C::RB, &bars[st], policy);
-    bulk_load(dst + C::STOK * C::RB, vc_src + (size_t)i * (C::STOK * C::RB), C::STOK * C::RB,
-              &bars[st], policy);
+    const size_t tok = (size_t)i * (kWarps * C::STOK);  // stage i of this warp
+    bulk_load(dst, kc_src + tok * C::RB, C::STOK * C::RB, &bars[st], policy);
+    bulk_load(dst + C::STOK * C::RB, vc_src + tok * C::RB, C::STOK * C::RB, &bars[st], policy);
     if constexpr (C::MB > 0) {
-      bulk_load(dst + 2 * C::STOK * C::RB, km_src + (size_t)i * (C::STOK * C::MB),
+      bulk_load(dst + 2 * C::STOK * C::RB, km_src + tok * C::MB, C::STOK * C::MB, &bars[st],
+                policy);
+      bulk_load(dst + 2 * C::STOK * C::RB + C::STOK * C::MB, vm_src + tok * C::MB,
                 C::STOK * C::MB, &bars[st], policy);
-      bulk_load(dst + 2 * C::STOK * C::RB + C::STOK * C::MB,
-                vm_src + (size_t)i * (C::STOK * C::MB), C::STOK * C::MB, &bars[st], policy);
     }
   };
 
   if (lane == 0) {
-    for (int s = 0; s < C::STAGES; ++s) mbar_init(&bars[s], 1);
-    fence_barrier_init();
     const int pre = min(n_tiles, C::STAGES);
-    for (int i = 0; i < pre; ++i) issue(i, i);
+    for (int i = 0; i < pre; ++i) issue(i, (st + i) % C::STAGES);
   }
 
-  // ---- the g query rows of this KV head, once per CTA, as fp16 in smem
+  // ---- the g query rows of this KV head, once per unit, as fp16 in smem
   // (bf16 queries are used through fp16: exact for |q| in [2^-14, 65504])
-  const int t = threadIdx.x;
   {
     const long long qbase = ((long long)b * a.q_heads + (long long)kvh * g) * D;
     if (t < g * (D / 8)) {
@@ -240,11 +269,16 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
     }
   }
   __syncthreads();
-  uint32_t qf[8][4];
+  // query fragments: kept in registers for the 3-CTA formats, re-read from
+  // shared memory (once per stage and k-step) for the 4-CTA ones
+  constexpr bool kQfRegs = C::MIN_CTAS == 3;
+  uint32_t qf[kQfRegs ? 8 : 1][4];
+  if constexpr (kQfRegs) {
 #pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    const uint4 v = qf_sm[ks * 32 + lane];
-    qf[ks][0] = v.x; qf[ks][1] = v.y; qf[ks][2] = v.z; qf[ks][3] = v.w;
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint4 v = qf_sm[ks * 32 + lane];
+      qf[ks][0] = v.x; qf[ks][1] = v.y; qf[ks][2] = v.z; qf[ks][3] = v.w;
+    }
   }
   const bool row0_ok = gid < R, row1_ok = gid + 8 < R;
   const float qs0 = (BITS != 16 && row0_ok) ? qs_sm[gid] : 0.f;
@@ -273,8 +307,8 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   constexpr float kLazy = 4.0f;
   float m_run = -INFINITY, l_part = 0.f;
   int failed_at = -1;
-  int st = 0;
-  uint32_t phase = 0;
+  const int st0 = st;
+  const uint32_t phase0 = phase;
 
   // One stage (SUB sub-tiles of 16 tokens): QK^T of every sub-tile, one
   // online-softmax update, then PV of every sub-tile.  Working on the
@@ -302,25 +336,52 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
 
     // ---- S = Qx * K^T for every 8-token n-tile of the stage
     float s_acc[NS][2][4];
+    if constexpr (kQfRegs) {
 #pragma unroll
-    for (int sub = 0; sub < NS; ++sub) {
+      for (int sub = 0; sub < NS; ++sub) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        s_acc[sub][nt][0] = s_acc[sub][nt][1] = s_acc[sub][nt][2] = s_acc[sub][nt][3] = 0.f;
-        uint32_t kw[C::KW];
-        load_chunk<C::KC, C::KW>(sK + ((sub * 2 + nt) * 8 + krow) * C::RB + tig * C::KC, kw);
-        uint32_t pr[16];
+        for (int nt = 0; nt < 2; ++nt) {
+          s_acc[sub][nt][0] = s_acc[sub][nt][1] = s_acc[sub][nt][2] = s_acc[sub][nt][3] = 0.f;
+          uint32_t kw[C::KW];
+          load_chunk<C::KC, C::KW>(sK + ((sub * 2 + nt) * 8 + krow) * C::RB + tig * C::KC, kw);
+          uint32_t pr[16];
 #pragma unroll
-        for (int w = 0; w < C::KW; ++w) {
-          uint32_t tmp[WP::kPairs];
-          WP::run(kw[w], tmp);
+          for (int w = 0; w < C::KW; ++w) {
+            uint32_t tmp[WP::kPairs];
+            WP::run(kw[w], tmp);
 #pragma unroll
-          for (int j = 0; j < WP::kPairs; ++j) pr[w * WP::kPairs + j] = tmp[j];
+            for (int j = 0; j < WP::kPairs; ++j) pr[w * WP::kPairs + j] = tmp[j];
+          }
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_f16(s_acc[sub][nt], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], pr[2 * ks],
+                    pr[2 * ks + 1]);
+        }
+      }
+    } else {
+      // k-step outermost: one shared-memory read of each query fragment
+      // feeds the MMAs of all n-tiles of the stage
+      uint32_t kw[NS][2][C::KW];
+#pragma unroll
+      for (int sub = 0; sub < NS; ++sub)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          s_acc[sub][nt][0] = s_acc[sub][nt][1] = s_acc[sub][nt][2] = s_acc[sub][nt][3] = 0.f;
+          load_chunk<C::KC, C::KW>(sK + ((sub * 2 + nt) * 8 + krow) * C::RB + tig * C::KC,
+                                   kw[sub][nt]);
         }
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_f16(s_acc[sub][nt], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], pr[2 * ks],
-                  pr[2 * ks + 1]);
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint4 q4 = qf_sm[ks * 32 + lane];
+        constexpr int P = WP::kPairs;
+#pragma unroll
+        for (int sub = 0; sub < NS; ++sub)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b0 = WP::one(kw[sub][nt][(2 * ks) / P], (2 * ks) % P);
+            const uint32_t b1 = WP::one(kw[sub][nt][(2 * ks + 1) / P], (2 * ks + 1) % P);
+            mma_f16(s_acc[sub][nt], q4.x, q4.y, q4.z, q4.w, b0, b1);
+          }
       }
     }
 
@@ -454,7 +515,7 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
     const uint8_t* sV = sK + C::STOK * C::RB;
     const uint8_t* sKm = sK + 2 * C::STOK * C::RB;
     const uint8_t* sVm = sKm + C::STOK * C::MB;
-    const int n_stage = min(C::STOK, w1 - (w0 + i * C::STOK));
+    const int n_stage = min(C::STOK, c1 - (w0 + i * kWarps * C::STOK));
     if (n_stage == C::STOK)
       stage_body(std::integral_constant<bool, true>(), sK, sV, sKm, sVm, C::STOK);
     else
@@ -468,11 +529,17 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   }
 
   if (failed_at >= 0) {
-    if (lane == 0) atomicOr(a.err, kErrWaitTimeout);
+    if (lane == 0) {
+      atomicOr(a.err, kErrWaitTimeout);
+      *fail_sm = 1;  // the CTA stops after this unit
+    }
     // drain the copies this warp issued and has not consumed (bounded)
     const int issued_end = min(n_tiles, failed_at + C::STAGES);
-    for (int i = failed_at; i < issued_end; ++i)
-      (void)mbar_wait_bounded(&bars[i % C::STAGES], (i / C::STAGES) & 1, 1u << 16);
+    for (int i = failed_at; i < issued_end; ++i) {
+      const int pos = st0 + i;
+      const uint32_t ph = phase0 ^ (uint32_t)((pos / C::STAGES) & 1);
+      (void)mbar_wait_bounded(&bars[pos % C::STAGES], ph, 1u << 16);
+    }
   }
 
   // ---- per-warp totals over the 4 lanes of a head
@@ -507,23 +574,34 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
     }
   }
   __syncthreads();
-  const int part = seg.part_base + split;
-  for (int h = 0; h < g; ++h) {
+  // per head: the max over the warps, each warp's weight 2^(m_w - M) and
+  // the total sum, computed once (thread h), then one FMA per warp per dim
+  float* wt = os + kWarps * 8 * D;  // [8][kWarps] weights, then M[8], L[8]
+  float* Mh = wt + 8 * kWarps;
+  float* Lh = Mh + 8;
+  if (t < g) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w)
-      if (ls[w * 8 + h] > 0.f) M = fmaxf(M, ms[w * 8 + h]);
-    float Ls = 0.f, O = 0.f;
-    if (M != -INFINITY) {
+      if (ls[w * 8 + t] > 0.f) M = fmaxf(M, ms[w * 8 + t]);
+    float Ls = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        if (ls[w * 8 + h] > 0.f) {
-          const float wt = exp2f(ms[w * 8 + h] - M);
-          Ls += wt * ls[w * 8 + h];
-          O += wt * os[(w * 8 + h) * D + t];
-        }
-      }
+    for (int w = 0; w < kWarps; ++w) {
+      const float x = (ls[w * 8 + t] > 0.f) ? exp2f(ms[w * 8 + t] - M) : 0.f;
+      wt[t * kWarps + w] = x;
+      Ls += x * ls[w * 8 + t];
     }
+    Mh[t] = M;
+    Lh[t] = Ls;
+  }
+  __syncthreads();
+  const int part = seg.part_base + split;
+#pragma unroll
+  for (int h = 0; h < g; ++h) {
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) O = fmaf(wt[h * kWarps + w], os[(w * 8 + h) * D + t], O);
+    const float M = Mh[h], Ls = Lh[h];
     const long long bh = (long long)b * a.q_heads + (long long)kvh * g + h;
     if (a.parts == 1) {
       a.out[bh * D + t] = (Ls > 0.f) ? O / Ls : 0.f;
@@ -536,6 +614,19 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
         a.part_ml[pi * 2 + 0] = M;
         a.part_ml[pi * 2 + 1] = Ls;
       }
+    }
+  }
+  }  // unit loop
+
+  // The last CTA to finish resets the counters for the next launch on this
+  // workspace (nothing waits on them).
+  if (t == 0) {
+    __threadfence();
+    const unsigned done = atomicAdd(&counters[1], 1u);
+    if (done == gridDim.x - 1) {
+      atomicExch(&counters[0], 0u);
+      atomicExch(&counters[1], 0u);
+      __threadfence();
     }
   }
 }
@@ -603,7 +694,9 @@ cudaError_t launch_split_g(const DecodeArgs& a, const SegView& seg, cudaStream_t
     attr_set.fetch_or(bit);
   }
   SplitParams P{a, seg};
-  dim3 grid(seg.n_split, a.kv_heads, a.batch);
+  const long long units = (long long)seg.n_split * a.kv_heads * a.batch;
+  const long long slots = 148LL * C::MIN_CTAS;  // one wave of persistent CTAs
+  const unsigned grid = (unsigned)(units < slots ? units : slots);
   decode_split_kernel<BITS, GE, GR><<<grid, kWarps * 32, C::SMEM, s>>>(P);
   return cudaGetLastError();
 }

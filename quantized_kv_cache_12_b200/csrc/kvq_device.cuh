@@ -128,6 +128,11 @@ struct WordPairs<4> {
   }
   __host__ __device__ static constexpr int dim(int j, int e) { return j + 4 * e; }
   __host__ __device__ static constexpr int exp(int j) { return 4 * (j & 1); }
+  // pair j alone (j a compile-time constant after unrolling)
+  __device__ __forceinline__ static uint32_t one(uint32_t w, int j) {
+    const uint32_t v = (j & 2) ? (w >> 8) : w;
+    return v & ((j & 1) ? 0x00F000F0u : 0x000F000Fu);
+  }
 };
 
 template <>
@@ -146,6 +151,10 @@ struct WordPairs<2> {
   }
   __host__ __device__ static constexpr int dim(int j, int e) { return j + 8 * e; }
   __host__ __device__ static constexpr int exp(int j) { return 2 * (j & 3); }
+  __device__ __forceinline__ static uint32_t one(uint32_t w, int j) {
+    const uint32_t v = (j & 4) ? (w >> 8) : w;
+    return v & (0x00030003u << (2 * (j & 3)));
+  }
 };
 
 template <>
@@ -157,6 +166,9 @@ struct WordPairs<8> {
   }
   __host__ __device__ static constexpr int dim(int j, int e) { return j + 2 * e; }
   __host__ __device__ static constexpr int exp(int) { return 0; }
+  __device__ __forceinline__ static uint32_t one(uint32_t w, int j) {
+    return (j ? (w >> 8) : w) & 0x00FF00FFu;
+  }
 };
 
 template <>
@@ -165,6 +177,7 @@ struct WordPairs<16> {
   __device__ __forceinline__ static void run(uint32_t w, uint32_t (&p)[1]) { p[0] = w; }
   __host__ __device__ static constexpr int dim(int, int e) { return e; }
   __host__ __device__ static constexpr int exp(int) { return 24; }
+  __device__ __forceinline__ static uint32_t one(uint32_t w, int) { return w; }
 };
 
 // Pairs across two tokens (V side): words a (token A) and b (token B) hold
