@@ -154,6 +154,28 @@ def run_reference(args, wl):
 
     import oracle
     import workloads
+    if wl.chunk_tokens:
+        sub = wl.scaled(batch=1, kv_heads=min(wl.kv_heads, 4), q_heads=min(wl.kv_heads, 4))
+        k, v = workloads.kv_tokens(sub, wl.context, "cpu")
+        q = workloads.queries(sub, "cpu")
+        prepared, counts = prepare_mixed_oracle(wl, k, v, q, sub)
+
+        def mixed_step(i):
+            qh, segs, lens = prepared[i % len(prepared)]
+            oracle.decode_attention(qh, False, segs, lens, 128 ** -0.5)
+        for i in range(args.warmup):
+            mixed_step(i)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            mixed_step(i)
+        el = time.perf_counter() - t0
+        value = args.steps / wl.kv_heads / el
+        sample = (f"each step: one (sequence, KV head) of {wl.name}: attention over its "
+                  f"{wl.n_chunks} chunks as FP16/INT4/INT2 segments ({int(counts[0])}/"
+                  f"{int(counts[1])}/{int(counts[2])} chunks); tokens/s = steps / kv_heads "
+                  f"({wl.kv_heads}) / seconds")
+        print(json.dumps(reference_line(args, wl, value, el, sample)), flush=True)
+        return
     sub = wl.scaled(batch=1, kv_heads=min(wl.kv_heads, 4),
                     q_heads=min(wl.kv_heads, 4) * wl.group_ratio)
     L = wl.context
@@ -190,7 +212,11 @@ def run_reference(args, wl):
     sample = (f"each step: one (sequence, KV head) of {wl.name} at {L + 1} tokens "
               f"(append 1 token + attention of {g} query heads); tokens/s = steps / kv_heads "
               f"({wl.kv_heads}) / seconds")
-    line = {
+    print(json.dumps(reference_line(args, wl, value, el, sample)), flush=True)
+
+
+def reference_line(args, wl, value, el, sample):
+    return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -201,7 +227,6 @@ def run_reference(args, wl):
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
 
 
 def workload_config(wl, extra=None):
@@ -256,9 +281,71 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
                       f"tokens/s = pairs / kv_heads / seconds"}
 
 
+def prepare_mixed_oracle(wl, k, v, q, wlr):
+    """Oracle inputs for (sequence 0, KV head h) pairs of the chunk-level mixed
+    workload: its own chunk classes (fp64 similarity), reorder and
+    quantization.  Returns (prepared pairs, class counts)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import workloads
+    emb, qemb = workloads.chunk_embeddings(wlr.scaled(batch=1), "cpu")
+    _, cls = oracle.chunk_assign(emb[0].numpy(), qemb[0].numpy(), wl.alpha, wl.beta)
+    perm, counts = oracle.chunk_partition(cls)
+    T = wl.chunk_tokens
+    prepared = []
+    for h in range(min(wl.kv_heads, 4)):
+        segs, lens, start = [], [], 0
+        for bits, cnt in zip((16,) + wl.low_bits, counts):
+            idx = perm[start:start + cnt]
+            start += cnt
+            tok = (idx[:, None] * T + np.arange(T)[None]).reshape(-1)
+            kk = k[0, h, torch.from_numpy(tok).to(k.device)].cpu().contiguous()
+            vv = v[0, h, torch.from_numpy(tok).to(v.device)].cpu().contiguous()
+            k16 = kk.view(torch.int16).numpy().view(np.uint16)[None, None]
+            v16 = vv.view(torch.int16).numpy().view(np.uint16)[None, None]
+            if bits == 16:
+                seg = dict(k_codes=k16.view(np.uint8).reshape(1, 1, -1, 256),
+                           v_codes=v16.view(np.uint8).reshape(1, 1, -1, 256), k_meta=None,
+                           v_meta=None, bits=16, group=128)
+            else:
+                kc, km = oracle.quantize_cache(k16, wl.group, bits)
+                vc, vm = oracle.quantize_cache(v16, wl.group, bits)
+                seg = dict(k_codes=kc, v_codes=vc, k_meta=km, v_meta=vm, bits=bits,
+                           group=wl.group)
+            segs.append(seg)
+            lens.append(np.array([len(tok)]))
+        qh = q[0:1, h:h + 1].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        prepared.append((qh, segs, lens))
+    return prepared, counts
+
+
+def cpu_baseline_mixed(wl, k, v, q, seconds: float, wlr):
+    """The oracle's timed fp64 attention over the three segments of sampled
+    (sequence, KV head) pairs of the chunk-level mixed workload."""
+    import oracle
+    prepared, counts = prepare_mixed_oracle(wl, k, v, q, wlr)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        qh, segs, lens = prepared[n % len(prepared)]
+        oracle.decode_attention(qh, False, segs, lens, 128 ** -0.5)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and n >= 2:
+            break
+    return {"value": n / wl.kv_heads / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} (sequence, KV head) attention steps of {wl.name} over its "
+                      f"{int(sum(counts))} chunks ({int(counts[0])} FP16, {int(counts[1])} INT4, "
+                      f"{int(counts[2])} INT2) cycling over {len(prepared)} heads, {el:.1f} s on "
+                      f"one host thread; tokens/s = pairs / kv_heads / seconds"}
+
+
 # ---------------------------------------------------------------- kvq arm
 
 def run_kvq(args, wl, rank, world, local_rank):
+    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -267,32 +354,52 @@ def run_kvq(args, wl, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    if wl.chunk_tokens:
-        raise SystemExit("bench: the chunk-level mixed-precision workload is a parity case here")
     B, H, Hq, D = wl.batch, wl.kv_heads, wl.q_heads, wl.head_dim
     ctx = wl.context
-    episode = wl.steps if wl.append else 1
-    max_tokens = workloads.round_up(ctx + episode + 1, 64)
+    episode = wl.steps if wl.append else min(wl.steps, 100)
     wlr = wl.scaled(seed=wl.seed + 1000 * rank)  # each rank its own sequences
 
     # ---- resident inputs (untimed set-up)
-    k, v = workloads.kv_tokens(wlr, ctx, dev)
-    cache = kvq.QuantizedKVCache.allocate(B, H, D, max_tokens, wl.bits, wl.group, dev)
-    cache.seq_lens.zero_()
-    kvq.kvq_quantize_append(cache, k, v, ctx, advance_seq_lens=True)
-    base_lens = cache.seq_lens.clone()
-    kn = torch.stack([torch.stack(workloads.kv_tokens(wlr, 1, dev, stream_extra=1 + e))
-                      for e in range(episode)])           # [E, 2, B, H, 1, D]
+    if wl.chunk_tokens:
+        # chunk-level mixed precision: search, reorder, quantize the prompt
+        # into FP16 / INT4 / INT2 segments once; each step attends over them
+        emb, qemb = workloads.chunk_embeddings(wlr, dev)
+        cbits = torch.empty((B, wl.n_chunks), dtype=torch.uint8, device=dev)
+        kvq.kvq_chunk_assign(emb, qemb, wl.alpha, wl.beta, cbits)
+        del emb, qemb
+        k, v = workloads.kv_tokens(wlr, ctx, dev)
+        segs = [kvq.QuantizedKVCache.allocate(B, H, D, workloads.round_up(ctx, 64), bits,
+                                              wl.group, dev) for bits in (16,) + wl.low_bits]
+        perm = torch.empty((B, wl.n_chunks), dtype=torch.int32, device=dev)
+        kvq.kvq_chunk_reorder(segs, k, v, wl.chunk_tokens, cbits, perm)
+        seg_lens = [c.seq_lens.cpu().numpy().astype(np.int64) for c in segs]
+        seg_bits = [c.bits for c in segs]
+        k_cpu_src = (k, v, cbits)
+        base_lens = None
+        kn = None
+    else:
+        max_tokens = workloads.round_up(ctx + episode + 1, 64)
+        k, v = workloads.kv_tokens(wlr, ctx, dev)
+        cache = kvq.QuantizedKVCache.allocate(B, H, D, max_tokens, wl.bits, wl.group, dev)
+        cache.seq_lens.zero_()
+        kvq.kvq_quantize_append(cache, k, v, ctx, advance_seq_lens=True)
+        base_lens = cache.seq_lens.clone()
+        segs = [cache]
+        seg_bits = [wl.bits]
+        seg_lens = None
+        k_cpu_src = None
+        kn = torch.stack([torch.stack(workloads.kv_tokens(wlr, 1, dev, stream_extra=1 + e))
+                          for e in range(episode)]) if wl.append else None  # [E, 2, B, H, 1, D]
     qs = torch.stack([workloads.queries(wlr, dev, step=e) for e in range(episode)])
-    hint = ctx + episode
+    hint = ctx + episode if wl.append else ctx
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
     lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
-    ws = kvq.alloc_workspace(cache, Hq, hint, device=dev)
-    ws_bytes = kvq.kvq_decode_workspace_bytes(cache, Hq, hint)
+    ws = kvq.alloc_workspace(segs, Hq, hint, device=dev)
+    ws_bytes = kvq.kvq_decode_workspace_bytes(segs, Hq, hint)
     bh = B * Hq
     parts = next(p for p in range(1, 1 << 16)
                  if 256 + (bh * p * 8 + 255) // 256 * 256 + bh * p * D * 4 == ws_bytes)
-    launches_per_step = (1 if wl.append else 0) + 1 + (1 if parts > 1 else 0)
+    launches_per_step = (1 if wl.append else 0) + len(segs) + (1 if parts > 1 else 0)
     stream = torch.cuda.current_stream()
 
     def step(s, ev=None):
@@ -303,13 +410,18 @@ def run_kvq(args, wl, rank, world, local_rank):
             kvq.kvq_quantize_append(cache, kn[e, 0], kn[e, 1], 1, advance_seq_lens=True)
         if ev is not None:
             ev[0].record(stream)
-        kvq.kvq_decode_partials(cache, qs[e], out, lse, ws, max_len_hint=hint)
+        kvq.kvq_decode_partials(segs, qs[e], out, lse, ws, max_len_hint=hint)
         if ev is not None:
             ev[1].record(stream)
-        kvq.kvq_decode_merge(cache, qs[e], out, lse, ws, max_len_hint=hint)
+        kvq.kvq_decode_merge(segs, qs[e], out, lse, ws, max_len_hint=hint)
 
-    def lens_at(s):
-        return ctx + (s % episode) + 1 if wl.append else ctx
+    def kv_bytes_at(s):
+        """Algorithmic K+V bytes of the split kernel(s) at step s."""
+        if seg_lens is not None:
+            return sum(int(ln.sum()) * H * bytes_per_head_token(bits, wl.group, D)
+                       for ln, bits in zip(seg_lens, seg_bits))
+        L = ctx + (s % episode) + 1 if wl.append else ctx
+        return B * H * L * bytes_per_head_token(wl.bits, wl.group, D)
 
     # ---- warm-up
     for s in range(args.warmup):
@@ -346,22 +458,22 @@ def run_kvq(args, wl, rank, world, local_rank):
     if sampler:
         sampler.stop()
 
-    bpt = bytes_per_head_token(wl.bits, wl.group, D)
-    kv_bytes = [B * H * lens_at(args.warmup + i) * bpt for i in range(args.steps)]
+    kv_bytes = [kv_bytes_at(args.warmup + i) for i in range(args.steps)]
     q_bytes = B * Hq * D * 2
     alg_bytes = sum(kv_bytes) + args.steps * q_bytes
     tokens = B * args.steps * world
     value = tokens / (ms / 1e3)
 
     # ---- end to end through the public call with pinned host buffers
-    kn_h = kn.cpu().pin_memory()
+    kn_h = kn.cpu().pin_memory() if kn is not None else None
     qs_h = qs.cpu().pin_memory()
-    k_d = torch.empty_like(kn[0, 0])
-    v_d = torch.empty_like(kn[0, 1])
+    k_d = torch.empty_like(kn[0, 0]) if kn is not None else None
+    v_d = torch.empty_like(kn[0, 1]) if kn is not None else None
     q_d = torch.empty_like(qs[0])
     out_h = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
     lse_h = torch.empty((B, Hq), dtype=torch.float32).pin_memory()
-    cache.seq_lens.copy_(base_lens)
+    if wl.append:
+        cache.seq_lens.copy_(base_lens)
 
     def e2e_step(s):
         e = s % episode
@@ -373,7 +485,7 @@ def run_kvq(args, wl, rank, world, local_rank):
         q_d.copy_(qs_h[e], non_blocking=True)
         if wl.append:
             kvq.kvq_quantize_append(cache, k_d, v_d, 1, advance_seq_lens=True)
-        kvq.kvq_decode_attention(cache, q_d, out, lse, ws, max_len_hint=hint)
+        kvq.kvq_decode_attention(segs, q_d, out, lse, ws, max_len_hint=hint)
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
 
@@ -394,7 +506,7 @@ def run_kvq(args, wl, rank, world, local_rank):
         t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e_ms = float(t.item())
-    h2d = (kn[0].numel() * 2 if wl.append else 0) + qs[0].numel() * 2
+    h2d = (kn[0].numel() * 2 if kn is not None else 0) + qs[0].numel() * 2
     d2h = out.numel() * 4 + lse.numel() * 4
 
     if rank != 0:
@@ -409,9 +521,14 @@ def run_kvq(args, wl, rank, world, local_rank):
         "config": workload_config(wl, {
             "global_batch": B * world, "parallelism": f"dp{world} (sequences sharded)",
             "cache_tokens_per_step": f"{ctx + 1}..{ctx + episode}" if wl.append else ctx,
+            **({"chunk_tokens": wl.chunk_tokens, "alpha": wl.alpha, "beta": wl.beta,
+                "segments": {f"bits{b}": int(ln.sum()) for b, ln in zip(seg_bits, seg_lens)}}
+               if seg_lens is not None else {}),
             "l2": f"inputs larger than L2: {sum(kv_bytes) / args.steps / 1e6:.0f} MB of packed "
                   f"K/V read per step per GPU (L2 126 MB)",
-            "step": "quantize-append 1 token/seq + split-K decode attention + LSE merge"}),
+            "step": ("quantize-append 1 token/seq + split-K decode attention + LSE merge"
+                     if wl.append else
+                     "split-K decode attention over the FP16/INT4/INT2 segments + LSE merge")}),
         "kv_read_gbs": sum(kv_bytes) / (ms / 1e3) / 1e9 * world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
@@ -425,8 +542,11 @@ def run_kvq(args, wl, rank, world, local_rank):
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, k, v, kn[0, 0], kn[0, 1], qs[0],
-                                            args.cpu_seconds)
+        if wl.chunk_tokens:
+            line["cpu_baseline"] = cpu_baseline_mixed(wl, k, v, qs[0], args.cpu_seconds, wlr)
+        else:
+            line["cpu_baseline"] = cpu_baseline(wl, k, v, kn[0, 0], kn[0, 1], qs[0],
+                                                args.cpu_seconds)
     return line
 
 
