@@ -56,15 +56,16 @@ kvq_status check_cache(const kvq_cache* c, bool allow16) {
 // unit.  The fixed cost -- the start of a unit waits for its query rows and
 // first copies -- was measured at about 400 tokens' worth of work.  The result depends only on
 // (sequences x KV heads, length), so it is cached per thread.
-int choose_splits(const kvq_cache& c, int max_len_hint) {
+int choose_splits(const kvq_cache& c, int max_len_hint, int ctas_per_sm) {
   const long long pairs = (long long)c.batch * c.kv_heads;
   long long len = c.max_tokens;
   if (max_len_hint > 0 && max_len_hint < len) len = max_len_hint;
   if (len <= 0 || pairs <= 0) return 1;
-  thread_local long long cached_pairs = -1, cached_len = -1;
+  thread_local long long cached_pairs = -1, cached_len = -1, cached_slots = -1;
   thread_local int cached_n = 1;
-  if (pairs == cached_pairs && len == cached_len) return cached_n;
-  constexpr long long kSlots = 148LL * 3, kOverhead = 400, kGran = 32, kMinTokens = 128;
+  const long long kSlots = 148LL * (ctas_per_sm > 0 ? ctas_per_sm : 3);
+  if (pairs == cached_pairs && len == cached_len && kSlots == cached_slots) return cached_n;
+  constexpr long long kOverhead = 400, kGran = 32, kMinTokens = 128;
   const long long cap = (len + kMinTokens - 1) / kMinTokens;
   long long best_n = 1, best_cost = -1;
   for (long long n = 1; n <= cap && n <= 4096; ++n) {
@@ -78,6 +79,7 @@ int choose_splits(const kvq_cache& c, int max_len_hint) {
   }
   cached_pairs = pairs;
   cached_len = len;
+  cached_slots = kSlots;
   cached_n = (int)best_n;
   return cached_n;
 }
@@ -87,10 +89,14 @@ struct SplitPlan {
   int parts;
 };
 
-kvq_status plan_splits(const kvq_cache* segs, int n_segs, int max_len_hint, SplitPlan* plan) {
+kvq_status plan_splits(const kvq_cache* segs, int n_segs, int q_heads, int max_len_hint,
+                       SplitPlan* plan) {
   plan->parts = 0;
+  const int g = q_heads / segs[0].kv_heads;
   for (int i = 0; i < n_segs; ++i) {
-    plan->n_split[i] = choose_splits(segs[i], max_len_hint);
+    const int bits = segs[i].k.bits;
+    const int ctas = kvq::decode_ctas_per_sm(bits, bits == 16 ? kD : segs[i].k.group_size, g);
+    plan->n_split[i] = choose_splits(segs[i], max_len_hint, ctas);
     plan->parts += plan->n_split[i];
   }
   return KVQ_OK;
@@ -198,7 +204,7 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache* segs, int32_t n_segs, int
   kvq_status st = check_segments(segs, n_segs, q_heads);
   if (st != KVQ_OK) return st;
   SplitPlan plan;
-  plan_splits(segs, n_segs, max_len_hint, &plan);
+  plan_splits(segs, n_segs, q_heads, max_len_hint, &plan);
   *bytes = workspace_for(segs, q_heads, plan.parts);
   return KVQ_OK;
 }
@@ -221,7 +227,7 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
   for (int i = 0; i < n_segs; ++i)
     if (segs[i].k.bits == 16 && q_dtype == KVQ_BF16) return KVQ_ERR_UNSUPPORTED;
   SplitPlan plan;
-  plan_splits(segs, n_segs, max_len_hint, &plan);
+  plan_splits(segs, n_segs, q_heads, max_len_hint, &plan);
   const size_t need = workspace_for(segs, q_heads, plan.parts);
   if (workspace == nullptr || workspace_bytes < need) return KVQ_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KVQ_ERR_INVALID_ARG;

@@ -27,6 +27,7 @@
 #include <atomic>
 #include <type_traits>
 
+#include "kvq_decode_common.cuh"
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
@@ -70,41 +71,6 @@ struct Cfg {
   static constexpr int CROSS = (BITS == 16) ? 2 : (BITS == 8 ? 4 : (BITS == 4 ? 8 : 16));
   static constexpr int PER_W = (NTG < CROSS) ? NTG : CROSS;  // V n-tiles per word
   static constexpr int EMAX = WordPairs<BITS>::kEmax;
-};
-
-// 2^n as an exact float constant (|n| <= 60).
-__host__ __device__ constexpr float pow2f(int n) {
-  return n >= 0 ? float(1ull << (n > 60 ? 60 : n)) : 1.0f / float(1ull << (-n > 60 ? 60 : -n));
-}
-
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-  return h2_as_u32(__floats2half2_rn(a, b));
-}
-
-// Load `n` bytes (1, 2 or a multiple of 4) of a lane's chunk into words.
-template <int NBYTES, int NW>
-__device__ __forceinline__ void load_chunk(const uint8_t* p, uint32_t (&w)[NW]) {
-  if constexpr (NBYTES == 1) {
-    w[0] = *p;
-  } else if constexpr (NBYTES == 2) {
-    w[0] = *reinterpret_cast<const uint16_t*>(p);
-  } else if constexpr (NBYTES % 16 == 0) {
-#pragma unroll
-    for (int i = 0; i < NBYTES / 16; ++i) {
-      uint4 v = reinterpret_cast<const uint4*>(p)[i];
-      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-    }
-  } else if constexpr (NBYTES == 8) {
-    uint2 v = *reinterpret_cast<const uint2*>(p);
-    w[0] = v.x; w[1] = v.y;
-  } else {
-    w[0] = *reinterpret_cast<const uint32_t*>(p);
-  }
-}
-
-struct SplitParams {
-  DecodeArgs a;
-  SegView seg;
 };
 
 // Token order inside an 8-token n-tile: MMA column n reads token row
@@ -174,12 +140,10 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   // stage's copy never runs past round_up(seq_len, 32) <= max_tokens)
   int L = seg.seq_lens[b];
   L = max(0, min(L, seg.max_tokens));
-  // a unit is `chunk` tokens (a multiple of the 32-token stage); its stages
-  // go to the four warps round-robin: warp w takes stages w, w + 4, ...
-  const int per_split = (L + seg.n_split - 1) / seg.n_split;
-  const int chunk = ((per_split + 31) / 32) * 32;
-  const int c0 = split * chunk;
-  const int c1 = min(c0 + chunk, L);
+  // a unit is a whole number of 32-token stages; its stages go to the four
+  // warps round-robin: warp w takes stages w, w + 4, ...
+  int c0, c1;
+  split_range(L, seg.n_split, split, c0, c1);
   const int unit_stages = (c1 > c0) ? (c1 - c0 + C::STOK - 1) / C::STOK : 0;
   const int n_tiles = (unit_stages > warp) ? (unit_stages - warp + kWarps - 1) / kWarps : 0;
   const int w0 = c0 + warp * C::STOK;  // first token of this warp's first stage
@@ -209,22 +173,7 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   }
 
   // ---- the g query rows of this KV head, once per unit, as fp16 in smem
-  // (bf16 queries are used through fp16: exact for |q| in [2^-14, 65504])
-  {
-    const long long qbase = ((long long)b * a.q_heads + (long long)kvh * g) * D;
-    if (t < g * (D / 8)) {
-      const uint4 raw = reinterpret_cast<const uint4*>(
-          static_cast<const uint16_t*>(a.q) + qbase)[t];
-      uint4 h16 = raw;
-      if (a.q_is_bf16) {
-        const __nv_bfloat162* bb = reinterpret_cast<const __nv_bfloat162*>(&raw);
-        __half2* hh = reinterpret_cast<__half2*>(&h16);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) hh[i] = __float22half2_rn(__bfloat1622float2(bb[i]));
-      }
-      reinterpret_cast<uint4*>(q_sm)[t] = h16;
-    }
-  }
+  stage_queries<g>(a, b, kvh, q_sm, t);
   __syncthreads();
   // sum of q over each (group, head) row, in the MMA's units (the QK MMA
   // returns 2^(EMAX - 24) * sum(q * c))
@@ -302,8 +251,10 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   float corr[C::NG];
 #pragma unroll
   for (int i = 0; i < C::NG; ++i) corr[i] = 0.f;
-  // m_run is a reference point, not the exact max: p = 2^(x - m_run) may
-  // reach 2^kLazy before the accumulators are rescaled
+  // m_run is a reference point at least as large as every score seen, so
+  // p = 2^(x - m_run) <= 1 and P' = p * s_V stays within fp16 range; it
+  // moves (with a rescale) only when a stage's max exceeds it, and then to
+  // that max + kLazy
   constexpr float kLazy = 4.0f;
   float m_run = -INFINITY, l_part = 0.f;
   int failed_at = -1;
@@ -426,18 +377,19 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
       }
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-    if (m_run == -INFINITY) {
-      m_run = tmax;  // nothing accumulated yet: no rescale needed
-    } else if (tmax > m_run + kLazy) {
-      const float alpha = fast_exp2(m_run - tmax);
+    if (tmax > m_run) {
+      const float m_new = tmax + kLazy;
+      if (m_run != -INFINITY) {  // nothing accumulated yet: no rescale needed
+        const float alpha = fast_exp2(m_run - m_new);
 #pragma unroll
-      for (int n = 0; n < 16; ++n)
+        for (int n = 0; n < 16; ++n)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) o_acc[n][c] *= alpha;
+          for (int c = 0; c < 4; ++c) o_acc[n][c] *= alpha;
 #pragma unroll
-      for (int gr = 0; gr < C::NG; ++gr) corr[gr] *= alpha;
-      l_part *= alpha;
-      m_run = tmax;
+        for (int gr = 0; gr < C::NG; ++gr) corr[gr] *= alpha;
+        l_part *= alpha;
+      }
+      m_run = m_new;
     }
     float p[NS][4];
 #pragma unroll
@@ -574,61 +526,10 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
     }
   }
   __syncthreads();
-  // per head: the max over the warps, each warp's weight 2^(m_w - M) and
-  // the total sum, computed once (thread h), then one FMA per warp per dim
-  float* wt = os + kWarps * 8 * D;  // [8][kWarps] weights, then M[8], L[8]
-  float* Mh = wt + 8 * kWarps;
-  float* Lh = Mh + 8;
-  if (t < g) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w)
-      if (ls[w * 8 + t] > 0.f) M = fmaxf(M, ms[w * 8 + t]);
-    float Ls = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float x = (ls[w * 8 + t] > 0.f) ? exp2f(ms[w * 8 + t] - M) : 0.f;
-      wt[t * kWarps + w] = x;
-      Ls += x * ls[w * 8 + t];
-    }
-    Mh[t] = M;
-    Lh[t] = Ls;
-  }
-  __syncthreads();
-  const int part = seg.part_base + split;
-#pragma unroll
-  for (int h = 0; h < g; ++h) {
-    float O = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) O = fmaf(wt[h * kWarps + w], os[(w * 8 + h) * D + t], O);
-    const float M = Mh[h], Ls = Lh[h];
-    const long long bh = (long long)b * a.q_heads + (long long)kvh * g + h;
-    if (a.parts == 1) {
-      a.out[bh * D + t] = (Ls > 0.f) ? O / Ls : 0.f;
-      if (a.lse != nullptr && t == 0)
-        a.lse[bh] = (Ls > 0.f) ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
-    } else {
-      const long long pi = bh * a.parts + part;
-      a.part_o[pi * D + t] = O;
-      if (t == 0) {
-        a.part_ml[pi * 2 + 0] = M;
-        a.part_ml[pi * 2 + 1] = Ls;
-      }
-    }
-  }
+  cta_merge_store<g>(a, ms, ls, os, os + kWarps * 8 * D, b, kvh, seg.part_base + split, t);
   }  // unit loop
 
-  // The last CTA to finish resets the counters for the next launch on this
-  // workspace (nothing waits on them).
-  if (t == 0) {
-    __threadfence();
-    const unsigned done = atomicAdd(&counters[1], 1u);
-    if (done == gridDim.x - 1) {
-      atomicExch(&counters[0], 0u);
-      atomicExch(&counters[1], 0u);
-      __threadfence();
-    }
-  }
+  if (t == 0) release_counters(counters);
 }
 
 // Merge the partial (m, l, o) of every split and segment (log-sum-exp).
@@ -705,7 +606,7 @@ template <int BITS, int GE>
 cudaError_t launch_split(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   constexpr int NG = kHeadDim / GE;
   switch (a.group_ratio) {
-    case 1: return launch_split_g<BITS, GE, 1>(a, seg, s);
+    case 1: return launch_decode_mha(a, seg, s);  // one head per KV head
     case 2: return launch_split_g<BITS, GE, 2>(a, seg, s);
     case 4:
       if constexpr (NG * 4 <= 16) return launch_split_g<BITS, GE, 4>(a, seg, s);
@@ -726,6 +627,13 @@ bool decode_supported(int bits, int group, int group_ratio) {
   if (!(bits == 2 || bits == 4 || bits == 8)) return false;
   if (!(group == 32 || group == 64 || group == 128)) return false;
   return (kHeadDim / group) * group_ratio <= 16;
+}
+
+int decode_ctas_per_sm(int bits, int group, int group_ratio) {
+  if (group_ratio == 1) return decode_mha_ctas_per_sm(bits, group);
+  (void)bits;
+  (void)group;
+  return Cfg<4, 64>::MIN_CTAS;  // the same for every format
 }
 
 int decode_smem_bytes(int bits, int group) {

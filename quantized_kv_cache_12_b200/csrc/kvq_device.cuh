@@ -160,14 +160,15 @@ struct WordPairs<2> {
 template <>
 struct WordPairs<8> {
   static constexpr int kPairs = 2, kDims = 4, kEmax = 0;
+  // bytes 1 and 3 are moved down by a byte permute with zero fill
   __device__ __forceinline__ static void run(uint32_t w, uint32_t (&p)[2]) {
     p[0] = w & 0x00FF00FFu;
-    p[1] = (w >> 8) & 0x00FF00FFu;
+    p[1] = prmt(w, 0u, 0x4341u);
   }
   __host__ __device__ static constexpr int dim(int j, int e) { return j + 2 * e; }
   __host__ __device__ static constexpr int exp(int) { return 0; }
   __device__ __forceinline__ static uint32_t one(uint32_t w, int j) {
-    return (j ? (w >> 8) : w) & 0x00FF00FFu;
+    return j ? prmt(w, 0u, 0x4341u) : (w & 0x00FF00FFu);
   }
 };
 
@@ -230,9 +231,9 @@ struct CrossPairs<8> {
     const uint32_t x = prmt(a, b, 0x5410u);  // [a.b0 a.b1 b.b0 b.b1]
     const uint32_t y = prmt(a, b, 0x7632u);  // [a.b2 a.b3 b.b2 b.b3]
     o[0] = x & 0x00FF00FFu;
-    o[1] = (x >> 8) & 0x00FF00FFu;
+    o[1] = prmt(x, 0u, 0x4341u);              // [x.b1 0 x.b3 0]
     o[2] = y & 0x00FF00FFu;
-    o[3] = (y >> 8) & 0x00FF00FFu;
+    o[3] = prmt(y, 0u, 0x4341u);
   }
   __host__ __device__ static constexpr int exp(int) { return 0; }
 };
