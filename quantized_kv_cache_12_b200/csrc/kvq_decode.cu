@@ -602,22 +602,6 @@ cudaError_t launch_split_g(const DecodeArgs& a, const SegView& seg, cudaStream_t
   return cudaGetLastError();
 }
 
-template <int BITS, int GE>
-cudaError_t launch_split(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
-  constexpr int NG = kHeadDim / GE;
-  switch (a.group_ratio) {
-    case 1: return launch_decode_mha(a, seg, s);  // one head per KV head
-    case 2: return launch_split_g<BITS, GE, 2>(a, seg, s);
-    case 4:
-      if constexpr (NG * 4 <= 16) return launch_split_g<BITS, GE, 4>(a, seg, s);
-      break;
-    case 8:
-      if constexpr (NG * 8 <= 16) return launch_split_g<BITS, GE, 8>(a, seg, s);
-      break;
-  }
-  return cudaErrorInvalidValue;
-}
-
 }  // namespace
 
 bool decode_supported(int bits, int group, int group_ratio) {
@@ -630,31 +614,20 @@ bool decode_supported(int bits, int group, int group_ratio) {
 }
 
 int decode_ctas_per_sm(int bits, int group, int group_ratio) {
-  if (group_ratio == 1) return decode_mha_ctas_per_sm(bits, group);
-  (void)bits;
-  (void)group;
+  if (decode_tm_supported(bits, group, group_ratio))
+    return decode_tm_ctas_per_sm(bits, group, group_ratio);
   return Cfg<4, 64>::MIN_CTAS;  // the same for every format
-}
-
-int decode_smem_bytes(int bits, int group) {
-#define KVQ_S(B, G_) \
-  if (bits == B && group == G_) return Cfg<B, G_>::SMEM;
-  KVQ_S(16, 128)
-  KVQ_S(8, 32) KVQ_S(8, 64) KVQ_S(8, 128)
-  KVQ_S(4, 32) KVQ_S(4, 64) KVQ_S(4, 128)
-  KVQ_S(2, 32) KVQ_S(2, 64) KVQ_S(2, 128)
-#undef KVQ_S
-  return 0;
 }
 
 cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   const int bits = seg.bits, group = (seg.bits == 16) ? kHeadDim : seg.group;
-#define KVQ_D(B, G_) \
-  if (bits == B && group == G_) return launch_split<B, G_>(a, seg, s);
-  KVQ_D(16, 128)
-  KVQ_D(8, 32) KVQ_D(8, 64) KVQ_D(8, 128)
-  KVQ_D(4, 32) KVQ_D(4, 64) KVQ_D(4, 128)
-  KVQ_D(2, 32) KVQ_D(2, 64) KVQ_D(2, 128)
+  // (group, head) columns that fit one 8-wide tile: tokens-on-M kernel
+  if (decode_tm_supported(bits, group, a.group_ratio)) return launch_decode_tm(a, seg, s);
+  // 16 (group, head) rows: this file's kernel
+#define KVQ_D(B, G_, R) \
+  if (bits == B && group == G_ && a.group_ratio == R) return launch_split_g<B, G_, R>(a, seg, s);
+  KVQ_D(8, 64, 8) KVQ_D(4, 64, 8) KVQ_D(2, 64, 8)
+  KVQ_D(8, 32, 4) KVQ_D(4, 32, 4) KVQ_D(2, 32, 4)
 #undef KVQ_D
   return cudaErrorInvalidValue;
 }

@@ -52,12 +52,13 @@ struct QuantArgs {
 // Per-bit-width launchers (kvq_quantize.cu, kvq_decode.cu, kvq_chunk.cu).
 cudaError_t launch_quantize(const QuantArgs& a, int bits, int group, cudaStream_t s);
 bool decode_supported(int bits, int group, int group_ratio);
-int decode_smem_bytes(int bits, int group);
 // resident decode CTAs per SM for a segment format and query-group ratio
 int decode_ctas_per_sm(int bits, int group, int group_ratio);
-int decode_mha_ctas_per_sm(int bits, int group);
+// the tokens-on-M kernel (kvq_decode_tm.cu): formats with NG * g <= 8
+bool decode_tm_supported(int bits, int group, int group_ratio);
+int decode_tm_ctas_per_sm(int bits, int group, int group_ratio);
 cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
-cudaError_t launch_decode_mha(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
+cudaError_t launch_decode_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_chunk_assign(const float* emb, const float* qemb, int batch, int n_chunks,
                                 int emb_dim, double alpha, double beta, double* sim,

@@ -111,10 +111,11 @@ def test_edge_lengths(kvq):
     np.testing.assert_allclose(o[1, 0], v1[0], atol=1e-5)
 
 
-def test_fp16_segment(kvq):
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_fp16_segment(kvq, g):
     """Raw fp16 rows (Cocktail's FP16 class), ragged lengths, NaN bytes past
-    the valid length."""
-    wl = workloads.WORKLOADS["cocktail_mixed"].scaled(kv_heads=3, q_heads=3)
+    the valid length, one to eight query heads per KV head."""
+    wl = workloads.WORKLOADS["cocktail_mixed"].scaled(kv_heads=3, q_heads=3 * g)
     lens = [45, 100]
     B = len(lens)
     k, v = workloads.kv_tokens(wl, 100, DEV, batch=B)
@@ -128,7 +129,58 @@ def test_fp16_segment(kvq):
     out, lse = _run(kvq, c, q)
     seg = oracle_segment(k, v, 16, 128)
     ref, lref = oracle.decode_attention(q_bits(q), False, [seg], [lens], 128 ** -0.5)
-    assert_close(out, ref, lse, lref, what="fp16 segment")
+    assert_close(out, ref, lse, lref, what=f"fp16 segment g{g}")
+
+
+@pytest.mark.parametrize("bits,G,g", [(2, 32, 1), (2, 32, 2), (4, 64, 4), (8, 128, 8),
+                                      (2, 64, 8), (4, 32, 4)])
+def test_large_magnitude_values(kvq, bits, G, g):
+    """V entries in the tens of thousands (INT2 scales near 3 * 10^4): the
+    weights p * s_V fed to the fp16 tensor-core operand must stay finite.
+    Compared after dividing by the magnitude, so the tolerance applies to the
+    N(0, 1)-sized values."""
+    mag = 500.0  # the x20 outlier channels reach ~45000, inside fp16 range
+    wl = workloads.WORKLOADS["long_gqa_int4"].scaled(kv_heads=2, q_heads=2 * g, bits=bits,
+                                                     group=G)
+    lens = [200, 97]
+    B = len(lens)
+    k, v = workloads.kv_tokens(wl, 200, DEV, batch=B)
+    v = (v.float() * mag).half()
+    assert torch.isfinite(v).all() and v.abs().max() > 2.0e4
+    q = workloads.queries(wl, DEV, batch=B)
+    c = kvq.QuantizedKVCache.allocate(B, 2, 128, 256, bits, G, DEV)
+    _poison(c)
+    fill_cache(kvq, c, k, v, lens)
+    out, lse = _run(kvq, c, q)
+    seg = oracle_segment(k, v, bits, G)
+    ref, lref = oracle.decode_attention(q_bits(q), q.dtype == torch.bfloat16, [seg], [lens],
+                                        128 ** -0.5)
+    assert_close(out / mag, ref / mag, lse, lref, what=f"large values bits{bits} G{G} g{g}")
+
+
+@pytest.mark.parametrize("bits,G,g", [(4, 128, 1), (4, 128, 2), (8, 128, 8), (4, 64, 4),
+                                      (2, 32, 2), (2, 64, 8)])
+def test_rising_scores_rescale(kvq, bits, G, g):
+    """Keys whose magnitude grows along the sequence make every head's running
+    max rise stage after stage, at different stages for different heads, so
+    the accumulators are rescaled many times."""
+    wl = workloads.WORKLOADS["long_gqa_int4"].scaled(kv_heads=2, q_heads=2 * g, bits=bits,
+                                                     group=G)
+    lens = [600, 333]
+    B = len(lens)
+    T = max(lens)
+    k, v = workloads.kv_tokens(wl, T, DEV, batch=B)
+    ramp = torch.linspace(0.2, 3.0, T, device=DEV).view(1, 1, T, 1)
+    k = (k.float() * ramp).half()
+    q = workloads.queries(wl, DEV, batch=B)
+    c = kvq.QuantizedKVCache.allocate(B, 2, 128, 640, bits, G, DEV)
+    _poison(c)
+    fill_cache(kvq, c, k, v, lens)
+    out, lse = _run(kvq, c, q, max_len_hint=64)  # one split: one long running max
+    seg = oracle_segment(k, v, bits, G)
+    ref, lref = oracle.decode_attention(q_bits(q), q.dtype == torch.bfloat16, [seg], [lens],
+                                        128 ** -0.5)
+    assert_close(out, ref, lse, lref, what=f"rising scores bits{bits} G{G} g{g}")
 
 
 def test_mixed_segments_equal_unchunked(kvq):
