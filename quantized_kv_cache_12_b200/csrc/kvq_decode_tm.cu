@@ -15,21 +15,28 @@
 // so the code conversions (the bulk of the instruction count) are done once
 // per token for all heads and groups, and no MMA row is padding.
 //
-// Lane roles (gid = lane / 4, tig = lane % 4), per 16-token sub-tile:
-//   QK: A rows gid, gid + 8 are tokens gid, gid + 8; the lane's k elements are
-//       its 32-dim chunk [32 tig, 32 tig + 32) of those tokens.  Accumulator
-//       columns 2 tig, 2 tig + 1 give the lane, for its two tokens, either the
-//       scores of heads 2 tig and 2 tig + 1 (NG = 1: two head slots), of head
-//       tig (NG = 2), or half of the score of head tig / 2 (NG = 4, completed
-//       by one shuffle).  The softmax runs here, per head slot.
-//   PV: k positions 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9 are tokens tig,
-//       tig + 4, tig + 8, tig + 12 (that order makes a warp's V loads one
-//       contiguous block); A rows gid, gid + 8 of m-tile mt are dims
-//       16 gid + mt and 16 gid + mt + 8, so a lane reads the 16 contiguous dims
-//       [16 gid, 16 gid + 16) of each of its four tokens; B column gid of
-//       n-tile nt is column nt * 8 + gid = (h, gr, part) of P'.
-// The output for head h and dim d sits in n-tile (h * 2NG + 2 group(d)) / 8,
-// lane (d / 16, (h * 2NG + 2 group(d)) % 8 / 2), columns hi + lo.
+// Lane roles (gid = lane / 4, tig = lane % 4), per 16-token sub-tile.  A
+// sub-tile's MMA rows r = 0 .. 15 are its tokens perm(r) = r ^ ((r >> 2) & 1)
+// (an order that keeps the shared-memory loads below free of bank
+// conflicts for the 2- and 4-bit formats).
+//   QK: A rows gid, gid + 8; the lane's k elements are its 32-dim chunk
+//       [32 tig, 32 tig + 32) of those two tokens.  B column c holds query
+//       head (c / CPH) mod g masked to group c mod NG, where CPH (columns per
+//       head) is chosen so that the two accumulator columns 2 tig, 2 tig + 1
+//       of a lane give it whole heads: the scores of heads 2 tig and 2 tig + 1
+//       (g = 8, NG = 1), or of one head, complete (NG <= 2) or in two halves
+//       added by one shuffle (NG = 4).  Unused columns repeat a head.  The
+//       online softmax and the weights P' = p * s_V (split into an fp16 high
+//       part and the negated fp16 remainder) are computed here, per owned
+//       head, for the lane's two tokens.
+//   PV: the weights go to the B operand by 8x8 transposes (movmatrix): B
+//       column 2 tig + part of n-tile b is (head, V group) combination (b, tig)
+//       of QK lane tig, so the accumulator columns 2 tig, 2 tig + 1 of a PV
+//       lane belong to the same lane position that owns their head: rescale
+//       factors and zero-point corrections never cross lanes.  A rows gid,
+//       gid + 8 of m-tile mt are dims 16 gid + mt and 16 gid + mt + 8; the k
+//       positions 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9 are rows 2 tig, 2 tig + 1,
+//       2 tig + 8, 2 tig + 9 of the sub-tile, whose V codes the lane converts.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -54,10 +61,13 @@ struct TmCfg {
   static constexpr int KW = KC / 4;
   static constexpr int VB = RB / 8;                    // V bytes of a lane (16 dims)
   static constexpr int VW = VB / 4;
-  static constexpr int NCQ = NG * GR;                  // QK columns (h, gr)
-  static constexpr int NCP = 2 * NCQ;                  // PV columns (h, gr, part)
-  static constexpr int NP = (NCP + 7) / 8;             // PV n-tiles
-  static constexpr int HS = (NG == 1 && GR > 1) ? 2 : 1;  // head slots of a QK lane
+  // QK columns per head (see the file comment), head slots of a QK lane,
+  // PV n-tiles, and lane positions whose (head, V group) combinations are
+  // distinct
+  static constexpr int CPH = (NG == 1 && GR == 8) ? 1 : ((NG == 4 || (NG == 2 && GR <= 2)) ? 4 : 2);
+  static constexpr int HS = CPH == 1 ? 2 : 1;
+  static constexpr int NP = (NG * GR + 3) / 4;
+  static constexpr int W = NG * GR < 4 ? NG * GR : 4;
   static constexpr int SUB = (BITS == 16) ? 1 : 2;     // 16-token sub-tiles per stage
   static constexpr int STOK = SUB * kTile;
   static constexpr int STAGE = 2 * STOK * RB + 2 * STOK * MB;
@@ -78,12 +88,37 @@ struct TmCfg {
   static constexpr int EMAX = WordPairs<BITS>::kEmax;
   // the warp merge reuses the stage buffers: m, l, o of kWarps x 8 rows
   static constexpr int MERGE_BYTES = (2 * kWarps * 8 + kWarps * 8 * D + 8 * (kWarps + 2)) * 4;
-  static_assert(NCQ <= 8, "at most eight (head, group) columns");
+  static_assert(NG * GR <= 8, "at most eight (head, group) combinations");
   static_assert(kWarps * STAGES * 8 <= HDR_Q, "mbarriers fit the header");
   static_assert(MERGE_BYTES <= kWarps * STAGES * STAGE, "merge scratch fits the stages");
   static_assert(WordPairs<BITS>::kPairs * KW == 16, "16 K pairs per lane and token");
   static_assert(CrossPairs<BITS>::kOut * VW == 16, "16 V dims per lane and token");
 };
+
+// Token of MMA row r (0 .. 15) of a 16-token sub-tile.
+__device__ __forceinline__ int tok_perm(int r) { return r ^ ((r >> 2) & 1); }
+
+// 8x8 transpose of 16-bit elements across the warp: lane (gid, tig) gets
+// elements (2 tig, gid) and (2 tig + 1, gid) of the matrix whose row gid,
+// columns 2 tig, 2 tig + 1 it passed in.
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+// Two weights as (hi, -lo) pairs: hi = fp16(x), -lo = fp16(hi - x), the
+// remainder formed exactly in fp32 from the fp16 hi.
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& r0, uint32_t& r1) {
+  const uint32_t hh = pack_h2(x0, x1);
+  float n0, n1;
+  asm("{.reg .f16 l, h;\n mov.b32 {l, h}, %2;\n sub.rn.f32.f16 %0, l, %3;\n"
+      " sub.rn.f32.f16 %1, h, %4;\n}"
+      : "=f"(n0), "=f"(n1)
+      : "r"(hh), "f"(x0), "f"(x1));
+  r0 = pack_h2(x0, n0);
+  r1 = pack_h2(x1, n1);
+}
 
 template <int BITS, int GE, int GR>
 __global__ void __launch_bounds__(kWarps * 32, TmCfg<BITS, GE, GR>::MIN_CTAS)
@@ -91,7 +126,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   using C = TmCfg<BITS, GE, GR>;
   using WP = WordPairs<BITS>;
   using XP = CrossPairs<BITS>;
-  constexpr int D = C::D, NG = C::NG, NP = C::NP, HS = C::HS;
+  constexpr int D = C::D, NG = C::NG, NP = C::NP, HS = C::HS, CPH = C::CPH;
   const DecodeArgs& a = P.a;
   const SegView& seg = P.seg;
 
@@ -102,47 +137,33 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::HDR_BARS) + warp * C::STAGES;
   __half* q_sm = reinterpret_cast<__half*>(smem + C::HDR_Q);      // [GR][D]
-  float* qs_sm = reinterpret_cast<float*>(smem + C::HDR_QS);      // [NCQ]
+  float* qs_sm = reinterpret_cast<float*>(smem + C::HDR_QS);      // [8] per QK column
   int* unit_sm = reinterpret_cast<int*>(smem + C::HDR_MISC);
   int* fail_sm = unit_sm + 1;
   uint8_t* stages = smem + C::HDR_BYTES + warp * C::STAGES * C::STAGE;
   uint32_t* counters = a.err + 1;  // [0] next unit, [1] CTAs done
 
   // ---- per-lane constants
-  // QK B column gid = (head qh, group qg); this lane's K chunk is in group kgrp
+  // QK B column gid: head (gid / CPH) mod g, group gid mod NG; the lane's K
+  // chunk lies in group kgrp
   const int kgrp = (32 * tig) / GE;
-  const bool qb_ok = gid < C::NCQ && (gid % NG) == kgrp;
-  const int qh = (gid < C::NCQ) ? gid / NG : 0;
-  // QK accumulator columns 2 tig, 2 tig + 1
-  const bool colA = 2 * tig < C::NCQ, colB = 2 * tig + 1 < C::NCQ;
-  const int meta_off = 4 * ((2 * tig) % NG);  // (s, z) of column 2 tig's group
-  // head of QK slot s of this lane (valid if < GR)
-  auto slot_head = [&](int s) { return NG == 1 ? 2 * tig + s : (2 * tig) / NG; };
-  // PV B column nt * 8 + gid: head hb, group gv (the same in every n-tile),
-  // part gid & 1; its head's scores sit in QK lanes with tig = ts
-  const int gv = (gid >> 1) % NG;
-  const float lo_sel = (gid & 1) ? 1.f : 0.f;
-  bool pv_ok[NP];
-  int ts[NP], sl[NP];
+  const bool qb_ok = (gid % NG) == kgrp;
+  const int qh = (gid / CPH) % GR;
+  // heads owned by this lane (slot s) and the group of each PV block b
+  int own_h[HS];
 #pragma unroll
-  for (int nt = 0; nt < NP; ++nt) {
-    const int col = nt * 8 + gid;
-    const int hb = col / (2 * NG);
-    pv_ok[nt] = col < C::NCP;
-    ts[nt] = pv_ok[nt] ? (hb * NG) / 2 : 0;
-    sl[nt] = (HS == 2) ? (hb & 1) : 0;
-  }
-  // PV accumulator columns nt * 8 + 2 tig (+1): head ho, group tig % NG; the
-  // lane holds outputs where that group is the group of its 16 dims
-  int ho[NP];
-  bool writer[NP];
+  for (int s = 0; s < HS; ++s) own_h[s] = (CPH == 1) ? 2 * tig + s : ((2 * tig) / CPH) % GR;
+  auto slot_of = [](int b) { return HS == 2 ? b : 0; };
+  int gv[NP];
 #pragma unroll
-  for (int nt = 0; nt < NP; ++nt) {
-    ho[nt] = (nt * 8 + 2 * tig) / (2 * NG);
-    writer[nt] = ho[nt] < GR && (tig % NG) == (16 * gid) / GE;
-  }
+  for (int b = 0; b < NP; ++b)
+    gv[b] = NG == 1 ? 0 : (NG == 2 ? (NP == 2 ? b : (tig & 1)) : (NP == 2 ? 2 * b + (tig & 1) : tig));
+  const bool distinct = tig < C::W;        // this lane's combinations are not repeats
+  const int dgrp = (16 * gid) / GE;        // group of the lane's 16 output dims
   const float score_scale = a.scale_log2 * pow2f(24 - C::EMAX);
-  const int vt[4] = {tig, tig + 4, tig + 8, tig + 12};  // PV tokens of this lane
+  // tokens of the lane's QK rows and PV k positions within a sub-tile
+  const int tq0 = tok_perm(gid);
+  const int tvA = tok_perm(2 * tig), tvB = tok_perm(2 * tig + 1);
 
   const uint64_t policy = l2_evict_first_policy();
   int st = 0;  // the stage ring (position and phase) runs on across units
@@ -202,16 +223,14 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   if constexpr (BITS != 16) {
     if (t < 64) {
       const int r = t >> 3, part = t & 7;
+      const __half* qr = q_sm + ((r / CPH) % GR) * D + (r % NG) * GE + part * (GE / 8);
       float acc = 0.f;
-      if (r < C::NCQ) {
-        const __half* qr = q_sm + (r / NG) * D + (r % NG) * GE + part * (GE / 8);
 #pragma unroll 4
-        for (int i = 0; i < GE / 8; ++i) acc += __half2float(qr[i]);
-      }
+      for (int i = 0; i < GE / 8; ++i) acc += __half2float(qr[i]);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-      if (r < C::NCQ && part == 0) qs_sm[r] = acc * pow2f(C::EMAX - 24);
+      if (part == 0) qs_sm[r] = acc * pow2f(C::EMAX - 24);
     }
   }
   __syncthreads();
@@ -233,21 +252,21 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
       }
     }
   }
-  const float qsA = (BITS != 16 && colA) ? qs_sm[2 * tig] : 0.f;
-  const float qsB = (BITS != 16 && colB) ? qs_sm[2 * tig + 1] : 0.f;
+  const float qsA = (BITS != 16) ? qs_sm[2 * tig] : 0.f;
+  const float qsB = (BITS != 16) ? qs_sm[2 * tig + 1] : 0.f;
 
-  // ---- running state.  m_ref (per head slot) is a reference point at least
-  // as large as every score seen, so p = 2^(x - m_ref) <= 1 and P' = p * s_V
-  // stays within fp16 range; it moves (with a rescale) only when a stage's
-  // max exceeds it, and then to that max + kLazy.
+  // ---- running state.  m_ref (per owned head) is a reference point at
+  // least as large as every score seen, so p = 2^(x - m_ref) <= 1 and
+  // P' = p * s_V stays within fp16 range; it moves (with a rescale) only when
+  // a stage's max exceeds it, and then to that max + kLazy.
   float o_acc[NP][8][4];
 #pragma unroll
-  for (int nt = 0; nt < NP; ++nt)
+  for (int nb = 0; nb < NP; ++nb)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) o_acc[nt][i][0] = o_acc[nt][i][1] = o_acc[nt][i][2] = o_acc[nt][i][3] = 0.f;
-  float corr[NP];  // sum of P' * z_V for B column nt * 8 + gid
+    for (int i = 0; i < 8; ++i) o_acc[nb][i][0] = o_acc[nb][i][1] = o_acc[nb][i][2] = o_acc[nb][i][3] = 0.f;
+  float corr[NP];  // sum of P' * z_V of combination (b, tig) over this lane's tokens
 #pragma unroll
-  for (int nt = 0; nt < NP; ++nt) corr[nt] = 0.f;
+  for (int nb = 0; nb < NP; ++nb) corr[nb] = 0.f;
   constexpr float kLazy = 4.0f;
   float m_ref[HS], l_part[HS];
 #pragma unroll
@@ -265,14 +284,16 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     constexpr int NS = C::SUB;
     auto valid = [&](int tok) { return FULL || tok < n_valid; };  // tok: 0 .. STOK-1
 
-    // ---- S^T = K * Qx^T per sub-tile: this lane's rows are tokens gid, gid + 8
+    // ---- S^T = K * Qx^T per sub-tile: rows gid, gid + 8
     float x[NS][HS][2];
 #pragma unroll
     for (int sub = 0; sub < NS; ++sub) {
-      float s_acc[4] = {0.f, 0.f, 0.f, 0.f};
+      // two accumulators (even and odd k-steps): two dependent MMA chains of
+      // four instead of one of eight
+      float s_acc[4] = {0.f, 0.f, 0.f, 0.f}, s_odd[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t k0[C::KW], k1[C::KW];
-      load_chunk<C::KC, C::KW>(sK + (sub * kTile + gid) * C::RB + tig * C::KC, k0);
-      load_chunk<C::KC, C::KW>(sK + (sub * kTile + gid + 8) * C::RB + tig * C::KC, k1);
+      load_chunk<C::KC, C::KW>(sK + (sub * kTile + tq0) * C::RB + tig * C::KC, k0);
+      load_chunk<C::KC, C::KW>(sK + (sub * kTile + tq0 + 8) * C::RB + tig * C::KC, k1);
       uint32_t p0[16], p1[16];
 #pragma unroll
       for (int w = 0; w < C::KW; ++w) {
@@ -287,41 +308,39 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
       }
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        mma_f16(s_acc, p0[2 * ks], p1[2 * ks], p0[2 * ks + 1], p1[2 * ks + 1], qb[ks][0],
-                qb[ks][1]);
-      // score = sum over the head's group columns of s_K * (S - z_K * qs);
+        mma_f16((ks & 1) ? s_odd : s_acc, p0[2 * ks], p1[2 * ks], p0[2 * ks + 1],
+                p1[2 * ks + 1], qb[ks][0], qb[ks][1]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) s_acc[c] += s_odd[c];
+      // the owned heads' scores: sum over their groups of s_K * (S - z_K * qs);
       // rows past the valid length may hold any bytes: masked below by select
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
+        const int tok = sub * kTile + tq0 + 8 * r;
         float v[HS];
         if constexpr (BITS == 16) {
           v[0] = s_acc[2 * r];
-          if constexpr (HS == 2) v[1] = s_acc[2 * r + 1];
+          if constexpr (HS == 2) v[HS - 1] = s_acc[2 * r + 1];
+        } else if constexpr (NG == 1) {
+          const float2 sz = __half22float2(*reinterpret_cast<const __half2*>(sKm + tok * C::MB));
+          v[0] = sz.x * fmaf(-sz.y, qsA, s_acc[2 * r]);
+          if constexpr (HS == 2) v[HS - 1] = sz.x * fmaf(-sz.y, qsB, s_acc[2 * r + 1]);
         } else {
-          const uint8_t* m = sKm + (sub * kTile + gid + 8 * r) * C::MB + meta_off;
-          if constexpr (NG == 1) {
-            const float2 sz = __half22float2(*reinterpret_cast<const __half2*>(m));
-            v[0] = colA ? sz.x * fmaf(-sz.y, qsA, s_acc[2 * r]) : 0.f;
-            if constexpr (HS == 2) v[1] = colB ? sz.x * fmaf(-sz.y, qsB, s_acc[2 * r + 1]) : 0.f;
-          } else {
-            v[0] = 0.f;
-            if (colA) {
-              const uint2 u = *reinterpret_cast<const uint2*>(m);
-              const float2 szA = __half22float2(u32_as_h2(u.x));
-              const float2 szB = __half22float2(u32_as_h2(u.y));
-              v[0] = fmaf(szB.x, fmaf(-szB.y, qsB, s_acc[2 * r + 1]),
-                          szA.x * fmaf(-szA.y, qsA, s_acc[2 * r]));
-            }
-            if constexpr (NG == 4) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-          }
+          const uint2 u = *reinterpret_cast<const uint2*>(
+              sKm + tok * C::MB + (NG == 4 ? 8 * (tig & 1) : 0));
+          const float2 szA = __half22float2(u32_as_h2(u.x));
+          const float2 szB = __half22float2(u32_as_h2(u.y));
+          v[0] = fmaf(szB.x, fmaf(-szB.y, qsB, s_acc[2 * r + 1]),
+                      szA.x * fmaf(-szA.y, qsA, s_acc[2 * r]));
+          if constexpr (NG == 4) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
         }
-        const bool ok = valid(sub * kTile + gid + 8 * r);
+        const bool ok = valid(tok);
 #pragma unroll
         for (int s = 0; s < HS; ++s) x[sub][s][r] = ok ? v[s] * score_scale : -INFINITY;
       }
     }
 
-    // ---- online softmax per head slot: max over the stage's tokens (rows
+    // ---- online softmax per owned head: max over the stage's tokens (rows
     // gid and gid + 8 of every sub-tile, then across gid)
     bool any_rescale = false;
     float alpha[HS];
@@ -342,106 +361,73 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         }
         m_ref[s] = m_new;
       }
-      l_part[s] *= alpha[s];
     }
     if (__any_sync(0xffffffffu, any_rescale)) {
-      // the PV accumulators (columns of head ho) and corrections (B column
-      // of head hb) take the factor of their head from its QK lane
+      // every factor is this lane's own: the accumulator columns of PV block
+      // b belong to the lane position that owns their head
 #pragma unroll
-      for (int nt = 0; nt < NP; ++nt) {
-        const int src_o = 4 * gid + (ho[nt] < GR ? (ho[nt] * NG) / 2 : 0);
-        const int src_b = 4 * gid + ts[nt];
-        float ao = __shfl_sync(0xffffffffu, alpha[0], src_o);
-        float ab = __shfl_sync(0xffffffffu, alpha[0], src_b);
-        if constexpr (HS == 2) {
-          const float ao1 = __shfl_sync(0xffffffffu, alpha[1], src_o);
-          const float ab1 = __shfl_sync(0xffffffffu, alpha[1], src_b);
-          ao = (ho[nt] & 1) ? ao1 : ao;
-          ab = sl[nt] ? ab1 : ab;
-        }
+      for (int s = 0; s < HS; ++s) l_part[s] *= alpha[s];
+#pragma unroll
+      for (int nb = 0; nb < NP; ++nb) {
+        const float al = alpha[slot_of(nb)];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) o_acc[nt][i][c] *= ao;
-        corr[nt] *= ab;
+          for (int c = 0; c < 4; ++c) o_acc[nb][i][c] *= al;
+        corr[nb] *= al;
       }
     }
-    // p in the QK layout (0 for masked tokens)
+
+    // ---- weights and O^T += V^T * P'^T per sub-tile
 #pragma unroll
-    for (int sub = 0; sub < NS; ++sub)
+    for (int sub = 0; sub < NS; ++sub) {
+      float p[HS][2];
 #pragma unroll
       for (int s = 0; s < HS; ++s)
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          x[sub][s][r] = fast_exp2(x[sub][s][r] - m_ref[s]);
-          l_part[s] += x[sub][s][r];
+          p[s][r] = fast_exp2(x[sub][s][r] - m_ref[s]);  // 0 for masked tokens
+          l_part[s] += p[s][r];
         }
-
-    // ---- O^T += V^T * P'^T per sub-tile
+      uint32_t bf0[NP], bf1[NP];
 #pragma unroll
-    for (int sub = 0; sub < NS; ++sub) {
-      // V (s, z) of this lane's four tokens for group gv
-      [[maybe_unused]] float2 szv[4];
-      if constexpr (BITS != 16) {
+      for (int nb = 0; nb < NP; ++nb) {
+        float pp[2];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          szv[k] = __half22float2(*reinterpret_cast<const __half2*>(
-              sVm + (sub * kTile + vt[k]) * C::MB + gv * 4));
-      }
-      uint32_t b0[NP], b1[NP];
-#pragma unroll
-      for (int nt = 0; nt < NP; ++nt) {
-        // p of head hb for tokens tig, tig + 4 (row 0 of QK lanes tig, tig + 4)
-        // and tig + 8, tig + 12 (row 1)
-        const int la = 4 * tig + ts[nt], lb = 4 * (tig + 4) + ts[nt];
-        float pv[4];
-        pv[0] = __shfl_sync(0xffffffffu, x[sub][0][0], la);
-        pv[1] = __shfl_sync(0xffffffffu, x[sub][0][0], lb);
-        pv[2] = __shfl_sync(0xffffffffu, x[sub][0][1], la);
-        pv[3] = __shfl_sync(0xffffffffu, x[sub][0][1], lb);
-        if constexpr (HS == 2) {
-          const float q0 = __shfl_sync(0xffffffffu, x[sub][HS - 1][0], la);
-          const float q1 = __shfl_sync(0xffffffffu, x[sub][HS - 1][0], lb);
-          const float q2 = __shfl_sync(0xffffffffu, x[sub][HS - 1][1], la);
-          const float q3 = __shfl_sync(0xffffffffu, x[sub][HS - 1][1], lb);
-          if (sl[nt]) {
-            pv[0] = q0; pv[1] = q1; pv[2] = q2; pv[3] = q3;
-          }
-        }
-        float pp[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int r = 0; r < 2; ++r) {
           if constexpr (BITS == 16) {
-            pp[k] = pv_ok[nt] ? pv[k] : 0.f;
+            pp[r] = p[slot_of(nb)][r];
           } else {
+            const int tok = sub * kTile + tq0 + 8 * r;
             // slots past the valid length may hold any bytes (NaN scales):
             // select, never multiply by a zero weight
-            const bool ok = pv_ok[nt] && valid(sub * kTile + vt[k]);
-            pp[k] = ok ? pv[k] * szv[k].x : 0.f;
-            corr[nt] = ok ? fmaf(pp[k], szv[k].y, corr[nt]) : corr[nt];
+            const float2 sz = __half22float2(*reinterpret_cast<const __half2*>(
+                sVm + tok * C::MB + gv[nb] * 4));
+            const bool ok = valid(tok);
+            pp[r] = ok ? p[slot_of(nb)][r] * sz.x : 0.f;
+            corr[nb] = ok ? fmaf(pp[r], sz.y, corr[nb]) : corr[nb];
           }
         }
-        // hi part in even columns, lo = P' - hi in odd ones
-        const float2 h01 = __half22float2(__floats2half2_rn(pp[0], pp[1]));
-        const float2 h23 = __half22float2(__floats2half2_rn(pp[2], pp[3]));
-        b0[nt] = pack_h2(fmaf(-lo_sel, h01.x, pp[0]), fmaf(-lo_sel, h01.y, pp[1]));
-        b1[nt] = pack_h2(fmaf(-lo_sel, h23.x, pp[2]), fmaf(-lo_sel, h23.y, pp[3]));
+        uint32_t r0, r1;
+        split_pair(pp[0], pp[1], r0, r1);
+        bf0[nb] = transpose8x8(r0);  // k positions 0 .. 7 (rows 0 .. 7)
+        bf1[nb] = transpose8x8(r1);  // k positions 8 .. 15
       }
 
       const uint8_t* vb = sV + sub * kTile * C::RB + gid * C::VB;
       uint32_t wA[C::VW], wB[C::VW], wC[C::VW], wD[C::VW];
-      load_chunk<C::VB, C::VW>(vb + vt[0] * C::RB, wA);
-      load_chunk<C::VB, C::VW>(vb + vt[1] * C::RB, wB);
-      load_chunk<C::VB, C::VW>(vb + vt[2] * C::RB, wC);
-      load_chunk<C::VB, C::VW>(vb + vt[3] * C::RB, wD);
+      load_chunk<C::VB, C::VW>(vb + tvA * C::RB, wA);
+      load_chunk<C::VB, C::VW>(vb + tvB * C::RB, wB);
+      load_chunk<C::VB, C::VW>(vb + (tvA + 8) * C::RB, wC);
+      load_chunk<C::VB, C::VW>(vb + (tvB + 8) * C::RB, wD);
       if constexpr (BITS == 16 && !FULL) {
         // raw fp16 rows past the valid length may hold anything: zero them
 #pragma unroll
         for (int w = 0; w < C::VW; ++w) {
-          wA[w] = valid(sub * kTile + vt[0]) ? wA[w] : 0u;
-          wB[w] = valid(sub * kTile + vt[1]) ? wB[w] : 0u;
-          wC[w] = valid(sub * kTile + vt[2]) ? wC[w] : 0u;
-          wD[w] = valid(sub * kTile + vt[3]) ? wD[w] : 0u;
+          wA[w] = valid(sub * kTile + tvA) ? wA[w] : 0u;
+          wB[w] = valid(sub * kTile + tvB) ? wB[w] : 0u;
+          wC[w] = valid(sub * kTile + tvA + 8) ? wC[w] : 0u;
+          wD[w] = valid(sub * kTile + tvB + 8) ? wD[w] : 0u;
         }
       }
       uint32_t xa[16], xc[16];
@@ -457,10 +443,10 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         }
       }
 #pragma unroll
-      for (int nt = 0; nt < NP; ++nt)
+      for (int nb = 0; nb < NP; ++nb)
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt)
-          mma_f16(o_acc[nt][mt], xa[mt], xa[mt + 8], xc[mt], xc[mt + 8], b0[nt], b1[nt]);
+          mma_f16(o_acc[nb][mt], xa[mt], xa[mt + 8], xc[mt], xc[mt + 8], bf0[nb], bf1[nb]);
     }
   };
 
@@ -500,46 +486,46 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     }
   }
 
-  // ---- warp totals: l over the token rows (gid), corrections over tig
+  // ---- warp totals: sums over the token rows (gid)
 #pragma unroll
   for (int s = 0; s < HS; ++s) {
     l_part[s] += __shfl_xor_sync(0xffffffffu, l_part[s], 4);
     l_part[s] += __shfl_xor_sync(0xffffffffu, l_part[s], 8);
     l_part[s] += __shfl_xor_sync(0xffffffffu, l_part[s], 16);
   }
-  float corr_t[NP];  // the correction of accumulator column nt * 8 + 2 tig
 #pragma unroll
-  for (int nt = 0; nt < NP; ++nt) {
-    corr[nt] += __shfl_xor_sync(0xffffffffu, corr[nt], 1);
-    corr[nt] += __shfl_xor_sync(0xffffffffu, corr[nt], 2);
-    corr_t[nt] = __shfl_sync(0xffffffffu, corr[nt], 8 * tig);
+  for (int nb = 0; nb < NP; ++nb) {
+    corr[nb] += __shfl_xor_sync(0xffffffffu, corr[nb], 4);
+    corr[nb] += __shfl_xor_sync(0xffffffffu, corr[nb], 8);
+    corr[nb] += __shfl_xor_sync(0xffffffffu, corr[nb], 16);
   }
 
   __syncthreads();
   float* ms = reinterpret_cast<float*>(smem + C::HDR_BYTES);  // [kWarps][8]
   float* ls = ms + kWarps * 8;                                 // [kWarps][8]
   float* os = ls + kWarps * 8;                                 // [kWarps][8][D]
-  if (gid == 0 && (NG != 4 || (tig & 1) == 0)) {
+  if (gid == 0 && distinct) {
+    // lanes owning the same head hold the same values: any may write
 #pragma unroll
     for (int s = 0; s < HS; ++s) {
-      const int h = slot_head(s);
-      if (h < GR) {
-        ms[warp * 8 + h] = m_ref[s];
-        ls[warp * 8 + h] = l_part[s];
-      }
+      ms[warp * 8 + own_h[s]] = m_ref[s];
+      ls[warp * 8 + own_h[s]] = l_part[s];
     }
   }
+  if (distinct) {
 #pragma unroll
-  for (int nt = 0; nt < NP; ++nt) {
-    if (writer[nt]) {
-      float* oh = os + (warp * 8 + ho[nt]) * D + 16 * gid;
+    for (int nb = 0; nb < NP; ++nb) {
+      if (gv[nb] == dgrp) {
+        float* oh = os + (warp * 8 + own_h[slot_of(nb)]) * D + 16 * gid;
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        // undo the subnormal code scale 2^(e - 24) of the row's dim
-        const float f0 = pow2f(24 - XP::exp(mt % XP::kOut));
-        const float f1 = pow2f(24 - XP::exp((mt + 8) % XP::kOut));
-        oh[mt] = fmaf(o_acc[nt][mt][0] + o_acc[nt][mt][1], f0, -corr_t[nt]);
-        oh[mt + 8] = fmaf(o_acc[nt][mt][2] + o_acc[nt][mt][3], f1, -corr_t[nt]);
+        for (int mt = 0; mt < 8; ++mt) {
+          // hi column minus the negated-remainder column, then undo the
+          // subnormal code scale 2^(e - 24) of the row's dim
+          const float f0 = pow2f(24 - XP::exp(mt % XP::kOut));
+          const float f1 = pow2f(24 - XP::exp((mt + 8) % XP::kOut));
+          oh[mt] = fmaf(o_acc[nb][mt][0] - o_acc[nb][mt][1], f0, -corr[nb]);
+          oh[mt + 8] = fmaf(o_acc[nb][mt][2] - o_acc[nb][mt][3], f1, -corr[nb]);
+        }
       }
     }
   }

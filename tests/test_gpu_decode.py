@@ -183,6 +183,41 @@ def test_rising_scores_rescale(kvq, bits, G, g):
     assert_close(out, ref, lse, lref, what=f"rising scores bits{bits} G{G} g{g}")
 
 
+@pytest.mark.parametrize("bits,G,g", [(8, 128, 1), (4, 64, 4), (2, 32, 1), (4, 128, 8),
+                                      (2, 64, 2), (4, 32, 4), (16, 128, 4)])
+def test_dominant_token_precision(kvq, bits, G, g):
+    """One token whose key is a large multiple of every query gets all the
+    weight: the output must equal that token's dequantized V to ~1e-6
+    relative.  The weights p * s_V enter the tensor cores as two fp16 parts;
+    rounding them to one fp16 value would show here as errors near 2^-12."""
+    wl = workloads.WORKLOADS["long_gqa_int4"].scaled(kv_heads=2, q_heads=2 * g, bits=bits,
+                                                     group=G)
+    lens = [150, 61]
+    B, T = len(lens), max(lens)
+    k, v = workloads.kv_tokens(wl, T, DEV, batch=B)
+    q = workloads.queries(wl, DEV, batch=B)
+    star = [97, 13]
+    qh = q.view(B, 2, g, 128).float().sum(2)  # per KV head: the sum of its queries
+    for bi, ts in enumerate(star):
+        kk = qh[bi] / qh[bi].norm(dim=-1, keepdim=True) * 60.0
+        k[bi, :, ts] = kk.half()
+    v = (v.float() * 4.0).half()
+    c = kvq.QuantizedKVCache.allocate(B, 2, 128, 192, bits, G, DEV)
+    _poison(c)
+    if bits == 16:
+        fill_fp16_segment(c, k, v, lens)
+    else:
+        fill_cache(kvq, c, k, v, lens)
+    out, _ = _run(kvq, c, q)
+    seg = oracle_segment(k, v, bits, G)
+    ref, _ = oracle.decode_attention(q_bits(q), q.dtype == torch.bfloat16, [seg], [lens],
+                                     128 ** -0.5)
+    o = out.cpu().numpy().astype(np.float64)
+    scale = np.abs(ref).max()
+    err = np.abs(o - ref).max() / scale
+    assert err < 2e-5, f"bits{bits} G{G} g{g}: max error {err:.2e} of max |out|"
+
+
 def test_mixed_segments_equal_unchunked(kvq):
     """Three segments (FP16, INT4, INT2) of one sequence merged by log-sum-exp
     equal attention over all their tokens (Cocktail page 3.2.3)."""
