@@ -353,6 +353,22 @@ def cpu_baseline_mixed(wl, k, v, q, seconds: float, wlr):
 
 # ---------------------------------------------------------------- kvq arm
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest of every rank's value (a job is as slow as its slowest
+    rank); `device` is where the backend wants its tensors."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(wl, rank: int):
+    """Weak scaling: every rank attends its own batch of sequences, drawn from
+    its own seeds; no sequence is shared, so no collective touches the data."""
+    return wl.scaled(seed=wl.seed + 1000 * rank)
+
+
 def run_kvq(args, wl, rank, world, local_rank):
     import numpy as np
     import torch
@@ -366,7 +382,7 @@ def run_kvq(args, wl, rank, world, local_rank):
     B, H, Hq, D = wl.batch, wl.kv_heads, wl.q_heads, wl.head_dim
     ctx = wl.context
     episode = wl.steps if wl.append else min(wl.steps, 100)
-    wlr = wl.scaled(seed=wl.seed + 1000 * rank)  # each rank its own sequences
+    wlr = rank_workload(wl, rank)
 
     # ---- resident inputs (untimed set-up)
     if wl.chunk_tokens:
@@ -462,9 +478,7 @@ def run_kvq(args, wl, rank, world, local_rank):
     split_ms = sum(a.elapsed_time(b) for a, b in evs)
     assert kvq.workspace_error_word(ws) == 0, "device wait gave up (error word set)"
     if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dev)
     clocks = sampler.summary(h0, h1) if sampler else None
     if sampler:
         sampler.stop()
@@ -514,9 +528,7 @@ def run_kvq(args, wl, rank, world, local_rank):
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, dev)
     h2d = (kn[0].numel() * 2 if kn is not None else 0) + qs[0].numel() * 2
     d2h = out.numel() * 4 + lse.numel() * 4
 
