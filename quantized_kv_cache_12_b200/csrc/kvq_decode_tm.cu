@@ -68,6 +68,11 @@ struct TmCfg {
   static constexpr int HS = CPH == 1 ? 2 : 1;
   static constexpr int NP = (NG * GR + 3) / 4;
   static constexpr int W = NG * GR < 4 ? NG * GR : 4;
+  // grouped PV (two groups, four heads): the m-tiles are split between the
+  // groups, and each multiplies only its own group's weights; a lane then
+  // reads CH = G / 8 contiguous dims of each group
+  static constexpr bool GPV = NG == 2 && GR == 4;
+  static constexpr int NO = GPV ? 1 : NP;              // accumulator n-tiles
   static constexpr int SUB = (BITS == 16) ? 1 : 2;     // 16-token sub-tiles per stage
   static constexpr int STOK = SUB * kTile;
   static constexpr int STAGE = 2 * STOK * RB + 2 * STOK * MB;
@@ -75,12 +80,16 @@ struct TmCfg {
   // of q, unit id and fail flag
   static constexpr int HDR_BARS = 0, HDR_Q = 512, HDR_QS = HDR_Q + GR * D * 2;
   static constexpr int HDR_MISC = HDR_QS + 64;
-  static constexpr int HDR_BYTES = ((HDR_MISC + 8 + 127) / 128) * 128;
-  // four CTAs per SM where the registers allow it (one PV n-tile) and three
-  // stages per warp fit in a quarter of the SM's shared memory
-  // (4 x (56 KB + 1 KB reserved) <= 228 KB), else three
+  // with two PV n-tiles the QK query fragments are read from shared memory
+  // (8 x 32 lanes x 8 B) instead of being held in 16 registers per thread
+  static constexpr bool QB_SMEM = false;
+  static constexpr int HDR_QF = HDR_MISC + 64;
+  static constexpr int HDR_BYTES = (((QB_SMEM ? HDR_QF + 8 * 32 * 8 : HDR_MISC + 8) + 127) / 128) * 128;
+  // four CTAs per SM (128 registers a thread) where two stages per warp fit
+  // in a quarter of the SM's shared memory (4 x (56 KB + 1 KB reserved)
+  // <= 228 KB), else three
   static constexpr int MIN_CTAS =
-      (NP == 1 && HDR_BYTES + kWarps * 3 * STAGE <= 56 * 1024) ? 4 : 3;
+      (NO == 1 && HDR_BYTES + kWarps * 3 * STAGE <= 56 * 1024) ? 4 : 3;
   static constexpr int SMEM_BUDGET = (MIN_CTAS == 4 ? 56 : 74) * 1024;
   static constexpr int STAGES_RAW = (SMEM_BUDGET - HDR_BYTES) / (kWarps * STAGE);
   static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 16 ? 16 : STAGES_RAW);
@@ -127,6 +136,8 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   using WP = WordPairs<BITS>;
   using XP = CrossPairs<BITS>;
   constexpr int D = C::D, NG = C::NG, NP = C::NP, HS = C::HS, CPH = C::CPH;
+  // grouped PV: dims of each group per lane, and their V bytes and words
+  constexpr int CH = GE / 8, VBG = CH * BITS / 8, VWG = VBG >= 4 ? VBG / 4 : 1;
   const DecodeArgs& a = P.a;
   const SegView& seg = P.seg;
 
@@ -140,6 +151,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   float* qs_sm = reinterpret_cast<float*>(smem + C::HDR_QS);      // [8] per QK column
   int* unit_sm = reinterpret_cast<int*>(smem + C::HDR_MISC);
   int* fail_sm = unit_sm + 1;
+  uint2* qf_sm = reinterpret_cast<uint2*>(smem + C::HDR_QF);     // [8 ks][32 lanes]
   uint8_t* stages = smem + C::HDR_BYTES + warp * C::STAGES * C::STAGE;
   uint32_t* counters = a.err + 1;  // [0] next unit, [1] CTAs done
 
@@ -236,7 +248,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   __syncthreads();
   // B fragments of QK: pair p = 2 ks + h of this lane's chunk, column gid;
   // each element scaled by 2^(EMAX - e) for the exponent e of its code
-  uint32_t qb[8][2];
+  uint32_t qb[C::QB_SMEM ? 1 : 8][2];
   {
     const __half* qrow = q_sm + qh * D + 32 * tig;
 #pragma unroll
@@ -248,9 +260,16 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         const int d0 = (p / WP::kPairs) * WP::kDims + WP::dim(j, 0);
         const int d1 = (p / WP::kPairs) * WP::kDims + WP::dim(j, 1);
         const float f = pow2f(C::EMAX - WP::exp(j));
-        qb[ks][h] = qb_ok ? pack_h2(__half2float(qrow[d0]) * f, __half2float(qrow[d1]) * f) : 0u;
+        const uint32_t v =
+            qb_ok ? pack_h2(__half2float(qrow[d0]) * f, __half2float(qrow[d1]) * f) : 0u;
+        if constexpr (C::QB_SMEM) {
+          if (warp == 0) reinterpret_cast<uint32_t*>(&qf_sm[ks * 32 + lane])[h] = v;
+        } else {
+          qb[ks][h] = v;
+        }
       }
     }
+    if constexpr (C::QB_SMEM) __syncthreads();
   }
   const float qsA = (BITS != 16) ? qs_sm[2 * tig] : 0.f;
   const float qsB = (BITS != 16) ? qs_sm[2 * tig + 1] : 0.f;
@@ -259,9 +278,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   // least as large as every score seen, so p = 2^(x - m_ref) <= 1 and
   // P' = p * s_V stays within fp16 range; it moves (with a rescale) only when
   // a stage's max exceeds it, and then to that max + kLazy.
-  float o_acc[NP][8][4];
+  float o_acc[C::NO][8][4];
 #pragma unroll
-  for (int nb = 0; nb < NP; ++nb)
+  for (int nb = 0; nb < C::NO; ++nb)
 #pragma unroll
     for (int i = 0; i < 8; ++i) o_acc[nb][i][0] = o_acc[nb][i][1] = o_acc[nb][i][2] = o_acc[nb][i][3] = 0.f;
   float corr[NP];  // sum of P' * z_V of combination (b, tig) over this lane's tokens
@@ -307,9 +326,19 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         }
       }
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t b0, b1;
+        if constexpr (C::QB_SMEM) {
+          const uint2 v = qf_sm[ks * 32 + lane];
+          b0 = v.x;
+          b1 = v.y;
+        } else {
+          b0 = qb[ks][0];
+          b1 = qb[ks][1];
+        }
         mma_f16((ks & 1) ? s_odd : s_acc, p0[2 * ks], p1[2 * ks], p0[2 * ks + 1],
-                p1[2 * ks + 1], qb[ks][0], qb[ks][1]);
+                p1[2 * ks + 1], b0, b1);
+      }
 #pragma unroll
       for (int c = 0; c < 4; ++c) s_acc[c] += s_odd[c];
       // the owned heads' scores: sum over their groups of s_K * (S - z_K * qs);
@@ -368,14 +397,15 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
 #pragma unroll
       for (int s = 0; s < HS; ++s) l_part[s] *= alpha[s];
 #pragma unroll
-      for (int nb = 0; nb < NP; ++nb) {
-        const float al = alpha[slot_of(nb)];
+      for (int nb = 0; nb < C::NO; ++nb) {
+        const float al = alpha[C::GPV ? 0 : slot_of(nb)];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
           for (int c = 0; c < 4; ++c) o_acc[nb][i][c] *= al;
-        corr[nb] *= al;
       }
+#pragma unroll
+      for (int nb = 0; nb < NP; ++nb) corr[nb] *= alpha[slot_of(nb)];
     }
 
     // ---- weights and O^T += V^T * P'^T per sub-tile
@@ -414,39 +444,69 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         bf1[nb] = transpose8x8(r1);  // k positions 8 .. 15
       }
 
-      const uint8_t* vb = sV + sub * kTile * C::RB + gid * C::VB;
-      uint32_t wA[C::VW], wB[C::VW], wC[C::VW], wD[C::VW];
-      load_chunk<C::VB, C::VW>(vb + tvA * C::RB, wA);
-      load_chunk<C::VB, C::VW>(vb + tvB * C::RB, wB);
-      load_chunk<C::VB, C::VW>(vb + (tvA + 8) * C::RB, wC);
-      load_chunk<C::VB, C::VW>(vb + (tvB + 8) * C::RB, wD);
-      if constexpr (BITS == 16 && !FULL) {
-        // raw fp16 rows past the valid length may hold anything: zero them
+      if constexpr (C::GPV) {
+        // m-tiles 4 gv .. 4 gv + 3 are group gv's dims: rows gid, gid + 8 of
+        // m-tile 4 gv + j are dims gv * G + gid * CH + j and + CH / 2
+#pragma unroll
+        for (int gq = 0; gq < NG; ++gq) {
+          const uint8_t* vb = sV + sub * kTile * C::RB + gq * (GE * BITS / 8) + gid * VBG;
+          uint32_t wA[VWG], wB[VWG], wC[VWG], wD[VWG];
+          load_chunk<VBG, VWG>(vb + tvA * C::RB, wA);
+          load_chunk<VBG, VWG>(vb + tvB * C::RB, wB);
+          load_chunk<VBG, VWG>(vb + (tvA + 8) * C::RB, wC);
+          load_chunk<VBG, VWG>(vb + (tvB + 8) * C::RB, wD);
+          uint32_t xa[VWG * XP::kOut], xc[VWG * XP::kOut];
+#pragma unroll
+          for (int w = 0; w < VWG; ++w) {
+            uint32_t ya[XP::kOut], yc[XP::kOut];
+            XP::run(wA[w], wB[w], ya);
+            XP::run(wC[w], wD[w], yc);
+#pragma unroll
+            for (int i = 0; i < XP::kOut; ++i) {
+              xa[w * XP::kOut + i] = ya[i];
+              xc[w * XP::kOut + i] = yc[i];
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < CH / 2; ++j)
+            mma_f16(o_acc[0][gq * (CH / 2) + j], xa[j], xa[j + CH / 2], xc[j],
+                    xc[j + CH / 2], bf0[gq], bf1[gq]);
+        }
+      } else {
+        const uint8_t* vb = sV + sub * kTile * C::RB + gid * C::VB;
+        uint32_t wA[C::VW], wB[C::VW], wC[C::VW], wD[C::VW];
+        load_chunk<C::VB, C::VW>(vb + tvA * C::RB, wA);
+        load_chunk<C::VB, C::VW>(vb + tvB * C::RB, wB);
+        load_chunk<C::VB, C::VW>(vb + (tvA + 8) * C::RB, wC);
+        load_chunk<C::VB, C::VW>(vb + (tvB + 8) * C::RB, wD);
+        if constexpr (BITS == 16 && !FULL) {
+          // raw fp16 rows past the valid length may hold anything: zero them
+#pragma unroll
+          for (int w = 0; w < C::VW; ++w) {
+            wA[w] = valid(sub * kTile + tvA) ? wA[w] : 0u;
+            wB[w] = valid(sub * kTile + tvB) ? wB[w] : 0u;
+            wC[w] = valid(sub * kTile + tvA + 8) ? wC[w] : 0u;
+            wD[w] = valid(sub * kTile + tvB + 8) ? wD[w] : 0u;
+          }
+        }
+        uint32_t xa[16], xc[16];
 #pragma unroll
         for (int w = 0; w < C::VW; ++w) {
-          wA[w] = valid(sub * kTile + tvA) ? wA[w] : 0u;
-          wB[w] = valid(sub * kTile + tvB) ? wB[w] : 0u;
-          wC[w] = valid(sub * kTile + tvA + 8) ? wC[w] : 0u;
-          wD[w] = valid(sub * kTile + tvB + 8) ? wD[w] : 0u;
+          uint32_t ya[XP::kOut], yc[XP::kOut];
+          XP::run(wA[w], wB[w], ya);
+          XP::run(wC[w], wD[w], yc);
+#pragma unroll
+          for (int i = 0; i < XP::kOut; ++i) {
+            xa[w * XP::kOut + i] = ya[i];
+            xc[w * XP::kOut + i] = yc[i];
+          }
         }
+#pragma unroll
+        for (int nb = 0; nb < NP; ++nb)
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt)
+            mma_f16(o_acc[nb][mt], xa[mt], xa[mt + 8], xc[mt], xc[mt + 8], bf0[nb], bf1[nb]);
       }
-      uint32_t xa[16], xc[16];
-#pragma unroll
-      for (int w = 0; w < C::VW; ++w) {
-        uint32_t ya[XP::kOut], yc[XP::kOut];
-        XP::run(wA[w], wB[w], ya);
-        XP::run(wC[w], wD[w], yc);
-#pragma unroll
-        for (int i = 0; i < XP::kOut; ++i) {
-          xa[w * XP::kOut + i] = ya[i];
-          xc[w * XP::kOut + i] = yc[i];
-        }
-      }
-#pragma unroll
-      for (int nb = 0; nb < NP; ++nb)
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-          mma_f16(o_acc[nb][mt], xa[mt], xa[mt + 8], xc[mt], xc[mt + 8], bf0[nb], bf1[nb]);
     }
   };
 
@@ -512,7 +572,20 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
       ls[warp * 8 + own_h[s]] = l_part[s];
     }
   }
-  if (distinct) {
+  if constexpr (C::GPV) {
+    // every lane: head tig (its own), 8 dims of each group
+    float* oh = os + (warp * 8 + own_h[0]) * D + gid * CH;
+#pragma unroll
+    for (int gq = 0; gq < NG; ++gq)
+#pragma unroll
+      for (int j = 0; j < CH / 2; ++j) {
+        const float f0 = pow2f(24 - XP::exp(j % XP::kOut));
+        const float f1 = pow2f(24 - XP::exp((j + CH / 2) % XP::kOut));
+        const float* o = o_acc[0][gq * (CH / 2) + j];
+        oh[gq * GE + j] = fmaf(o[0] - o[1], f0, -corr[gq]);
+        oh[gq * GE + j + CH / 2] = fmaf(o[2] - o[3], f1, -corr[gq]);
+      }
+  } else if (distinct) {
 #pragma unroll
     for (int nb = 0; nb < NP; ++nb) {
       if (gv[nb] == dgrp) {
