@@ -422,28 +422,34 @@ def run_kvq(args, wl, rank, world, local_rank):
     ws = kvq.alloc_workspace(segs, Hq, hint, device=dev)
     ws_bytes = kvq.kvq_decode_workspace_bytes(segs, Hq, hint)
     bh = B * Hq
-    parts = next(p for p in range(1, 1 << 16)
-                 if 256 + (bh * p * 8 + 255) // 256 * 256 + bh * p * D * 4 == ws_bytes)
-    launches_per_step = (1 if wl.append else 0) + len(segs) + (1 if parts > 1 else 0)
+    r256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+
+    def ws_for(p):  # kvq_decode_workspace_bytes' layout for p partials
+        return 256 + r256(B * 4) + r256(bh * p * 8) + r256(bh * p * D * 4)
+    parts = next(p for p in range(1, 1 << 16) if ws_for(p) == ws_bytes)
+    # kernels of the library per step: one split-K launch per segment (the
+    # append runs inside it), then the merge when there are several partials
+    launches_per_step = len(segs) + (1 if parts > 1 else 0)
     stream = torch.cuda.current_stream()
 
-    # a step = [append] + split-K partials + merge, each a separate call so
-    # the partials kernel can be timed on its own
-    def append_fn(e):
-        if e == 0:
-            cache.seq_lens.copy_(base_lens, non_blocking=True)
-        kvq.kvq_quantize_append(cache, kn[e, 0], kn[e, 1], 1, advance_seq_lens=True)
+    def reset_fn(e):  # the episode restarts from the prefilled lengths
+        cache.seq_lens.copy_(base_lens, non_blocking=True)
 
-    def partials_fn(e):
-        kvq.kvq_decode_partials(segs, qs[e], out, lse, ws, max_len_hint=hint)
+    def partials_fn(e):  # the timed kernel(s): append + split-K attention
+        if wl.append:
+            kvq.kvq_decode_step_partials(cache, kn[e, 0], kn[e, 1], qs[e], out, lse, ws,
+                                         max_len_hint=hint)
+        else:
+            kvq.kvq_decode_partials(segs, qs[e], out, lse, ws, max_len_hint=hint)
 
     def merge_fn(e):
         kvq.kvq_decode_merge(segs, qs[e], out, lse, ws, max_len_hint=hint)
 
-    phases = ([append_fn] if wl.append else []) + [partials_fn, merge_fn]
+    def phases_at(e):
+        return ([reset_fn] if wl.append and e == 0 else []) + [partials_fn, merge_fn]
 
     def step(s):
-        for f in phases:
+        for f in phases_at(s % episode):
             f(s % episode)
 
     def kv_bytes_at(s):
@@ -467,7 +473,7 @@ def run_kvq(args, wl, rank, world, local_rank):
     with torch.cuda.stream(cap):
         for e in range(episode):
             row = []
-            for f in phases:
+            for f in phases_at(e):
                 g = torch.cuda.CUDAGraph()
                 g.capture_begin()
                 f(e)
@@ -476,15 +482,15 @@ def run_kvq(args, wl, rank, world, local_rank):
             graphs.append(row)
     stream.wait_stream(cap)
     torch.cuda.synchronize()
-    i_part = phases.index(partials_fn)
 
     def step_graphs(s, ev=None):
         row = graphs[s % episode]
         for j, g in enumerate(row):
-            if ev is not None and j == i_part:
+            timed = j == len(row) - 2  # the partials phase
+            if ev is not None and timed:
                 ev[0].record(stream)
             g.replay()
-            if ev is not None and j == i_part:
+            if ev is not None and timed:
                 ev[1].record(stream)
 
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -543,8 +549,9 @@ def run_kvq(args, wl, rank, world, local_rank):
             v_d.copy_(kn_h[e, 1], non_blocking=True)
         q_d.copy_(qs_h[e], non_blocking=True)
         if wl.append:
-            kvq.kvq_quantize_append(cache, k_d, v_d, 1, advance_seq_lens=True)
-        kvq.kvq_decode_attention(segs, q_d, out, lse, ws, max_len_hint=hint)
+            kvq.kvq_decode_step(cache, k_d, v_d, q_d, out, lse, ws, max_len_hint=hint)
+        else:
+            kvq.kvq_decode_attention(segs, q_d, out, lse, ws, max_len_hint=hint)
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
 
@@ -582,11 +589,11 @@ def run_kvq(args, wl, rank, world, local_rank):
                 "segments": {f"bits{b}": int(ln.sum()) for b, ln in zip(seg_bits, seg_lens)}}
                if seg_lens is not None else {}),
             "launch": "each phase of a step replayed from a CUDA graph captured once per "
-                      "episode position; events around the attention-partials replay",
+                      "episode position; events around the split-K replay",
             "l2": f"inputs larger than L2: {sum(kv_bytes) / args.steps / 1e6:.0f} MB of packed "
                   f"K/V read per step per GPU (L2 126 MB)",
-            "step": ("quantize-append 1 token/seq + split-K decode attention + LSE merge"
-                     if wl.append else
+            "step": ("kvq_decode_step: quantize-on-write of 1 token/seq inside the split-K "
+                     "decode attention kernel, then the LSE merge" if wl.append else
                      "split-K decode attention over the FP16/INT4/INT2 segments + LSE merge")}),
         "kv_read_gbs": sum(kv_bytes) / (ms / 1e3) / 1e9 * world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -149,12 +149,14 @@ kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k_new,
                                int32_t advance_seq_lens, void *stream);
 
 /*
- * Workspace bytes that kvq_decode_attention needs for these segments and
- * arguments (host-only).  The workspace holds the per-split partial
- * results (m, l, o) merged by log-sum-exp and a 256-byte header whose
- * first 32-bit word is a sticky device error flag (nonzero after a kernel
- * gave up a bounded wait; the library never clears it), followed by the
- * work counters of the persistent decode kernel.
+ * Workspace bytes that kvq_decode_attention (and kvq_decode_step) need for
+ * these segments and arguments (host-only).  The workspace holds a 256-byte
+ * header whose first 32-bit word is a sticky device error flag (nonzero
+ * after a kernel gave up a bounded wait; the library never clears it),
+ * followed by the work counters of the persistent decode kernel; then one
+ * counter per sequence, used by the decode step; then the per-split
+ * partial results (m, l, o) merged by log-sum-exp.  Every counter is back
+ * at zero when a call's kernels finish.
  */
 kvq_status kvq_decode_workspace_bytes(const kvq_cache *segs, int32_t n_segs,
                                       int32_t q_heads, int32_t max_len_hint,
@@ -179,10 +181,14 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache *segs, int32_t n_segs,
  *   max_len_hint: an upper bound of the seq_lens used to pick the split
  *        count (<= 0: max_tokens); results are correct for any seq_lens.
  *   workspace: device, >= kvq_decode_workspace_bytes(same arguments),
- *        256-byte aligned, zero-filled before its first use (its header
- *        holds work counters that the kernels return to zero at the end of
- *        every call, so it stays reusable without clearing).
+ *        256-byte aligned, zero-filled before its first use and again
+ *        before a call on a cache of another batch size (its front holds
+ *        counters that the kernels return to zero at the end of every call,
+ *        at offsets that depend on the batch size only; it stays reusable
+ *        without clearing across lengths, hints and segments).
  * A sequence with no tokens gives out = 0 and lse = -inf.
+ * The call is one split-K kernel launch per segment, then one merge kernel
+ * when the plan has more than one partial.
  * Supported: head_dim 128; g in 1..8; bits 2/4/8 with G 32/64/128, and bits
  * 16 with fp16 q.  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED,
  * KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA.
@@ -193,6 +199,47 @@ kvq_status kvq_decode_attention(const kvq_cache *segs, int32_t n_segs,
                                 float *out, float *lse, int32_t max_len_hint,
                                 void *workspace, size_t workspace_bytes,
                                 void *stream);
+
+/*
+ * One decode step of one cache: quantize-on-write of one new token per
+ * (sequence, KV head) -- the Oaken page's pipeline, where the quantizer sits
+ * in the write path to memory (section 3.2.3), with the quantize formula of
+ * the Cocktail page, 3.2.2, exactly as kvq_quantize_append computes it --
+ * then kvq_decode_attention over the cache including that token.  It is the
+ * same as kvq_quantize_append(cache, k_new, v_new, 1, advance = 1) followed
+ * by kvq_decode_attention, with the same results bit for bit in the cache,
+ * but for the tokens-on-M formats ((head_dim / G) * g <= 8) the append runs
+ * inside the split-K kernel: the unit whose token range covers the new
+ * position writes it, and the last unit of each sequence advances
+ * seq_lens[b].
+ *   cache: one segment, bits 2, 4 or 8.
+ *   k_new, v_new: device fp16 [batch][kv_heads][1][head_dim], 16-byte
+ *        aligned.  A sequence already at max_tokens keeps its length and
+ *        the token is not written (as in kvq_quantize_append).
+ *   q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint, workspace:
+ *        as kvq_decode_attention; max_len_hint should bound the lengths
+ *        after the append.
+ * Errors (nothing enqueued): KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED
+ * (bits 16), KVQ_ERR_WORKSPACE; KVQ_ERR_CUDA after a failed launch.
+ */
+kvq_status kvq_decode_step(const kvq_cache *cache, const void *k_new,
+                           const void *v_new, const void *q, kvq_dtype q_dtype,
+                           int32_t q_heads, float softmax_scale, float *out,
+                           float *lse, int32_t max_len_hint, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+/*
+ * The first half of kvq_decode_step -- the append and the split-K partials
+ * -- for callers that time or overlap the halves; follow it with
+ * kvq_decode_merge(cache, 1, ...) on the same stream.  Same arguments,
+ * checks and errors as kvq_decode_step.
+ */
+kvq_status kvq_decode_step_partials(const kvq_cache *cache, const void *k_new,
+                                    const void *v_new, const void *q,
+                                    kvq_dtype q_dtype, int32_t q_heads,
+                                    float softmax_scale, float *out, float *lse,
+                                    int32_t max_len_hint, void *workspace,
+                                    size_t workspace_bytes, void *stream);
 
 /*
  * The two halves of kvq_decode_attention, for callers that time or overlap

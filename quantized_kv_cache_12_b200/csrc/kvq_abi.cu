@@ -15,6 +15,7 @@ namespace {
 constexpr int kD = 128;
 constexpr size_t kHeaderBytes = 256;
 
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool valid_group(int g) { return g == 32 || g == 64 || g == 128; }
@@ -121,14 +122,42 @@ kvq_status check_segments(const kvq_cache* segs, int n_segs, int q_heads) {
   return KVQ_OK;
 }
 
-size_t workspace_for(const kvq_cache* segs, int q_heads, int parts) {
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+// Workspace layout: header (error word, work counters); the per-sequence
+// unit counters of the decode step, at an offset and size that depend only
+// on batch; then the partial (m, l) and o, whose sizes follow the split
+// plan.  Every counter returns to zero by the end of each launch, so one
+// zero fill lasts for any number of calls on caches of one batch size.
+struct WsLayout {
+  size_t seq_cnt, ml, o, total;
+};
+
+size_t counter_bytes(const kvq_cache* segs) {
+  return round256((size_t)segs[0].batch * sizeof(uint32_t));
+}
+
+WsLayout workspace_layout(const kvq_cache* segs, int q_heads, int parts) {
   const size_t bh = (size_t)segs[0].batch * q_heads;
-  const size_t ml = bh * parts * 2 * sizeof(float);
-  const size_t o = bh * parts * kD * sizeof(float);
-  return kHeaderBytes + ((ml + 255) / 256) * 256 + o;
+  WsLayout w;
+  w.seq_cnt = kHeaderBytes;
+  w.ml = kHeaderBytes + counter_bytes(segs);
+  w.o = w.ml + round256(bh * parts * 2 * sizeof(float));
+  w.total = w.o + round256(bh * parts * kD * sizeof(float));
+  return w;
+}
+
+size_t workspace_for(const kvq_cache* segs, int q_heads, int parts) {
+  return workspace_layout(segs, q_heads, parts).total;
 }
 
 }  // namespace
+
+namespace kvq {
+size_t decode_zeroed_prefix_bytes(const kvq_cache* segs) {
+  return kHeaderBytes + counter_bytes(segs);
+}
+}  // namespace kvq
 
 extern "C" {
 
@@ -215,10 +244,16 @@ namespace {
 
 enum DecodeStage { kPartials = 1, kMerge = 2, kBoth = 3 };
 
+// One decode attention (stages kBoth), or only its partials or its merge,
+// or (stages 0) only the argument checks.  k_new/v_new (with a single
+// segment of a tokens-on-M format) make it a decode step: the kernel also
+// quantizes one new token per (sequence, KV head) into the cache and
+// advances seq_lens.
 kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
                          kvq_dtype q_dtype, int32_t q_heads, float softmax_scale, float* out,
                          float* lse, int32_t max_len_hint, void* workspace,
-                         size_t workspace_bytes, void* stream, int stages) {
+                         size_t workspace_bytes, void* stream, int stages,
+                         const void* k_new = nullptr, const void* v_new = nullptr) {
   kvq_status st = check_segments(segs, n_segs, q_heads);
   if (st != KVQ_OK) return st;
   if (q == nullptr || out == nullptr || !aligned16(q)) return KVQ_ERR_INVALID_ARG;
@@ -231,10 +266,10 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
   const size_t need = workspace_for(segs, q_heads, plan.parts);
   if (workspace == nullptr || workspace_bytes < need) return KVQ_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KVQ_ERR_INVALID_ARG;
+  if (stages == 0) return KVQ_OK;  // arguments checked, nothing enqueued
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t bh = (size_t)segs[0].batch * q_heads;
-  const size_t ml_bytes = ((bh * plan.parts * 2 * sizeof(float) + 255) / 256) * 256;
+  const WsLayout lay = workspace_layout(segs, q_heads, plan.parts);
   kvq::DecodeArgs a;
   a.batch = segs[0].batch;
   a.kv_heads = segs[0].kv_heads;
@@ -245,10 +280,13 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
   a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
   a.parts = plan.parts;
   a.err = reinterpret_cast<uint32_t*>(ws);
-  a.part_ml = reinterpret_cast<float*>(ws + kHeaderBytes);
-  a.part_o = reinterpret_cast<float*>(ws + kHeaderBytes + ml_bytes);
+  a.part_ml = reinterpret_cast<float*>(ws + lay.ml);
+  a.part_o = reinterpret_cast<float*>(ws + lay.o);
   a.out = out;
   a.lse = lse;
+  a.seq_cnt = reinterpret_cast<uint32_t*>(ws + lay.seq_cnt);
+  a.k_new = static_cast<const __half*>(k_new);
+  a.v_new = static_cast<const __half*>(v_new);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int base = 0;
   for (int i = 0; i < n_segs; ++i) {
@@ -298,6 +336,56 @@ kvq_status kvq_decode_merge(const kvq_cache* segs, int32_t n_segs, const void* q
                             size_t workspace_bytes, void* stream) {
   return decode_stages(segs, n_segs, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
                        workspace, workspace_bytes, stream, kMerge);
+}
+
+}  // extern "C"
+
+namespace {
+
+// The decode step (stages kBoth) or its first half (kPartials).
+kvq_status decode_step_stages(const kvq_cache* cache, const void* k_new, const void* v_new,
+                              const void* q, kvq_dtype q_dtype, int32_t q_heads,
+                              float softmax_scale, float* out, float* lse, int32_t max_len_hint,
+                              void* workspace, size_t workspace_bytes, void* stream, int stages) {
+  kvq_status st = check_segments(cache, 1, q_heads);
+  if (st != KVQ_OK) return st;
+  if (cache->k.bits == 16) return KVQ_ERR_UNSUPPORTED;
+  if (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new))
+    return KVQ_ERR_INVALID_ARG;
+  const int g = q_heads / cache->kv_heads;
+  if (kvq::decode_tm_supported(cache->k.bits, cache->k.group_size, g))
+    return decode_stages(cache, 1, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
+                         workspace, workspace_bytes, stream, stages, k_new, v_new);
+  // formats of the 16-row kernel: the append kernel, then the attention
+  // (every argument is checked before the first launch)
+  st = decode_stages(cache, 1, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
+                     workspace, workspace_bytes, stream, 0);
+  if (st != KVQ_OK) return st;
+  st = kvq_quantize_append(cache, k_new, v_new, 1, 1, stream);
+  if (st != KVQ_OK) return st;
+  return decode_stages(cache, 1, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
+                       workspace, workspace_bytes, stream, stages);
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_step(const kvq_cache* cache, const void* k_new, const void* v_new,
+                           const void* q, kvq_dtype q_dtype, int32_t q_heads, float softmax_scale,
+                           float* out, float* lse, int32_t max_len_hint, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return decode_step_stages(cache, k_new, v_new, q, q_dtype, q_heads, softmax_scale, out, lse,
+                            max_len_hint, workspace, workspace_bytes, stream, kBoth);
+}
+
+kvq_status kvq_decode_step_partials(const kvq_cache* cache, const void* k_new, const void* v_new,
+                                    const void* q, kvq_dtype q_dtype, int32_t q_heads,
+                                    float softmax_scale, float* out, float* lse,
+                                    int32_t max_len_hint, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  return decode_step_stages(cache, k_new, v_new, q, q_dtype, q_heads, softmax_scale, out, lse,
+                            max_len_hint, workspace, workspace_bytes, stream, kPartials);
 }
 
 kvq_status kvq_chunk_assign(const float* chunk_emb, const float* query_emb, int32_t batch,

@@ -527,6 +527,8 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   }
   __syncthreads();
   cta_merge_store<g>(a, ms, ls, os, os + kWarps * 8 * D, b, kvh, seg.part_base + split, t);
+  // the merge wrote the stage buffers: order that before the next unit's copies
+  fence_proxy_async_smem();
   }  // unit loop
 
   if (t == 0) release_counters(counters);

@@ -1,8 +1,9 @@
 // kvq_decode_common.cuh -- pieces shared by the two decode-attention kernels
-// (the grouped-query kernel in kvq_decode.cu and the one-head-per-KV-head
-// kernel in kvq_decode_mha.cu): operand packing, the persistent work-unit
-// loop's bookkeeping, and the in-CTA log-sum-exp merge of the four warps'
-// partial results with its store to the output or to a split partial.
+// (the tokens-on-M kernel in kvq_decode_tm.cu and the 16-row kernel in
+// kvq_decode.cu): operand packing, the persistent work-unit loop's
+// bookkeeping, the in-CTA log-sum-exp merge of the four warps' partial
+// results with its store to the output or to a split partial, and the
+// sequence-length advance of a decode step.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -128,6 +129,18 @@ __device__ __forceinline__ void cta_merge_store(const DecodeArgs& a, const float
         a.part_ml[pi * 2 + 1] = Ls;
       }
     }
+  }
+}
+
+// Decode step: after a unit of sequence b finished (thread 0 calls this),
+// the last of the sequence's `units_per_seq` units advances seq_lens[b] to
+// `new_len`; every unit of b read the old length at its start.
+__device__ __forceinline__ void advance_if_last(const DecodeArgs& a, const SegView& seg, int b,
+                                                int units_per_seq, int new_len) {
+  const unsigned prev = atomicAdd(&a.seq_cnt[b], 1u);
+  if (prev == (unsigned)units_per_seq - 1) {
+    const_cast<int32_t*>(seg.seq_lens)[b] = new_len;
+    a.seq_cnt[b] = 0u;
   }
 }
 

@@ -46,6 +46,7 @@
 #include "kvq_decode_common.cuh"
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
+#include "kvq_quant_core.cuh"
 
 namespace kvq {
 
@@ -80,11 +81,15 @@ struct TmCfg {
   // of q, unit id and fail flag
   static constexpr int HDR_BARS = 0, HDR_Q = 512, HDR_QS = HDR_Q + GR * D * 2;
   static constexpr int HDR_MISC = HDR_QS + 64;
+  // decode step: the new token's K and V rows (codes, then meta), each at a
+  // 16-byte aligned stride (the quantizer stores up to 8 bytes at a time)
+  static constexpr int NEW_STRIDE = ((RB + MB + 15) / 16) * 16;
+  static constexpr int HDR_NEW = HDR_MISC + 64;
   // with two PV n-tiles the QK query fragments are read from shared memory
   // (8 x 32 lanes x 8 B) instead of being held in 16 registers per thread
   static constexpr bool QB_SMEM = false;
-  static constexpr int HDR_QF = HDR_MISC + 64;
-  static constexpr int HDR_BYTES = (((QB_SMEM ? HDR_QF + 8 * 32 * 8 : HDR_MISC + 8) + 127) / 128) * 128;
+  static constexpr int HDR_QF = HDR_NEW + 2 * NEW_STRIDE;
+  static constexpr int HDR_BYTES = (((QB_SMEM ? HDR_QF + 8 * 32 * 8 : HDR_QF) + 127) / 128) * 128;
   // four CTAs per SM (128 registers a thread) where two stages per warp fit
   // in a quarter of the SM's shared memory (4 x (56 KB + 1 KB reserved)
   // <= 228 KB), else three
@@ -100,6 +105,7 @@ struct TmCfg {
   static_assert(NG * GR <= 8, "at most eight (head, group) combinations");
   static_assert(kWarps * STAGES * 8 <= HDR_Q, "mbarriers fit the header");
   static_assert(MERGE_BYTES <= kWarps * STAGES * STAGE, "merge scratch fits the stages");
+  static_assert(HDR_NEW % 16 == 0 && NEW_STRIDE % 16 == 0, "aligned new-token rows");
   static_assert(WordPairs<BITS>::kPairs * KW == 16, "16 K pairs per lane and token");
   static_assert(CrossPairs<BITS>::kOut * VW == 16, "16 V dims per lane and token");
 };
@@ -151,6 +157,8 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   float* qs_sm = reinterpret_cast<float*>(smem + C::HDR_QS);      // [8] per QK column
   int* unit_sm = reinterpret_cast<int*>(smem + C::HDR_MISC);
   int* fail_sm = unit_sm + 1;
+  // decode step: the new token's quantized K and V rows (codes, then meta)
+  uint8_t* new_sm = smem + C::HDR_NEW;
   uint2* qf_sm = reinterpret_cast<uint2*>(smem + C::HDR_QF);     // [8 ks][32 lanes]
   uint8_t* stages = smem + C::HDR_BYTES + warp * C::STAGES * C::STAGE;
   uint32_t* counters = a.err + 1;  // [0] next unit, [1] CTAs done
@@ -197,13 +205,23 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   const int kvh = (unit / seg.n_split) % a.kv_heads;
   const int b = unit / (seg.n_split * a.kv_heads);
 
-  int L = seg.seq_lens[b];
-  L = max(0, min(L, seg.max_tokens));
+  // a decode step appends one token at position L_old (dropped when the
+  // cache is full) and attends over it too
+  const int L_old = max(0, min(seg.seq_lens[b], seg.max_tokens));
+  const bool step = a.k_new != nullptr;
+  const int L = (step && L_old < seg.max_tokens) ? L_old + 1 : L_old;
   int c0, c1;
   split_range(L, seg.n_split, split, c0, c1);
   const int unit_stages = (c1 > c0) ? (c1 - c0 + C::STOK - 1) / C::STOK : 0;
   const int n_tiles = (unit_stages > warp) ? (unit_stages - warp + kWarps - 1) / kWarps : 0;
   const int w0 = c0 + warp * C::STOK;  // first token of this warp's first stage
+  // this unit writes the new token; the warp holding its stage patches the
+  // stage in shared memory after the copy lands (the copy may read the row
+  // before or after the global store)
+  const bool append_here = step && L > L_old && c0 <= L_old && L_old < c1;
+  const int patch_stage = (L_old - c0) / C::STOK;
+  const int patch_i = (append_here && patch_stage % kWarps == warp) ? patch_stage / kWarps : -1;
+  const int patch_row = (L_old - c0) % C::STOK;
 
   const long long row0 = ((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0;
   const uint8_t* kc_src = seg.k_codes + row0 * C::RB;
@@ -226,6 +244,25 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   if (lane == 0) {
     const int pre = min(n_tiles, C::STAGES);
     for (int i = 0; i < pre; ++i) issue(i, (st + i) % C::STAGES);
+  }
+
+  // ---- decode step: quantize the new K (lanes 0-15) and V (16-31) rows of
+  // this KV head into shared memory, then copy them to the cache
+  if constexpr (BITS != 16) {
+    if (append_here && warp == 0) {
+      const int vh = lane >> 4, l16 = lane & 15;
+      const __half* src = (vh ? a.v_new : a.k_new) + ((long long)b * a.kv_heads + kvh) * D;
+      uint8_t* row = new_sm + vh * C::NEW_STRIDE;
+      quantize_slice<BITS, GE>(src, row, row + C::RB, l16, true);
+      __syncwarp();
+      const long long dst = ((long long)b * a.kv_heads + kvh) * seg.max_tokens + L_old;
+      uint8_t* gc = const_cast<uint8_t*>(vh ? seg.v_codes : seg.k_codes) + dst * C::RB;
+      uint8_t* gm = const_cast<uint8_t*>(vh ? seg.v_meta : seg.k_meta) + dst * C::MB;
+      for (int i = l16; i < C::RB / 4; i += 16)
+        reinterpret_cast<uint32_t*>(gc)[i] = reinterpret_cast<const uint32_t*>(row)[i];
+      if (l16 < C::MB / 4)
+        reinterpret_cast<uint32_t*>(gm)[l16] = reinterpret_cast<const uint32_t*>(row + C::RB)[l16];
+    }
   }
 
   // ---- the g query rows of this KV head, once per unit
@@ -519,6 +556,28 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     const uint8_t* sV = sK + C::STOK * C::RB;
     const uint8_t* sKm = sK + 2 * C::STOK * C::RB;
     const uint8_t* sVm = sKm + C::STOK * C::MB;
+    if constexpr (BITS != 16) {
+      if (i == patch_i) {
+        // the new token's row, from the quantized copy in shared memory
+        uint32_t* dK = reinterpret_cast<uint32_t*>(stages + st * C::STAGE + patch_row * C::RB);
+        uint32_t* dV = dK + C::STOK * C::RB / 4;
+        uint32_t* dKm = reinterpret_cast<uint32_t*>(stages + st * C::STAGE + 2 * C::STOK * C::RB +
+                                                    patch_row * C::MB);
+        uint32_t* dVm = dKm + C::STOK * C::MB / 4;
+        const uint32_t* nK = reinterpret_cast<const uint32_t*>(new_sm);
+        const uint32_t* nV = reinterpret_cast<const uint32_t*>(new_sm + C::NEW_STRIDE);
+        for (int j = lane; j < C::RB / 4; j += 32) {
+          dK[j] = nK[j];
+          dV[j] = nV[j];
+        }
+        if (lane < C::MB / 4) {
+          dKm[lane] = nK[C::RB / 4 + lane];
+          dVm[lane] = nV[C::RB / 4 + lane];
+        }
+        fence_proxy_async_smem();  // before the ring refills this stage
+        __syncwarp();
+      }
+    }
     const int n_stage = min(C::STOK, c1 - (w0 + i * kWarps * C::STOK));
     if (n_stage == C::STOK)
       stage_body(std::integral_constant<bool, true>(), sK, sV, sKm, sVm, C::STOK);
@@ -604,6 +663,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   }
   __syncthreads();
   cta_merge_store<GR>(a, ms, ls, os, os + kWarps * 8 * D, b, kvh, seg.part_base + split, t);
+  if (step && t == 0) advance_if_last(a, seg, b, seg.n_split * a.kv_heads, L);
+  // the merge wrote the stage buffers: order that before the next unit's copies
+  fence_proxy_async_smem();
   }  // unit loop
 
   if (t == 0) release_counters(counters);

@@ -35,6 +35,13 @@ struct DecodeArgs {
   float* out;            // [batch][q_heads][head_dim]
   float* lse;            // [batch][q_heads] or null
   uint32_t* err;         // sticky device error word
+  // decode step: one new token per (sequence, KV head), quantized into the
+  // cache by the unit whose token range covers its position; seq_cnt[b]
+  // counts finished units of sequence b, and the last one advances
+  // seq_lens[b] (null k_new: no append)
+  const __half* k_new;   // [batch][kv_heads][head_dim] fp16
+  const __half* v_new;
+  uint32_t* seq_cnt;
 };
 
 struct QuantArgs {
@@ -60,6 +67,9 @@ int decode_tm_ctas_per_sm(int bits, int group, int group_ratio);
 cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s);
+// leading workspace bytes that hold the header and the counters (they must
+// be zero before a call whose cache shape differs from the previous call's)
+size_t decode_zeroed_prefix_bytes(const kvq_cache* segs);
 cudaError_t launch_chunk_assign(const float* emb, const float* qemb, int batch, int n_chunks,
                                 int emb_dim, double alpha, double beta, double* sim,
                                 uint8_t* bits, cudaStream_t s);

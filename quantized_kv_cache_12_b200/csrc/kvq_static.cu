@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "kvq.h"
+#include "kvq_internal.h"
 
 namespace {
 
@@ -55,10 +56,11 @@ extern "C" kvq_status kvq_decode_attention_noalloc(const kvq_cache* segs, int32_
   void* scratch = nullptr;
   st = scratch_address(&scratch);
   if (st != KVQ_OK) return st;
-  // The array keeps the previous call's contents.  The split kernels rewrite
-  // every partial they hand to the merge, so only the error word has to
-  // start at zero.
-  if (cudaMemsetAsync(scratch, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // The array keeps the previous call's contents, which may have had another
+  // layout.  The split kernels rewrite every partial they hand to the merge;
+  // the error word and the counters (at the front) start at zero.
+  if (cudaMemsetAsync(scratch, 0, kvq::decode_zeroed_prefix_bytes(segs),
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KVQ_ERR_CUDA;
   return kvq_decode_attention(segs, n_segs, q, q_dtype, q_heads, softmax_scale, out, lse,
                               max_len_hint, scratch, KVQ_STATIC_SCRATCH_BYTES, stream);

@@ -63,6 +63,8 @@ def _load():
     lib.kvq_decode_workspace_bytes.argtypes = [cp, i32, i32, i32, ctypes.POINTER(sz)]
     for name in ("kvq_decode_attention", "kvq_decode_partials", "kvq_decode_merge"):
         getattr(lib, name).argtypes = [cp, i32, P, ctypes.c_int, i32, f32, P, P, i32, P, sz, P]
+    for name in ("kvq_decode_step", "kvq_decode_step_partials"):
+        getattr(lib, name).argtypes = [cp, P, P, P, ctypes.c_int, i32, f32, P, P, i32, P, sz, P]
     lib.kvq_decode_attention_noalloc.argtypes = [cp, i32, P, ctypes.c_int, i32, f32, P, P,
                                                  i32, P]
     lib.kvq_decode_attention_noalloc.restype = ctypes.c_int
@@ -70,7 +72,8 @@ def _load():
     lib.kvq_chunk_reorder.argtypes = [cp, P, P, i32, i32, P, P, P]
     for name in ("kvq_plane_bytes", "kvq_quantize_append", "kvq_decode_workspace_bytes",
                  "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_merge",
-                 "kvq_chunk_assign", "kvq_chunk_reorder"):
+                 "kvq_decode_step", "kvq_decode_step_partials", "kvq_chunk_assign",
+                 "kvq_chunk_reorder"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -174,6 +177,35 @@ def kvq_decode_merge(segs, q: torch.Tensor, out: torch.Tensor, lse: Optional[tor
                      max_len_hint: int = 0, stream=None):
     _decode_call(lib.kvq_decode_merge, "kvq_decode_merge", segs, q, out, lse, workspace,
                  softmax_scale, max_len_hint, stream)
+
+
+def _step_call(fn, name, cache, k_new, v_new, q, out, lse, workspace, softmax_scale,
+               max_len_hint, stream):
+    arr = _caches(cache)
+    dt = KVQ_BF16 if q.dtype == torch.bfloat16 else KVQ_F16
+    scale = softmax_scale if softmax_scale is not None else q.shape[2] ** -0.5
+    _check(fn(arr, _ptr(k_new), _ptr(v_new), _ptr(q), dt, int(q.shape[1]), float(scale),
+              _ptr(out), _ptr(lse), int(max_len_hint), _ptr(workspace),
+              workspace.numel() * workspace.element_size(), _stream(stream)), name)
+
+
+def kvq_decode_step(cache, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+                    out: torch.Tensor, lse: Optional[torch.Tensor], workspace: torch.Tensor,
+                    softmax_scale: Optional[float] = None, max_len_hint: int = 0, stream=None):
+    """Append one token per (sequence, KV head) -- quantized into the cache --
+    and attend over the cache including it; advances cache.seq_lens."""
+    _step_call(lib.kvq_decode_step, "kvq_decode_step", cache, k_new, v_new, q, out, lse,
+               workspace, softmax_scale, max_len_hint, stream)
+
+
+def kvq_decode_step_partials(cache, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+                             out: torch.Tensor, lse: Optional[torch.Tensor],
+                             workspace: torch.Tensor, softmax_scale: Optional[float] = None,
+                             max_len_hint: int = 0, stream=None):
+    """The append and the split-K partials of kvq_decode_step; follow with
+    kvq_decode_merge."""
+    _step_call(lib.kvq_decode_step_partials, "kvq_decode_step_partials", cache, k_new, v_new,
+               q, out, lse, workspace, softmax_scale, max_len_hint, stream)
 
 
 def kvq_decode_attention_noalloc(segs, q: torch.Tensor, out: torch.Tensor,

@@ -165,6 +165,32 @@ def test_decode_workspace_and_argument_checks(kvq):
     assert st == kvq.KVQ_ERR_UNSUPPORTED  # bf16 queries with raw fp16 keys
 
 
+def test_decode_step_rejects_bad_arguments(kvq):
+    """kvq_decode_step checks everything on the host before its first launch,
+    on both of its paths (one fused launch, or append then attention)."""
+    lib = kvq.lib
+    fake = ctypes.c_void_p(0x70000)
+    ws = ctypes.c_void_p(0x80000)
+    for kv_heads, q_heads in ((8, 32), (2, 16)):  # g = 4 (fused), g = 8 with G64 (two launches)
+        c = _fake_cache(kvq, batch=4, kv_heads=kv_heads, max_tokens=8192)
+        arr = (kvq.kvq_cache * 1)(c)
+        n = kvq.kvq_decode_workspace_bytes(c, q_heads)
+
+        def step(k_new, v_new, q, ws_bytes, scale=0.088):
+            return lib.kvq_decode_step(arr, k_new, v_new, q, 0, q_heads, ctypes.c_float(scale),
+                                       fake, None, 0, ws, ws_bytes, None)
+        assert step(None, fake, fake, n) == kvq.KVQ_ERR_INVALID_ARG
+        assert step(fake, ctypes.c_void_p(0x70004), fake, n) == kvq.KVQ_ERR_INVALID_ARG
+        assert step(fake, fake, None, n) == kvq.KVQ_ERR_INVALID_ARG
+        assert step(fake, fake, fake, n, scale=-1.0) == kvq.KVQ_ERR_INVALID_ARG
+        assert step(fake, fake, fake, 64) == kvq.KVQ_ERR_WORKSPACE
+    c16 = _fake_cache(kvq, bits=16, batch=4, kv_heads=8, max_tokens=8192)
+    arr16 = (kvq.kvq_cache * 1)(c16)
+    st = lib.kvq_decode_step(arr16, fake, fake, fake, 0, 32, ctypes.c_float(0.088), fake, None, 0,
+                             ws, 1 << 30, None)
+    assert st == kvq.KVQ_ERR_UNSUPPORTED  # raw fp16 caches take no quantized append
+
+
 def test_chunk_entry_points_reject_bad_arguments(kvq):
     lib = kvq.lib
     fake = ctypes.c_void_p(0x10000)
