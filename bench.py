@@ -464,40 +464,61 @@ def run_kvq(args, wl, rank, world, local_rank):
     for s in range(args.warmup):
         step(s)
     torch.cuda.synchronize()
-    # ---- every phase of every episode position as a CUDA graph, so the
-    # timed loop is paced by the device, not by the Python calls (capture
-    # records the launches without running them)
+    # ---- every episode position as one CUDA graph (reset at the start of an
+    # episode, split-K partials, merge), so the timed loop is paced by the
+    # device and the merge is a programmatic dependent of the split-K kernel
+    # inside the graph.  Event-record nodes inside each graph bracket the
+    # split-K launch; after the loop each pair holds the time of its graph's
+    # last replay (the last `episode` steps of the timed region).
+    from cuda.bindings import runtime as cudart
+
+    split_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(episode)]
+    for e0, e1 in split_evs:  # create the events before the capture
+        e0.record(stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+
+    def record_in_graph(ev, st):
+        err, = cudart.cudaEventRecordWithFlags(ev.cuda_event, st.cuda_stream,
+                                               cudart.cudaEventRecordExternal)
+        if err != cudart.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaEventRecordWithFlags: {err}")
+
     graphs = []
     cap = torch.cuda.Stream(dev)
+    side = torch.cuda.Stream(dev)  # the end-of-split record branches off here
+    fork, join = torch.cuda.Event(), torch.cuda.Event()
     cap.wait_stream(stream)
     with torch.cuda.stream(cap):
         for e in range(episode):
-            row = []
-            for f in phases_at(e):
-                g = torch.cuda.CUDAGraph()
-                g.capture_begin()
-                f(e)
-                g.capture_end()
-                row.append(g)
-            graphs.append(row)
+            g = torch.cuda.CUDAGraph()
+            g.capture_begin()
+            if wl.append and e == 0:
+                reset_fn(e)
+            record_in_graph(split_evs[e][0], cap)
+            partials_fn(e)
+            # the end event hangs off the split-K node on a branch, so the
+            # merge still follows that node directly (programmatic edge)
+            fork.record(cap)
+            side.wait_event(fork)
+            record_in_graph(split_evs[e][1], side)
+            join.record(side)
+            merge_fn(e)
+            cap.wait_event(join)
+            g.capture_end()
+            graphs.append(g)
     stream.wait_stream(cap)
     torch.cuda.synchronize()
-
-    def step_graphs(s, ev=None):
-        row = graphs[s % episode]
-        for j, g in enumerate(row):
-            timed = j == len(row) - 2  # the partials phase
-            if ev is not None and timed:
-                ev[0].record(stream)
-            g.replay()
-            if ev is not None and timed:
-                ev[1].record(stream)
+    # one full episode of replays (uploads the graphs; the state returns to
+    # the same episode position)
+    for j in range(episode):
+        graphs[(args.warmup + j) % episode].replay()
+    torch.cuda.synchronize()
 
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_id) if rank == 0 else None
     time.sleep(0.3 if sampler else 0)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -507,7 +528,7 @@ def run_kvq(args, wl, rank, world, local_rank):
     torch.cuda.nvtx.range_push("kvq_timed")  # lets a profiler select the timed launches
     t_start.record(stream)
     for i in range(args.steps):
-        step_graphs(args.warmup + i, evs[i])
+        graphs[(args.warmup + i) % episode].replay()
     t_end.record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -515,7 +536,9 @@ def run_kvq(args, wl, rank, world, local_rank):
         dist.barrier()
     h1 = time.time()
     ms = t_start.elapsed_time(t_end)
-    split_ms = sum(a.elapsed_time(b) for a, b in evs)
+    # the split-K time of each graph's last replay in the timed region
+    last_step = {(args.warmup + i) % episode: args.warmup + i for i in range(args.steps)}
+    split_us = {e: split_evs[e][0].elapsed_time(split_evs[e][1]) * 1e3 for e in last_step}
     assert kvq.workspace_error_word(ws) == 0, "device wait gave up (error word set)"
     if world > 1:
         ms = max_over_ranks(ms, dev)
@@ -525,46 +548,76 @@ def run_kvq(args, wl, rank, world, local_rank):
 
     kv_bytes = [kv_bytes_at(args.warmup + i) for i in range(args.steps)]
     q_bytes = B * Hq * D * 2
-    alg_bytes = sum(kv_bytes) + args.steps * q_bytes
+    # roofline over the timed split-K launches: their algorithmic bytes over
+    # their summed device time
+    split_bytes = sum(kv_bytes_at(s_) + q_bytes for s_ in last_step.values())
+    split_total_us = sum(split_us.values())
     tokens = B * args.steps * world
     value = tokens / (ms / 1e3)
 
-    # ---- end to end through the public call with pinned host buffers
+    # ---- end to end through the public call with pinned host buffers: every
+    # step copies its inputs in (the new K/V token and q) and its results out
+    # (out, lse).  The copies run on two copy streams, double-buffered, so a
+    # step's input copy overlaps the previous step's attention and its output
+    # copy overlaps the next one's; the attention calls stay in order on the
+    # compute stream.
     kn_h = kn.cpu().pin_memory() if kn is not None else None
     qs_h = qs.cpu().pin_memory()
-    k_d = torch.empty_like(kn[0, 0]) if kn is not None else None
-    v_d = torch.empty_like(kn[0, 1]) if kn is not None else None
-    q_d = torch.empty_like(qs[0])
-    out_h = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
-    lse_h = torch.empty((B, Hq), dtype=torch.float32).pin_memory()
+    k_d = [torch.empty_like(kn[0, 0]) for _ in range(2)] if kn is not None else None
+    v_d = [torch.empty_like(kn[0, 1]) for _ in range(2)] if kn is not None else None
+    q_d = [torch.empty_like(qs[0]) for _ in range(2)]
+    out_d = [torch.empty_like(out) for _ in range(2)]
+    lse_d = [torch.empty_like(lse) for _ in range(2)]
+    out_h = [torch.empty((B, Hq, D), dtype=torch.float32).pin_memory() for _ in range(2)]
+    lse_h = [torch.empty((B, Hq), dtype=torch.float32).pin_memory() for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    out_read = [torch.cuda.Event() for _ in range(2)]
     if wl.append:
         cache.seq_lens.copy_(base_lens)
 
-    def e2e_step(s):
-        e = s % episode
+    def e2e_step(s, n):  # n: steps since the start of this loop
+        e, j = s % episode, n % 2
+        with torch.cuda.stream(s_in):
+            if n >= 2:
+                s_in.wait_event(done[j])  # step n-2 no longer reads buffer j
+            if wl.append:
+                k_d[j].copy_(kn_h[e, 0], non_blocking=True)
+                v_d[j].copy_(kn_h[e, 1], non_blocking=True)
+            q_d[j].copy_(qs_h[e], non_blocking=True)
+            in_ready[j].record(s_in)
+        stream.wait_event(in_ready[j])
+        if n >= 2:
+            stream.wait_event(out_read[j])  # step n-2's results were copied out
         if wl.append:
             if e == 0:
                 cache.seq_lens.copy_(base_lens, non_blocking=True)
-            k_d.copy_(kn_h[e, 0], non_blocking=True)
-            v_d.copy_(kn_h[e, 1], non_blocking=True)
-        q_d.copy_(qs_h[e], non_blocking=True)
-        if wl.append:
-            kvq.kvq_decode_step(cache, k_d, v_d, q_d, out, lse, ws, max_len_hint=hint)
+            kvq.kvq_decode_step(cache, k_d[j], v_d[j], q_d[j], out_d[j], lse_d[j], ws,
+                                max_len_hint=hint)
         else:
-            kvq.kvq_decode_attention(segs, q_d, out, lse, ws, max_len_hint=hint)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+            kvq.kvq_decode_attention(segs, q_d[j], out_d[j], lse_d[j], ws, max_len_hint=hint)
+        done[j].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done[j])
+            out_h[j].copy_(out_d[j], non_blocking=True)
+            lse_h[j].copy_(lse_d[j], non_blocking=True)
+            out_read[j].record(s_out)
 
-    for s in range(args.warmup):
-        e2e_step(s)
+    for n in range(args.warmup):
+        e2e_step(n, n)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
     for i in range(args.steps):
-        e2e_step(args.warmup + i)
+        e2e_step(args.warmup + i, i)
+    for j in range(2):  # the region ends after the last results reached the host
+        stream.wait_event(out_read[j])
     e1.record(stream)
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
@@ -576,7 +629,7 @@ def run_kvq(args, wl, rank, world, local_rank):
     if rank != 0:
         return None
     peak, peak_kind = measured_peak()
-    achieved = alg_bytes / (split_ms / 1e3) / 1e9
+    achieved = split_bytes / (split_total_us / 1e6) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
@@ -588,8 +641,9 @@ def run_kvq(args, wl, rank, world, local_rank):
             **({"chunk_tokens": wl.chunk_tokens, "alpha": wl.alpha, "beta": wl.beta,
                 "segments": {f"bits{b}": int(ln.sum()) for b, ln in zip(seg_bits, seg_lens)}}
                if seg_lens is not None else {}),
-            "launch": "each phase of a step replayed from a CUDA graph captured once per "
-                      "episode position; events around the split-K replay",
+            "launch": "each step replayed from one CUDA graph per episode position "
+                      "(split-K kernel, then the merge as a programmatic dependent); "
+                      "event-record nodes in the graph time the split-K launch",
             "l2": f"inputs larger than L2: {sum(kv_bytes) / args.steps / 1e6:.0f} MB of packed "
                   f"K/V read per step per GPU (L2 126 MB)",
             "step": ("kvq_decode_step: quantize-on-write of 1 token/seq inside the split-K "
@@ -600,10 +654,14 @@ def run_kvq(args, wl, rank, world, local_rank):
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                      "traffic": recorded_traffic(wl.name), "kernel": split_kernel_name(wl),
-                     "alg_bytes_per_launch": alg_bytes / args.steps,
-                     "avg_launch_us": split_ms / args.steps * 1e3},
+                     "alg_bytes_per_launch": split_bytes / len(last_step),
+                     "avg_launch_us": split_total_us / len(last_step),
+                     "launches_timed": len(last_step)},
         "e2e": {"value": B * args.steps * world / (e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "kvq_decode_step (append workloads) or kvq_decode_attention through the "
+                        "Python binding; pinned host buffers, copies double-buffered on two "
+                        "copy streams"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }

@@ -66,7 +66,7 @@ int choose_splits(const kvq_cache& c, int max_len_hint, int ctas_per_sm) {
   thread_local int cached_n = 1;
   const long long kSlots = 148LL * (ctas_per_sm > 0 ? ctas_per_sm : 3);
   if (pairs == cached_pairs && len == cached_len && kSlots == cached_slots) return cached_n;
-  constexpr long long kOverhead = 400, kGran = 32, kMinTokens = 128;
+  constexpr long long kOverhead = 200, kGran = 32, kMinTokens = 128;
   const long long cap = (len + kMinTokens - 1) / kMinTokens;
   long long best_n = 1, best_cost = -1;
   for (long long n = 1; n <= cap && n <= 4096; ++n) {

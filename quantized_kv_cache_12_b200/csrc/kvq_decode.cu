@@ -92,6 +92,7 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   const SegView& seg = P.seg;
 
   extern __shared__ __align__(128) uint8_t smem[];
+  grid_dependents_may_launch();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -535,27 +536,38 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
 }
 
 // Merge the partial (m, l, o) of every split and segment (log-sum-exp).
-// One CTA per (sequence, query head); the 128 threads first reduce the max
-// and the weights over the partials together, then each thread sums one
-// output dim over the partials.
-__global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs a) {
-  extern __shared__ float w_sm[];  // [parts] weights 2^(m_p - M)
-  __shared__ float red[kHeadDim / 32];
+// One CTA of 128 x PG threads per (sequence, query head): all threads
+// reduce the max and the weights over the partials together; thread
+// (group j, dim d) then sums dim d over the partials j, j + PG, j + 2 PG, ...
+// with four independent sums (several loads in flight), and group 0 adds the
+// groups' sums.  It is launched as a programmatic dependent of the split-K
+// kernels: the launch overlaps their tail, and griddepcontrol.wait holds
+// every thread until they have completed and their stores are visible.
+template <int PG>
+__global__ void __launch_bounds__(kHeadDim * PG) decode_merge_kernel(const DecodeArgs a) {
+  extern __shared__ float w_sm[];  // [parts] weights 2^(m_p - M), then [PG][D] sums
+  __shared__ float red[4 * PG];
+  grid_dependency_wait();
+  constexpr int NT = kHeadDim * PG, NW = NT / 32;
   const long long bh = blockIdx.x;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const float* ml = a.part_ml + bh * a.parts * 2;
-  const float* po = a.part_o + bh * a.parts * kHeadDim;
+  const int d = t % kHeadDim, grp = t / kHeadDim;
+  const int P = a.parts;
+  const float* ml = a.part_ml + bh * P * 2;
+  const float* po = a.part_o + bh * P * kHeadDim;
   float m = -INFINITY;
-  for (int p = t; p < a.parts; p += kHeadDim)
+  for (int p = t; p < P; p += NT)
     if (ml[2 * p + 1] > 0.f) m = fmaxf(m, ml[2 * p]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) red[warp] = m;
   __syncthreads();
-  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  float M = red[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) M = fmaxf(M, red[w]);
   __syncthreads();
   float l = 0.f;
-  for (int p = t; p < a.parts; p += kHeadDim) {
+  for (int p = t; p < P; p += NT) {
     const float lp = ml[2 * p + 1];
     const float w = (lp > 0.f && M != -INFINITY) ? exp2f(ml[2 * p] - M) : 0.f;
     w_sm[p] = w;
@@ -565,18 +577,28 @@ __global__ void __launch_bounds__(kHeadDim) decode_merge_kernel(const DecodeArgs
   for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   if (lane == 0) red[warp] = l;
   __syncthreads();
-  const float L = red[0] + red[1] + red[2] + red[3];
+  float L = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) L += red[w];
   float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
-  int p = 0;
-  for (; p + 4 <= a.parts; p += 4) {
-    O0 = fmaf(w_sm[p], po[(long long)p * kHeadDim + t], O0);
-    O1 = fmaf(w_sm[p + 1], po[(long long)(p + 1) * kHeadDim + t], O1);
-    O2 = fmaf(w_sm[p + 2], po[(long long)(p + 2) * kHeadDim + t], O2);
-    O3 = fmaf(w_sm[p + 3], po[(long long)(p + 3) * kHeadDim + t], O3);
+  int p = grp;
+  for (; p + 3 * PG < P; p += 4 * PG) {
+    O0 = fmaf(w_sm[p], po[(long long)p * kHeadDim + d], O0);
+    O1 = fmaf(w_sm[p + PG], po[(long long)(p + PG) * kHeadDim + d], O1);
+    O2 = fmaf(w_sm[p + 2 * PG], po[(long long)(p + 2 * PG) * kHeadDim + d], O2);
+    O3 = fmaf(w_sm[p + 3 * PG], po[(long long)(p + 3 * PG) * kHeadDim + d], O3);
   }
-  for (; p < a.parts; ++p) O0 = fmaf(w_sm[p], po[(long long)p * kHeadDim + t], O0);
-  const float O = (O0 + O1) + (O2 + O3);
-  a.out[bh * kHeadDim + t] = (L > 0.f) ? O / L : 0.f;
+  for (; p < P; p += PG) O0 = fmaf(w_sm[p], po[(long long)p * kHeadDim + d], O0);
+  float O = (O0 + O1) + (O2 + O3);
+  if constexpr (PG > 1) {
+    float* osm = w_sm + P;
+    osm[grp * kHeadDim + d] = O;
+    __syncthreads();
+    if (grp != 0) return;
+#pragma unroll
+    for (int j = 1; j < PG; ++j) O += osm[j * kHeadDim + d];
+  }
+  a.out[bh * kHeadDim + d] = (L > 0.f) ? O / L : 0.f;
   if (a.lse != nullptr && t == 0)
     a.lse[bh] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
@@ -634,15 +656,33 @@ cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaS
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)a.parts * sizeof(float);
+template <int PG>
+cudaError_t launch_merge_pg(const DecodeArgs& a, cudaStream_t s) {
+  const size_t smem = ((size_t)a.parts + (PG > 1 ? PG * kHeadDim : 0)) * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_merge_kernel,
+    cudaError_t e = cudaFuncSetAttribute(decode_merge_kernel<PG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  decode_merge_kernel<<<(unsigned)((long long)a.batch * a.q_heads), kHeadDim, smem, s>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long long)a.batch * a.q_heads));
+  cfg.blockDim = dim3(kHeadDim * PG);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_merge_kernel<PG>, a);
+}
+
+cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s) {
+  // more partials: more thread groups, so that each thread's chain of
+  // dependent loads stays short
+  if (a.parts >= 48) return launch_merge_pg<4>(a, s);
+  if (a.parts >= 16) return launch_merge_pg<2>(a, s);
+  return launch_merge_pg<1>(a, s);
 }
 
 }  // namespace kvq

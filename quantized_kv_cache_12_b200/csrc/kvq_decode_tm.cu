@@ -148,6 +148,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   const SegView& seg = P.seg;
 
   extern __shared__ __align__(128) uint8_t smem[];
+  grid_dependents_may_launch();
   const int t = threadIdx.x;
   const int warp = t >> 5, lane = t & 31;
   const int gid = lane >> 2, tig = lane & 3;

@@ -64,6 +64,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization after this one may be scheduled once every CTA of this one
+// has executed the trigger (or exited) ...
+__device__ __forceinline__ void grid_dependents_may_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// ... and waits here until this one has completed and its memory operations
+// are visible (a no-op for a kernel launched without that attribute).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- bulk copy
 // One-dimensional bulk copy global -> shared, completion counted on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.  No multicast.
