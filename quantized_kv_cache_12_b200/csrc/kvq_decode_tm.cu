@@ -224,25 +224,30 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   const int patch_i = (append_here && patch_stage % kWarps == warp) ? patch_stage / kWarps : -1;
   const int patch_row = (L_old - c0) % C::STOK;
 
+  // A stage is filled by one bulk copy per plane (K codes, V codes, K meta,
+  // V meta), issued side by side by lanes 0 .. NCOPY-1: lane j holds its
+  // plane's source for this warp's first stage, its per-stage stride, its
+  // byte count and its offset inside a stage.
+  constexpr int NCOPY = C::MB > 0 ? 4 : 2;
   const long long row0 = ((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0;
-  const uint8_t* kc_src = seg.k_codes + row0 * C::RB;
-  const uint8_t* vc_src = seg.v_codes + row0 * C::RB;
-  const uint8_t* km_src = seg.k_meta + row0 * C::MB;
-  const uint8_t* vm_src = seg.v_meta + row0 * C::MB;
+  const int cp_j = lane < NCOPY ? lane : 0;
+  const int cp_rb = (cp_j < 2) ? C::RB : C::MB;  // bytes per token of the plane
+  const uint8_t* cp_src = (cp_j == 0 ? seg.k_codes : cp_j == 1 ? seg.v_codes
+                           : cp_j == 2 ? seg.k_meta : seg.v_meta) + row0 * cp_rb;
+  const uint32_t cp_off = cp_j == 0 ? 0u : cp_j == 1 ? (uint32_t)(C::STOK * C::RB)
+                          : cp_j == 2 ? (uint32_t)(2 * C::STOK * C::RB)
+                                      : (uint32_t)(2 * C::STOK * C::RB + C::STOK * C::MB);
+  const uint32_t cp_bytes = (uint32_t)(C::STOK * cp_rb);
+  const size_t cp_stride = (size_t)(kWarps * C::STOK) * cp_rb;
+  // stage i of this warp into ring slot st (all lanes call it together)
   auto issue = [&](int i, int st) {
-    uint8_t* dst = stages + st * C::STAGE;
-    mbar_arrive_expect_tx(&bars[st], C::STAGE);
-    const size_t tok = (size_t)i * (kWarps * C::STOK);
-    bulk_load(dst, kc_src + tok * C::RB, C::STOK * C::RB, &bars[st], policy);
-    bulk_load(dst + C::STOK * C::RB, vc_src + tok * C::RB, C::STOK * C::RB, &bars[st], policy);
-    if constexpr (C::MB > 0) {
-      bulk_load(dst + 2 * C::STOK * C::RB, km_src + tok * C::MB, C::STOK * C::MB, &bars[st],
-                policy);
-      bulk_load(dst + 2 * C::STOK * C::RB + C::STOK * C::MB, vm_src + tok * C::MB,
-                C::STOK * C::MB, &bars[st], policy);
-    }
+    if (lane == 0) mbar_arrive_expect_tx(&bars[st], C::STAGE);
+    __syncwarp();
+    if (lane < NCOPY)
+      bulk_load(stages + st * C::STAGE + cp_off, cp_src + (size_t)i * cp_stride, cp_bytes,
+                &bars[st], policy);
   };
-  if (lane == 0) {
+  {
     const int pre = min(n_tiles, C::STAGES);
     for (int i = 0; i < pre; ++i) issue(i, (st + i) % C::STAGES);
   }
@@ -585,7 +590,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     else
       stage_body(std::integral_constant<bool, false>(), sK, sV, sKm, sVm, n_stage);
     __syncwarp();
-    if (lane == 0 && i + C::STAGES < n_tiles) issue(i + C::STAGES, st);
+    if (i + C::STAGES < n_tiles) issue(i + C::STAGES, st);
     if (++st == C::STAGES) {
       st = 0;
       phase ^= 1u;
