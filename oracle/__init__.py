@@ -59,6 +59,15 @@ def _load():
         lib.kvqo_attention_blocks.argtypes = [P, i32, P, P, i32, f64, P, i32, P, P]
         lib.kvqo_attention_packed.argtypes = [P, i32, i32, P, P, i32, P, P, i32, i32,
                                               i64, i32, f64, P, P]
+        lib.kvqo_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.kvqo_e4m3_to_f64.restype = f64
+        lib.kvqo_f32_to_e4m3.argtypes = [ctypes.c_float]
+        lib.kvqo_f32_to_e4m3.restype = ctypes.c_uint8
+        lib.kvqo_quantize_group_fp8.argtypes = [P, i32, P, P]
+        lib.kvqo_quantize_rows_fp8.argtypes = [P, i64, i32, i32, P, P]
+        lib.kvqo_dequantize_rows_fmt.argtypes = [P, P, i64, i32, i32, i32, i32, P]
+        lib.kvqo_attention_packed_fmt.argtypes = [P, i32, i32, P, P, i32, P, P, i32, i32, i32,
+                                                  i64, i32, f64, P, P]
         lib.kvqo_chunk_assign.argtypes = [P, P, i32, i32, f64, f64, P, P]
         lib.kvqo_chunk_partition.argtypes = [P, i32, P, P]
         lib.kvqo_kv_elements.argtypes = [u64, u64, u64, u64, u64]
@@ -119,29 +128,65 @@ def quantize_group(x16, bits: int):
     return code, int(s[0]), int(z[0])
 
 
-def quantize_rows(x16, group: int, bits: int):
+def quantize_rows(x16, group: int, bits: int, fmt: str = "int"):
     """Token rows [N, D] of fp16 bit patterns -> (codes [N, D*bits/8] uint8,
-    meta [N, D/G, 2] uint16 holding the (scale, zero) fp16 patterns)."""
+    meta [N, D/G, 2] uint16 holding the (scale, zero) fp16 patterns).
+    fmt "fp8": E4M3 codes (bits 8) with zero point 0 (KV-cache page, FP8)."""
     lib = _load()
     x16 = _c(x16, np.uint16)
     N, D = x16.shape
     codes = np.zeros((N, D * bits // 8), np.uint8)
     ng = D // group if bits != 16 else 1
     meta = np.zeros((N, ng, 2), np.uint16)
-    lib.kvqo_quantize_rows(_p(x16), N, D, group, bits, _p(codes), _p(meta))
+    if fmt == "fp8":
+        assert bits == 8
+        lib.kvqo_quantize_rows_fp8(_p(x16), N, D, group, _p(codes), _p(meta))
+    else:
+        lib.kvqo_quantize_rows(_p(x16), N, D, group, bits, _p(codes), _p(meta))
     return codes, meta
 
 
-def dequantize_rows(codes, meta, D: int, group: int, bits: int) -> np.ndarray:
-    """Packed rows -> fp64 [N, D], x_hat = (c - z) * s (exact in fp64)."""
+def dequantize_rows(codes, meta, D: int, group: int, bits: int, fmt: str = "int") -> np.ndarray:
+    """Packed rows -> fp64 [N, D]: x_hat = (c - z) * s, or e4m3(c) * s for
+    fmt "fp8" (both exact in fp64)."""
     lib = _load()
     codes = _c(codes, np.uint8)
     N = codes.shape[0]
     meta = _c(meta if meta is not None else np.zeros((N, 1, 2), np.uint16), np.uint16)
     out = np.zeros((N, D), np.float64)
-    lib.kvqo_dequantize_rows(_p(codes), _p(meta), N, D, group if bits != 16 else D, bits,
-                             _p(out))
+    lib.kvqo_dequantize_rows_fmt(_p(codes), _p(meta), N, D, group if bits != 16 else D, bits,
+                                 int(fmt == "fp8"), _p(out))
     return out
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 (KV-cache page, FP8 KV cache; reading R14 in kvq_oracle.c)
+# --------------------------------------------------------------------------
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """E4M3 codes (uint8) -> fp64 values (NaN for S.1111.111)."""
+    lib = _load()
+    c = _c(codes, np.uint8).ravel()
+    return np.array([lib.kvqo_e4m3_to_f64(int(v)) for v in c], np.float64).reshape(
+        np.shape(codes))
+
+
+def f32_to_e4m3(x) -> np.ndarray:
+    """fp32 values -> nearest E4M3 codes, ties to even, saturating at 448."""
+    lib = _load()
+    x = _c(x, np.float32)
+    return np.array([lib.kvqo_f32_to_e4m3(float(v)) for v in x.ravel()], np.uint8).reshape(
+        x.shape)
+
+
+def quantize_group_fp8(x16):
+    """One group of fp16 bit patterns -> (E4M3 codes uint8[G], s16)."""
+    lib = _load()
+    x16 = _c(x16, np.uint16)
+    code = np.zeros(x16.size, np.uint8)
+    s = np.zeros(1, np.uint16)
+    lib.kvqo_quantize_group_fp8(_p(x16), x16.size, _p(code), _p(s))
+    return code, int(s[0])
 
 
 # --------------------------------------------------------------------------
@@ -232,12 +277,12 @@ def kv_elements(layers: int, kv_heads: int, head_dim: int, seq_len: int, batch: 
 # Whole-cache helpers built from the functions above
 # --------------------------------------------------------------------------
 
-def quantize_cache(x16, group: int, bits: int):
+def quantize_cache(x16, group: int, bits: int, fmt: str = "int"):
     """x16 [..., T, D] fp16 patterns -> codes [..., T, D*bits/8], meta [..., T, D/G, 2]."""
     x16 = _c(x16, np.uint16)
     lead = x16.shape[:-1]
     D = x16.shape[-1]
-    codes, meta = quantize_rows(x16.reshape(-1, D), group, bits)
+    codes, meta = quantize_rows(x16.reshape(-1, D), group, bits, fmt)
     return (codes.reshape(*lead, D * bits // 8),
             meta.reshape(*lead, meta.shape[-2], 2))
 
@@ -248,7 +293,8 @@ def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: fl
 
     q16: [B, Hq, D] fp16/bf16 patterns.  segments: list of dicts with numpy
     arrays ``k_codes``/``v_codes`` [B, Hkv, T, row_bytes], ``k_meta``/``v_meta``
-    [B, Hkv, T, D/G, 2] (None for bits 16), ``bits``, ``group``.
+    [B, Hkv, T, D/G, 2] (None for bits 16), ``bits``, ``group`` and optionally
+    ``fmt`` ("int", the default, or "fp8").
     seq_lens_per_seg: list of int arrays [B].  The segments of a sequence are
     concatenated in token order (attention does not depend on the order).
     pairs: optional list of (b, kv_head) to evaluate; others stay NaN.
@@ -269,8 +315,9 @@ def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: fl
             bits, G = seg["bits"], seg["group"]
             km = seg["k_meta"][b, h, :L] if bits != 16 else None
             vm = seg["v_meta"][b, h, :L] if bits != 16 else None
-            Ks.append(dequantize_rows(seg["k_codes"][b, h, :L], km, D, G, bits))
-            Vs.append(dequantize_rows(seg["v_codes"][b, h, :L], vm, D, G, bits))
+            fmt = seg.get("fmt", "int")
+            Ks.append(dequantize_rows(seg["k_codes"][b, h, :L], km, D, G, bits, fmt))
+            Vs.append(dequantize_rows(seg["v_codes"][b, h, :L], vm, D, G, bits, fmt))
         K = np.concatenate(Ks, 0)
         V = np.concatenate(Vs, 0)
         qh = q16[b, h * g:(h + 1) * g]

@@ -28,6 +28,10 @@
  *   [P5] TurboQuant page (bhfrc.com news 57821): 1.2 (KV element count
  *        worked example); 2.3 (per-group scaling, dequantization inside
  *        the attention matmul).
+ *   [P2'] The KV-cache page above, "主流KV Cache量化方案对比" item 1 (FP8
+ *        KV cache, E4M3 or E5M2, 2x compression) and "实践中的调优建议"
+ *        (dynamic quantization: the scale is computed from the current
+ *        vectors at every step).
  *
  * Readings taken where the pages are silent (each one also listed in the
  * design notes):
@@ -51,6 +55,13 @@
  *       are taken over the chunks of one sequence; all in fp64.
  *   R9  Reorder order: FP16 chunks, then INT4, then INT2, each class in
  *       ascending original chunk index.
+ *   R14 FP8 codes are E4M3 in the variant without infinities (bias 7, three
+ *       mantissa bits, largest finite 448, S.1111.111 is NaN).  Scales are
+ *       dynamic and per group of G along head_dim of each token, like the
+ *       integer formats: s = max(amax / 448, 1e-5) in fp32, stored in fp16
+ *       rounded toward +infinity (so |x / s| <= 448), zero point 0; each
+ *       code is x / s (one fp32 division) rounded to the nearest E4M3 value,
+ *       ties to even, saturating at +-448; x_hat = e4m3(code) * s.
  */
 #include <math.h>
 #include <stdint.h>
@@ -234,6 +245,87 @@ void kvqo_quantize_rows(const uint16_t *x, int64_t n_rows, int D, int G,
     free(tmp);
 }
 
+/* ------------------------------------------------------------------------ */
+/* FP8 E4M3 ([P2'] item 1; R14), written from the format definition.       */
+/* ------------------------------------------------------------------------ */
+
+/* Value of an E4M3 code: (-1)^S * 2^(E-7) * (1 + M/8) for E >= 1, and
+ * (-1)^S * 2^-6 * M/8 for E = 0; E = 15 with M = 7 is NaN. */
+double kvqo_e4m3_to_f64(uint8_t c)
+{
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp((double)(8 + m), e - 10);
+    return sgn ? -v : v;
+}
+
+/* Nearest E4M3 code to an fp32 value, ties to even, magnitudes past the
+ * largest finite value (448) saturated to it; NaN gives S.1111.111. */
+uint8_t kvqo_f32_to_e4m3(float x)
+{
+    if (isnan(x))
+        return 0x7F;
+    uint8_t sgn = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    /* the spacing of E4M3 values around a: 2^-9 below 2^-6, else 2^(e-3) */
+    int e = (a > 0.0) ? (int)floor(log2(a)) : -100;
+    if (a > 0.0 && ldexp(1.0, e) > a) /* guard log2 rounding */
+        e -= 1;
+    if (a > 0.0 && ldexp(1.0, e + 1) <= a)
+        e += 1;
+    double quantum = ldexp(1.0, (e < -6 ? -6 : e) - 3);
+    double r = rint(a / quantum) * quantum; /* a / quantum is exact */
+    if (r > 448.0)
+        r = 448.0;
+    if (r == 0.0)
+        return sgn;
+    int re = (int)floor(log2(r));
+    if (ldexp(1.0, re) > r)
+        re -= 1;
+    if (re < -6)
+        return (uint8_t)(sgn | (uint8_t)(r / ldexp(1.0, -9))); /* subnormal */
+    int m = (int)(r / ldexp(1.0, re - 3)) - 8;
+    return (uint8_t)(sgn | ((re + 7) << 3) | m);
+}
+
+/* One group of G binary16 values to E4M3 codes with scale s (R14). */
+void kvqo_quantize_group_fp8(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
+{
+    float amax = 0.0f;
+    for (int j = 0; j < G; ++j) {
+        float v = fabsf(kvqo_f16_to_f32(x[j]));
+        if (v > amax)
+            amax = v;
+    }
+    float s32 = amax / 448.0f;
+    if (s32 < 1e-5f)
+        s32 = 1e-5f;
+    uint16_t s16 = kvqo_f32_to_f16_up(s32);
+    float s = kvqo_f16_to_f32(s16);
+    for (int j = 0; j < G; ++j)
+        code[j] = kvqo_f32_to_e4m3(kvqo_f16_to_f32(x[j]) / s);
+    *s_out = s16;
+}
+
+/* Token rows to E4M3 codes (one byte per element) and (s, 0) fp16 pairs per
+ * group of G along the row. */
+void kvqo_quantize_rows_fp8(const uint16_t *x, int64_t n_rows, int D, int G, uint8_t *codes,
+                            uint16_t *meta)
+{
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int g = 0; g < D / G; ++g) {
+            uint16_t s16;
+            kvqo_quantize_group_fp8(x + r * D + g * G, G, codes + r * D + g * G, &s16);
+            meta[(r * (D / G) + g) * 2 + 0] = s16;
+            meta[(r * (D / G) + g) * 2 + 1] = 0; /* zero point 0 */
+        }
+}
+
 /* Unpack code e of a packed row (R7). */
 static unsigned kvqo_code_at(const uint8_t *row, int e, int bits)
 {
@@ -243,8 +335,26 @@ static unsigned kvqo_code_at(const uint8_t *row, int e, int bits)
 
 /*
  * Dequantize n_rows packed rows: x_hat = (c - z) * s, evaluated in fp64,
- * where it is exact (|c - z| < 2^17 and s has 11 significant bits).
+ * where it is exact (|c - z| < 2^17 and s has 11 significant bits); with
+ * fp8 != 0 the codes are E4M3 and x_hat = e4m3(c) * s (R14), also exact.
  */
+void kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *meta,
+                          int64_t n_rows, int D, int G, int bits, double *out);
+
+void kvqo_dequantize_rows_fmt(const uint8_t *codes, const uint16_t *meta, int64_t n_rows,
+                              int D, int G, int bits, int fp8, double *out)
+{
+    if (fp8) {
+        for (int64_t r = 0; r < n_rows; ++r)
+            for (int e = 0; e < D; ++e) {
+                double s = (double)kvqo_f16_to_f32(meta[(r * (D / G) + e / G) * 2 + 0]);
+                out[r * D + e] = kvqo_e4m3_to_f64(codes[r * D + e]) * s;
+            }
+        return;
+    }
+    kvqo_dequantize_rows(codes, meta, n_rows, D, G, bits, out);
+}
+
 void kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *meta,
                           int64_t n_rows, int D, int G, int bits, double *out)
 {
@@ -390,12 +500,29 @@ void kvqo_attention_blocks(const double *q, int g, const double *K,
  * the fp64 attention above is applied.  q16: [g][D] binary16 or bfloat16
  * bit patterns (q_is_bf16).
  */
+void kvqo_attention_packed_fmt(const uint16_t *q16, int q_is_bf16, int g,
+                               const uint8_t *k_codes, const uint16_t *k_meta, int k_bits,
+                               const uint8_t *v_codes, const uint16_t *v_meta, int v_bits,
+                               int fp8, int G, int64_t L, int D, double scale, double *o,
+                               double *lse);
+
 void kvqo_attention_packed(const uint16_t *q16, int q_is_bf16, int g,
                            const uint8_t *k_codes, const uint16_t *k_meta,
                            int k_bits, const uint8_t *v_codes,
                            const uint16_t *v_meta, int v_bits, int G,
                            int64_t L, int D, double scale, double *o,
                            double *lse)
+{
+    kvqo_attention_packed_fmt(q16, q_is_bf16, g, k_codes, k_meta, k_bits, v_codes, v_meta,
+                              v_bits, 0, G, L, D, scale, o, lse);
+}
+
+/* The same with a code format: fp8 != 0 means E4M3 codes for K and V. */
+void kvqo_attention_packed_fmt(const uint16_t *q16, int q_is_bf16, int g,
+                               const uint8_t *k_codes, const uint16_t *k_meta, int k_bits,
+                               const uint8_t *v_codes, const uint16_t *v_meta, int v_bits,
+                               int fp8, int G, int64_t L, int D, double scale, double *o,
+                               double *lse)
 {
     double *q = (double *)malloc((size_t)g * D * sizeof(double));
     for (int64_t i = 0; i < (int64_t)g * D; ++i)
@@ -405,8 +532,8 @@ void kvqo_attention_packed(const uint16_t *q16, int q_is_bf16, int g,
     double *V = (double *)malloc((size_t)(L > 0 ? L : 1) * D * sizeof(double));
     int Gk = (k_bits == 16) ? D : G;
     int Gv = (v_bits == 16) ? D : G;
-    kvqo_dequantize_rows(k_codes, k_meta, L, D, Gk, k_bits, K);
-    kvqo_dequantize_rows(v_codes, v_meta, L, D, Gv, v_bits, V);
+    kvqo_dequantize_rows_fmt(k_codes, k_meta, L, D, Gk, k_bits, fp8, K);
+    kvqo_dequantize_rows_fmt(v_codes, v_meta, L, D, Gv, v_bits, fp8, V);
     kvqo_attention(q, g, K, V, L, D, scale, o, lse);
     free(q);
     free(K);

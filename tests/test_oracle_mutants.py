@@ -46,6 +46,13 @@ MUTANTS = [
      "static const uint8_t order[3] = {16, 2, 4};"),
     ("f16 rounding truncates", "if (rest > 0x1000u || (rest == 0x1000u && (h & 1u)))",
      "if (rest > 0x1000u)"),
+    ("e4m3 ties away from zero", "double r = rint(a / quantum) * quantum;",
+     "double r = round(a / quantum) * quantum;"),
+    ("e4m3 without subnormal spacing", "double quantum = ldexp(1.0, (e < -6 ? -6 : e) - 3);",
+     "double quantum = ldexp(1.0, e - 3);"),
+    ("e4m3 exponent bias 8", "v = ldexp((double)(8 + m), e - 10);",
+     "v = ldexp((double)(8 + m), e - 11);"),
+    ("fp8 scale from another maximum", "float s32 = amax / 448.0f;", "float s32 = amax / 464.0f;"),
 ]
 
 
@@ -120,6 +127,22 @@ def _pins(o):
     ob, lb = o.attention_blocks(q, K * 3, V, 0.2, [0, 7, 7, 30, 50])
     od, ld = o.attention(q, K * 3, V, 0.2)
     yield "blocks equal direct", bool(np.allclose(ob, od, atol=1e-12) and np.allclose(lb, ld, atol=1e-12))
+
+    f8 = _golden("fp8_worked_example.json")
+    ok = True
+    for g in f8["groups"]:
+        code, s16 = o.quantize_group_fp8(np.asarray(g["x"], np.float16).view(np.uint16))
+        ok &= code.tolist() == g["codes"] and s16 == int(g["s16"], 16)
+    yield "fp8 worked groups", bool(ok)
+    codes = np.arange(256, dtype=np.uint8)
+    v8 = o.e4m3_to_f64(codes)
+    t8 = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    yield "e4m3 decode vs torch", bool(np.all((v8 == t8) | (np.isnan(v8) & np.isnan(t8))))
+    fin = np.unique(t8[~np.isnan(t8)])
+    mids = np.concatenate([(fin[:-1] + fin[1:]) / 2, rng.standard_normal(2000) * 30]).astype(np.float32)
+    mids = np.clip(mids, -448, 448)
+    yield "e4m3 encode vs torch", bool(np.array_equal(
+        o.f32_to_e4m3(mids), torch.from_numpy(mids).to(torch.float8_e4m3fn).view(torch.uint8).numpy()))
 
     t = _golden("chunk_threshold_toy.json")
     sim, cls = o.chunk_assign(np.array(t["chunks"], np.float32), np.array(t["query"], np.float32),
