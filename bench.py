@@ -194,22 +194,22 @@ def run_reference(args, wl):
     g = wl.group_ratio
     prepared = []
     for h in range(sub.kv_heads):
-        kc, km = oracle.quantize_rows(k[0, h].numpy().view(np.uint16), wl.group, wl.bits)
-        vc, vm = oracle.quantize_rows(v[0, h].numpy().view(np.uint16), wl.group, wl.bits)
+        kc, km = oracle.quantize_rows(k[0, h].numpy().view(np.uint16), wl.group, wl.bits, wl.fmt)
+        vc, vm = oracle.quantize_rows(v[0, h].numpy().view(np.uint16), wl.group, wl.bits, wl.fmt)
         qh = q[0, h * g:(h + 1) * g].contiguous().view(torch.int16).numpy().view(np.uint16)
         prepared.append((kc, km, vc, vm, qh, kn[0, h].numpy().view(np.uint16),
                          vn[0, h].numpy().view(np.uint16)))
 
     def step(i):
         kc, km, vc, vm, qh, knew, vnew = prepared[i % len(prepared)]
-        ck, mk = oracle.quantize_rows(knew, wl.group, wl.bits)
-        cv, mv = oracle.quantize_rows(vnew, wl.group, wl.bits)
+        ck, mk = oracle.quantize_rows(knew, wl.group, wl.bits, wl.fmt)
+        cv, mv = oracle.quantize_rows(vnew, wl.group, wl.bits, wl.fmt)
         kc2 = np.concatenate([kc, ck])
         km2 = np.concatenate([km, mk])
         vc2 = np.concatenate([vc, cv])
         vm2 = np.concatenate([vm, mv])
         oracle.attention_packed(qh, wl.q_dtype == "bf16", kc2, km2, wl.bits, vc2, vm2, wl.bits,
-                                wl.group, L + 1, 128 ** -0.5)
+                                wl.group, L + 1, 128 ** -0.5, wl.fmt)
 
     for i in range(args.warmup):
         step(i)
@@ -229,7 +229,8 @@ def reference_line(args, wl, value, el, sample):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": DTYPE[wl.bits], "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3" if wl.fmt == "fp8" else DTYPE[wl.bits],
+        "data": "synthetic",
         "config": workload_config(wl),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
@@ -242,6 +243,7 @@ def workload_config(wl, extra=None):
     cfg = {"workload": wl.name, "batch_per_gpu": wl.batch, "q_heads": wl.q_heads,
            "kv_heads": wl.kv_heads, "head_dim": wl.head_dim, "context": wl.context,
            "bits": wl.bits, "group": wl.group, "q_dtype": wl.q_dtype,
+           **({"format": "fp8 e4m3"} if wl.fmt == "fp8" else {}),
            "episode_steps": wl.steps if wl.append else 0}
     if extra:
         cfg.update(extra)
@@ -263,8 +265,8 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
     for b, h in pairs:
         kk = k[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
         vv = v[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-        kc, km = oracle.quantize_rows(kk, wl.group, wl.bits)
-        vc, vm = oracle.quantize_rows(vv, wl.group, wl.bits)
+        kc, km = oracle.quantize_rows(kk, wl.group, wl.bits, wl.fmt)
+        vc, vm = oracle.quantize_rows(vv, wl.group, wl.bits, wl.fmt)
         qh = q[b, h * g:(h + 1) * g].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
         knew = kn[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
         vnew = vn[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
@@ -274,12 +276,12 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
     t0 = time.perf_counter()
     while True:
         kc, km, vc, vm, qh, knew, vnew = prepared[n % len(prepared)]
-        ck, mk = oracle.quantize_rows(knew, wl.group, wl.bits)
-        cv, mv = oracle.quantize_rows(vnew, wl.group, wl.bits)
+        ck, mk = oracle.quantize_rows(knew, wl.group, wl.bits, wl.fmt)
+        cv, mv = oracle.quantize_rows(vnew, wl.group, wl.bits, wl.fmt)
         oracle.attention_packed(qh, wl.q_dtype == "bf16", np.concatenate([kc, ck]),
                                 np.concatenate([km, mk]), wl.bits, np.concatenate([vc, cv]),
                                 np.concatenate([vm, mv]), wl.bits, wl.group, L + 1,
-                                128 ** -0.5)
+                                128 ** -0.5, fmt=wl.fmt)
         n += 1
         el = time.perf_counter() - t0
         if el >= seconds and n >= 2:
@@ -406,7 +408,9 @@ def run_kvq(args, wl, rank, world, local_rank):
     else:
         max_tokens = workloads.round_up(ctx + episode + 1, 64)
         k, v = workloads.kv_tokens(wlr, ctx, dev)
-        cache = kvq.QuantizedKVCache.allocate(B, H, D, max_tokens, wl.bits, wl.group, dev)
+        cache = kvq.QuantizedKVCache.allocate(
+            B, H, D, max_tokens, wl.bits, wl.group, dev,
+            fmt=kvq.KVQ_FMT_FP8_E4M3 if wl.fmt == "fp8" else kvq.KVQ_FMT_INT)
         cache.seq_lens.zero_()
         kvq.kvq_quantize_append(cache, k, v, ctx, advance_seq_lens=True)
         base_lens = cache.seq_lens.clone()
@@ -653,7 +657,7 @@ def run_kvq(args, wl, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": DTYPE[wl.bits], "data": "synthetic",
+        "dtype": "e4m3" if wl.fmt == "fp8" else DTYPE[wl.bits], "data": "synthetic",
         "config": workload_config(wl, {
             "global_batch": B * world, "parallelism": f"dp{world} (sequences sharded)",
             "cache_tokens_per_step": f"{ctx + 1}..{ctx + episode}" if wl.append else ctx,

@@ -66,6 +66,12 @@ typedef enum kvq_status {
 
 typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
 
+/* Code format of a plane. */
+typedef enum kvq_format {
+    KVQ_FMT_INT = 0,      /* asymmetric integer codes: x_hat = (c - z) * s    */
+    KVQ_FMT_FP8_E4M3 = 1  /* FP8 E4M3 codes, bits 8: x_hat = e4m3(c) * s      */
+} kvq_format;
+
 /*
  * One K or V plane of a cache (one bit-width).
  *   bits 2, 4, 8: codes  u8  [batch][kv_heads][max_tokens][head_dim*bits/8],
@@ -74,6 +80,11 @@ typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
  *                 meta  f16 [batch][kv_heads][max_tokens][head_dim/G][2],
  *                 the pair (scale, zero point) of each group, groups of G
  *                 consecutive head_dim elements of one token row.
+ *   bits 8 with fmt KVQ_FMT_FP8_E4M3: one E4M3 code per element (bias 7,
+ *                 no infinities, largest finite 448), the same meta layout
+ *                 with zero point 0 (the KV-cache page's FP8 KV cache, with
+ *                 the scale of each group computed from the values written,
+ *                 that page's dynamic quantization).
  *   bits 16:      codes f16 [batch][kv_heads][max_tokens][head_dim] raw
  *                 values (Cocktail's FP16 class); meta unused (may be NULL).
  * Both buffers 16-byte aligned.
@@ -83,6 +94,7 @@ typedef struct kvq_plane {
     int32_t group_size; /* G: 32, 64 or 128, dividing head_dim (bits < 16)  */
     void *codes;        /* device                                           */
     void *meta;         /* device; NULL when bits == 16                     */
+    int32_t fmt;        /* kvq_format; KVQ_FMT_FP8_E4M3 needs bits 8        */
 } kvq_plane;
 
 /*

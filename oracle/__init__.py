@@ -224,8 +224,9 @@ def attention_blocks(q, K, V, scale: float, bounds: Sequence[int]):
 
 
 def attention_packed(q16, q_is_bf16: bool, k_codes, k_meta, k_bits: int, v_codes, v_meta,
-                     v_bits: int, group: int, L: int, scale: float):
-    """Attention of g query heads over one packed (sequence, KV head) cache."""
+                     v_bits: int, group: int, L: int, scale: float, fmt: str = "int"):
+    """Attention of g query heads over one packed (sequence, KV head) cache
+    (fmt "fp8": E4M3 codes for K and V)."""
     lib = _load()
     q16 = _c(q16, np.uint16)
     g, D = q16.shape
@@ -235,9 +236,9 @@ def attention_packed(q16, q_is_bf16: bool, k_codes, k_meta, k_bits: int, v_codes
     vm = _c(v_meta, np.uint16) if v_bits != 16 else np.zeros(1, np.uint16)
     o = np.zeros((g, D), np.float64)
     lse = np.zeros(g, np.float64)
-    lib.kvqo_attention_packed(_p(q16), int(bool(q_is_bf16)), g, _p(kc), _p(km), k_bits,
-                              _p(vc), _p(vm), v_bits, group, L, D, float(scale), _p(o),
-                              _p(lse))
+    lib.kvqo_attention_packed_fmt(_p(q16), int(bool(q_is_bf16)), g, _p(kc), _p(km), k_bits,
+                                  _p(vc), _p(vm), v_bits, int(fmt == "fp8"), group, L, D,
+                                  float(scale), _p(o), _p(lse))
     return o, lse
 
 

@@ -20,8 +20,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool valid_group(int g) { return g == 32 || g == 64 || g == 128; }
 
+// The kernels' template tag of a plane's format: its bit width, or kE4M3.
+int kernel_bits(const kvq_plane& p) { return p.fmt == KVQ_FMT_FP8_E4M3 ? kvq::kE4M3 : p.bits; }
+
 kvq_status check_plane(const kvq_plane& p, int head_dim, bool allow16) {
   if (p.codes == nullptr || !aligned16(p.codes)) return KVQ_ERR_INVALID_ARG;
+  if (p.fmt != KVQ_FMT_INT && p.fmt != KVQ_FMT_FP8_E4M3) return KVQ_ERR_INVALID_ARG;
+  if (p.fmt == KVQ_FMT_FP8_E4M3 && p.bits != 8) return KVQ_ERR_UNSUPPORTED;
   if (p.bits == 16) {
     if (!allow16) return KVQ_ERR_UNSUPPORTED;
     return KVQ_OK;
@@ -43,7 +48,7 @@ kvq_status check_cache(const kvq_cache* c, bool allow16) {
   if (s != KVQ_OK) return s;
   s = check_plane(c->v, c->head_dim, allow16);
   if (s != KVQ_OK) return s;
-  if (c->k.bits != c->v.bits) return KVQ_ERR_UNSUPPORTED;
+  if (c->k.bits != c->v.bits || c->k.fmt != c->v.fmt) return KVQ_ERR_UNSUPPORTED;
   if (c->k.bits != 16 && c->k.group_size != c->v.group_size) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }
@@ -95,7 +100,7 @@ kvq_status plan_splits(const kvq_cache* segs, int n_segs, int q_heads, int max_l
   plan->parts = 0;
   const int g = q_heads / segs[0].kv_heads;
   for (int i = 0; i < n_segs; ++i) {
-    const int bits = segs[i].k.bits;
+    const int bits = kernel_bits(segs[i].k);
     const int ctas = kvq::decode_ctas_per_sm(bits, bits == 16 ? kD : segs[i].k.group_size, g);
     plan->n_split[i] = choose_splits(segs[i], max_len_hint, ctas);
     plan->parts += plan->n_split[i];
@@ -115,7 +120,7 @@ kvq_status check_segments(const kvq_cache* segs, int n_segs, int q_heads) {
   if (q_heads <= 0 || q_heads % segs[0].kv_heads != 0) return KVQ_ERR_INVALID_ARG;
   const int g = q_heads / segs[0].kv_heads;
   for (int i = 0; i < n_segs; ++i) {
-    const int bits = segs[i].k.bits;
+    const int bits = kernel_bits(segs[i].k);
     if (!kvq::decode_supported(bits, bits == 16 ? kD : segs[i].k.group_size, g))
       return KVQ_ERR_UNSUPPORTED;
   }
@@ -222,7 +227,7 @@ kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const 
   a.max_tokens = cache->max_tokens;
   a.n_new = n_new;
   a.advance = advance_seq_lens != 0;
-  cudaError_t e = kvq::launch_quantize(a, cache->k.bits, cache->k.group_size,
+  cudaError_t e = kvq::launch_quantize(a, kernel_bits(cache->k), cache->k.group_size,
                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
@@ -296,7 +301,7 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
     v.k_meta = static_cast<const uint8_t*>(segs[i].k.meta);
     v.v_meta = static_cast<const uint8_t*>(segs[i].v.meta);
     v.seq_lens = segs[i].seq_lens;
-    v.bits = segs[i].k.bits;
+    v.bits = kernel_bits(segs[i].k);
     v.group = segs[i].k.bits == 16 ? kD : segs[i].k.group_size;
     v.max_tokens = segs[i].max_tokens;
     v.n_split = plan.n_split[i];
@@ -353,7 +358,7 @@ kvq_status decode_step_stages(const kvq_cache* cache, const void* k_new, const v
   if (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new))
     return KVQ_ERR_INVALID_ARG;
   const int g = q_heads / cache->kv_heads;
-  if (kvq::decode_tm_supported(cache->k.bits, cache->k.group_size, g))
+  if (kvq::decode_tm_supported(kernel_bits(cache->k), cache->k.group_size, g))
     return decode_stages(cache, 1, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
                          workspace, workspace_bytes, stream, stages, k_new, v_new);
   // formats of the 16-row kernel: the append kernel, then the attention
@@ -412,7 +417,8 @@ kvq_status kvq_chunk_reorder(const kvq_cache* segs, const void* k_src, const voi
   for (int i = 0; i < 3; ++i) {
     kvq_status st = check_cache(&segs[i], true);
     if (st != KVQ_OK) return st;
-    if (segs[i].k.bits != want_bits[i]) return KVQ_ERR_INVALID_ARG;
+    if (segs[i].k.bits != want_bits[i] || segs[i].k.fmt != KVQ_FMT_INT)
+      return KVQ_ERR_INVALID_ARG;
     if (segs[i].batch != segs[0].batch || segs[i].kv_heads != segs[0].kv_heads)
       return KVQ_ERR_INVALID_ARG;
   }

@@ -56,7 +56,7 @@ template <int BITS, int GE, int GR>
 struct TmCfg {
   static constexpr int D = kHeadDim;
   static constexpr int NG = D / GE;                    // groups per token
-  static constexpr int RB = D * BITS / 8;              // code bytes per token
+  static constexpr int RB = D * code_bits(BITS) / 8;   // code bytes per token
   static constexpr int MB = (BITS == 16) ? 0 : NG * 4; // (s, z) bytes per token
   static constexpr int KC = RB / 4;                    // K bytes of a lane (32 dims)
   static constexpr int KW = KC / 4;
@@ -143,7 +143,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   using XP = CrossPairs<BITS>;
   constexpr int D = C::D, NG = C::NG, NP = C::NP, HS = C::HS, CPH = C::CPH;
   // grouped PV: dims of each group per lane, and their V bytes and words
-  constexpr int CH = GE / 8, VBG = CH * BITS / 8, VWG = VBG >= 4 ? VBG / 4 : 1;
+  constexpr int CH = GE / 8, VBG = CH * code_bits(BITS) / 8, VWG = VBG >= 4 ? VBG / 4 : 1;
   const DecodeArgs& a = P.a;
   const SegView& seg = P.seg;
 
@@ -345,6 +345,21 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     constexpr bool FULL = decltype(full_tag)::value;
     constexpr int NS = C::SUB;
     auto valid = [&](int tok) { return FULL || tok < n_valid; };  // tok: 0 .. STOK-1
+    // V rows past the valid length may hold any bytes.  Integer codes are
+    // finite and meet a zero weight; raw fp16 and e4m3 bytes can be NaN or
+    // Inf, which a zero weight does not cancel in the MMA: zero those words.
+    auto zero_invalid = [&](int sub, auto& wA, auto& wB, auto& wC, auto& wD) {
+      if constexpr ((BITS == 16 || BITS == kE4M3) && !FULL) {
+        constexpr int NW = sizeof(wA) / sizeof(wA[0]);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          wA[w] = valid(sub * kTile + tvA) ? wA[w] : 0u;
+          wB[w] = valid(sub * kTile + tvB) ? wB[w] : 0u;
+          wC[w] = valid(sub * kTile + tvA + 8) ? wC[w] : 0u;
+          wD[w] = valid(sub * kTile + tvB + 8) ? wD[w] : 0u;
+        }
+      }
+    };
 
     // ---- S^T = K * Qx^T per sub-tile: rows gid, gid + 8
     float x[NS][HS][2];
@@ -492,12 +507,14 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         // m-tile 4 gv + j are dims gv * G + gid * CH + j and + CH / 2
 #pragma unroll
         for (int gq = 0; gq < NG; ++gq) {
-          const uint8_t* vb = sV + sub * kTile * C::RB + gq * (GE * BITS / 8) + gid * VBG;
+          const uint8_t* vb =
+              sV + sub * kTile * C::RB + gq * (GE * code_bits(BITS) / 8) + gid * VBG;
           uint32_t wA[VWG], wB[VWG], wC[VWG], wD[VWG];
           load_chunk<VBG, VWG>(vb + tvA * C::RB, wA);
           load_chunk<VBG, VWG>(vb + tvB * C::RB, wB);
           load_chunk<VBG, VWG>(vb + (tvA + 8) * C::RB, wC);
           load_chunk<VBG, VWG>(vb + (tvB + 8) * C::RB, wD);
+          zero_invalid(sub, wA, wB, wC, wD);
           uint32_t xa[VWG * XP::kOut], xc[VWG * XP::kOut];
 #pragma unroll
           for (int w = 0; w < VWG; ++w) {
@@ -522,16 +539,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         load_chunk<C::VB, C::VW>(vb + tvB * C::RB, wB);
         load_chunk<C::VB, C::VW>(vb + (tvA + 8) * C::RB, wC);
         load_chunk<C::VB, C::VW>(vb + (tvB + 8) * C::RB, wD);
-        if constexpr (BITS == 16 && !FULL) {
-          // raw fp16 rows past the valid length may hold anything: zero them
-#pragma unroll
-          for (int w = 0; w < C::VW; ++w) {
-            wA[w] = valid(sub * kTile + tvA) ? wA[w] : 0u;
-            wB[w] = valid(sub * kTile + tvB) ? wB[w] : 0u;
-            wC[w] = valid(sub * kTile + tvA + 8) ? wC[w] : 0u;
-            wD[w] = valid(sub * kTile + tvB + 8) ? wD[w] : 0u;
-          }
-        }
+        zero_invalid(sub, wA, wB, wC, wD);
         uint32_t xa[16], xc[16];
 #pragma unroll
         for (int w = 0; w < C::VW; ++w) {
@@ -709,7 +717,9 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   X(8, 64, 1) X(8, 64, 2) X(8, 64, 4)                                  \
   X(4, 64, 1) X(4, 64, 2) X(4, 64, 4)                                  \
   X(2, 64, 1) X(2, 64, 2) X(2, 64, 4)                                  \
-  X(8, 32, 1) X(8, 32, 2) X(4, 32, 1) X(4, 32, 2) X(2, 32, 1) X(2, 32, 2)
+  X(8, 32, 1) X(8, 32, 2) X(4, 32, 1) X(4, 32, 2) X(2, 32, 1) X(2, 32, 2)                  \
+  X(kE4M3, 128, 1) X(kE4M3, 128, 2) X(kE4M3, 128, 4) X(kE4M3, 128, 8)  \
+  X(kE4M3, 64, 1) X(kE4M3, 64, 2) X(kE4M3, 64, 4) X(kE4M3, 32, 1) X(kE4M3, 32, 2)
 
 }  // namespace
 

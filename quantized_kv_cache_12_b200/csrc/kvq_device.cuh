@@ -7,6 +7,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "kvq_internal.h"
+
 namespace kvq {
 
 constexpr int kHeadDim = 128;  // head_dim supported by this build
@@ -200,6 +202,30 @@ struct WordPairs<16> {
   __device__ __forceinline__ static uint32_t one(uint32_t w, int) { return w; }
 };
 
+// Two E4M3 codes (low byte, high byte) to an fp16 pair (low half, high
+// half); exact, every E4M3 value being an fp16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t v16) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((uint16_t)v16));
+  return r;
+}
+
+// FP8 E4M3 word (dims 0..3): pair j = dims (2j, 2j + 1), the values
+// themselves (factor 1, like raw fp16).
+template <>
+struct WordPairs<kE4M3> {
+  static constexpr int kPairs = 2, kDims = 4, kEmax = 24;
+  __device__ __forceinline__ static void run(uint32_t w, uint32_t (&p)[2]) {
+    p[0] = e4m3x2_to_h2(w & 0xFFFFu);
+    p[1] = e4m3x2_to_h2(w >> 16);
+  }
+  __host__ __device__ static constexpr int dim(int j, int e) { return 2 * j + e; }
+  __host__ __device__ static constexpr int exp(int) { return 24; }
+  __device__ __forceinline__ static uint32_t one(uint32_t w, int j) {
+    return e4m3x2_to_h2(j ? (w >> 16) : (w & 0xFFFFu));
+  }
+};
+
 // Pairs across two tokens (V side): words a (token A) and b (token B) hold
 // the same dims; out[i] = half2(code_A[dim i], code_B[dim i]) for the dims of
 // the word in order, with the subnormal exponent exp(i).
@@ -255,6 +281,20 @@ struct CrossPairs<8> {
     o[3] = prmt(y, 0u, 0x4341u);
   }
   __host__ __device__ static constexpr int exp(int) { return 0; }
+};
+
+template <>
+struct CrossPairs<kE4M3> {
+  static constexpr int kOut = 4;
+  __device__ __forceinline__ static void run(uint32_t a, uint32_t b, uint32_t (&o)[4]) {
+    const uint32_t x = prmt(a, b, 0x5140u);  // [a.b0 b.b0 a.b1 b.b1]
+    const uint32_t y = prmt(a, b, 0x7362u);  // [a.b2 b.b2 a.b3 b.b3]
+    o[0] = e4m3x2_to_h2(x & 0xFFFFu);
+    o[1] = e4m3x2_to_h2(x >> 16);
+    o[2] = e4m3x2_to_h2(y & 0xFFFFu);
+    o[3] = e4m3x2_to_h2(y >> 16);
+  }
+  __host__ __device__ static constexpr int exp(int) { return 24; }
 };
 
 template <>

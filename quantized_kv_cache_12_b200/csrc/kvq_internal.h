@@ -10,6 +10,11 @@
 
 namespace kvq {
 
+// Kernel template tag of the FP8 E4M3 code format (8-bit codes); the integer
+// formats use their bit width (2, 4, 8) and raw fp16 rows use 16.
+constexpr int kE4M3 = 0x108;
+__host__ __device__ constexpr int code_bits(int tag) { return tag & 0xFF; }
+
 // One K/V plane pair of one cache segment, as the kernels see it.
 struct SegView {
   const uint8_t* k_codes;

@@ -31,7 +31,7 @@ __device__ __forceinline__ RowRef locate_row(const QuantArgs& a, long long r, in
   const long long rr = is_v ? r - per : r;
   const int t = (int)(rr % a.n_new);
   const long long bh = rr / a.n_new;  // b * kv_heads + h
-  constexpr int RB = kHeadDim * BITS / 8;
+  constexpr int RB = kHeadDim * code_bits(BITS) / 8;
   constexpr int MB = (kHeadDim / G) * 4;
   const int pos = base_pos + t;
   RowRef ref;
@@ -127,6 +127,7 @@ cudaError_t launch_quantize(const QuantArgs& a, int bits, int group, cudaStream_
   KVQ_Q(8, 32) KVQ_Q(8, 64) KVQ_Q(8, 128)
   KVQ_Q(4, 32) KVQ_Q(4, 64) KVQ_Q(4, 128)
   KVQ_Q(2, 32) KVQ_Q(2, 64) KVQ_Q(2, 128)
+  KVQ_Q(kE4M3, 32) KVQ_Q(kE4M3, 64) KVQ_Q(kE4M3, 128)
 #undef KVQ_Q
   return cudaErrorInvalidValue;
 }

@@ -24,6 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libkvq.so")
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, \
     KVQ_ERR_CUDA = range(6)
 KVQ_F16, KVQ_BF16 = 0, 1
+KVQ_FMT_INT, KVQ_FMT_FP8_E4M3 = 0, 1
 HEADER_BYTES = 256  # workspace header: sticky device error word first
 
 
@@ -35,7 +36,7 @@ class KvqError(RuntimeError):
 
 class kvq_plane(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32),
-                ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p)]
+                ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("fmt", ctypes.c_int32)]
 
 
 class kvq_cache(ctypes.Structure):
@@ -247,7 +248,8 @@ class QuantizedKVCache:
 
     codes: uint8 [B, H_kv, max_tokens, head_dim*bits/8];
     meta: fp16 [B, H_kv, max_tokens, head_dim/G, 2] (scale, zero), None for bits 16;
-    seq_lens: int32 [B] on the device.
+    seq_lens: int32 [B] on the device; fmt: KVQ_FMT_INT, or KVQ_FMT_FP8_E4M3
+    (bits 8: E4M3 codes, zero points 0).
     """
     batch: int
     kv_heads: int
@@ -260,9 +262,11 @@ class QuantizedKVCache:
     k_meta: Optional[torch.Tensor]
     v_meta: Optional[torch.Tensor]
     seq_lens: torch.Tensor
+    fmt: int = KVQ_FMT_INT
 
     @classmethod
-    def allocate(cls, batch, kv_heads, head_dim, max_tokens, bits, group_size, device="cuda"):
+    def allocate(cls, batch, kv_heads, head_dim, max_tokens, bits, group_size, device="cuda",
+                 fmt: int = KVQ_FMT_INT):
         rb = head_dim * bits // 8
         shape = (batch, kv_heads, max_tokens, rb)
         k = torch.empty(shape, dtype=torch.uint8, device=device)
@@ -273,16 +277,17 @@ class QuantizedKVCache:
             km = torch.empty(mshape, dtype=torch.float16, device=device)
             vm = torch.empty(mshape, dtype=torch.float16, device=device)
         lens = torch.zeros(batch, dtype=torch.int32, device=device)
-        return cls(batch, kv_heads, head_dim, max_tokens, bits, group_size, k, v, km, vm, lens)
+        return cls(batch, kv_heads, head_dim, max_tokens, bits, group_size, k, v, km, vm, lens,
+                   fmt)
 
     def struct(self) -> kvq_cache:
         c = kvq_cache()
         c.batch, c.kv_heads, c.head_dim, c.max_tokens = (self.batch, self.kv_heads,
                                                          self.head_dim, self.max_tokens)
         c.k = kvq_plane(self.bits, self.group_size, self.k_codes.data_ptr(),
-                        self.k_meta.data_ptr() if self.k_meta is not None else None)
+                        self.k_meta.data_ptr() if self.k_meta is not None else None, self.fmt)
         c.v = kvq_plane(self.bits, self.group_size, self.v_codes.data_ptr(),
-                        self.v_meta.data_ptr() if self.v_meta is not None else None)
+                        self.v_meta.data_ptr() if self.v_meta is not None else None, self.fmt)
         c.seq_lens = self.seq_lens.data_ptr()
         return c
 

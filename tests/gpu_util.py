@@ -35,16 +35,16 @@ def fill_fp16_segment(cache, k: torch.Tensor, v: torch.Tensor, lens):
     cache.seq_lens.copy_(torch.as_tensor(np.asarray(lens, np.int32), device=cache.seq_lens.device))
 
 
-def oracle_segment(k: torch.Tensor, v: torch.Tensor, bits: int, group: int):
-    """The oracle's own packed cache of the same fp16 inputs."""
+def oracle_segment(k: torch.Tensor, v: torch.Tensor, bits: int, group: int, fmt: str = "int"):
+    """The oracle's own packed cache of the same fp16 inputs (fmt "fp8": E4M3)."""
     k16, v16 = f16_bits(k), f16_bits(v)
     if bits == 16:
         kc = k16.view(np.uint8).reshape(*k16.shape[:3], -1)
         vc = v16.view(np.uint8).reshape(*v16.shape[:3], -1)
         return dict(k_codes=kc, v_codes=vc, k_meta=None, v_meta=None, bits=16, group=128)
-    kc, km = oracle.quantize_cache(k16, group, bits)
-    vc, vm = oracle.quantize_cache(v16, group, bits)
-    return dict(k_codes=kc, v_codes=vc, k_meta=km, v_meta=vm, bits=bits, group=group)
+    kc, km = oracle.quantize_cache(k16, group, bits, fmt)
+    vc, vm = oracle.quantize_cache(v16, group, bits, fmt)
+    return dict(k_codes=kc, v_codes=vc, k_meta=km, v_meta=vm, bits=bits, group=group, fmt=fmt)
 
 
 def assert_close(out: torch.Tensor, ref: np.ndarray, lse=None, lse_ref=None, mask=None,

@@ -191,6 +191,28 @@ def test_decode_step_rejects_bad_arguments(kvq):
     assert st == kvq.KVQ_ERR_UNSUPPORTED  # raw fp16 caches take no quantized append
 
 
+def test_fp8_planes_validated(kvq):
+    """KVQ_FMT_FP8_E4M3 needs bits 8 and the same format on K and V; unknown
+    formats are rejected; FP8 decode is built for (head_dim / G) * g <= 8."""
+    fake = ctypes.c_void_p(0x60000)
+
+    def append_status(c):
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, 1, 1, None)
+    c = _fake_cache(kvq, bits=4)
+    c.k.fmt = c.v.fmt = kvq.KVQ_FMT_FP8_E4M3
+    assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
+    c = _fake_cache(kvq, bits=8)
+    c.k.fmt = c.v.fmt = 7
+    assert append_status(c) == kvq.KVQ_ERR_INVALID_ARG
+    c = _fake_cache(kvq, bits=8)
+    c.k.fmt = kvq.KVQ_FMT_FP8_E4M3
+    assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
+    c = _fake_cache(kvq, bits=8, group=64, kv_heads=2)
+    c.k.fmt = c.v.fmt = kvq.KVQ_FMT_FP8_E4M3
+    assert kvq.kvq_decode_workspace_bytes(c, 8) > 0   # g = 4: tokens-on-M kernel
+    assert _status(kvq.kvq_decode_workspace_bytes, c, 16) == kvq.KVQ_ERR_UNSUPPORTED  # g = 8
+
+
 def test_chunk_entry_points_reject_bad_arguments(kvq):
     lib = kvq.lib
     fake = ctypes.c_void_p(0x10000)

@@ -68,6 +68,7 @@ class DecodeWorkload:
     alpha: float = 0.0
     beta: float = 0.0
     low_bits: Tuple[int, ...] = ()   # bit-widths of the two quantized classes
+    fmt: str = "int"          # code format: "int" (asymmetric integer) or "fp8" (E4M3, bits 8)
 
     @property
     def group_ratio(self) -> int:
@@ -102,6 +103,16 @@ WORKLOADS = {
         context=32768, bits=4, group=32, q_dtype="f16", steps=100, append=False, seed=4,
         chunk_tokens=32, emb_dim=768, query_pool=20, query_noise=0.1, alpha=0.6, beta=0.1,
         low_bits=(4, 2)),
+    # the FP8 E4M3 variant of the KV-cache page, on the Llama-2 and Llama-3 shapes
+    "llama2_7b_mha_fp8": DecodeWorkload(
+        name="llama2_7b_mha_fp8", batch=16, q_heads=32, kv_heads=32, head_dim=128,
+        context=4096, bits=8, group=128, q_dtype="bf16", steps=100, append=True, seed=2,
+        k_outliers=Outliers(factor=10.0, fraction=0.01),
+        v_outliers=Outliers(factor=10.0, fraction=0.01), fmt="fp8"),
+    "llama3_8b_gqa_fp8": DecodeWorkload(
+        name="llama3_8b_gqa_fp8", batch=32, q_heads=32, kv_heads=8, head_dim=128,
+        context=8192, bits=8, group=64, q_dtype="f16", steps=100, append=True, seed=3,
+        k_outliers=Outliers(factor=15.0, per_head=4), v_sigma=0.5, fmt="fp8"),
     "long_gqa_int4": DecodeWorkload(
         name="long_gqa_int4", batch=1, q_heads=32, kv_heads=8, head_dim=128,
         context=131072, bits=4, group=64, q_dtype="f16", steps=256, append=True, seed=5,
