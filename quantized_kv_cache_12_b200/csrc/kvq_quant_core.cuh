@@ -9,20 +9,20 @@
 //   code = clamp(rint(x / s) + z, 0, qmax).
 // Every step is one IEEE fp32 operation with round-to-nearest-even (explicit
 // intrinsics, so no contraction can change a result), which makes codes,
-// scales and zero points reproducible bit for bit.
+// scales and zero points reproducible bit for bit.  The per-element division
+// by s is a correction step on a product with RN(1/s) that returns the IEEE
+// quotient exactly (div_rn below), and the rounding and clamping of the code
+// use an equivalent order that needs no conversion instruction.
 #pragma once
 
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "kvq_device.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
 
-// One thread holds 8 consecutive fp16 values of a token row; the G/8
-// threads of a group are consecutive lanes (groups never straddle a row).
-// Returns the packed codes of the 8 values (BITS bits each, element j at
-// bit offset BITS*j) and the (scale, zero) half2 of the group.
 // Two fp32 values to E4M3 codes, each rounded to the nearest E4M3 value
 // (ties to even) and saturated at +-448; `lo` goes to the low byte.
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
@@ -31,81 +31,175 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return r;
 }
 
-template <int BITS, int G>
-__device__ __forceinline__ void quantize8(const uint4 raw, uint32_t& codes_lo,
-                                          uint32_t& codes_hi, uint32_t& meta) {
-  static_assert(G % 8 == 0 && G >= 16 && G <= 256, "group size");
-  const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-  float x[8];
+// x / d rounded to nearest-even fp32 (the IEEE quotient), given r = RN(1/d):
+// q0 = RN(x r) approximates x / d within one ulp, the remainder x - q0 d is
+// exact in one fma, and RN(q0 + (x - q0 d) r) is the correctly rounded
+// quotient (Markstein's theorem: P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990).  Used with fp16-valued x and d, where no step under- or overflows;
+// the identity with IEEE division holds for every pair of 11-bit
+// significands, which covers every fp16 x and d up to a power of two.  A zero
+// quotient comes out +0 whatever the sign of x.
+__device__ __forceinline__ float div_rn(float x, float d, float r) {
+  const float q0 = __fmul_rn(x, r);
+  const float e = __fmaf_rn(-q0, d, x);
+  return __fmaf_rn(e, r, q0);
+}
+
+// Packed code words of NV values of a BITS-bit format (at least one word).
+template <int BITS, int NV>
+__host__ __device__ constexpr int code_words() {
+  return (NV * code_bits(BITS) + 31) / 32;
+}
+
+// Pack codes held in the low CB bits of u[] (the bits above them may hold
+// anything) into words, element j at bit offset CB * j.
+template <int CB, int NV>
+__device__ __forceinline__ void pack_codes(const uint32_t (&u)[NV], uint32_t* w) {
+  if constexpr (CB == 8) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __half22float2(h2[i]);
+    for (int i = 0; i < NV / 4; ++i)
+      w[i] = __byte_perm(__byte_perm(u[4 * i], u[4 * i + 1], 0x0040),
+                         __byte_perm(u[4 * i + 2], u[4 * i + 3], 0x0040), 0x5410);
+  } else if constexpr (CB == 4) {
+    // four codes as bytes, then each byte pair folded into one byte
+#pragma unroll
+    for (int i = 0; i < NV / 8; ++i) {
+      uint32_t t[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int o = 8 * i + 4 * h;
+        const uint32_t b = __byte_perm(__byte_perm(u[o], u[o + 1], 0x0040),
+                                       __byte_perm(u[o + 2], u[o + 3], 0x0040), 0x5410) &
+                           0x0F0F0F0Fu;
+        t[h] = b | (b >> 4);  // bytes 0 and 2 hold code pairs
+      }
+      w[i] = __byte_perm(t[0], t[1], 0x6420);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < code_words<CB, NV>(); ++i) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int j = 0; j < 16 && 16 * i + j < NV; ++j) x |= (u[16 * i + j] & 3u) << (2 * j);
+      w[i] = x;
+    }
+  }
+}
+
+// One thread holds NV (8 or 16) consecutive fp16 values of a token row; the
+// G / NV threads of a group are consecutive lanes (groups never straddle a
+// row).  Produces the packed codes of the NV values (BITS bits each, element
+// j at bit offset BITS * j) and the (scale, zero) half2 of the group.
+template <int BITS, int G, int NV>
+__device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
+                                              uint32_t (&codes)[code_words<BITS, NV>()],
+                                              uint32_t& meta) {
+  static_assert(NV == 8 || NV == 16, "values per thread");
+  static_assert(G % NV == 0 && G / NV <= 32 && G <= kHeadDim, "group size");
+  constexpr int NH = NV / 2;
+  constexpr int GL = G / NV;  // lanes per group
+  const __half2* h2 = reinterpret_cast<const __half2*>(&raw[0]);
+  float x[NV];
+#pragma unroll
+  for (int i = 0; i < NH; ++i) {
+    const float2 f = __half22float2(h2[i]);
     x[2 * i] = f.x;
     x[2 * i + 1] = f.y;
   }
   if constexpr (BITS == kE4M3) {
     // FP8 E4M3 (the KV-cache page's FP8 KV cache, dynamic scale): s = max(
     // amax / 448, 1e-5) stored in fp16 rounded up, so |x / s| <= 448;
-    // code = E4M3 of the fp32 quotient x / s; zero point 0.
-    float amax = 0.f;
+    // code = E4M3 of the fp32 quotient x / s; zero point 0.  The group's
+    // |max| is taken on the fp16 values (exact).
+    __half2 am = __habs2(h2[0]);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    for (int i = 1; i < NH; ++i) am = __hmax2(am, __habs2(h2[i]));
+    am = __hmax2(am, __lowhigh2highlow(am));
 #pragma unroll
-    for (int off = 1; off < G / 8; off <<= 1)
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    float s32 = __fdiv_rn(amax, 448.0f);
-    s32 = fmaxf(s32, 1e-5f);
+    for (int off = 1; off < GL; off <<= 1)
+      am = __hmax2(am, u32_as_h2(__shfl_xor_sync(0xffffffffu, h2_as_u32(am), off)));
+    constexpr float kInv448 = 1.0f / 448.0f;
+    const float s32 = fmaxf(div_rn(__low2float(am), 448.0f, kInv448), 1e-5f);
     const __half s16 = __float2half_ru(s32);
     const float s = __half2float(s16);
-    uint32_t c[4];
+    const float r = __frcp_rn(s);
+    uint32_t c[NH];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) c[i] = e4m3x2(__fdiv_rn(x[2 * i], s), __fdiv_rn(x[2 * i + 1], s));
-    codes_lo = c[0] | (c[1] << 16);
-    codes_hi = c[2] | (c[3] << 16);
-    const __half2 sz = __halves2half2(s16, __float2half_rn(0.f));
-    meta = *reinterpret_cast<const uint32_t*>(&sz);
+    for (int i = 0; i < NH; ++i)
+      c[i] = e4m3x2(copysignf(div_rn(x[2 * i], s, r), x[2 * i]),
+                    copysignf(div_rn(x[2 * i + 1], s, r), x[2 * i + 1]));
+#pragma unroll
+    for (int i = 0; i < NH / 2; ++i) codes[i] = __byte_perm(c[2 * i], c[2 * i + 1], 0x5410);
+    meta = h2_as_u32(__halves2half2(s16, __float2half_rn(0.f)));
   } else {
-    float mn = x[0], mx = x[0];
+    // group (min, -max) as one fp16 pair: one shuffle and one min per step
+    __half2 lo2 = h2[0], hi2 = h2[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) {
-      mn = fminf(mn, x[i]);
-      mx = fmaxf(mx, x[i]);
+    for (int i = 1; i < NH; ++i) {
+      lo2 = __hmin2(lo2, h2[i]);
+      hi2 = __hmax2(hi2, h2[i]);
     }
+    __half2 mm = __halves2half2(__hmin(__low2half(lo2), __high2half(lo2)),
+                                __hneg(__hmax(__low2half(hi2), __high2half(hi2))));
 #pragma unroll
-    for (int off = 1; off < G / 8; off <<= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    }
-    constexpr float qmax = float((1 << code_bits(BITS)) - 1);
-    float s32 = __fdiv_rn(__fsub_rn(mx, mn), qmax);
-    s32 = fmaxf(s32, 1e-5f);
+    for (int off = 1; off < GL; off <<= 1)
+      mm = __hmin2(mm, u32_as_h2(__shfl_xor_sync(0xffffffffu, h2_as_u32(mm), off)));
+    const float mn = __low2float(mm), mx = -__high2float(mm);
+    constexpr int qmax_i = (1 << code_bits(BITS)) - 1;
+    constexpr float qmax = float(qmax_i);
+    constexpr float kInvQmax = 1.0f / qmax;
+    const float s32 = fmaxf(div_rn(__fsub_rn(mx, mn), qmax, kInvQmax), 1e-5f);
     const __half s16 = __float2half_ru(s32);
     const float s = __half2float(s16);
-    float zf = __fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.0f);
+    const float r = __frcp_rn(s);
+    float zf = __fadd_rn(rintf(div_rn(-mn, s, r)), 0.0f);
     zf = fminf(fmaxf(zf, -65504.0f), 65504.0f);
     const __half z16 = __float2half_rn(zf);
-    const float z = __half2float(z16);
-
-    uint32_t c[8];
+    const float z = __half2float(z16);  // an integer
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds |v| < 2^22 to an integer
+    uint32_t u[NV];
+    // code = clamp(rint(x / s) + z, 0, qmax).
+    if (__all_sync(0xffffffffu, fabsf(zf) <= 2048.0f)) {
+      // z is exact in fp16 and equals -rint(RN(mn / s)) (rounding and rint
+      // are monotone and odd-symmetric), so every code of the group is >= 0
+      // and every quotient lies within 2048 + qmax + 2 of zero: only the
+      // upper clamp is needed, on rint(q) + 1.5 * 2^23 + z, whose low
+      // mantissa bits then hold the code.
+      constexpr float kTop = kMagic + qmax;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float v = __fadd_rn(rintf(__fdiv_rn(x[i], s)), z);
-      v = fminf(fmaxf(v, 0.0f), qmax);
-      c[i] = static_cast<uint32_t>(v);
-    }
-    if (code_bits(BITS) == 8) {
-      codes_lo = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-      codes_hi = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+      for (int i = 0; i < NV; ++i) {
+        const float a = __fadd_rn(__fadd_rn(div_rn(x[i], s, r), kMagic), z);
+        u[i] = __float_as_uint(fminf(a, kTop));
+      }
     } else {
-      uint32_t w = 0;
+      // Clamping the quotient to [-z, qmax - z] first gives the same code (z
+      // is an integer: a quotient below -z rounds to at most -z, one above
+      // qmax - z to at least qmax - z) and bounds it well inside +-2^22.
+      const float lo = -z, hi = __fadd_rn(qmax, -z);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) w |= c[i] << (code_bits(BITS) * i);
-      codes_lo = w;
-      codes_hi = 0;
+      for (int i = 0; i < NV; ++i) {
+        const float q = fminf(fmaxf(div_rn(x[i], s, r), lo), hi);
+        u[i] = __float_as_uint(__fadd_rn(__fadd_rn(q, kMagic), z));
+      }
     }
-    const __half2 sz = __halves2half2(s16, z16);
-    meta = *reinterpret_cast<const uint32_t*>(&sz);
+    pack_codes<code_bits(BITS), NV>(u, codes);
+    meta = h2_as_u32(__halves2half2(s16, z16));
   }
+}
+
+// quantize_vals for 8 values per thread: codes in (codes_lo, codes_hi).
+template <int BITS, int G>
+__device__ __forceinline__ void quantize8(const uint4 raw, uint32_t& codes_lo,
+                                          uint32_t& codes_hi, uint32_t& meta) {
+  const uint4 r[1] = {raw};
+  uint32_t w[code_words<BITS, 8>()];
+  quantize_vals<BITS, G, 8>(r, w, meta);
+  codes_lo = w[0];
+  if constexpr (code_words<BITS, 8>() > 1)
+    codes_hi = w[1];
+  else
+    codes_hi = 0;
 }
 
 // Quantize one 16-byte slice of a row and store it.  lane16 = index of the

@@ -70,24 +70,95 @@ __global__ void __launch_bounds__(1024) quantize_append_kernel(const QuantArgs a
   }
 }
 
-// Bulk quantize (prefill): grid-stride over all rows.  Reads each thread's
-// sequence length once per row; lengths are advanced by a separate kernel.
+// Bulk quantize (prefill).  Work unit: kUnitRows consecutive tokens of one
+// (side, sequence, KV head) plane row, whose fp16 rows are contiguous in the
+// input and whose codes and (s, z) are contiguous in the cache.  A warp takes
+// units round-robin, four rows per step (8 lanes x 32 bytes per row, 16
+// values per lane), and loads the next unit's rows before it quantizes the
+// current one, so every lane keeps 64 bytes of reads in flight.
+constexpr int kUnitRows = 8;
+constexpr int kBulkNV = 16;                           // values per lane
+constexpr int kBulkLanes = kHeadDim / kBulkNV;        // lanes per row
+constexpr int kBulkRowsPerStep = 32 / kBulkLanes;     // rows per warp step
+constexpr int kBulkSteps = kUnitRows / kBulkRowsPerStep;
+
+struct BulkUnit {
+  uint4 raw[kBulkSteps][kBulkNV / 8];
+  long long dst_row;  // cache row of position 0 of the unit's plane row
+  int t0, base, is_v;
+};
+
+__device__ __forceinline__ void bulk_fetch(const QuantArgs& a, int u, int units_per_row, int li,
+                                           int ri, BulkUnit& w) {
+  const int planes = a.batch * a.kv_heads;
+  const int p = u / units_per_row;
+  const int j = u - p * units_per_row;
+  const bool is_v = p >= planes;
+  const int bh = is_v ? p - planes : p;
+  w.t0 = j * kUnitRows;
+  w.base = a.seq_lens[bh / a.kv_heads];
+  w.dst_row = (long long)bh * a.max_tokens;
+  w.is_v = is_v;
+  const uint4* src = reinterpret_cast<const uint4*>(
+      (is_v ? a.v_new : a.k_new) + ((long long)bh * a.n_new + w.t0) * kHeadDim);
+#pragma unroll
+  for (int k = 0; k < kBulkSteps; ++k) {
+    const int row = kBulkRowsPerStep * k + ri;
+    const bool in = w.t0 + row < a.n_new;
+#pragma unroll
+    for (int c = 0; c < kBulkNV / 8; ++c)
+      w.raw[k][c] = in ? __ldcs(src + row * (kHeadDim / 8) + li * (kBulkNV / 8) + c)
+                       : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 template <int BITS, int G>
-__global__ void __launch_bounds__(256) quantize_bulk_kernel(const QuantArgs a) {
-  const long long rows = 2LL * a.batch * a.kv_heads * a.n_new;
-  const int lane16 = threadIdx.x & 15;
-  const long long rows_per_step = (long long)gridDim.x * (blockDim.x / 16);
-  const long long first = (long long)blockIdx.x * (blockDim.x / 16) + (threadIdx.x >> 4);
-  // trip count is uniform across the warp (both half-warps take the same steps)
-  const long long warp_first = first & ~1LL;
-  for (long long r = first; warp_first + (r - first) < rows; r += rows_per_step) {
-    const bool in = r < rows;
-    const long long rs = in ? r : 0;
-    const long long per = (long long)a.batch * a.kv_heads * a.n_new;
-    const long long rr = rs >= per ? rs - per : rs;
-    const int b = (int)(rr / ((long long)a.kv_heads * a.n_new));
-    RowRef ref = locate_row<BITS, G>(a, rs, a.seq_lens[b]);
-    quantize_slice<BITS, G>(ref.src, ref.codes, ref.meta, lane16, in && ref.active);
+__device__ __forceinline__ void bulk_work(const QuantArgs& a, int li, int ri, const BulkUnit& w) {
+  constexpr int RB = kHeadDim * code_bits(BITS) / 8;
+  constexpr int MB = (kHeadDim / G) * 4;
+  constexpr int NW = code_words<BITS, kBulkNV>();
+  uint8_t* codes = w.is_v ? a.v_codes : a.k_codes;
+  uint8_t* meta = w.is_v ? a.v_meta : a.k_meta;
+#pragma unroll
+  for (int k = 0; k < kBulkSteps; ++k) {
+    const int t = w.t0 + kBulkRowsPerStep * k + ri;
+    const int pos = w.base + t;
+    uint32_t cw[NW], m;
+    quantize_vals<BITS, G, kBulkNV>(w.raw[k], cw, m);
+    if (t < a.n_new && pos < a.max_tokens) {
+      const long long row = w.dst_row + pos;
+      uint8_t* cr = codes + row * RB;
+      if constexpr (NW == 4) {
+        reinterpret_cast<uint4*>(cr)[li] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      } else if constexpr (NW == 2) {
+        reinterpret_cast<uint2*>(cr)[li] = make_uint2(cw[0], cw[1]);
+      } else {
+        reinterpret_cast<uint32_t*>(cr)[li] = cw[0];
+      }
+      constexpr int GL = G / kBulkNV;  // lanes per group
+      if ((li % GL) == 0) reinterpret_cast<uint32_t*>(meta + row * MB)[li / GL] = m;
+    }
+  }
+}
+
+template <int BITS, int G>
+__global__ void __launch_bounds__(256) quantize_bulk_kernel(const QuantArgs a, int units_per_row,
+                                                            int n_units) {
+  const int lane = threadIdx.x & 31;
+  const int li = lane % kBulkLanes, ri = lane / kBulkLanes;
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  int u = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // uniform across the warp
+  BulkUnit A, B;
+  if (u < n_units) bulk_fetch(a, u, units_per_row, li, ri, A);
+  while (u < n_units) {
+    const int u1 = u + nw;
+    if (u1 < n_units) bulk_fetch(a, u1, units_per_row, li, ri, B);
+    bulk_work<BITS, G>(a, li, ri, A);
+    if (u1 >= n_units) break;
+    const int u2 = u1 + nw;
+    if (u2 < n_units) bulk_fetch(a, u2, units_per_row, li, ri, A);
+    bulk_work<BITS, G>(a, li, ri, B);
+    u = u2;
   }
 }
 
@@ -107,11 +178,23 @@ cudaError_t launch_q(const QuantArgs& a, cudaStream_t s) {
     quantize_append_kernel<BITS, G><<<a.batch, threads, 0, s>>>(a);
     return cudaGetLastError();
   }
-  const long long rows = (long long)a.batch * rows_per_seq;
-  long long blocks = (rows + 15) / 16;
-  const long long cap = 148LL * 8;  // 8 resident 256-thread CTAs per SM
-  if (blocks > cap) blocks = cap;
-  quantize_bulk_kernel<BITS, G><<<(unsigned)blocks, 256, 0, s>>>(a);
+  const int units_per_row = (a.n_new + kUnitRows - 1) / kUnitRows;
+  const long long n_units = 2LL * a.batch * a.kv_heads * units_per_row;
+  if (n_units > 0x7fffffffLL) return cudaErrorInvalidValue;
+  static int slots = 0;  // resident 256-thread CTAs on the device
+  if (slots == 0) {
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_bulk_kernel<BITS, G>,
+                                                        256, 0);
+    if (e != cudaSuccess) return e;
+    slots = sms * (per_sm > 0 ? per_sm : 1);
+  }
+  long long blocks = (n_units + 7) / 8;
+  if (blocks > slots) blocks = slots;
+  quantize_bulk_kernel<BITS, G><<<(unsigned)blocks, 256, 0, s>>>(a, units_per_row, (int)n_units);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !a.advance) return e;
   advance_seq_lens_kernel<<<(a.batch + 127) / 128, 128, 0, s>>>(a.seq_lens, a.batch, a.n_new,

@@ -163,3 +163,80 @@ def test_prefill_full_size_long_context_sampled(kvq):
         ec, em = oracle.quantize_rows(x, 64, 4)
         assert np.array_equal(codes[0, h, t].cpu().numpy(), ec)
         assert np.array_equal(_meta_bits(meta[0, h, t]), em)
+
+
+# ---- the bulk (prefill) kernel: more than 512 rows per sequence
+
+
+def _alloc_fmt(kvq, B, H, max_tokens, bits, G, fmt):
+    f = kvq.KVQ_FMT_FP8_E4M3 if fmt == "fp8" else kvq.KVQ_FMT_INT
+    c = kvq.QuantizedKVCache.allocate(B, H, 128, max_tokens, bits, G, DEV, fmt=f)
+    c.k_codes.fill_(0xA5)
+    c.v_codes.fill_(0x5A)
+    c.k_meta.view(torch.int16).fill_(-1)
+    c.v_meta.view(torch.int16).fill_(-1)
+    return c
+
+
+BULK_FORMATS = [(b, G, "int") for b in (2, 4, 8) for G in (32, 64, 128)] + \
+               [(8, G, "fp8") for G in (32, 64, 128)]
+
+
+@pytest.mark.parametrize("bits,G,fmt", BULK_FORMATS)
+def test_bulk_kernel_ragged_starts_and_capacity(kvq, bits, G, fmt):
+    """77 tokens per (sequence, KV head) over 4 heads (616 rows per
+    sequence: the bulk kernel), appended at start positions 0, 3 and 60 of a
+    128-token cache: the third sequence's last 9 tokens fall past capacity
+    and are dropped; every written row equals the oracle's, every other slot
+    keeps its bytes."""
+    B, H, T, cap = 3, 4, 77, 128
+    wl = workloads.WORKLOADS["llama3_8b_gqa_int4"].scaled(batch=B, kv_heads=H, q_heads=H)
+    k, v = workloads.kv_tokens(wl, T, DEV)
+    c = _alloc_fmt(kvq, B, H, cap, bits, G, fmt)
+    start = [0, 3, 60]
+    c.seq_lens.copy_(torch.tensor(start, dtype=torch.int32))
+    kvq.kvq_quantize_append(c, k, v, T, advance_seq_lens=True)
+    assert c.seq_lens.tolist() == [min(s + T, cap) for s in start]
+    kc, km = oracle.quantize_cache(f16_bits(k), G, bits, fmt)
+    vc, vm = oracle.quantize_cache(f16_bits(v), G, bits, fmt)
+    for b in range(B):
+        n = min(T, cap - start[b])
+        p = slice(start[b], start[b] + n)
+        assert np.array_equal(c.k_codes[b, :, p].cpu().numpy(), kc[b, :, :n])
+        assert np.array_equal(c.v_codes[b, :, p].cpu().numpy(), vc[b, :, :n])
+        assert np.array_equal(_meta_bits(c.k_meta[b, :, p]), km[b, :, :n])
+        assert np.array_equal(_meta_bits(c.v_meta[b, :, p]), vm[b, :, :n])
+        assert (c.k_codes[b, :, :start[b]] == 0xA5).all()
+        assert (c.v_codes[b, :, start[b] + n:] == 0x5A).all()
+        assert (c.k_meta[b, :, start[b] + n:].view(torch.int16) == -1).all()
+
+
+@pytest.mark.parametrize("bits,G,fmt", [(8, 128, "int"), (4, 64, "int"), (2, 32, "int"),
+                                        (4, 128, "int"), (8, 64, "fp8")])
+def test_bulk_kernel_scale_sweep_and_adversarial(kvq, bits, G, fmt):
+    """Groups whose magnitudes sweep the fp16 range (2^-24 .. 2^15, so the
+    scale runs from its 1e-5 floor to above 100), offsets that push the zero
+    point to its clamp, and the hand-picked adversarial rows, all through the
+    bulk kernel; codes, scales and zero points byte for byte."""
+    rng = np.random.default_rng(7)
+    rows = []
+    for e in range(-24, 16):
+        for off in (0.0, 3.0, -40.0):
+            x = rng.standard_normal(128) * 2.0 ** e + off * 2.0 ** max(e, 0)
+            rows.append(np.clip(x, -65504, 65504).astype(np.float16))
+    rows = np.concatenate([np.stack(rows), _adversarial_rows()])
+    n = rows.shape[0]  # rows per head: 4 heads x 2 sides x n > 512 rows per sequence
+    H = 4
+    k = torch.from_numpy(np.stack([rows] * H)).to(DEV).view(1, H, n, 128).contiguous()
+    v = torch.from_numpy(np.stack([rows[::-1]] * H)).to(DEV).view(1, H, n, 128).contiguous()
+    k[0, 1] = -k[0, 1]
+    c = _alloc_fmt(kvq, 1, H, 192, bits, G, fmt)
+    c.seq_lens.zero_()
+    kvq.kvq_quantize_append(c, k, v, n, advance_seq_lens=True)
+    assert torch.isfinite(k.float()).all()
+    kc, km = oracle.quantize_cache(f16_bits(k), G, bits, fmt)
+    vc, vm = oracle.quantize_cache(f16_bits(v), G, bits, fmt)
+    assert np.array_equal(c.k_codes[:, :, :n].cpu().numpy(), kc)
+    assert np.array_equal(_meta_bits(c.k_meta[:, :, :n]), km)
+    assert np.array_equal(c.v_codes[:, :, :n].cpu().numpy(), vc)
+    assert np.array_equal(_meta_bits(c.v_meta[:, :, :n]), vm)
