@@ -46,48 +46,59 @@ __device__ __forceinline__ float div_rn(float x, float d, float r) {
   return __fmaf_rn(e, r, q0);
 }
 
+// div_rn on two values at once: x2 = (x0, x1), nd2 = (-d, -d), r2 = (r, r)
+// (q0 * -d + x is the same fma as -q0 * d + x).
+__device__ __forceinline__ uint64_t div_rn2(uint64_t x2, uint64_t nd2, uint64_t r2) {
+  const uint64_t q0 = f2_mul(x2, r2);
+  const uint64_t e = f2_fma(q0, nd2, x2);
+  return f2_fma(e, r2, q0);
+}
+
 // Packed code words of NV values of a BITS-bit format (at least one word).
 template <int BITS, int NV>
 __host__ __device__ constexpr int code_words() {
   return (NV * code_bits(BITS) + 31) / 32;
 }
 
-// Pack codes held in the low CB bits of u[] (the bits above them may hold
-// anything) into words, element j at bit offset CB * j.
+// Pack codes into words, element j at bit offset CB * j.  t[i] holds the
+// codes of elements i (low lane) and i + NV / 2 (high lane) as fp32 integers
+// in [0, 2^CB).  Adjacent registers are merged lane by lane, c_even +
+// 2^(width) * c_odd, an exact fp32 fma while values stay below 2^24, until a
+// lane holds 16 bits of codes (8 for 8 values of 2 bits); adding 1.5 * 2^23
+// then puts them in the low mantissa bits, and byte permutes assemble the
+// words.
 template <int CB, int NV>
-__device__ __forceinline__ void pack_codes(const uint32_t (&u)[NV], uint32_t* w) {
-  if constexpr (CB == 8) {
+__device__ __forceinline__ void pack_codes(uint64_t (&t)[NV / 2], uint32_t* w) {
+  constexpr int NH = NV / 2;
+  constexpr int L = (16 / CB < NH) ? 16 / CB : NH;  // codes per lane chunk
+  constexpr int LEVELS = L == 1 ? 0 : L == 2 ? 1 : L == 4 ? 2 : 3;
+  constexpr int N = NH / L;                          // chunk registers
 #pragma unroll
-    for (int i = 0; i < NV / 4; ++i)
-      w[i] = __byte_perm(__byte_perm(u[4 * i], u[4 * i + 1], 0x0040),
-                         __byte_perm(u[4 * i + 2], u[4 * i + 3], 0x0040), 0x5410);
-  } else if constexpr (CB == 4) {
-    // four codes as bytes, then each byte pair folded into one byte
+  for (int lev = 0; lev < LEVELS; ++lev) {
+    const float mult = float(1u << (CB << lev));
+    const uint64_t m = f2_pack(mult, mult);
 #pragma unroll
-    for (int i = 0; i < NV / 8; ++i) {
-      uint32_t t[2];
+    for (int j = 0; j < (NH >> (lev + 1)); ++j) t[j] = f2_fma(t[2 * j + 1], m, t[2 * j]);
+  }
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t m2 = f2_pack(kMagic, kMagic);
+  uint32_t c[2 * N];  // chunks in element order: the low lanes, then the high lanes
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int o = 8 * i + 4 * h;
-        const uint32_t b = __byte_perm(__byte_perm(u[o], u[o + 1], 0x0040),
-                                       __byte_perm(u[o + 2], u[o + 3], 0x0040), 0x5410) &
-                           0x0F0F0F0Fu;
-        t[h] = b | (b >> 4);  // bytes 0 and 2 hold code pairs
-      }
-      w[i] = __byte_perm(t[0], t[1], 0x6420);
-    }
+  for (int j = 0; j < N; ++j) {
+    const float2 f = f2_unpack(f2_add(t[j], m2));
+    c[j] = __float_as_uint(f.x);
+    c[N + j] = __float_as_uint(f.y);
+  }
+  if constexpr (CB * L == 16) {
+#pragma unroll
+    for (int k = 0; k < N; ++k) w[k] = __byte_perm(c[2 * k], c[2 * k + 1], 0x5410);
   } else {
-#pragma unroll
-    for (int i = 0; i < code_words<CB, NV>(); ++i) {
-      uint32_t x = 0;
-#pragma unroll
-      for (int j = 0; j < 16 && 16 * i + j < NV; ++j) x |= (u[16 * i + j] & 3u) << (2 * j);
-      w[i] = x;
-    }
+    static_assert(CB * L == 8 && N == 1, "8-bit chunks only for 8 values of 2 bits");
+    w[0] = __byte_perm(c[0], c[1], 0x0040) & 0xFFFFu;
   }
 }
 
-// One thread holds NV (8 or 16) consecutive fp16 values of a token row; the
+// One thread holds NV (8, 16 or 32) consecutive fp16 values of a token row; the
 // G / NV threads of a group are consecutive lanes (groups never straddle a
 // row).  Produces the packed codes of the NV values (BITS bits each, element
 // j at bit offset BITS * j) and the (scale, zero) half2 of the group.
@@ -95,7 +106,7 @@ template <int BITS, int G, int NV>
 __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
                                               uint32_t (&codes)[code_words<BITS, NV>()],
                                               uint32_t& meta) {
-  static_assert(NV == 8 || NV == 16, "values per thread");
+  static_assert(NV == 8 || NV == 16 || NV == 32, "values per thread");
   static_assert(G % NV == 0 && G / NV <= 32 && G <= kHeadDim, "group size");
   constexpr int NH = NV / 2;
   constexpr int GL = G / NV;  // lanes per group
@@ -124,11 +135,13 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
     const __half s16 = __float2half_ru(s32);
     const float s = __half2float(s16);
     const float r = __frcp_rn(s);
+    const uint64_t r2 = f2_pack(r, r), nd2 = f2_pack(-s, -s);
     uint32_t c[NH];
 #pragma unroll
-    for (int i = 0; i < NH; ++i)
-      c[i] = e4m3x2(copysignf(div_rn(x[2 * i], s, r), x[2 * i]),
-                    copysignf(div_rn(x[2 * i + 1], s, r), x[2 * i + 1]));
+    for (int i = 0; i < NH; ++i) {
+      const float2 q = f2_unpack(div_rn2(f2_pack(x[2 * i], x[2 * i + 1]), nd2, r2));
+      c[i] = e4m3x2(copysignf(q.x, x[2 * i]), copysignf(q.y, x[2 * i + 1]));
+    }
 #pragma unroll
     for (int i = 0; i < NH / 2; ++i) codes[i] = __byte_perm(c[2 * i], c[2 * i + 1], 0x5410);
     meta = h2_as_u32(__halves2half2(s16, __float2half_rn(0.f)));
@@ -158,32 +171,36 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
     const __half z16 = __float2half_rn(zf);
     const float z = __half2float(z16);  // an integer
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds |v| < 2^22 to an integer
-    uint32_t u[NV];
-    // code = clamp(rint(x / s) + z, 0, qmax).
-    if (__all_sync(0xffffffffu, fabsf(zf) <= 2048.0f)) {
+    // pair i of the packed arithmetic holds elements i and i + NH
+    const uint64_t r2 = f2_pack(r, r), nd2 = f2_pack(-s, -s);
+    const uint64_t m2 = f2_pack(kMagic, kMagic);
+    const float zm = z - kMagic;  // exact: an integer of magnitude below 2^24
+    const uint64_t zm2 = f2_pack(zm, zm);
+    uint64_t t[NH];  // codes as fp32 integers
+    // code = clamp(rint(x / s) + z, 0, qmax); (q + 1.5 * 2^23) + (z - 1.5 *
+    // 2^23) is rint(q) + z exactly for |q| < 2^22.
+    const float top = __fadd_rn(__fadd_rn(div_rn(mx, s, r), kMagic), zm);
+    if (__all_sync(0xffffffffu, fabsf(zf) <= 2048.0f && top <= qmax)) {
       // z is exact in fp16 and equals -rint(RN(mn / s)) (rounding and rint
-      // are monotone and odd-symmetric), so every code of the group is >= 0
-      // and every quotient lies within 2048 + qmax + 2 of zero: only the
-      // upper clamp is needed, on rint(q) + 1.5 * 2^23 + z, whose low
-      // mantissa bits then hold the code.
-      constexpr float kTop = kMagic + qmax;
+      // are monotone and odd-symmetric), so every code of the group is >= 0,
+      // the group's largest code (at its max) is <= qmax, and every quotient
+      // lies within 2048 + qmax + 2 of zero: no clamp is needed.
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const float a = __fadd_rn(__fadd_rn(div_rn(x[i], s, r), kMagic), z);
-        u[i] = __float_as_uint(fminf(a, kTop));
-      }
+      for (int i = 0; i < NH; ++i)
+        t[i] = f2_add(f2_add(div_rn2(f2_pack(x[i], x[i + NH]), nd2, r2), m2), zm2);
     } else {
       // Clamping the quotient to [-z, qmax - z] first gives the same code (z
       // is an integer: a quotient below -z rounds to at most -z, one above
       // qmax - z to at least qmax - z) and bounds it well inside +-2^22.
       const float lo = -z, hi = __fadd_rn(qmax, -z);
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const float q = fminf(fmaxf(div_rn(x[i], s, r), lo), hi);
-        u[i] = __float_as_uint(__fadd_rn(__fadd_rn(q, kMagic), z));
+      for (int i = 0; i < NH; ++i) {
+        const float2 q = f2_unpack(div_rn2(f2_pack(x[i], x[i + NH]), nd2, r2));
+        const uint64_t qc = f2_pack(fminf(fmaxf(q.x, lo), hi), fminf(fmaxf(q.y, lo), hi));
+        t[i] = f2_add(f2_add(qc, m2), zm2);
       }
     }
-    pack_codes<code_bits(BITS), NV>(u, codes);
+    pack_codes<code_bits(BITS), NV>(t, codes);
     meta = h2_as_u32(__halves2half2(s16, z16));
   }
 }

@@ -72,94 +72,212 @@ __global__ void __launch_bounds__(1024) quantize_append_kernel(const QuantArgs a
 
 // Bulk quantize (prefill).  Work unit: kUnitRows consecutive tokens of one
 // (side, sequence, KV head) plane row, whose fp16 rows are contiguous in the
-// input and whose codes and (s, z) are contiguous in the cache.  A warp takes
-// units round-robin, four rows per step (8 lanes x 32 bytes per row, 16
-// values per lane), and loads the next unit's rows before it quantizes the
-// current one, so every lane keeps 64 bytes of reads in flight.
-constexpr int kUnitRows = 8;
-constexpr int kBulkNV = 16;                           // values per lane
-constexpr int kBulkLanes = kHeadDim / kBulkNV;        // lanes per row
-constexpr int kBulkRowsPerStep = 32 / kBulkLanes;     // rows per warp step
-constexpr int kBulkSteps = kUnitRows / kBulkRowsPerStep;
+// input and whose codes and (s, z) are contiguous in the cache.  Each warp
+// takes a contiguous range of units, one unit per step (4 lanes x 64 bytes
+// per row, 32 values per lane), and keeps the next kBulkDepth - 1 units in
+// flight as cp.async copies into its own shared-memory ring: each copy
+// instruction moves 64 contiguous bytes of every row of the unit, and after
+// its own copy group has landed and a warp barrier, each lane reads its 64
+// bytes of a row.
+constexpr int kBulkNV = 32;                       // values per lane
+constexpr int kBulkLanes = kHeadDim / kBulkNV;    // lanes per row
+constexpr int kUnitRows = 32 / kBulkLanes;        // rows per unit = per warp step
+constexpr int kBulkDepth = 4;                     // ring slots per warp
+constexpr int kBulkWarps = 4;                     // warps per CTA
+constexpr int kUnitBytes = kUnitRows * kHeadDim * 2;
 
-struct BulkUnit {
-  uint4 raw[kBulkSteps][kBulkNV / 8];
-  long long dst_row;  // cache row of position 0 of the unit's plane row
-  int t0, base, is_v;
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// A position in a warp's unit sequence: plane row (side, b, h) and unit j
+// within it, plus this lane's token t.  Moving one unit steps the addresses
+// derived from it by a constant; they are rebuilt from (side, b, h, j) only
+// when the position enters the next plane row.
+struct BulkPos {
+  int side, b, h, j, t;
+  __device__ __forceinline__ void start(const QuantArgs& a, int u, int units_per_row, int ri) {
+    const int p = u / units_per_row;
+    j = u - p * units_per_row;
+    const int planes = a.batch * a.kv_heads;
+    side = p >= planes;
+    const int bh = side ? p - planes : p;
+    b = bh / a.kv_heads;
+    h = bh - b * a.kv_heads;
+    t = j * kUnitRows + ri;
+  }
+  // true when the next unit is in the same plane row (t advanced), false
+  // when the position moved to the next plane row (t reset)
+  __device__ __forceinline__ bool step(const QuantArgs& a, int units_per_row, int ri) {
+    if (++j < units_per_row) {
+      t += kUnitRows;
+      return true;
+    }
+    j = 0;
+    t = ri;
+    if (++h == a.kv_heads) {
+      h = 0;
+      if (++b == a.batch) {
+        b = 0;
+        ++side;
+      }
+    }
+    return false;
+  }
+  __device__ __forceinline__ long long bh(const QuantArgs& a) const {
+    return (long long)b * a.kv_heads + h;
+  }
 };
 
-__device__ __forceinline__ void bulk_fetch(const QuantArgs& a, int u, int units_per_row, int li,
-                                           int ri, BulkUnit& w) {
-  const int planes = a.batch * a.kv_heads;
-  const int p = u / units_per_row;
-  const int j = u - p * units_per_row;
-  const bool is_v = p >= planes;
-  const int bh = is_v ? p - planes : p;
-  w.t0 = j * kUnitRows;
-  w.base = a.seq_lens[bh / a.kv_heads];
-  w.dst_row = (long long)bh * a.max_tokens;
-  w.is_v = is_v;
-  const uint4* src = reinterpret_cast<const uint4*>(
-      (is_v ? a.v_new : a.k_new) + ((long long)bh * a.n_new + w.t0) * kHeadDim);
-#pragma unroll
-  for (int k = 0; k < kBulkSteps; ++k) {
-    const int row = kBulkRowsPerStep * k + ri;
-    const bool in = w.t0 + row < a.n_new;
-#pragma unroll
-    for (int c = 0; c < kBulkNV / 8; ++c)
-      w.raw[k][c] = in ? __ldcs(src + row * (kHeadDim / 8) + li * (kBulkNV / 8) + c)
-                       : make_uint4(0u, 0u, 0u, 0u);
+// The copy side: chunk 0 of this lane's input row.
+struct BulkSrc {
+  BulkPos p;
+  const uint4* src;
+  __device__ __forceinline__ void locate(const QuantArgs& a) {
+    src = reinterpret_cast<const uint4*>((p.side ? a.v_new : a.k_new) +
+                                         (p.bh(a) * a.n_new + p.t) * kHeadDim);
   }
-}
+  __device__ __forceinline__ void advance(const QuantArgs& a, int units_per_row, int ri) {
+    if (p.step(a, units_per_row, ri))
+      src += kUnitRows * (kHeadDim / 8);
+    else
+      locate(a);
+  }
+};
 
+// The write side: this lane's code bytes and its row's (s, z) words.  Rows
+// at or past max_tokens are never written, so their addresses may run past
+// the cache.
 template <int BITS, int G>
-__device__ __forceinline__ void bulk_work(const QuantArgs& a, int li, int ri, const BulkUnit& w) {
-  constexpr int RB = kHeadDim * code_bits(BITS) / 8;
-  constexpr int MB = (kHeadDim / G) * 4;
-  constexpr int NW = code_words<BITS, kBulkNV>();
-  uint8_t* codes = w.is_v ? a.v_codes : a.k_codes;
-  uint8_t* meta = w.is_v ? a.v_meta : a.k_meta;
-#pragma unroll
-  for (int k = 0; k < kBulkSteps; ++k) {
-    const int t = w.t0 + kBulkRowsPerStep * k + ri;
-    const int pos = w.base + t;
-    uint32_t cw[NW], m;
-    quantize_vals<BITS, G, kBulkNV>(w.raw[k], cw, m);
-    if (t < a.n_new && pos < a.max_tokens) {
-      const long long row = w.dst_row + pos;
-      uint8_t* cr = codes + row * RB;
-      if constexpr (NW == 4) {
-        reinterpret_cast<uint4*>(cr)[li] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      } else if constexpr (NW == 2) {
-        reinterpret_cast<uint2*>(cr)[li] = make_uint2(cw[0], cw[1]);
-      } else {
-        reinterpret_cast<uint32_t*>(cr)[li] = cw[0];
-      }
-      constexpr int GL = G / kBulkNV;  // lanes per group
-      if ((li % GL) == 0) reinterpret_cast<uint32_t*>(meta + row * MB)[li / GL] = m;
+struct BulkDst {
+  static constexpr int RB = kHeadDim * code_bits(BITS) / 8;
+  static constexpr int MB = (kHeadDim / G) * 4;
+  static constexpr int LB = RB / kBulkLanes;  // code bytes per lane
+  BulkPos p;
+  int pos;
+  uint8_t* codes;
+  uint8_t* meta;
+  __device__ __forceinline__ void locate(const QuantArgs& a, int li) {
+    pos = a.seq_lens[p.b] + p.t;
+    const long long row = p.bh(a) * a.max_tokens + pos;
+    codes = (p.side ? a.v_codes : a.k_codes) + row * RB + li * LB;
+    meta = (p.side ? a.v_meta : a.k_meta) + row * MB;
+  }
+  __device__ __forceinline__ void advance(const QuantArgs& a, int units_per_row, int ri,
+                                          int li) {
+    if (p.step(a, units_per_row, ri)) {
+      pos += kUnitRows;
+      codes += kUnitRows * RB;
+      meta += kUnitRows * MB;
+    } else {
+      locate(a, li);
     }
   }
+};
+
+// Ring offset of 16-byte chunk k (0..15) of row ri of a unit: k XOR (ri & 7)
+// within the row.  A copy step (lane (ri, li) moves chunk 4c + li) and a read
+// step (lane (ri, li) reads chunk 4li + c) then each put exactly four chunks
+// on every group of four banks: four wavefronts for 512 bytes, the minimum.
+__device__ __forceinline__ uint32_t bulk_slot_off(int ri, int k) {
+  return (uint32_t)(ri * (kHeadDim * 2) + ((k ^ (ri & 7)) * 16));
+}
+
+__device__ __forceinline__ void bulk_issue(const QuantArgs& a, const BulkSrc& c,
+                                           const uint32_t (&soff)[kBulkNV / 8], int li,
+                                           uint32_t slot) {
+  if (c.p.t < a.n_new) {
+#pragma unroll
+    for (int k = 0; k < kBulkNV / 8; ++k) cp_async16(slot + soff[k], c.src + k * kBulkLanes + li);
+  }
+  cp_async_commit();
 }
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(256) quantize_bulk_kernel(const QuantArgs a, int units_per_row,
-                                                            int n_units) {
-  const int lane = threadIdx.x & 31;
-  const int li = lane % kBulkLanes, ri = lane / kBulkLanes;
-  const int nw = gridDim.x * (blockDim.x >> 5);
-  int u = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // uniform across the warp
-  BulkUnit A, B;
-  if (u < n_units) bulk_fetch(a, u, units_per_row, li, ri, A);
-  while (u < n_units) {
-    const int u1 = u + nw;
-    if (u1 < n_units) bulk_fetch(a, u1, units_per_row, li, ri, B);
-    bulk_work<BITS, G>(a, li, ri, A);
-    if (u1 >= n_units) break;
-    const int u2 = u1 + nw;
-    if (u2 < n_units) bulk_fetch(a, u2, units_per_row, li, ri, A);
-    bulk_work<BITS, G>(a, li, ri, B);
-    u = u2;
+__device__ __forceinline__ void bulk_work(const QuantArgs& a, int li, const BulkDst<BITS, G>& c,
+                                          const uint32_t (&roff)[kBulkNV / 8],
+                                          const uint8_t* slot) {
+  constexpr int NW = code_words<BITS, kBulkNV>();
+  const bool in = c.p.t < a.n_new;
+  uint4 raw[kBulkNV / 8];
+#pragma unroll
+  for (int k = 0; k < kBulkNV / 8; ++k)
+    raw[k] = in ? *reinterpret_cast<const uint4*>(slot + roff[k]) : make_uint4(0u, 0u, 0u, 0u);
+  uint32_t cw[NW], m;
+  quantize_vals<BITS, G, kBulkNV>(raw, cw, m);
+  if (in && c.pos < a.max_tokens) {
+    if constexpr (NW == 8) {
+      reinterpret_cast<uint4*>(c.codes)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      reinterpret_cast<uint4*>(c.codes)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    } else if constexpr (NW == 4) {
+      *reinterpret_cast<uint4*>(c.codes) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    } else {
+      *reinterpret_cast<uint2*>(c.codes) = make_uint2(cw[0], cw[1]);
+    }
+    constexpr int GL = G / kBulkNV;  // lanes per group
+    if ((li % GL) == 0) reinterpret_cast<uint32_t*>(c.meta)[li / GL] = m;
   }
+}
+
+template <int BITS, int G>
+__global__ void __launch_bounds__(kBulkWarps * 32) quantize_bulk_kernel(const QuantArgs a,
+                                                                        int units_per_row,
+                                                                        int n_units,
+                                                                        int units_per_warp) {
+  __shared__ __align__(16) uint8_t ring[kBulkWarps][kBulkDepth][kUnitBytes];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int li = lane % kBulkLanes, ri = lane / kBulkLanes;
+  const long long gw = (long long)blockIdx.x * kBulkWarps + warp;
+  const long long first_ll = gw * units_per_warp;
+  if (first_ll >= n_units) return;  // the whole warp
+  const int first = (int)first_ll;
+  const int n = min(units_per_warp, n_units - first);
+  const uint32_t ring0 = (uint32_t)__cvta_generic_to_shared(&ring[warp][0][0]);
+  // this lane's chunk offsets in a ring slot: the chunks it copies, the
+  // chunks it reads
+  uint32_t soff[kBulkNV / 8], roff[kBulkNV / 8];
+#pragma unroll
+  for (int k = 0; k < kBulkNV / 8; ++k) {
+    soff[k] = bulk_slot_off(ri, k * kBulkLanes + li);
+    roff[k] = bulk_slot_off(ri, li * (kBulkNV / 8) + k);
+  }
+  BulkSrc ic;  // next unit to copy
+  ic.p.start(a, first, units_per_row, ri);
+  ic.locate(a);
+  BulkDst<BITS, G> wc;  // next unit to quantize
+  wc.p = ic.p;
+  wc.locate(a, li);
+#pragma unroll
+  for (int k = 0; k < kBulkDepth - 1; ++k) {
+    if (k < n) {
+      bulk_issue(a, ic, soff, li, ring0 + k * kUnitBytes);
+      ic.advance(a, units_per_row, ri);
+    } else {
+      cp_async_commit();  // empty group: the wait count stays uniform
+    }
+  }
+  for (int i = 0; i < n; ++i) {
+    cp_async_wait<kBulkDepth - 2>();  // this lane's copies of unit i have landed
+    __syncwarp();                     // ... and every lane's; unit i - 1 is read
+    // refill the slot of unit i - 1 (read in the previous step) with unit
+    // i + kBulkDepth - 1
+    if (i + kBulkDepth - 1 < n) {
+      bulk_issue(a, ic, soff, li, ring0 + ((i + kBulkDepth - 1) % kBulkDepth) * kUnitBytes);
+      ic.advance(a, units_per_row, ri);
+    } else {
+      cp_async_commit();
+    }
+    bulk_work<BITS, G>(a, li, wc, roff, &ring[warp][i % kBulkDepth][0]);
+    wc.advance(a, units_per_row, ri, li);
+  }
+  cp_async_wait<0>();
 }
 
 __global__ void advance_seq_lens_kernel(int32_t* seq_lens, int batch, int n_new,
@@ -180,21 +298,24 @@ cudaError_t launch_q(const QuantArgs& a, cudaStream_t s) {
   }
   const int units_per_row = (a.n_new + kUnitRows - 1) / kUnitRows;
   const long long n_units = 2LL * a.batch * a.kv_heads * units_per_row;
-  if (n_units > 0x7fffffffLL) return cudaErrorInvalidValue;
-  static int slots = 0;  // resident 256-thread CTAs on the device
+  if (n_units > 0x3fffffffLL) return cudaErrorInvalidValue;
+  static int slots = 0;  // resident CTAs on the device
   if (slots == 0) {
     int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_bulk_kernel<BITS, G>,
-                                                        256, 0);
+                                                        kBulkWarps * 32, 0);
     if (e != cudaSuccess) return e;
     slots = sms * (per_sm > 0 ? per_sm : 1);
   }
-  long long blocks = (n_units + 7) / 8;
-  if (blocks > slots) blocks = slots;
-  quantize_bulk_kernel<BITS, G><<<(unsigned)blocks, 256, 0, s>>>(a, units_per_row, (int)n_units);
+  // every resident warp takes an equal contiguous range of units
+  const long long warps = (long long)slots * kBulkWarps;
+  const long long per_warp = (n_units + warps - 1) / warps;
+  const long long blocks = (n_units + per_warp * kBulkWarps - 1) / (per_warp * kBulkWarps);
+  quantize_bulk_kernel<BITS, G><<<(unsigned)blocks, kBulkWarps * 32, 0, s>>>(
+      a, units_per_row, (int)n_units, (int)per_warp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !a.advance) return e;
   advance_seq_lens_kernel<<<(a.batch + 127) / 128, 128, 0, s>>>(a.seq_lens, a.batch, a.n_new,
