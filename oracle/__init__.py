@@ -65,6 +65,8 @@ def _load():
         lib.kvqo_f32_to_e4m3.restype = ctypes.c_uint8
         lib.kvqo_quantize_group_fp8.argtypes = [P, i32, P, P]
         lib.kvqo_quantize_rows_fp8.argtypes = [P, i64, i32, i32, P, P]
+        lib.kvqo_quantize_group_sym8.argtypes = [P, i32, P, P]
+        lib.kvqo_quantize_rows_sym8.argtypes = [P, i64, i32, i32, P, P]
         lib.kvqo_dequantize_rows_fmt.argtypes = [P, P, i64, i32, i32, i32, i32, P]
         lib.kvqo_attention_packed_fmt.argtypes = [P, i32, i32, P, P, i32, P, P, i32, i32, i32,
                                                   i64, i32, f64, P, P]
@@ -128,10 +130,16 @@ def quantize_group(x16, bits: int):
     return code, int(s[0]), int(z[0])
 
 
+# code formats of the C functions' `fmt` argument
+FMT_CODES = {"int": 0, "fp8": 1, "sym8": 2}
+
+
 def quantize_rows(x16, group: int, bits: int, fmt: str = "int"):
     """Token rows [N, D] of fp16 bit patterns -> (codes [N, D*bits/8] uint8,
     meta [N, D/G, 2] uint16 holding the (scale, zero) fp16 patterns).
-    fmt "fp8": E4M3 codes (bits 8) with zero point 0 (KV-cache page, FP8)."""
+    fmt "fp8": E4M3 codes (bits 8) with zero point 0 (KV-cache page, FP8);
+    fmt "sym8": symmetric INT8, two's complement codes (bits 8) with zero
+    point 0 (KV-cache page, INT8 item)."""
     lib = _load()
     x16 = _c(x16, np.uint16)
     N, D = x16.shape
@@ -141,21 +149,25 @@ def quantize_rows(x16, group: int, bits: int, fmt: str = "int"):
     if fmt == "fp8":
         assert bits == 8
         lib.kvqo_quantize_rows_fp8(_p(x16), N, D, group, _p(codes), _p(meta))
+    elif fmt == "sym8":
+        assert bits == 8
+        lib.kvqo_quantize_rows_sym8(_p(x16), N, D, group, _p(codes), _p(meta))
     else:
+        assert fmt == "int", fmt
         lib.kvqo_quantize_rows(_p(x16), N, D, group, bits, _p(codes), _p(meta))
     return codes, meta
 
 
 def dequantize_rows(codes, meta, D: int, group: int, bits: int, fmt: str = "int") -> np.ndarray:
-    """Packed rows -> fp64 [N, D]: x_hat = (c - z) * s, or e4m3(c) * s for
-    fmt "fp8" (both exact in fp64)."""
+    """Packed rows -> fp64 [N, D]: x_hat = (c - z) * s, e4m3(c) * s for
+    fmt "fp8", int8(c) * s for fmt "sym8" (all exact in fp64)."""
     lib = _load()
     codes = _c(codes, np.uint8)
     N = codes.shape[0]
     meta = _c(meta if meta is not None else np.zeros((N, 1, 2), np.uint16), np.uint16)
     out = np.zeros((N, D), np.float64)
     lib.kvqo_dequantize_rows_fmt(_p(codes), _p(meta), N, D, group if bits != 16 else D, bits,
-                                 int(fmt == "fp8"), _p(out))
+                                 FMT_CODES[fmt], _p(out))
     return out
 
 
@@ -186,6 +198,21 @@ def quantize_group_fp8(x16):
     code = np.zeros(x16.size, np.uint8)
     s = np.zeros(1, np.uint16)
     lib.kvqo_quantize_group_fp8(_p(x16), x16.size, _p(code), _p(s))
+    return code, int(s[0])
+
+
+# --------------------------------------------------------------------------
+# Symmetric INT8 (KV-cache page, INT8 item; reading R15 in kvq_oracle.c)
+# --------------------------------------------------------------------------
+
+def quantize_group_sym8(x16):
+    """One group of fp16 bit patterns -> (int8 codes as uint8[G] two's
+    complement bytes, s16)."""
+    lib = _load()
+    x16 = _c(x16, np.uint16)
+    code = np.zeros(x16.size, np.uint8)
+    s = np.zeros(1, np.uint16)
+    lib.kvqo_quantize_group_sym8(_p(x16), x16.size, _p(code), _p(s))
     return code, int(s[0])
 
 
@@ -226,7 +253,7 @@ def attention_blocks(q, K, V, scale: float, bounds: Sequence[int]):
 def attention_packed(q16, q_is_bf16: bool, k_codes, k_meta, k_bits: int, v_codes, v_meta,
                      v_bits: int, group: int, L: int, scale: float, fmt: str = "int"):
     """Attention of g query heads over one packed (sequence, KV head) cache
-    (fmt "fp8": E4M3 codes for K and V)."""
+    (fmt "fp8": E4M3 codes for K and V; "sym8": symmetric INT8)."""
     lib = _load()
     q16 = _c(q16, np.uint16)
     g, D = q16.shape
@@ -237,7 +264,7 @@ def attention_packed(q16, q_is_bf16: bool, k_codes, k_meta, k_bits: int, v_codes
     o = np.zeros((g, D), np.float64)
     lse = np.zeros(g, np.float64)
     lib.kvqo_attention_packed_fmt(_p(q16), int(bool(q_is_bf16)), g, _p(kc), _p(km), k_bits,
-                                  _p(vc), _p(vm), v_bits, int(fmt == "fp8"), group, L, D,
+                                  _p(vc), _p(vm), v_bits, FMT_CODES[fmt], group, L, D,
                                   float(scale), _p(o), _p(lse))
     return o, lse
 
@@ -295,7 +322,7 @@ def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: fl
     q16: [B, Hq, D] fp16/bf16 patterns.  segments: list of dicts with numpy
     arrays ``k_codes``/``v_codes`` [B, Hkv, T, row_bytes], ``k_meta``/``v_meta``
     [B, Hkv, T, D/G, 2] (None for bits 16), ``bits``, ``group`` and optionally
-    ``fmt`` ("int", the default, or "fp8").
+    ``fmt`` ("int", the default, "fp8" or "sym8").
     seq_lens_per_seg: list of int arrays [B].  The segments of a sequence are
     concatenated in token order (attention does not depend on the order).
     pairs: optional list of (b, kv_head) to evaluate; others stay NaN.

@@ -29,9 +29,10 @@
  *        worked example); 2.3 (per-group scaling, dequantization inside
  *        the attention matmul).
  *   [P2'] The KV-cache page above, "主流KV Cache量化方案对比" item 1 (FP8
- *        KV cache, E4M3 or E5M2, 2x compression) and "实践中的调优建议"
- *        (dynamic quantization: the scale is computed from the current
- *        vectors at every step).
+ *        KV cache, E4M3 or E5M2, 2x compression), item 2 (INT8 quantization
+ *        with a symmetric scale amax / 127, round, clamp to [-128, 127]) and
+ *        "实践中的调优建议" (dynamic quantization: the scale is computed from
+ *        the current vectors at every step).
  *
  * Readings taken where the pages are silent (each one also listed in the
  * design notes):
@@ -62,6 +63,18 @@
  *       rounded toward +infinity (so |x / s| <= 448), zero point 0; each
  *       code is x / s (one fp32 division) rounded to the nearest E4M3 value,
  *       ties to even, saturating at +-448; x_hat = e4m3(code) * s.
+ *   R15 Symmetric INT8 ([P2'] item 2): the listing reduces the scale over
+ *       head_dim of each token while its prose says per channel; the group
+ *       runs along head_dim per token like every other format (G = head_dim
+ *       is the listing's per-token scale).  s = max(amax / 127, 1e-5) in
+ *       fp32, stored in fp16 rounded toward +infinity (R2), zero point 0;
+ *       code = clamp(round(x / s), -128, 127) with one fp32 division by the
+ *       stored scale (R3) and round-half-to-even (R1), stored as a two's
+ *       complement byte; x_hat = code * s.  With the rounded-up scale
+ *       |x / s| <= 127, so the clamp never acts; it is kept as written.
+ *
+ * Code formats (the `fmt` arguments): 0 asymmetric integer codes of `bits`
+ * bits (R1-R7), 1 E4M3 (R14), 2 symmetric INT8 (R15).
  */
 #include <math.h>
 #include <stdint.h>
@@ -326,6 +339,46 @@ void kvqo_quantize_rows_fp8(const uint16_t *x, int64_t n_rows, int D, int G, uin
         }
 }
 
+/* Symmetric INT8 ([P2'] item 2; R15): one group of G binary16 values to
+ * two's complement codes with scale s. */
+void kvqo_quantize_group_sym8(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
+{
+    float amax = 0.0f;
+    for (int j = 0; j < G; ++j) {
+        float v = fabsf(kvqo_f16_to_f32(x[j]));
+        if (v > amax)
+            amax = v;
+    }
+    float s32 = amax / 127.0f;
+    if (s32 < 1e-5f)
+        s32 = 1e-5f;
+    uint16_t s16 = kvqo_f32_to_f16_up(s32);
+    float s = kvqo_f16_to_f32(s16);
+    for (int j = 0; j < G; ++j) {
+        float c = rintf(kvqo_f16_to_f32(x[j]) / s);
+        if (c < -128.0f)
+            c = -128.0f;
+        if (c > 127.0f)
+            c = 127.0f;
+        code[j] = (uint8_t)(int8_t)c;
+    }
+    *s_out = s16;
+}
+
+/* Token rows to symmetric INT8 codes (one byte per element) and (s, 0) fp16
+ * pairs per group of G along the row. */
+void kvqo_quantize_rows_sym8(const uint16_t *x, int64_t n_rows, int D, int G, uint8_t *codes,
+                             uint16_t *meta)
+{
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int g = 0; g < D / G; ++g) {
+            uint16_t s16;
+            kvqo_quantize_group_sym8(x + r * D + g * G, G, codes + r * D + g * G, &s16);
+            meta[(r * (D / G) + g) * 2 + 0] = s16;
+            meta[(r * (D / G) + g) * 2 + 1] = 0; /* zero point 0 */
+        }
+}
+
 /* Unpack code e of a packed row (R7). */
 static unsigned kvqo_code_at(const uint8_t *row, int e, int bits)
 {
@@ -336,19 +389,22 @@ static unsigned kvqo_code_at(const uint8_t *row, int e, int bits)
 /*
  * Dequantize n_rows packed rows: x_hat = (c - z) * s, evaluated in fp64,
  * where it is exact (|c - z| < 2^17 and s has 11 significant bits); with
- * fp8 != 0 the codes are E4M3 and x_hat = e4m3(c) * s (R14), also exact.
+ * fmt 1 the codes are E4M3 and x_hat = e4m3(c) * s (R14), with fmt 2 they
+ * are two's complement bytes and x_hat = c * s (R15), both also exact.
  */
 void kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *meta,
                           int64_t n_rows, int D, int G, int bits, double *out);
 
 void kvqo_dequantize_rows_fmt(const uint8_t *codes, const uint16_t *meta, int64_t n_rows,
-                              int D, int G, int bits, int fp8, double *out)
+                              int D, int G, int bits, int fmt, double *out)
 {
-    if (fp8) {
+    if (fmt == 1 || fmt == 2) {
         for (int64_t r = 0; r < n_rows; ++r)
             for (int e = 0; e < D; ++e) {
                 double s = (double)kvqo_f16_to_f32(meta[(r * (D / G) + e / G) * 2 + 0]);
-                out[r * D + e] = kvqo_e4m3_to_f64(codes[r * D + e]) * s;
+                uint8_t c = codes[r * D + e];
+                double v = (fmt == 1) ? kvqo_e4m3_to_f64(c) : (double)(int8_t)c;
+                out[r * D + e] = v * s;
             }
         return;
     }
@@ -503,7 +559,7 @@ void kvqo_attention_blocks(const double *q, int g, const double *K,
 void kvqo_attention_packed_fmt(const uint16_t *q16, int q_is_bf16, int g,
                                const uint8_t *k_codes, const uint16_t *k_meta, int k_bits,
                                const uint8_t *v_codes, const uint16_t *v_meta, int v_bits,
-                               int fp8, int G, int64_t L, int D, double scale, double *o,
+                               int fmt, int G, int64_t L, int D, double scale, double *o,
                                double *lse);
 
 void kvqo_attention_packed(const uint16_t *q16, int q_is_bf16, int g,
@@ -517,11 +573,11 @@ void kvqo_attention_packed(const uint16_t *q16, int q_is_bf16, int g,
                               v_bits, 0, G, L, D, scale, o, lse);
 }
 
-/* The same with a code format: fp8 != 0 means E4M3 codes for K and V. */
+/* The same with a code format for K and V (fmt as in the header). */
 void kvqo_attention_packed_fmt(const uint16_t *q16, int q_is_bf16, int g,
                                const uint8_t *k_codes, const uint16_t *k_meta, int k_bits,
                                const uint8_t *v_codes, const uint16_t *v_meta, int v_bits,
-                               int fp8, int G, int64_t L, int D, double scale, double *o,
+                               int fmt, int G, int64_t L, int D, double scale, double *o,
                                double *lse)
 {
     double *q = (double *)malloc((size_t)g * D * sizeof(double));
@@ -532,8 +588,8 @@ void kvqo_attention_packed_fmt(const uint16_t *q16, int q_is_bf16, int g,
     double *V = (double *)malloc((size_t)(L > 0 ? L : 1) * D * sizeof(double));
     int Gk = (k_bits == 16) ? D : G;
     int Gv = (v_bits == 16) ? D : G;
-    kvqo_dequantize_rows_fmt(k_codes, k_meta, L, D, Gk, k_bits, fp8, K);
-    kvqo_dequantize_rows_fmt(v_codes, v_meta, L, D, Gv, v_bits, fp8, V);
+    kvqo_dequantize_rows_fmt(k_codes, k_meta, L, D, Gk, k_bits, fmt, K);
+    kvqo_dequantize_rows_fmt(v_codes, v_meta, L, D, Gv, v_bits, fmt, V);
     kvqo_attention(q, g, K, V, L, D, scale, o, lse);
     free(q);
     free(K);

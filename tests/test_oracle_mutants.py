@@ -53,6 +53,13 @@ MUTANTS = [
     ("e4m3 exponent bias 8", "v = ldexp((double)(8 + m), e - 10);",
      "v = ldexp((double)(8 + m), e - 11);"),
     ("fp8 scale from another maximum", "float s32 = amax / 448.0f;", "float s32 = amax / 464.0f;"),
+    ("sym8 ties away from zero", "float c = rintf(kvqo_f16_to_f32(x[j]) / s);",
+     "float c = roundf(kvqo_f16_to_f32(x[j]) / s);"),
+    ("sym8 scale over 128 levels", "float s32 = amax / 127.0f;", "float s32 = amax / 128.0f;"),
+    ("sym8 offset-binary codes", "code[j] = (uint8_t)(int8_t)c;",
+     "code[j] = (uint8_t)(int)(c + 128.0f);"),
+    ("sym8 dequant unsigned", "double v = (fmt == 1) ? kvqo_e4m3_to_f64(c) : (double)(int8_t)c;",
+     "double v = (fmt == 1) ? kvqo_e4m3_to_f64(c) : (double)c;"),
 ]
 
 
@@ -143,6 +150,17 @@ def _pins(o):
     mids = np.clip(mids, -448, 448)
     yield "e4m3 encode vs torch", bool(np.array_equal(
         o.f32_to_e4m3(mids), torch.from_numpy(mids).to(torch.float8_e4m3fn).view(torch.uint8).numpy()))
+
+    s8 = _golden("sym8_worked_example.json")
+    ok = True
+    for g in s8["groups"]:
+        code, s16 = o.quantize_group_sym8(np.asarray(g["x"], np.float16).view(np.uint16))
+        ok &= code.tolist() == g["codes"] and s16 == int(g["s16"], 16)
+    yield "sym8 worked groups", bool(ok)
+    c8 = np.array([[0, 1, 127, 128, 255]], np.uint8)
+    m8 = np.array([[[np.float16(0.5).view(np.uint16), 0]]], np.uint16)
+    yield "sym8 dequant", o.dequantize_rows(c8, m8, 5, 5, 8, "sym8").tolist() == [
+        [0.0, 0.5, 63.5, -64.0, -0.5]]
 
     t = _golden("chunk_threshold_toy.json")
     sim, cls = o.chunk_assign(np.array(t["chunks"], np.float32), np.array(t["query"], np.float32),
