@@ -33,6 +33,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "quantized-KV decode attention tokens/s; KV-read GB/s as % of B200 HBM peak"
 DTYPE = {2: "u2", 4: "u4", 8: "u8", 16: "f16"}
+# code formats: arithmetic type, JSON name, and the library's format code
+FMT_DTYPE = {"fp8": "e4m3", "sym8": "s8"}
+FMT_NAME = {"fp8": "fp8 e4m3", "sym8": "symmetric int8"}
+FMT_CODE = {"int": 0, "fp8": 1, "sym8": 2}  # KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
@@ -229,7 +233,7 @@ def reference_line(args, wl, value, el, sample):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3" if wl.fmt == "fp8" else DTYPE[wl.bits],
+        "vs_baseline": None, "dtype": FMT_DTYPE.get(wl.fmt, DTYPE[wl.bits]),
         "data": "synthetic",
         "config": workload_config(wl),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
@@ -243,7 +247,7 @@ def workload_config(wl, extra=None):
     cfg = {"workload": wl.name, "batch_per_gpu": wl.batch, "q_heads": wl.q_heads,
            "kv_heads": wl.kv_heads, "head_dim": wl.head_dim, "context": wl.context,
            "bits": wl.bits, "group": wl.group, "q_dtype": wl.q_dtype,
-           **({"format": "fp8 e4m3"} if wl.fmt == "fp8" else {}),
+           **({"format": FMT_NAME[wl.fmt]} if wl.fmt != "int" else {}),
            "episode_steps": wl.steps if wl.append else 0}
     if extra:
         cfg.update(extra)
@@ -410,7 +414,7 @@ def run_kvq(args, wl, rank, world, local_rank):
         k, v = workloads.kv_tokens(wlr, ctx, dev)
         cache = kvq.QuantizedKVCache.allocate(
             B, H, D, max_tokens, wl.bits, wl.group, dev,
-            fmt=kvq.KVQ_FMT_FP8_E4M3 if wl.fmt == "fp8" else kvq.KVQ_FMT_INT)
+            fmt=FMT_CODE[wl.fmt])
         cache.seq_lens.zero_()
         kvq.kvq_quantize_append(cache, k, v, ctx, advance_seq_lens=True)
         base_lens = cache.seq_lens.clone()
@@ -657,7 +661,7 @@ def run_kvq(args, wl, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3" if wl.fmt == "fp8" else DTYPE[wl.bits], "data": "synthetic",
+        "dtype": FMT_DTYPE.get(wl.fmt, DTYPE[wl.bits]), "data": "synthetic",
         "config": workload_config(wl, {
             "global_batch": B * world, "parallelism": f"dp{world} (sequences sharded)",
             "cache_tokens_per_step": f"{ctx + 1}..{ctx + episode}" if wl.append else ctx,

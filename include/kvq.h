@@ -69,7 +69,8 @@ typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
 /* Code format of a plane. */
 typedef enum kvq_format {
     KVQ_FMT_INT = 0,      /* asymmetric integer codes: x_hat = (c - z) * s    */
-    KVQ_FMT_FP8_E4M3 = 1  /* FP8 E4M3 codes, bits 8: x_hat = e4m3(c) * s      */
+    KVQ_FMT_FP8_E4M3 = 1, /* FP8 E4M3 codes, bits 8: x_hat = e4m3(c) * s      */
+    KVQ_FMT_INT8_SYM = 2  /* symmetric INT8 codes, bits 8: x_hat = c * s      */
 } kvq_format;
 
 /*
@@ -85,6 +86,11 @@ typedef enum kvq_format {
  *                 with zero point 0 (the KV-cache page's FP8 KV cache, with
  *                 the scale of each group computed from the values written,
  *                 that page's dynamic quantization).
+ *   bits 8 with fmt KVQ_FMT_INT8_SYM: one two's complement int8 code per
+ *                 element, the same meta layout with zero point 0 (the
+ *                 KV-cache page's INT8 item: s = amax / 127 of the group,
+ *                 floored at 1e-5 and stored in fp16 rounded up; code =
+ *                 round-half-even(x / s), clamped to [-128, 127]).
  *   bits 16:      codes f16 [batch][kv_heads][max_tokens][head_dim] raw
  *                 values (Cocktail's FP16 class); meta unused (may be NULL).
  * Both buffers 16-byte aligned.
@@ -94,7 +100,7 @@ typedef struct kvq_plane {
     int32_t group_size; /* G: 32, 64 or 128, dividing head_dim (bits < 16)  */
     void *codes;        /* device                                           */
     void *meta;         /* device; NULL when bits == 16                     */
-    int32_t fmt;        /* kvq_format; KVQ_FMT_FP8_E4M3 needs bits 8        */
+    int32_t fmt;        /* kvq_format; the FP8 and INT8_SYM formats: bits 8 */
 } kvq_plane;
 
 /*

@@ -20,13 +20,16 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool valid_group(int g) { return g == 32 || g == 64 || g == 128; }
 
-// The kernels' template tag of a plane's format: its bit width, or kE4M3.
-int kernel_bits(const kvq_plane& p) { return p.fmt == KVQ_FMT_FP8_E4M3 ? kvq::kE4M3 : p.bits; }
+// The kernels' template tag of a plane's format: its bit width, kE4M3 or kSym8.
+int kernel_bits(const kvq_plane& p) {
+  return p.fmt == KVQ_FMT_FP8_E4M3 ? kvq::kE4M3 : p.fmt == KVQ_FMT_INT8_SYM ? kvq::kSym8 : p.bits;
+}
 
 kvq_status check_plane(const kvq_plane& p, int head_dim, bool allow16) {
   if (p.codes == nullptr || !aligned16(p.codes)) return KVQ_ERR_INVALID_ARG;
-  if (p.fmt != KVQ_FMT_INT && p.fmt != KVQ_FMT_FP8_E4M3) return KVQ_ERR_INVALID_ARG;
-  if (p.fmt == KVQ_FMT_FP8_E4M3 && p.bits != 8) return KVQ_ERR_UNSUPPORTED;
+  if (p.fmt != KVQ_FMT_INT && p.fmt != KVQ_FMT_FP8_E4M3 && p.fmt != KVQ_FMT_INT8_SYM)
+    return KVQ_ERR_INVALID_ARG;
+  if (p.fmt != KVQ_FMT_INT && p.bits != 8) return KVQ_ERR_UNSUPPORTED;
   if (p.bits == 16) {
     if (!allow16) return KVQ_ERR_UNSUPPORTED;
     return KVQ_OK;

@@ -141,6 +141,14 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   using C = TmCfg<BITS, GE, GR>;
   using WP = WordPairs<BITS>;
   using XP = CrossPairs<BITS>;
+  // the zero point the codes are read against: symmetric INT8 codes are read
+  // as offset binary (c + 128) with a stored zero point of 0
+  auto zero_of = [](float z) {
+    if constexpr (BITS == kSym8)
+      return z + 128.0f;
+    else
+      return z;
+  };
   constexpr int D = C::D, NG = C::NG, NP = C::NP, HS = C::HS, CPH = C::CPH;
   // grouped PV: dims of each group per lane, and their V bytes and words
   constexpr int CH = GE / 8, VBG = CH * code_bits(BITS) / 8, VWG = VBG >= 4 ? VBG / 4 : 1;
@@ -410,15 +418,15 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
           if constexpr (HS == 2) v[HS - 1] = s_acc[2 * r + 1];
         } else if constexpr (NG == 1) {
           const float2 sz = __half22float2(*reinterpret_cast<const __half2*>(sKm + tok * C::MB));
-          v[0] = sz.x * fmaf(-sz.y, qsA, s_acc[2 * r]);
-          if constexpr (HS == 2) v[HS - 1] = sz.x * fmaf(-sz.y, qsB, s_acc[2 * r + 1]);
+          v[0] = sz.x * fmaf(-zero_of(sz.y), qsA, s_acc[2 * r]);
+          if constexpr (HS == 2) v[HS - 1] = sz.x * fmaf(-zero_of(sz.y), qsB, s_acc[2 * r + 1]);
         } else {
           const uint2 u = *reinterpret_cast<const uint2*>(
               sKm + tok * C::MB + (NG == 4 ? 8 * (tig & 1) : 0));
           const float2 szA = __half22float2(u32_as_h2(u.x));
           const float2 szB = __half22float2(u32_as_h2(u.y));
-          v[0] = fmaf(szB.x, fmaf(-szB.y, qsB, s_acc[2 * r + 1]),
-                      szA.x * fmaf(-szA.y, qsA, s_acc[2 * r]));
+          v[0] = fmaf(szB.x, fmaf(-zero_of(szB.y), qsB, s_acc[2 * r + 1]),
+                      szA.x * fmaf(-zero_of(szA.y), qsA, s_acc[2 * r]));
           if constexpr (NG == 4) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
         }
         const bool ok = valid(tok);
@@ -493,7 +501,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
                 sVm + tok * C::MB + gv[nb] * 4));
             const bool ok = valid(tok);
             pp[r] = ok ? p[slot_of(nb)][r] * sz.x : 0.f;
-            corr[nb] = ok ? fmaf(pp[r], sz.y, corr[nb]) : corr[nb];
+            corr[nb] = ok ? fmaf(pp[r], zero_of(sz.y), corr[nb]) : corr[nb];
           }
         }
         uint32_t r0, r1;
@@ -719,7 +727,9 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   X(2, 64, 1) X(2, 64, 2) X(2, 64, 4)                                  \
   X(8, 32, 1) X(8, 32, 2) X(4, 32, 1) X(4, 32, 2) X(2, 32, 1) X(2, 32, 2)                  \
   X(kE4M3, 128, 1) X(kE4M3, 128, 2) X(kE4M3, 128, 4) X(kE4M3, 128, 8)  \
-  X(kE4M3, 64, 1) X(kE4M3, 64, 2) X(kE4M3, 64, 4) X(kE4M3, 32, 1) X(kE4M3, 32, 2)
+  X(kE4M3, 64, 1) X(kE4M3, 64, 2) X(kE4M3, 64, 4) X(kE4M3, 32, 1) X(kE4M3, 32, 2) \
+  X(kSym8, 128, 1) X(kSym8, 128, 2) X(kSym8, 128, 4) X(kSym8, 128, 8)  \
+  X(kSym8, 64, 1) X(kSym8, 64, 2) X(kSym8, 64, 4) X(kSym8, 32, 1) X(kSym8, 32, 2)
 
 }  // namespace
 

@@ -231,6 +231,23 @@ struct WordPairs<16> {
   __device__ __forceinline__ static uint32_t one(uint32_t w, int) { return w; }
 };
 
+// Symmetric INT8 word (two's complement bytes): bit 7 of every byte flipped
+// gives the offset-binary code c + 128, read like the 8-bit integer codes
+// with a zero point of 128.
+template <>
+struct WordPairs<kSym8> {
+  static constexpr int kPairs = 2, kDims = 4, kEmax = 0;
+  __device__ __forceinline__ static void run(uint32_t w, uint32_t (&p)[2]) {
+    p[0] = (w & 0x00FF00FFu) ^ 0x00800080u;
+    p[1] = prmt(w, 0u, 0x4341u) ^ 0x00800080u;
+  }
+  __host__ __device__ static constexpr int dim(int j, int e) { return j + 2 * e; }
+  __host__ __device__ static constexpr int exp(int) { return 0; }
+  __device__ __forceinline__ static uint32_t one(uint32_t w, int j) {
+    return (j ? prmt(w, 0u, 0x4341u) : (w & 0x00FF00FFu)) ^ 0x00800080u;
+  }
+};
+
 // Two E4M3 codes (low byte, high byte) to an fp16 pair (low half, high
 // half); exact, every E4M3 value being an fp16 value.
 __device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t v16) {
@@ -308,6 +325,20 @@ struct CrossPairs<8> {
     o[1] = prmt(x, 0u, 0x4341u);              // [x.b1 0 x.b3 0]
     o[2] = y & 0x00FF00FFu;
     o[3] = prmt(y, 0u, 0x4341u);
+  }
+  __host__ __device__ static constexpr int exp(int) { return 0; }
+};
+
+template <>
+struct CrossPairs<kSym8> {
+  static constexpr int kOut = 4;
+  __device__ __forceinline__ static void run(uint32_t a, uint32_t b, uint32_t (&o)[4]) {
+    const uint32_t x = prmt(a, b, 0x5410u);  // [a.b0 a.b1 b.b0 b.b1]
+    const uint32_t y = prmt(a, b, 0x7632u);  // [a.b2 a.b3 b.b2 b.b3]
+    o[0] = (x & 0x00FF00FFu) ^ 0x00800080u;  // offset binary, as in WordPairs<kSym8>
+    o[1] = prmt(x, 0u, 0x4341u) ^ 0x00800080u;
+    o[2] = (y & 0x00FF00FFu) ^ 0x00800080u;
+    o[3] = prmt(y, 0u, 0x4341u) ^ 0x00800080u;
   }
   __host__ __device__ static constexpr int exp(int) { return 0; }
 };

@@ -13,6 +13,8 @@ namespace kvq {
 // Kernel template tag of the FP8 E4M3 code format (8-bit codes); the integer
 // formats use their bit width (2, 4, 8) and raw fp16 rows use 16.
 constexpr int kE4M3 = 0x108;
+// symmetric INT8 codes (two's complement bytes, zero point 0); code_bits 8
+constexpr int kSym8 = 0x208;
 __host__ __device__ constexpr int code_bits(int tag) { return tag & 0xFF; }
 
 // One K/V plane pair of one cache segment, as the kernels see it.

@@ -118,11 +118,8 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
     x[2 * i] = f.x;
     x[2 * i + 1] = f.y;
   }
-  if constexpr (BITS == kE4M3) {
-    // FP8 E4M3 (the KV-cache page's FP8 KV cache, dynamic scale): s = max(
-    // amax / 448, 1e-5) stored in fp16 rounded up, so |x / s| <= 448;
-    // code = E4M3 of the fp32 quotient x / s; zero point 0.  The group's
-    // |max| is taken on the fp16 values (exact).
+  if constexpr (BITS == kE4M3 || BITS == kSym8) {
+    // the group's |max|, taken on the fp16 values (exact)
     __half2 am = __habs2(h2[0]);
 #pragma unroll
     for (int i = 1; i < NH; ++i) am = __hmax2(am, __habs2(h2[i]));
@@ -130,6 +127,34 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
 #pragma unroll
     for (int off = 1; off < GL; off <<= 1)
       am = __hmax2(am, u32_as_h2(__shfl_xor_sync(0xffffffffu, h2_as_u32(am), off)));
+    if constexpr (BITS == kSym8) {
+      // Symmetric INT8 (the KV-cache page's INT8 item): s = max(amax / 127,
+      // 1e-5) stored in fp16 rounded up, so |x / s| <= 127 and the clamp to
+      // [-128, 127] never acts; code = rint(x / s) as a two's complement
+      // byte; zero point 0.  The codes go through the integer packing as
+      // c + 128 in [1, 255]; flipping bit 7 of every byte then gives c.
+      constexpr float kInv127 = 1.0f / 127.0f;
+      constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+      const float s32 = fmaxf(div_rn(__low2float(am), 127.0f, kInv127), 1e-5f);
+      const __half s16 = __float2half_ru(s32);
+      const float s = __half2float(s16);
+      const float r = __frcp_rn(s);
+      const uint64_t r2 = f2_pack(r, r), nd2 = f2_pack(-s, -s);
+      const uint64_t m2 = f2_pack(kMagic, kMagic);
+      const uint64_t om2 = f2_pack(128.0f - kMagic, 128.0f - kMagic);
+      uint64_t t[NH];  // pair i holds elements i and i + NH
+#pragma unroll
+      for (int i = 0; i < NH; ++i)
+        t[i] = f2_add(f2_add(div_rn2(f2_pack(x[i], x[i + NH]), nd2, r2), m2), om2);
+      pack_codes<8, NV>(t, codes);
+#pragma unroll
+      for (int i = 0; i < code_words<BITS, NV>(); ++i) codes[i] ^= 0x80808080u;
+      meta = h2_as_u32(__halves2half2(s16, __float2half_rn(0.f)));
+      return;
+    }
+    // FP8 E4M3 (the KV-cache page's FP8 KV cache, dynamic scale): s = max(
+    // amax / 448, 1e-5) stored in fp16 rounded up, so |x / s| <= 448;
+    // code = E4M3 of the fp32 quotient x / s; zero point 0.
     constexpr float kInv448 = 1.0f / 448.0f;
     const float s32 = fmaxf(div_rn(__low2float(am), 448.0f, kInv448), 1e-5f);
     const __half s16 = __float2half_ru(s32);

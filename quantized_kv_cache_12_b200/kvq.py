@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libkvq.so")
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, \
     KVQ_ERR_CUDA = range(6)
 KVQ_F16, KVQ_BF16 = 0, 1
-KVQ_FMT_INT, KVQ_FMT_FP8_E4M3 = 0, 1
+KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM = 0, 1, 2
 HEADER_BYTES = 256  # workspace header: sticky device error word first
 
 
@@ -248,8 +248,9 @@ class QuantizedKVCache:
 
     codes: uint8 [B, H_kv, max_tokens, head_dim*bits/8];
     meta: fp16 [B, H_kv, max_tokens, head_dim/G, 2] (scale, zero), None for bits 16;
-    seq_lens: int32 [B] on the device; fmt: KVQ_FMT_INT, or KVQ_FMT_FP8_E4M3
-    (bits 8: E4M3 codes, zero points 0).
+    seq_lens: int32 [B] on the device; fmt: KVQ_FMT_INT, KVQ_FMT_FP8_E4M3
+    (bits 8: E4M3 codes, zero points 0) or KVQ_FMT_INT8_SYM (bits 8: two's
+    complement codes, zero points 0).
     """
     batch: int
     kv_heads: int

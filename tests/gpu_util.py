@@ -36,7 +36,8 @@ def fill_fp16_segment(cache, k: torch.Tensor, v: torch.Tensor, lens):
 
 
 def oracle_segment(k: torch.Tensor, v: torch.Tensor, bits: int, group: int, fmt: str = "int"):
-    """The oracle's own packed cache of the same fp16 inputs (fmt "fp8": E4M3)."""
+    """The oracle's own packed cache of the same fp16 inputs (fmt "fp8": E4M3,
+    "sym8": symmetric INT8)."""
     k16, v16 = f16_bits(k), f16_bits(v)
     if bits == 16:
         kc = k16.view(np.uint8).reshape(*k16.shape[:3], -1)

@@ -213,6 +213,28 @@ def test_fp8_planes_validated(kvq):
     assert _status(kvq.kvq_decode_workspace_bytes, c, 16) == kvq.KVQ_ERR_UNSUPPORTED  # g = 8
 
 
+def test_sym8_planes_validated(kvq):
+    """KVQ_FMT_INT8_SYM needs bits 8 and the same format on K and V; its
+    decode is built for the same (G, g) as FP8."""
+    fake = ctypes.c_void_p(0x60000)
+
+    def append_status(c):
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, 1, 1, None)
+    c = _fake_cache(kvq, bits=2)
+    c.k.fmt = c.v.fmt = kvq.KVQ_FMT_INT8_SYM
+    assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
+    c = _fake_cache(kvq, bits=8)
+    c.k.fmt = kvq.KVQ_FMT_INT8_SYM
+    c.v.fmt = kvq.KVQ_FMT_INT
+    assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
+    c = _fake_cache(kvq, bits=8, group=128, kv_heads=2)
+    c.k.fmt = c.v.fmt = kvq.KVQ_FMT_INT8_SYM
+    assert kvq.kvq_decode_workspace_bytes(c, 16) > 0   # g = 8, G = 128
+    c = _fake_cache(kvq, bits=8, group=32, kv_heads=2)
+    c.k.fmt = c.v.fmt = kvq.KVQ_FMT_INT8_SYM
+    assert _status(kvq.kvq_decode_workspace_bytes, c, 8) == kvq.KVQ_ERR_UNSUPPORTED  # 4 x 4
+
+
 def test_chunk_entry_points_reject_bad_arguments(kvq):
     lib = kvq.lib
     fake = ctypes.c_void_p(0x10000)

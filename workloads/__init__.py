@@ -68,7 +68,8 @@ class DecodeWorkload:
     alpha: float = 0.0
     beta: float = 0.0
     low_bits: Tuple[int, ...] = ()   # bit-widths of the two quantized classes
-    fmt: str = "int"          # code format: "int" (asymmetric integer) or "fp8" (E4M3, bits 8)
+    fmt: str = "int"          # code format: "int" (asymmetric integer), "fp8" (E4M3, bits 8)
+    #                           or "sym8" (symmetric INT8, bits 8)
 
     @property
     def group_ratio(self) -> int:
@@ -113,6 +114,11 @@ WORKLOADS = {
         name="llama3_8b_gqa_fp8", batch=32, q_heads=32, kv_heads=8, head_dim=128,
         context=8192, bits=8, group=64, q_dtype="f16", steps=100, append=True, seed=3,
         k_outliers=Outliers(factor=15.0, per_head=4), v_sigma=0.5, fmt="fp8"),
+    "llama2_7b_mha_sym8": DecodeWorkload(
+        name="llama2_7b_mha_sym8", batch=16, q_heads=32, kv_heads=32, head_dim=128,
+        context=4096, bits=8, group=128, q_dtype="bf16", steps=100, append=True, seed=2,
+        k_outliers=Outliers(factor=10.0, fraction=0.01),
+        v_outliers=Outliers(factor=10.0, fraction=0.01), fmt="sym8"),
     "long_gqa_int4": DecodeWorkload(
         name="long_gqa_int4", batch=1, q_heads=32, kv_heads=8, head_dim=128,
         context=131072, bits=4, group=64, q_dtype="f16", steps=256, append=True, seed=5,
