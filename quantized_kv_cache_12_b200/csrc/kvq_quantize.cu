@@ -182,12 +182,14 @@ struct BulkDst {
   }
 };
 
-// Ring offset of 16-byte chunk k (0..15) of row ri of a unit: k XOR (ri & 7)
-// within the row.  A copy step (lane (ri, li) moves chunk 4c + li) and a read
-// step (lane (ri, li) reads chunk 4li + c) then each put exactly four chunks
-// on every group of four banks: four wavefronts for 512 bytes, the minimum.
+// Ring offset of 16-byte chunk k (0..15) of row ri of a unit: position
+// k ^ (bit 3 of k) ^ (6 for odd rows) within the row.  16-byte shared-memory
+// accesses are served eight lanes (two rows) at a time; for a copy step
+// (lane (ri, li) moves chunk 4c + li) and for a read step (lane (ri, li)
+// reads chunk 4li + c) the eight chunks of each such pair of rows then fall
+// in eight different groups of four banks: no bank conflicts.
 __device__ __forceinline__ uint32_t bulk_slot_off(int ri, int k) {
-  return (uint32_t)(ri * (kHeadDim * 2) + ((k ^ (ri & 7)) * 16));
+  return (uint32_t)(ri * (kHeadDim * 2) + ((k ^ ((k >> 3) & 1) ^ ((ri & 1) * 6)) * 16));
 }
 
 __device__ __forceinline__ void bulk_issue(const QuantArgs& a, const BulkSrc& c,
