@@ -66,6 +66,8 @@ def _load():
         lib.kvqo_quantize_group_fp8.argtypes = [P, i32, P, P]
         lib.kvqo_quantize_rows_fp8.argtypes = [P, i64, i32, i32, P, P]
         lib.kvqo_quantize_group_sym8.argtypes = [P, i32, P, P]
+        lib.kvqo_quantize_block_channels.argtypes = [P, i32, i32, i32, P, P]
+        lib.kvqo_dequantize_block_channels.argtypes = [P, P, i32, i32, i32, P]
         lib.kvqo_quantize_rows_sym8.argtypes = [P, i64, i32, i32, P, P]
         lib.kvqo_dequantize_rows_fmt.argtypes = [P, P, i64, i32, i32, i32, i32, P]
         lib.kvqo_attention_packed_fmt.argtypes = [P, i32, i32, P, P, i32, P, P, i32, i32, i32,
@@ -217,6 +219,67 @@ def quantize_group_sym8(x16):
 
 
 # --------------------------------------------------------------------------
+# Per-channel K (KV-cache page, INT8 item: the Key quantized per channel;
+# reading R16 in kvq_oracle.c): blocks of KPC_BLOCK tokens, one (s, z) per
+# channel and block
+# --------------------------------------------------------------------------
+
+KPC_BLOCK = 32
+
+
+def quantize_block_channels(x16, bits: int):
+    """One block of token rows [T, D] (fp16 patterns) -> (codes [T, D*bits/8],
+    meta [D, 2] uint16 (s, z) per channel)."""
+    lib = _load()
+    x16 = _c(x16, np.uint16)
+    T, D = x16.shape
+    codes = np.zeros((T, D * bits // 8), np.uint8)
+    meta = np.zeros((D, 2), np.uint16)
+    lib.kvqo_quantize_block_channels(_p(x16), T, D, bits, _p(codes), _p(meta))
+    return codes, meta
+
+
+def dequantize_block_channels(codes, meta, D: int, bits: int) -> np.ndarray:
+    """One block's codes [T, D*bits/8] and meta [D, 2] -> fp64 [T, D]."""
+    lib = _load()
+    codes = _c(codes, np.uint8)
+    meta = _c(meta, np.uint16)
+    T = codes.shape[0]
+    out = np.zeros((T, D), np.float64)
+    lib.kvqo_dequantize_block_channels(_p(codes), _p(meta), T, D, bits, _p(out))
+    return out
+
+
+def quantize_cache_channels(x16, bits: int):
+    """x16 [..., T, D] with T a multiple of KPC_BLOCK -> codes [..., T, D*bits/8],
+    meta [..., T / KPC_BLOCK, D, 2]."""
+    x16 = _c(x16, np.uint16)
+    lead, (T, D) = x16.shape[:-2], x16.shape[-2:]
+    assert T % KPC_BLOCK == 0, T
+    flat = x16.reshape(-1, T // KPC_BLOCK, KPC_BLOCK, D)
+    codes = np.zeros((flat.shape[0], T, D * bits // 8), np.uint8)
+    meta = np.zeros((flat.shape[0], T // KPC_BLOCK, D, 2), np.uint16)
+    for i in range(flat.shape[0]):
+        for blk in range(T // KPC_BLOCK):
+            c, m = quantize_block_channels(flat[i, blk], bits)
+            codes[i, blk * KPC_BLOCK:(blk + 1) * KPC_BLOCK] = c
+            meta[i, blk] = m
+    return (codes.reshape(*lead, T, D * bits // 8),
+            meta.reshape(*lead, T // KPC_BLOCK, D, 2))
+
+
+def dequantize_channels(codes, meta, L: int, D: int, bits: int) -> np.ndarray:
+    """The first L tokens (L a multiple of KPC_BLOCK) of one (sequence, KV
+    head) of a per-channel K plane -> fp64 [L, D]."""
+    assert L % KPC_BLOCK == 0, L
+    out = np.zeros((L, D), np.float64)
+    for blk in range(L // KPC_BLOCK):
+        r = slice(blk * KPC_BLOCK, (blk + 1) * KPC_BLOCK)
+        out[r] = dequantize_block_channels(codes[r], meta[blk], D, bits)
+    return out
+
+
+# --------------------------------------------------------------------------
 # fp64 attention (score definition: KVO-LLM page 3.2; chunked + merge:
 # Cocktail page 3.2.3)
 # --------------------------------------------------------------------------
@@ -322,7 +385,9 @@ def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: fl
     q16: [B, Hq, D] fp16/bf16 patterns.  segments: list of dicts with numpy
     arrays ``k_codes``/``v_codes`` [B, Hkv, T, row_bytes], ``k_meta``/``v_meta``
     [B, Hkv, T, D/G, 2] (None for bits 16), ``bits``, ``group`` and optionally
-    ``fmt`` ("int", the default, "fp8" or "sym8").
+    ``fmt`` ("int", the default, "fp8" or "sym8") and ``k_channels`` (True: K
+    is per-channel, ``k_meta`` [B, Hkv, T / KPC_BLOCK, D, 2], lengths multiples
+    of KPC_BLOCK).
     seq_lens_per_seg: list of int arrays [B].  The segments of a sequence are
     concatenated in token order (attention does not depend on the order).
     pairs: optional list of (b, kv_head) to evaluate; others stay NaN.
@@ -341,10 +406,14 @@ def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: fl
         for seg, lens in zip(segments, seq_lens_per_seg):
             L = int(lens[b])
             bits, G = seg["bits"], seg["group"]
-            km = seg["k_meta"][b, h, :L] if bits != 16 else None
             vm = seg["v_meta"][b, h, :L] if bits != 16 else None
             fmt = seg.get("fmt", "int")
-            Ks.append(dequantize_rows(seg["k_codes"][b, h, :L], km, D, G, bits, fmt))
+            if seg.get("k_channels", False):
+                Ks.append(dequantize_channels(seg["k_codes"][b, h, :L], seg["k_meta"][b, h], L,
+                                              D, bits))
+            else:
+                km = seg["k_meta"][b, h, :L] if bits != 16 else None
+                Ks.append(dequantize_rows(seg["k_codes"][b, h, :L], km, D, G, bits, fmt))
             Vs.append(dequantize_rows(seg["v_codes"][b, h, :L], vm, D, G, bits, fmt))
         K = np.concatenate(Ks, 0)
         V = np.concatenate(Vs, 0)

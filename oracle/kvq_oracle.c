@@ -72,6 +72,16 @@
  *       stored scale (R3) and round-half-to-even (R1), stored as a two's
  *       complement byte; x_hat = code * s.  With the rounded-up scale
  *       |x / s| <= 127, so the clamp never acts; it is kept as written.
+ *   R16 Per-channel K ([P2'] item 2: the Key is more sensitive to
+ *       quantization error and is quantized per channel, the Value per
+ *       token).  K is grouped per channel over blocks of 32 consecutive
+ *       tokens of one (sequence, KV head): each channel of a block has its
+ *       own (s, z), from the asymmetric formula of R1-R5 over the block's 32
+ *       values of that channel.  Codes stay packed along token rows (R7);
+ *       the (s, z) pairs are stored per block and channel.  Only complete
+ *       blocks are quantized: the tokens of an unfinished block stay in
+ *       fp16 (a separate fp16 segment) until the block is complete.  V keeps
+ *       its per-token groups along head_dim (R6).
  *
  * Code formats (the `fmt` arguments): 0 asymmetric integer codes of `bits`
  * bits (R1-R7), 1 E4M3 (R14), 2 symmetric INT8 (R15).
@@ -430,6 +440,50 @@ void kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *meta,
             out[r * D + e] = (c - z) * s;
         }
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Per-channel K ([P2'] item 2: the Key quantized per channel; R16)         */
+/* ------------------------------------------------------------------------ */
+
+/* One block of T token rows x [T][D] (binary16) of one (sequence, KV head):
+ * the T values of channel d form one group, quantized with the asymmetric
+ * formula of R1-R5 (kvqo_quantize_group).  codes: [T][D*bits/8], packed
+ * along each token row (R7); meta: [D][2], the (s, z) of each channel. */
+void kvqo_quantize_block_channels(const uint16_t *x, int T, int D, int bits, uint8_t *codes,
+                                  uint16_t *meta)
+{
+    const int64_t row_bytes = (int64_t)D * bits / 8;
+    uint16_t *col = (uint16_t *)malloc((size_t)T * sizeof(uint16_t));
+    uint8_t *tmp = (uint8_t *)malloc((size_t)T);
+    memset(codes, 0, (size_t)(T * row_bytes));
+    for (int d = 0; d < D; ++d) {
+        for (int t = 0; t < T; ++t)
+            col[t] = x[(int64_t)t * D + d];
+        uint16_t s16, z16;
+        kvqo_quantize_group(col, T, bits, tmp, &s16, &z16);
+        meta[d * 2 + 0] = s16;
+        meta[d * 2 + 1] = z16;
+        const int bitpos = d * bits;
+        for (int t = 0; t < T; ++t)
+            codes[t * row_bytes + bitpos / 8] |= (uint8_t)(tmp[t] << (bitpos % 8));
+    }
+    free(col);
+    free(tmp);
+}
+
+/* x_hat[t][d] = (c[t][d] - z_d) * s_d of one block, in fp64 (exact). */
+void kvqo_dequantize_block_channels(const uint8_t *codes, const uint16_t *meta, int T, int D,
+                                    int bits, double *out)
+{
+    const int64_t row_bytes = (int64_t)D * bits / 8;
+    for (int t = 0; t < T; ++t)
+        for (int d = 0; d < D; ++d) {
+            double s = (double)kvqo_f16_to_f32(meta[d * 2 + 0]);
+            double z = (double)kvqo_f16_to_f32(meta[d * 2 + 1]);
+            double c = (double)kvqo_code_at(codes + t * row_bytes, d, bits);
+            out[(int64_t)t * D + d] = (c - z) * s;
+        }
 }
 
 /* ------------------------------------------------------------------------ */

@@ -60,6 +60,12 @@ MUTANTS = [
      "code[j] = (uint8_t)(int)(c + 128.0f);"),
     ("sym8 dequant unsigned", "double v = (fmt == 1) ? kvqo_e4m3_to_f64(c) : (double)(int8_t)c;",
      "double v = (fmt == 1) ? kvqo_e4m3_to_f64(c) : (double)c;"),
+    ("per-channel block read transposed", "col[t] = x[(int64_t)t * D + d];",
+     "col[t] = x[(int64_t)d * T + t];"),
+    ("per-channel codes at the token offset", "codes[t * row_bytes + bitpos / 8] |= (uint8_t)(tmp[t] << (bitpos % 8));",
+     "codes[d * (row_bytes / 4) + (t * bits) / 8] |= (uint8_t)(tmp[t] << ((t * bits) % 8));"),
+    ("per-channel dequant ignores the zero point", "out[(int64_t)t * D + d] = (c - z) * s;",
+     "out[(int64_t)t * D + d] = c * s;"),
 ]
 
 
@@ -161,6 +167,22 @@ def _pins(o):
     m8 = np.array([[[np.float16(0.5).view(np.uint16), 0]]], np.uint16)
     yield "sym8 dequant", o.dequantize_rows(c8, m8, 5, 5, 8, "sym8").tolist() == [
         [0.0, 0.5, 63.5, -64.0, -0.5]]
+
+    rng_k = np.random.default_rng(5)
+    xk = (rng_k.standard_normal((32, 128)) * 3).astype(np.float16)
+    xk[:, 5] = np.linspace(-40, 90, 32)
+    ck, mk = o.quantize_block_channels(xk.view(np.uint16), 4)
+    ctr, mtr = o.quantize_rows(np.ascontiguousarray(xk.T).view(np.uint16), 32, 4)
+    jj = np.arange(128)
+    un = (ck[:, jj // 2].astype(np.int64) >> ((jj % 2) * 4)) & 15
+    jt = np.arange(32)
+    unt = (ctr[:, jt // 2].astype(np.int64) >> ((jt % 2) * 4)) & 15
+    yield "per-channel = transposed per-token", bool(np.array_equal(mk, mtr[:, 0, :])
+                                                      and np.array_equal(un, unt.T))
+    xh = o.dequantize_block_channels(ck, mk, 128, 4)
+    sk = mk[:, 0].view(np.float16).astype(np.float64)
+    yield "per-channel half-step bound", bool(np.all(np.abs(xk.astype(np.float64) - xh)
+                                                     <= sk[None, :] / 2 * (1 + 2.0**-12)))
 
     t = _golden("chunk_threshold_toy.json")
     sim, cls = o.chunk_assign(np.array(t["chunks"], np.float32), np.array(t["query"], np.float32),
