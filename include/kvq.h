@@ -73,6 +73,15 @@ typedef enum kvq_format {
     KVQ_FMT_INT8_SYM = 2  /* symmetric INT8 codes, bits 8: x_hat = c * s      */
 } kvq_format;
 
+/* Grouping axis of a plane's (scale, zero point) pairs. */
+typedef enum kvq_axis {
+    KVQ_AXIS_TOKEN = 0,   /* groups of G along head_dim within a token row    */
+    KVQ_AXIS_CHANNEL = 1  /* K only: one group per channel over each block of */
+                          /* KVQ_CHANNEL_BLOCK consecutive tokens             */
+} kvq_axis;
+
+#define KVQ_CHANNEL_BLOCK 32
+
 /*
  * One K or V plane of a cache (one bit-width).
  *   bits 2, 4, 8: codes  u8  [batch][kv_heads][max_tokens][head_dim*bits/8],
@@ -91,6 +100,14 @@ typedef enum kvq_format {
  *                 KV-cache page's INT8 item: s = amax / 127 of the group,
  *                 floored at 1e-5 and stored in fp16 rounded up; code =
  *                 round-half-even(x / s), clamped to [-128, 127]).
+ *   axis KVQ_AXIS_CHANNEL (K plane, fmt KVQ_FMT_INT, bits 2, 4 or 8): the
+ *                 KV-cache page's advice to quantize the Key per channel.
+ *                 Codes as above; meta f16 [batch][kv_heads][max_tokens /
+ *                 KVQ_CHANNEL_BLOCK][head_dim][2], the (scale, zero point) of
+ *                 channel d over the block's tokens (same formula as the
+ *                 token groups); group_size is not used for this plane.
+ *                 Only whole blocks are quantized: the tokens of an
+ *                 unfinished block belong in a separate bits-16 segment.
  *   bits 16:      codes f16 [batch][kv_heads][max_tokens][head_dim] raw
  *                 values (Cocktail's FP16 class); meta unused (may be NULL).
  * Both buffers 16-byte aligned.
@@ -101,6 +118,7 @@ typedef struct kvq_plane {
     void *codes;        /* device                                           */
     void *meta;         /* device; NULL when bits == 16                     */
     int32_t fmt;        /* kvq_format; the FP8 and INT8_SYM formats: bits 8 */
+    int32_t axis;       /* kvq_axis; KVQ_AXIS_CHANNEL on the K plane only   */
 } kvq_plane;
 
 /*
@@ -158,8 +176,11 @@ uint64_t kvq_kv_elements(uint64_t layers, uint64_t kv_heads, uint64_t head_dim,
  *                 (capped at max_tokens), in stream order.
  * Tokens whose position would reach max_tokens are not written (the
  * kernel checks on the device).  Both planes must have bits 2, 4 or 8 and
- * the same group size.  Errors: KVQ_ERR_INVALID_ARG (nulls, n_new < 1,
- * misalignment), KVQ_ERR_CAPACITY (n_new > max_tokens),
+ * the same group size.  With a per-channel K plane (KVQ_AXIS_CHANNEL)
+ * n_new must be a multiple of KVQ_CHANNEL_BLOCK, and so must seq_lens[b]
+ * on the device: a sequence whose length is not is neither written nor
+ * advanced.  Errors: KVQ_ERR_INVALID_ARG (nulls, n_new < 1, misalignment,
+ * n_new off a block boundary), KVQ_ERR_CAPACITY (n_new > max_tokens),
  * KVQ_ERR_UNSUPPORTED, KVQ_ERR_CUDA.
  */
 kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k_new,

@@ -25,17 +25,22 @@ int kernel_bits(const kvq_plane& p) {
   return p.fmt == KVQ_FMT_FP8_E4M3 ? kvq::kE4M3 : p.fmt == KVQ_FMT_INT8_SYM ? kvq::kSym8 : p.bits;
 }
 
-kvq_status check_plane(const kvq_plane& p, int head_dim, bool allow16) {
+kvq_status check_plane(const kvq_plane& p, int head_dim, bool allow16, bool is_k) {
   if (p.codes == nullptr || !aligned16(p.codes)) return KVQ_ERR_INVALID_ARG;
   if (p.fmt != KVQ_FMT_INT && p.fmt != KVQ_FMT_FP8_E4M3 && p.fmt != KVQ_FMT_INT8_SYM)
     return KVQ_ERR_INVALID_ARG;
+  if (p.axis != KVQ_AXIS_TOKEN && p.axis != KVQ_AXIS_CHANNEL) return KVQ_ERR_INVALID_ARG;
   if (p.fmt != KVQ_FMT_INT && p.bits != 8) return KVQ_ERR_UNSUPPORTED;
+  if (p.axis == KVQ_AXIS_CHANNEL &&
+      (!is_k || p.fmt != KVQ_FMT_INT || !(p.bits == 2 || p.bits == 4 || p.bits == 8)))
+    return KVQ_ERR_UNSUPPORTED;
   if (p.bits == 16) {
     if (!allow16) return KVQ_ERR_UNSUPPORTED;
     return KVQ_OK;
   }
   if (!(p.bits == 2 || p.bits == 4 || p.bits == 8)) return KVQ_ERR_UNSUPPORTED;
-  if (!valid_group(p.group_size) || head_dim % p.group_size != 0) return KVQ_ERR_UNSUPPORTED;
+  if (p.axis == KVQ_AXIS_TOKEN && (!valid_group(p.group_size) || head_dim % p.group_size != 0))
+    return KVQ_ERR_UNSUPPORTED;
   if (p.meta == nullptr || !aligned16(p.meta)) return KVQ_ERR_INVALID_ARG;
   return KVQ_OK;
 }
@@ -47,12 +52,13 @@ kvq_status check_cache(const kvq_cache* c, bool allow16) {
   if (c->head_dim != kD) return KVQ_ERR_UNSUPPORTED;
   if (c->max_tokens % 64 != 0) return KVQ_ERR_INVALID_ARG;
   if (c->seq_lens == nullptr) return KVQ_ERR_INVALID_ARG;
-  kvq_status s = check_plane(c->k, c->head_dim, allow16);
+  kvq_status s = check_plane(c->k, c->head_dim, allow16, true);
   if (s != KVQ_OK) return s;
-  s = check_plane(c->v, c->head_dim, allow16);
+  s = check_plane(c->v, c->head_dim, allow16, false);
   if (s != KVQ_OK) return s;
   if (c->k.bits != c->v.bits || c->k.fmt != c->v.fmt) return KVQ_ERR_UNSUPPORTED;
-  if (c->k.bits != 16 && c->k.group_size != c->v.group_size) return KVQ_ERR_UNSUPPORTED;
+  if (c->k.bits != 16 && c->k.axis == KVQ_AXIS_TOKEN && c->k.group_size != c->v.group_size)
+    return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }
 
@@ -104,7 +110,8 @@ kvq_status plan_splits(const kvq_cache* segs, int n_segs, int q_heads, int max_l
   const int g = q_heads / segs[0].kv_heads;
   for (int i = 0; i < n_segs; ++i) {
     const int bits = kernel_bits(segs[i].k);
-    const int ctas = kvq::decode_ctas_per_sm(bits, bits == 16 ? kD : segs[i].k.group_size, g);
+    const int ctas = kvq::decode_ctas_per_sm(bits, bits == 16 ? kD : segs[i].v.group_size, g,
+                                             segs[i].k.axis == KVQ_AXIS_CHANNEL);
     plan->n_split[i] = choose_splits(segs[i], max_len_hint, ctas);
     plan->parts += plan->n_split[i];
   }
@@ -124,7 +131,8 @@ kvq_status check_segments(const kvq_cache* segs, int n_segs, int q_heads) {
   const int g = q_heads / segs[0].kv_heads;
   for (int i = 0; i < n_segs; ++i) {
     const int bits = kernel_bits(segs[i].k);
-    if (!kvq::decode_supported(bits, bits == 16 ? kD : segs[i].k.group_size, g))
+    const bool kpc = segs[i].k.axis == KVQ_AXIS_CHANNEL;
+    if (!kvq::decode_supported(bits, bits == 16 ? kD : segs[i].v.group_size, g, kpc))
       return KVQ_ERR_UNSUPPORTED;
   }
   return KVQ_OK;
@@ -230,6 +238,9 @@ kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const 
   a.max_tokens = cache->max_tokens;
   a.n_new = n_new;
   a.advance = advance_seq_lens != 0;
+  a.side0 = 0;
+  a.k_channels = cache->k.axis == KVQ_AXIS_CHANNEL;
+  if (a.k_channels && n_new % KVQ_CHANNEL_BLOCK != 0) return KVQ_ERR_INVALID_ARG;
   cudaError_t e = kvq::launch_quantize(a, kernel_bits(cache->k), cache->k.group_size,
                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
@@ -305,7 +316,8 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
     v.v_meta = static_cast<const uint8_t*>(segs[i].v.meta);
     v.seq_lens = segs[i].seq_lens;
     v.bits = kernel_bits(segs[i].k);
-    v.group = segs[i].k.bits == 16 ? kD : segs[i].k.group_size;
+    v.group = segs[i].k.bits == 16 ? kD : segs[i].v.group_size;
+    v.k_channels = segs[i].k.axis == KVQ_AXIS_CHANNEL;
     v.max_tokens = segs[i].max_tokens;
     v.n_split = plan.n_split[i];
     v.part_base = base;
@@ -358,6 +370,9 @@ kvq_status decode_step_stages(const kvq_cache* cache, const void* k_new, const v
   kvq_status st = check_segments(cache, 1, q_heads);
   if (st != KVQ_OK) return st;
   if (cache->k.bits == 16) return KVQ_ERR_UNSUPPORTED;
+  // a per-channel K block is quantized only once it is complete: single
+  // tokens go to a separate fp16 segment
+  if (cache->k.axis == KVQ_AXIS_CHANNEL) return KVQ_ERR_UNSUPPORTED;
   if (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new))
     return KVQ_ERR_INVALID_ARG;
   const int g = q_heads / cache->kv_heads;
@@ -420,7 +435,8 @@ kvq_status kvq_chunk_reorder(const kvq_cache* segs, const void* k_src, const voi
   for (int i = 0; i < 3; ++i) {
     kvq_status st = check_cache(&segs[i], true);
     if (st != KVQ_OK) return st;
-    if (segs[i].k.bits != want_bits[i] || segs[i].k.fmt != KVQ_FMT_INT)
+    if (segs[i].k.bits != want_bits[i] || segs[i].k.fmt != KVQ_FMT_INT ||
+        segs[i].k.axis != KVQ_AXIS_TOKEN)
       return KVQ_ERR_INVALID_ARG;
     if (segs[i].batch != segs[0].batch || segs[i].kv_heads != segs[0].kv_heads)
       return KVQ_ERR_INVALID_ARG;

@@ -628,8 +628,9 @@ cudaError_t launch_split_g(const DecodeArgs& a, const SegView& seg, cudaStream_t
 
 }  // namespace
 
-bool decode_supported(int bits, int group, int group_ratio) {
-  if (bits == kE4M3 || bits == kSym8) return decode_tm_supported(bits, group, group_ratio);
+bool decode_supported(int bits, int group, int group_ratio, bool kpc) {
+  if (kpc || bits == kE4M3 || bits == kSym8)
+    return decode_tm_supported(bits, group, group_ratio, kpc);
   if (!(group_ratio == 1 || group_ratio == 2 || group_ratio == 4 || group_ratio == 8))
     return false;
   if (bits == 16) return true;
@@ -638,16 +639,18 @@ bool decode_supported(int bits, int group, int group_ratio) {
   return (kHeadDim / group) * group_ratio <= 16;
 }
 
-int decode_ctas_per_sm(int bits, int group, int group_ratio) {
-  if (decode_tm_supported(bits, group, group_ratio))
-    return decode_tm_ctas_per_sm(bits, group, group_ratio);
+int decode_ctas_per_sm(int bits, int group, int group_ratio, bool kpc) {
+  if (decode_tm_supported(bits, group, group_ratio, kpc))
+    return decode_tm_ctas_per_sm(bits, group, group_ratio, kpc);
   return Cfg<4, 64>::MIN_CTAS;  // the same for every format
 }
 
 cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   const int bits = seg.bits, group = (seg.bits == 16) ? kHeadDim : seg.group;
   // (group, head) columns that fit one 8-wide tile: tokens-on-M kernel
-  if (decode_tm_supported(bits, group, a.group_ratio)) return launch_decode_tm(a, seg, s);
+  if (decode_tm_supported(bits, group, a.group_ratio, seg.k_channels))
+    return launch_decode_tm(a, seg, s);
+  if (seg.k_channels) return cudaErrorInvalidValue;
   // 16 (group, head) rows: this file's kernel
 #define KVQ_D(B, G_, R) \
   if (bits == B && group == G_ && a.group_ratio == R) return launch_split_g<B, G_, R>(a, seg, s);

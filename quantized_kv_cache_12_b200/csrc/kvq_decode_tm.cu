@@ -733,7 +733,8 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
 
 }  // namespace
 
-bool decode_tm_supported(int bits, int group, int group_ratio) {
+bool decode_tm_supported(int bits, int group, int group_ratio, bool kpc) {
+  if (kpc) return false;
 #define KVQ_X(B, G_, R) \
   if (bits == B && group == G_ && group_ratio == R) return true;
   KVQ_TM_FORMATS(KVQ_X)
@@ -741,7 +742,8 @@ bool decode_tm_supported(int bits, int group, int group_ratio) {
   return false;
 }
 
-int decode_tm_ctas_per_sm(int bits, int group, int group_ratio) {
+int decode_tm_ctas_per_sm(int bits, int group, int group_ratio, bool kpc) {
+  if (kpc) return 0;
 #define KVQ_X(B, G_, R) \
   if (bits == B && group == G_ && group_ratio == R) return TmCfg<B, G_, R>::MIN_CTAS;
   KVQ_TM_FORMATS(KVQ_X)

@@ -29,6 +29,7 @@ struct SegView {
   int32_t max_tokens;
   int32_t n_split;       // CTAs per (sequence, KV head) for this segment
   int32_t part_base;     // index of this segment's first partial
+  int32_t k_channels;    // K grouped per channel over kChannelBlock-token blocks
 };
 
 struct DecodeArgs {
@@ -61,16 +62,25 @@ struct QuantArgs {
   int32_t* seq_lens;
   int32_t batch, kv_heads, max_tokens, n_new;
   int32_t advance;
+  // per-channel K (K plane grouped per channel over blocks of
+  // kChannelBlock tokens): the per-token kernels then write V only (side0 =
+  // 1), and a sequence whose length is not a multiple of the block is not
+  // written and not advanced
+  int32_t side0;
+  int32_t k_channels;
 };
+// tokens per block of a per-channel K plane
+constexpr int kChannelBlock = 32;
 
 // Per-bit-width launchers (kvq_quantize.cu, kvq_decode.cu, kvq_chunk.cu).
 cudaError_t launch_quantize(const QuantArgs& a, int bits, int group, cudaStream_t s);
-bool decode_supported(int bits, int group, int group_ratio);
+// kpc: the K plane is grouped per channel (group is then V's group size)
+bool decode_supported(int bits, int group, int group_ratio, bool kpc = false);
 // resident decode CTAs per SM for a segment format and query-group ratio
-int decode_ctas_per_sm(int bits, int group, int group_ratio);
+int decode_ctas_per_sm(int bits, int group, int group_ratio, bool kpc = false);
 // the tokens-on-M kernel (kvq_decode_tm.cu): formats with NG * g <= 8
-bool decode_tm_supported(int bits, int group, int group_ratio);
-int decode_tm_ctas_per_sm(int bits, int group, int group_ratio);
+bool decode_tm_supported(int bits, int group, int group_ratio, bool kpc = false);
+int decode_tm_ctas_per_sm(int bits, int group, int group_ratio, bool kpc = false);
 cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s);

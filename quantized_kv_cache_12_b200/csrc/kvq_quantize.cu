@@ -50,11 +50,12 @@ template <int BITS, int G>
 __global__ void __launch_bounds__(1024) quantize_append_kernel(const QuantArgs a) {
   const int b = blockIdx.x;
   const int base = a.seq_lens[b];
+  if (a.k_channels && base % kChannelBlock != 0) return;  // not written, not advanced
   const int rows_per_side = a.kv_heads * a.n_new;
   const int rows = 2 * rows_per_side;
   const int lane16 = threadIdx.x & 15;
   const long long per = (long long)a.batch * rows_per_side;
-  for (int r0 = 0; r0 < rows; r0 += blockDim.x / 16) {
+  for (int r0 = a.side0 * rows_per_side; r0 < rows; r0 += blockDim.x / 16) {
     const int r = r0 + (int)(threadIdx.x >> 4);
     const bool in = r < rows;
     const int rs = in ? r : 0;
@@ -162,10 +163,13 @@ struct BulkDst {
   static constexpr int LB = RB / kBulkLanes;  // code bytes per lane
   BulkPos p;
   int pos;
+  bool skip;  // a per-channel-K cache's sequence off a block boundary
   uint8_t* codes;
   uint8_t* meta;
   __device__ __forceinline__ void locate(const QuantArgs& a, int li) {
-    pos = a.seq_lens[p.b] + p.t;
+    const int base = a.seq_lens[p.b];
+    skip = a.k_channels && base % kChannelBlock != 0;
+    pos = base + p.t;
     const long long row = p.bh(a) * a.max_tokens + pos;
     codes = (p.side ? a.v_codes : a.k_codes) + row * RB + li * LB;
     meta = (p.side ? a.v_meta : a.k_meta) + row * MB;
@@ -214,7 +218,7 @@ __device__ __forceinline__ void bulk_work(const QuantArgs& a, int li, const Bulk
     raw[k] = in ? *reinterpret_cast<const uint4*>(slot + roff[k]) : make_uint4(0u, 0u, 0u, 0u);
   uint32_t cw[NW], m;
   quantize_vals<BITS, G, kBulkNV>(raw, cw, m);
-  if (in && c.pos < a.max_tokens) {
+  if (in && c.pos < a.max_tokens && !c.skip) {
     if constexpr (NW == 8) {
       reinterpret_cast<uint4*>(c.codes)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
       reinterpret_cast<uint4*>(c.codes)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
@@ -250,8 +254,8 @@ __global__ void __launch_bounds__(kBulkWarps * 32) quantize_bulk_kernel(const Qu
     soff[k] = bulk_slot_off(ri, k * kBulkLanes + li);
     roff[k] = bulk_slot_off(ri, li * (kBulkNV / 8) + k);
   }
-  BulkSrc ic;  // next unit to copy
-  ic.p.start(a, first, units_per_row, ri);
+  BulkSrc ic;  // next unit to copy (units of side 0 precede those of side 1)
+  ic.p.start(a, first + a.side0 * a.batch * a.kv_heads * units_per_row, units_per_row, ri);
   ic.locate(a);
   BulkDst<BITS, G> wc;  // next unit to quantize
   wc.p = ic.p;
@@ -283,14 +287,87 @@ __global__ void __launch_bounds__(kBulkWarps * 32) quantize_bulk_kernel(const Qu
 }
 
 __global__ void advance_seq_lens_kernel(int32_t* seq_lens, int batch, int n_new,
-                                        int max_tokens) {
+                                        int max_tokens, int k_channels) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < batch) seq_lens[b] = min(seq_lens[b] + n_new, max_tokens);
+  if (b < batch && !(k_channels && seq_lens[b] % kChannelBlock != 0))
+    seq_lens[b] = min(seq_lens[b] + n_new, max_tokens);
+}
+
+// Per-channel K (the KV-cache page's INT8 item: the Key quantized per
+// channel): one CTA per block of kChannelBlock new tokens of one (sequence,
+// KV head), thread d owning channel d.  The block's rows are staged in shared
+// memory; each channel's min, max, scale, zero point and codes follow the
+// same fp32 steps as the per-token groups (IEEE division, round half to
+// even), then the codes are packed along the token rows.  A sequence whose
+// length is not a multiple of the block is skipped; blocks at or past
+// max_tokens (a multiple of 64) are dropped whole.
+template <int BITS>
+__global__ void __launch_bounds__(kHeadDim) quantize_k_channels_kernel(const QuantArgs a) {
+  constexpr int D = kHeadDim, TB = kChannelBlock, RB = D * BITS / 8;
+  constexpr int EPW = 32 / BITS;  // codes per 32-bit word
+  __shared__ __align__(16) __half xs[TB][D];
+  __shared__ uint8_t cs[TB][D];
+  const int bh = blockIdx.y;
+  const int j = blockIdx.x;
+  const int b = bh / a.kv_heads;
+  const int base = a.seq_lens[b];
+  if (base % TB != 0) return;
+  const int pos0 = base + j * TB;
+  if (pos0 >= a.max_tokens) return;
+  const uint4* src = reinterpret_cast<const uint4*>(a.k_new + ((long long)bh * a.n_new + j * TB) * D);
+  for (int i = threadIdx.x; i < TB * D / 8; i += blockDim.x)
+    reinterpret_cast<uint4*>(&xs[0][0])[i] = src[i];
+  __syncthreads();
+  const int d = threadIdx.x;
+  float mn = __half2float(xs[0][d]), mx = mn;
+  for (int t = 1; t < TB; ++t) {
+    const float v = __half2float(xs[t][d]);
+    mn = v < mn ? v : mn;
+    mx = v > mx ? v : mx;
+  }
+  constexpr float qmax = float((1 << BITS) - 1);
+  const float s32 = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), qmax), 1e-5f);
+  const __half s16 = __float2half_ru(s32);
+  const float s = __half2float(s16);
+  float zf = __fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.0f);
+  zf = fminf(fmaxf(zf, -65504.0f), 65504.0f);
+  const __half z16 = __float2half_rn(zf);
+  const float z = __half2float(z16);
+  for (int t = 0; t < TB; ++t) {
+    const float c = __fadd_rn(rintf(__fdiv_rn(__half2float(xs[t][d]), s)), z);
+    cs[t][d] = (uint8_t)fminf(fmaxf(c, 0.0f), qmax);
+  }
+  const long long blk = (long long)bh * (a.max_tokens / TB) + pos0 / TB;
+  reinterpret_cast<__half2*>(a.k_meta)[blk * D + d] = __halves2half2(s16, z16);
+  __syncthreads();
+  for (int i = threadIdx.x; i < TB * RB / 4; i += blockDim.x) {
+    const int t = i / (RB / 4), w = i % (RB / 4);
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < EPW; ++e) word |= (uint32_t)cs[t][w * EPW + e] << (e * BITS);
+    reinterpret_cast<uint32_t*>(a.k_codes + ((long long)bh * a.max_tokens + pos0 + t) * RB)[w] =
+        word;
+  }
 }
 
 template <int BITS, int G>
-cudaError_t launch_q(const QuantArgs& a, cudaStream_t s) {
-  const int rows_per_seq = 2 * a.kv_heads * a.n_new;
+cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
+  QuantArgs a = a_in;
+  if (a.k_channels) {
+    // K: whole blocks, per channel; then the per-token kernels write V only
+    if constexpr (BITS == 2 || BITS == 4 || BITS == 8) {
+      if (a.n_new % kChannelBlock != 0 || (long long)a.batch * a.kv_heads > 65535)
+        return cudaErrorInvalidValue;
+      const dim3 grid(a.n_new / kChannelBlock, a.batch * a.kv_heads);
+      quantize_k_channels_kernel<BITS><<<grid, kHeadDim, 0, s>>>(a);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      a.side0 = 1;
+    } else {
+      return cudaErrorInvalidValue;
+    }
+  }
+  const int rows_per_seq = (2 - a.side0) * a.kv_heads * a.n_new;
   if (rows_per_seq <= 512) {
     // one pass over the sequence's rows when they fit in one CTA
     int threads = ((rows_per_seq * 16 + 63) / 64) * 64;
@@ -299,7 +376,7 @@ cudaError_t launch_q(const QuantArgs& a, cudaStream_t s) {
     return cudaGetLastError();
   }
   const int units_per_row = (a.n_new + kUnitRows - 1) / kUnitRows;
-  const long long n_units = 2LL * a.batch * a.kv_heads * units_per_row;
+  const long long n_units = (2LL - a.side0) * a.batch * a.kv_heads * units_per_row;
   if (n_units > 0x3fffffffLL) return cudaErrorInvalidValue;
   static int slots = 0;  // resident CTAs on the device
   if (slots == 0) {
@@ -321,7 +398,7 @@ cudaError_t launch_q(const QuantArgs& a, cudaStream_t s) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !a.advance) return e;
   advance_seq_lens_kernel<<<(a.batch + 127) / 128, 128, 0, s>>>(a.seq_lens, a.batch, a.n_new,
-                                                               a.max_tokens);
+                                                               a.max_tokens, a.k_channels);
   return cudaGetLastError();
 }
 

@@ -25,6 +25,8 @@ KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORK
     KVQ_ERR_CUDA = range(6)
 KVQ_F16, KVQ_BF16 = 0, 1
 KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM = 0, 1, 2
+KVQ_AXIS_TOKEN, KVQ_AXIS_CHANNEL = 0, 1
+KVQ_CHANNEL_BLOCK = 32
 HEADER_BYTES = 256  # workspace header: sticky device error word first
 
 
@@ -36,7 +38,8 @@ class KvqError(RuntimeError):
 
 class kvq_plane(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32),
-                ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("fmt", ctypes.c_int32)]
+                ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("fmt", ctypes.c_int32),
+                ("axis", ctypes.c_int32)]
 
 
 class kvq_cache(ctypes.Structure):
@@ -251,6 +254,9 @@ class QuantizedKVCache:
     seq_lens: int32 [B] on the device; fmt: KVQ_FMT_INT, KVQ_FMT_FP8_E4M3
     (bits 8: E4M3 codes, zero points 0) or KVQ_FMT_INT8_SYM (bits 8: two's
     complement codes, zero points 0).
+    k_axis: KVQ_AXIS_TOKEN, or KVQ_AXIS_CHANNEL (K grouped per channel over
+    blocks of KVQ_CHANNEL_BLOCK tokens: k_meta fp16 [B, H_kv,
+    max_tokens / KVQ_CHANNEL_BLOCK, head_dim, 2]; group_size is V's).
     """
     batch: int
     kv_heads: int
@@ -264,10 +270,11 @@ class QuantizedKVCache:
     v_meta: Optional[torch.Tensor]
     seq_lens: torch.Tensor
     fmt: int = KVQ_FMT_INT
+    k_axis: int = KVQ_AXIS_TOKEN
 
     @classmethod
     def allocate(cls, batch, kv_heads, head_dim, max_tokens, bits, group_size, device="cuda",
-                 fmt: int = KVQ_FMT_INT):
+                 fmt: int = KVQ_FMT_INT, k_axis: int = KVQ_AXIS_TOKEN):
         rb = head_dim * bits // 8
         shape = (batch, kv_heads, max_tokens, rb)
         k = torch.empty(shape, dtype=torch.uint8, device=device)
@@ -275,20 +282,24 @@ class QuantizedKVCache:
         km = vm = None
         if bits != 16:
             mshape = (batch, kv_heads, max_tokens, head_dim // group_size, 2)
-            km = torch.empty(mshape, dtype=torch.float16, device=device)
+            kshape = ((batch, kv_heads, max_tokens // KVQ_CHANNEL_BLOCK, head_dim, 2)
+                      if k_axis == KVQ_AXIS_CHANNEL else mshape)
+            km = torch.empty(kshape, dtype=torch.float16, device=device)
             vm = torch.empty(mshape, dtype=torch.float16, device=device)
         lens = torch.zeros(batch, dtype=torch.int32, device=device)
         return cls(batch, kv_heads, head_dim, max_tokens, bits, group_size, k, v, km, vm, lens,
-                   fmt)
+                   fmt, k_axis)
 
     def struct(self) -> kvq_cache:
         c = kvq_cache()
         c.batch, c.kv_heads, c.head_dim, c.max_tokens = (self.batch, self.kv_heads,
                                                          self.head_dim, self.max_tokens)
         c.k = kvq_plane(self.bits, self.group_size, self.k_codes.data_ptr(),
-                        self.k_meta.data_ptr() if self.k_meta is not None else None, self.fmt)
+                        self.k_meta.data_ptr() if self.k_meta is not None else None, self.fmt,
+                        self.k_axis)
         c.v = kvq_plane(self.bits, self.group_size, self.v_codes.data_ptr(),
-                        self.v_meta.data_ptr() if self.v_meta is not None else None, self.fmt)
+                        self.v_meta.data_ptr() if self.v_meta is not None else None, self.fmt,
+                        KVQ_AXIS_TOKEN)
         c.seq_lens = self.seq_lens.data_ptr()
         return c
 

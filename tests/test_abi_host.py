@@ -235,6 +235,38 @@ def test_sym8_planes_validated(kvq):
     assert _status(kvq.kvq_decode_workspace_bytes, c, 8) == kvq.KVQ_ERR_UNSUPPORTED  # 4 x 4
 
 
+def test_channel_axis_validated(kvq):
+    """KVQ_AXIS_CHANNEL is for the K plane of an integer-code cache only; an
+    append to it must be whole 32-token blocks; the one-call decode step does
+    not take it (single tokens go to an fp16 segment); unknown axes are
+    rejected."""
+    fake = ctypes.c_void_p(0x60000)
+
+    def append_status(c, n):
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, n, 1, None)
+    c = _fake_cache(kvq, bits=4)
+    c.k.axis = kvq.KVQ_AXIS_CHANNEL
+    assert append_status(c, 5) == kvq.KVQ_ERR_INVALID_ARG      # not a whole block
+    c.k.group_size = 7                                          # not used on that plane
+    assert append_status(c, 33) == kvq.KVQ_ERR_INVALID_ARG
+    c = _fake_cache(kvq, bits=4)
+    c.v.axis = kvq.KVQ_AXIS_CHANNEL
+    assert append_status(c, 32) == kvq.KVQ_ERR_UNSUPPORTED     # V stays per token
+    c = _fake_cache(kvq, bits=8)
+    c.k.axis = kvq.KVQ_AXIS_CHANNEL
+    c.k.fmt = c.v.fmt = kvq.KVQ_FMT_FP8_E4M3
+    assert append_status(c, 32) == kvq.KVQ_ERR_UNSUPPORTED     # integer codes only
+    c = _fake_cache(kvq, bits=4)
+    c.k.axis = 3
+    assert append_status(c, 32) == kvq.KVQ_ERR_INVALID_ARG
+    c = _fake_cache(kvq, bits=4, group=64, kv_heads=2)
+    c.k.axis = kvq.KVQ_AXIS_CHANNEL
+    ws = ctypes.c_void_p(0x80000)
+    st = kvq.lib.kvq_decode_step((kvq.kvq_cache * 1)(c), fake, fake, fake, kvq.KVQ_F16, 8,
+                                 ctypes.c_float(0.08), fake, None, 0, ws, 1 << 30, None)
+    assert st == kvq.KVQ_ERR_UNSUPPORTED
+
+
 def test_chunk_entry_points_reject_bad_arguments(kvq):
     lib = kvq.lib
     fake = ctypes.c_void_p(0x10000)
