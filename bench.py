@@ -63,10 +63,13 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def bytes_per_head_token(bits: int, group: int, head_dim: int = 128) -> int:
-    """K plus V bytes of one (sequence, KV head, token): codes + (s, z) pairs."""
+def bytes_per_head_token(bits: int, group: int, head_dim: int = 128,
+                         k_channels: bool = False) -> int:
+    """K plus V bytes of one (sequence, KV head, token): codes + (s, z) pairs
+    (per-channel K: head_dim pairs per 32-token block, 16 bytes a token)."""
     meta = 0 if bits == 16 else (head_dim // group) * 4
-    return 2 * (head_dim * bits // 8 + meta)
+    kmeta = head_dim * 4 // 32 if k_channels else meta
+    return 2 * (head_dim * bits // 8) + meta + kmeta
 
 
 def kernel_source_hash() -> str:
@@ -159,6 +162,28 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- reference arm
 
+def channel_oracle_pairs(wl, k, v, q, pairs):
+    """Oracle inputs of (sequence, KV head) pairs of a per-channel-K workload:
+    K quantized per channel over 32-token blocks, V per token; each entry is
+    (q patterns [1, g, D], the one-pair segment, its length)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    g = wl.group_ratio
+    out = []
+    for b, h in pairs:
+        kk = k[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        vv = v[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        kc, km = oracle.quantize_cache_channels(kk, wl.bits)
+        vc, vm = oracle.quantize_rows(vv, wl.group, wl.bits)
+        seg = dict(k_codes=kc[None, None], k_meta=km[None, None], v_codes=vc[None, None],
+                   v_meta=vm[None, None], bits=wl.bits, group=wl.group, k_channels=True)
+        qh = q[b, h * g:(h + 1) * g].cpu().contiguous().view(torch.int16).numpy()
+        out.append((qh.view(np.uint16)[None], seg, [np.array([kk.shape[0]])]))
+    return out
+
+
 def run_reference(args, wl):
     """The CPU oracle as it stands, on this host's cores: each step attends
     one (sequence, KV head) of the workload after appending one token."""
@@ -187,6 +212,28 @@ def run_reference(args, wl):
                   f"{wl.n_chunks} chunks as FP16/INT4/INT2 segments ({int(counts[0])}/"
                   f"{int(counts[1])}/{int(counts[2])} chunks); tokens/s = steps / kv_heads "
                   f"({wl.kv_heads}) / seconds")
+        print(json.dumps(reference_line(args, wl, value, el, sample)), flush=True)
+        return
+    if wl.k_axis == "channel":
+        sub = wl.scaled(batch=1, kv_heads=min(wl.kv_heads, 4),
+                        q_heads=min(wl.kv_heads, 4) * wl.group_ratio)
+        k, v = workloads.kv_tokens(sub, wl.context, "cpu")
+        q = workloads.queries(sub, "cpu")
+        prepared = channel_oracle_pairs(wl, k, v, q, [(0, h) for h in range(sub.kv_heads)])
+
+        def kpc_step(i):
+            qh, seg, lens = prepared[i % len(prepared)]
+            oracle.decode_attention(qh, wl.q_dtype == "bf16", [seg], lens, 128 ** -0.5)
+        for i in range(args.warmup):
+            kpc_step(i)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            kpc_step(i)
+        el = time.perf_counter() - t0
+        value = args.steps / wl.kv_heads / el
+        sample = (f"each step: one (sequence, KV head) of {wl.name}: attention of "
+                  f"{wl.group_ratio} query heads over {wl.context} tokens, K per channel; "
+                  f"tokens/s = steps / kv_heads ({wl.kv_heads}) / seconds")
         print(json.dumps(reference_line(args, wl, value, el, sample)), flush=True)
         return
     sub = wl.scaled(batch=1, kv_heads=min(wl.kv_heads, 4),
@@ -248,6 +295,7 @@ def workload_config(wl, extra=None):
            "kv_heads": wl.kv_heads, "head_dim": wl.head_dim, "context": wl.context,
            "bits": wl.bits, "group": wl.group, "q_dtype": wl.q_dtype,
            **({"format": FMT_NAME[wl.fmt]} if wl.fmt != "int" else {}),
+           **({"k_grouping": "per channel, 32-token blocks"} if wl.k_axis == "channel" else {}),
            "episode_steps": wl.steps if wl.append else 0}
     if extra:
         cfg.update(extra)
@@ -265,6 +313,21 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
     import oracle
     g = wl.group_ratio
     pairs = [(b, h) for b in range(min(wl.batch, 2)) for h in range(min(wl.kv_heads, 4))]
+    if wl.k_axis == "channel":
+        prep = channel_oracle_pairs(wl, k, v, q, pairs)
+        n = 0
+        t0 = time.perf_counter()
+        while True:
+            qh, seg, lens = prep[n % len(prep)]
+            oracle.decode_attention(qh, wl.q_dtype == "bf16", [seg], lens, 128 ** -0.5)
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds and n >= 2:
+                break
+        return {"value": n / wl.kv_heads / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": f"{n} (sequence, KV head) attentions of {wl.name} over "
+                          f"{k.shape[2]} tokens (K per channel) cycling over {len(prep)} pairs, "
+                          f"{el:.1f} s on one host thread; tokens/s = pairs / kv_heads / seconds"}
     prepared = []
     for b, h in pairs:
         kk = k[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
@@ -389,6 +452,7 @@ def run_kvq(args, wl, rank, world, local_rank):
     ctx = wl.context
     episode = wl.steps if wl.append else min(wl.steps, 100)
     wlr = rank_workload(wl, rank)
+    kpc = wl.k_axis == "channel"  # K grouped per channel over 32-token blocks
 
     # ---- resident inputs (untimed set-up)
     prefill = None  # set by the single-cache set-up below
@@ -414,7 +478,7 @@ def run_kvq(args, wl, rank, world, local_rank):
         k, v = workloads.kv_tokens(wlr, ctx, dev)
         cache = kvq.QuantizedKVCache.allocate(
             B, H, D, max_tokens, wl.bits, wl.group, dev,
-            fmt=FMT_CODE[wl.fmt])
+            fmt=FMT_CODE[wl.fmt], k_axis=1 if kpc else 0)
         cache.seq_lens.zero_()
         kvq.kvq_quantize_append(cache, k, v, ctx, advance_seq_lens=True)
         base_lens = cache.seq_lens.clone()
@@ -431,7 +495,7 @@ def run_kvq(args, wl, rank, world, local_rank):
         pf_ev[1].record()
         torch.cuda.synchronize()
         pf_us = pf_ev[0].elapsed_time(pf_ev[1]) * 1e3 / pf_reps
-        pf_bytes = B * H * ctx * (2 * D * 2 + bytes_per_head_token(wl.bits, wl.group, D))
+        pf_bytes = B * H * ctx * (2 * D * 2 + bytes_per_head_token(wl.bits, wl.group, D, kpc))
         prefill = {"tokens": B * ctx, "us": pf_us, "bytes": pf_bytes,
                    "gbs": pf_bytes / (pf_us / 1e6) / 1e9, "kernel": "quantize_bulk_kernel",
                    "note": "fp16 K and V read + packed codes and (s, z) written, per launch "
@@ -485,7 +549,7 @@ def run_kvq(args, wl, rank, world, local_rank):
             return sum(int(ln.sum()) * H * bytes_per_head_token(bits, wl.group, D)
                        for ln, bits in zip(seg_lens, seg_bits))
         L = ctx + (s % episode) + 1 if wl.append else ctx
-        return B * H * L * bytes_per_head_token(wl.bits, wl.group, D)
+        return B * H * L * bytes_per_head_token(wl.bits, wl.group, D, kpc)
 
     # ---- warm-up (eager; also makes the one-time kernel attribute settings)
     for s in range(args.warmup):
@@ -697,7 +761,8 @@ def run_kvq(args, wl, rank, world, local_rank):
         if wl.chunk_tokens:
             line["cpu_baseline"] = cpu_baseline_mixed(wl, k, v, qs[0], args.cpu_seconds, wlr)
         else:
-            line["cpu_baseline"] = cpu_baseline(wl, k, v, kn[0, 0], kn[0, 1], qs[0],
+            line["cpu_baseline"] = cpu_baseline(wl, k, v, kn[0, 0] if kn is not None else None,
+                                                kn[0, 1] if kn is not None else None, qs[0],
                                                 args.cpu_seconds)
     return line
 

@@ -52,12 +52,16 @@ namespace kvq {
 
 namespace {
 
-template <int BITS, int GE, int GR>
+template <int BITS, int GE, int GR, bool KPC = false>
 struct TmCfg {
   static constexpr int D = kHeadDim;
-  static constexpr int NG = D / GE;                    // groups per token
+  static constexpr int NG = D / GE;                    // V groups per token (and K's, per token)
   static constexpr int RB = D * code_bits(BITS) / 8;   // code bytes per token
   static constexpr int MB = (BITS == 16) ? 0 : NG * 4; // (s, z) bytes per token
+  // K meta bytes per token: per-channel K (KPC) stores D (s, z) pairs per
+  // block of kChannelBlock tokens, i.e. 16 bytes per token, and a stage is
+  // one block
+  static constexpr int MBK = KPC ? D * 4 / kChannelBlock : MB;
   static constexpr int KC = RB / 4;                    // K bytes of a lane (32 dims)
   static constexpr int KW = KC / 4;
   static constexpr int VB = RB / 8;                    // V bytes of a lane (16 dims)
@@ -76,7 +80,7 @@ struct TmCfg {
   static constexpr int NO = GPV ? 1 : NP;              // accumulator n-tiles
   static constexpr int SUB = (BITS == 16) ? 1 : 2;     // 16-token sub-tiles per stage
   static constexpr int STOK = SUB * kTile;
-  static constexpr int STAGE = 2 * STOK * RB + 2 * STOK * MB;
+  static constexpr int STAGE = 2 * STOK * RB + STOK * (MBK + MB);
   // header: mbarriers (<= 512 B), the g query rows as fp16, the column sums
   // of q, unit id and fail flag
   static constexpr int HDR_BARS = 0, HDR_Q = 512, HDR_QS = HDR_Q + GR * D * 2;
@@ -108,6 +112,11 @@ struct TmCfg {
   static_assert(HDR_NEW % 16 == 0 && NEW_STRIDE % 16 == 0, "aligned new-token rows");
   static_assert(WordPairs<BITS>::kPairs * KW == 16, "16 K pairs per lane and token");
   static_assert(CrossPairs<BITS>::kOut * VW == 16, "16 V dims per lane and token");
+  // per-channel K: a stage is one block, and lane tig owns head tig % g with
+  // its QK columns 2 tig (hi part) and 2 tig + 1 (lo part)
+  static_assert(!KPC || ((BITS == 2 || BITS == 4 || BITS == 8) && STOK == kChannelBlock &&
+                         CPH == 2 && HS == 1),
+                "per-channel K: integer codes, one block per stage, two columns per head");
 };
 
 // Token of MMA row r (0 .. 15) of a 16-token sub-tile.
@@ -135,10 +144,10 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& r0, uin
   r1 = pack_h2(x1, n1);
 }
 
-template <int BITS, int GE, int GR>
-__global__ void __launch_bounds__(kWarps * 32, TmCfg<BITS, GE, GR>::MIN_CTAS)
+template <int BITS, int GE, int GR, bool KPC>
+__global__ void __launch_bounds__(kWarps * 32, TmCfg<BITS, GE, GR, KPC>::MIN_CTAS)
 decode_tm_kernel(const __grid_constant__ SplitParams P) {
-  using C = TmCfg<BITS, GE, GR>;
+  using C = TmCfg<BITS, GE, GR, KPC>;
   using WP = WordPairs<BITS>;
   using XP = CrossPairs<BITS>;
   // the zero point the codes are read against: symmetric INT8 codes are read
@@ -239,12 +248,12 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   constexpr int NCOPY = C::MB > 0 ? 4 : 2;
   const long long row0 = ((long long)b * a.kv_heads + kvh) * seg.max_tokens + w0;
   const int cp_j = lane < NCOPY ? lane : 0;
-  const int cp_rb = (cp_j < 2) ? C::RB : C::MB;  // bytes per token of the plane
+  const int cp_rb = (cp_j < 2) ? C::RB : (cp_j == 2 ? C::MBK : C::MB);  // bytes per token
   const uint8_t* cp_src = (cp_j == 0 ? seg.k_codes : cp_j == 1 ? seg.v_codes
                            : cp_j == 2 ? seg.k_meta : seg.v_meta) + row0 * cp_rb;
   const uint32_t cp_off = cp_j == 0 ? 0u : cp_j == 1 ? (uint32_t)(C::STOK * C::RB)
                           : cp_j == 2 ? (uint32_t)(2 * C::STOK * C::RB)
-                                      : (uint32_t)(2 * C::STOK * C::RB + C::STOK * C::MB);
+                                      : (uint32_t)(2 * C::STOK * C::RB + C::STOK * C::MBK);
   const uint32_t cp_bytes = (uint32_t)(C::STOK * cp_rb);
   const size_t cp_stride = (size_t)(kWarps * C::STOK) * cp_rb;
   // stage i of this warp into ring slot st (all lanes call it together)
@@ -262,7 +271,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
 
   // ---- decode step: quantize the new K (lanes 0-15) and V (16-31) rows of
   // this KV head into shared memory, then copy them to the cache
-  if constexpr (BITS != 16) {
+  if constexpr (BITS != 16 && !KPC) {
     if (append_here && warp == 0) {
       const int vh = lane >> 4, l16 = lane & 15;
       const __half* src = (vh ? a.v_new : a.k_new) + ((long long)b * a.kv_heads + kvh) * D;
@@ -283,7 +292,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   stage_queries<GR>(a, b, kvh, q_sm, t);
   __syncthreads();
   // column sums of q in the QK MMA's units (it returns 2^(EMAX - 24) sum q c)
-  if constexpr (BITS != 16) {
+  if constexpr (BITS != 16 && !KPC) {
     if (t < 64) {
       const int r = t >> 3, part = t & 7;
       const __half* qr = q_sm + ((r / CPH) % GR) * D + (r % NG) * GE + part * (GE / 8);
@@ -300,7 +309,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   // B fragments of QK: pair p = 2 ks + h of this lane's chunk, column gid;
   // each element scaled by 2^(EMAX - e) for the exponent e of its code
   uint32_t qb[C::QB_SMEM ? 1 : 8][2];
-  {
+  if constexpr (!KPC) {
     const __half* qrow = q_sm + qh * D + 32 * tig;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -322,8 +331,46 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     }
     if constexpr (C::QB_SMEM) __syncthreads();
   }
-  const float qsA = (BITS != 16) ? qs_sm[2 * tig] : 0.f;
-  const float qsB = (BITS != 16) ? qs_sm[2 * tig + 1] : 0.f;
+  const float qsA = (BITS != 16 && !KPC) ? qs_sm[2 * tig] : 0.f;
+  const float qsB = (BITS != 16 && !KPC) ? qs_sm[2 * tig + 1] : 0.f;
+
+  // Per-channel K: the QK B fragments of a block are q * s_d for the block's
+  // channel scales, in two fp16 parts (hi in the even columns, lo = the fp32
+  // remainder in the odd ones: q * s is exact in fp32, hi + lo keeps 22
+  // bits), each element times 2^(EMAX - e) as above; the zero points enter
+  // as the block's bias sum_d q_d s_d z_d per head, in the MMA's units.
+  float kbias = 0.f;
+  auto kpc_rebuild = [&](const uint8_t* sKm) {
+    if constexpr (KPC) {
+      const __half* qrow = q_sm + qh * D + 32 * tig;
+      const __half2* szr = reinterpret_cast<const __half2*>(sKm) + 32 * tig;  // (s, z) of its channels
+      const bool lo_part = gid & 1;
+      float bp = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int p = 2 * ks + h;
+          const int j = p % WP::kPairs;
+          const int d0 = (p / WP::kPairs) * WP::kDims + WP::dim(j, 0);
+          const int d1 = (p / WP::kPairs) * WP::kDims + WP::dim(j, 1);
+          const float f = pow2f(C::EMAX - WP::exp(j));
+          const float2 sz0 = __half22float2(szr[d0]), sz1 = __half22float2(szr[d1]);
+          const float qs0 = __half2float(qrow[d0]) * sz0.x, qs1 = __half2float(qrow[d1]) * sz1.x;
+          bp = fmaf(qs0, sz0.y, fmaf(qs1, sz1.y, bp));
+          const float v0 = qs0 * f, v1 = qs1 * f;
+          const uint32_t hh = pack_h2(v0, v1);
+          const float2 hf = __half22float2(u32_as_h2(hh));
+          qb[ks][h] = lo_part ? pack_h2(v0 - hf.x, v1 - hf.y) : hh;
+        }
+      }
+      // the head's sum over its 128 channels: the four lanes of this gid,
+      // then from a lane holding the owned head (gid = 2 h)
+      bp += __shfl_xor_sync(0xffffffffu, bp, 1);
+      bp += __shfl_xor_sync(0xffffffffu, bp, 2);
+      kbias = __shfl_sync(0xffffffffu, bp, 8 * own_h[0]) * pow2f(C::EMAX - 24);
+    }
+  };
 
   // ---- running state.  m_ref (per owned head) is a reference point at
   // least as large as every score seen, so p = 2^(x - m_ref) <= 1 and
@@ -352,6 +399,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
                         const uint8_t* sVm, int n_valid) {
     constexpr bool FULL = decltype(full_tag)::value;
     constexpr int NS = C::SUB;
+    kpc_rebuild(sKm);
     auto valid = [&](int tok) { return FULL || tok < n_valid; };  // tok: 0 .. STOK-1
     // V rows past the valid length may hold any bytes.  Integer codes are
     // finite and meet a zero weight; raw fp16 and e4m3 bytes can be NaN or
@@ -416,6 +464,8 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         if constexpr (BITS == 16) {
           v[0] = s_acc[2 * r];
           if constexpr (HS == 2) v[HS - 1] = s_acc[2 * r + 1];
+        } else if constexpr (KPC) {
+          v[0] = s_acc[2 * r] + s_acc[2 * r + 1] - kbias;
         } else if constexpr (NG == 1) {
           const float2 sz = __half22float2(*reinterpret_cast<const __half2*>(sKm + tok * C::MB));
           v[0] = sz.x * fmaf(-zero_of(sz.y), qsA, s_acc[2 * r]);
@@ -577,8 +627,8 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     const uint8_t* sK = stages + st * C::STAGE;
     const uint8_t* sV = sK + C::STOK * C::RB;
     const uint8_t* sKm = sK + 2 * C::STOK * C::RB;
-    const uint8_t* sVm = sKm + C::STOK * C::MB;
-    if constexpr (BITS != 16) {
+    const uint8_t* sVm = sKm + C::STOK * C::MBK;
+    if constexpr (BITS != 16 && !KPC) {
       if (i == patch_i) {
         // the new token's row, from the quantized copy in shared memory
         uint32_t* dK = reinterpret_cast<uint32_t*>(stages + st * C::STAGE + patch_row * C::RB);
@@ -693,9 +743,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   if (t == 0) release_counters(counters);
 }
 
-template <int BITS, int GE, int GR>
+template <int BITS, int GE, int GR, bool KPC>
 cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
-  using C = TmCfg<BITS, GE, GR>;
+  using C = TmCfg<BITS, GE, GR, KPC>;
   // the shared-memory opt-in is a per-device function attribute: set it once
   // per device (bit i of the mask = device i)
   static std::atomic<unsigned long long> attr_set{0};
@@ -703,7 +753,7 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tm_kernel<BITS, GE, GR>,
+    cudaError_t e = cudaFuncSetAttribute(decode_tm_kernel<BITS, GE, GR, KPC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
@@ -712,9 +762,13 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   const long long units = (long long)seg.n_split * a.kv_heads * a.batch;
   const long long slots = 148LL * C::MIN_CTAS;  // one wave of persistent CTAs
   const unsigned grid = (unsigned)(units < slots ? units : slots);
-  decode_tm_kernel<BITS, GE, GR><<<grid, kWarps * 32, C::SMEM, s>>>(P);
+  decode_tm_kernel<BITS, GE, GR, KPC><<<grid, kWarps * 32, C::SMEM, s>>>(P);
   return cudaGetLastError();
 }
+
+// Per-channel K (G is V's group size): the (bits, G, g) whose QK columns
+// give lane tig head tig % g in two columns (see TmCfg).
+#define KVQ_TM_KPC_FORMATS(X) X(4, 64, 4) X(8, 128, 1) X(4, 128, 4) X(4, 128, 1)
 
 // Every (bits, G, g) with NG * g <= 8 that the cache formats allow.
 #define KVQ_TM_FORMATS(X)                                              \
@@ -734,20 +788,29 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
 }  // namespace
 
 bool decode_tm_supported(int bits, int group, int group_ratio, bool kpc) {
-  if (kpc) return false;
 #define KVQ_X(B, G_, R) \
   if (bits == B && group == G_ && group_ratio == R) return true;
+  if (kpc) {
+    KVQ_TM_KPC_FORMATS(KVQ_X)
+    return false;
+  }
   KVQ_TM_FORMATS(KVQ_X)
 #undef KVQ_X
   return false;
 }
 
 int decode_tm_ctas_per_sm(int bits, int group, int group_ratio, bool kpc) {
-  if (kpc) return 0;
 #define KVQ_X(B, G_, R) \
-  if (bits == B && group == G_ && group_ratio == R) return TmCfg<B, G_, R>::MIN_CTAS;
+  if (bits == B && group == G_ && group_ratio == R) return TmCfg<B, G_, R, false>::MIN_CTAS;
+#define KVQ_XK(B, G_, R) \
+  if (bits == B && group == G_ && group_ratio == R) return TmCfg<B, G_, R, true>::MIN_CTAS;
+  if (kpc) {
+    KVQ_TM_KPC_FORMATS(KVQ_XK)
+    return 0;
+  }
   KVQ_TM_FORMATS(KVQ_X)
 #undef KVQ_X
+#undef KVQ_XK
   return 0;
 }
 
@@ -755,9 +818,16 @@ cudaError_t launch_decode_tm(const DecodeArgs& a, const SegView& seg, cudaStream
   const int bits = seg.bits, group = (seg.bits == 16) ? kHeadDim : seg.group;
   const int g = a.group_ratio;
 #define KVQ_X(B, G_, R) \
-  if (bits == B && group == G_ && g == R) return launch_tm<B, G_, R>(a, seg, s);
+  if (bits == B && group == G_ && g == R) return launch_tm<B, G_, R, false>(a, seg, s);
+#define KVQ_XK(B, G_, R) \
+  if (bits == B && group == G_ && g == R) return launch_tm<B, G_, R, true>(a, seg, s);
+  if (seg.k_channels) {
+    KVQ_TM_KPC_FORMATS(KVQ_XK)
+    return cudaErrorInvalidValue;
+  }
   KVQ_TM_FORMATS(KVQ_X)
 #undef KVQ_X
+#undef KVQ_XK
   return cudaErrorInvalidValue;
 }
 

@@ -62,3 +62,56 @@ def test_quantize_channels_bit_exact(kvq, bits, G, H, T):
         assert np.array_equal(c.v_meta[b, :, p].cpu().numpy().view(np.uint16), vm[b, :, :n])
         assert (c.k_codes[b, :, :st] == 0xA5).all()
         assert (c.k_meta[b, :, :st // TB].view(torch.int16) == -1).all()
+
+
+def _kpc_segment(k, v, bits, G):
+    kc, km = oracle.quantize_cache_channels(f16_bits(k), bits)
+    vc, vm = oracle.quantize_cache(f16_bits(v), G, bits)
+    return dict(k_codes=kc, k_meta=km, v_codes=vc, v_meta=vm, bits=bits, group=G,
+                k_channels=True)
+
+
+@pytest.mark.parametrize("bits,G,g", [(4, 64, 4), (8, 128, 1), (4, 128, 4), (4, 128, 1)])
+def test_decode_attention_channels(kvq, bits, G, g):
+    """Attention over a per-channel-K cache (lengths on block boundaries, one
+    sequence empty), then together with an fp16 residual segment holding
+    each sequence's unfinished block: the KIVI-style pair."""
+    from gpu_util import assert_close, fill_cache, fill_fp16_segment, q_bits
+    H = 2
+    wl = workloads.WORKLOADS["llama3_8b_gqa_int4"].scaled(kv_heads=H, q_heads=H * g, bits=bits,
+                                                          group=G)
+    lens = [320, 64, 0, 32]
+    B, T = len(lens), max(lens)
+    k, v = workloads.kv_tokens(wl, T, DEV, batch=B)
+    k[1, 0, 40, 3] = 250.0  # an outlier channel value inside one block
+    q = workloads.queries(wl, DEV, batch=B)
+    c = _alloc(kvq, B, H, 320, bits, G)
+    fill_cache(kvq, c, k, v, lens)
+    seg = _kpc_segment(k, v, bits, G)
+    ws = kvq.alloc_workspace(c, H * g, 0, device=DEV)
+    out = torch.full((B, H * g, 128), float("nan"), device=DEV)
+    lse = torch.full((B, H * g), float("nan"), device=DEV)
+    kvq.kvq_decode_attention(c, q, out, lse, ws)
+    torch.cuda.synchronize()
+    assert kvq.workspace_error_word(ws) == 0
+    ref, lref = oracle.decode_attention(q_bits(q), False, [seg], [lens], 128 ** -0.5)
+    mask = np.array([n > 0 for n in lens])
+    assert_close(out, ref, lse, lref, mask=mask, what=f"kpc b{bits} G{G} g{g}")
+    # with the unfinished blocks in an fp16 segment
+    rlens = [17, 31, 5, 0]
+    kr, vr = workloads.kv_tokens(wl, 32, DEV, stream_extra=7, batch=B)
+    r = kvq.QuantizedKVCache.allocate(B, H, 128, 64, 16, 128, DEV)
+    fill_fp16_segment(r, kr, vr, rlens)
+    segs = [c, r]
+    ws2 = kvq.alloc_workspace(segs, H * g, 0, device=DEV)
+    out2 = torch.full((B, H * g, 128), float("nan"), device=DEV)
+    lse2 = torch.full((B, H * g), float("nan"), device=DEV)
+    kvq.kvq_decode_attention(segs, q, out2, lse2, ws2)
+    torch.cuda.synchronize()
+    assert kvq.workspace_error_word(ws2) == 0
+    rseg = dict(k_codes=f16_bits(kr).view(np.uint8).reshape(B, H, 32, -1),
+                v_codes=f16_bits(vr).view(np.uint8).reshape(B, H, 32, -1), k_meta=None,
+                v_meta=None, bits=16, group=128)
+    ref2, lref2 = oracle.decode_attention(q_bits(q), False, [seg, rseg], [lens, rlens],
+                                          128 ** -0.5)
+    assert_close(out2, ref2, lse2, lref2, what=f"kpc + fp16 residual b{bits} G{G} g{g}")

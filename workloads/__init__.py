@@ -70,6 +70,8 @@ class DecodeWorkload:
     low_bits: Tuple[int, ...] = ()   # bit-widths of the two quantized classes
     fmt: str = "int"          # code format: "int" (asymmetric integer), "fp8" (E4M3, bits 8)
     #                           or "sym8" (symmetric INT8, bits 8)
+    k_axis: str = "token"     # K grouping: "token" (groups along head_dim) or "channel"
+    #                           (per channel over 32-token blocks; attention only)
 
     @property
     def group_ratio(self) -> int:
@@ -119,6 +121,10 @@ WORKLOADS = {
         context=4096, bits=8, group=128, q_dtype="bf16", steps=100, append=True, seed=2,
         k_outliers=Outliers(factor=10.0, fraction=0.01),
         v_outliers=Outliers(factor=10.0, fraction=0.01), fmt="sym8"),
+    "llama3_8b_gqa_int4_kpc": DecodeWorkload(
+        name="llama3_8b_gqa_int4_kpc", batch=32, q_heads=32, kv_heads=8, head_dim=128,
+        context=8192, bits=4, group=64, q_dtype="f16", steps=100, append=False, seed=3,
+        k_outliers=Outliers(factor=15.0, per_head=4), v_sigma=0.5, k_axis="channel"),
     "long_gqa_int4": DecodeWorkload(
         name="long_gqa_int4", batch=1, q_heads=32, kv_heads=8, head_dim=128,
         context=131072, bits=4, group=64, q_dtype="f16", steps=256, append=True, seed=5,
