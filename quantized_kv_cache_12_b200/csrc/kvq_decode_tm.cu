@@ -93,7 +93,9 @@ struct TmCfg {
   // (8 x 32 lanes x 8 B) instead of being held in 16 registers per thread
   static constexpr bool QB_SMEM = false;
   static constexpr int HDR_QF = HDR_NEW + 2 * NEW_STRIDE;
-  static constexpr int HDR_BYTES = (((QB_SMEM ? HDR_QF + 8 * 32 * 8 : HDR_QF) + 127) / 128) * 128;
+  // per-channel K: the g query rows times each dim's 2^(EMAX - e), fp16
+  static constexpr int QF_BYTES = QB_SMEM ? 8 * 32 * 8 : (KPC ? GR * D * 2 : 0);
+  static constexpr int HDR_BYTES = ((HDR_QF + QF_BYTES + 127) / 128) * 128;
   // four CTAs per SM (128 registers a thread) where two stages per warp fit
   // in a quarter of the SM's shared memory (4 x (56 KB + 1 KB reserved)
   // <= 228 KB), else three
@@ -340,35 +342,79 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   // bits), each element times 2^(EMAX - e) as above; the zero points enter
   // as the block's bias sum_d q_d s_d z_d per head, in the MMA's units.
   float kbias = 0.f;
+  __half* qf_tab = reinterpret_cast<__half*>(smem + C::HDR_QF);  // [GR][D] (per-channel K)
+  if constexpr (KPC) {
+    // q * 2^(EMAX - e) of each dim, once per unit (lanes of one head and
+    // chunk write the same values)
+    const __half* qrow = q_sm + qh * D + 32 * tig;
+    __half* qfrow = qf_tab + qh * D + 32 * tig;
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      const int j = p % WP::kPairs;
+      const int blk = (p / WP::kPairs) * WP::kDims;
+      const float f = pow2f(C::EMAX - WP::exp(j));
+      qfrow[blk + WP::dim(j, 0)] = __float2half_rn(__half2float(qrow[blk + WP::dim(j, 0)]) * f);
+      qfrow[blk + WP::dim(j, 1)] = __float2half_rn(__half2float(qrow[blk + WP::dim(j, 1)]) * f);
+    }
+    __syncthreads();
+  }
+  // d = fp32 a * b + c for fp16 a, b (the product is exact)
+  auto fma_h = [](__half a, __half b, float c) {
+    float d;
+    asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(__half_as_ushort(a)),
+        "h"(__half_as_ushort(b)), "f"(c));
+    return d;
+  };
   auto kpc_rebuild = [&](const uint8_t* sKm) {
     if constexpr (KPC) {
-      const __half* qrow = q_sm + qh * D + 32 * tig;
+      constexpr int KD = WP::kDims;  // dims of one code word
+      const __half* qfrow = qf_tab + qh * D + 32 * tig;
       const __half2* szr = reinterpret_cast<const __half2*>(sKm) + 32 * tig;  // (s, z) of its channels
       const bool lo_part = gid & 1;
-      float bp = 0.f;
+      // bias terms by pair position j: their query values carry 2^(EMAX - e_j)
+      float bpj[WP::kPairs];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
+      for (int j = 0; j < WP::kPairs; ++j) bpj[j] = 0.f;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int p = 2 * ks + h;
-          const int j = p % WP::kPairs;
-          const int d0 = (p / WP::kPairs) * WP::kDims + WP::dim(j, 0);
-          const int d1 = (p / WP::kPairs) * WP::kDims + WP::dim(j, 1);
-          const float f = pow2f(C::EMAX - WP::exp(j));
-          const float2 sz0 = __half22float2(szr[d0]), sz1 = __half22float2(szr[d1]);
-          const float qs0 = __half2float(qrow[d0]) * sz0.x, qs1 = __half2float(qrow[d1]) * sz1.x;
-          bp = fmaf(qs0, sz0.y, fmaf(qs1, sz1.y, bp));
-          const float v0 = qs0 * f, v1 = qs1 * f;
-          const uint32_t hh = pack_h2(v0, v1);
-          const float2 hf = __half22float2(u32_as_h2(hh));
-          qb[ks][h] = lo_part ? pack_h2(v0 - hf.x, v1 - hf.y) : hh;
+      for (int wb = 0; wb < 32 / KD; ++wb) {
+        // this word block's query values and (s, z) pairs, in vector loads
+        __half qd[KD];
+        __half2 szd[KD];
+#pragma unroll
+        for (int i = 0; i < KD; i += 8)
+          *reinterpret_cast<uint4*>(&qd[i]) = *reinterpret_cast<const uint4*>(qfrow + wb * KD + i);
+        if constexpr (KD == 4)
+          *reinterpret_cast<uint2*>(&qd[0]) = *reinterpret_cast<const uint2*>(qfrow + wb * KD);
+#pragma unroll
+        for (int i = 0; i < KD; i += 4)
+          *reinterpret_cast<uint4*>(&szd[i]) = *reinterpret_cast<const uint4*>(szr + wb * KD + i);
+#pragma unroll
+        for (int j = 0; j < WP::kPairs; ++j) {
+          const int p = wb * WP::kPairs + j;
+          const __half2 sz0 = szd[WP::dim(j, 0)], sz1 = szd[WP::dim(j, 1)];
+          const __half q0 = qd[WP::dim(j, 0)], q1 = qd[WP::dim(j, 1)];
+          const __half2 hi = __hmul2(__halves2half2(q0, q1), __lows2half2(sz0, sz1));
+          const float r0 = fma_h(q0, __low2half(sz0), -__low2float(hi));
+          const float r1 = fma_h(q1, __low2half(sz1), -__high2float(hi));
+          const __half2 lo = __floats2half2_rn(r0, r1);
+          float b = bpj[j];
+          b = fma_h(__low2half(hi), __high2half(sz0), b);
+          b = fma_h(__high2half(hi), __high2half(sz1), b);
+          b = fma_h(__low2half(lo), __high2half(sz0), b);
+          bpj[j] = fma_h(__high2half(lo), __high2half(sz1), b);
+          qb[p / 2][p % 2] = h2_as_u32(lo_part ? lo : hi);
         }
       }
-      // the head's sum over its 128 channels: the four lanes of this gid,
-      // then from a lane holding the owned head (gid = 2 h)
+      // in the MMA's units, 2^(EMAX - 24) sum q s z: each term's query value
+      // already carries 2^(EMAX - e_j), so it takes 2^(e_j - 24); then the
+      // head's sum over its 128 channels (the four lanes of this gid), read
+      // from a lane holding the owned head (gid = 2 h)
+      float bp = 0.f;
+#pragma unroll
+      for (int j = 0; j < WP::kPairs; ++j) bp = fmaf(bpj[j], pow2f(WP::exp(j) - 24), bp);
       bp += __shfl_xor_sync(0xffffffffu, bp, 1);
       bp += __shfl_xor_sync(0xffffffffu, bp, 2);
-      kbias = __shfl_sync(0xffffffffu, bp, 8 * own_h[0]) * pow2f(C::EMAX - 24);
+      kbias = __shfl_sync(0xffffffffu, bp, 8 * own_h[0]);
     }
   };
 

@@ -297,7 +297,7 @@ __global__ void advance_seq_lens_kernel(int32_t* seq_lens, int batch, int n_new,
 // channel): one CTA per block of kChannelBlock new tokens of one (sequence,
 // KV head), thread d owning channel d.  The block's rows are staged in shared
 // memory; each channel's min, max, scale, zero point and codes follow the
-// same fp32 steps as the per-token groups (IEEE division, round half to
+// same fp32 steps as the per-token groups (the IEEE quotient, round half to
 // even), then the codes are packed along the token rows.  A sequence whose
 // length is not a multiple of the block is skipped; blocks at or past
 // max_tokens (a multiple of 64) are dropped whole.
@@ -329,12 +329,14 @@ __global__ void __launch_bounds__(kHeadDim) quantize_k_channels_kernel(const Qua
   const float s32 = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), qmax), 1e-5f);
   const __half s16 = __float2half_ru(s32);
   const float s = __half2float(s16);
-  float zf = __fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.0f);
+  const float r = __frcp_rn(s);  // x / s below: the correction step on RN(1/s) (IEEE quotient)
+  float zf = __fadd_rn(rintf(div_rn(-mn, s, r)), 0.0f);
   zf = fminf(fmaxf(zf, -65504.0f), 65504.0f);
   const __half z16 = __float2half_rn(zf);
   const float z = __half2float(z16);
+#pragma unroll 8
   for (int t = 0; t < TB; ++t) {
-    const float c = __fadd_rn(rintf(__fdiv_rn(__half2float(xs[t][d]), s)), z);
+    const float c = __fadd_rn(rintf(div_rn(__half2float(xs[t][d]), s, r)), z);
     cs[t][d] = (uint8_t)fminf(fmaxf(c, 0.0f), qmax);
   }
   const long long blk = (long long)bh * (a.max_tokens / TB) + pos0 / TB;
