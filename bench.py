@@ -128,6 +128,13 @@ class ClockSampler:
             if len(parts) == 6:
                 self.samples.append((time.time(), parts))
 
+    def wait_first(self, timeout_s: float):
+        """Return once the first sample has arrived (nvidia-smi takes a moment
+        to start), or after timeout_s."""
+        t_end = time.time() + timeout_s
+        while self.proc is not None and not self.samples and time.time() < t_end:
+            time.sleep(0.02)
+
     def stop(self):
         if self.proc is not None:
             self.proc.terminate()
@@ -609,7 +616,8 @@ def run_kvq(args, wl, rank, world, local_rank):
 
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_id) if rank == 0 else None
-    time.sleep(0.3 if sampler else 0)
+    if sampler:
+        sampler.wait_first(10.0)  # sampling is running before the timed region opens
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     if world > 1:
