@@ -463,19 +463,46 @@ def run_kvq(args, wl, rank, world, local_rank):
 
     # ---- resident inputs (untimed set-up)
     prefill = None  # set by the single-cache set-up below
+    chunk_timing = None  # set by the chunk-level mixed set-up below
     if wl.chunk_tokens:
         # chunk-level mixed precision: search, reorder, quantize the prompt
         # into FP16 / INT4 / INT2 segments once; each step attends over them
         emb, qemb = workloads.chunk_embeddings(wlr, dev)
         cbits = torch.empty((B, wl.n_chunks), dtype=torch.uint8, device=dev)
         kvq.kvq_chunk_assign(emb, qemb, wl.alpha, wl.beta, cbits)
-        del emb, qemb
         k, v = workloads.kv_tokens(wlr, ctx, dev)
         segs = [kvq.QuantizedKVCache.allocate(B, H, D, workloads.round_up(ctx, 64), bits,
                                               wl.group, dev) for bits in (16,) + wl.low_bits]
         perm = torch.empty((B, wl.n_chunks), dtype=torch.int32, device=dev)
         kvq.kvq_chunk_reorder(segs, k, v, wl.chunk_tokens, cbits, perm)
         seg_lens = [c.seq_lens.cpu().numpy().astype(np.int64) for c in segs]
+        # the chunk search and the reorder (one-off per prompt), timed on their
+        # own, 3 launches each: the search reads the chunk and query embeddings
+        # once; the reorder reads the fp16 K and V once and writes each class's
+        # codes and (s, z) once
+        ca_ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        torch.cuda.synchronize()
+        ca_ev[0].record()
+        for _ in range(3):
+            kvq.kvq_chunk_assign(emb, qemb, wl.alpha, wl.beta, cbits)
+        ca_ev[1].record()
+        for _ in range(3):
+            kvq.kvq_chunk_reorder(segs, k, v, wl.chunk_tokens, cbits, perm)
+        ca_ev[2].record()
+        torch.cuda.synchronize()
+        assign_us = ca_ev[0].elapsed_time(ca_ev[1]) * 1e3 / 3
+        reorder_us = ca_ev[1].elapsed_time(ca_ev[2]) * 1e3 / 3
+        assign_bytes = emb.numel() * 4 + qemb.numel() * 4
+        reorder_bytes = B * H * ctx * 2 * D * 2 + sum(
+            int(ln.sum()) * H * bytes_per_head_token(c.bits, wl.group, D)
+            for ln, c in zip(seg_lens, segs))
+        chunk_timing = {"assign_us": assign_us, "assign_bytes": assign_bytes,
+                        "reorder_us": reorder_us, "reorder_bytes": reorder_bytes,
+                        "reorder_gbs": reorder_bytes / (reorder_us / 1e6) / 1e9,
+                        "kernels": "chunk_assign_kernel, chunk_partition_kernel + chunk_bulk_kernel",
+                        "note": "3 launches each; reorder bytes: fp16 K and V read + every "
+                                "segment's codes and (s, z) written"}
+        del emb, qemb
         seg_bits = [c.bits for c in segs]
         k_cpu_src = (k, v, cbits)
         base_lens = None
@@ -763,6 +790,8 @@ def run_kvq(args, wl, rank, world, local_rank):
                         "copy streams"},
         "gpu_launches": launches_per_step * args.steps,
         **({"prefill_quantize": {**prefill, "frac": prefill["gbs"] / peak}} if prefill else {}),
+        **({"chunk_reorder": {**chunk_timing, "frac": chunk_timing["reorder_gbs"] / peak}}
+           if chunk_timing else {}),
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

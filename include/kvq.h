@@ -347,7 +347,9 @@ kvq_status kvq_decode_attention_noalloc(const kvq_cache *segs, int32_t n_segs,
  *   query_emb: device fp32 [batch][emb_dim]
  *   sim_out:   device fp64 [batch][n_chunks], or NULL
  *   chunk_bits_out: device u8 [batch][n_chunks] (16, 4 or 2)
- * n_chunks <= 4096.  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_CUDA.
+ * n_chunks <= 4096; emb_dim a multiple of 4, at most 4096; chunk_emb 16-byte
+ * aligned.  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED (emb_dim),
+ * KVQ_ERR_CUDA.
  */
 kvq_status kvq_chunk_assign(const float *chunk_emb, const float *query_emb,
                             int32_t batch, int32_t n_chunks, int32_t emb_dim,

@@ -418,6 +418,8 @@ kvq_status kvq_chunk_assign(const float* chunk_emb, const float* query_emb, int3
     return KVQ_ERR_INVALID_ARG;
   if (batch <= 0 || n_chunks <= 0 || n_chunks > 4096 || emb_dim <= 0) return KVQ_ERR_INVALID_ARG;
   if (!isfinite(alpha) || !isfinite(beta)) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(chunk_emb)) return KVQ_ERR_INVALID_ARG;
+  if (emb_dim % 4 != 0 || emb_dim > 4096) return KVQ_ERR_UNSUPPORTED;
   cudaError_t e = kvq::launch_chunk_assign(chunk_emb, query_emb, batch, n_chunks, emb_dim, alpha,
                                            beta, sim_out, chunk_bits_out,
                                            static_cast<cudaStream_t>(stream));

@@ -244,6 +244,31 @@ __device__ __forceinline__ void quantize8(const uint4 raw, uint32_t& codes_lo,
     codes_hi = 0;
 }
 
+// ---- the bulk kernels' shared-memory ring (prefill quantize, chunk
+// reorder): per-lane cp.async copies of 16 bytes, committed in groups
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Ring offset of 16-byte chunk k (0..15) of row ri of a unit: position
+// k ^ (bit 3 of k) ^ (6 for odd rows) within the row.  16-byte shared-memory
+// accesses are served eight lanes (two rows) at a time; for a copy step
+// (lane (ri, li) moves chunk 4c + li) and for a read step (lane (ri, li)
+// reads chunk 4li + c) the eight chunks of each such pair of rows then fall
+// in eight different groups of four banks: no bank conflicts.
+__device__ __forceinline__ uint32_t bulk_slot_off(int ri, int k) {
+  return (uint32_t)(ri * (kHeadDim * 2) + ((k ^ ((k >> 3) & 1) ^ ((ri & 1) * 6)) * 16));
+}
+
+
 // Quantize one 16-byte slice of a row and store it.  lane16 = index of the
 // slice within the 128-value row (0..15); all 32 lanes of the warp must call
 // this together (the group reduction uses warp shuffles); `active` false

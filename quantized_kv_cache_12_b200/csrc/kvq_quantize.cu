@@ -87,17 +87,6 @@ constexpr int kBulkDepth = 4;                     // ring slots per warp
 constexpr int kBulkWarps = 4;                     // warps per CTA
 constexpr int kUnitBytes = kUnitRows * kHeadDim * 2;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // A position in a warp's unit sequence: plane row (side, b, h) and unit j
 // within it, plus this lane's token t.  Moving one unit steps the addresses
 // derived from it by a constant; they are rebuilt from (side, b, h, j) only
@@ -185,16 +174,6 @@ struct BulkDst {
     }
   }
 };
-
-// Ring offset of 16-byte chunk k (0..15) of row ri of a unit: position
-// k ^ (bit 3 of k) ^ (6 for odd rows) within the row.  16-byte shared-memory
-// accesses are served eight lanes (two rows) at a time; for a copy step
-// (lane (ri, li) moves chunk 4c + li) and for a read step (lane (ri, li)
-// reads chunk 4li + c) the eight chunks of each such pair of rows then fall
-// in eight different groups of four banks: no bank conflicts.
-__device__ __forceinline__ uint32_t bulk_slot_off(int ri, int k) {
-  return (uint32_t)(ri * (kHeadDim * 2) + ((k ^ ((k >> 3) & 1) ^ ((ri & 1) * 6)) * 16));
-}
 
 __device__ __forceinline__ void bulk_issue(const QuantArgs& a, const BulkSrc& c,
                                            const uint32_t (&soff)[kBulkNV / 8], int li,

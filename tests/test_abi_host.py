@@ -274,6 +274,13 @@ def test_chunk_entry_points_reject_bad_arguments(kvq):
         kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_chunk_assign(fake, fake, 8, 5000, 768, 0.6, 0.1, None, fake, None) == \
         kvq.KVQ_ERR_INVALID_ARG
+    # the staged embedding copies need 16-byte rows and fit emb_dim <= 4096
+    assert lib.kvq_chunk_assign(fake, fake, 8, 1024, 770, 0.6, 0.1, None, fake, None) == \
+        kvq.KVQ_ERR_UNSUPPORTED
+    assert lib.kvq_chunk_assign(fake, fake, 8, 1024, 4100, 0.6, 0.1, None, fake, None) == \
+        kvq.KVQ_ERR_UNSUPPORTED
+    assert lib.kvq_chunk_assign(ctypes.c_void_p(0x10004), fake, 8, 1024, 768, 0.6, 0.1, None,
+                                fake, None) == kvq.KVQ_ERR_INVALID_ARG
     segs = (kvq.kvq_cache * 3)(_fake_cache(kvq, bits=16, max_tokens=1024),
                                _fake_cache(kvq, bits=4, group=32, max_tokens=1024),
                                _fake_cache(kvq, bits=2, group=32, max_tokens=1024))

@@ -37,6 +37,25 @@ def test_chunk_assign_bit_exact(kvq):
         assert counts[0] >= 1 and counts.sum() == n
 
 
+def test_chunk_assign_rounds_and_partial_tile(kvq):
+    """More chunks than threads of the CTA (several rounds) and an embedding
+    width that leaves a partial last tile: similarities bit for bit."""
+    B, n, E = 2, 2500, 100
+    g = torch.Generator(device=DEV)
+    g.manual_seed(17)
+    emb = torch.randn((B, n, E), generator=g, device=DEV)
+    qemb = torch.randn((B, E), generator=g, device=DEV)
+    bits = torch.zeros((B, n), dtype=torch.uint8, device=DEV)
+    sim = torch.zeros((B, n), dtype=torch.float64, device=DEV)
+    kvq.kvq_chunk_assign(emb, qemb, 0.6, 0.1, bits, sim)
+    torch.cuda.synchronize()
+    e, qe = emb.cpu().numpy(), qemb.cpu().numpy()
+    for b in range(B):
+        s_ref, c_ref = oracle.chunk_assign(e[b], qe[b], 0.6, 0.1)
+        assert np.array_equal(sim[b].cpu().numpy().view(np.uint64), s_ref.view(np.uint64))
+        assert np.array_equal(bits[b].cpu().numpy(), c_ref)
+
+
 def test_chunk_assign_threshold_toy(kvq, golden_dir):
     import json
     import os
@@ -185,3 +204,15 @@ def test_cocktail_full_size_sampled(kvq):
                                         128 ** -0.5)
         ref[b, h], lref[b, h], mask[b, h] = r[0, 0], lr[0, 0], True
     assert_close(out, ref, lse, lref, mask=mask, what="cocktail full size")
+
+
+@pytest.mark.parametrize("G", [64, 128])
+def test_reorder_chunk16_groups(kvq, G):
+    """16-token chunks (two 8-row units each) and the larger group sizes:
+    gathered rows and codes byte for byte against the oracle's partition."""
+    wl = workloads.WORKLOADS["cocktail_mixed"].scaled(kv_heads=2, q_heads=2, chunk_tokens=16)
+    B, H, ctx = 3, 2, 1024
+    rng = np.random.default_rng(3)
+    cbits = rng.choice(np.array([16, 4, 2], np.uint8), size=(B, ctx // 16), p=[0.2, 0.3, 0.5])
+    cbits[2, :] = 4
+    _check_reorder(kvq, wl, B, H, ctx, cbits, G=G)
