@@ -687,15 +687,25 @@ def run_kvq(args, wl, rank, world, local_rank):
     # step's input copy overlaps the previous step's attention and its output
     # copy overlaps the next one's; the attention calls stay in order on the
     # compute stream.
-    kn_h = kn.cpu().pin_memory() if kn is not None else None
-    qs_h = qs.cpu().pin_memory()
-    k_d = [torch.empty_like(kn[0, 0]) for _ in range(2)] if kn is not None else None
-    v_d = [torch.empty_like(kn[0, 1]) for _ in range(2)] if kn is not None else None
-    q_d = [torch.empty_like(qs[0]) for _ in range(2)]
-    out_d = [torch.empty_like(out) for _ in range(2)]
-    lse_d = [torch.empty_like(lse) for _ in range(2)]
-    out_h = [torch.empty((B, Hq, D), dtype=torch.float32).pin_memory() for _ in range(2)]
-    lse_h = [torch.empty((B, Hq), dtype=torch.float32).pin_memory() for _ in range(2)]
+    # inputs of a step (new K and V token, q) in one pinned host row and one
+    # device slot, results (out, lse) likewise: one copy each way per step
+    nk = kn[0, 0].numel() if kn is not None else 0  # fp16 elements of k_new (= v_new)
+    nq = qs[0].numel()
+    in_h = torch.empty((episode, 2 * nk + nq), dtype=torch.float16).pin_memory()
+    for e in range(episode):
+        if kn is not None:
+            in_h[e, :nk].copy_(kn[e, 0].reshape(-1))
+            in_h[e, nk:2 * nk].copy_(kn[e, 1].reshape(-1))
+        in_h[e, 2 * nk:].copy_(qs[e].reshape(-1))
+    in_d = [torch.empty(2 * nk + nq, dtype=torch.float16, device=dev) for _ in range(2)]
+    k_d = [b[:nk].view(kn[0, 0].shape) for b in in_d] if kn is not None else None
+    v_d = [b[nk:2 * nk].view(kn[0, 1].shape) for b in in_d] if kn is not None else None
+    q_d = [b[2 * nk:].view(qs[0].shape) for b in in_d]
+    no, nl = out.numel(), lse.numel()
+    res_d = [torch.empty(no + nl, dtype=torch.float32, device=dev) for _ in range(2)]
+    out_d = [r[:no].view(out.shape) for r in res_d]
+    lse_d = [r[no:].view(lse.shape) for r in res_d]
+    res_h = [torch.empty(no + nl, dtype=torch.float32).pin_memory() for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     in_ready = [torch.cuda.Event() for _ in range(2)]
     done = [torch.cuda.Event() for _ in range(2)]
@@ -707,11 +717,8 @@ def run_kvq(args, wl, rank, world, local_rank):
         e, j = s % episode, n % 2
         with torch.cuda.stream(s_in):
             if n >= 2:
-                s_in.wait_event(done[j])  # step n-2 no longer reads buffer j
-            if wl.append:
-                k_d[j].copy_(kn_h[e, 0], non_blocking=True)
-                v_d[j].copy_(kn_h[e, 1], non_blocking=True)
-            q_d[j].copy_(qs_h[e], non_blocking=True)
+                s_in.wait_event(done[j])  # step n-2 no longer reads slot j
+            in_d[j].copy_(in_h[e], non_blocking=True)
             in_ready[j].record(s_in)
         stream.wait_event(in_ready[j])
         if n >= 2:
@@ -726,8 +733,7 @@ def run_kvq(args, wl, rank, world, local_rank):
         done[j].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(done[j])
-            out_h[j].copy_(out_d[j], non_blocking=True)
-            lse_h[j].copy_(lse_d[j], non_blocking=True)
+            res_h[j].copy_(res_d[j], non_blocking=True)
             out_read[j].record(s_out)
 
     for n in range(args.warmup):
@@ -786,8 +792,8 @@ def run_kvq(args, wl, rank, world, local_rank):
         "e2e": {"value": B * args.steps * world / (e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "kvq_decode_step (append workloads) or kvq_decode_attention through the "
-                        "Python binding; pinned host buffers, copies double-buffered on two "
-                        "copy streams"},
+                        "Python binding; pinned host buffers, one input and one result copy per "
+                        "step, double-buffered on two copy streams"},
         "gpu_launches": launches_per_step * args.steps,
         **({"prefill_quantize": {**prefill, "frac": prefill["gbs"] / peak}} if prefill else {}),
         **({"chunk_reorder": {**chunk_timing, "frac": chunk_timing["reorder_gbs"] / peak}}

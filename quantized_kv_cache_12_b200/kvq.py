@@ -105,7 +105,9 @@ def _check(status: int, where: str):
 
 
 def _caches(segs) -> ctypes.Array:
-    if isinstance(segs, (QuantizedKVCache, kvq_cache)):
+    if isinstance(segs, QuantizedKVCache):
+        return segs.struct_array()
+    if isinstance(segs, kvq_cache):
         segs = [segs]
     arr = (kvq_cache * len(segs))()
     for i, s in enumerate(segs):
@@ -289,6 +291,15 @@ class QuantizedKVCache:
         lens = torch.zeros(batch, dtype=torch.int32, device=device)
         return cls(batch, kv_heads, head_dim, max_tokens, bits, group_size, k, v, km, vm, lens,
                    fmt, k_axis)
+
+    def struct_array(self) -> ctypes.Array:
+        """A one-element kvq_cache array for this cache, built on first use
+        (the planes' tensors are allocated once and never replaced)."""
+        arr = self.__dict__.get("_struct_array")
+        if arr is None:
+            arr = (kvq_cache * 1)(self.struct())
+            self.__dict__["_struct_array"] = arr
+        return arr
 
     def struct(self) -> kvq_cache:
         c = kvq_cache()
