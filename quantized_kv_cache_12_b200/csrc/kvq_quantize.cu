@@ -283,9 +283,8 @@ __global__ void advance_seq_lens_kernel(int32_t* seq_lens, int batch, int n_new,
 template <int BITS>
 __global__ void __launch_bounds__(kHeadDim) quantize_k_channels_kernel(const QuantArgs a) {
   constexpr int D = kHeadDim, TB = kChannelBlock, RB = D * BITS / 8;
-  constexpr int EPW = 32 / BITS;  // codes per 32-bit word
   __shared__ __align__(16) __half xs[TB][D];
-  __shared__ uint8_t cs[TB][D];
+  __shared__ __align__(16) uint8_t cs[TB][D];
   const int bh = blockIdx.y;
   const int j = blockIdx.x;
   const int b = bh / a.kv_heads;
@@ -298,34 +297,69 @@ __global__ void __launch_bounds__(kHeadDim) quantize_k_channels_kernel(const Qua
     reinterpret_cast<uint4*>(&xs[0][0])[i] = src[i];
   __syncthreads();
   const int d = threadIdx.x;
-  float mn = __half2float(xs[0][d]), mx = mn;
+  float x[TB];
+#pragma unroll
+  for (int t = 0; t < TB; ++t) x[t] = __half2float(xs[t][d]);
+  float mn = x[0], mx = x[0];
+#pragma unroll
   for (int t = 1; t < TB; ++t) {
-    const float v = __half2float(xs[t][d]);
-    mn = v < mn ? v : mn;
-    mx = v > mx ? v : mx;
+    mn = x[t] < mn ? x[t] : mn;
+    mx = x[t] > mx ? x[t] : mx;
   }
-  constexpr float qmax = float((1 << BITS) - 1);
-  const float s32 = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), qmax), 1e-5f);
+  constexpr int qmax_i = (1 << BITS) - 1;
+  constexpr float qmax = float(qmax_i), kInvQmax = 1.0f / qmax;
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  // x / d below: the correction step on RN(1/d), the IEEE quotient
+  const float s32 = fmaxf(div_rn(__fsub_rn(mx, mn), qmax, kInvQmax), 1e-5f);
   const __half s16 = __float2half_ru(s32);
   const float s = __half2float(s16);
-  const float r = __frcp_rn(s);  // x / s below: the correction step on RN(1/s) (IEEE quotient)
+  const float r = __frcp_rn(s);
   float zf = __fadd_rn(rintf(div_rn(-mn, s, r)), 0.0f);
   zf = fminf(fmaxf(zf, -65504.0f), 65504.0f);
   const __half z16 = __float2half_rn(zf);
   const float z = __half2float(z16);
-#pragma unroll 8
-  for (int t = 0; t < TB; ++t) {
-    const float c = __fadd_rn(rintf(div_rn(__half2float(xs[t][d]), s, r)), z);
-    cs[t][d] = (uint8_t)fminf(fmaxf(c, 0.0f), qmax);
+  const float zm = z - kMagic;
+  // code = clamp(rint(x / s) + z, 0, qmax): (q + M) + z is M + the code, whose
+  // low mantissa bits are the code, when the channel needs no clamp (|z| <=
+  // 2048 and its top code, (q_max + M) + (z - M), <= qmax; see the per-token
+  // quantizer), else with the quotient clamped first
+  const float top = __fadd_rn(__fadd_rn(div_rn(mx, s, r), kMagic), zm);
+  if (fabsf(zf) <= 2048.0f && top <= qmax) {
+#pragma unroll
+    for (int t = 0; t < TB; ++t)
+      cs[t][d] = (uint8_t)__float_as_uint(__fadd_rn(__fadd_rn(div_rn(x[t], s, r), kMagic), z));
+  } else {
+    const float lo = -z, hi = __fadd_rn(qmax, -z);
+#pragma unroll
+    for (int t = 0; t < TB; ++t) {
+      const float q = fminf(fmaxf(div_rn(x[t], s, r), lo), hi);
+      cs[t][d] = (uint8_t)__float_as_uint(__fadd_rn(__fadd_rn(q, kMagic), z));
+    }
   }
   const long long blk = (long long)bh * (a.max_tokens / TB) + pos0 / TB;
   reinterpret_cast<__half2*>(a.k_meta)[blk * D + d] = __halves2half2(s16, z16);
   __syncthreads();
+  // rows of codes: whole words read from the byte codes
   for (int i = threadIdx.x; i < TB * RB / 4; i += blockDim.x) {
     const int t = i / (RB / 4), w = i % (RB / 4);
-    uint32_t word = 0;
+    uint32_t word;
+    if constexpr (BITS == 8) {
+      word = *reinterpret_cast<const uint32_t*>(&cs[t][4 * w]);
+    } else if constexpr (BITS == 4) {
+      const uint2 v = *reinterpret_cast<const uint2*>(&cs[t][8 * w]);
+      const uint32_t a0 = v.x | (v.x >> 4), a1 = v.y | (v.y >> 4);  // bytes 0, 2: code pairs
+      word = __byte_perm(a0, a1, 0x6420);
+    } else {
+      const uint4 v = *reinterpret_cast<const uint4*>(&cs[t][16 * w]);
+      const uint32_t q4[4] = {v.x, v.y, v.z, v.w};
+      uint32_t b[4];
 #pragma unroll
-    for (int e = 0; e < EPW; ++e) word |= (uint32_t)cs[t][w * EPW + e] << (e * BITS);
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t c1 = q4[k] | (q4[k] >> 6);  // bytes 0, 2: code pairs
+        b[k] = c1 | (c1 >> 12);                    // byte 0: four codes
+      }
+      word = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    }
     reinterpret_cast<uint32_t*>(a.k_codes + ((long long)bh * a.max_tokens + pos0 + t) * RB)[w] =
         word;
   }
