@@ -74,7 +74,10 @@ def bytes_per_head_token(bits: int, group: int, head_dim: int = 128,
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("kvq_decode.cu", "kvq_decode_tm.cu", "kvq_decode_common.cuh", "kvq_device.cuh"):
+    # the decode kernels' sources and the headers they compile (the fused
+    # append's quantizer included)
+    for f in ("kvq_decode.cu", "kvq_decode_tm.cu", "kvq_decode_common.cuh", "kvq_device.cuh",
+              "kvq_quant_core.cuh", "kvq_internal.h"):
         with open(os.path.join(ROOT, "quantized_kv_cache_12_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
