@@ -129,7 +129,7 @@ typedef struct kvq_plane {
 typedef struct kvq_cache {
     int32_t batch;
     int32_t kv_heads;
-    int32_t head_dim;   /* 128 in this build                                */
+    int32_t head_dim;   /* 128 (the kernels are compiled for it)            */
     int32_t max_tokens; /* token capacity per (sequence, KV head)           */
     kvq_plane k;
     kvq_plane v;
@@ -149,7 +149,7 @@ const char *kvq_version(void);
  * bytes per element), per plane and layer, with bits/8 bytes per element
  * plus 4 bytes of (scale, zero) per group.
  * Returns KVQ_ERR_INVALID_ARG on non-positive sizes or null outputs,
- * KVQ_ERR_UNSUPPORTED on a (bits, G, head_dim) this build does not pack.
+ * KVQ_ERR_UNSUPPORTED on a (bits, G, head_dim) the library does not pack.
  */
 kvq_status kvq_plane_bytes(int32_t batch, int32_t kv_heads, int32_t head_dim,
                            int32_t max_tokens, int32_t bits, int32_t group_size,

@@ -29,7 +29,7 @@ def declared_functions():
     return sorted(names)
 
 
-def test_header_declares_the_north_star_entry_points():
+def test_header_declares_the_three_hot_path_entry_points():
     names = declared_functions()
     for n in ("kvq_quantize_append", "kvq_decode_attention", "kvq_chunk_reorder"):
         assert n in names
