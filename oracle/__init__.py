@@ -66,6 +66,12 @@ def _load():
         lib.kvqo_quantize_group_fp8.argtypes = [P, i32, P, P]
         lib.kvqo_quantize_rows_fp8.argtypes = [P, i64, i32, i32, P, P]
         lib.kvqo_quantize_group_sym8.argtypes = [P, i32, P, P]
+        lib.kvqo_e5m2_to_f64.restype = ctypes.c_double
+        lib.kvqo_e5m2_to_f64.argtypes = [ctypes.c_uint8]
+        lib.kvqo_f32_to_e5m2.restype = ctypes.c_uint8
+        lib.kvqo_f32_to_e5m2.argtypes = [ctypes.c_float]
+        lib.kvqo_quantize_group_e5m2.argtypes = [P, i32, P, P]
+        lib.kvqo_quantize_rows_e5m2.argtypes = [P, i64, i32, i32, P, P]
         lib.kvqo_quantize_block_channels.argtypes = [P, i32, i32, i32, P, P]
         lib.kvqo_dequantize_block_channels.argtypes = [P, P, i32, i32, i32, P]
         lib.kvqo_quantize_rows_sym8.argtypes = [P, i64, i32, i32, P, P]
@@ -133,7 +139,7 @@ def quantize_group(x16, bits: int):
 
 
 # code formats of the C functions' `fmt` argument
-FMT_CODES = {"int": 0, "fp8": 1, "sym8": 2}
+FMT_CODES = {"int": 0, "fp8": 1, "sym8": 2, "e5m2": 3}
 
 
 def quantize_rows(x16, group: int, bits: int, fmt: str = "int"):
@@ -141,7 +147,8 @@ def quantize_rows(x16, group: int, bits: int, fmt: str = "int"):
     meta [N, D/G, 2] uint16 holding the (scale, zero) fp16 patterns).
     fmt "fp8": E4M3 codes (bits 8) with zero point 0 (KV-cache page, FP8);
     fmt "sym8": symmetric INT8, two's complement codes (bits 8) with zero
-    point 0 (KV-cache page, INT8 item)."""
+    point 0 (KV-cache page, INT8 item); fmt "e5m2": E5M2 codes (bits 8) with
+    zero point 0 (KV-cache page, FP8)."""
     lib = _load()
     x16 = _c(x16, np.uint16)
     N, D = x16.shape
@@ -154,6 +161,9 @@ def quantize_rows(x16, group: int, bits: int, fmt: str = "int"):
     elif fmt == "sym8":
         assert bits == 8
         lib.kvqo_quantize_rows_sym8(_p(x16), N, D, group, _p(codes), _p(meta))
+    elif fmt == "e5m2":
+        assert bits == 8
+        lib.kvqo_quantize_rows_e5m2(_p(x16), N, D, group, _p(codes), _p(meta))
     else:
         assert fmt == "int", fmt
         lib.kvqo_quantize_rows(_p(x16), N, D, group, bits, _p(codes), _p(meta))
@@ -162,7 +172,8 @@ def quantize_rows(x16, group: int, bits: int, fmt: str = "int"):
 
 def dequantize_rows(codes, meta, D: int, group: int, bits: int, fmt: str = "int") -> np.ndarray:
     """Packed rows -> fp64 [N, D]: x_hat = (c - z) * s, e4m3(c) * s for
-    fmt "fp8", int8(c) * s for fmt "sym8" (all exact in fp64)."""
+    fmt "fp8", int8(c) * s for fmt "sym8", e5m2(c) * s for fmt "e5m2" (all
+    exact in fp64)."""
     lib = _load()
     codes = _c(codes, np.uint8)
     N = codes.shape[0]
@@ -200,6 +211,32 @@ def quantize_group_fp8(x16):
     code = np.zeros(x16.size, np.uint8)
     s = np.zeros(1, np.uint16)
     lib.kvqo_quantize_group_fp8(_p(x16), x16.size, _p(code), _p(s))
+    return code, int(s[0])
+
+
+def e5m2_to_f64(codes) -> np.ndarray:
+    """E5M2 codes (uint8) -> fp64 values (infinities and NaN in E = 31)."""
+    lib = _load()
+    c = _c(codes, np.uint8).ravel()
+    return np.array([lib.kvqo_e5m2_to_f64(int(v)) for v in c], np.float64).reshape(
+        np.shape(codes))
+
+
+def f32_to_e5m2(x) -> np.ndarray:
+    """fp32 values -> nearest E5M2 codes, ties to even, saturating at 57344."""
+    lib = _load()
+    x = _c(x, np.float32)
+    return np.array([lib.kvqo_f32_to_e5m2(float(v)) for v in x.ravel()], np.uint8).reshape(
+        x.shape)
+
+
+def quantize_group_e5m2(x16):
+    """One group of fp16 bit patterns -> (E5M2 codes uint8[G], s16)."""
+    lib = _load()
+    x16 = _c(x16, np.uint16)
+    code = np.zeros(x16.size, np.uint8)
+    s = np.zeros(1, np.uint16)
+    lib.kvqo_quantize_group_e5m2(_p(x16), x16.size, _p(code), _p(s))
     return code, int(s[0])
 
 
@@ -316,7 +353,7 @@ def attention_blocks(q, K, V, scale: float, bounds: Sequence[int]):
 def attention_packed(q16, q_is_bf16: bool, k_codes, k_meta, k_bits: int, v_codes, v_meta,
                      v_bits: int, group: int, L: int, scale: float, fmt: str = "int"):
     """Attention of g query heads over one packed (sequence, KV head) cache
-    (fmt "fp8": E4M3 codes for K and V; "sym8": symmetric INT8)."""
+    (fmt "fp8": E4M3 codes for K and V; "sym8": symmetric INT8; "e5m2": E5M2)."""
     lib = _load()
     q16 = _c(q16, np.uint16)
     g, D = q16.shape
@@ -385,7 +422,7 @@ def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: fl
     q16: [B, Hq, D] fp16/bf16 patterns.  segments: list of dicts with numpy
     arrays ``k_codes``/``v_codes`` [B, Hkv, T, row_bytes], ``k_meta``/``v_meta``
     [B, Hkv, T, D/G, 2] (None for bits 16), ``bits``, ``group`` and optionally
-    ``fmt`` ("int", the default, "fp8" or "sym8") and ``k_channels`` (True: K
+    ``fmt`` ("int", the default, "fp8", "sym8" or "e5m2") and ``k_channels`` (True: K
     is per-channel, ``k_meta`` [B, Hkv, T / KPC_BLOCK, D, 2], lengths multiples
     of KPC_BLOCK).
     seq_lens_per_seg: list of int arrays [B].  The segments of a sequence are

@@ -82,9 +82,14 @@
  *       blocks are quantized: the tokens of an unfinished block stay in
  *       fp16 (a separate fp16 segment) until the block is complete.  V keeps
  *       its per-token groups along head_dim (R6).
+ *   R17 FP8 E5M2 ([P2'] item 1 names E5M2 beside E4M3): the format with
+ *       bias 15, two mantissa bits, largest finite 57344, infinities and NaN
+ *       in E = 31; the scale as R14 with 57344 for 448 (s = max(amax /
+ *       57344, 1e-5), fp16 rounded up); codes the nearest E5M2 value of x /
+ *       s, ties to even, saturating at +-57344 (never an infinity).
  *
  * Code formats (the `fmt` arguments): 0 asymmetric integer codes of `bits`
- * bits (R1-R7), 1 E4M3 (R14), 2 symmetric INT8 (R15).
+ * bits (R1-R7), 1 E4M3 (R14), 2 symmetric INT8 (R15), 3 E5M2 (R17).
  */
 #include <math.h>
 #include <stdint.h>
@@ -349,6 +354,84 @@ void kvqo_quantize_rows_fp8(const uint16_t *x, int64_t n_rows, int D, int G, uin
         }
 }
 
+/* ------------------------------------------------------------------------ */
+/* FP8 E5M2 ([P2'] item 1; R17), written from the format definition.       */
+/* ------------------------------------------------------------------------ */
+
+/* Value of an E5M2 code: (-1)^S * 2^(E-15) * (1 + M/4) for 1 <= E <= 30,
+ * (-1)^S * 2^-14 * M/4 for E = 0; E = 31 is infinity (M = 0) or NaN. */
+double kvqo_e5m2_to_f64(uint8_t c)
+{
+    int sgn = c >> 7, e = (c >> 2) & 31, m = c & 3;
+    double v;
+    if (e == 31)
+        v = (m == 0) ? INFINITY : NAN;
+    else if (e == 0)
+        v = ldexp((double)m, -16);
+    else
+        v = ldexp((double)(4 + m), e - 17);
+    return sgn ? -v : v;
+}
+
+/* Nearest E5M2 code to an fp32 value, ties to even, magnitudes past the
+ * largest finite value (57344) saturated to it; NaN gives S.11111.11. */
+uint8_t kvqo_f32_to_e5m2(float x)
+{
+    if (isnan(x))
+        return 0x7F;
+    uint8_t sgn = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    /* the spacing of E5M2 values around a: 2^-16 below 2^-14, else 2^(e-2) */
+    int e = (a > 0.0) ? (int)floor(log2(a)) : -100;
+    if (a > 0.0 && ldexp(1.0, e) > a) /* guard log2 rounding */
+        e -= 1;
+    if (a > 0.0 && ldexp(1.0, e + 1) <= a)
+        e += 1;
+    double quantum = ldexp(1.0, (e < -14 ? -14 : e) - 2);
+    double r = rint(a / quantum) * quantum; /* a / quantum is exact */
+    if (r > 57344.0)
+        r = 57344.0;
+    if (r == 0.0)
+        return sgn;
+    int re = (int)floor(log2(r));
+    if (re < -14)
+        return (uint8_t)(sgn | (uint8_t)(r / ldexp(1.0, -16))); /* subnormal */
+    int m = (int)(r / ldexp(1.0, re - 2)) - 4;
+    return (uint8_t)(sgn | ((re + 15) << 2) | m);
+}
+
+/* One group of G binary16 values to E5M2 codes with scale s (R17). */
+void kvqo_quantize_group_e5m2(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
+{
+    float amax = 0.0f;
+    for (int j = 0; j < G; ++j) {
+        float v = fabsf(kvqo_f16_to_f32(x[j]));
+        if (v > amax)
+            amax = v;
+    }
+    float s32 = amax / 57344.0f;
+    if (s32 < 1e-5f)
+        s32 = 1e-5f;
+    uint16_t s16 = kvqo_f32_to_f16_up(s32);
+    float s = kvqo_f16_to_f32(s16);
+    for (int j = 0; j < G; ++j)
+        code[j] = kvqo_f32_to_e5m2(kvqo_f16_to_f32(x[j]) / s);
+    *s_out = s16;
+}
+
+/* Token rows to E5M2 codes and (s, 0) fp16 pairs per group of G. */
+void kvqo_quantize_rows_e5m2(const uint16_t *x, int64_t n_rows, int D, int G, uint8_t *codes,
+                             uint16_t *meta)
+{
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int g = 0; g < D / G; ++g) {
+            uint16_t s16;
+            kvqo_quantize_group_e5m2(x + r * D + g * G, G, codes + r * D + g * G, &s16);
+            meta[(r * (D / G) + g) * 2 + 0] = s16;
+            meta[(r * (D / G) + g) * 2 + 1] = 0; /* zero point 0 */
+        }
+}
+
 /* Symmetric INT8 ([P2'] item 2; R15): one group of G binary16 values to
  * two's complement codes with scale s. */
 void kvqo_quantize_group_sym8(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
@@ -400,7 +483,8 @@ static unsigned kvqo_code_at(const uint8_t *row, int e, int bits)
  * Dequantize n_rows packed rows: x_hat = (c - z) * s, evaluated in fp64,
  * where it is exact (|c - z| < 2^17 and s has 11 significant bits); with
  * fmt 1 the codes are E4M3 and x_hat = e4m3(c) * s (R14), with fmt 2 they
- * are two's complement bytes and x_hat = c * s (R15), both also exact.
+ * are two's complement bytes and x_hat = c * s (R15), with fmt 3 E5M2 and
+ * x_hat = e5m2(c) * s (R17), all also exact.
  */
 void kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *meta,
                           int64_t n_rows, int D, int G, int bits, double *out);
@@ -408,12 +492,13 @@ void kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *meta,
 void kvqo_dequantize_rows_fmt(const uint8_t *codes, const uint16_t *meta, int64_t n_rows,
                               int D, int G, int bits, int fmt, double *out)
 {
-    if (fmt == 1 || fmt == 2) {
+    if (fmt == 1 || fmt == 2 || fmt == 3) {
         for (int64_t r = 0; r < n_rows; ++r)
             for (int e = 0; e < D; ++e) {
                 double s = (double)kvqo_f16_to_f32(meta[(r * (D / G) + e / G) * 2 + 0]);
                 uint8_t c = codes[r * D + e];
-                double v = (fmt == 1) ? kvqo_e4m3_to_f64(c) : (double)(int8_t)c;
+                double v = (fmt == 1) ? kvqo_e4m3_to_f64(c)
+                           : (fmt == 3) ? kvqo_e5m2_to_f64(c) : (double)(int8_t)c;
                 out[r * D + e] = v * s;
             }
         return;

@@ -58,14 +58,18 @@ MUTANTS = [
     ("sym8 scale over 128 levels", "float s32 = amax / 127.0f;", "float s32 = amax / 128.0f;"),
     ("sym8 offset-binary codes", "code[j] = (uint8_t)(int8_t)c;",
      "code[j] = (uint8_t)(int)(c + 128.0f);"),
-    ("sym8 dequant unsigned", "double v = (fmt == 1) ? kvqo_e4m3_to_f64(c) : (double)(int8_t)c;",
-     "double v = (fmt == 1) ? kvqo_e4m3_to_f64(c) : (double)c;"),
+    ("sym8 dequant unsigned", ": (fmt == 3) ? kvqo_e5m2_to_f64(c) : (double)(int8_t)c;",
+     ": (fmt == 3) ? kvqo_e5m2_to_f64(c) : (double)c;"),
     ("per-channel block read transposed", "col[t] = x[(int64_t)t * D + d];",
      "col[t] = x[(int64_t)d * T + t];"),
     ("per-channel codes at the token offset", "codes[t * row_bytes + bitpos / 8] |= (uint8_t)(tmp[t] << (bitpos % 8));",
      "codes[d * (row_bytes / 4) + (t * bits) / 8] |= (uint8_t)(tmp[t] << ((t * bits) % 8));"),
     ("per-channel dequant ignores the zero point", "out[(int64_t)t * D + d] = (c - z) * s;",
      "out[(int64_t)t * D + d] = c * s;"),
+    ("e5m2 ties away from zero", "double quantum = ldexp(1.0, (e < -14 ? -14 : e) - 2);\n    double r = rint(a / quantum) * quantum;",
+     "double quantum = ldexp(1.0, (e < -14 ? -14 : e) - 2);\n    double r = round(a / quantum) * quantum;"),
+    ("e5m2 exponent bias 16", "v = ldexp((double)(4 + m), e - 17);", "v = ldexp((double)(4 + m), e - 18);"),
+    ("e5m2 scale from the E4M3 maximum", "float s32 = amax / 57344.0f;", "float s32 = amax / 448.0f;"),
 ]
 
 
@@ -183,6 +187,21 @@ def _pins(o):
     sk = mk[:, 0].view(np.float16).astype(np.float64)
     yield "per-channel half-step bound", bool(np.all(np.abs(xk.astype(np.float64) - xh)
                                                      <= sk[None, :] / 2 * (1 + 2.0**-12)))
+
+    e5 = _golden("e5m2_worked_example.json")
+    ok = True
+    for g in e5["groups"]:
+        code, s16 = o.quantize_group_e5m2(np.asarray(g["x"], np.float16).view(np.uint16))
+        ok &= code.tolist() == g["codes"] and s16 == int(g["s16"], 16)
+    yield "e5m2 worked group", bool(ok)
+    c5 = np.arange(256, dtype=np.uint8)
+    v5 = o.e5m2_to_f64(c5)
+    t5 = torch.from_numpy(c5).view(torch.float8_e5m2).float().numpy().astype(np.float64)
+    yield "e5m2 decode vs torch", bool(np.all((v5 == t5) | (np.isnan(v5) & np.isnan(t5))))
+    f5 = np.unique(t5[np.isfinite(t5)])
+    m5 = np.clip((f5[:-1] + f5[1:]) / 2, -57344, 57344).astype(np.float32)
+    yield "e5m2 encode vs torch", bool(np.array_equal(
+        o.f32_to_e5m2(m5), torch.from_numpy(m5).to(torch.float8_e5m2).view(torch.uint8).numpy()))
 
     t = _golden("chunk_threshold_toy.json")
     sim, cls = o.chunk_assign(np.array(t["chunks"], np.float32), np.array(t["query"], np.float32),
