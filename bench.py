@@ -34,9 +34,10 @@ sys.path.insert(0, ROOT)
 METRIC = "quantized-KV decode attention tokens/s; KV-read GB/s as % of B200 HBM peak"
 DTYPE = {2: "u2", 4: "u4", 8: "u8", 16: "f16"}
 # code formats: arithmetic type, JSON name, and the library's format code
-FMT_DTYPE = {"fp8": "e4m3", "sym8": "s8"}
-FMT_NAME = {"fp8": "fp8 e4m3", "sym8": "symmetric int8"}
-FMT_CODE = {"int": 0, "fp8": 1, "sym8": 2}  # KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM
+FMT_DTYPE = {"fp8": "e4m3", "sym8": "s8", "e5m2": "e5m2"}
+FMT_NAME = {"fp8": "fp8 e4m3", "sym8": "symmetric int8", "e5m2": "fp8 e5m2"}
+# KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM, KVQ_FMT_FP8_E5M2
+FMT_CODE = {"int": 0, "fp8": 1, "sym8": 2, "e5m2": 3}
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 

@@ -70,7 +70,8 @@ typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1 } kvq_dtype;
 typedef enum kvq_format {
     KVQ_FMT_INT = 0,      /* asymmetric integer codes: x_hat = (c - z) * s    */
     KVQ_FMT_FP8_E4M3 = 1, /* FP8 E4M3 codes, bits 8: x_hat = e4m3(c) * s      */
-    KVQ_FMT_INT8_SYM = 2  /* symmetric INT8 codes, bits 8: x_hat = c * s      */
+    KVQ_FMT_INT8_SYM = 2, /* symmetric INT8 codes, bits 8: x_hat = c * s      */
+    KVQ_FMT_FP8_E5M2 = 3  /* FP8 E5M2 codes, bits 8: x_hat = e5m2(c) * s      */
 } kvq_format;
 
 /* Grouping axis of a plane's (scale, zero point) pairs. */
@@ -95,6 +96,10 @@ typedef enum kvq_axis {
  *                 with zero point 0 (the KV-cache page's FP8 KV cache, with
  *                 the scale of each group computed from the values written,
  *                 that page's dynamic quantization).
+ *   bits 8 with fmt KVQ_FMT_FP8_E5M2: one E5M2 code per element (bias 15,
+ *                 largest finite 57344), the same meta layout with zero
+ *                 point 0; the scale of each group is its |max| / 57344
+ *                 (floored at 1e-5, fp16 rounded up), codes saturate.
  *   bits 8 with fmt KVQ_FMT_INT8_SYM: one two's complement int8 code per
  *                 element, the same meta layout with zero point 0 (the
  *                 KV-cache page's INT8 item: s = amax / 127 of the group,

@@ -22,12 +22,16 @@ bool valid_group(int g) { return g == 32 || g == 64 || g == 128; }
 
 // The kernels' template tag of a plane's format: its bit width, kE4M3 or kSym8.
 int kernel_bits(const kvq_plane& p) {
-  return p.fmt == KVQ_FMT_FP8_E4M3 ? kvq::kE4M3 : p.fmt == KVQ_FMT_INT8_SYM ? kvq::kSym8 : p.bits;
+  return p.fmt == KVQ_FMT_FP8_E4M3   ? kvq::kE4M3
+         : p.fmt == KVQ_FMT_FP8_E5M2 ? kvq::kE5M2
+         : p.fmt == KVQ_FMT_INT8_SYM ? kvq::kSym8
+                                     : p.bits;
 }
 
 kvq_status check_plane(const kvq_plane& p, int head_dim, bool allow16, bool is_k) {
   if (p.codes == nullptr || !aligned16(p.codes)) return KVQ_ERR_INVALID_ARG;
-  if (p.fmt != KVQ_FMT_INT && p.fmt != KVQ_FMT_FP8_E4M3 && p.fmt != KVQ_FMT_INT8_SYM)
+  if (p.fmt != KVQ_FMT_INT && p.fmt != KVQ_FMT_FP8_E4M3 && p.fmt != KVQ_FMT_INT8_SYM &&
+      p.fmt != KVQ_FMT_FP8_E5M2)
     return KVQ_ERR_INVALID_ARG;
   if (p.axis != KVQ_AXIS_TOKEN && p.axis != KVQ_AXIS_CHANNEL) return KVQ_ERR_INVALID_ARG;
   if (p.fmt != KVQ_FMT_INT && p.bits != 8) return KVQ_ERR_UNSUPPORTED;

@@ -629,7 +629,7 @@ cudaError_t launch_split_g(const DecodeArgs& a, const SegView& seg, cudaStream_t
 }  // namespace
 
 bool decode_supported(int bits, int group, int group_ratio, bool kpc) {
-  if (kpc || bits == kE4M3 || bits == kSym8)
+  if (kpc || bits == kE4M3 || bits == kE5M2 || bits == kSym8)
     return decode_tm_supported(bits, group, group_ratio, kpc);
   if (!(group_ratio == 1 || group_ratio == 2 || group_ratio == 4 || group_ratio == 8))
     return false;

@@ -448,10 +448,10 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     kpc_rebuild(sKm);
     auto valid = [&](int tok) { return FULL || tok < n_valid; };  // tok: 0 .. STOK-1
     // V rows past the valid length may hold any bytes.  Integer codes are
-    // finite and meet a zero weight; raw fp16 and e4m3 bytes can be NaN or
+    // finite and meet a zero weight; raw fp16 and FP8 bytes can be NaN or
     // Inf, which a zero weight does not cancel in the MMA: zero those words.
     auto zero_invalid = [&](int sub, auto& wA, auto& wB, auto& wC, auto& wD) {
-      if constexpr ((BITS == 16 || BITS == kE4M3) && !FULL) {
+      if constexpr ((BITS == 16 || BITS == kE4M3 || BITS == kE5M2) && !FULL) {
         constexpr int NW = sizeof(wA) / sizeof(wA[0]);
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
@@ -829,7 +829,9 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   X(kE4M3, 128, 1) X(kE4M3, 128, 2) X(kE4M3, 128, 4) X(kE4M3, 128, 8)  \
   X(kE4M3, 64, 1) X(kE4M3, 64, 2) X(kE4M3, 64, 4) X(kE4M3, 32, 1) X(kE4M3, 32, 2) \
   X(kSym8, 128, 1) X(kSym8, 128, 2) X(kSym8, 128, 4) X(kSym8, 128, 8)  \
-  X(kSym8, 64, 1) X(kSym8, 64, 2) X(kSym8, 64, 4) X(kSym8, 32, 1) X(kSym8, 32, 2)
+  X(kSym8, 64, 1) X(kSym8, 64, 2) X(kSym8, 64, 4) X(kSym8, 32, 1) X(kSym8, 32, 2) \
+  X(kE5M2, 128, 1) X(kE5M2, 128, 2) X(kE5M2, 128, 4) X(kE5M2, 128, 8)  \
+  X(kE5M2, 64, 1) X(kE5M2, 64, 2) X(kE5M2, 64, 4) X(kE5M2, 32, 1) X(kE5M2, 32, 2)
 
 }  // namespace
 

@@ -11,7 +11,7 @@
 
 namespace kvq {
 
-constexpr int kHeadDim = 128;  // head_dim supported by this build
+constexpr int kHeadDim = 128;  // the head_dim the kernels are compiled for
 constexpr int kTile = 16;      // tokens per warp step (one m16n8k16 K-extent)
 constexpr int kWarps = 4;      // consumer warps per decode CTA
 
@@ -231,6 +231,23 @@ struct WordPairs<16> {
   __device__ __forceinline__ static uint32_t one(uint32_t w, int) { return w; }
 };
 
+// FP8 E5M2 word (dims 0..3): an E5M2 code is the high byte of the fp16 of
+// the same value, so a byte permute with zero fill gives pair j = dims
+// (2j, 2j + 1), the values themselves (factor 1, like raw fp16).
+template <>
+struct WordPairs<kE5M2> {
+  static constexpr int kPairs = 2, kDims = 4, kEmax = 24;
+  __device__ __forceinline__ static void run(uint32_t w, uint32_t (&p)[2]) {
+    p[0] = prmt(w, 0u, 0x1404u);  // [0 w.b0 0 w.b1]
+    p[1] = prmt(w, 0u, 0x3424u);  // [0 w.b2 0 w.b3]
+  }
+  __host__ __device__ static constexpr int dim(int j, int e) { return 2 * j + e; }
+  __host__ __device__ static constexpr int exp(int) { return 24; }
+  __device__ __forceinline__ static uint32_t one(uint32_t w, int j) {
+    return prmt(w, 0u, j ? 0x3424u : 0x1404u);
+  }
+};
+
 // Symmetric INT8 word (two's complement bytes): bit 7 of every byte flipped
 // gives the offset-binary code c + 128, read like the 8-bit integer codes
 // with a zero point of 128.
@@ -341,6 +358,20 @@ struct CrossPairs<kSym8> {
     o[3] = prmt(y, 0u, 0x4341u) ^ 0x00800080u;
   }
   __host__ __device__ static constexpr int exp(int) { return 0; }
+};
+
+template <>
+struct CrossPairs<kE5M2> {
+  static constexpr int kOut = 4;
+  __device__ __forceinline__ static void run(uint32_t a, uint32_t b, uint32_t (&o)[4]) {
+    const uint32_t x = prmt(a, b, 0x5140u);  // [a.b0 b.b0 a.b1 b.b1]
+    const uint32_t y = prmt(a, b, 0x7362u);  // [a.b2 b.b2 a.b3 b.b3]
+    o[0] = prmt(x, 0u, 0x1404u);              // [0 a.b0 0 b.b0]: fp16 of the codes
+    o[1] = prmt(x, 0u, 0x3424u);
+    o[2] = prmt(y, 0u, 0x1404u);
+    o[3] = prmt(y, 0u, 0x3424u);
+  }
+  __host__ __device__ static constexpr int exp(int) { return 24; }
 };
 
 template <>

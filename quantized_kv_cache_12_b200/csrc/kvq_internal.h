@@ -15,6 +15,8 @@ namespace kvq {
 constexpr int kE4M3 = 0x108;
 // symmetric INT8 codes (two's complement bytes, zero point 0); code_bits 8
 constexpr int kSym8 = 0x208;
+// FP8 E5M2 codes (bias 15, two mantissa bits); code_bits 8
+constexpr int kE5M2 = 0x308;
 __host__ __device__ constexpr int code_bits(int tag) { return tag & 0xFF; }
 
 // One K/V plane pair of one cache segment, as the kernels see it.

@@ -31,6 +31,13 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return r;
 }
 
+// The same for E5M2 codes, saturated at +-57344.
+__device__ __forceinline__ uint32_t e5m2x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // x / d rounded to nearest-even fp32 (the IEEE quotient), given r = RN(1/d):
 // q0 = RN(x r) approximates x / d within one ulp, the remainder x - q0 d is
 // exact in one fma, and RN(q0 + (x - q0 d) r) is the correctly rounded
@@ -118,7 +125,7 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
     x[2 * i] = f.x;
     x[2 * i + 1] = f.y;
   }
-  if constexpr (BITS == kE4M3 || BITS == kSym8) {
+  if constexpr (BITS == kE4M3 || BITS == kE5M2 || BITS == kSym8) {
     // the group's |max|, taken on the fp16 values (exact)
     __half2 am = __habs2(h2[0]);
 #pragma unroll
@@ -152,11 +159,13 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
       meta = h2_as_u32(__halves2half2(s16, __float2half_rn(0.f)));
       return;
     }
-    // FP8 E4M3 (the KV-cache page's FP8 KV cache, dynamic scale): s = max(
-    // amax / 448, 1e-5) stored in fp16 rounded up, so |x / s| <= 448;
-    // code = E4M3 of the fp32 quotient x / s; zero point 0.
-    constexpr float kInv448 = 1.0f / 448.0f;
-    const float s32 = fmaxf(div_rn(__low2float(am), 448.0f, kInv448), 1e-5f);
+    // FP8 (the KV-cache page's FP8 KV cache, dynamic scale): s = max(amax /
+    // F, 1e-5) stored in fp16 rounded up, so |x / s| <= F, the format's
+    // largest finite value (E4M3 448, E5M2 57344); code = the FP8 value of
+    // the fp32 quotient x / s; zero point 0.
+    constexpr float kMaxF = BITS == kE4M3 ? 448.0f : 57344.0f;
+    constexpr float kInvMax = 1.0f / kMaxF;
+    const float s32 = fmaxf(div_rn(__low2float(am), kMaxF, kInvMax), 1e-5f);
     const __half s16 = __float2half_ru(s32);
     const float s = __half2float(s16);
     const float r = __frcp_rn(s);
@@ -165,7 +174,10 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
 #pragma unroll
     for (int i = 0; i < NH; ++i) {
       const float2 q = f2_unpack(div_rn2(f2_pack(x[2 * i], x[2 * i + 1]), nd2, r2));
-      c[i] = e4m3x2(copysignf(q.x, x[2 * i]), copysignf(q.y, x[2 * i + 1]));
+      if constexpr (BITS == kE4M3)
+        c[i] = e4m3x2(copysignf(q.x, x[2 * i]), copysignf(q.y, x[2 * i + 1]));
+      else
+        c[i] = e5m2x2(copysignf(q.x, x[2 * i]), copysignf(q.y, x[2 * i + 1]));
     }
 #pragma unroll
     for (int i = 0; i < NH / 2; ++i) codes[i] = __byte_perm(c[2 * i], c[2 * i + 1], 0x5410);

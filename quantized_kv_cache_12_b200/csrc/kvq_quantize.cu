@@ -427,6 +427,7 @@ cudaError_t launch_quantize(const QuantArgs& a, int bits, int group, cudaStream_
   KVQ_Q(2, 32) KVQ_Q(2, 64) KVQ_Q(2, 128)
   KVQ_Q(kE4M3, 32) KVQ_Q(kE4M3, 64) KVQ_Q(kE4M3, 128)
   KVQ_Q(kSym8, 32) KVQ_Q(kSym8, 64) KVQ_Q(kSym8, 128)
+  KVQ_Q(kE5M2, 32) KVQ_Q(kE5M2, 64) KVQ_Q(kE5M2, 128)
 #undef KVQ_Q
   return cudaErrorInvalidValue;
 }

@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libkvq.so")
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, \
     KVQ_ERR_CUDA = range(6)
 KVQ_F16, KVQ_BF16 = 0, 1
-KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM = 0, 1, 2
+KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM, KVQ_FMT_FP8_E5M2 = 0, 1, 2, 3
 KVQ_AXIS_TOKEN, KVQ_AXIS_CHANNEL = 0, 1
 KVQ_CHANNEL_BLOCK = 32
 HEADER_BYTES = 256  # workspace header: sticky device error word first
@@ -254,8 +254,9 @@ class QuantizedKVCache:
     codes: uint8 [B, H_kv, max_tokens, head_dim*bits/8];
     meta: fp16 [B, H_kv, max_tokens, head_dim/G, 2] (scale, zero), None for bits 16;
     seq_lens: int32 [B] on the device; fmt: KVQ_FMT_INT, KVQ_FMT_FP8_E4M3
-    (bits 8: E4M3 codes, zero points 0) or KVQ_FMT_INT8_SYM (bits 8: two's
-    complement codes, zero points 0).
+    (bits 8: E4M3 codes, zero points 0), KVQ_FMT_FP8_E5M2 (bits 8: E5M2 codes,
+    zero points 0) or KVQ_FMT_INT8_SYM (bits 8: two's complement codes, zero
+    points 0).
     k_axis: KVQ_AXIS_TOKEN, or KVQ_AXIS_CHANNEL (K grouped per channel over
     blocks of KVQ_CHANNEL_BLOCK tokens: k_meta fp16 [B, H_kv,
     max_tokens / KVQ_CHANNEL_BLOCK, head_dim, 2]; group_size is V's).

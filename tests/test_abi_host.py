@@ -213,6 +213,26 @@ def test_fp8_planes_validated(kvq):
     assert _status(kvq.kvq_decode_workspace_bytes, c, 16) == kvq.KVQ_ERR_UNSUPPORTED  # g = 8
 
 
+def test_e5m2_planes_validated(kvq):
+    """KVQ_FMT_FP8_E5M2 needs bits 8 and the same format on K and V; its decode
+    is built for the same (G, g) as E4M3."""
+    fake = ctypes.c_void_p(0x60000)
+
+    def append_status(c):
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, 1, 1, None)
+    c = _fake_cache(kvq, bits=4)
+    c.k.fmt = c.v.fmt = kvq.KVQ_FMT_FP8_E5M2
+    assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
+    c = _fake_cache(kvq, bits=8)
+    c.k.fmt = kvq.KVQ_FMT_FP8_E5M2
+    c.v.fmt = kvq.KVQ_FMT_FP8_E4M3
+    assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
+    c = _fake_cache(kvq, bits=8, group=64, kv_heads=2)
+    c.k.fmt = c.v.fmt = kvq.KVQ_FMT_FP8_E5M2
+    assert kvq.kvq_decode_workspace_bytes(c, 8) > 0   # g = 4
+    assert _status(kvq.kvq_decode_workspace_bytes, c, 16) == kvq.KVQ_ERR_UNSUPPORTED  # g = 8
+
+
 def test_sym8_planes_validated(kvq):
     """KVQ_FMT_INT8_SYM needs bits 8 and the same format on K and V; its
     decode is built for the same (G, g) as FP8."""

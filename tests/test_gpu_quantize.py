@@ -169,7 +169,7 @@ def test_prefill_full_size_long_context_sampled(kvq):
 
 
 def _alloc_fmt(kvq, B, H, max_tokens, bits, G, fmt):
-    f = kvq.KVQ_FMT_FP8_E4M3 if fmt == "fp8" else kvq.KVQ_FMT_INT
+    f = {"fp8": kvq.KVQ_FMT_FP8_E4M3, "e5m2": kvq.KVQ_FMT_FP8_E5M2}.get(fmt, kvq.KVQ_FMT_INT)
     c = kvq.QuantizedKVCache.allocate(B, H, 128, max_tokens, bits, G, DEV, fmt=f)
     c.k_codes.fill_(0xA5)
     c.v_codes.fill_(0x5A)
@@ -179,7 +179,7 @@ def _alloc_fmt(kvq, B, H, max_tokens, bits, G, fmt):
 
 
 BULK_FORMATS = [(b, G, "int") for b in (2, 4, 8) for G in (32, 64, 128)] + \
-               [(8, G, "fp8") for G in (32, 64, 128)]
+               [(8, G, f) for G in (32, 64, 128) for f in ("fp8", "e5m2")]
 
 
 @pytest.mark.parametrize("bits,G,fmt", BULK_FORMATS)
@@ -212,7 +212,7 @@ def test_bulk_kernel_ragged_starts_and_capacity(kvq, bits, G, fmt):
 
 
 @pytest.mark.parametrize("bits,G,fmt", [(8, 128, "int"), (4, 64, "int"), (2, 32, "int"),
-                                        (4, 128, "int"), (8, 64, "fp8")])
+                                        (4, 128, "int"), (8, 64, "fp8"), (8, 32, "e5m2")])
 def test_bulk_kernel_scale_sweep_and_adversarial(kvq, bits, G, fmt):
     """Groups whose magnitudes sweep the fp16 range (2^-24 .. 2^15, so the
     scale runs from its 1e-5 floor to above 100), offsets that push the zero

@@ -68,8 +68,8 @@ class DecodeWorkload:
     alpha: float = 0.0
     beta: float = 0.0
     low_bits: Tuple[int, ...] = ()   # bit-widths of the two quantized classes
-    fmt: str = "int"          # code format: "int" (asymmetric integer), "fp8" (E4M3, bits 8)
-    #                           or "sym8" (symmetric INT8, bits 8)
+    fmt: str = "int"          # code format: "int" (asymmetric integer), "fp8" (E4M3, bits 8),
+    #                           "e5m2" (E5M2, bits 8) or "sym8" (symmetric INT8, bits 8)
     k_axis: str = "token"     # K grouping: "token" (groups along head_dim) or "channel"
     #                           (per channel over 32-token blocks; attention only)
 
@@ -116,6 +116,10 @@ WORKLOADS = {
         name="llama3_8b_gqa_fp8", batch=32, q_heads=32, kv_heads=8, head_dim=128,
         context=8192, bits=8, group=64, q_dtype="f16", steps=100, append=True, seed=3,
         k_outliers=Outliers(factor=15.0, per_head=4), v_sigma=0.5, fmt="fp8"),
+    "llama3_8b_gqa_e5m2": DecodeWorkload(
+        name="llama3_8b_gqa_e5m2", batch=32, q_heads=32, kv_heads=8, head_dim=128,
+        context=8192, bits=8, group=64, q_dtype="f16", steps=100, append=True, seed=3,
+        k_outliers=Outliers(factor=15.0, per_head=4), v_sigma=0.5, fmt="e5m2"),
     "llama2_7b_mha_sym8": DecodeWorkload(
         name="llama2_7b_mha_sym8", batch=16, q_heads=32, kv_heads=32, head_dim=128,
         context=4096, bits=8, group=128, q_dtype="bf16", steps=100, append=True, seed=2,
