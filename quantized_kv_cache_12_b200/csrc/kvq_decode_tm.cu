@@ -106,6 +106,12 @@ struct TmCfg {
   static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 16 ? 16 : STAGES_RAW);
   static constexpr int SMEM = HDR_BYTES + kWarps * STAGES * STAGE;
   static constexpr int EMAX = WordPairs<BITS>::kEmax;
+  // FP8 weights P' = p * s_V carry an exact 2^8 (E4M3) or 2^14 (E5M2): their
+  // scales (|max| / 448, / 57344) would otherwise put small weights among the
+  // fp16 subnormals, where the (hi, lo) split loses its bits; the largest
+  // scale times the factor stays below 65504.  The output undoes it.
+  static constexpr float PSCALE = BITS == kE4M3 ? 256.0f : (BITS == kE5M2 ? 16384.0f : 1.0f);
+  static constexpr float INV_PSCALE = 1.0f / PSCALE;
   // the warp merge reuses the stage buffers: m, l, o of kWarps x 8 rows
   static constexpr int MERGE_BYTES = (2 * kWarps * 8 + kWarps * 8 * D + 8 * (kWarps + 2)) * 4;
   static_assert(NG * GR <= 8, "at most eight (head, group) combinations");
@@ -596,7 +602,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
             const float2 sz = __half22float2(*reinterpret_cast<const __half2*>(
                 sVm + tok * C::MB + gv[nb] * 4));
             const bool ok = valid(tok);
-            pp[r] = ok ? p[slot_of(nb)][r] * sz.x : 0.f;
+            pp[r] = ok ? p[slot_of(nb)][r] * (sz.x * C::PSCALE) : 0.f;
+            // in the weights' units: PSCALE is 1 for every format with a
+            // zero point (the FP8 formats, lifted, have zero points of 0)
             corr[nb] = ok ? fmaf(pp[r], zero_of(sz.y), corr[nb]) : corr[nb];
           }
         }
@@ -756,8 +764,8 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     for (int gq = 0; gq < NG; ++gq)
 #pragma unroll
       for (int j = 0; j < CH / 2; ++j) {
-        const float f0 = pow2f(24 - XP::exp(j % XP::kOut));
-        const float f1 = pow2f(24 - XP::exp((j + CH / 2) % XP::kOut));
+        const float f0 = pow2f(24 - XP::exp(j % XP::kOut)) * C::INV_PSCALE;
+        const float f1 = pow2f(24 - XP::exp((j + CH / 2) % XP::kOut)) * C::INV_PSCALE;
         const float* o = o_acc[0][gq * (CH / 2) + j];
         oh[gq * GE + j] = fmaf(o[0] - o[1], f0, -corr[gq]);
         oh[gq * GE + j + CH / 2] = fmaf(o[2] - o[3], f1, -corr[gq]);
@@ -771,8 +779,8 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         for (int mt = 0; mt < 8; ++mt) {
           // hi column minus the negated-remainder column, then undo the
           // subnormal code scale 2^(e - 24) of the row's dim
-          const float f0 = pow2f(24 - XP::exp(mt % XP::kOut));
-          const float f1 = pow2f(24 - XP::exp((mt + 8) % XP::kOut));
+          const float f0 = pow2f(24 - XP::exp(mt % XP::kOut)) * C::INV_PSCALE;
+          const float f1 = pow2f(24 - XP::exp((mt + 8) % XP::kOut)) * C::INV_PSCALE;
           oh[mt] = fmaf(o_acc[nb][mt][0] - o_acc[nb][mt][1], f0, -corr[nb]);
           oh[mt + 8] = fmaf(o_acc[nb][mt][2] - o_acc[nb][mt][3], f1, -corr[nb]);
         }
