@@ -76,9 +76,10 @@ def bytes_per_head_token(bits: int, group: int, head_dim: int = 128,
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     # the decode kernels' sources and the headers they compile (the fused
-    # append's quantizer included)
+    # append's quantizer included), and the host code whose split plan picks
+    # the kernel build and the units of a launch
     for f in ("kvq_decode.cu", "kvq_decode_tm.cu", "kvq_decode_common.cuh", "kvq_device.cuh",
-              "kvq_quant_core.cuh", "kvq_internal.h"):
+              "kvq_quant_core.cuh", "kvq_internal.h", "kvq_abi.cu"):
         with open(os.path.join(ROOT, "quantized_kv_cache_12_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

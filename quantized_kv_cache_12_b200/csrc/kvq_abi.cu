@@ -67,23 +67,28 @@ kvq_status check_cache(const kvq_cache* c, bool allow16) {
 }
 
 // Split count of one segment.  A (sequence, KV head, split) is one unit of
-// work; the decode kernel runs one wave of persistent CTAs (three per SM,
-// 444 on a B200) that take units from a counter.  With equal units the
-// kernel takes ceil(units / 444) unit-times, so the count minimises
-// ceil(units / 444) x (tokens per unit + a fixed per-unit cost), tokens per
+// work; the decode kernel runs one wave of persistent CTAs (S = 148 x the
+// format's CTAs per SM) that take units from a counter.  With equal units
+// the kernel takes ceil(units / S) unit-times, so the count minimises
+// ceil(units / S) x (tokens per unit + a fixed per-unit cost), tokens per
 // unit being rounded up to the 32-token stage, with at least 128 tokens per
 // unit.  The fixed cost -- the start of a unit waits for its query rows and
-// first copies -- was measured at about 400 tokens' worth of work.  The result depends only on
-// (sequences x KV heads, length), so it is cached per thread.
+// first copies -- was measured at about 200 tokens' worth of work.  The
+// result depends only on (sequences x KV heads, length, S), so the last few
+// are cached per thread.
 int choose_splits(const kvq_cache& c, int max_len_hint, int ctas_per_sm) {
   const long long pairs = (long long)c.batch * c.kv_heads;
   long long len = c.max_tokens;
   if (max_len_hint > 0 && max_len_hint < len) len = max_len_hint;
   if (len <= 0 || pairs <= 0) return 1;
-  thread_local long long cached_pairs = -1, cached_len = -1, cached_slots = -1;
-  thread_local int cached_n = 1;
+  constexpr int kCache = 4;
+  thread_local long long cached_pairs[kCache] = {-1, -1, -1, -1}, cached_len[kCache],
+                                               cached_slots[kCache];
+  thread_local int cached_n[kCache], cache_next = 0;
   const long long kSlots = 148LL * (ctas_per_sm > 0 ? ctas_per_sm : 3);
-  if (pairs == cached_pairs && len == cached_len && kSlots == cached_slots) return cached_n;
+  for (int e = 0; e < kCache; ++e)
+    if (pairs == cached_pairs[e] && len == cached_len[e] && kSlots == cached_slots[e])
+      return cached_n[e];
   constexpr long long kOverhead = 200, kGran = 32, kMinTokens = 128;
   const long long cap = (len + kMinTokens - 1) / kMinTokens;
   long long best_n = 1, best_cost = -1;
@@ -96,15 +101,18 @@ int choose_splits(const kvq_cache& c, int max_len_hint, int ctas_per_sm) {
       best_n = n;
     }
   }
-  cached_pairs = pairs;
-  cached_len = len;
-  cached_slots = kSlots;
-  cached_n = (int)best_n;
-  return cached_n;
+  const int e = cache_next;
+  cache_next = (cache_next + 1) % kCache;
+  cached_pairs[e] = pairs;
+  cached_len[e] = len;
+  cached_slots[e] = kSlots;
+  cached_n[e] = (int)best_n;
+  return cached_n[e];
 }
 
 struct SplitPlan {
   int n_split[16];
+  int wide[16];  // the segment runs its format's five-CTAs-per-SM build
   int parts;
 };
 
@@ -114,9 +122,20 @@ kvq_status plan_splits(const kvq_cache* segs, int n_segs, int q_heads, int max_l
   const int g = q_heads / segs[0].kv_heads;
   for (int i = 0; i < n_segs; ++i) {
     const int bits = kernel_bits(segs[i].k);
-    const int ctas = kvq::decode_ctas_per_sm(bits, bits == 16 ? kD : segs[i].v.group_size, g,
-                                             segs[i].k.axis == KVQ_AXIS_CHANNEL);
+    const int group = bits == 16 ? kD : segs[i].v.group_size;
+    const bool kpc = segs[i].k.axis == KVQ_AXIS_CHANNEL;
+    const int ctas = kvq::decode_ctas_per_sm(bits, group, g, kpc);
     plan->n_split[i] = choose_splits(segs[i], max_len_hint, ctas);
+    plan->wide[i] = 0;
+    // the five-CTA build where its own plan needs more than one wave
+    const int wide = kvq::decode_tm_wide_ctas_per_sm(bits, group, g, kpc);
+    if (wide > 0) {
+      const int n = choose_splits(segs[i], max_len_hint, wide);
+      if ((long long)segs[i].batch * segs[i].kv_heads * n > 148LL * wide) {
+        plan->n_split[i] = n;
+        plan->wide[i] = 1;
+      }
+    }
     plan->parts += plan->n_split[i];
   }
   return KVQ_OK;
@@ -324,6 +343,7 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
     v.k_channels = segs[i].k.axis == KVQ_AXIS_CHANNEL;
     v.max_tokens = segs[i].max_tokens;
     v.n_split = plan.n_split[i];
+    v.wide = plan.wide[i];
     v.part_base = base;
     base += plan.n_split[i];
     if ((stages & kPartials) && kvq::launch_decode_segment(a, v, s) != cudaSuccess)

@@ -52,7 +52,7 @@ namespace kvq {
 
 namespace {
 
-template <int BITS, int GE, int GR, bool KPC = false>
+template <int BITS, int GE, int GR, bool KPC = false, int OCC = 0>
 struct TmCfg {
   static constexpr int D = kHeadDim;
   static constexpr int NG = D / GE;                    // V groups per token (and K's, per token)
@@ -96,12 +96,13 @@ struct TmCfg {
   // per-channel K: the g query rows times each dim's 2^(EMAX - e), fp16
   static constexpr int QF_BYTES = QB_SMEM ? 8 * 32 * 8 : (KPC ? GR * D * 2 : 0);
   static constexpr int HDR_BYTES = ((HDR_QF + QF_BYTES + 127) / 128) * 128;
-  // four CTAs per SM (128 registers a thread) where two stages per warp fit
-  // in a quarter of the SM's shared memory (4 x (56 KB + 1 KB reserved)
-  // <= 228 KB), else three
+  // four CTAs per SM (128 registers a thread) where three stages per warp
+  // fit in a quarter of the SM's shared memory (4 x (56 KB + 1 KB reserved)
+  // <= 228 KB), else three; OCC > 0 asks for that many instead (five: 102
+  // registers a thread and 44 KB, which leaves two stages per warp)
   static constexpr int MIN_CTAS =
-      (NO == 1 && HDR_BYTES + kWarps * 3 * STAGE <= 56 * 1024) ? 4 : 3;
-  static constexpr int SMEM_BUDGET = (MIN_CTAS == 4 ? 56 : 74) * 1024;
+      OCC > 0 ? OCC : ((NO == 1 && HDR_BYTES + kWarps * 3 * STAGE <= 56 * 1024) ? 4 : 3);
+  static constexpr int SMEM_BUDGET = (MIN_CTAS >= 5 ? 44 : (MIN_CTAS == 4 ? 56 : 74)) * 1024;
   static constexpr int STAGES_RAW = (SMEM_BUDGET - HDR_BYTES) / (kWarps * STAGE);
   static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 16 ? 16 : STAGES_RAW);
   static constexpr int SMEM = HDR_BYTES + kWarps * STAGES * STAGE;
@@ -152,10 +153,10 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& r0, uin
   r1 = pack_h2(x1, n1);
 }
 
-template <int BITS, int GE, int GR, bool KPC>
-__global__ void __launch_bounds__(kWarps * 32, TmCfg<BITS, GE, GR, KPC>::MIN_CTAS)
+template <int BITS, int GE, int GR, bool KPC, int OCC>
+__global__ void __launch_bounds__(kWarps * 32, TmCfg<BITS, GE, GR, KPC, OCC>::MIN_CTAS)
 decode_tm_kernel(const __grid_constant__ SplitParams P) {
-  using C = TmCfg<BITS, GE, GR, KPC>;
+  using C = TmCfg<BITS, GE, GR, KPC, OCC>;
   using WP = WordPairs<BITS>;
   using XP = CrossPairs<BITS>;
   // the zero point the codes are read against: symmetric INT8 codes are read
@@ -797,9 +798,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   if (t == 0) release_counters(counters);
 }
 
-template <int BITS, int GE, int GR, bool KPC>
+template <int BITS, int GE, int GR, bool KPC, int OCC = 0>
 cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
-  using C = TmCfg<BITS, GE, GR, KPC>;
+  using C = TmCfg<BITS, GE, GR, KPC, OCC>;
   // the shared-memory opt-in is a per-device function attribute: set it once
   // per device (bit i of the mask = device i)
   static std::atomic<unsigned long long> attr_set{0};
@@ -807,7 +808,7 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tm_kernel<BITS, GE, GR, KPC>,
+    cudaError_t e = cudaFuncSetAttribute(decode_tm_kernel<BITS, GE, GR, KPC, OCC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
@@ -816,13 +817,20 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   const long long units = (long long)seg.n_split * a.kv_heads * a.batch;
   const long long slots = 148LL * C::MIN_CTAS;  // one wave of persistent CTAs
   const unsigned grid = (unsigned)(units < slots ? units : slots);
-  decode_tm_kernel<BITS, GE, GR, KPC><<<grid, kWarps * 32, C::SMEM, s>>>(P);
+  decode_tm_kernel<BITS, GE, GR, KPC, OCC><<<grid, kWarps * 32, C::SMEM, s>>>(P);
   return cudaGetLastError();
 }
 
 // Per-channel K (G is V's group size): the (bits, G, g) whose QK columns
 // give lane tig head tig % g in two columns (see TmCfg).
 #define KVQ_TM_KPC_FORMATS(X) X(4, 64, 4) X(8, 128, 1) X(4, 128, 4) X(4, 128, 1)
+
+// Formats also built at five CTAs per SM (two stages per warp): with more
+// units than one wave of those CTAs, the finer split shortens the last
+// wave by more than the shallower copy pipeline costs; with one wave or
+// less the three-stage kernel is faster.
+#define KVQ_TM_WIDE_FORMATS(X) X(4, 64, 4)
+constexpr int kWideCtas = 5;
 
 // Every (bits, G, g) with NG * g <= 8 that the cache formats allow.
 #define KVQ_TM_FORMATS(X)                                              \
@@ -870,9 +878,25 @@ int decode_tm_ctas_per_sm(int bits, int group, int group_ratio, bool kpc) {
   return 0;
 }
 
+int decode_tm_wide_ctas_per_sm(int bits, int group, int group_ratio, bool kpc) {
+  if (kpc) return 0;
+#define KVQ_X(B, G_, R) \
+  if (bits == B && group == G_ && group_ratio == R) return TmCfg<B, G_, R, false, kWideCtas>::MIN_CTAS;
+  KVQ_TM_WIDE_FORMATS(KVQ_X)
+#undef KVQ_X
+  return 0;
+}
+
 cudaError_t launch_decode_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   const int bits = seg.bits, group = (seg.bits == 16) ? kHeadDim : seg.group;
   const int g = a.group_ratio;
+  if (seg.wide) {
+#define KVQ_X(B, G_, R) \
+  if (!seg.k_channels && bits == B && group == G_ && g == R) return launch_tm<B, G_, R, false, kWideCtas>(a, seg, s);
+    KVQ_TM_WIDE_FORMATS(KVQ_X)
+#undef KVQ_X
+    return cudaErrorInvalidValue;
+  }
 #define KVQ_X(B, G_, R) \
   if (bits == B && group == G_ && g == R) return launch_tm<B, G_, R, false>(a, seg, s);
 #define KVQ_XK(B, G_, R) \

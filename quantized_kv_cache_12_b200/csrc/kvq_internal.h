@@ -32,6 +32,7 @@ struct SegView {
   int32_t n_split;       // CTAs per (sequence, KV head) for this segment
   int32_t part_base;     // index of this segment's first partial
   int32_t k_channels;    // K grouped per channel over kChannelBlock-token blocks
+  int32_t wide;          // run the five-CTAs-per-SM build of the format
 };
 
 struct DecodeArgs {
@@ -83,6 +84,8 @@ int decode_ctas_per_sm(int bits, int group, int group_ratio, bool kpc = false);
 // the tokens-on-M kernel (kvq_decode_tm.cu): formats with NG * g <= 8
 bool decode_tm_supported(int bits, int group, int group_ratio, bool kpc = false);
 int decode_tm_ctas_per_sm(int bits, int group, int group_ratio, bool kpc = false);
+// CTAs per SM of the format's five-CTA build, 0 where it has none
+int decode_tm_wide_ctas_per_sm(int bits, int group, int group_ratio, bool kpc = false);
 cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s);
