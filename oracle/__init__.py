@@ -80,6 +80,9 @@ def _load():
                                                   i64, i32, f64, P, P]
         lib.kvqo_chunk_assign.argtypes = [P, P, i32, i32, f64, f64, P, P]
         lib.kvqo_chunk_partition.argtypes = [P, i32, P, P]
+        f32 = ctypes.c_float
+        lib.kvqo_oaken_quantize_rows.argtypes = [P, i64, i32, f32, i32, f32, i32, P, P]
+        lib.kvqo_oaken_dequantize_rows.argtypes = [P, P, i64, i32, f32, i32, f32, P]
         lib.kvqo_kv_elements.argtypes = [u64, u64, u64, u64, u64]
         lib.kvqo_kv_elements.restype = u64
         _lib = lib
@@ -317,6 +320,48 @@ def dequantize_channels(codes, meta, L: int, D: int, bits: int) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Oaken group-shift codec ("大模型KV缓存量化技术：原理、优化与实践" page,
+# sections 3.1, 3.2.1, 3.2.2; reading R18 in kvq_oracle.c)
+# --------------------------------------------------------------------------
+
+OAKEN_SLOTS = 16
+
+
+def oaken_quantize_rows(x16, s_in: float, z_in: int, s_out: float, outer_bits: int):
+    """Token rows [N, D] (fp16 patterns) -> (codes [N, D/2] uint8, slots
+    [N, OAKEN_SLOTS] uint16) with the plane's offline parameters."""
+    lib = _load()
+    x16 = _c(x16, np.uint16)
+    N, D = x16.shape
+    codes = np.zeros((N, D // 2), np.uint8)
+    slots = np.zeros((N, OAKEN_SLOTS), np.uint16)
+    lib.kvqo_oaken_quantize_rows(_p(x16), N, D, float(s_in), int(z_in), float(s_out),
+                                 int(outer_bits), _p(codes), _p(slots))
+    return codes, slots
+
+
+def oaken_dequantize_rows(codes, slots, D: int, s_in: float, z_in: int, s_out: float):
+    """codes [N, D/2], slots [N, OAKEN_SLOTS] -> fp64 [N, D]."""
+    lib = _load()
+    codes = _c(codes, np.uint8)
+    slots = _c(slots, np.uint16)
+    N = codes.shape[0]
+    out = np.zeros((N, D), np.float64)
+    lib.kvqo_oaken_dequantize_rows(_p(codes), _p(slots), N, D, float(s_in), int(z_in),
+                                   float(s_out), _p(out))
+    return out
+
+
+def oaken_quantize_cache(x16, params):
+    """x16 [..., T, D] -> codes [..., T, D/2], slots [..., T, OAKEN_SLOTS];
+    params = (s_in, z_in, s_out, outer_bits)."""
+    x16 = _c(x16, np.uint16)
+    lead, D = x16.shape[:-1], x16.shape[-1]
+    codes, slots = oaken_quantize_rows(x16.reshape(-1, D), *params)
+    return codes.reshape(*lead, D // 2), slots.reshape(*lead, OAKEN_SLOTS)
+
+
+# --------------------------------------------------------------------------
 # fp64 attention (score definition: KVO-LLM page 3.2; chunked + merge:
 # Cocktail page 3.2.3)
 # --------------------------------------------------------------------------
@@ -422,9 +467,11 @@ def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: fl
     q16: [B, Hq, D] fp16/bf16 patterns.  segments: list of dicts with numpy
     arrays ``k_codes``/``v_codes`` [B, Hkv, T, row_bytes], ``k_meta``/``v_meta``
     [B, Hkv, T, D/G, 2] (None for bits 16), ``bits``, ``group`` and optionally
-    ``fmt`` ("int", the default, "fp8", "sym8" or "e5m2") and ``k_channels`` (True: K
-    is per-channel, ``k_meta`` [B, Hkv, T / KPC_BLOCK, D, 2], lengths multiples
-    of KPC_BLOCK).
+    ``fmt`` ("int", the default, "fp8", "sym8", "e5m2" or "oaken") and ``k_channels``
+    (True: K is per-channel, ``k_meta`` [B, Hkv, T / KPC_BLOCK, D, 2], lengths
+    multiples of KPC_BLOCK).  An "oaken" segment holds the outlier slots
+    [B, Hkv, T, OAKEN_SLOTS] in ``k_meta``/``v_meta`` and the planes' offline
+    parameters (s_in, z_in, s_out, outer_bits) in ``k_oaken``/``v_oaken``.
     seq_lens_per_seg: list of int arrays [B].  The segments of a sequence are
     concatenated in token order (attention does not depend on the order).
     pairs: optional list of (b, kv_head) to evaluate; others stay NaN.
@@ -445,6 +492,13 @@ def decode_attention(q16, q_is_bf16: bool, segments, seq_lens_per_seg, scale: fl
             bits, G = seg["bits"], seg["group"]
             vm = seg["v_meta"][b, h, :L] if bits != 16 else None
             fmt = seg.get("fmt", "int")
+            if fmt == "oaken":
+                kp, vp = seg["k_oaken"], seg["v_oaken"]
+                Ks.append(oaken_dequantize_rows(seg["k_codes"][b, h, :L], seg["k_meta"][b, h, :L],
+                                                D, kp[0], kp[1], kp[2]))
+                Vs.append(oaken_dequantize_rows(seg["v_codes"][b, h, :L], seg["v_meta"][b, h, :L],
+                                                D, vp[0], vp[1], vp[2]))
+                continue
             if seg.get("k_channels", False):
                 Ks.append(dequantize_channels(seg["k_codes"][b, h, :L], seg["k_meta"][b, h], L,
                                               D, bits))

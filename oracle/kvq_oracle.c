@@ -13,7 +13,11 @@
  *
  * Sources (page title, section):
  *   [P1] "大模型KV缓存量化技术：原理、优化与实践", section 2.1 (static global
- *        quantization: scale = (max - min) / (2^bits - 1)).
+ *        quantization: scale = (max - min) / (2^bits - 1)); sections 3.1
+ *        (Oaken: offline thresholds, online group-shift quantization,
+ *        dense-sparse encoding), 3.2.1 (threshold zones and their widths)
+ *        and 3.2.2 (group shift: Delta = value - T_hi or value - T_lo,
+ *        dequantized as T + Delta * scale).
  *   [P2] "大模型推理加速之KV Cache量化压缩原理与工程实现": the KV-cache size
  *        formula (2 * layers * kv_heads * head_dim * seq_len * batch * bytes);
  *        "常见问题排查" (scale clamped to at least 1e-5); INT4 asymmetric
@@ -87,9 +91,34 @@
  *       in E = 31; the scale as R14 with 57344 for 448 (s = max(amax /
  *       57344, 1e-5), fp16 rounded up); codes the nearest E5M2 value of x /
  *       s, ties to even, saturating at +-57344 (never an infinity).
+ *   R18 Oaken group-shift codec ([P1] 3.1 online phase, 3.2.1 zones,
+ *       3.2.2 group shift).  The thresholds are fixed offline per plane and
+ *       given as an inner scale s_in (an fp16 value) and an integer inner
+ *       zero point z_in in [0, 15]: T_lo = -z_in * s_in, T_hi = (15 - z_in)
+ *       * s_in, both exact in fp32, so the thresholds sit on the inner grid.
+ *       The outer scale s_out > 0 and the outer width b in {5, 6, 7} are
+ *       fixed offline too.  Per element v (fp16 read exactly into fp32):
+ *         T_lo <= v <= T_hi: c = clamp(rint(v / s_in) + z_in, 0, 15) (the
+ *           listing's quantize(value, inner_scale), with R1, R5), no
+ *           outlier.  The page's inner and middle zones (both 4-bit) are
+ *           this one quantizer: the listing has a single non-outer branch.
+ *         v > T_hi: c = 15 and the outlier Delta = v - T_hi (one fp32
+ *           subtraction) is kept as m = min(rint(Delta / s_out), 2^b - 1).
+ *         v < T_lo: c = 0, Delta = v - T_lo, m = min(rint(-Delta / s_out),
+ *           2^b - 1), kept as -m.
+ *       Dense-sparse storage: the codes c are packed like 4-bit integer
+ *       codes (R7).  A row's outliers go, in ascending dim order, to 16
+ *       slots of 16 bits each (low byte the dim, high byte the signed m as
+ *       a two's complement byte).  Slots after the last outlier hold 0.
+ *       Outliers after the 16th are dropped, so those elements reconstruct
+ *       to their threshold.  x_hat = (c - z_in) * s_in + d * s_out, where d
+ *       is the element's signed slot value (0 without a slot).  For an
+ *       outlier that is T_hi + m * s_out or T_lo - m * s_out: the page's
+ *       dequantization T + Delta_hat.
  *
  * Code formats (the `fmt` arguments): 0 asymmetric integer codes of `bits`
- * bits (R1-R7), 1 E4M3 (R14), 2 symmetric INT8 (R15), 3 E5M2 (R17).
+ * bits (R1-R7), 1 E4M3 (R14), 2 symmetric INT8 (R15), 3 E5M2 (R17).  The
+ * Oaken codec (R18) has functions of its own.
  */
 #include <math.h>
 #include <stdint.h>
@@ -470,6 +499,87 @@ void kvqo_quantize_rows_sym8(const uint16_t *x, int64_t n_rows, int D, int G, ui
             meta[(r * (D / G) + g) * 2 + 0] = s16;
             meta[(r * (D / G) + g) * 2 + 1] = 0; /* zero point 0 */
         }
+}
+
+/* Oaken group-shift codec ([P1] 3.1, 3.2.2; R18): one row of D binary16
+ * values to packed 4-bit codes (D / 2 bytes) and 16 outlier slots. */
+#define KVQO_OAKEN_SLOTS 16
+
+void kvqo_oaken_quantize_row(const uint16_t *x, int D, float s_in, int z_in, float s_out,
+                             int outer_bits, uint8_t *codes, uint16_t *slots)
+{
+    const float z = (float)z_in;
+    const float t_lo = -z * s_in;
+    const float t_hi = (15.0f - z) * s_in;
+    const float m_max = (float)((1 << outer_bits) - 1);
+    int n_slot = 0;
+    memset(codes, 0, (size_t)D / 2);
+    for (int i = 0; i < KVQO_OAKEN_SLOTS; ++i)
+        slots[i] = 0;
+    for (int j = 0; j < D; ++j) {
+        const float v = kvqo_f16_to_f32(x[j]);
+        unsigned c;
+        int outlier = 0, d = 0;
+        if (v > t_hi) { /* outer zone, high side: shift by T_hi */
+            const float delta = v - t_hi;
+            float m = rintf(delta / s_out);
+            if (m > m_max)
+                m = m_max;
+            c = 15;
+            outlier = 1;
+            d = (int)m;
+        } else if (v < t_lo) { /* outer zone, low side: shift by T_lo */
+            const float delta = v - t_lo;
+            float m = rintf(-delta / s_out);
+            if (m > m_max)
+                m = m_max;
+            c = 0;
+            outlier = 1;
+            d = -(int)m;
+        } else { /* inner and middle zones: the 4-bit inner quantizer */
+            float cf = rintf(v / s_in) + z;
+            if (cf < 0.0f)
+                cf = 0.0f;
+            if (cf > 15.0f)
+                cf = 15.0f;
+            c = (unsigned)cf;
+        }
+        codes[j / 2] |= (uint8_t)(c << ((j % 2) * 4));
+        if (outlier && n_slot < KVQO_OAKEN_SLOTS) {
+            slots[n_slot] = (uint16_t)((unsigned)j | ((unsigned)(uint8_t)(int8_t)d << 8));
+            ++n_slot;
+        }
+    }
+}
+
+void kvqo_oaken_quantize_rows(const uint16_t *x, int64_t n_rows, int D, float s_in, int z_in,
+                              float s_out, int outer_bits, uint8_t *codes, uint16_t *slots)
+{
+    for (int64_t r = 0; r < n_rows; ++r)
+        kvqo_oaken_quantize_row(x + r * D, D, s_in, z_in, s_out, outer_bits,
+                                codes + r * (D / 2), slots + r * KVQO_OAKEN_SLOTS);
+}
+
+/* x_hat = (c - z_in) * s_in + d * s_out in fp64 (R18); the dense part is the
+ * threshold for an outlier, the slot adds its shifted magnitude. */
+void kvqo_oaken_dequantize_rows(const uint8_t *codes, const uint16_t *slots, int64_t n_rows,
+                                int D, float s_in, int z_in, float s_out, double *out)
+{
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint8_t *row = codes + r * (D / 2);
+        double *o = out + r * D;
+        for (int j = 0; j < D; ++j) {
+            const unsigned c = (row[j / 2] >> ((j % 2) * 4)) & 15u;
+            o[j] = ((double)c - (double)z_in) * (double)s_in;
+        }
+        for (int i = 0; i < KVQO_OAKEN_SLOTS; ++i) {
+            const uint16_t w = slots[r * KVQO_OAKEN_SLOTS + i];
+            const int j = w & 0xff;
+            const int d = (int8_t)(uint8_t)(w >> 8);
+            if (j < D)
+                o[j] += (double)d * (double)s_out;
+        }
+    }
 }
 
 /* Unpack code e of a packed row (R7). */

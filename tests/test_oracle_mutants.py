@@ -70,6 +70,14 @@ MUTANTS = [
      "double quantum = ldexp(1.0, (e < -14 ? -14 : e) - 2);\n    double r = round(a / quantum) * quantum;"),
     ("e5m2 exponent bias 16", "v = ldexp((double)(4 + m), e - 17);", "v = ldexp((double)(4 + m), e - 18);"),
     ("e5m2 scale from the E4M3 maximum", "float s32 = amax / 57344.0f;", "float s32 = amax / 448.0f;"),
+    ("oaken high side shifted by the low threshold", "const float delta = v - t_hi;",
+     "const float delta = v - t_lo;"),
+    ("oaken outer ties away from zero", "float m = rintf(delta / s_out);", "float m = roundf(delta / s_out);"),
+    ("oaken inner zero point dropped", "float cf = rintf(v / s_in) + z;", "float cf = rintf(v / s_in);"),
+    ("oaken upper threshold one step high", "const float t_hi = (15.0f - z) * s_in;",
+     "const float t_hi = (16.0f - z) * s_in;"),
+    ("oaken outer magnitude one bit short", "const float m_max = (float)((1 << outer_bits) - 1);",
+     "const float m_max = (float)((1 << (outer_bits - 1)) - 1);"),
 ]
 
 
@@ -202,6 +210,15 @@ def _pins(o):
     m5 = np.clip((f5[:-1] + f5[1:]) / 2, -57344, 57344).astype(np.float32)
     yield "e5m2 encode vs torch", bool(np.array_equal(
         o.f32_to_e5m2(m5), torch.from_numpy(m5).to(torch.float8_e5m2).view(torch.uint8).numpy()))
+
+    ok = True
+    for r in _golden("oaken_worked_example.json")["rows"]:
+        x = np.asarray(r["x"], np.float16).view(np.uint16)[None]
+        c, sl = o.oaken_quantize_rows(x, r["s_in"], r["z_in"], r["s_out"], r["outer_bits"])
+        xh = o.oaken_dequantize_rows(c, sl, x.shape[1], r["s_in"], r["z_in"], r["s_out"])
+        ok &= (c[0].tolist() == r["codes"] and sl[0].tolist() == [int(v, 16) for v in r["slots"]]
+               and xh[0].tolist() == r["x_hat"])
+    yield "oaken worked rows", bool(ok)
 
     t = _golden("chunk_threshold_toy.json")
     sim, cls = o.chunk_assign(np.array(t["chunks"], np.float32), np.array(t["query"], np.float32),
