@@ -34,10 +34,12 @@ sys.path.insert(0, ROOT)
 METRIC = "quantized-KV decode attention tokens/s; KV-read GB/s as % of B200 HBM peak"
 DTYPE = {2: "u2", 4: "u4", 8: "u8", 16: "f16"}
 # code formats: arithmetic type, JSON name, and the library's format code
-FMT_DTYPE = {"fp8": "e4m3", "sym8": "s8", "e5m2": "e5m2"}
-FMT_NAME = {"fp8": "fp8 e4m3", "sym8": "symmetric int8", "e5m2": "fp8 e5m2"}
-# KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM, KVQ_FMT_FP8_E5M2
-FMT_CODE = {"int": 0, "fp8": 1, "sym8": 2, "e5m2": 3}
+FMT_DTYPE = {"fp8": "e4m3", "sym8": "s8", "e5m2": "e5m2", "oaken": "u4"}
+FMT_NAME = {"fp8": "fp8 e4m3", "sym8": "symmetric int8", "e5m2": "fp8 e5m2",
+            "oaken": "oaken group-shift (4-bit dense + 16 outlier slots)"}
+# KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM, KVQ_FMT_FP8_E5M2, KVQ_FMT_OAKEN
+FMT_CODE = {"int": 0, "fp8": 1, "sym8": 2, "e5m2": 3, "oaken": 4}
+OAKEN_SLOTS = 16
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
@@ -65,9 +67,12 @@ def measured_peak():
 
 
 def bytes_per_head_token(bits: int, group: int, head_dim: int = 128,
-                         k_channels: bool = False) -> int:
+                         k_channels: bool = False, fmt: str = "int") -> int:
     """K plus V bytes of one (sequence, KV head, token): codes + (s, z) pairs
-    (per-channel K: head_dim pairs per 32-token block, 16 bytes a token)."""
+    (per-channel K: head_dim pairs per 32-token block, 16 bytes a token;
+    the Oaken codec: 4-bit codes + 16 two-byte outlier slots per row)."""
+    if fmt == "oaken":
+        return 2 * (head_dim // 2 + 2 * OAKEN_SLOTS)
     meta = 0 if bits == 16 else (head_dim // group) * 4
     kmeta = head_dim * 4 // 32 if k_channels else meta
     return 2 * (head_dim * bits // 8) + meta + kmeta
@@ -89,6 +94,8 @@ def split_kernel_name(wl) -> str:
     """The decode kernel the library picks for this workload's formats: the
     tokens-on-M kernel when (head_dim / G) * g <= 8, else the 16-row one."""
     g = wl.q_heads // wl.kv_heads
+    if wl.fmt == "oaken":
+        return "oaken_decode_kernel"
     groups = [128, wl.group] if wl.chunk_tokens else [wl.group]  # + the FP16 segment
     ok = all((128 // G) * g <= 8 for G in groups)
     return "decode_tm_kernel" if ok else "decode_split_kernel"
@@ -174,23 +181,34 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- reference arm
 
-def channel_oracle_pairs(wl, k, v, q, pairs):
-    """Oracle inputs of (sequence, KV head) pairs of a per-channel-K workload:
-    K quantized per channel over 32-token blocks, V per token; each entry is
-    (q patterns [1, g, D], the one-pair segment, its length)."""
+def segment_oracle_pairs(wl, k, v, q, pairs):
+    """Oracle inputs of (sequence, KV head) pairs of an attention-only
+    workload: K per channel over 32-token blocks and V per token, or both
+    planes in the Oaken codec; each entry is (q patterns [1, g, D], the
+    one-pair segment, its length)."""
     import numpy as np
     import torch
 
     import oracle
+    import workloads
     g = wl.group_ratio
     out = []
+    if wl.fmt == "oaken":
+        kp, vp = workloads.oaken_params(wl, "k"), workloads.oaken_params(wl, "v")
     for b, h in pairs:
         kk = k[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
         vv = v[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-        kc, km = oracle.quantize_cache_channels(kk, wl.bits)
-        vc, vm = oracle.quantize_rows(vv, wl.group, wl.bits)
-        seg = dict(k_codes=kc[None, None], k_meta=km[None, None], v_codes=vc[None, None],
-                   v_meta=vm[None, None], bits=wl.bits, group=wl.group, k_channels=True)
+        if wl.fmt == "oaken":
+            kc, km = oracle.oaken_quantize_rows(kk, *kp)
+            vc, vm = oracle.oaken_quantize_rows(vv, *vp)
+            seg = dict(k_codes=kc[None, None], k_meta=km[None, None], v_codes=vc[None, None],
+                       v_meta=vm[None, None], bits=4, group=128, fmt="oaken", k_oaken=kp,
+                       v_oaken=vp)
+        else:
+            kc, km = oracle.quantize_cache_channels(kk, wl.bits)
+            vc, vm = oracle.quantize_rows(vv, wl.group, wl.bits)
+            seg = dict(k_codes=kc[None, None], k_meta=km[None, None], v_codes=vc[None, None],
+                       v_meta=vm[None, None], bits=wl.bits, group=wl.group, k_channels=True)
         qh = q[b, h * g:(h + 1) * g].cpu().contiguous().view(torch.int16).numpy()
         out.append((qh.view(np.uint16)[None], seg, [np.array([kk.shape[0]])]))
     return out
@@ -226,12 +244,12 @@ def run_reference(args, wl):
                   f"({wl.kv_heads}) / seconds")
         print(json.dumps(reference_line(args, wl, value, el, sample)), flush=True)
         return
-    if wl.k_axis == "channel":
+    if wl.k_axis == "channel" or wl.fmt == "oaken":
         sub = wl.scaled(batch=1, kv_heads=min(wl.kv_heads, 4),
                         q_heads=min(wl.kv_heads, 4) * wl.group_ratio)
         k, v = workloads.kv_tokens(sub, wl.context, "cpu")
         q = workloads.queries(sub, "cpu")
-        prepared = channel_oracle_pairs(wl, k, v, q, [(0, h) for h in range(sub.kv_heads)])
+        prepared = segment_oracle_pairs(wl, k, v, q, [(0, h) for h in range(sub.kv_heads)])
 
         def kpc_step(i):
             qh, seg, lens = prepared[i % len(prepared)]
@@ -243,8 +261,9 @@ def run_reference(args, wl):
             kpc_step(i)
         el = time.perf_counter() - t0
         value = args.steps / wl.kv_heads / el
+        how = "Oaken codec" if wl.fmt == "oaken" else "K per channel"
         sample = (f"each step: one (sequence, KV head) of {wl.name}: attention of "
-                  f"{wl.group_ratio} query heads over {wl.context} tokens, K per channel; "
+                  f"{wl.group_ratio} query heads over {wl.context} tokens, {how}; "
                   f"tokens/s = steps / kv_heads ({wl.kv_heads}) / seconds")
         print(json.dumps(reference_line(args, wl, value, el, sample)), flush=True)
         return
@@ -325,8 +344,8 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
     import oracle
     g = wl.group_ratio
     pairs = [(b, h) for b in range(min(wl.batch, 2)) for h in range(min(wl.kv_heads, 4))]
-    if wl.k_axis == "channel":
-        prep = channel_oracle_pairs(wl, k, v, q, pairs)
+    if wl.k_axis == "channel" or wl.fmt == "oaken":
+        prep = segment_oracle_pairs(wl, k, v, q, pairs)
         n = 0
         t0 = time.perf_counter()
         while True:
@@ -338,7 +357,9 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
                 break
         return {"value": n / wl.kv_heads / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                 "sample": f"{n} (sequence, KV head) attentions of {wl.name} over "
-                          f"{k.shape[2]} tokens (K per channel) cycling over {len(prep)} pairs, "
+                          f"{k.shape[2]} tokens ("
+                          f"{'Oaken codec' if wl.fmt == 'oaken' else 'K per channel'}) "
+                          f"cycling over {len(prep)} pairs, "
                           f"{el:.1f} s on one host thread; tokens/s = pairs / kv_heads / seconds"}
     prepared = []
     for b, h in pairs:
@@ -515,9 +536,11 @@ def run_kvq(args, wl, rank, world, local_rank):
     else:
         max_tokens = workloads.round_up(ctx + episode + 1, 64)
         k, v = workloads.kv_tokens(wlr, ctx, dev)
+        oaken = ({"k_oaken": workloads.oaken_params(wl, "k"),
+                  "v_oaken": workloads.oaken_params(wl, "v")} if wl.fmt == "oaken" else {})
         cache = kvq.QuantizedKVCache.allocate(
             B, H, D, max_tokens, wl.bits, wl.group, dev,
-            fmt=FMT_CODE[wl.fmt], k_axis=1 if kpc else 0)
+            fmt=FMT_CODE[wl.fmt], k_axis=1 if kpc else 0, **oaken)
         cache.seq_lens.zero_()
         kvq.kvq_quantize_append(cache, k, v, ctx, advance_seq_lens=True)
         base_lens = cache.seq_lens.clone()
@@ -534,9 +557,12 @@ def run_kvq(args, wl, rank, world, local_rank):
         pf_ev[1].record()
         torch.cuda.synchronize()
         pf_us = pf_ev[0].elapsed_time(pf_ev[1]) * 1e3 / pf_reps
-        pf_bytes = B * H * ctx * (2 * D * 2 + bytes_per_head_token(wl.bits, wl.group, D, kpc))
+        pf_bytes = B * H * ctx * (2 * D * 2 + bytes_per_head_token(wl.bits, wl.group, D, kpc,
+                                                                   wl.fmt))
         prefill = {"tokens": B * ctx, "us": pf_us, "bytes": pf_bytes,
-                   "gbs": pf_bytes / (pf_us / 1e6) / 1e9, "kernel": "quantize_bulk_kernel",
+                   "gbs": pf_bytes / (pf_us / 1e6) / 1e9,
+                   "kernel": ("oaken_quantize_kernel" if wl.fmt == "oaken"
+                              else "quantize_bulk_kernel"),
                    "note": "fp16 K and V read + packed codes and (s, z) written, per launch "
                            "(3 launches, each after a 4-byte seq_lens reset)"}
         segs = [cache]
@@ -588,7 +614,7 @@ def run_kvq(args, wl, rank, world, local_rank):
             return sum(int(ln.sum()) * H * bytes_per_head_token(bits, wl.group, D)
                        for ln, bits in zip(seg_lens, seg_bits))
         L = ctx + (s % episode) + 1 if wl.append else ctx
-        return B * H * L * bytes_per_head_token(wl.bits, wl.group, D, kpc)
+        return B * H * L * bytes_per_head_token(wl.bits, wl.group, D, kpc, wl.fmt)
 
     # ---- warm-up (eager; also makes the one-time kernel attribute settings)
     for s in range(args.warmup):

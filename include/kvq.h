@@ -71,7 +71,8 @@ typedef enum kvq_format {
     KVQ_FMT_INT = 0,      /* asymmetric integer codes: x_hat = (c - z) * s    */
     KVQ_FMT_FP8_E4M3 = 1, /* FP8 E4M3 codes, bits 8: x_hat = e4m3(c) * s      */
     KVQ_FMT_INT8_SYM = 2, /* symmetric INT8 codes, bits 8: x_hat = c * s      */
-    KVQ_FMT_FP8_E5M2 = 3  /* FP8 E5M2 codes, bits 8: x_hat = e5m2(c) * s      */
+    KVQ_FMT_FP8_E5M2 = 3, /* FP8 E5M2 codes, bits 8: x_hat = e5m2(c) * s      */
+    KVQ_FMT_OAKEN = 4     /* Oaken group-shift codes, bits 4 (see below)     */
 } kvq_format;
 
 /* Grouping axis of a plane's (scale, zero point) pairs. */
@@ -82,6 +83,27 @@ typedef enum kvq_axis {
 } kvq_axis;
 
 #define KVQ_CHANNEL_BLOCK 32
+
+/* Outlier slots per token row of a KVQ_FMT_OAKEN plane. */
+#define KVQ_OAKEN_SLOTS 16
+
+/*
+ * Offline parameters of a KVQ_FMT_OAKEN plane (the "大模型KV缓存量化技术：
+ * 原理、优化与实践" page, section 3.1: thresholds fixed before deployment,
+ * applied online; 3.2.1: outer zone 5-7 bits, inner and middle 4 bits).
+ *   inner_scale s_in: a positive fp16 value (held here as a float);
+ *   inner_zero z_in: integer in [0, 15]; the thresholds are T_lo = -z_in *
+ *     s_in and T_hi = (15 - z_in) * s_in, both on the inner grid;
+ *   outer_scale s_out: positive and finite;
+ *   outer_bits b: 5, 6 or 7 (outlier magnitudes up to 2^b - 1).
+ * Ignored for the other formats.
+ */
+typedef struct kvq_oaken {
+    float inner_scale;
+    int32_t inner_zero;
+    float outer_scale;
+    int32_t outer_bits;
+} kvq_oaken;
 
 /*
  * One K or V plane of a cache (one bit-width).
@@ -113,6 +135,22 @@ typedef enum kvq_axis {
  *                 token groups); group_size is not used for this plane.
  *                 Only whole blocks are quantized: the tokens of an
  *                 unfinished block belong in a separate bits-16 segment.
+ *   bits 4 with fmt KVQ_FMT_OAKEN (group_size = head_dim): the Oaken
+ *                 group-shift codec of the same page's sections 3.1, 3.2.1
+ *                 and 3.2.2, with the plane's offline kvq_oaken parameters.
+ *                 Per element v: T_lo <= v <= T_hi gives c = clamp(rne(v /
+ *                 s_in) + z_in, 0, 15); v > T_hi gives c = 15 and an outlier
+ *                 m = min(rne((v - T_hi) / s_out), 2^b - 1); v < T_lo gives
+ *                 c = 0 and an outlier -min(rne((T_lo - v) / s_out), 2^b - 1)
+ *                 (fp32, one subtraction and one division each).  Codes
+ *                 are packed like 4-bit codes.  meta u16
+ *                 [batch][kv_heads][max_tokens][KVQ_OAKEN_SLOTS] holds the
+ *                 row's outliers in ascending dim order (low byte the dim,
+ *                 high byte the signed magnitude as a two's complement
+ *                 byte), then zeros; outliers after the KVQ_OAKEN_SLOTS-th
+ *                 are dropped.  x_hat = (c - z_in) * s_in + d * s_out with d
+ *                 the element's slot value (0 without one): the page's
+ *                 T_hi + Delta * scale and T_lo + Delta * scale.
  *   bits 16:      codes f16 [batch][kv_heads][max_tokens][head_dim] raw
  *                 values (Cocktail's FP16 class); meta unused (may be NULL).
  * Both buffers 16-byte aligned.
@@ -124,6 +162,7 @@ typedef struct kvq_plane {
     void *meta;         /* device; NULL when bits == 16                     */
     int32_t fmt;        /* kvq_format; the FP8 and INT8_SYM formats: bits 8 */
     int32_t axis;       /* kvq_axis; KVQ_AXIS_CHANNEL on the K plane only   */
+    kvq_oaken oaken;    /* KVQ_FMT_OAKEN only                               */
 } kvq_plane;
 
 /*

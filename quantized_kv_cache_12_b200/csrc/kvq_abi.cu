@@ -20,20 +20,44 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool valid_group(int g) { return g == 32 || g == 64 || g == 128; }
 
-// The kernels' template tag of a plane's format: its bit width, kE4M3 or kSym8.
+// The kernels' template tag of a plane's format: its bit width, or kE4M3, kE5M2,
+// kSym8 or kOaken.
 int kernel_bits(const kvq_plane& p) {
   return p.fmt == KVQ_FMT_FP8_E4M3   ? kvq::kE4M3
          : p.fmt == KVQ_FMT_FP8_E5M2 ? kvq::kE5M2
          : p.fmt == KVQ_FMT_INT8_SYM ? kvq::kSym8
+         : p.fmt == KVQ_FMT_OAKEN    ? kvq::kOaken
                                      : p.bits;
+}
+
+// An Oaken plane's offline parameters: s_in a positive fp16 value, z_in in
+// [0, 15], s_out positive and finite, b in 5..7.
+bool valid_oaken(const kvq_oaken& o) {
+  if (!(o.inner_scale > 0.0f) || !isfinite(o.inner_scale)) return false;
+  if (__half2float(__float2half_rn(o.inner_scale)) != o.inner_scale) return false;
+  if (o.inner_zero < 0 || o.inner_zero > 15) return false;
+  if (!(o.outer_scale > 0.0f) || !isfinite(o.outer_scale)) return false;
+  return o.outer_bits >= 5 && o.outer_bits <= 7;
+}
+
+kvq::OakenParams oaken_params(const kvq_plane& p) {
+  return kvq::make_oaken_params(p.oaken.inner_scale, p.oaken.inner_zero, p.oaken.outer_scale,
+                                p.oaken.outer_bits);
 }
 
 kvq_status check_plane(const kvq_plane& p, int head_dim, bool allow16, bool is_k) {
   if (p.codes == nullptr || !aligned16(p.codes)) return KVQ_ERR_INVALID_ARG;
   if (p.fmt != KVQ_FMT_INT && p.fmt != KVQ_FMT_FP8_E4M3 && p.fmt != KVQ_FMT_INT8_SYM &&
-      p.fmt != KVQ_FMT_FP8_E5M2)
+      p.fmt != KVQ_FMT_FP8_E5M2 && p.fmt != KVQ_FMT_OAKEN)
     return KVQ_ERR_INVALID_ARG;
   if (p.axis != KVQ_AXIS_TOKEN && p.axis != KVQ_AXIS_CHANNEL) return KVQ_ERR_INVALID_ARG;
+  if (p.fmt == KVQ_FMT_OAKEN) {
+    if (p.bits != 4 || p.axis != KVQ_AXIS_TOKEN || p.group_size != head_dim)
+      return KVQ_ERR_UNSUPPORTED;
+    if (!valid_oaken(p.oaken)) return KVQ_ERR_INVALID_ARG;
+    if (p.meta == nullptr || !aligned16(p.meta)) return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+  }
   if (p.fmt != KVQ_FMT_INT && p.bits != 8) return KVQ_ERR_UNSUPPORTED;
   if (p.axis == KVQ_AXIS_CHANNEL &&
       (!is_k || p.fmt != KVQ_FMT_INT || !(p.bits == 2 || p.bits == 4 || p.bits == 8)))
@@ -264,6 +288,13 @@ kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const 
   a.side0 = 0;
   a.k_channels = cache->k.axis == KVQ_AXIS_CHANNEL;
   if (a.k_channels && n_new % KVQ_CHANNEL_BLOCK != 0) return KVQ_ERR_INVALID_ARG;
+  if (cache->k.fmt == KVQ_FMT_OAKEN) {
+    a.k_oaken = oaken_params(cache->k);
+    a.v_oaken = oaken_params(cache->v);
+    return kvq::launch_oaken_quantize(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KVQ_OK
+               : KVQ_ERR_CUDA;
+  }
   cudaError_t e = kvq::launch_quantize(a, kernel_bits(cache->k), cache->k.group_size,
                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
@@ -344,6 +375,10 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
     v.max_tokens = segs[i].max_tokens;
     v.n_split = plan.n_split[i];
     v.wide = plan.wide[i];
+    if (segs[i].k.fmt == KVQ_FMT_OAKEN) {
+      v.k_oaken = oaken_params(segs[i].k);
+      v.v_oaken = oaken_params(segs[i].v);
+    }
     v.part_base = base;
     base += plan.n_split[i];
     if ((stages & kPartials) && kvq::launch_decode_segment(a, v, s) != cudaSuccess)

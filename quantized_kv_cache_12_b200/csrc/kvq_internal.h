@@ -17,7 +17,17 @@ constexpr int kE4M3 = 0x108;
 constexpr int kSym8 = 0x208;
 // FP8 E5M2 codes (bias 15, two mantissa bits); code_bits 8
 constexpr int kE5M2 = 0x308;
+// the Oaken group-shift codec (4-bit dense codes plus outlier slots)
+constexpr int kOaken = 0x404;
 __host__ __device__ constexpr int code_bits(int tag) { return tag & 0xFF; }
+
+// A KVQ_FMT_OAKEN plane's offline parameters as the kernels use them:
+// T_lo = -z s_in, T_hi = (15 - z) s_in, r_in = 1 / s_in (rounded to
+// nearest), outlier magnitudes up to m_max = 2^b - 1.
+struct OakenParams {
+  float s_in, r_in, z, t_lo, t_hi, s_out, m_max;
+};
+OakenParams make_oaken_params(float s_in, int z_in, float s_out, int outer_bits);
 
 // One K/V plane pair of one cache segment, as the kernels see it.
 struct SegView {
@@ -33,6 +43,7 @@ struct SegView {
   int32_t part_base;     // index of this segment's first partial
   int32_t k_channels;    // K grouped per channel over kChannelBlock-token blocks
   int32_t wide;          // run the five-CTAs-per-SM build of the format
+  OakenParams k_oaken, v_oaken;  // bits == kOaken: the planes' parameters
 };
 
 struct DecodeArgs {
@@ -71,6 +82,7 @@ struct QuantArgs {
   // written and not advanced
   int32_t side0;
   int32_t k_channels;
+  OakenParams k_oaken, v_oaken;  // Oaken planes (launch_oaken_quantize)
 };
 // tokens per block of a per-channel K plane
 constexpr int kChannelBlock = 32;
@@ -89,6 +101,12 @@ int decode_tm_wide_ctas_per_sm(int bits, int group, int group_ratio, bool kpc = 
 cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s);
+// the Oaken codec (kvq_oaken.cu): quantize-on-write of both planes (and the
+// seq_lens advance), and its decode-attention kernel (g = 1, 2, 4, 8)
+cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s);
+bool decode_oaken_supported(int group_ratio);
+int decode_oaken_ctas_per_sm(int group_ratio);
+cudaError_t launch_decode_oaken(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 // leading workspace bytes that hold the header and the counters (they must
 // be zero before a call whose cache shape differs from the previous call's)
 size_t decode_zeroed_prefix_bytes(const kvq_cache* segs);

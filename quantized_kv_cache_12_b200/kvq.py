@@ -24,9 +24,10 @@ LIB_PATH = os.path.join(_PKG, "libkvq.so")
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, \
     KVQ_ERR_CUDA = range(6)
 KVQ_F16, KVQ_BF16 = 0, 1
-KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM, KVQ_FMT_FP8_E5M2 = 0, 1, 2, 3
+KVQ_FMT_INT, KVQ_FMT_FP8_E4M3, KVQ_FMT_INT8_SYM, KVQ_FMT_FP8_E5M2, KVQ_FMT_OAKEN = 0, 1, 2, 3, 4
 KVQ_AXIS_TOKEN, KVQ_AXIS_CHANNEL = 0, 1
 KVQ_CHANNEL_BLOCK = 32
+KVQ_OAKEN_SLOTS = 16
 HEADER_BYTES = 256  # workspace header: sticky device error word first
 
 
@@ -36,10 +37,15 @@ class KvqError(RuntimeError):
         super().__init__(f"{where}: {kvq_status_string(status)} (status {status})")
 
 
+class kvq_oaken(ctypes.Structure):
+    _fields_ = [("inner_scale", ctypes.c_float), ("inner_zero", ctypes.c_int32),
+                ("outer_scale", ctypes.c_float), ("outer_bits", ctypes.c_int32)]
+
+
 class kvq_plane(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32),
                 ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("fmt", ctypes.c_int32),
-                ("axis", ctypes.c_int32)]
+                ("axis", ctypes.c_int32), ("oaken", kvq_oaken)]
 
 
 class kvq_cache(ctypes.Structure):
@@ -260,6 +266,10 @@ class QuantizedKVCache:
     k_axis: KVQ_AXIS_TOKEN, or KVQ_AXIS_CHANNEL (K grouped per channel over
     blocks of KVQ_CHANNEL_BLOCK tokens: k_meta fp16 [B, H_kv,
     max_tokens / KVQ_CHANNEL_BLOCK, head_dim, 2]; group_size is V's).
+    fmt KVQ_FMT_OAKEN (bits 4, group_size = head_dim): meta holds the outlier
+    slots, int16 [B, H_kv, max_tokens, KVQ_OAKEN_SLOTS] (16-bit words), and
+    k_oaken / v_oaken the planes' offline (inner_scale, inner_zero,
+    outer_scale, outer_bits).
     """
     batch: int
     kv_heads: int
@@ -274,16 +284,23 @@ class QuantizedKVCache:
     seq_lens: torch.Tensor
     fmt: int = KVQ_FMT_INT
     k_axis: int = KVQ_AXIS_TOKEN
+    k_oaken: Optional[tuple] = None
+    v_oaken: Optional[tuple] = None
 
     @classmethod
     def allocate(cls, batch, kv_heads, head_dim, max_tokens, bits, group_size, device="cuda",
-                 fmt: int = KVQ_FMT_INT, k_axis: int = KVQ_AXIS_TOKEN):
+                 fmt: int = KVQ_FMT_INT, k_axis: int = KVQ_AXIS_TOKEN, k_oaken=None,
+                 v_oaken=None):
         rb = head_dim * bits // 8
         shape = (batch, kv_heads, max_tokens, rb)
         k = torch.empty(shape, dtype=torch.uint8, device=device)
         v = torch.empty(shape, dtype=torch.uint8, device=device)
         km = vm = None
-        if bits != 16:
+        if fmt == KVQ_FMT_OAKEN:
+            sshape = (batch, kv_heads, max_tokens, KVQ_OAKEN_SLOTS)
+            km = torch.empty(sshape, dtype=torch.int16, device=device)
+            vm = torch.empty(sshape, dtype=torch.int16, device=device)
+        elif bits != 16:
             mshape = (batch, kv_heads, max_tokens, head_dim // group_size, 2)
             kshape = ((batch, kv_heads, max_tokens // KVQ_CHANNEL_BLOCK, head_dim, 2)
                       if k_axis == KVQ_AXIS_CHANNEL else mshape)
@@ -291,7 +308,7 @@ class QuantizedKVCache:
             vm = torch.empty(mshape, dtype=torch.float16, device=device)
         lens = torch.zeros(batch, dtype=torch.int32, device=device)
         return cls(batch, kv_heads, head_dim, max_tokens, bits, group_size, k, v, km, vm, lens,
-                   fmt, k_axis)
+                   fmt, k_axis, k_oaken, v_oaken)
 
     def struct_array(self) -> ctypes.Array:
         """A one-element kvq_cache array for this cache, built on first use
@@ -308,10 +325,10 @@ class QuantizedKVCache:
                                                          self.head_dim, self.max_tokens)
         c.k = kvq_plane(self.bits, self.group_size, self.k_codes.data_ptr(),
                         self.k_meta.data_ptr() if self.k_meta is not None else None, self.fmt,
-                        self.k_axis)
+                        self.k_axis, kvq_oaken(*(self.k_oaken or (0.0, 0, 0.0, 0))))
         c.v = kvq_plane(self.bits, self.group_size, self.v_codes.data_ptr(),
                         self.v_meta.data_ptr() if self.v_meta is not None else None, self.fmt,
-                        KVQ_AXIS_TOKEN)
+                        KVQ_AXIS_TOKEN, kvq_oaken(*(self.v_oaken or (0.0, 0, 0.0, 0))))
         c.seq_lens = self.seq_lens.data_ptr()
         return c
 

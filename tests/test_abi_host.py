@@ -314,3 +314,66 @@ def test_chunk_entry_points_reject_bad_arguments(kvq):
     wrong = (kvq.kvq_cache * 3)(segs[1], segs[0], segs[2])
     assert lib.kvq_chunk_reorder(wrong, fake, fake, 1024, 32, fake, fake, None) == \
         kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_oaken_planes_validated(kvq):
+    """KVQ_FMT_OAKEN needs bits 4, group_size = head_dim, the token axis, the
+    same format on K and V, and offline parameters in range (inner_scale a
+    positive fp16 value, inner_zero in [0, 15], outer_scale positive and
+    finite, outer_bits 5 to 7); its decode is built for g = 1, 2, 4, 8."""
+    fake = ctypes.c_void_p(0x60000)
+
+    def oaken_cache(kp=(0.25, 8, 0.5, 5), vp=(0.125, 3, 0.05, 7), bits=4, group=128, kv_heads=2):
+        c = _fake_cache(kvq, bits=bits, group=group, kv_heads=kv_heads)
+        c.k.fmt = c.v.fmt = kvq.KVQ_FMT_OAKEN
+        c.k.oaken = kvq.kvq_oaken(*kp)
+        c.v.oaken = kvq.kvq_oaken(*vp)
+        return c
+
+    def append_status(c):
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, 1, 1, None)
+
+    for g in (1, 2, 4, 8):
+        assert kvq.kvq_decode_workspace_bytes(oaken_cache(), 2 * g) > 0
+    assert _status(kvq.kvq_decode_workspace_bytes, oaken_cache(), 6) == kvq.KVQ_ERR_UNSUPPORTED
+    assert append_status(oaken_cache(bits=8)) == kvq.KVQ_ERR_UNSUPPORTED
+    assert append_status(oaken_cache(group=64)) == kvq.KVQ_ERR_UNSUPPORTED
+    for bad in [(0.3, 8, 0.5, 5),            # not an fp16 value
+                (0.0, 8, 0.5, 5), (float("nan"), 8, 0.5, 5),
+                (0.25, -1, 0.5, 5), (0.25, 16, 0.5, 5),
+                (0.25, 8, 0.0, 5), (0.25, 8, float("inf"), 5),
+                (0.25, 8, 0.5, 4), (0.25, 8, 0.5, 8)]:
+        assert append_status(oaken_cache(kp=bad)) == kvq.KVQ_ERR_INVALID_ARG, bad
+        assert append_status(oaken_cache(vp=bad)) == kvq.KVQ_ERR_INVALID_ARG, bad
+    c = oaken_cache()
+    c.k.meta = None
+    assert append_status(c) == kvq.KVQ_ERR_INVALID_ARG
+    c = oaken_cache()
+    c.v.fmt = kvq.KVQ_FMT_INT
+    c.v.bits = 4
+    assert append_status(c) in (kvq.KVQ_ERR_UNSUPPORTED, kvq.KVQ_ERR_INVALID_ARG)
+    c = oaken_cache()
+    c.k.axis = kvq.KVQ_AXIS_CHANNEL
+    assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_struct_layout_matches_the_header(kvq, tmp_path):
+    """The binding's ctypes structs have the header's sizes and offsets (a C
+    program built from include/kvq.h prints them)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc missing")
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include "kvq.h"\nint main(void) {\n'
+                   ' printf("%zu %zu %zu %zu %zu\\n", sizeof(kvq_plane), sizeof(kvq_cache),'
+                   ' offsetof(kvq_plane, oaken), offsetof(kvq_cache, v),'
+                   ' offsetof(kvq_cache, seq_lens));\n return 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)],
+                   check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    want = [ctypes.sizeof(kvq.kvq_plane), ctypes.sizeof(kvq.kvq_cache),
+            kvq.kvq_plane.oaken.offset, kvq.kvq_cache.v.offset, kvq.kvq_cache.seq_lens.offset]
+    assert got == want

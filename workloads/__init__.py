@@ -69,7 +69,9 @@ class DecodeWorkload:
     beta: float = 0.0
     low_bits: Tuple[int, ...] = ()   # bit-widths of the two quantized classes
     fmt: str = "int"          # code format: "int" (asymmetric integer), "fp8" (E4M3, bits 8),
-    #                           "e5m2" (E5M2, bits 8) or "sym8" (symmetric INT8, bits 8)
+    #                           "e5m2" (E5M2, bits 8), "sym8" (symmetric INT8, bits 8) or
+    #                           "oaken" (group-shift codec, bits 4, group = head_dim)
+    outer_bits: int = 5       # "oaken": bits of an outlier's shifted magnitude
     k_axis: str = "token"     # K grouping: "token" (groups along head_dim) or "channel"
     #                           (per channel over 32-token blocks; attention only)
 
@@ -129,6 +131,10 @@ WORKLOADS = {
         name="llama3_8b_gqa_int4_kpc", batch=32, q_heads=32, kv_heads=8, head_dim=128,
         context=8192, bits=4, group=64, q_dtype="f16", steps=100, append=False, seed=3,
         k_outliers=Outliers(factor=15.0, per_head=4), v_sigma=0.5, k_axis="channel"),
+    "llama3_8b_gqa_oaken": DecodeWorkload(
+        name="llama3_8b_gqa_oaken", batch=32, q_heads=32, kv_heads=8, head_dim=128,
+        context=8192, bits=4, group=128, q_dtype="f16", steps=100, append=False, seed=3,
+        k_outliers=Outliers(factor=15.0, per_head=4), v_sigma=0.5, fmt="oaken"),
     "long_gqa_int4": DecodeWorkload(
         name="long_gqa_int4", batch=1, q_heads=32, kv_heads=8, head_dim=128,
         context=131072, bits=4, group=64, q_dtype="f16", steps=256, append=True, seed=5,
@@ -208,3 +214,32 @@ def chunk_embeddings(wl: DecodeWorkload, device, batch: Optional[int] = None):
 
 def round_up(x: int, m: int) -> int:
     return (x + m - 1) // m * m
+
+
+# stream of the calibration sample behind the Oaken planes' offline parameters
+_CALIBRATION_EXTRA = 1 << 20
+
+
+def oaken_params(wl: DecodeWorkload, which: str, n_tokens: int = 512):
+    """Offline parameters (inner_scale, inner_zero, outer_scale, outer_bits)
+    of the K ("k") or V ("v") plane of an "oaken" workload, from percentile
+    statistics of a calibration sample drawn like the workload's rows (an
+    independent stream, one sequence): the 2.5th and 97.5th percentiles
+    bound the 4-bit band, so about 5% of the values fall in the outer zone;
+    inner_scale is the smallest fp16 value with 15 steps spanning that band;
+    inner_zero puts the low percentile on the grid; outer_scale lets the
+    sample's extremes reach the largest outlier magnitude."""
+    k, v = kv_tokens(wl, n_tokens, "cpu", stream_extra=_CALIBRATION_EXTRA, batch=1)
+    x = (k if which == "k" else v).float().flatten()
+    lo = float(torch.quantile(x, 0.025))
+    hi = float(torch.quantile(x, 0.975))
+    span = torch.tensor((hi - lo) / 15.0, dtype=torch.float32)
+    s16 = span.half()
+    if s16.float() < span:
+        s16 = torch.nextafter(s16, torch.tensor(float("inf"), dtype=torch.float16))
+    s_in = float(s16)
+    z_in = int(min(max(round(-lo / s_in), 0), 15))
+    t_lo, t_hi = -z_in * s_in, (15 - z_in) * s_in
+    reach = max(float(x.max()) - t_hi, t_lo - float(x.min()), s_in)
+    s_out = float(torch.tensor(reach / ((1 << wl.outer_bits) - 1), dtype=torch.float32))
+    return s_in, z_in, s_out, wl.outer_bits
