@@ -84,7 +84,7 @@ def kernel_source_hash() -> str:
     # append's quantizer included), and the host code whose split plan picks
     # the kernel build and the units of a launch
     for f in ("kvq_decode.cu", "kvq_decode_tm.cu", "kvq_decode_common.cuh", "kvq_device.cuh",
-              "kvq_quant_core.cuh", "kvq_internal.h", "kvq_abi.cu"):
+              "kvq_quant_core.cuh", "kvq_internal.h", "kvq_abi.cu", "kvq_oaken.cu"):
         with open(os.path.join(ROOT, "quantized_kv_cache_12_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
