@@ -194,6 +194,8 @@ const char *kvq_version(void);
  * plus 4 bytes of (scale, zero) per group.
  * Returns KVQ_ERR_INVALID_ARG on non-positive sizes or null outputs,
  * KVQ_ERR_UNSUPPORTED on a (bits, G, head_dim) the library does not pack.
+ * (A KVQ_FMT_OAKEN plane's codes are those of bits 4; its meta holds
+ * KVQ_OAKEN_SLOTS * 2 bytes per token row instead of (scale, zero) pairs.)
  */
 kvq_status kvq_plane_bytes(int32_t batch, int32_t kv_heads, int32_t head_dim,
                            int32_t max_tokens, int32_t bits, int32_t group_size,
@@ -220,7 +222,9 @@ uint64_t kvq_kv_elements(uint64_t layers, uint64_t kv_heads, uint64_t head_dim,
  *                 (capped at max_tokens), in stream order.
  * Tokens whose position would reach max_tokens are not written (the
  * kernel checks on the device).  Both planes must have bits 2, 4 or 8 and
- * the same group size.  With a per-channel K plane (KVQ_AXIS_CHANNEL)
+ * the same group size.  KVQ_FMT_OAKEN planes (bits 4, G = head_dim) are
+ * encoded with their kvq_oaken parameters by one quantize kernel (half a
+ * warp per token row), then seq_lens advances.  With a per-channel K plane (KVQ_AXIS_CHANNEL)
  * n_new must be a multiple of KVQ_CHANNEL_BLOCK, and so must seq_lens[b]
  * on the device: a sequence whose length is not is neither written nor
  * advanced.  Errors: KVQ_ERR_INVALID_ARG (nulls, n_new < 1, misalignment,
@@ -273,7 +277,8 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache *segs, int32_t n_segs,
  * The call is one split-K kernel launch per segment, then one merge kernel
  * when the plan has more than one partial.
  * Supported: head_dim 128; g in 1..8; bits 2/4/8 with G 32/64/128, and bits
- * 16 with fp16 q.  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED,
+ * 16 with fp16 q; KVQ_FMT_OAKEN segments with g = 1, 2, 4 or 8 (their own
+ * split-K kernel, the codes' dense part plus the outlier slots).  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED,
  * KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA.
  */
 kvq_status kvq_decode_attention(const kvq_cache *segs, int32_t n_segs,
@@ -294,7 +299,8 @@ kvq_status kvq_decode_attention(const kvq_cache *segs, int32_t n_segs,
  * but for the tokens-on-M formats ((head_dim / G) * g <= 8) the append runs
  * inside the split-K kernel: the unit whose token range covers the new
  * position writes it, and the last unit of each sequence advances
- * seq_lens[b].
+ * seq_lens[b].  Other formats (KVQ_FMT_OAKEN included) run the two calls
+ * as two launches on the stream.
  *   cache: one segment, bits 2, 4 or 8.
  *   k_new, v_new: device fp16 [batch][kv_heads][1][head_dim], 16-byte
  *        aligned.  A sequence already at max_tokens keeps its length and

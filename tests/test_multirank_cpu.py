@@ -46,7 +46,7 @@ def _max_worker(rank, world, port, out):
 def test_max_over_ranks_gloo():
     """Every rank gets the slowest rank's time."""
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.start_processes(_max_worker, args=(world, port, out), nprocs=world, start_method="spawn")
     assert dict(out) == {0: 4.5, 1: 4.5}
 
@@ -84,7 +84,7 @@ def test_ranks_attend_disjoint_sequences_gloo():
     """Weak scaling shards by sequence: the ranks' inputs differ, and each
     rank's output is exactly what one process computes for those sequences."""
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.start_processes(_shard_worker, args=(world, port, out), nprocs=world, start_method="spawn")
     k0, k1 = out["k"]
     assert not np.array_equal(k0, k1)
