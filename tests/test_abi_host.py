@@ -377,3 +377,24 @@ def test_struct_layout_matches_the_header(kvq, tmp_path):
     want = [ctypes.sizeof(kvq.kvq_plane), ctypes.sizeof(kvq.kvq_cache),
             kvq.kvq_plane.oaken.offset, kvq.kvq_cache.v.offset, kvq.kvq_cache.seq_lens.offset]
     assert got == want
+
+
+def test_split_plan_per_workload(kvq):
+    """The host split plan (a wave model over 148 SMs x the format's CTAs
+    per SM, plus the five-CTA build of INT4 G64 g = 4 where its own plan
+    spans more than one wave), read back through the workspace size: the
+    partials per (sequence, query head) at the benchmark's shapes."""
+    def parts(B, H, Hq, max_tokens, hint, bits=4, group=64, fmt=0):
+        c = _fake_cache(kvq, bits=bits, group=group, max_tokens=max_tokens, batch=B, kv_heads=H)
+        c.k.fmt = c.v.fmt = fmt
+        if fmt == kvq.KVQ_FMT_OAKEN:
+            c.k.oaken = c.v.oaken = kvq.kvq_oaken(0.25, 8, 0.5, 5)
+        ws = kvq.kvq_decode_workspace_bytes(c, Hq, hint)
+        r256 = lambda n: (n + 255) // 256 * 256
+        return next(p for p in range(1, 4096)
+                    if 256 + r256(B * 4) + r256(B * Hq * p * 8) + r256(B * Hq * p * 128 * 4) == ws)
+    assert parts(32, 8, 32, 8320, 8292) == 5        # Llama-3 GQA INT4: five-CTA build, 1.7 waves
+    assert parts(16, 8, 32, 8320, 8292) == 9        # half the batch: the four-CTA build, 2 waves
+    assert parts(1, 8, 32, 131392, 131328) == 74    # long context: one wave of the four-CTA build
+    assert parts(16, 32, 32, 4224, 4196, bits=8, group=128) == 4   # Llama-2 MHA: 2048 units
+    assert parts(32, 8, 32, 8320, 8192, group=128, fmt=kvq.KVQ_FMT_OAKEN) == 5
