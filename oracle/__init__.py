@@ -54,6 +54,7 @@ def _load():
         lib.kvqo_f16_to_f32_array.argtypes = [P, i64, P]
         lib.kvqo_quantize_group.argtypes = [P, i32, i32, P, P, P]
         lib.kvqo_quantize_rows.argtypes = [P, i64, i32, i32, i32, P, P]
+        lib.kvqo_quantize_rows_any.argtypes = [P, i32, i64, i32, i32, i32, i32, P, P]
         lib.kvqo_dequantize_rows.argtypes = [P, P, i64, i32, i32, i32, P]
         lib.kvqo_attention.argtypes = [P, i32, P, P, i64, i32, f64, P, P]
         lib.kvqo_attention_blocks.argtypes = [P, i32, P, P, i32, f64, P, i32, P, P]
@@ -145,19 +146,27 @@ def quantize_group(x16, bits: int):
 FMT_CODES = {"int": 0, "fp8": 1, "sym8": 2, "e5m2": 3}
 
 
-def quantize_rows(x16, group: int, bits: int, fmt: str = "int"):
+def quantize_rows(x16, group: int, bits: int, fmt: str = "int", in_dtype: str = "f16"):
     """Token rows [N, D] of fp16 bit patterns -> (codes [N, D*bits/8] uint8,
     meta [N, D/G, 2] uint16 holding the (scale, zero) fp16 patterns).
     fmt "fp8": E4M3 codes (bits 8) with zero point 0 (KV-cache page, FP8);
     fmt "sym8": symmetric INT8, two's complement codes (bits 8) with zero
     point 0 (KV-cache page, INT8 item); fmt "e5m2": E5M2 codes (bits 8) with
-    zero point 0 (KV-cache page, FP8)."""
+    zero point 0 (KV-cache page, FP8).  in_dtype "bf16": the rows are
+    bfloat16 bit patterns, read exactly into fp32 like the fp16 ones (the
+    same arithmetic follows)."""
     lib = _load()
     x16 = _c(x16, np.uint16)
     N, D = x16.shape
     codes = np.zeros((N, D * bits // 8), np.uint8)
     ng = D // group if bits != 16 else 1
     meta = np.zeros((N, ng, 2), np.uint16)
+    if in_dtype == "bf16":
+        assert bits != 16, "raw rows hold fp16 values"
+        lib.kvqo_quantize_rows_any(_p(x16), 1, N, D, group, bits, FMT_CODES[fmt], _p(codes),
+                                   _p(meta))
+        return codes, meta
+    assert in_dtype == "f16", in_dtype
     if fmt == "fp8":
         assert bits == 8
         lib.kvqo_quantize_rows_fp8(_p(x16), N, D, group, _p(codes), _p(meta))
@@ -450,12 +459,13 @@ def kv_elements(layers: int, kv_heads: int, head_dim: int, seq_len: int, batch: 
 # Whole-cache helpers built from the functions above
 # --------------------------------------------------------------------------
 
-def quantize_cache(x16, group: int, bits: int, fmt: str = "int"):
-    """x16 [..., T, D] fp16 patterns -> codes [..., T, D*bits/8], meta [..., T, D/G, 2]."""
+def quantize_cache(x16, group: int, bits: int, fmt: str = "int", in_dtype: str = "f16"):
+    """x16 [..., T, D] fp16 (or, with in_dtype "bf16", bfloat16) patterns ->
+    codes [..., T, D*bits/8], meta [..., T, D/G, 2]."""
     x16 = _c(x16, np.uint16)
     lead = x16.shape[:-1]
     D = x16.shape[-1]
-    codes, meta = quantize_rows(x16.reshape(-1, D), group, bits, fmt)
+    codes, meta = quantize_rows(x16.reshape(-1, D), group, bits, fmt, in_dtype)
     return (codes.reshape(*lead, D * bits // 8),
             meta.reshape(*lead, meta.shape[-2], 2))
 

@@ -219,20 +219,28 @@ float kvqo_bf16_to_f32(uint16_t h)
 /* Group-wise asymmetric quantization ([P4] 3.2.2, [P1] 2.1, [P2], [P5] 2.3) */
 /* ------------------------------------------------------------------------ */
 
+/* Value of the j-th input element: binary16 or bfloat16 bit patterns, both
+ * read exactly into fp32. */
+static float kvqo_in(const uint16_t *x, int j, int in_bf16)
+{
+    return in_bf16 ? kvqo_bf16_to_f32(x[j]) : kvqo_f16_to_f32(x[j]);
+}
+
 /*
- * Quantize one group x[0..G-1] (binary16 bit patterns) to `bits`-bit codes.
- * Writes the G unpacked codes, and the fp16 bit patterns of s and z.
+ * Quantize one group x[0..G-1] (binary16 bit patterns, or bfloat16 with
+ * in_bf16) to `bits`-bit codes.  Writes the G unpacked codes, and the fp16
+ * bit patterns of s and z.
  */
-void kvqo_quantize_group(const uint16_t *x, int G, int bits,
-                         uint8_t *code, uint16_t *s_out, uint16_t *z_out)
+static void kvqo_quantize_group_in(const uint16_t *x, int in_bf16, int G, int bits,
+                                   uint8_t *code, uint16_t *s_out, uint16_t *z_out)
 {
     const float qmax = (float)((1 << bits) - 1);
 
-    /* min and max of the group, in fp32 (exact for fp16 inputs) */
-    float mn = kvqo_f16_to_f32(x[0]);
+    /* min and max of the group, in fp32 (exact for fp16 and bf16 inputs) */
+    float mn = kvqo_in(x, 0, in_bf16);
     float mx = mn;
     for (int j = 1; j < G; ++j) {
-        float v = kvqo_f16_to_f32(x[j]);
+        float v = kvqo_in(x, j, in_bf16);
         if (v < mn)
             mn = v;
         if (v > mx)
@@ -257,7 +265,7 @@ void kvqo_quantize_group(const uint16_t *x, int G, int bits,
 
     /* quant(x) = round(x / s) + z, clamped to the code range (R5) */
     for (int j = 0; j < G; ++j) {
-        float c = rintf(kvqo_f16_to_f32(x[j]) / s) + z;
+        float c = rintf(kvqo_in(x, j, in_bf16) / s) + z;
         if (c < 0.0f)
             c = 0.0f;
         if (c > qmax)
@@ -268,14 +276,20 @@ void kvqo_quantize_group(const uint16_t *x, int G, int bits,
     *z_out = z16;
 }
 
+void kvqo_quantize_group(const uint16_t *x, int G, int bits,
+                         uint8_t *code, uint16_t *s_out, uint16_t *z_out)
+{
+    kvqo_quantize_group_in(x, 0, G, bits, code, s_out, z_out);
+}
+
 /*
  * Quantize n_rows token rows of D fp16 values, groups of G along the row
  * (R6).  codes: [n_rows][D*bits/8] packed (R7); meta: [n_rows][D/G][2]
  * binary16 (scale, zero).  bits == 16 stores the fp16 row unchanged and
  * writes no meta (the FP16 class of [P4] 3.1.1).
  */
-void kvqo_quantize_rows(const uint16_t *x, int64_t n_rows, int D, int G,
-                        int bits, uint8_t *codes, uint16_t *meta)
+static void kvqo_quantize_rows_in(const uint16_t *x, int in_bf16, int64_t n_rows, int D,
+                                  int G, int bits, uint8_t *codes, uint16_t *meta)
 {
     const int64_t row_bytes = (int64_t)D * bits / 8;
     uint8_t *tmp = (uint8_t *)malloc((size_t)G);
@@ -289,7 +303,7 @@ void kvqo_quantize_rows(const uint16_t *x, int64_t n_rows, int D, int G,
         memset(cr, 0, (size_t)row_bytes);
         for (int g = 0; g < D / G; ++g) {
             uint16_t s16, z16;
-            kvqo_quantize_group(xr + g * G, G, bits, tmp, &s16, &z16);
+            kvqo_quantize_group_in(xr + g * G, in_bf16, G, bits, tmp, &s16, &z16);
             meta[(r * (D / G) + g) * 2 + 0] = s16;
             meta[(r * (D / G) + g) * 2 + 1] = z16;
             for (int j = 0; j < G; ++j) {
@@ -300,6 +314,12 @@ void kvqo_quantize_rows(const uint16_t *x, int64_t n_rows, int D, int G,
         }
     }
     free(tmp);
+}
+
+void kvqo_quantize_rows(const uint16_t *x, int64_t n_rows, int D, int G,
+                        int bits, uint8_t *codes, uint16_t *meta)
+{
+    kvqo_quantize_rows_in(x, 0, n_rows, D, G, bits, codes, meta);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -351,11 +371,12 @@ uint8_t kvqo_f32_to_e4m3(float x)
 }
 
 /* One group of G binary16 values to E4M3 codes with scale s (R14). */
-void kvqo_quantize_group_fp8(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
+static void kvqo_quantize_group_fp8_in(const uint16_t *x, int in_bf16, int G, uint8_t *code,
+                                       uint16_t *s_out)
 {
     float amax = 0.0f;
     for (int j = 0; j < G; ++j) {
-        float v = fabsf(kvqo_f16_to_f32(x[j]));
+        float v = fabsf(kvqo_in(x, j, in_bf16));
         if (v > amax)
             amax = v;
     }
@@ -365,8 +386,13 @@ void kvqo_quantize_group_fp8(const uint16_t *x, int G, uint8_t *code, uint16_t *
     uint16_t s16 = kvqo_f32_to_f16_up(s32);
     float s = kvqo_f16_to_f32(s16);
     for (int j = 0; j < G; ++j)
-        code[j] = kvqo_f32_to_e4m3(kvqo_f16_to_f32(x[j]) / s);
+        code[j] = kvqo_f32_to_e4m3(kvqo_in(x, j, in_bf16) / s);
     *s_out = s16;
+}
+
+void kvqo_quantize_group_fp8(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
+{
+    kvqo_quantize_group_fp8_in(x, 0, G, code, s_out);
 }
 
 /* Token rows to E4M3 codes (one byte per element) and (s, 0) fp16 pairs per
@@ -430,11 +456,12 @@ uint8_t kvqo_f32_to_e5m2(float x)
 }
 
 /* One group of G binary16 values to E5M2 codes with scale s (R17). */
-void kvqo_quantize_group_e5m2(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
+static void kvqo_quantize_group_e5m2_in(const uint16_t *x, int in_bf16, int G, uint8_t *code,
+                                       uint16_t *s_out)
 {
     float amax = 0.0f;
     for (int j = 0; j < G; ++j) {
-        float v = fabsf(kvqo_f16_to_f32(x[j]));
+        float v = fabsf(kvqo_in(x, j, in_bf16));
         if (v > amax)
             amax = v;
     }
@@ -444,8 +471,13 @@ void kvqo_quantize_group_e5m2(const uint16_t *x, int G, uint8_t *code, uint16_t 
     uint16_t s16 = kvqo_f32_to_f16_up(s32);
     float s = kvqo_f16_to_f32(s16);
     for (int j = 0; j < G; ++j)
-        code[j] = kvqo_f32_to_e5m2(kvqo_f16_to_f32(x[j]) / s);
+        code[j] = kvqo_f32_to_e5m2(kvqo_in(x, j, in_bf16) / s);
     *s_out = s16;
+}
+
+void kvqo_quantize_group_e5m2(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
+{
+    kvqo_quantize_group_e5m2_in(x, 0, G, code, s_out);
 }
 
 /* Token rows to E5M2 codes and (s, 0) fp16 pairs per group of G. */
@@ -463,11 +495,12 @@ void kvqo_quantize_rows_e5m2(const uint16_t *x, int64_t n_rows, int D, int G, ui
 
 /* Symmetric INT8 ([P2'] item 2; R15): one group of G binary16 values to
  * two's complement codes with scale s. */
-void kvqo_quantize_group_sym8(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
+static void kvqo_quantize_group_sym8_in(const uint16_t *x, int in_bf16, int G, uint8_t *code,
+                                        uint16_t *s_out)
 {
     float amax = 0.0f;
     for (int j = 0; j < G; ++j) {
-        float v = fabsf(kvqo_f16_to_f32(x[j]));
+        float v = fabsf(kvqo_in(x, j, in_bf16));
         if (v > amax)
             amax = v;
     }
@@ -477,7 +510,7 @@ void kvqo_quantize_group_sym8(const uint16_t *x, int G, uint8_t *code, uint16_t 
     uint16_t s16 = kvqo_f32_to_f16_up(s32);
     float s = kvqo_f16_to_f32(s16);
     for (int j = 0; j < G; ++j) {
-        float c = rintf(kvqo_f16_to_f32(x[j]) / s);
+        float c = rintf(kvqo_in(x, j, in_bf16) / s);
         if (c < -128.0f)
             c = -128.0f;
         if (c > 127.0f)
@@ -485,6 +518,11 @@ void kvqo_quantize_group_sym8(const uint16_t *x, int G, uint8_t *code, uint16_t 
         code[j] = (uint8_t)(int8_t)c;
     }
     *s_out = s16;
+}
+
+void kvqo_quantize_group_sym8(const uint16_t *x, int G, uint8_t *code, uint16_t *s_out)
+{
+    kvqo_quantize_group_sym8_in(x, 0, G, code, s_out);
 }
 
 /* Token rows to symmetric INT8 codes (one byte per element) and (s, 0) fp16
@@ -496,6 +534,37 @@ void kvqo_quantize_rows_sym8(const uint16_t *x, int64_t n_rows, int D, int G, ui
         for (int g = 0; g < D / G; ++g) {
             uint16_t s16;
             kvqo_quantize_group_sym8(x + r * D + g * G, G, codes + r * D + g * G, &s16);
+            meta[(r * (D / G) + g) * 2 + 0] = s16;
+            meta[(r * (D / G) + g) * 2 + 1] = 0; /* zero point 0 */
+        }
+}
+
+/*
+ * Token rows of D values (binary16 bit patterns, or bfloat16 with in_bf16:
+ * the KV-cache page's caches hold either; both read exactly into fp32), one
+ * group of G along the row, in any of the token-grouped formats: fmt 0
+ * asymmetric integer codes of `bits` bits, 1 FP8 E4M3, 2 symmetric INT8,
+ * 3 FP8 E5M2 (bits 8).  codes: [n_rows][D*bits/8]; meta: [n_rows][D/G][2].
+ * Every format runs the arithmetic above on the fp32 values unchanged.
+ */
+void kvqo_quantize_rows_any(const uint16_t *x, int in_bf16, int64_t n_rows, int D, int G,
+                            int bits, int fmt, uint8_t *codes, uint16_t *meta)
+{
+    if (fmt == 0) {
+        kvqo_quantize_rows_in(x, in_bf16, n_rows, D, G, bits, codes, meta);
+        return;
+    }
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int g = 0; g < D / G; ++g) {
+            uint16_t s16;
+            const uint16_t *xg = x + r * D + g * G;
+            uint8_t *cg = codes + r * D + g * G;
+            if (fmt == 1)
+                kvqo_quantize_group_fp8_in(xg, in_bf16, G, cg, &s16);
+            else if (fmt == 2)
+                kvqo_quantize_group_sym8_in(xg, in_bf16, G, cg, &s16);
+            else
+                kvqo_quantize_group_e5m2_in(xg, in_bf16, G, cg, &s16);
             meta[(r * (D / G) + g) * 2 + 0] = s16;
             meta[(r * (D / G) + g) * 2 + 1] = 0; /* zero point 0 */
         }

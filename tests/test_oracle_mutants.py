@@ -22,8 +22,10 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 # (name, original text, mutated text)
 MUTANTS = [
-    ("round half away from zero", "float c = rintf(kvqo_f16_to_f32(x[j]) / s) + z;",
-     "float c = roundf(kvqo_f16_to_f32(x[j]) / s) + z;"),
+    ("bf16 read as fp16", "return in_bf16 ? kvqo_bf16_to_f32(x[j]) : kvqo_f16_to_f32(x[j]);",
+     "return kvqo_f16_to_f32(x[j]);"),
+    ("round half away from zero", "float c = rintf(kvqo_in(x, j, in_bf16) / s) + z;",
+     "float c = roundf(kvqo_in(x, j, in_bf16) / s) + z;"),
     ("scale rounded to nearest", "uint16_t s16 = kvqo_f32_to_f16_up(s32);",
      "uint16_t s16 = kvqo_f32_to_f16(s32);"),
     ("zero point clamped to code range", "    uint16_t z16 = kvqo_f32_to_f16(zf);",
@@ -53,8 +55,8 @@ MUTANTS = [
     ("e4m3 exponent bias 8", "v = ldexp((double)(8 + m), e - 10);",
      "v = ldexp((double)(8 + m), e - 11);"),
     ("fp8 scale from another maximum", "float s32 = amax / 448.0f;", "float s32 = amax / 464.0f;"),
-    ("sym8 ties away from zero", "float c = rintf(kvqo_f16_to_f32(x[j]) / s);",
-     "float c = roundf(kvqo_f16_to_f32(x[j]) / s);"),
+    ("sym8 ties away from zero", "float c = rintf(kvqo_in(x, j, in_bf16) / s);",
+     "float c = roundf(kvqo_in(x, j, in_bf16) / s);"),
     ("sym8 scale over 128 levels", "float s32 = amax / 127.0f;", "float s32 = amax / 128.0f;"),
     ("sym8 offset-binary codes", "code[j] = (uint8_t)(int8_t)c;",
      "code[j] = (uint8_t)(int)(c + 128.0f);"),
@@ -210,6 +212,13 @@ def _pins(o):
     m5 = np.clip((f5[:-1] + f5[1:]) / 2, -57344, 57344).astype(np.float32)
     yield "e5m2 encode vs torch", bool(np.array_equal(
         o.f32_to_e5m2(m5), torch.from_numpy(m5).to(torch.float8_e5m2).view(torch.uint8).numpy()))
+
+    b = _golden("bf16_worked_example.json")
+    pat = np.array([int(h, 16) for h in b["bf16_patterns"]], np.uint16)[None]
+    cb, mb = o.quantize_rows(pat, b["group"], b["bits"], in_dtype="bf16")
+    ub = [(int(cb[0, j // 2]) >> (4 * (j % 2))) & 15 for j in range(b["group"])]
+    yield "bf16 worked group", (ub == b["codes"] and int(mb[0, 0, 0]) == int(b["scale_f16"], 16)
+                                and int(mb[0, 0, 1]) == int(b["zero_f16"], 16))
 
     ok = True
     for r in _golden("oaken_worked_example.json")["rows"]:
