@@ -1,13 +1,13 @@
 #!/usr/bin/env python
 """Decode-step benchmark of the quantized KV cache on B200.
 
-One step = quantize-on-write of one new token per sequence
-(kvq_quantize_append) + decode attention of one query per sequence over the
-whole packed cache (kvq_decode_partials + kvq_decode_merge, i.e.
-kvq_decode_attention).  Default workload: the Llama-2-7B-shaped MHA layer
-(batch 16, 32 heads, head_dim 128, context 4096, INT8 group 128, bf16
+One step = quantize-on-write of one new token per sequence + decode
+attention of one query per sequence over the whole packed cache
+(kvq_decode_step: the split-K kernel with the append inside it, then the
+log-sum-exp merge kernel).  Default workload: the Llama-3-8B-shaped GQA layer (batch 32,
+32 query / 8 KV heads, head_dim 128, context 8192, INT4 group 64, fp16
 queries); the cache length runs through the workload's 100-step episode
-(4097 .. 4196 tokens) and restarts, so any --steps keeps the same shape.
+(8193 .. 8292 tokens) and restarts, so any --steps keeps the same shape.
 
 Prints one JSON line (rank 0): tokens/s over all ranks (device-timed, max
 over ranks), the roofline of the split-K attention kernel against the
@@ -47,10 +47,10 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--steps", type=int, default=15000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
-    p.add_argument("--workload", default="llama2_7b_mha_int8")
+    p.add_argument("--workload", default="llama3_8b_gqa_int4")
     p.add_argument("--batch", type=int, default=0,
                    help="override the workload's batch (smaller cases for profiling)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -215,8 +215,9 @@ def segment_oracle_pairs(wl, k, v, q, pairs):
 
 
 def run_reference(args, wl):
-    """The CPU oracle as it stands, on this host's cores: each step attends
-    one (sequence, KV head) of the workload after appending one token."""
+    """The CPU oracle as it stands, on this host's cores (one thread per
+    core): each step attends one (sequence, KV head) of the workload after
+    appending one token."""
     import numpy as np
     import torch
 
@@ -233,10 +234,7 @@ def run_reference(args, wl):
             oracle.decode_attention(qh, False, segs, lens, 128 ** -0.5)
         for i in range(args.warmup):
             mixed_step(i)
-        t0 = time.perf_counter()
-        for i in range(args.steps):
-            mixed_step(i)
-        el = time.perf_counter() - t0
+        el = run_steps_parallel(mixed_step, args.steps)
         value = args.steps / wl.kv_heads / el
         sample = (f"each step: one (sequence, KV head) of {wl.name}: attention over its "
                   f"{wl.n_chunks} chunks as FP16/INT4/INT2 segments ({int(counts[0])}/"
@@ -256,10 +254,7 @@ def run_reference(args, wl):
             oracle.decode_attention(qh, wl.q_dtype == "bf16", [seg], lens, 128 ** -0.5)
         for i in range(args.warmup):
             kpc_step(i)
-        t0 = time.perf_counter()
-        for i in range(args.steps):
-            kpc_step(i)
-        el = time.perf_counter() - t0
+        el = run_steps_parallel(kpc_step, args.steps)
         value = args.steps / wl.kv_heads / el
         how = "Oaken codec" if wl.fmt == "oaken" else "K per channel"
         sample = (f"each step: one (sequence, KV head) of {wl.name}: attention of "
@@ -295,10 +290,7 @@ def run_reference(args, wl):
 
     for i in range(args.warmup):
         step(i)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        step(i)
-    el = time.perf_counter() - t0
+    el = run_steps_parallel(step, args.steps)
     value = args.steps / wl.kv_heads / el
     sample = (f"each step: one (sequence, KV head) of {wl.name} at {L + 1} tokens "
               f"(append 1 token + attention of {g} query heads); tokens/s = steps / kv_heads "
@@ -306,7 +298,25 @@ def run_reference(args, wl):
     print(json.dumps(reference_line(args, wl, value, el, sample)), flush=True)
 
 
+def run_steps_parallel(step, steps: int) -> float:
+    """Run step(0) .. step(steps - 1) on one host thread per core (thread i
+    takes steps i, i + n, ...; the oracle's C calls release the interpreter
+    lock); returns the elapsed seconds."""
+    import threading
+    n = max(1, min(os.cpu_count() or 1, steps))
+    t0 = time.perf_counter()
+    ts = [threading.Thread(target=lambda i=i: [step(j) for j in range(i, steps, n)])
+          for i in range(n)]
+    for th in ts:
+        th.start()
+    for th in ts:
+        th.join()
+    return time.perf_counter() - t0
+
+
 def reference_line(args, wl, value, el, sample):
+    threads = max(1, min(os.cpu_count() or 1, args.steps))
+    sample = f"{sample}; steps spread over {threads} host threads (one per core)"
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -314,8 +324,9 @@ def reference_line(args, wl, value, el, sample):
         "vs_baseline": None, "dtype": FMT_DTYPE.get(wl.fmt, DTYPE[wl.bits]),
         "data": "synthetic",
         "config": workload_config(wl),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(os.cpu_count() or 1,
+                                                                           args.steps),
+                         "nproc": os.cpu_count(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -335,9 +346,52 @@ def workload_config(wl, extra=None):
 
 # ---------------------------------------------------------------- CPU baseline
 
+def time_oracle_jobs(jobs, seconds: float, threads: int):
+    """Run the oracle jobs round-robin on `threads` host threads for about
+    `seconds` (each thread at least one job); returns (jobs done, seconds).
+    The oracle is C called through ctypes, which releases the interpreter
+    lock for the call, so the threads run on separate cores."""
+    import threading
+    done = [0] * threads
+    t0 = time.perf_counter()
+
+    def worker(i):
+        n = 0
+        while True:
+            jobs[(i + n * threads) % len(jobs)]()
+            n += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+        done[i] = n
+    ts = [threading.Thread(target=worker, args=(i,)) for i in range(threads)]
+    for th in ts:
+        th.start()
+    for th in ts:
+        th.join()
+    return sum(done), time.perf_counter() - t0
+
+
+def oracle_baseline(wl, jobs, seconds: float, what: str):
+    """The oracle as it stands on a bounded sample: one host thread, then
+    every host core (one thread per core).  tokens/s = (sequence, KV head)
+    jobs / kv_heads / seconds (a job is one sequence's work for one KV head)."""
+    nproc = os.cpu_count() or 1
+    n1, el1 = time_oracle_jobs(jobs, seconds, 1)
+    nn, eln = time_oracle_jobs(jobs, seconds, nproc)
+    single = {"value": n1 / wl.kv_heads / el1, "unit": "tokens/s", "cores": 1,
+              "sample": f"{n1} {what} cycling over {len(jobs)} (sequence, KV head) pairs, "
+                        f"{el1:.1f} s on one host thread"}
+    return {"value": nn / wl.kv_heads / eln, "unit": "tokens/s", "cores": nproc,
+            "nproc": nproc, "kind": "oracle",
+            "sample": f"{nn} {what} cycling over {len(jobs)} (sequence, KV head) pairs, "
+                      f"{eln:.1f} s on {nproc} host threads (one per core, nproc = {nproc}); "
+                      f"tokens/s = jobs / kv_heads / seconds",
+            "single_thread": single}
+
+
 def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
-    """The oracle (single-threaded C, fp64 attention) on a bounded sample of
-    the same inputs: (sequence, KV head) pairs, each one append + attention."""
+    """The oracle (C, fp64 attention) on a bounded sample of the same inputs:
+    (sequence, KV head) pairs, each one append + attention."""
     import numpy as np
     import torch
 
@@ -346,22 +400,16 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
     pairs = [(b, h) for b in range(min(wl.batch, 2)) for h in range(min(wl.kv_heads, 4))]
     if wl.k_axis == "channel" or wl.fmt == "oaken":
         prep = segment_oracle_pairs(wl, k, v, q, pairs)
-        n = 0
-        t0 = time.perf_counter()
-        while True:
-            qh, seg, lens = prep[n % len(prep)]
-            oracle.decode_attention(qh, wl.q_dtype == "bf16", [seg], lens, 128 ** -0.5)
-            n += 1
-            el = time.perf_counter() - t0
-            if el >= seconds and n >= 2:
-                break
-        return {"value": n / wl.kv_heads / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                "sample": f"{n} (sequence, KV head) attentions of {wl.name} over "
-                          f"{k.shape[2]} tokens ("
-                          f"{'Oaken codec' if wl.fmt == 'oaken' else 'K per channel'}) "
-                          f"cycling over {len(prep)} pairs, "
-                          f"{el:.1f} s on one host thread; tokens/s = pairs / kv_heads / seconds"}
-    prepared = []
+
+        def job_of(qh, seg, lens):
+            return lambda: oracle.decode_attention(qh, wl.q_dtype == "bf16", [seg], lens,
+                                                   128 ** -0.5)
+        jobs = [job_of(*p) for p in prep]
+        how = "Oaken codec" if wl.fmt == "oaken" else "K per channel"
+        return oracle_baseline(wl, jobs, seconds,
+                               f"attentions of {wl.name} over {k.shape[2]} tokens ({how})")
+    L = k.shape[2]
+    jobs = []
     for b, h in pairs:
         kk = k[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
         vv = v[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
@@ -370,26 +418,17 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
         qh = q[b, h * g:(h + 1) * g].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
         knew = kn[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
         vnew = vn[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-        prepared.append((kc, km, vc, vm, qh, knew, vnew))
-    L = k.shape[2]
-    n = 0
-    t0 = time.perf_counter()
-    while True:
-        kc, km, vc, vm, qh, knew, vnew = prepared[n % len(prepared)]
-        ck, mk = oracle.quantize_rows(knew, wl.group, wl.bits, wl.fmt)
-        cv, mv = oracle.quantize_rows(vnew, wl.group, wl.bits, wl.fmt)
-        oracle.attention_packed(qh, wl.q_dtype == "bf16", np.concatenate([kc, ck]),
-                                np.concatenate([km, mk]), wl.bits, np.concatenate([vc, cv]),
-                                np.concatenate([vm, mv]), wl.bits, wl.group, L + 1,
-                                128 ** -0.5, fmt=wl.fmt)
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds and n >= 2:
-            break
-    return {"value": n / wl.kv_heads / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} (sequence, KV head) decode steps of {wl.name} at {L + 1} tokens "
-                      f"cycling over {len(prepared)} pairs, {el:.1f} s on one host thread; "
-                      f"tokens/s = pairs / kv_heads / seconds"}
+
+        def job(kc=kc, km=km, vc=vc, vm=vm, qh=qh, knew=knew, vnew=vnew):
+            ck, mk = oracle.quantize_rows(knew, wl.group, wl.bits, wl.fmt)
+            cv, mv = oracle.quantize_rows(vnew, wl.group, wl.bits, wl.fmt)
+            oracle.attention_packed(qh, wl.q_dtype == "bf16", np.concatenate([kc, ck]),
+                                    np.concatenate([km, mk]), wl.bits,
+                                    np.concatenate([vc, cv]), np.concatenate([vm, mv]),
+                                    wl.bits, wl.group, L + 1, 128 ** -0.5, fmt=wl.fmt)
+        jobs.append(job)
+    return oracle_baseline(wl, jobs, seconds,
+                           f"decode steps (append + attention) of {wl.name} at {L + 1} tokens")
 
 
 def prepare_mixed_oracle(wl, k, v, q, wlr):
@@ -437,20 +476,14 @@ def cpu_baseline_mixed(wl, k, v, q, seconds: float, wlr):
     (sequence, KV head) pairs of the chunk-level mixed workload."""
     import oracle
     prepared, counts = prepare_mixed_oracle(wl, k, v, q, wlr)
-    n = 0
-    t0 = time.perf_counter()
-    while True:
-        qh, segs, lens = prepared[n % len(prepared)]
-        oracle.decode_attention(qh, False, segs, lens, 128 ** -0.5)
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds and n >= 2:
-            break
-    return {"value": n / wl.kv_heads / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} (sequence, KV head) attention steps of {wl.name} over its "
-                      f"{int(sum(counts))} chunks ({int(counts[0])} FP16, {int(counts[1])} INT4, "
-                      f"{int(counts[2])} INT2) cycling over {len(prepared)} heads, {el:.1f} s on "
-                      f"one host thread; tokens/s = pairs / kv_heads / seconds"}
+
+    def job_of(qh, segs, lens):
+        return lambda: oracle.decode_attention(qh, False, segs, lens, 128 ** -0.5)
+    jobs = [job_of(*p) for p in prepared]
+    return oracle_baseline(wl, jobs, seconds,
+                           f"attention steps of {wl.name} over its {int(sum(counts))} chunks "
+                           f"({int(counts[0])} FP16, {int(counts[1])} INT4, {int(counts[2])} "
+                           f"INT2)")
 
 
 # ---------------------------------------------------------------- kvq arm
@@ -825,6 +858,12 @@ def run_kvq(args, wl, rank, world, local_rank):
                 "path": "kvq_decode_step (append workloads) or kvq_decode_attention through the "
                         "Python binding; pinned host buffers, one input and one result copy per "
                         "step, double-buffered on two copy streams"},
+        # device latency of one step and of its kernel(s), and of the prefill
+        # quantize of the whole context (for the 256-token tiny workload, the
+        # latency-bound case, these are the figures that matter)
+        "latency_us": {"step": ms / args.steps * 1e3,
+                       "decode_kernels": split_total_us / len(last_step),
+                       **({"prefill_quantize": prefill["us"]} if prefill else {})},
         "gpu_launches": launches_per_step * args.steps,
         **({"prefill_quantize": {**prefill, "frac": prefill["gbs"] / peak}} if prefill else {}),
         **({"chunk_reorder": {**chunk_timing, "frac": chunk_timing["reorder_gbs"] / peak}}

@@ -215,9 +215,21 @@ uint64_t kvq_kv_elements(uint64_t layers, uint64_t kv_heads, uint64_t head_dim,
  * seq_lens[b] .. seq_lens[b] + n_new - 1 of each sequence's K and V planes
  * (quantize-on-write: Cocktail page 3.2.2 formula; Oaken's write pipeline,
  * jsqmd.com news 825302 section 3.2.3, quantizes inside the memory write).
- *   k_new, v_new: device fp16 [batch][kv_heads][n_new][head_dim], 16-byte
- *                 aligned.  n_new = 1 is the decode-step append; n_new = the
- *                 prompt length is the bulk prefill (with seq_lens = 0).
+ *   k_new, v_new: device [batch][kv_heads][n_new][head_dim] of kv_dtype
+ *                 values, 16-byte aligned.  n_new = 1 is the decode-step
+ *                 append; n_new = the prompt length is the bulk prefill
+ *                 (with seq_lens = 0).
+ *   kv_dtype:     KVQ_F16 or KVQ_BF16.  Values of either type are widened to
+ *                 fp32 exactly and go through the same fp32 steps, so a bf16
+ *                 row holding fp16-representable values gives the codes of
+ *                 its fp16 form.  bf16 input is taken by the token-grouped
+ *                 formats (asymmetric integer, FP8 E4M3/E5M2, symmetric
+ *                 INT8); a per-channel K plane or an Oaken plane with bf16
+ *                 input returns KVQ_ERR_UNSUPPORTED.  bf16 values reach
+ *                 beyond fp16: a group is encodable when its scale fits fp16
+ *                 ((max - min) / (2^bits - 1), or |max| / 448, / 57344,
+ *                 / 127, at most 65504) and its values are below 2^64 in
+ *                 magnitude; the codes of other groups are unspecified.
  *   advance_seq_lens: nonzero adds n_new to seq_lens[b] after the write
  *                 (capped at max_tokens), in stream order.
  * Tokens whose position would reach max_tokens are not written (the
@@ -228,12 +240,13 @@ uint64_t kvq_kv_elements(uint64_t layers, uint64_t kv_heads, uint64_t head_dim,
  * n_new must be a multiple of KVQ_CHANNEL_BLOCK, and so must seq_lens[b]
  * on the device: a sequence whose length is not is neither written nor
  * advanced.  Errors: KVQ_ERR_INVALID_ARG (nulls, n_new < 1, misalignment,
- * n_new off a block boundary), KVQ_ERR_CAPACITY (n_new > max_tokens),
- * KVQ_ERR_UNSUPPORTED, KVQ_ERR_CUDA.
+ * n_new off a block boundary, an unknown kv_dtype), KVQ_ERR_CAPACITY (n_new >
+ * max_tokens), KVQ_ERR_UNSUPPORTED, KVQ_ERR_CUDA.
  */
 kvq_status kvq_quantize_append(const kvq_cache *cache, const void *k_new,
-                               const void *v_new, int32_t n_new,
-                               int32_t advance_seq_lens, void *stream);
+                               const void *v_new, kvq_dtype kv_dtype,
+                               int32_t n_new, int32_t advance_seq_lens,
+                               void *stream);
 
 /*
  * Workspace bytes that kvq_decode_attention (and kvq_decode_step) need for
@@ -261,8 +274,18 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache *segs, int32_t n_segs,
  *   segs: 1 segment, or several segments of one mixed-precision cache (same
  *         batch, kv_heads, head_dim; each its own bits, planes, seq_lens).
  *   q: device [batch][q_heads][head_dim] fp16 or bf16 (q_dtype), 16-byte
- *      aligned; bf16 values are used as fp16 (exact for magnitudes in
- *      [2^-14, 65504]).
+ *      aligned.  The kernels feed q to fp16 tensor-core operands, lifted by
+ *      a power of two that depends on the code format (up to 2^6 for 2-bit
+ *      codes); a query row whose largest element would leave the fp16 range
+ *      that way is staged scaled down by a power of two and its scores are
+ *      scaled back, so every finite query gives finite scores.  bf16
+ *      elements are rounded to fp16 after that scaling (exact where the
+ *      scaled magnitude is at least 2^-14).  A score is formed per group as
+ *      s * (sum q c - z * sum q), the code sum accumulated by the tensor
+ *      cores in fp32, so its absolute error grows with s * |z| * max |q_j|
+ *      rather than with the score itself: with 2-bit codes, query elements
+ *      beyond about 1000 in magnitude can take the attention outside a
+ *      1e-3 relative error.
  *   out: device fp32 [batch][q_heads][head_dim]; lse: device fp32
  *        [batch][q_heads] natural log, or NULL.
  *   max_len_hint: an upper bound of the seq_lens used to pick the split
@@ -294,7 +317,7 @@ kvq_status kvq_decode_attention(const kvq_cache *segs, int32_t n_segs,
  * in the write path to memory (section 3.2.3), with the quantize formula of
  * the Cocktail page, 3.2.2, exactly as kvq_quantize_append computes it --
  * then kvq_decode_attention over the cache including that token.  It is the
- * same as kvq_quantize_append(cache, k_new, v_new, 1, advance = 1) followed
+ * same as kvq_quantize_append(cache, k_new, v_new, KVQ_F16, 1, advance = 1) followed
  * by kvq_decode_attention, with the same results bit for bit in the cache,
  * but for the tokens-on-M formats ((head_dim / G) * g <= 8) the append runs
  * inside the split-K kernel: the unit whose token range covers the new
@@ -374,9 +397,12 @@ kvq_status kvq_decode_merge(const kvq_cache *segs, int32_t n_segs,
  *    more scratch than KVQ_STATIC_SCRATCH_BYTES (kvq_decode_workspace_bytes
  *    with the same arguments tells how much it needs).
  *  - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library
- *    call.  The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current and caches it; make
- *    that first call before any stream capture.
+ *    call.  Every call looks up the array's device address
+ *    (cudaGetSymbolAddress) with the caller's device current; the first
+ *    call on a device is the one that loads the library's module there, so
+ *    make that first call before any stream capture.
+ *  - Arguments are all checked before the array is touched: a non-OK
+ *    status means nothing was enqueued.
  *  - Every call shares the one array, which keeps the last call's contents
  *    (the error word is cleared at the start of each call).  Calls whose
  *    work overlaps on the GPU -- on different streams, or from different

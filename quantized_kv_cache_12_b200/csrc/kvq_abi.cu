@@ -5,7 +5,10 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
+
+#include <atomic>
 
 #include "kvq.h"
 #include "kvq_internal.h"
@@ -91,28 +94,14 @@ kvq_status check_cache(const kvq_cache* c, bool allow16) {
 }
 
 // Split count of one segment.  A (sequence, KV head, split) is one unit of
-// work; the decode kernel runs one wave of persistent CTAs (S = 148 x the
-// format's CTAs per SM) that take units from a counter.  With equal units
-// the kernel takes ceil(units / S) unit-times, so the count minimises
-// ceil(units / S) x (tokens per unit + a fixed per-unit cost), tokens per
-// unit being rounded up to the 32-token stage, with at least 128 tokens per
-// unit.  The fixed cost -- the start of a unit waits for its query rows and
-// first copies -- was measured at about 200 tokens' worth of work.  The
-// result depends only on (sequences x KV heads, length, S), so the last few
-// are cached per thread.
-int choose_splits(const kvq_cache& c, int max_len_hint, int ctas_per_sm) {
-  const long long pairs = (long long)c.batch * c.kv_heads;
-  long long len = c.max_tokens;
-  if (max_len_hint > 0 && max_len_hint < len) len = max_len_hint;
-  if (len <= 0 || pairs <= 0) return 1;
-  constexpr int kCache = 4;
-  thread_local long long cached_pairs[kCache] = {-1, -1, -1, -1}, cached_len[kCache],
-                                               cached_slots[kCache];
-  thread_local int cached_n[kCache], cache_next = 0;
-  const long long kSlots = 148LL * (ctas_per_sm > 0 ? ctas_per_sm : 3);
-  for (int e = 0; e < kCache; ++e)
-    if (pairs == cached_pairs[e] && len == cached_len[e] && kSlots == cached_slots[e])
-      return cached_n[e];
+// work; the decode kernels run one wave of persistent CTAs (S = SMs x the format's CTAs per SM) that take units from
+// a counter.  With equal units the kernel takes ceil(units / S) unit-times,
+// so the count minimises ceil(units / S) x (tokens per unit + a fixed
+// per-unit cost), tokens per unit being rounded up to the 32-token stage,
+// with at least 128 tokens per unit.  The fixed cost -- the start of a unit
+// waits for its query rows and first copies -- was measured at about 200
+// tokens' worth of work.
+int choose_splits_uncached(long long pairs, long long len, long long kSlots) {
   constexpr long long kOverhead = 200, kGran = 32, kMinTokens = 128;
   const long long cap = (len + kMinTokens - 1) / kMinTokens;
   long long best_n = 1, best_cost = -1;
@@ -125,13 +114,32 @@ int choose_splits(const kvq_cache& c, int max_len_hint, int ctas_per_sm) {
       best_n = n;
     }
   }
-  const int e = cache_next;
-  cache_next = (cache_next + 1) % kCache;
-  cached_pairs[e] = pairs;
-  cached_len[e] = len;
-  cached_slots[e] = kSlots;
-  cached_n[e] = (int)best_n;
-  return cached_n[e];
+  return (int)best_n;
+}
+
+// The search above costs a few microseconds for long sequences, and every
+// decode call plans its splits: the last few answers are kept per host
+// thread (the inputs are a handful of integers, so a hit is exact).
+int choose_splits(const kvq_cache& c, int max_len_hint, int ctas_per_sm, int sms) {
+  const long long pairs = (long long)c.batch * c.kv_heads;
+  long long len = c.max_tokens;
+  if (max_len_hint > 0 && max_len_hint < len) len = max_len_hint;
+  if (len <= 0 || pairs <= 0) return 1;
+  const long long kSlots = (long long)sms * (ctas_per_sm > 0 ? ctas_per_sm : 3);
+  struct Memo {
+    long long pairs, len, slots;
+    int n;
+  };
+  constexpr int kMemo = 8;
+  thread_local Memo memo[kMemo] = {};
+  thread_local int next = 0;
+  for (int i = 0; i < kMemo; ++i)
+    if (memo[i].n > 0 && memo[i].pairs == pairs && memo[i].len == len && memo[i].slots == kSlots)
+      return memo[i].n;
+  const int n = choose_splits_uncached(pairs, len, kSlots);
+  memo[next] = Memo{pairs, len, kSlots, n};
+  next = (next + 1) % kMemo;
+  return n;
 }
 
 struct SplitPlan {
@@ -144,18 +152,19 @@ kvq_status plan_splits(const kvq_cache* segs, int n_segs, int q_heads, int max_l
                        SplitPlan* plan) {
   plan->parts = 0;
   const int g = q_heads / segs[0].kv_heads;
+  const int sms = kvq::device_sm_count();
   for (int i = 0; i < n_segs; ++i) {
     const int bits = kernel_bits(segs[i].k);
     const int group = bits == 16 ? kD : segs[i].v.group_size;
     const bool kpc = segs[i].k.axis == KVQ_AXIS_CHANNEL;
     const int ctas = kvq::decode_ctas_per_sm(bits, group, g, kpc);
-    plan->n_split[i] = choose_splits(segs[i], max_len_hint, ctas);
+    plan->n_split[i] = choose_splits(segs[i], max_len_hint, ctas, sms);
     plan->wide[i] = 0;
     // the five-CTA build where its own plan needs more than one wave
     const int wide = kvq::decode_tm_wide_ctas_per_sm(bits, group, g, kpc);
     if (wide > 0) {
-      const int n = choose_splits(segs[i], max_len_hint, wide);
-      if ((long long)segs[i].batch * segs[i].kv_heads * n > 148LL * wide) {
+      const int n = choose_splits(segs[i], max_len_hint, wide, sms);
+      if ((long long)segs[i].batch * segs[i].kv_heads * n > (long long)sms * wide) {
         plan->n_split[i] = n;
         plan->wide[i] = 1;
       }
@@ -217,6 +226,36 @@ size_t workspace_for(const kvq_cache* segs, int q_heads, int parts) {
 }  // namespace
 
 namespace kvq {
+// The device's streaming multiprocessors, read once per device
+// (cudaDevAttrMultiProcessorCount).  KVQ_NUM_SMS in the environment
+// overrides it, for planning on a host without that device; with neither,
+// kDefaultSms (B200).
+int device_sm_count() {
+  static int env_sms = -1;  // -1: not read yet, 0: unset
+  if (env_sms < 0) {
+    const char* e = getenv("KVQ_NUM_SMS");
+    const long v = e != nullptr ? strtol(e, nullptr, 10) : 0;
+    env_sms = (v > 0 && v <= 4096) ? (int)v : 0;
+  }
+  if (env_sms > 0) return env_sms;
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cached[kMaxDev];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();  // no device here: clear the sticky-free error state
+    return kDefaultSms;
+  }
+  int n = cached[dev].load();
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      return kDefaultSms;
+    }
+    cached[dev].store(n);
+  }
+  return n;
+}
+
 size_t decode_zeroed_prefix_bytes(const kvq_cache* segs) {
   return kHeaderBytes + counter_bytes(segs);
 }
@@ -265,14 +304,21 @@ uint64_t kvq_kv_elements(uint64_t layers, uint64_t kv_heads, uint64_t head_dim,
 }
 
 kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const void* v_new,
-                               int32_t n_new, int32_t advance_seq_lens, void* stream) {
+                               kvq_dtype kv_dtype, int32_t n_new, int32_t advance_seq_lens,
+                               void* stream) {
   kvq_status st = check_cache(cache, false);
   if (st != KVQ_OK) return st;
   if (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new))
     return KVQ_ERR_INVALID_ARG;
+  if (kv_dtype != KVQ_F16 && kv_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
   if (n_new < 1) return KVQ_ERR_INVALID_ARG;
   if (n_new > cache->max_tokens) return KVQ_ERR_CAPACITY;
+  // bf16 input: the token-grouped formats only
+  if (kv_dtype == KVQ_BF16 &&
+      (cache->k.fmt == KVQ_FMT_OAKEN || cache->k.axis == KVQ_AXIS_CHANNEL))
+    return KVQ_ERR_UNSUPPORTED;
   kvq::QuantArgs a;
+  a.in_bf16 = kv_dtype == KVQ_BF16;
   a.k_new = static_cast<const __half*>(k_new);
   a.v_new = static_cast<const __half*>(v_new);
   a.k_codes = static_cast<uint8_t*>(cache->k.codes);
@@ -375,6 +421,7 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
     v.max_tokens = segs[i].max_tokens;
     v.n_split = plan.n_split[i];
     v.wide = plan.wide[i];
+    v.sms = kvq::device_sm_count();
     if (segs[i].k.fmt == KVQ_FMT_OAKEN) {
       v.k_oaken = oaken_params(segs[i].k);
       v.v_oaken = oaken_params(segs[i].v);
@@ -390,6 +437,17 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
 }
 
 }  // namespace
+
+namespace kvq {
+// kvq_decode_attention's argument checks alone (nothing enqueued).
+kvq_status decode_check_args(const kvq_cache* segs, int32_t n_segs, const void* q,
+                             kvq_dtype q_dtype, int32_t q_heads, float softmax_scale, float* out,
+                             float* lse, int32_t max_len_hint, void* workspace,
+                             size_t workspace_bytes) {
+  return decode_stages(segs, n_segs, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
+                       workspace, workspace_bytes, nullptr, 0);
+}
+}  // namespace kvq
 
 extern "C" {
 
@@ -443,7 +501,7 @@ kvq_status decode_step_stages(const kvq_cache* cache, const void* k_new, const v
   st = decode_stages(cache, 1, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
                      workspace, workspace_bytes, stream, 0);
   if (st != KVQ_OK) return st;
-  st = kvq_quantize_append(cache, k_new, v_new, 1, 1, stream);
+  st = kvq_quantize_append(cache, k_new, v_new, KVQ_F16, 1, 1, stream);
   if (st != KVQ_OK) return st;
   return decode_stages(cache, 1, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
                        workspace, workspace_bytes, stream, stages);

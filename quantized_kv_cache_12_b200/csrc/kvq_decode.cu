@@ -109,6 +109,7 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   uint8_t* stages = smem + C::HDR_BYTES + warp * C::STAGES * C::STAGE;
   int* unit_sm = reinterpret_cast<int*>(smem + C::HDR_MISC);
   int* fail_sm = unit_sm + 1;
+  int* qexp_sm = unit_sm + 8;  // [8] power-of-two shift of each staged query row
   uint32_t* counters = a.err + 1;  // [0] next unit, [1] CTAs done
 
   const uint64_t policy = l2_evict_first_policy();
@@ -174,7 +175,7 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   }
 
   // ---- the g query rows of this KV head, once per unit, as fp16 in smem
-  stage_queries<g>(a, b, kvh, q_sm, t);
+  stage_queries<g, C::EMAX - WP::exp(0)>(a, b, kvh, q_sm, qexp_sm, t);
   __syncthreads();
   // sum of q over each (group, head) row, in the MMA's units (the QK MMA
   // returns 2^(EMAX - 24) * sum(q * c))
@@ -236,8 +237,9 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   const int gr0 = row0_ok ? (gid >> lg) : 0;
   const int gr1 = row1_ok ? ((gid + 8) >> lg) : 0;
   const bool head_ok = gid < g;  // this lane's PV rows are a real head
-  // log2-domain softmax scale including the MMA's 2^(24 - EMAX)
-  const float score_scale = a.scale_log2 * pow2f(24 - C::EMAX);
+  // log2-domain softmax scale including the MMA's 2^(24 - EMAX), and the
+  // query row's shift: every score of this lane is head gid % g's
+  const float score_scale = a.scale_log2 * pow2f(24 - C::EMAX) * unshift(qexp_sm[gid & (g - 1)]);
   // this lane's token rows within a tile: MMA columns 2*tig, 2*tig+1 of the
   // two n-tiles, in the rho order
   const int tokA = rho(2 * tig), tokB = rho(2 * tig + 1);
@@ -580,6 +582,9 @@ __global__ void __launch_bounds__(kHeadDim * PG) decode_merge_kernel(const Decod
   float L = 0.f;
 #pragma unroll
   for (int w = 0; w < NW; ++w) L += red[w];
+  // every partial's o is finite (a split with no tokens stores 0), so a
+  // weight of 0 contributes exactly nothing; the loads stay independent of
+  // the weights
   float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
   int p = grp;
   for (; p + 3 * PG < P; p += 4 * PG) {
@@ -620,7 +625,7 @@ cudaError_t launch_split_g(const DecodeArgs& a, const SegView& seg, cudaStream_t
   }
   SplitParams P{a, seg};
   const long long units = (long long)seg.n_split * a.kv_heads * a.batch;
-  const long long slots = 148LL * C::MIN_CTAS;  // one wave of persistent CTAs
+  const long long slots = (long long)seg.sms * C::MIN_CTAS;  // one wave of persistent CTAs
   const unsigned grid = (unsigned)(units < slots ? units : slots);
   decode_split_kernel<BITS, GE, GR><<<grid, kWarps * 32, C::SMEM, s>>>(P);
   return cudaGetLastError();

@@ -50,24 +50,62 @@ __device__ __forceinline__ void load_chunk(const uint8_t* p, uint32_t (&w)[NW]) 
 }
 
 // The query rows of KV head `kvh` of sequence `b` (g rows of head_dim) into
-// shared memory as fp16.  bf16 queries are used through fp16, which is exact
-// for |q| in [2^-14, 65504].  Threads 0 .. g * 16 - 1 take part.
-template <int G>
+// shared memory as fp16, row h times 2^sh[h]: the kernels lift a query
+// element by up to 2^QUP before it becomes an fp16 tensor-core operand, so
+// sh[h] <= 0 is the largest value that keeps 2^QUP times the row's largest
+// |q| below 2^15.  A row with max |q| < 2^(15 - QUP) has sh = 0 and is stored
+// as it is (fp16 queries exactly; bf16 queries exactly for magnitudes in
+// [2^-14, 65504]); a larger row loses only the bits of its elements that
+// fall below 2^-24 after the shift.  The caller multiplies the row's scores
+// by 2^-sh[h].  All threads of the CTA call this (rows are half-warps of
+// threads 0 .. g * 16 - 1); qexp[h] receives sh[h].
+template <int G, int QUP>
 __device__ __forceinline__ void stage_queries(const DecodeArgs& a, int b, int kvh, __half* q_sm,
-                                              int t) {
+                                              int* qexp, int t) {
+  static_assert(G * (kHeadDim / 8) <= kWarps * 32, "one thread per 8 query elements");
   const long long qbase = ((long long)b * a.q_heads + (long long)kvh * G) * kHeadDim;
-  if (t < G * (kHeadDim / 8)) {
-    const uint4 raw = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.q) + qbase)[t];
-    uint4 h16 = raw;
-    if (a.q_is_bf16) {
-      const __nv_bfloat162* bb = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      __half2* hh = reinterpret_cast<__half2*>(&h16);
+  const bool mine = t < G * (kHeadDim / 8);
+  uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+  if (mine) raw = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.q) + qbase)[t];
+  // the row's largest magnitude as a bit pattern with the sign cleared (for
+  // fp16 and bf16 alike, the order of these patterns is the order of the
+  // magnitudes), over the thread's 8 elements, then its half-warp
+  constexpr uint32_t kAbs = 0x7FFF7FFFu;
+  uint32_t m = __vmaxu2(__vmaxu2(raw.x & kAbs, raw.y & kAbs), __vmaxu2(raw.z & kAbs, raw.w & kAbs));
+  m = max(m & 0xFFFFu, m >> 16);
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  if (mine) {
+    // floor(log2) of the largest magnitude (its biased exponent field; a
+    // subnormal gives the smallest normal exponent, which is small enough)
+    const int e = a.q_is_bf16 ? (int)(m >> 7) - 127 : (int)(m >> 10) - 15;
+    const int sh = e >= 15 - QUP ? max(14 - QUP - e, -120) : 0;
+    if (sh == 0 && !a.q_is_bf16) {
+      reinterpret_cast<uint4*>(q_sm)[t] = raw;
+    } else {
+      const float sc = __int_as_float((127 + sh) << 23);  // 2^sh, exact
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      uint4 h16;
+      uint32_t* hw = reinterpret_cast<uint32_t*>(&h16);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) hh[i] = __float22half2_rn(__bfloat1622float2(bb[i]));
+      for (int i = 0; i < 4; ++i) {
+        float2 x;
+        if (a.q_is_bf16)
+          x = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+        else
+          x = __half22float2(u32_as_h2(w[i]));
+        hw[i] = h2_as_u32(__floats2half2_rn(x.x * sc, x.y * sc));
+      }
+      reinterpret_cast<uint4*>(q_sm)[t] = h16;
     }
-    reinterpret_cast<uint4*>(q_sm)[t] = h16;
+    if ((t & 15) == 0) qexp[t >> 4] = sh;
   }
 }
+
+// 2^-sh for a row exponent of stage_queries (exact).
+__device__ __forceinline__ float unshift(int sh) { return __int_as_float((127 - sh) << 23); }
 
 // Token range [c0, c1) of split `split` of a sequence of length L: the splits
 // are whole 32-token stages, so a stage's copy never runs past

@@ -153,6 +153,12 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& r0, uin
   r1 = pack_h2(x1, n1);
 }
 
+// Centre two 8-bit codes held as fp16 subnormals c * 2^-24: c - 128, exact
+// (|c - 128| <= 128).
+__device__ __forceinline__ uint32_t center8(uint32_t v) {
+  return h2_as_u32(__hsub2(u32_as_h2(v), u32_as_h2(0x00800080u)));
+}
+
 template <int BITS, int GE, int GR, bool KPC, int OCC>
 __global__ void __launch_bounds__(kWarps * 32, TmCfg<BITS, GE, GR, KPC, OCC>::MIN_CTAS)
 decode_tm_kernel(const __grid_constant__ SplitParams P) {
@@ -160,12 +166,29 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   using WP = WordPairs<BITS>;
   using XP = CrossPairs<BITS>;
   // the zero point the codes are read against: symmetric INT8 codes are read
-  // as offset binary (c + 128) with a stored zero point of 0
+  // as offset binary (c + 128) with a stored zero point of 0.  On the V side
+  // 8-bit codes enter the tensor cores centred (c - 128, so symmetric INT8
+  // codes end up as c itself, with z = 0): the PV products are summed over
+  // a whole split, and offset codes near 128 would make those sums large
+  // while the output is their small difference
+  constexpr bool CENTER8 = BITS == 8 || BITS == kSym8;
   auto zero_of = [](float z) {
     if constexpr (BITS == kSym8)
       return z + 128.0f;
     else
       return z;
+  };
+  auto zero_of_v = [](float z) {
+    if constexpr (BITS == 8)
+      return z - 128.0f;
+    else
+      return z;
+  };
+  auto cen = [](uint32_t v) {
+    if constexpr (CENTER8)
+      return center8(v);
+    else
+      return v;
   };
   constexpr int D = C::D, NG = C::NG, NP = C::NP, HS = C::HS, CPH = C::CPH;
   // grouped PV: dims of each group per lane, and their V bytes and words
@@ -182,8 +205,10 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::HDR_BARS) + warp * C::STAGES;
   __half* q_sm = reinterpret_cast<__half*>(smem + C::HDR_Q);      // [GR][D]
   float* qs_sm = reinterpret_cast<float*>(smem + C::HDR_QS);      // [8] per QK column
+  float* hsc_sm = qs_sm + 8;  // [8] score scale of each query head
   int* unit_sm = reinterpret_cast<int*>(smem + C::HDR_MISC);
   int* fail_sm = unit_sm + 1;
+  int* qexp_sm = unit_sm + 8;  // [8] power-of-two shift of each staged query row
   // decode step: the new token's quantized K and V rows (codes, then meta)
   uint8_t* new_sm = smem + C::HDR_NEW;
   uint2* qf_sm = reinterpret_cast<uint2*>(smem + C::HDR_QF);     // [8 ks][32 lanes]
@@ -208,6 +233,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   const bool distinct = tig < C::W;        // this lane's combinations are not repeats
   const int dgrp = (16 * gid) / GE;        // group of the lane's 16 output dims
   const float score_scale = a.scale_log2 * pow2f(24 - C::EMAX);
+  // the largest power of two a query element is lifted by before it becomes
+  // an fp16 operand: 2^(EMAX - e) for the code exponent e = 0
+  constexpr int QUP = C::EMAX - WP::exp(0);
   // tokens of the lane's QK rows and PV k positions within a sub-tile
   const int tq0 = tok_perm(gid);
   const int tvA = tok_perm(2 * tig), tvB = tok_perm(2 * tig + 1);
@@ -297,9 +325,12 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     }
   }
 
-  // ---- the g query rows of this KV head, once per unit
-  stage_queries<GR>(a, b, kvh, q_sm, t);
+  // ---- the g query rows of this KV head, once per unit, and each head's
+  // score scale (undoing its row's power-of-two shift), read from shared
+  // memory where it is used rather than held in registers across the loop
+  stage_queries<GR, QUP>(a, b, kvh, q_sm, qexp_sm, t);
   __syncthreads();
+  if (t >= 64 && t < 64 + GR) hsc_sm[t - 64] = score_scale * unshift(qexp_sm[t - 64]);
   // column sums of q in the QK MMA's units (it returns 2^(EMAX - 24) sum q c)
   if constexpr (BITS != 16 && !KPC) {
     if (t < 64) {
@@ -534,30 +565,41 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         }
         const bool ok = valid(tok);
 #pragma unroll
-        for (int s = 0; s < HS; ++s) x[sub][s][r] = ok ? v[s] * score_scale : -INFINITY;
+        for (int s = 0; s < HS; ++s) x[sub][s][r] = ok ? v[s] * hsc_sm[own_h[s]] : -INFINITY;
       }
     }
 
     // ---- online softmax per owned head: max over the stage's tokens (rows
-    // gid and gid + 8 of every sub-tile, then across gid)
+    // gid and gid + 8 of every sub-tile, then across gid).  The reference
+    // point moves rarely, so a warp vote first asks whether any lane's own
+    // scores exceed it; only then are the maxima reduced across the rows.
     bool any_rescale = false;
     float alpha[HS];
+    float lmax[HS];
+    bool up = false;
 #pragma unroll
     for (int s = 0; s < HS; ++s) {
-      float tmax = -INFINITY;
+      lmax[s] = -INFINITY;
 #pragma unroll
-      for (int sub = 0; sub < NS; ++sub) tmax = fmaxf(tmax, fmaxf(x[sub][s][0], x[sub][s][1]));
-      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
-      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+      for (int sub = 0; sub < NS; ++sub) lmax[s] = fmaxf(lmax[s], fmaxf(x[sub][s][0], x[sub][s][1]));
+      up |= lmax[s] > m_ref[s];
       alpha[s] = 1.f;
-      if (tmax > m_ref[s]) {
-        const float m_new = tmax + kLazy;
-        if (m_ref[s] != -INFINITY) {
-          alpha[s] = fast_exp2(m_ref[s] - m_new);
-          any_rescale = true;
+    }
+    if (__any_sync(0xffffffffu, up)) {
+#pragma unroll
+      for (int s = 0; s < HS; ++s) {
+        float tmax = lmax[s];
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+        if (tmax > m_ref[s]) {
+          const float m_new = tmax + kLazy;
+          if (m_ref[s] != -INFINITY) {
+            alpha[s] = fast_exp2(m_ref[s] - m_new);
+            any_rescale = true;
+          }
+          m_ref[s] = m_new;
         }
-        m_ref[s] = m_new;
       }
     }
     if (__any_sync(0xffffffffu, any_rescale)) {
@@ -606,7 +648,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
             pp[r] = ok ? p[slot_of(nb)][r] * (sz.x * C::PSCALE) : 0.f;
             // in the weights' units: PSCALE is 1 for every format with a
             // zero point (the FP8 formats, lifted, have zero points of 0)
-            corr[nb] = ok ? fmaf(pp[r], zero_of(sz.y), corr[nb]) : corr[nb];
+            corr[nb] = ok ? fmaf(pp[r], zero_of_v(sz.y), corr[nb]) : corr[nb];
           }
         }
         uint32_t r0, r1;
@@ -636,8 +678,8 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
             XP::run(wC[w], wD[w], yc);
 #pragma unroll
             for (int i = 0; i < XP::kOut; ++i) {
-              xa[w * XP::kOut + i] = ya[i];
-              xc[w * XP::kOut + i] = yc[i];
+              xa[w * XP::kOut + i] = cen(ya[i]);
+              xc[w * XP::kOut + i] = cen(yc[i]);
             }
           }
 #pragma unroll
@@ -661,8 +703,8 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
           XP::run(wC[w], wD[w], yc);
 #pragma unroll
           for (int i = 0; i < XP::kOut; ++i) {
-            xa[w * XP::kOut + i] = ya[i];
-            xc[w * XP::kOut + i] = yc[i];
+            xa[w * XP::kOut + i] = cen(ya[i]);
+            xc[w * XP::kOut + i] = cen(yc[i]);
           }
         }
 #pragma unroll
@@ -815,7 +857,7 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   }
   SplitParams P{a, seg};
   const long long units = (long long)seg.n_split * a.kv_heads * a.batch;
-  const long long slots = 148LL * C::MIN_CTAS;  // one wave of persistent CTAs
+  const long long slots = (long long)seg.sms * C::MIN_CTAS;  // one wave of persistent CTAs
   const unsigned grid = (unsigned)(units < slots ? units : slots);
   decode_tm_kernel<BITS, GE, GR, KPC, OCC><<<grid, kWarps * 32, C::SMEM, s>>>(P);
   return cudaGetLastError();

@@ -13,7 +13,7 @@ namespace kvq {
 
 constexpr int kHeadDim = 128;  // the head_dim the kernels are compiled for
 constexpr int kTile = 16;      // tokens per warp step (one m16n8k16 K-extent)
-constexpr int kWarps = 4;      // consumer warps per decode CTA
+constexpr int kWarps = kWarpsPerCta;  // consumer warps per decode CTA
 
 // Device error flag bits (sticky word at the start of the decode workspace).
 constexpr uint32_t kErrWaitTimeout = 1u;

@@ -39,12 +39,18 @@ struct SegView {
   int32_t bits;
   int32_t group;
   int32_t max_tokens;
-  int32_t n_split;       // CTAs per (sequence, KV head) for this segment
-  int32_t part_base;     // index of this segment's first partial
+  int32_t n_split;       // units per (sequence, KV head): 16-row and Oaken kernels
+  int32_t part_base;     // index of this segment's first partial slot
   int32_t k_channels;    // K grouped per channel over kChannelBlock-token blocks
   int32_t wide;          // run the five-CTAs-per-SM build of the format
+  int32_t sms;           // streaming multiprocessors of the device
   OakenParams k_oaken, v_oaken;  // bits == kOaken: the planes' parameters
 };
+
+// warps of a decode CTA
+constexpr int kWarpsPerCta = 4;
+// SM count assumed when no device can be queried (a B200 has 148)
+constexpr int kDefaultSms = 148;
 
 struct DecodeArgs {
   int32_t batch, kv_heads, q_heads, group_ratio;
@@ -82,6 +88,8 @@ struct QuantArgs {
   // written and not advanced
   int32_t side0;
   int32_t k_channels;
+  // k_new and v_new hold bf16 values (else fp16); token-grouped formats only
+  int32_t in_bf16;
   OakenParams k_oaken, v_oaken;  // Oaken planes (launch_oaken_quantize)
 };
 // tokens per block of a per-channel K plane
@@ -107,6 +115,14 @@ cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s);
 bool decode_oaken_supported(int group_ratio);
 int decode_oaken_ctas_per_sm(int group_ratio);
 cudaError_t launch_decode_oaken(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
+// kvq_decode_attention's argument checks only: KVQ_OK means a call with the
+// same arguments enqueues its kernels (kvq_abi.cu)
+kvq_status decode_check_args(const kvq_cache* segs, int32_t n_segs, const void* q,
+                             kvq_dtype q_dtype, int32_t q_heads, float softmax_scale, float* out,
+                             float* lse, int32_t max_len_hint, void* workspace,
+                             size_t workspace_bytes);
+// streaming multiprocessors of the current device (kvq_abi.cu)
+int device_sm_count();
 // leading workspace bytes that hold the header and the counters (they must
 // be zero before a call whose cache shape differs from the previous call's)
 size_t decode_zeroed_prefix_bytes(const kvq_cache* segs);

@@ -168,14 +168,18 @@ __global__ void __launch_bounds__(kWarps * 32) oaken_decode_kernel(const __grid_
   const int bh = unit / n_split;
   const int b = bh / a.kv_heads, kvh = bh % a.kv_heads;
 
-  // the query rows, fp16 -> fp32 [D][G]
-  __half* qh = reinterpret_cast<__half*>(sm + C::QH_OFF);
+  // the query rows as fp32 [D][G], straight from the fp16 or bf16 inputs
+  // (exact; this kernel's arithmetic is fp32 throughout)
   float* qf = sm + C::Q_OFF;
-  stage_queries<G>(a, b, kvh, qh, t);
-  __syncthreads();
-  for (int i = t; i < D * G; i += kWarps * 32) {
-    const int j = i / G, h = i % G;
-    qf[i] = __half2float(qh[h * D + j]);
+  {
+    const uint16_t* qg = static_cast<const uint16_t*>(a.q) +
+                         ((long long)b * a.q_heads + (long long)kvh * G) * D;
+    for (int i = t; i < D * G; i += kWarps * 32) {
+      const int j = i / G, h = i % G;
+      const uint16_t u = qg[h * D + j];
+      qf[i] = a.q_is_bf16 ? __uint_as_float((uint32_t)u << 16)
+                          : __half2float(__ushort_as_half(u));
+    }
   }
   __syncthreads();
 
@@ -376,7 +380,8 @@ OakenParams make_oaken_params(float s_in, int z_in, float s_out, int outer_bits)
 cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s) {
   const long long rows = 2LL * a.batch * a.kv_heads * a.n_new;
   const long long blocks = (rows + 15) / 16;
-  const unsigned grid = (unsigned)(blocks < 148LL * 8 ? blocks : 148LL * 8);
+  const long long cap = (long long)device_sm_count() * 8;
+  const unsigned grid = (unsigned)(blocks < cap ? blocks : cap);
   oaken_quantize_kernel<<<grid, 256, 0, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !a.advance) return e;

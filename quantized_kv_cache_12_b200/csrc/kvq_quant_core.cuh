@@ -15,6 +15,7 @@
 // use an equivalent order that needs no conversion instruction.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -105,35 +106,72 @@ __device__ __forceinline__ void pack_codes(uint64_t (&t)[NV / 2], uint32_t* w) {
   }
 }
 
-// One thread holds NV (8, 16 or 32) consecutive fp16 values of a token row; the
-// G / NV threads of a group are consecutive lanes (groups never straddle a
-// row).  Produces the packed codes of the NV values (BITS bits each, element
-// j at bit offset BITS * j) and the (scale, zero) half2 of the group.
-template <int BITS, int G, int NV>
+// A pair of 16-bit input values in one 32-bit word: binary16 (BF false) or
+// bfloat16 (BF true).  Both widen to fp32 exactly, and their pairwise min and
+// max are exact; the sign bit is bit 15 of each half in both formats.
+template <bool BF>
+struct InPair {
+  static __device__ __forceinline__ float2 widen(uint32_t w) {
+    if constexpr (BF)
+      return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    else
+      return __half22float2(u32_as_h2(w));
+  }
+  static __device__ __forceinline__ uint32_t min2(uint32_t a, uint32_t b) {
+    if constexpr (BF) {
+      const __nv_bfloat162 r = __hmin2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                       *reinterpret_cast<const __nv_bfloat162*>(&b));
+      return *reinterpret_cast<const uint32_t*>(&r);
+    } else {
+      return h2_as_u32(__hmin2(u32_as_h2(a), u32_as_h2(b)));
+    }
+  }
+  static __device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b) {
+    if constexpr (BF) {
+      const __nv_bfloat162 r = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                       *reinterpret_cast<const __nv_bfloat162*>(&b));
+      return *reinterpret_cast<const uint32_t*>(&r);
+    } else {
+      return h2_as_u32(__hmax2(u32_as_h2(a), u32_as_h2(b)));
+    }
+  }
+  static __device__ __forceinline__ uint32_t swap(uint32_t a) { return __byte_perm(a, 0, 0x1032); }
+};
+
+// One thread holds NV (8, 16 or 32) consecutive 16-bit values of a token row
+// (fp16, or bf16 with BF); the G / NV threads of a group are consecutive lanes
+// (groups never straddle a row).  Produces the packed codes of the NV values
+// (BITS bits each, element j at bit offset BITS * j) and the (scale, zero)
+// half2 of the group.  Every value is widened to fp32 exactly, so both input
+// types go through the same fp32 steps.
+template <int BITS, int G, int NV, bool BF = false>
 __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
                                               uint32_t (&codes)[code_words<BITS, NV>()],
                                               uint32_t& meta) {
   static_assert(NV == 8 || NV == 16 || NV == 32, "values per thread");
   static_assert(G % NV == 0 && G / NV <= 32 && G <= kHeadDim, "group size");
+  using P = InPair<BF>;
   constexpr int NH = NV / 2;
   constexpr int GL = G / NV;  // lanes per group
-  const __half2* h2 = reinterpret_cast<const __half2*>(&raw[0]);
+  const uint32_t* w2 = reinterpret_cast<const uint32_t*>(&raw[0]);
   float x[NV];
 #pragma unroll
   for (int i = 0; i < NH; ++i) {
-    const float2 f = __half22float2(h2[i]);
+    const float2 f = P::widen(w2[i]);
     x[2 * i] = f.x;
     x[2 * i + 1] = f.y;
   }
   if constexpr (BITS == kE4M3 || BITS == kE5M2 || BITS == kSym8) {
-    // the group's |max|, taken on the fp16 values (exact)
-    __half2 am = __habs2(h2[0]);
+    // the group's |max|, taken on the 16-bit values (exact): clearing the
+    // sign bits is |.| in both formats
+    uint32_t am = w2[0] & 0x7FFF7FFFu;
 #pragma unroll
-    for (int i = 1; i < NH; ++i) am = __hmax2(am, __habs2(h2[i]));
-    am = __hmax2(am, __lowhigh2highlow(am));
+    for (int i = 1; i < NH; ++i) am = P::max2(am, w2[i] & 0x7FFF7FFFu);
+    am = P::max2(am, P::swap(am));
 #pragma unroll
     for (int off = 1; off < GL; off <<= 1)
-      am = __hmax2(am, u32_as_h2(__shfl_xor_sync(0xffffffffu, h2_as_u32(am), off)));
+      am = P::max2(am, __shfl_xor_sync(0xffffffffu, am, off));
+    const float amax = P::widen(am).x;
     if constexpr (BITS == kSym8) {
       // Symmetric INT8 (the KV-cache page's INT8 item): s = max(amax / 127,
       // 1e-5) stored in fp16 rounded up, so |x / s| <= 127 and the clamp to
@@ -142,7 +180,7 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
       // c + 128 in [1, 255]; flipping bit 7 of every byte then gives c.
       constexpr float kInv127 = 1.0f / 127.0f;
       constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-      const float s32 = fmaxf(div_rn(__low2float(am), 127.0f, kInv127), 1e-5f);
+      const float s32 = fmaxf(div_rn(amax, 127.0f, kInv127), 1e-5f);
       const __half s16 = __float2half_ru(s32);
       const float s = __half2float(s16);
       const float r = __frcp_rn(s);
@@ -165,7 +203,7 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
     // the fp32 quotient x / s; zero point 0.
     constexpr float kMaxF = BITS == kE4M3 ? 448.0f : 57344.0f;
     constexpr float kInvMax = 1.0f / kMaxF;
-    const float s32 = fmaxf(div_rn(__low2float(am), kMaxF, kInvMax), 1e-5f);
+    const float s32 = fmaxf(div_rn(amax, kMaxF, kInvMax), 1e-5f);
     const __half s16 = __float2half_ru(s32);
     const float s = __half2float(s16);
     const float r = __frcp_rn(s);
@@ -183,19 +221,21 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
     for (int i = 0; i < NH / 2; ++i) codes[i] = __byte_perm(c[2 * i], c[2 * i + 1], 0x5410);
     meta = h2_as_u32(__halves2half2(s16, __float2half_rn(0.f)));
   } else {
-    // group (min, -max) as one fp16 pair: one shuffle and one min per step
-    __half2 lo2 = h2[0], hi2 = h2[0];
+    // group (min, -max) as one 16-bit pair: one shuffle and one min per step
+    uint32_t lo2 = w2[0], hi2 = w2[0];
 #pragma unroll
     for (int i = 1; i < NH; ++i) {
-      lo2 = __hmin2(lo2, h2[i]);
-      hi2 = __hmax2(hi2, h2[i]);
+      lo2 = P::min2(lo2, w2[i]);
+      hi2 = P::max2(hi2, w2[i]);
     }
-    __half2 mm = __halves2half2(__hmin(__low2half(lo2), __high2half(lo2)),
-                                __hneg(__hmax(__low2half(hi2), __high2half(hi2))));
+    lo2 = P::min2(lo2, P::swap(lo2));
+    hi2 = P::max2(hi2, P::swap(hi2)) ^ 0x80008000u;  // -max in both halves
+    uint32_t mm = __byte_perm(lo2, hi2, 0x7610);      // (min, -max)
 #pragma unroll
     for (int off = 1; off < GL; off <<= 1)
-      mm = __hmin2(mm, u32_as_h2(__shfl_xor_sync(0xffffffffu, h2_as_u32(mm), off)));
-    const float mn = __low2float(mm), mx = -__high2float(mm);
+      mm = P::min2(mm, __shfl_xor_sync(0xffffffffu, mm, off));
+    const float2 mmf = P::widen(mm);
+    const float mn = mmf.x, mx = -mmf.y;
     constexpr int qmax_i = (1 << code_bits(BITS)) - 1;
     constexpr float qmax = float(qmax_i);
     constexpr float kInvQmax = 1.0f / qmax;
@@ -243,12 +283,12 @@ __device__ __forceinline__ void quantize_vals(const uint4 (&raw)[NV / 8],
 }
 
 // quantize_vals for 8 values per thread: codes in (codes_lo, codes_hi).
-template <int BITS, int G>
+template <int BITS, int G, bool BF = false>
 __device__ __forceinline__ void quantize8(const uint4 raw, uint32_t& codes_lo,
                                           uint32_t& codes_hi, uint32_t& meta) {
   const uint4 r[1] = {raw};
   uint32_t w[code_words<BITS, 8>()];
-  quantize_vals<BITS, G, 8>(r, w, meta);
+  quantize_vals<BITS, G, 8, BF>(r, w, meta);
   codes_lo = w[0];
   if constexpr (code_words<BITS, 8>() > 1)
     codes_hi = w[1];
@@ -281,17 +321,17 @@ __device__ __forceinline__ uint32_t bulk_slot_off(int ri, int k) {
 }
 
 
-// Quantize one 16-byte slice of a row and store it.  lane16 = index of the
-// slice within the 128-value row (0..15); all 32 lanes of the warp must call
+// Quantize one 16-byte slice of a row (fp16 values, or bf16 with BF) and
+// store it.  lane16 = index of the slice within the 128-value row (0..15); all 32 lanes of the warp must call
 // this together (the group reduction uses warp shuffles); `active` false
 // lanes load nothing and store nothing.
-template <int BITS, int G>
+template <int BITS, int G, bool BF = false>
 __device__ __forceinline__ void quantize_slice(const __half* src_row, uint8_t* codes_row,
                                                uint8_t* meta_row, int lane16, bool active) {
   uint4 raw = make_uint4(0u, 0u, 0u, 0u);
   if (active) raw = __ldg(reinterpret_cast<const uint4*>(src_row) + lane16);
   uint32_t lo, hi, meta;
-  quantize8<BITS, G>(raw, lo, hi, meta);
+  quantize8<BITS, G, BF>(raw, lo, hi, meta);
   if (!active) return;
   if (code_bits(BITS) == 8) {
     reinterpret_cast<uint2*>(codes_row)[lane16] = make_uint2(lo, hi);

@@ -2,8 +2,9 @@
 // cache (Cocktail page 3.2.2 formula; Oaken page 3.2.3 pipeline, where the
 // quantizer sits inside the memory write).
 //
-// Layout of a thread's work: a token row of 128 fp16 values is 16 lanes x 16
-// bytes; a warp quantizes two rows per step.  The row's groups are reduced
+// Layout of a thread's work: a token row of 128 16-bit values (fp16, or bf16
+// through the BF template flag) is 16 lanes x 16 bytes; a warp quantizes two
+// rows per step.  The row's groups are reduced
 // with warp shuffles, codes are packed in registers and written with one
 // 2/4/8-byte store per lane, and the group leader writes (scale, zero).
 #include <cuda_runtime.h>
@@ -46,7 +47,7 @@ __device__ __forceinline__ RowRef locate_row(const QuantArgs& a, long long r, in
 // Decode-step append: one CTA per sequence handles all of its rows, then
 // advances seq_lens[b] itself (every thread has read the old value before
 // the barrier, so the update cannot race with the writes).
-template <int BITS, int G>
+template <int BITS, int G, bool BF>
 __global__ void __launch_bounds__(1024) quantize_append_kernel(const QuantArgs a) {
   const int b = blockIdx.x;
   const int base = a.seq_lens[b];
@@ -63,7 +64,7 @@ __global__ void __launch_bounds__(1024) quantize_append_kernel(const QuantArgs a
         (rs < rows_per_side) ? (long long)b * rows_per_side + rs
                              : per + (long long)b * rows_per_side + (rs - rows_per_side);
     RowRef ref = locate_row<BITS, G>(a, global_row, base);
-    quantize_slice<BITS, G>(ref.src, ref.codes, ref.meta, lane16, in && ref.active);
+    quantize_slice<BITS, G, BF>(ref.src, ref.codes, ref.meta, lane16, in && ref.active);
   }
   if (a.advance) {
     __syncthreads();
@@ -185,7 +186,7 @@ __device__ __forceinline__ void bulk_issue(const QuantArgs& a, const BulkSrc& c,
   cp_async_commit();
 }
 
-template <int BITS, int G>
+template <int BITS, int G, bool BF>
 __device__ __forceinline__ void bulk_work(const QuantArgs& a, int li, const BulkDst<BITS, G>& c,
                                           const uint32_t (&roff)[kBulkNV / 8],
                                           const uint8_t* slot) {
@@ -196,7 +197,7 @@ __device__ __forceinline__ void bulk_work(const QuantArgs& a, int li, const Bulk
   for (int k = 0; k < kBulkNV / 8; ++k)
     raw[k] = in ? *reinterpret_cast<const uint4*>(slot + roff[k]) : make_uint4(0u, 0u, 0u, 0u);
   uint32_t cw[NW], m;
-  quantize_vals<BITS, G, kBulkNV>(raw, cw, m);
+  quantize_vals<BITS, G, kBulkNV, BF>(raw, cw, m);
   if (in && c.pos < a.max_tokens && !c.skip) {
     if constexpr (NW == 8) {
       reinterpret_cast<uint4*>(c.codes)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
@@ -211,7 +212,7 @@ __device__ __forceinline__ void bulk_work(const QuantArgs& a, int li, const Bulk
   }
 }
 
-template <int BITS, int G>
+template <int BITS, int G, bool BF>
 __global__ void __launch_bounds__(kBulkWarps * 32) quantize_bulk_kernel(const QuantArgs a,
                                                                         int units_per_row,
                                                                         int n_units,
@@ -259,7 +260,7 @@ __global__ void __launch_bounds__(kBulkWarps * 32) quantize_bulk_kernel(const Qu
     } else {
       cp_async_commit();
     }
-    bulk_work<BITS, G>(a, li, wc, roff, &ring[warp][i % kBulkDepth][0]);
+    bulk_work<BITS, G, BF>(a, li, wc, roff, &ring[warp][i % kBulkDepth][0]);
     wc.advance(a, units_per_row, ri, li);
   }
   cp_async_wait<0>();
@@ -365,12 +366,12 @@ __global__ void __launch_bounds__(kHeadDim) quantize_k_channels_kernel(const Qua
   }
 }
 
-template <int BITS, int G>
+template <int BITS, int G, bool BF>
 cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
   QuantArgs a = a_in;
   if (a.k_channels) {
     // K: whole blocks, per channel; then the per-token kernels write V only
-    if constexpr (BITS == 2 || BITS == 4 || BITS == 8) {
+    if constexpr ((BITS == 2 || BITS == 4 || BITS == 8) && !BF) {
       if (a.n_new % kChannelBlock != 0 || (long long)a.batch * a.kv_heads > 65535)
         return cudaErrorInvalidValue;
       const dim3 grid(a.n_new / kChannelBlock, a.batch * a.kv_heads);
@@ -387,28 +388,26 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
     // one pass over the sequence's rows when they fit in one CTA
     int threads = ((rows_per_seq * 16 + 63) / 64) * 64;
     if (threads > 1024) threads = 1024;
-    quantize_append_kernel<BITS, G><<<a.batch, threads, 0, s>>>(a);
+    quantize_append_kernel<BITS, G, BF><<<a.batch, threads, 0, s>>>(a);
     return cudaGetLastError();
   }
   const int units_per_row = (a.n_new + kUnitRows - 1) / kUnitRows;
   const long long n_units = (2LL - a.side0) * a.batch * a.kv_heads * units_per_row;
   if (n_units > 0x3fffffffLL) return cudaErrorInvalidValue;
-  static int slots = 0;  // resident CTAs on the device
-  if (slots == 0) {
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_bulk_kernel<BITS, G>,
-                                                        kBulkWarps * 32, 0);
+  static int per_sm = 0;  // resident CTAs per SM of this kernel
+  if (per_sm == 0) {
+    int r = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &r, quantize_bulk_kernel<BITS, G, BF>, kBulkWarps * 32, 0);
     if (e != cudaSuccess) return e;
-    slots = sms * (per_sm > 0 ? per_sm : 1);
+    per_sm = r > 0 ? r : 1;
   }
+  const long long slots = (long long)device_sm_count() * per_sm;
   // every resident warp takes an equal contiguous range of units
   const long long warps = (long long)slots * kBulkWarps;
   const long long per_warp = (n_units + warps - 1) / warps;
   const long long blocks = (n_units + per_warp * kBulkWarps - 1) / (per_warp * kBulkWarps);
-  quantize_bulk_kernel<BITS, G><<<(unsigned)blocks, kBulkWarps * 32, 0, s>>>(
+  quantize_bulk_kernel<BITS, G, BF><<<(unsigned)blocks, kBulkWarps * 32, 0, s>>>(
       a, units_per_row, (int)n_units, (int)per_warp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !a.advance) return e;
@@ -420,8 +419,9 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_quantize(const QuantArgs& a, int bits, int group, cudaStream_t s) {
-#define KVQ_Q(B, G_) \
-  if (bits == B && group == G_) return launch_q<B, G_>(a, s);
+#define KVQ_Q(B, G_)                                              \
+  if (bits == B && group == G_)                                   \
+    return a.in_bf16 ? launch_q<B, G_, true>(a, s) : launch_q<B, G_, false>(a, s);
   KVQ_Q(8, 32) KVQ_Q(8, 64) KVQ_Q(8, 128)
   KVQ_Q(4, 32) KVQ_Q(4, 64) KVQ_Q(4, 128)
   KVQ_Q(2, 32) KVQ_Q(2, 64) KVQ_Q(2, 128)

@@ -21,24 +21,19 @@ namespace {
 // KVQ_STATIC_SCRATCH_BYTES until the process exits.
 static __device__ __align__(256) unsigned char g_decode_scratch[KVQ_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
 
 // In host code the array's name is only a host-side stand-in, not a device
-// address, so the device address is looked up once per device, with that
-// device current, and cached.
+// address, so the device address is looked up with the caller's device
+// current.  It is looked up on every call (a host-side table read once the
+// module is loaded), so a call after a device reset sees the reloaded
+// module's array.
 kvq_status scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr)
-      return KVQ_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr)
+    return KVQ_ERR_CUDA;
+  *out = p;
   return KVQ_OK;
 }
 
@@ -56,9 +51,13 @@ extern "C" kvq_status kvq_decode_attention_noalloc(const kvq_cache* segs, int32_
   void* scratch = nullptr;
   st = scratch_address(&scratch);
   if (st != KVQ_OK) return st;
+  // every argument is checked before anything touches the shared array
+  st = kvq::decode_check_args(segs, n_segs, q, q_dtype, q_heads, softmax_scale, out, lse,
+                              max_len_hint, scratch, KVQ_STATIC_SCRATCH_BYTES);
+  if (st != KVQ_OK) return st;
   // The array keeps the previous call's contents, which may have had another
-  // layout.  The split kernels rewrite every partial they hand to the merge;
-  // the error word and the counters (at the front) start at zero.
+  // layout.  The decode kernels rewrite every partial slot they hand to a
+  // merge; the error word and the counters (at the front) start at zero.
   if (cudaMemsetAsync(scratch, 0, kvq::decode_zeroed_prefix_bytes(segs),
                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KVQ_ERR_CUDA;

@@ -69,7 +69,7 @@ def _load():
                                     ctypes.POINTER(sz)]
     lib.kvq_kv_elements.argtypes = [ctypes.c_uint64] * 5
     lib.kvq_kv_elements.restype = ctypes.c_uint64
-    lib.kvq_quantize_append.argtypes = [cp, P, P, i32, i32, P]
+    lib.kvq_quantize_append.argtypes = [cp, P, P, i32, i32, i32, P]
     lib.kvq_decode_workspace_bytes.argtypes = [cp, i32, i32, i32, ctypes.POINTER(sz)]
     for name in ("kvq_decode_attention", "kvq_decode_partials", "kvq_decode_merge"):
         getattr(lib, name).argtypes = [cp, i32, P, ctypes.c_int, i32, f32, P, P, i32, P, sz, P]
@@ -145,8 +145,13 @@ def kvq_kv_elements(layers, kv_heads, head_dim, seq_len, batch) -> int:
 
 def kvq_quantize_append(cache, k_new: torch.Tensor, v_new: torch.Tensor, n_new: int,
                         advance_seq_lens: bool = True, stream=None):
+    """k_new and v_new are fp16 or bf16 (both the same); the dtype is passed
+    as kvq_dtype."""
+    if k_new.dtype != v_new.dtype or k_new.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("kvq_quantize_append: k_new and v_new must both be float16 or bfloat16")
+    dt = KVQ_BF16 if k_new.dtype == torch.bfloat16 else KVQ_F16
     arr = _caches(cache)
-    _check(lib.kvq_quantize_append(arr, _ptr(k_new), _ptr(v_new), int(n_new),
+    _check(lib.kvq_quantize_append(arr, _ptr(k_new), _ptr(v_new), dt, int(n_new),
                                    int(bool(advance_seq_lens)), _stream(stream)),
            "kvq_quantize_append")
 

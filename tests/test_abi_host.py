@@ -5,6 +5,8 @@ import ctypes
 import json
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -103,7 +105,11 @@ def test_quantize_append_rejects_bad_arguments(kvq):
     S = kvq.kvq_quantize_append
     ok_ptr = 0x60000
 
-    class T:  # minimal tensor stand-in: only data_ptr() is used
+    import torch
+
+    class T:  # minimal tensor stand-in: only data_ptr() and dtype are used
+        dtype = torch.float16
+
         def __init__(self, p):
             self.p = p
 
@@ -127,6 +133,39 @@ def test_quantize_append_rejects_bad_arguments(kvq):
     c2 = _fake_cache(kvq)
     c2.v.group_size = 32
     assert _status(S, c2, T(ok_ptr), T(ok_ptr), 1) == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_quantize_append_kv_dtype(kvq):
+    """kv_dtype is KVQ_F16 or KVQ_BF16; bf16 input is refused for per-channel
+    K and Oaken planes (token-grouped formats only); the binding passes the
+    tensors' dtype and refuses mixed or other dtypes before calling."""
+    import torch
+    fake = ctypes.c_void_p(0x60000)
+
+    def st(c, dt, n=1):
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, dt, n, 1, None)
+    assert st(_fake_cache(kvq), 2) == kvq.KVQ_ERR_INVALID_ARG
+    assert st(_fake_cache(kvq), -1) == kvq.KVQ_ERR_INVALID_ARG
+    assert st(_fake_cache(kvq), kvq.KVQ_BF16, n=0) == kvq.KVQ_ERR_INVALID_ARG
+    assert st(_fake_cache(kvq, bits=3), kvq.KVQ_BF16) == kvq.KVQ_ERR_UNSUPPORTED
+    c = _fake_cache(kvq, bits=4)
+    c.k.axis = kvq.KVQ_AXIS_CHANNEL
+    assert st(c, kvq.KVQ_BF16, n=32) == kvq.KVQ_ERR_UNSUPPORTED
+    c = _fake_cache(kvq, bits=4, group=128)
+    c.k.fmt = c.v.fmt = kvq.KVQ_FMT_OAKEN
+    c.k.oaken = kvq.kvq_oaken(0.25, 8, 0.5, 5)
+    c.v.oaken = kvq.kvq_oaken(0.125, 3, 0.05, 7)
+    assert st(c, kvq.KVQ_BF16) == kvq.KVQ_ERR_UNSUPPORTED
+
+    class T:
+        def __init__(self, dtype):
+            self.dtype = dtype
+
+        def data_ptr(self):
+            return 0x60000
+    for a, b in ((torch.float16, torch.bfloat16), (torch.float32, torch.float32)):
+        with pytest.raises(TypeError):
+            kvq.kvq_quantize_append(_fake_cache(kvq), T(a), T(b), 1)
 
 
 def test_decode_workspace_and_argument_checks(kvq):
@@ -197,7 +236,7 @@ def test_fp8_planes_validated(kvq):
     fake = ctypes.c_void_p(0x60000)
 
     def append_status(c):
-        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, 1, 1, None)
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, kvq.KVQ_F16, 1, 1, None)
     c = _fake_cache(kvq, bits=4)
     c.k.fmt = c.v.fmt = kvq.KVQ_FMT_FP8_E4M3
     assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
@@ -219,7 +258,7 @@ def test_e5m2_planes_validated(kvq):
     fake = ctypes.c_void_p(0x60000)
 
     def append_status(c):
-        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, 1, 1, None)
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, kvq.KVQ_F16, 1, 1, None)
     c = _fake_cache(kvq, bits=4)
     c.k.fmt = c.v.fmt = kvq.KVQ_FMT_FP8_E5M2
     assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
@@ -239,7 +278,7 @@ def test_sym8_planes_validated(kvq):
     fake = ctypes.c_void_p(0x60000)
 
     def append_status(c):
-        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, 1, 1, None)
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, kvq.KVQ_F16, 1, 1, None)
     c = _fake_cache(kvq, bits=2)
     c.k.fmt = c.v.fmt = kvq.KVQ_FMT_INT8_SYM
     assert append_status(c) == kvq.KVQ_ERR_UNSUPPORTED
@@ -263,7 +302,7 @@ def test_channel_axis_validated(kvq):
     fake = ctypes.c_void_p(0x60000)
 
     def append_status(c, n):
-        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, n, 1, None)
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, kvq.KVQ_F16, n, 1, None)
     c = _fake_cache(kvq, bits=4)
     c.k.axis = kvq.KVQ_AXIS_CHANNEL
     assert append_status(c, 5) == kvq.KVQ_ERR_INVALID_ARG      # not a whole block
@@ -331,7 +370,7 @@ def test_oaken_planes_validated(kvq):
         return c
 
     def append_status(c):
-        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, 1, 1, None)
+        return kvq.lib.kvq_quantize_append((kvq.kvq_cache * 1)(c), fake, fake, kvq.KVQ_F16, 1, 1, None)
 
     for g in (1, 2, 4, 8):
         assert kvq.kvq_decode_workspace_bytes(oaken_cache(), 2 * g) > 0
@@ -379,22 +418,50 @@ def test_struct_layout_matches_the_header(kvq, tmp_path):
     assert got == want
 
 
+def _plan_parts(kvq, B, H, Hq, max_tokens, hint, bits=4, group=64, fmt=0):
+    """Partials per (sequence, query head) of a split plan, read back through
+    the workspace size: header, per-sequence counters, then (m, l) and o of
+    every partial."""
+    c = _fake_cache(kvq, bits=bits, group=group, max_tokens=max_tokens, batch=B, kv_heads=H)
+    c.k.fmt = c.v.fmt = fmt
+    if fmt == kvq.KVQ_FMT_OAKEN:
+        c.k.oaken = c.v.oaken = kvq.kvq_oaken(0.25, 8, 0.5, 5)
+    ws = kvq.kvq_decode_workspace_bytes(c, Hq, hint)
+    r256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    return next(p for p in range(1, 4096)
+                if 256 + r256(B * 4) + r256(B * Hq * p * 8) + r256(B * Hq * p * 128 * 4) == ws)
+
+
 def test_split_plan_per_workload(kvq):
-    """The host split plan (a wave model over 148 SMs x the format's CTAs
-    per SM, plus the five-CTA build of INT4 G64 g = 4 where its own plan
-    spans more than one wave), read back through the workspace size: the
-    partials per (sequence, query head) at the benchmark's shapes."""
-    def parts(B, H, Hq, max_tokens, hint, bits=4, group=64, fmt=0):
-        c = _fake_cache(kvq, bits=bits, group=group, max_tokens=max_tokens, batch=B, kv_heads=H)
-        c.k.fmt = c.v.fmt = fmt
-        if fmt == kvq.KVQ_FMT_OAKEN:
-            c.k.oaken = c.v.oaken = kvq.kvq_oaken(0.25, 8, 0.5, 5)
-        ws = kvq.kvq_decode_workspace_bytes(c, Hq, hint)
-        r256 = lambda n: (n + 255) // 256 * 256
-        return next(p for p in range(1, 4096)
-                    if 256 + r256(B * 4) + r256(B * Hq * p * 8) + r256(B * Hq * p * 128 * 4) == ws)
+    """The host split plan (a wave model over the device's SMs x the format's
+    CTAs per SM -- 148 on a host without that device -- plus the five-CTA
+    build of INT4 G64 g = 4 where its own plan spans more than one wave), at
+    the benchmark's shapes: the partials per (sequence, query head)."""
+    parts = lambda *a, **k: _plan_parts(kvq, *a, **k)  # noqa: E731
     assert parts(32, 8, 32, 8320, 8292) == 5        # Llama-3 GQA INT4: five-CTA build, 1.7 waves
     assert parts(16, 8, 32, 8320, 8292) == 9        # half the batch: the four-CTA build, 2 waves
     assert parts(1, 8, 32, 131392, 131328) == 74    # long context: one wave of the four-CTA build
     assert parts(16, 32, 32, 4224, 4196, bits=8, group=128) == 4   # Llama-2 MHA: 2048 units
     assert parts(32, 8, 32, 8320, 8192, group=128, fmt=kvq.KVQ_FMT_OAKEN) == 5
+
+
+def test_split_plan_follows_the_sm_count(tmp_path):
+    """The plan reads the device's SM count; KVQ_NUM_SMS overrides it (read
+    once per process, so the check runs in a child process).  With 74 SMs,
+    worked by hand from the wave model cost ceil(units / slots) x (tokens per
+    unit + 200): Llama-3 GQA INT4 (256 pairs) takes the five-CTA build (370
+    slots) at four splits -- cost 3 waves x (2080 + 200) = 6840 against 8520
+    for one split and 7080 for seven -- as its 1024 units exceed one wave;
+    the long context (8 pairs, four-CTA build, 296 slots) takes 37 splits,
+    the most that fit one wave (cost 3752 against 3984 for 74), and the
+    five-CTA plan (46 splits, 368 units) fits one wave, so it is not taken."""
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from quantized_kv_cache_12_b200 import kvq\n"
+        "import tests.test_abi_host as t\n"
+        "print(t._plan_parts(kvq, 32, 8, 32, 8320, 8292), "
+        "t._plan_parts(kvq, 1, 8, 32, 131392, 131328))\n" % ROOT)
+    env = dict(os.environ, KVQ_NUM_SMS="74")
+    out = subprocess.run([sys.executable, "-c", code], env=env, cwd=ROOT, check=True,
+                         capture_output=True, text=True).stdout.split()
+    assert out == ["4", "37"]

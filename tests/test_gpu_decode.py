@@ -305,3 +305,71 @@ def test_full_size_llama3_gqa_int4_sampled(kvq):
 
 def test_full_size_long_context_sampled(kvq):
     _full_size(kvq, "long_gqa_int4", [(0, 0), (0, 5)])
+
+
+def _large_query_case(kvq, bits, G, g, q_dtype, mag, zero_channel):
+    """K, V and queries N(0, 1), then one query element per head at `mag`
+    (dim 5).
+    With zero_channel, K's dim 5 is 0 on every token and dims 0..G-1 are
+    |N(0, 1)|, so that group's minimum is 0, its zero point +0 and dim 5's
+    code exactly 0: the large element contributes exactly nothing, and any
+    overflow of it inside the kernel shows as NaN."""
+    H, B, T = 2, 2, 200
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(77)
+    k = torch.randn((B, H, T, 128), generator=gen, device=DEV).half()
+    v = torch.randn((B, H, T, 128), generator=gen, device=DEV).half()
+    if zero_channel:
+        k[..., :G] = k[..., :G].abs()
+        k[..., 5] = 0.0
+    else:
+        # the large element meets a key channel scaled so that q_5 k_5 stays
+        # near N(0, 20^2): moderate scores, as the tensor cores' accumulation
+        # (not fp32 rounding alone) limits the precision of much larger ones
+        k[..., 5] = (k[..., 5].float() * (20.0 / mag)).half()
+    qf = torch.randn((B, H * g, 128), generator=gen, device=DEV)
+    qf[..., 5] = mag
+    qf[:, ::2, 5] = -mag  # both signs
+    q = qf.to(torch.bfloat16 if q_dtype == "bf16" else torch.float16)
+    assert torch.isfinite(q).all()
+    lens = [T, 151]
+    c = kvq.QuantizedKVCache.allocate(B, H, 128, 256, bits, G, DEV)
+    _poison(c)
+    fill_cache(kvq, c, k, v, lens)
+    out, lse = _run(kvq, c, q)
+    seg = oracle_segment(k, v, bits, G)
+    ref, lref = oracle.decode_attention(q_bits(q), q_dtype == "bf16", [seg], [lens],
+                                        128 ** -0.5)
+    return out, lse, ref, lref
+
+
+@pytest.mark.parametrize("bits,G,g,q_dtype,mag", [
+    (2, 32, 2, "f16", 2000.0), (2, 128, 8, "f16", 2000.0), (4, 64, 4, "f16", 5000.0),
+    (4, 128, 1, "f16", 60000.0), (4, 64, 8, "f16", 5000.0), (2, 32, 4, "f16", 2000.0),
+    (8, 128, 1, "f16", 60000.0), (4, 64, 4, "bf16", 1.0e5), (8, 128, 1, "bf16", 3.0e5),
+    (2, 32, 2, "bf16", 1.0e6)])
+def test_large_query_elements_do_not_overflow(kvq, bits, G, g, q_dtype, mag):
+    """A query element the kernels lift past the fp16 range (INT2 codes lift
+    query elements by up to 2^6, INT4 by 2^4) or a bf16 query above 65504:
+    the staged row is scaled down by a power of two and its scores scaled
+    back up, so the result is finite and within the attention tolerance of
+    the oracle (the large element meets exact-zero codes here, so the fp32
+    scores are as well conditioned as for N(0, 1) queries)."""
+    out, lse, ref, lref = _large_query_case(kvq, bits, G, g, q_dtype, mag, zero_channel=True)
+    assert_close(out, ref, lse, lref, what=f"large q bits{bits} G{G} g{g} {q_dtype} {mag}")
+
+
+@pytest.mark.parametrize("bits,G,g,mag", [(4, 64, 4, 5000.0), (2, 32, 2, 2000.0),
+                                          (4, 64, 8, 5000.0), (2, 128, 8, 1000.0)])
+def test_large_query_elements_meet_real_keys(kvq, bits, G, g, mag):
+    """The same large elements against keys whose channel 5 is scaled to
+    keep the products q_5 k_5 moderate: the large elements still meet real,
+    nonzero codes (and would overflow without the row shift), and the
+    result is within the attention tolerance.  A score is formed as
+    s (sum q c - z sum q) with the codes' sum accumulated by the tensor
+    cores, so its absolute error grows with |q_5| z rather than with the
+    score: with 2-bit groups of 128 and eight heads per KV head the
+    tolerance holds up to |q_5| of about 1000 (the header states the
+    limit)."""
+    out, lse, ref, lref = _large_query_case(kvq, bits, G, g, "f16", mag, zero_channel=False)
+    assert_close(out, ref, lse, lref, what=f"large q, real keys bits{bits} G{G} g{g}")

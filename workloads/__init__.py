@@ -169,8 +169,9 @@ def outlier_mask(wl: DecodeWorkload, which: str) -> torch.Tensor:
 
 
 def kv_tokens(wl: DecodeWorkload, n_tokens: int, device, stream_extra: int = 0,
-              batch: Optional[int] = None):
-    """Fresh K and V rows, fp16 [B, kv_heads, n_tokens, head_dim].
+              batch: Optional[int] = None, dtype: torch.dtype = torch.float16):
+    """Fresh K and V rows [B, kv_heads, n_tokens, head_dim] of ``dtype``
+    (fp16, or bf16: the same fp32 draws rounded to the other type).
 
     ``stream_extra`` selects an independent stream (0 = the prompt/context,
     1 + step = the token appended at that decode step)."""
@@ -182,7 +183,7 @@ def kv_tokens(wl: DecodeWorkload, n_tokens: int, device, stream_extra: int = 0,
         x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
         x.mul_(sigma)
         x.mul_(outlier_mask(wl, which).to(device)[None, :, None, :])
-        out.append(x.to(torch.float16))
+        out.append(x.to(dtype))
     return out[0], out[1]
 
 
