@@ -94,8 +94,8 @@ def split_kernel_name(wl) -> str:
     """The decode kernel the library picks for this workload's formats: the
     tokens-on-M kernel when (head_dim / G) * g <= 8, else the 16-row one."""
     g = wl.q_heads // wl.kv_heads
-    if wl.fmt == "oaken":
-        return "oaken_decode_kernel"
+    if wl.fmt == "oaken":  # one (s, z) per plane: a single group per token
+        return "decode_tm_kernel"
     groups = [128, wl.group] if wl.chunk_tokens else [wl.group]  # + the FP16 segment
     ok = all((128 // G) * g <= 8 for G in groups)
     return "decode_tm_kernel" if ok else "decode_split_kernel"
@@ -844,7 +844,9 @@ def run_kvq(args, wl, rank, world, local_rank):
                   f"K/V read per step per GPU (L2 126 MB)",
             "step": ("kvq_decode_step: quantize-on-write of 1 token/seq inside the split-K "
                      "decode attention kernel, then the LSE merge" if wl.append else
-                     "split-K decode attention over the FP16/INT4/INT2 segments + LSE merge")}),
+                     "split-K decode attention over the FP16/INT4/INT2 segments + LSE merge"
+                     if wl.chunk_tokens else
+                     "split-K decode attention over the prefilled cache + LSE merge")}),
         "kv_read_gbs": sum(kv_bytes) / (ms / 1e3) / 1e9 * world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,

@@ -94,22 +94,33 @@ kvq_status check_cache(const kvq_cache* c, bool allow16) {
 }
 
 // Split count of one segment.  A (sequence, KV head, split) is one unit of
-// work; the decode kernels run one wave of persistent CTAs (S = SMs x the format's CTAs per SM) that take units from
-// a counter.  With equal units the kernel takes ceil(units / S) unit-times,
-// so the count minimises ceil(units / S) x (tokens per unit + a fixed
-// per-unit cost), tokens per unit being rounded up to the 32-token stage,
-// with at least 128 tokens per unit.  The fixed cost -- the start of a unit
-// waits for its query rows and first copies -- was measured at about 200
-// tokens' worth of work.
-int choose_splits_uncached(long long pairs, long long len, long long kSlots) {
-  constexpr long long kOverhead = 200, kGran = 32, kMinTokens = 128;
+// work; the decode kernels run one wave of persistent CTAs (C per SM, the
+// format's occupancy) that take units from a counter, so each SM works
+// through about u = ceil(units / SMs) units in rounds of up to C at a time.
+// An SM's throughput is shared by its resident CTAs and saturates at about
+// three of them, so a round of c < 3 units runs at c/3 of the SM's rate.
+// The count minimises the SM's time, sum over its rounds of c x (tokens per
+// unit + a fixed per-unit cost) / min(1, c/3), tokens per unit being rounded
+// up to the 32-token stage, with at least 128 tokens per unit.  The fixed
+// cost -- the start of a unit waits for its query rows and first copies,
+// its end merges the warps -- is about 300 tokens' worth of work.  Both
+// constants were fitted to split-count sweeps on B200 (INT4, INT8, FP8,
+// per-channel K; 8 to 512 (sequence, head) pairs, 4k to 131k tokens).
+int choose_splits_uncached(long long pairs, long long len, int sms, int ctas) {
+  constexpr long long kOverhead = 300, kGran = 32, kMinTokens = 128;
+  constexpr double kSat = 3.0;
   const long long cap = (len + kMinTokens - 1) / kMinTokens;
-  long long best_n = 1, best_cost = -1;
+  long long best_n = 1;
+  double best_cost = -1.0;
   for (long long n = 1; n <= cap && n <= 4096; ++n) {
     const long long chunk = ((len + n - 1) / n + kGran - 1) / kGran * kGran;
-    const long long waves = (pairs * n + kSlots - 1) / kSlots;
-    const long long cost = waves * (chunk + kOverhead);
-    if (best_cost < 0 || cost < best_cost) {
+    const long long u = (pairs * n + sms - 1) / sms;  // units of the busiest SM
+    const long long full = u / ctas, rest = u % ctas;
+    const double c_full = (double)ctas, c_rest = (double)rest;
+    double rounds = (double)full * c_full / (c_full < kSat ? c_full / kSat : 1.0);
+    if (rest > 0) rounds += c_rest / (c_rest < kSat ? c_rest / kSat : 1.0);
+    const double cost = rounds * (double)(chunk + kOverhead);
+    if (best_cost < 0 || cost < best_cost * (1.0 - 1e-9)) {
       best_cost = cost;
       best_n = n;
     }
@@ -125,26 +136,26 @@ int choose_splits(const kvq_cache& c, int max_len_hint, int ctas_per_sm, int sms
   long long len = c.max_tokens;
   if (max_len_hint > 0 && max_len_hint < len) len = max_len_hint;
   if (len <= 0 || pairs <= 0) return 1;
-  const long long kSlots = (long long)sms * (ctas_per_sm > 0 ? ctas_per_sm : 3);
+  const int ctas = ctas_per_sm > 0 ? ctas_per_sm : 3;
   struct Memo {
-    long long pairs, len, slots;
-    int n;
+    long long pairs, len;
+    int sms, ctas, n;
   };
   constexpr int kMemo = 8;
   thread_local Memo memo[kMemo] = {};
   thread_local int next = 0;
   for (int i = 0; i < kMemo; ++i)
-    if (memo[i].n > 0 && memo[i].pairs == pairs && memo[i].len == len && memo[i].slots == kSlots)
+    if (memo[i].n > 0 && memo[i].pairs == pairs && memo[i].len == len && memo[i].sms == sms &&
+        memo[i].ctas == ctas)
       return memo[i].n;
-  const int n = choose_splits_uncached(pairs, len, kSlots);
-  memo[next] = Memo{pairs, len, kSlots, n};
+  const int n = choose_splits_uncached(pairs, len, sms, ctas);
+  memo[next] = Memo{pairs, len, sms, ctas, n};
   next = (next + 1) % kMemo;
   return n;
 }
 
 struct SplitPlan {
   int n_split[16];
-  int wide[16];  // the segment runs its format's five-CTAs-per-SM build
   int parts;
 };
 
@@ -159,16 +170,6 @@ kvq_status plan_splits(const kvq_cache* segs, int n_segs, int q_heads, int max_l
     const bool kpc = segs[i].k.axis == KVQ_AXIS_CHANNEL;
     const int ctas = kvq::decode_ctas_per_sm(bits, group, g, kpc);
     plan->n_split[i] = choose_splits(segs[i], max_len_hint, ctas, sms);
-    plan->wide[i] = 0;
-    // the five-CTA build where its own plan needs more than one wave
-    const int wide = kvq::decode_tm_wide_ctas_per_sm(bits, group, g, kpc);
-    if (wide > 0) {
-      const int n = choose_splits(segs[i], max_len_hint, wide, sms);
-      if ((long long)segs[i].batch * segs[i].kv_heads * n > (long long)sms * wide) {
-        plan->n_split[i] = n;
-        plan->wide[i] = 1;
-      }
-    }
     plan->parts += plan->n_split[i];
   }
   return KVQ_OK;
@@ -420,7 +421,6 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
     v.k_channels = segs[i].k.axis == KVQ_AXIS_CHANNEL;
     v.max_tokens = segs[i].max_tokens;
     v.n_split = plan.n_split[i];
-    v.wide = plan.wide[i];
     v.sms = kvq::device_sm_count();
     if (segs[i].k.fmt == KVQ_FMT_OAKEN) {
       v.k_oaken = oaken_params(segs[i].k);
@@ -493,10 +493,14 @@ kvq_status decode_step_stages(const kvq_cache* cache, const void* k_new, const v
   if (k_new == nullptr || v_new == nullptr || !aligned16(k_new) || !aligned16(v_new))
     return KVQ_ERR_INVALID_ARG;
   const int g = q_heads / cache->kv_heads;
-  if (kvq::decode_tm_supported(kernel_bits(cache->k), cache->k.group_size, g))
+  // the tokens-on-M kernel quantizes the new token itself, except for the
+  // Oaken codec, whose row encoding (the outlier slots) has its own kernel
+  if (cache->k.fmt != KVQ_FMT_OAKEN &&
+      kvq::decode_tm_supported(kernel_bits(cache->k), cache->k.group_size, g))
     return decode_stages(cache, 1, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
                          workspace, workspace_bytes, stream, stages, k_new, v_new);
-  // formats of the 16-row kernel: the append kernel, then the attention
+  // formats of the 16-row kernel and the Oaken codec: the append kernel,
+  // then the attention
   // (every argument is checked before the first launch)
   st = decode_stages(cache, 1, q, q_dtype, q_heads, softmax_scale, out, lse, max_len_hint,
                      workspace, workspace_bytes, stream, 0);

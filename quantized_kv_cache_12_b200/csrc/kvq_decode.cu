@@ -634,8 +634,7 @@ cudaError_t launch_split_g(const DecodeArgs& a, const SegView& seg, cudaStream_t
 }  // namespace
 
 bool decode_supported(int bits, int group, int group_ratio, bool kpc) {
-  if (bits == kOaken) return !kpc && group == kHeadDim && decode_oaken_supported(group_ratio);
-  if (kpc || bits == kE4M3 || bits == kE5M2 || bits == kSym8)
+  if (kpc || bits == kE4M3 || bits == kE5M2 || bits == kSym8 || bits == kOaken)
     return decode_tm_supported(bits, group, group_ratio, kpc);
   if (!(group_ratio == 1 || group_ratio == 2 || group_ratio == 4 || group_ratio == 8))
     return false;
@@ -646,7 +645,6 @@ bool decode_supported(int bits, int group, int group_ratio, bool kpc) {
 }
 
 int decode_ctas_per_sm(int bits, int group, int group_ratio, bool kpc) {
-  if (bits == kOaken) return decode_oaken_ctas_per_sm(group_ratio);
   if (decode_tm_supported(bits, group, group_ratio, kpc))
     return decode_tm_ctas_per_sm(bits, group, group_ratio, kpc);
   return Cfg<4, 64>::MIN_CTAS;  // the same for every format
@@ -654,7 +652,6 @@ int decode_ctas_per_sm(int bits, int group, int group_ratio, bool kpc) {
 
 cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   const int bits = seg.bits, group = (seg.bits == 16) ? kHeadDim : seg.group;
-  if (bits == kOaken) return launch_decode_oaken(a, seg, s);
   // (group, head) columns that fit one 8-wide tile: tokens-on-M kernel
   if (decode_tm_supported(bits, group, a.group_ratio, seg.k_channels))
     return launch_decode_tm(a, seg, s);

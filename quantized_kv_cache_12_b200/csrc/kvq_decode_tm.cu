@@ -52,12 +52,16 @@ namespace kvq {
 
 namespace {
 
-template <int BITS, int GE, int GR, bool KPC = false, int OCC = 0>
+template <int BITS, int GE, int GR, bool KPC = false>
 struct TmCfg {
   static constexpr int D = kHeadDim;
+  // the Oaken codec: 4-bit dense codes with one (s, z) per plane, and a
+  // row's outlier slots in place of per-token (s, z) pairs
+  static constexpr bool OAK = BITS == kOaken;
   static constexpr int NG = D / GE;                    // V groups per token (and K's, per token)
   static constexpr int RB = D * code_bits(BITS) / 8;   // code bytes per token
-  static constexpr int MB = (BITS == 16) ? 0 : NG * 4; // (s, z) bytes per token
+  static constexpr int MB =                            // (s, z) (or slot) bytes per token
+      (BITS == 16) ? 0 : (OAK ? KVQ_OAKEN_SLOTS * 2 : NG * 4);
   // K meta bytes per token: per-channel K (KPC) stores D (s, z) pairs per
   // block of kChannelBlock tokens, i.e. 16 bytes per token, and a stage is
   // one block
@@ -93,16 +97,18 @@ struct TmCfg {
   // (8 x 32 lanes x 8 B) instead of being held in 16 registers per thread
   static constexpr bool QB_SMEM = false;
   static constexpr int HDR_QF = HDR_NEW + 2 * NEW_STRIDE;
-  // per-channel K: the g query rows times each dim's 2^(EMAX - e), fp16
-  static constexpr int QF_BYTES = QB_SMEM ? 8 * 32 * 8 : (KPC ? GR * D * 2 : 0);
+  // per-channel K: the g query rows times each dim's 2^(EMAX - e), fp16;
+  // Oaken: the query table [D][GR] fp32 of the K slots' products, and each
+  // warp's slot scores [32 tokens][GR] fp32
+  static constexpr int QF_BYTES =
+      QB_SMEM ? 8 * 32 * 8 : (KPC ? GR * D * 2 : (OAK ? (D + kWarps * 32) * GR * 4 : 0));
   static constexpr int HDR_BYTES = ((HDR_QF + QF_BYTES + 127) / 128) * 128;
   // four CTAs per SM (128 registers a thread) where three stages per warp
   // fit in a quarter of the SM's shared memory (4 x (56 KB + 1 KB reserved)
-  // <= 228 KB), else three; OCC > 0 asks for that many instead (five: 102
-  // registers a thread and 44 KB, which leaves two stages per warp)
+  // <= 228 KB), else three
   static constexpr int MIN_CTAS =
-      OCC > 0 ? OCC : ((NO == 1 && HDR_BYTES + kWarps * 3 * STAGE <= 56 * 1024) ? 4 : 3);
-  static constexpr int SMEM_BUDGET = (MIN_CTAS >= 5 ? 44 : (MIN_CTAS == 4 ? 56 : 74)) * 1024;
+      (NO == 1 && HDR_BYTES + kWarps * 3 * STAGE <= 56 * 1024) ? 4 : 3;
+  static constexpr int SMEM_BUDGET = (MIN_CTAS == 4 ? 56 : 74) * 1024;
   static constexpr int STAGES_RAW = (SMEM_BUDGET - HDR_BYTES) / (kWarps * STAGE);
   static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 16 ? 16 : STAGES_RAW);
   static constexpr int SMEM = HDR_BYTES + kWarps * STAGES * STAGE;
@@ -126,6 +132,11 @@ struct TmCfg {
   static_assert(!KPC || ((BITS == 2 || BITS == 4 || BITS == 8) && STOK == kChannelBlock &&
                          CPH == 2 && HS == 1),
                 "per-channel K: integer codes, one block per stage, two columns per head");
+  // Oaken: one group per token (the plane's (s, z)), and the V slots'
+  // scatter tile of one 16-token sub-tile (128 dims x 16 tokens of fp16)
+  // fits the stage's code bytes
+  static_assert(!OAK || (NG == 1 && !GPV && 2 * STOK * RB >= D * kTile * 2 && SUB == 2),
+                "Oaken: one group per token, scatter tile inside the stage's codes");
 };
 
 // Token of MMA row r (0 .. 15) of a 16-token sub-tile.
@@ -159,12 +170,13 @@ __device__ __forceinline__ uint32_t center8(uint32_t v) {
   return h2_as_u32(__hsub2(u32_as_h2(v), u32_as_h2(0x00800080u)));
 }
 
-template <int BITS, int GE, int GR, bool KPC, int OCC>
-__global__ void __launch_bounds__(kWarps * 32, TmCfg<BITS, GE, GR, KPC, OCC>::MIN_CTAS)
+template <int BITS, int GE, int GR, bool KPC>
+__global__ void __launch_bounds__(kWarps * 32, TmCfg<BITS, GE, GR, KPC>::MIN_CTAS)
 decode_tm_kernel(const __grid_constant__ SplitParams P) {
-  using C = TmCfg<BITS, GE, GR, KPC, OCC>;
+  using C = TmCfg<BITS, GE, GR, KPC>;
   using WP = WordPairs<BITS>;
   using XP = CrossPairs<BITS>;
+  constexpr bool OAK = C::OAK;
   // the zero point the codes are read against: symmetric INT8 codes are read
   // as offset binary (c + 128) with a stored zero point of 0.  On the V side
   // 8-bit codes enter the tensor cores centred (c - 128, so symmetric INT8
@@ -307,8 +319,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   }
 
   // ---- decode step: quantize the new K (lanes 0-15) and V (16-31) rows of
-  // this KV head into shared memory, then copy them to the cache
-  if constexpr (BITS != 16 && !KPC) {
+  // this KV head into shared memory, then copy them to the cache (the
+  // Oaken codec appends with its own kernel before the attention)
+  if constexpr (BITS != 16 && !KPC && !OAK) {
     if (append_here && warp == 0) {
       const int vh = lane >> 4, l16 = lane & 15;
       const __half* src = (vh ? a.v_new : a.k_new) + ((long long)b * a.kv_heads + kvh) * D;
@@ -345,6 +358,15 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
       if (part == 0) qs_sm[r] = acc * pow2f(C::EMAX - 24);
     }
   }
+  // Oaken: the K slots' query table, otab[j][h] = q_h,j s_out in the QK
+  // MMA's units (2^(EMAX - 24) times the staged, shifted query)
+  float* otab = reinterpret_cast<float*>(smem + C::HDR_QF);             // [D][GR]
+  float* spx = otab + D * GR + warp * 32 * GR;                          // [32][GR]
+  if constexpr (OAK) {
+    const float f = pow2f(C::EMAX - 24) * seg.k_oaken.s_out;
+    for (int i = t; i < D * GR; i += kWarps * 32)
+      otab[i] = __half2float(q_sm[(i % GR) * D + i / GR]) * f;
+  }
   __syncthreads();
   // B fragments of QK: pair p = 2 ks + h of this lane's chunk, column gid;
   // each element scaled by 2^(EMAX - e) for the exponent e of its code
@@ -373,6 +395,10 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   }
   const float qsA = (BITS != 16 && !KPC) ? qs_sm[2 * tig] : 0.f;
   const float qsB = (BITS != 16 && !KPC) ? qs_sm[2 * tig + 1] : 0.f;
+  // Oaken planes' parameters (unused for the other formats)
+  const float ks_in = seg.k_oaken.s_in, kz_in = seg.k_oaken.z;
+  const float vs_in = seg.v_oaken.s_in, vz_in = seg.v_oaken.z;
+  const float v_ratio = seg.v_oaken.s_out / seg.v_oaken.s_in;
 
   // Per-channel K: the QK B fragments of a block are q * s_d for the block's
   // channel scales, in two fp16 parts (hi in the even columns, lo = the fp32
@@ -484,6 +510,41 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     constexpr bool FULL = decltype(full_tag)::value;
     constexpr int NS = C::SUB;
     kpc_rebuild(sKm);
+    if constexpr (OAK) {
+      // the K outlier slots' score terms, lane = token of the stage: sum
+      // over its slots of d * otab[dim] for every query head, into spx
+      // (a slot is the dim in its low byte, the signed shift in its high
+      // byte; an empty slot is 0 and adds 0; rows past the valid length may
+      // hold any bytes, their scores are masked below)
+      const uint4* sl = reinterpret_cast<const uint4*>(sKm + lane * C::MB);
+      const uint4 s0 = sl[0], s1 = sl[1];
+      const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      float acc[GR];
+#pragma unroll
+      for (int h = 0; h < GR; ++h) acc[h] = 0.f;
+#pragma unroll
+      for (int k = 0; k < KVQ_OAKEN_SLOTS; ++k) {
+        const uint32_t u = (k & 1) ? (sw[k >> 1] >> 16) : sw[k >> 1];
+        const float d = (float)(int)(int8_t)(uint8_t)(u >> 8);
+        const float* tr = otab + (u & 0x7Fu) * GR;
+        if constexpr (GR % 4 == 0) {
+#pragma unroll
+          for (int h = 0; h < GR; h += 4) {
+            const float4 tv = *reinterpret_cast<const float4*>(tr + h);
+            acc[h] = fmaf(d, tv.x, acc[h]);
+            acc[h + 1] = fmaf(d, tv.y, acc[h + 1]);
+            acc[h + 2] = fmaf(d, tv.z, acc[h + 2]);
+            acc[h + 3] = fmaf(d, tv.w, acc[h + 3]);
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < GR; ++h) acc[h] = fmaf(d, tr[h], acc[h]);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < GR; ++h) spx[lane * GR + h] = acc[h];
+      __syncwarp();
+    }
     auto valid = [&](int tok) { return FULL || tok < n_valid; };  // tok: 0 .. STOK-1
     // V rows past the valid length may hold any bytes.  Integer codes are
     // finite and meet a zero weight; raw fp16 and FP8 bytes can be NaN or
@@ -550,6 +611,12 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
           if constexpr (HS == 2) v[HS - 1] = s_acc[2 * r + 1];
         } else if constexpr (KPC) {
           v[0] = s_acc[2 * r] + s_acc[2 * r + 1] - kbias;
+        } else if constexpr (OAK) {
+          // the plane's (s_in, z_in), plus the token's slot terms
+          const float* sp = spx + tok * GR;
+          v[0] = fmaf(ks_in, fmaf(-kz_in, qsA, s_acc[2 * r]), sp[own_h[0]]);
+          if constexpr (HS == 2)
+            v[HS - 1] = fmaf(ks_in, fmaf(-kz_in, qsB, s_acc[2 * r + 1]), sp[own_h[HS - 1]]);
         } else if constexpr (NG == 1) {
           const float2 sz = __half22float2(*reinterpret_cast<const __half2*>(sKm + tok * C::MB));
           v[0] = sz.x * fmaf(-zero_of(sz.y), qsA, s_acc[2 * r]);
@@ -620,6 +687,8 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     }
 
     // ---- weights and O^T += V^T * P'^T per sub-tile
+    float p_keep[OAK ? NS : 1][HS][2];  // Oaken: the weights, for the V slots below
+    (void)p_keep;
 #pragma unroll
     for (int sub = 0; sub < NS; ++sub) {
       float p[HS][2];
@@ -629,6 +698,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         for (int r = 0; r < 2; ++r) {
           p[s][r] = fast_exp2(x[sub][s][r] - m_ref[s]);  // 0 for masked tokens
           l_part[s] += p[s][r];
+          if constexpr (OAK) p_keep[sub][s][r] = p[s][r];
         }
       uint32_t bf0[NP], bf1[NP];
 #pragma unroll
@@ -636,7 +706,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         float pp[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          if constexpr (BITS == 16) {
+          if constexpr (BITS == 16 || OAK) {
+            // raw fp16; or the Oaken codec, whose one V scale and zero
+            // point are applied at the output (z_in times the weights' sum)
             pp[r] = p[slot_of(nb)][r];
           } else {
             const int tok = sub * kTile + tq0 + 8 * r;
@@ -714,6 +786,73 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
             mma_f16(o_acc[nb][mt], xa[mt], xa[mt + 8], xc[mt], xc[mt + 8], bf0[nb], bf1[nb]);
       }
     }
+
+    if constexpr (OAK) {
+      // ---- the V outlier slots: O^T += Vd^T * P_sp^T per sub-tile, into the
+      // same accumulators.  Vd is the sub-tile's slots scattered into a
+      // dense fp16 tile [128 dims][16 tokens] (d * 2^(e - 24), the exponent
+      // of the dim's code position, so the output scale of the dense codes
+      // applies), built in the stage's code bytes, which both products have
+      // consumed; P_sp = p * s_out / s_in in the dense weights' (hi, -lo)
+      // layout, so that the output's s_in gives s_out * d.  Tile row of dim
+      // j: (j % 16) * 8 + j / 16, the rows of one m-tile's 8x8 blocks being
+      // consecutive; the two 16-byte halves of a row (tokens 0-7, 8-15)
+      // swap when bit 2 of the row is set, which keeps the 8x8 loads free
+      // of bank conflicts.
+      uint8_t* vd = const_cast<uint8_t*>(sK);
+      const uint32_t vd_sm = smem_u32(vd);
+      const int tt = lane & 15, hf = lane >> 4;  // scatter: token tt, slots 8 hf .. 8 hf + 7
+      const int kap = tok_perm(tt);              // its k position in the products
+      const int mq = lane >> 3, i8 = lane & 7;   // 8x8 load: block mq, row i8
+#pragma unroll
+      for (int sub = 0; sub < NS; ++sub) {
+        uint32_t bs0[NP], bs1[NP];
+#pragma unroll
+        for (int nb = 0; nb < NP; ++nb) {
+          uint32_t r0, r1;
+          split_pair(p_keep[sub][slot_of(nb)][0] * v_ratio, p_keep[sub][slot_of(nb)][1] * v_ratio,
+                     r0, r1);
+          bs0[nb] = transpose8x8(r0);
+          bs1[nb] = transpose8x8(r1);
+        }
+        __syncwarp();  // every lane is done reading the tile (codes or slots)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          reinterpret_cast<uint4*>(vd)[i * 32 + lane] = make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
+        {
+          const uint4 w = *reinterpret_cast<const uint4*>(sVm + (sub * kTile + tt) * C::MB +
+                                                          hf * 16);
+          const uint32_t sw[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t u = (k & 1) ? (sw[k >> 1] >> 16) : sw[k >> 1];
+            const int d = (int)(int8_t)(uint8_t)(u >> 8);
+            if (d != 0) {
+              const uint32_t j = u & 0x7Fu;
+              const uint32_t row = (j & 15u) * 8u + (j >> 4);
+              const uint32_t half16 = (uint32_t)(kap >> 3) ^ ((j >> 6) & 1u);
+              const float e = (j & 1u) ? 0x1p-20f : 0x1p-24f;
+              *reinterpret_cast<__half*>(vd + row * 32u + half16 * 16u + (kap & 7) * 2) =
+                  __float2half_rn((float)d * e);
+            }
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const uint32_t row = (uint32_t)((mt + 8 * (mq & 1)) * 8 + i8);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4(vd_sm + row * 32u + ((uint32_t)((mq >> 1) ^ ((i8 >> 2) & 1)) << 4), a0, a1,
+                      a2, a3);
+#pragma unroll
+          for (int nb = 0; nb < NP; ++nb) mma_f16(o_acc[nb][mt], a0, a1, a2, a3, bs0[nb], bs1[nb]);
+        }
+      }
+      // the tile was written through the generic proxy; the ring's next bulk
+      // copy into this stage comes through the async proxy
+      fence_proxy_async_smem();
+    }
   };
 
   for (int i = 0; i < n_tiles; ++i) {
@@ -725,7 +864,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
     const uint8_t* sV = sK + C::STOK * C::RB;
     const uint8_t* sKm = sK + 2 * C::STOK * C::RB;
     const uint8_t* sVm = sKm + C::STOK * C::MBK;
-    if constexpr (BITS != 16 && !KPC) {
+    if constexpr (BITS != 16 && !KPC && !OAK) {
       if (i == patch_i) {
         // the new token's row, from the quantized copy in shared memory
         uint32_t* dK = reinterpret_cast<uint32_t*>(stages + st * C::STAGE + patch_row * C::RB);
@@ -822,10 +961,13 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
         for (int mt = 0; mt < 8; ++mt) {
           // hi column minus the negated-remainder column, then undo the
           // subnormal code scale 2^(e - 24) of the row's dim
+          // (Oaken: the plane's z_in times the weights' sum, and its s_in)
           const float f0 = pow2f(24 - XP::exp(mt % XP::kOut)) * C::INV_PSCALE;
           const float f1 = pow2f(24 - XP::exp((mt + 8) % XP::kOut)) * C::INV_PSCALE;
-          oh[mt] = fmaf(o_acc[nb][mt][0] - o_acc[nb][mt][1], f0, -corr[nb]);
-          oh[mt + 8] = fmaf(o_acc[nb][mt][2] - o_acc[nb][mt][3], f1, -corr[nb]);
+          const float cz = OAK ? vz_in * l_part[slot_of(nb)] : corr[nb];
+          const float osc = OAK ? vs_in : 1.f;
+          oh[mt] = osc * fmaf(o_acc[nb][mt][0] - o_acc[nb][mt][1], f0, -cz);
+          oh[mt + 8] = osc * fmaf(o_acc[nb][mt][2] - o_acc[nb][mt][3], f1, -cz);
         }
       }
     }
@@ -840,9 +982,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   if (t == 0) release_counters(counters);
 }
 
-template <int BITS, int GE, int GR, bool KPC, int OCC = 0>
+template <int BITS, int GE, int GR, bool KPC>
 cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
-  using C = TmCfg<BITS, GE, GR, KPC, OCC>;
+  using C = TmCfg<BITS, GE, GR, KPC>;
   // the shared-memory opt-in is a per-device function attribute: set it once
   // per device (bit i of the mask = device i)
   static std::atomic<unsigned long long> attr_set{0};
@@ -850,7 +992,7 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tm_kernel<BITS, GE, GR, KPC, OCC>,
+    cudaError_t e = cudaFuncSetAttribute(decode_tm_kernel<BITS, GE, GR, KPC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
@@ -859,20 +1001,13 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   const long long units = (long long)seg.n_split * a.kv_heads * a.batch;
   const long long slots = (long long)seg.sms * C::MIN_CTAS;  // one wave of persistent CTAs
   const unsigned grid = (unsigned)(units < slots ? units : slots);
-  decode_tm_kernel<BITS, GE, GR, KPC, OCC><<<grid, kWarps * 32, C::SMEM, s>>>(P);
+  decode_tm_kernel<BITS, GE, GR, KPC><<<grid, kWarps * 32, C::SMEM, s>>>(P);
   return cudaGetLastError();
 }
 
 // Per-channel K (G is V's group size): the (bits, G, g) whose QK columns
 // give lane tig head tig % g in two columns (see TmCfg).
 #define KVQ_TM_KPC_FORMATS(X) X(4, 64, 4) X(8, 128, 1) X(4, 128, 4) X(4, 128, 1)
-
-// Formats also built at five CTAs per SM (two stages per warp): with more
-// units than one wave of those CTAs, the finer split shortens the last
-// wave by more than the shallower copy pipeline costs; with one wave or
-// less the three-stage kernel is faster.
-#define KVQ_TM_WIDE_FORMATS(X) X(4, 64, 4)
-constexpr int kWideCtas = 5;
 
 // Every (bits, G, g) with NG * g <= 8 that the cache formats allow.
 #define KVQ_TM_FORMATS(X)                                              \
@@ -889,7 +1024,8 @@ constexpr int kWideCtas = 5;
   X(kSym8, 128, 1) X(kSym8, 128, 2) X(kSym8, 128, 4) X(kSym8, 128, 8)  \
   X(kSym8, 64, 1) X(kSym8, 64, 2) X(kSym8, 64, 4) X(kSym8, 32, 1) X(kSym8, 32, 2) \
   X(kE5M2, 128, 1) X(kE5M2, 128, 2) X(kE5M2, 128, 4) X(kE5M2, 128, 8)  \
-  X(kE5M2, 64, 1) X(kE5M2, 64, 2) X(kE5M2, 64, 4) X(kE5M2, 32, 1) X(kE5M2, 32, 2)
+  X(kE5M2, 64, 1) X(kE5M2, 64, 2) X(kE5M2, 64, 4) X(kE5M2, 32, 1) X(kE5M2, 32, 2) \
+  X(kOaken, 128, 1) X(kOaken, 128, 2) X(kOaken, 128, 4) X(kOaken, 128, 8)
 
 }  // namespace
 
@@ -920,25 +1056,9 @@ int decode_tm_ctas_per_sm(int bits, int group, int group_ratio, bool kpc) {
   return 0;
 }
 
-int decode_tm_wide_ctas_per_sm(int bits, int group, int group_ratio, bool kpc) {
-  if (kpc) return 0;
-#define KVQ_X(B, G_, R) \
-  if (bits == B && group == G_ && group_ratio == R) return TmCfg<B, G_, R, false, kWideCtas>::MIN_CTAS;
-  KVQ_TM_WIDE_FORMATS(KVQ_X)
-#undef KVQ_X
-  return 0;
-}
-
 cudaError_t launch_decode_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   const int bits = seg.bits, group = (seg.bits == 16) ? kHeadDim : seg.group;
   const int g = a.group_ratio;
-  if (seg.wide) {
-#define KVQ_X(B, G_, R) \
-  if (!seg.k_channels && bits == B && group == G_ && g == R) return launch_tm<B, G_, R, false, kWideCtas>(a, seg, s);
-    KVQ_TM_WIDE_FORMATS(KVQ_X)
-#undef KVQ_X
-    return cudaErrorInvalidValue;
-  }
 #define KVQ_X(B, G_, R) \
   if (bits == B && group == G_ && g == R) return launch_tm<B, G_, R, false>(a, seg, s);
 #define KVQ_XK(B, G_, R) \

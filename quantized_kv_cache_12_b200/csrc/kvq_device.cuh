@@ -108,6 +108,16 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Four 8x8 tiles of 16-bit elements from shared memory, in the register
+// layout of an m16n8k16 A operand: lane i supplies the address of row i % 8
+// of tile i / 8 (16 contiguous bytes); tile t lands in r[t].
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                            uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 // ---------------------------------------------------------------- bit casts
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
   return *reinterpret_cast<uint32_t*>(&h);
@@ -289,6 +299,10 @@ struct WordPairs<kE4M3> {
   }
 };
 
+// The Oaken codec's dense part is 4-bit codes packed like INT4.
+template <>
+struct WordPairs<kOaken> : WordPairs<4> {};
+
 // Pairs across two tokens (V side): words a (token A) and b (token B) hold
 // the same dims; out[i] = half2(code_A[dim i], code_B[dim i]) for the dims of
 // the word in order, with the subnormal exponent exp(i).
@@ -313,6 +327,9 @@ struct CrossPairs<4> {
   }
   __host__ __device__ static constexpr int exp(int i) { return 4 * (i & 1); }
 };
+
+template <>
+struct CrossPairs<kOaken> : CrossPairs<4> {};
 
 template <>
 struct CrossPairs<2> {

@@ -39,10 +39,9 @@ struct SegView {
   int32_t bits;
   int32_t group;
   int32_t max_tokens;
-  int32_t n_split;       // units per (sequence, KV head): 16-row and Oaken kernels
+  int32_t n_split;       // units (splits) per (sequence, KV head)
   int32_t part_base;     // index of this segment's first partial slot
   int32_t k_channels;    // K grouped per channel over kChannelBlock-token blocks
-  int32_t wide;          // run the five-CTAs-per-SM build of the format
   int32_t sms;           // streaming multiprocessors of the device
   OakenParams k_oaken, v_oaken;  // bits == kOaken: the planes' parameters
 };
@@ -104,17 +103,12 @@ int decode_ctas_per_sm(int bits, int group, int group_ratio, bool kpc = false);
 // the tokens-on-M kernel (kvq_decode_tm.cu): formats with NG * g <= 8
 bool decode_tm_supported(int bits, int group, int group_ratio, bool kpc = false);
 int decode_tm_ctas_per_sm(int bits, int group, int group_ratio, bool kpc = false);
-// CTAs per SM of the format's five-CTA build, 0 where it has none
-int decode_tm_wide_ctas_per_sm(int bits, int group, int group_ratio, bool kpc = false);
 cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s);
 // the Oaken codec (kvq_oaken.cu): quantize-on-write of both planes (and the
 // seq_lens advance), and its decode-attention kernel (g = 1, 2, 4, 8)
 cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s);
-bool decode_oaken_supported(int group_ratio);
-int decode_oaken_ctas_per_sm(int group_ratio);
-cudaError_t launch_decode_oaken(const DecodeArgs& a, const SegView& seg, cudaStream_t s);
 // kvq_decode_attention's argument checks only: KVQ_OK means a call with the
 // same arguments enqueues its kernels (kvq_abi.cu)
 kvq_status decode_check_args(const kvq_cache* segs, int32_t n_segs, const void* q,

@@ -433,28 +433,39 @@ def _plan_parts(kvq, B, H, Hq, max_tokens, hint, bits=4, group=64, fmt=0):
 
 
 def test_split_plan_per_workload(kvq):
-    """The host split plan (a wave model over the device's SMs x the format's
-    CTAs per SM -- 148 on a host without that device -- plus the five-CTA
-    build of INT4 G64 g = 4 where its own plan spans more than one wave), at
-    the benchmark's shapes: the partials per (sequence, query head)."""
+    """The host split plan at the benchmark's shapes (148 SMs on a host
+    without a device), as partials per (sequence, query head).  The plan
+    minimises the busiest SM's time: u = ceil(units / SMs) units in rounds of
+    up to C (the format's CTAs per SM), a round of c < 3 units at c/3 of the
+    SM's rate, each unit (tokens rounded up to 32) + 300 tokens of fixed cost:
+      Llama-3 GQA INT4 (256 pairs, L 8292, C 4): 4 splits, u = 7, rounds 4 + 3,
+        7 x (2080 + 300) = 16660; 2 splits cost 4 x 4460 = 17840, 6 splits
+        11 x 1708 = 18788, 5 splits (4 + 4 + a lone unit) 11 x 1964 = 21604.
+      half that batch (128 pairs): 3 splits, u = 3, 3 x 3084 = 9252 against
+        4 x 2380 = 9520 for 4.
+      long context (8 pairs, L 131328): 55 splits, u = 3, 3 x (2400 + 300) =
+        8100 against 4 x (1792 + 300) = 8368 for 74.
+      Llama-2 MHA INT8 (512 pairs, L 4196, C 3): 4 splits, u = 14, rounds
+        3 + 3 + 3 + 3 + 2 (at 2/3 rate), 15 x 1356 = 20340 against
+        12 x 1708 = 20496 for 3.
+      Oaken codec (256 pairs, L 8192, C 3): 5 splits, u = 9, 9 x 1964 =
+        17676 against 6 x 3052 = 18312 for 3."""
     parts = lambda *a, **k: _plan_parts(kvq, *a, **k)  # noqa: E731
-    assert parts(32, 8, 32, 8320, 8292) == 5        # Llama-3 GQA INT4: five-CTA build, 1.7 waves
-    assert parts(16, 8, 32, 8320, 8292) == 9        # half the batch: the four-CTA build, 2 waves
-    assert parts(1, 8, 32, 131392, 131328) == 74    # long context: one wave of the four-CTA build
-    assert parts(16, 32, 32, 4224, 4196, bits=8, group=128) == 4   # Llama-2 MHA: 2048 units
+    assert parts(32, 8, 32, 8320, 8292) == 4
+    assert parts(16, 8, 32, 8320, 8292) == 3
+    assert parts(1, 8, 32, 131392, 131328) == 55
+    assert parts(16, 32, 32, 4224, 4196, bits=8, group=128) == 4
     assert parts(32, 8, 32, 8320, 8192, group=128, fmt=kvq.KVQ_FMT_OAKEN) == 5
 
 
 def test_split_plan_follows_the_sm_count(tmp_path):
     """The plan reads the device's SM count; KVQ_NUM_SMS overrides it (read
     once per process, so the check runs in a child process).  With 74 SMs,
-    worked by hand from the wave model cost ceil(units / slots) x (tokens per
-    unit + 200): Llama-3 GQA INT4 (256 pairs) takes the five-CTA build (370
-    slots) at four splits -- cost 3 waves x (2080 + 200) = 6840 against 8520
-    for one split and 7080 for seven -- as its 1024 units exceed one wave;
-    the long context (8 pairs, four-CTA build, 296 slots) takes 37 splits,
-    the most that fit one wave (cost 3752 against 3984 for 74), and the
-    five-CTA plan (46 splits, 368 units) fits one wave, so it is not taken."""
+    worked by hand from the same cost: Llama-3 GQA INT4 (256 pairs, 4 CTAs
+    per SM) takes 2 splits -- u = 7, rounds 4 + 3, 7 x 4460 = 31220, against
+    4 x 8620 = 34480 for one split and (12 + 3) x 2380 = 35700 for four --
+    and the long context (8 pairs) takes 37 splits -- u = 4, 4 x 3852 =
+    15408, against (4 + 3) x 2700 = 18900 for 55."""
     code = (
         "import sys; sys.path.insert(0, %r)\n"
         "from quantized_kv_cache_12_b200 import kvq\n"
@@ -464,4 +475,4 @@ def test_split_plan_follows_the_sm_count(tmp_path):
     env = dict(os.environ, KVQ_NUM_SMS="74")
     out = subprocess.run([sys.executable, "-c", code], env=env, cwd=ROOT, check=True,
                          capture_output=True, text=True).stdout.split()
-    assert out == ["4", "37"]
+    assert out == ["2", "37"]
