@@ -18,9 +18,13 @@
 // outlier the dense part is its threshold and the slot adds the shift.
 //
 // Kernels:
-//   oaken_quantize_kernel: quantize-on-write, half a warp per row (8 dims a
-//     lane), the outliers' slots placed by a shuffle scan of the lanes'
-//     counts.  HBM-bound: 256 B read and 96 B written per row.
+//   oaken_quantize_kernel: quantize-on-write of a few rows per sequence
+//     (the decode-step append), half a warp per row (8 dims a lane), the
+//     outliers' slots placed by a shuffle scan of the lanes' counts.
+//   oaken_bulk_kernel: the prefill, on the bulk quantizer's load ring (four
+//     lanes per row, 32 dims a lane), dense codes branch-free, outliers in
+//     a compact per-lane loop.  HBM-bound: 256 B read and 96 B written per
+//     row.
 //   The decode attention over these planes is the tokens-on-M kernel's
 //     (kvq_decode_tm.cu): the dense codes through the tensor cores like
 //     INT4 with the plane's one (s, z), the K slots as per-token score
@@ -30,6 +34,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include "kvq_bulk.cuh"
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 #include "kvq_quant_core.cuh"
@@ -122,6 +127,104 @@ __global__ void __launch_bounds__(256) oaken_quantize_kernel(const QuantArgs a) 
   }
 }
 
+// Bulk (prefill) encoder: the bulk ring's units (kUnitRows consecutive rows
+// of one (side, sequence, KV head) plane row, 4 lanes per row, 32
+// consecutive dims a lane).  The dense codes of all 32 values are computed
+// branch-free on clamped values, rint(clamp(v, T_lo, T_hi) / s_in) + z_in
+// (the thresholds divide to exactly -z_in and 15 - z_in, so an outlier gets
+// its threshold's code and an inner value its own), with packed f32x2
+// arithmetic; the clamped values also flag the outliers.  Each lane then
+// settles its own outliers in a compact loop (dim order, after the row's
+// earlier lanes: an exclusive scan of the four lanes' counts), writing them
+// into the warp's slot rows in shared memory, whose zeros stand for the
+// empty slots; the rows go out as 8-byte stores.
+using OakDst = BulkDst<kRowBytes, kSlotBytes>;
+
+__device__ __forceinline__ void oaken_work(const QuantArgs& a, int li, int ri, const OakDst& c,
+                                           const uint32_t (&roff)[kBulkNV / 8],
+                                           const uint8_t* slot, uint16_t* sbuf) {
+  static_assert(kBulkNV == 32 && kBulkLanes == 4 && kSlots == 16, "lane and slot layout");
+  const bool in = c.p.t < a.n_new;
+  const OakenParams& p = c.p.side ? a.v_oaken : a.k_oaken;
+  uint4 raw[kBulkNV / 8];
+#pragma unroll
+  for (int k = 0; k < kBulkNV / 8; ++k)
+    raw[k] = in ? *reinterpret_cast<const uint4*>(slot + roff[k]) : make_uint4(0u, 0u, 0u, 0u);
+  const __half2* h2 = reinterpret_cast<const __half2*>(&raw[0]);
+  float x[kBulkNV];
+#pragma unroll
+  for (int i = 0; i < kBulkNV / 2; ++i) {
+    const float2 f = __half22float2(h2[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t r2 = f2_pack(p.r_in, p.r_in), nd2 = f2_pack(-p.s_in, -p.s_in);
+  const uint64_t m2 = f2_pack(kMagic, kMagic);
+  const float zm = p.z - kMagic;
+  const uint64_t zm2 = f2_pack(zm, zm);
+  uint64_t t[kBulkNV / 2];  // pair i: elements i and i + 16
+  uint32_t omask = 0;       // bit j: element j is an outlier
+#pragma unroll
+  for (int i = 0; i < kBulkNV / 2; ++i) {
+    const float v0 = x[i], v1 = x[i + kBulkNV / 2];
+    const float c0 = fminf(fmaxf(v0, p.t_lo), p.t_hi), c1 = fminf(fmaxf(v1, p.t_lo), p.t_hi);
+    omask |= ((uint32_t)(c0 != v0) << i) | ((uint32_t)(c1 != v1) << (i + kBulkNV / 2));
+    // quotients in [-z_in, 15 - z_in]: (q + M) + (z_in - M) is rint(q) + z_in
+    t[i] = f2_add(f2_add(div_rn2(f2_pack(c0, c1), nd2, r2), m2), zm2);
+  }
+  uint32_t cw[code_words<4, kBulkNV>()];
+  pack_codes<4, kBulkNV>(t, cw);
+  if (!in) omask = 0;
+  // slot positions: exclusive scan of the row's four lanes' counts
+  const int cnt = __popc(omask);
+  int incl = cnt;
+  {
+    const int u1 = __shfl_up_sync(0xffffffffu, incl, 1, kBulkLanes);
+    if (li >= 1) incl += u1;
+    const int u2 = __shfl_up_sync(0xffffffffu, incl, 2, kBulkLanes);
+    if (li >= 2) incl += u2;
+  }
+  uint16_t* srow = sbuf + ri * kSlots;
+  reinterpret_cast<uint2*>(srow)[li] = make_uint2(0u, 0u);  // slots 4 li .. 4 li + 3
+  __syncwarp();
+  int k = incl - cnt;
+  while (omask != 0u) {
+    const int j = __ffs(omask) - 1;
+    omask &= omask - 1u;
+    if (k < kSlots) {
+      const float v = __half2float(*reinterpret_cast<const __half*>(
+          slot + bulk_slot_off(ri, li * (kBulkNV / 8) + (j >> 3)) + (j & 7) * 2));
+      const bool hi = v > p.t_hi;
+      const float m = fminf(rintf(__fdiv_rn(hi ? v - p.t_hi : -(v - p.t_lo), p.s_out)), p.m_max);
+      const int d = hi ? (int)m : -(int)m;
+      srow[k] = (uint16_t)((uint32_t)(kBulkNV * li + j) | ((uint32_t)(uint8_t)(int8_t)d << 8));
+    }
+    ++k;
+  }
+  __syncwarp();
+  if (in && c.pos < a.max_tokens) {
+    *reinterpret_cast<uint4*>(c.codes) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    reinterpret_cast<uint2*>(c.meta)[li] = reinterpret_cast<const uint2*>(srow)[li];
+  }
+  __syncwarp();  // the slot rows are rewritten by the next unit
+}
+
+__global__ void __launch_bounds__(kBulkWarps * 32) oaken_bulk_kernel(const QuantArgs a,
+                                                                     int units_per_row,
+                                                                     int n_units,
+                                                                     int units_per_warp) {
+  __shared__ __align__(16) uint8_t ring[kBulkWarps][kBulkDepth][kUnitBytes];
+  __shared__ __align__(16) uint16_t sbuf[kBulkWarps][kUnitRows][kSlots];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int li = lane % kBulkLanes, ri = lane / kBulkLanes;
+  bulk_loop<OakDst>(a, units_per_row, n_units, units_per_warp, &ring[warp][0][0],
+                    [&](const OakDst& c, const uint32_t (&roff)[kBulkNV / 8],
+                        const uint8_t* slot) {
+                      oaken_work(a, li, ri, c, roff, slot, &sbuf[warp][0][0]);
+                    });
+}
+
 __global__ void oaken_advance_kernel(int32_t* seq_lens, int batch, int n_new, int max_tokens) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < batch) seq_lens[b] = min(seq_lens[b] + n_new, max_tokens);
@@ -142,12 +245,28 @@ OakenParams make_oaken_params(float s_in, int z_in, float s_out, int outer_bits)
 }
 
 cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s) {
-  const long long rows = 2LL * a.batch * a.kv_heads * a.n_new;
-  const long long blocks = (rows + 15) / 16;
-  const long long cap = (long long)device_sm_count() * 8;
-  const unsigned grid = (unsigned)(blocks < cap ? blocks : cap);
-  oaken_quantize_kernel<<<grid, 256, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (2LL * a.kv_heads * a.n_new <= 512) {
+    // a few rows per sequence (the decode-step append): half a warp per row
+    const long long rows = 2LL * a.batch * a.kv_heads * a.n_new;
+    const long long blocks = (rows + 15) / 16;
+    const long long cap = (long long)device_sm_count() * 8;
+    const unsigned grid = (unsigned)(blocks < cap ? blocks : cap);
+    oaken_quantize_kernel<<<grid, 256, 0, s>>>(a);
+  } else {
+    static int per_sm = 0;  // resident CTAs per SM of the bulk kernel
+    if (per_sm == 0) {
+      int r = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, oaken_bulk_kernel, kBulkWarps * 32, 0);
+      if (e != cudaSuccess) return e;
+      per_sm = r > 0 ? r : 1;
+    }
+    BulkShape sh;
+    if (!bulk_shape(a, per_sm, &sh)) return cudaErrorInvalidValue;
+    oaken_bulk_kernel<<<sh.blocks, kBulkWarps * 32, 0, s>>>(a, sh.units_per_row, sh.n_units,
+                                                            sh.per_warp);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess || !a.advance) return e;
   oaken_advance_kernel<<<(a.batch + 127) / 128, 128, 0, s>>>(a.seq_lens, a.batch, a.n_new,
                                                              a.max_tokens);
