@@ -519,30 +519,31 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
       const uint4* sl = reinterpret_cast<const uint4*>(sKm + lane * C::MB);
       const uint4 s0 = sl[0], s1 = sl[1];
       const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      float acc[GR];
+      if constexpr (GR % 2 == 0) {
+        // heads in pairs: packed f32x2 products
+        uint64_t acc[GR / 2];
 #pragma unroll
-      for (int h = 0; h < GR; ++h) acc[h] = 0.f;
+        for (int h = 0; h < GR / 2; ++h) acc[h] = 0ull;
 #pragma unroll
-      for (int k = 0; k < KVQ_OAKEN_SLOTS; ++k) {
-        const uint32_t u = (k & 1) ? (sw[k >> 1] >> 16) : sw[k >> 1];
-        const float d = (float)(int)(int8_t)(uint8_t)(u >> 8);
-        const float* tr = otab + (u & 0x7Fu) * GR;
-        if constexpr (GR % 4 == 0) {
+        for (int k = 0; k < KVQ_OAKEN_SLOTS; ++k) {
+          const uint32_t u = (k & 1) ? (sw[k >> 1] >> 16) : sw[k >> 1];
+          const float d = (float)(int)(int8_t)(uint8_t)(u >> 8);
+          const uint64_t d2 = f2_pack(d, d);
+          const uint64_t* tr = reinterpret_cast<const uint64_t*>(otab + (u & 0x7Fu) * GR);
 #pragma unroll
-          for (int h = 0; h < GR; h += 4) {
-            const float4 tv = *reinterpret_cast<const float4*>(tr + h);
-            acc[h] = fmaf(d, tv.x, acc[h]);
-            acc[h + 1] = fmaf(d, tv.y, acc[h + 1]);
-            acc[h + 2] = fmaf(d, tv.z, acc[h + 2]);
-            acc[h + 3] = fmaf(d, tv.w, acc[h + 3]);
-          }
-        } else {
-#pragma unroll
-          for (int h = 0; h < GR; ++h) acc[h] = fmaf(d, tr[h], acc[h]);
+          for (int h = 0; h < GR / 2; ++h) acc[h] = f2_fma(d2, tr[h], acc[h]);
         }
-      }
 #pragma unroll
-      for (int h = 0; h < GR; ++h) spx[lane * GR + h] = acc[h];
+        for (int h = 0; h < GR / 2; ++h) reinterpret_cast<uint64_t*>(spx + lane * GR)[h] = acc[h];
+      } else {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < KVQ_OAKEN_SLOTS; ++k) {
+          const uint32_t u = (k & 1) ? (sw[k >> 1] >> 16) : sw[k >> 1];
+          acc = fmaf((float)(int)(int8_t)(uint8_t)(u >> 8), otab[u & 0x7Fu], acc);
+        }
+        spx[lane] = acc;
+      }
       __syncwarp();
     }
     auto valid = [&](int tok) { return FULL || tok < n_valid; };  // tok: 0 .. STOK-1
@@ -804,6 +805,11 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
       const int tt = lane & 15, hf = lane >> 4;  // scatter: token tt, slots 8 hf .. 8 hf + 7
       const int kap = tok_perm(tt);              // its k position in the products
       const int mq = lane >> 3, i8 = lane & 7;   // 8x8 load: block mq, row i8
+      // an empty slot (0: dim 0, shift 0) must not overwrite a real outlier
+      // at dim 0 of the same token: its store goes to a spare byte pair in
+      // the consumed K slots
+      __half* spare = reinterpret_cast<__half*>(const_cast<uint8_t*>(sKm)) + lane;
+      const uint32_t kap_bits = ((uint32_t)(kap >> 3) << 4) | ((uint32_t)(kap & 7) << 1);
 #pragma unroll
       for (int sub = 0; sub < NS; ++sub) {
         uint32_t bs0[NP], bs1[NP];
@@ -828,14 +834,14 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
           for (int k = 0; k < 8; ++k) {
             const uint32_t u = (k & 1) ? (sw[k >> 1] >> 16) : sw[k >> 1];
             const int d = (int)(int8_t)(uint8_t)(u >> 8);
-            if (d != 0) {
-              const uint32_t j = u & 0x7Fu;
-              const uint32_t row = (j & 15u) * 8u + (j >> 4);
-              const uint32_t half16 = (uint32_t)(kap >> 3) ^ ((j >> 6) & 1u);
-              const float e = (j & 1u) ? 0x1p-20f : 0x1p-24f;
-              *reinterpret_cast<__half*>(vd + row * 32u + half16 * 16u + (kap & 7) * 2) =
-                  __float2half_rn((float)d * e);
-            }
+            const uint32_t j = u & 0x7Fu;
+            // byte offset: row (j % 16) * 8 + j / 16 of 32 bytes, the row's
+            // half for the token (swapped when bit 2 of the row, j's bit 6,
+            // is set), the token's pair of bytes
+            const uint32_t off = ((j & 15u) << 8) | ((j >> 4) << 5) | (((j >> 2) & 16u) ^ kap_bits);
+            // d * 2^(e - 24): the exact fp16 integer d times a power of two
+            const __half hv = __hmul(__int2half_rn(d), __ushort_as_half((j & 1u) ? 0x0010 : 0x0001));
+            *(d != 0 ? reinterpret_cast<__half*>(vd + off) : spare) = hv;
           }
         }
         __syncwarp();

@@ -129,32 +129,65 @@ __global__ void __launch_bounds__(256) oaken_quantize_kernel(const QuantArgs a) 
 
 // Bulk (prefill) encoder: the bulk ring's units (kUnitRows consecutive rows
 // of one (side, sequence, KV head) plane row, 4 lanes per row, 32
-// consecutive dims a lane).  The dense codes of all 32 values are computed
-// branch-free on clamped values, rint(clamp(v, T_lo, T_hi) / s_in) + z_in
-// (the thresholds divide to exactly -z_in and 15 - z_in, so an outlier gets
-// its threshold's code and an inner value its own), with packed f32x2
-// arithmetic; the clamped values also flag the outliers.  Each lane then
-// settles its own outliers in a compact loop (dim order, after the row's
-// earlier lanes: an exclusive scan of the four lanes' counts), writing them
-// into the warp's slot rows in shared memory, whose zeros stand for the
-// empty slots; the rows go out as 8-byte stores.
+// consecutive dims a lane).  Per pair of fp16 values: clamped to the
+// thresholds in fp16 (th = the largest fp16 <= T_hi, tl = the smallest >=
+// T_lo: an fp16 value lies outside [T_lo, T_hi] exactly when it lies outside
+// [tl, th]), the clamp also flagging the outliers; then the dense code
+// rint(clamped / s_in) + z_in in packed f32x2 arithmetic -- an inner value
+// keeps its own code, and th and tl divide to within 15/1024 of 15 - z_in
+// and -z_in, so an outlier gets its threshold's code.  The outliers of the
+// warp's 8 rows are then listed in shared memory (each with its row, its
+// place among the row's outliers in dim order -- a scan of the row's lanes
+// -- and its dim) and settled 32 at a time across the whole warp; the slot
+// rows are assembled in shared memory, whose zeros stand for the empty
+// slots, and go out as 8-byte stores.
 using OakDst = BulkDst<kRowBytes, kSlotBytes>;
+constexpr int kOakList = kUnitRows * kSlots;  // outliers a unit can keep
 
-__device__ __forceinline__ void oaken_work(const QuantArgs& a, int li, int ri, const OakDst& c,
+struct OakUnitParams {
+  float s_in, r_in, z, t_lo, t_hi, s_out, m_max;
+  uint32_t tl2, th2;  // fp16 pairs (tl, tl) and (th, th)
+};
+
+__device__ __forceinline__ OakUnitParams oaken_unit_params(const OakenParams& p) {
+  OakUnitParams u;
+  u.s_in = p.s_in;
+  u.r_in = p.r_in;
+  u.z = p.z;
+  u.t_lo = p.t_lo;
+  u.t_hi = p.t_hi;
+  u.s_out = p.s_out;
+  u.m_max = p.m_max;
+  const __half tl = __float2half_ru(p.t_lo), th = __float2half_rd(p.t_hi);
+  u.tl2 = h2_as_u32(__halves2half2(tl, tl));
+  u.th2 = h2_as_u32(__halves2half2(th, th));
+  return u;
+}
+
+__device__ __forceinline__ void oaken_work(const QuantArgs& a, int lane, const OakDst& c,
                                            const uint32_t (&roff)[kBulkNV / 8],
-                                           const uint8_t* slot, uint16_t* sbuf) {
+                                           const uint8_t* slot, uint16_t* sbuf,
+                                           uint16_t* olist) {
   static_assert(kBulkNV == 32 && kBulkLanes == 4 && kSlots == 16, "lane and slot layout");
+  const int li = lane % kBulkLanes, ri = lane / kBulkLanes;
   const bool in = c.p.t < a.n_new;
-  const OakenParams& p = c.p.side ? a.v_oaken : a.k_oaken;
+  // the unit's plane parameters in registers (one side per unit)
+  const OakUnitParams p = oaken_unit_params(c.p.side ? a.v_oaken : a.k_oaken);
   uint4 raw[kBulkNV / 8];
 #pragma unroll
   for (int k = 0; k < kBulkNV / 8; ++k)
     raw[k] = in ? *reinterpret_cast<const uint4*>(slot + roff[k]) : make_uint4(0u, 0u, 0u, 0u);
-  const __half2* h2 = reinterpret_cast<const __half2*>(&raw[0]);
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&raw[0]);  // pair i: elements 2i, 2i + 1
+  // clamp in fp16; bit i / 16 + i of omask: element 2i / 2i + 1 is an outlier
+  // (reordered to dim order below)
   float x[kBulkNV];
+  uint32_t omask = 0;
 #pragma unroll
   for (int i = 0; i < kBulkNV / 2; ++i) {
-    const float2 f = __half22float2(h2[i]);
+    const __half2 h = u32_as_h2(w[i]);
+    const __half2 cl = __hmin2(__hmax2(h, u32_as_h2(p.tl2)), u32_as_h2(p.th2));
+    omask |= __hne2_mask(cl, h) & (0x00010001u << i);
+    const float2 f = __half22float2(cl);
     x[2 * i] = f.x;
     x[2 * i + 1] = f.y;
   }
@@ -163,20 +196,25 @@ __device__ __forceinline__ void oaken_work(const QuantArgs& a, int li, int ri, c
   const uint64_t m2 = f2_pack(kMagic, kMagic);
   const float zm = p.z - kMagic;
   const uint64_t zm2 = f2_pack(zm, zm);
-  uint64_t t[kBulkNV / 2];  // pair i: elements i and i + 16
-  uint32_t omask = 0;       // bit j: element j is an outlier
+  uint64_t t[kBulkNV / 2];  // pair i: elements i and i + 16 (the packing's order)
 #pragma unroll
-  for (int i = 0; i < kBulkNV / 2; ++i) {
-    const float v0 = x[i], v1 = x[i + kBulkNV / 2];
-    const float c0 = fminf(fmaxf(v0, p.t_lo), p.t_hi), c1 = fminf(fmaxf(v1, p.t_lo), p.t_hi);
-    omask |= ((uint32_t)(c0 != v0) << i) | ((uint32_t)(c1 != v1) << (i + kBulkNV / 2));
-    // quotients in [-z_in, 15 - z_in]: (q + M) + (z_in - M) is rint(q) + z_in
-    t[i] = f2_add(f2_add(div_rn2(f2_pack(c0, c1), nd2, r2), m2), zm2);
-  }
+  for (int i = 0; i < kBulkNV / 2; ++i)
+    // quotients within [-z_in, 15 - z_in]: (q + M) + (z_in - M) is rint(q) + z_in
+    t[i] = f2_add(f2_add(div_rn2(f2_pack(x[i], x[i + kBulkNV / 2]), nd2, r2), m2), zm2);
   uint32_t cw[code_words<4, kBulkNV>()];
   pack_codes<4, kBulkNV>(t, cw);
   if (!in) omask = 0;
-  // slot positions: exclusive scan of the row's four lanes' counts
+  // bit j: element j (dim 32 li + j) is an outlier -- the even elements'
+  // bits spread to the even positions, the odd ones' to the odd
+  auto spread = [](uint32_t v) {  // bit i of a 16-bit value to bit 2i
+    v = (v | (v << 8)) & 0x00FF00FFu;
+    v = (v | (v << 4)) & 0x0F0F0F0Fu;
+    v = (v | (v << 2)) & 0x33333333u;
+    return (v | (v << 1)) & 0x55555555u;
+  };
+  omask = spread(omask & 0xFFFFu) | (spread(omask >> 16) << 1);
+  // places among the row's outliers (dim order: lanes in order); the first
+  // kSlots are kept, and the kept ones get places in the warp's list
   const int cnt = __popc(omask);
   int incl = cnt;
   {
@@ -185,29 +223,45 @@ __device__ __forceinline__ void oaken_work(const QuantArgs& a, int li, int ri, c
     const int u2 = __shfl_up_sync(0xffffffffu, incl, 2, kBulkLanes);
     if (li >= 2) incl += u2;
   }
+  const int kept = max(0, min(cnt, kSlots - (incl - cnt)));
+  int wincl = kept;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, wincl, off);
+    if (lane >= off) wincl += u;
+  }
+  const int total = __shfl_sync(0xffffffffu, wincl, 31);
   uint16_t* srow = sbuf + ri * kSlots;
   reinterpret_cast<uint2*>(srow)[li] = make_uint2(0u, 0u);  // slots 4 li .. 4 li + 3
-  __syncwarp();
-  int k = incl - cnt;
-  while (omask != 0u) {
-    const int j = __ffs(omask) - 1;
-    omask &= omask - 1u;
-    if (k < kSlots) {
-      const float v = __half2float(*reinterpret_cast<const __half*>(
-          slot + bulk_slot_off(ri, li * (kBulkNV / 8) + (j >> 3)) + (j & 7) * 2));
-      const bool hi = v > p.t_hi;
-      const float m = fminf(rintf(__fdiv_rn(hi ? v - p.t_hi : -(v - p.t_lo), p.s_out)), p.m_max);
-      const int d = hi ? (int)m : -(int)m;
-      srow[k] = (uint16_t)((uint32_t)(kBulkNV * li + j) | ((uint32_t)(uint8_t)(int8_t)d << 8));
+  // list entry: row (bits 0-2), place in the row (bits 3-7), dim (bits 8-14);
+  // outliers past the row's kSlots-th are dropped (their dense code is
+  // their threshold's)
+  {
+    int k = incl - cnt, e = wincl - kept;
+    uint32_t m = omask;
+    for (int n = 0; n < kept; ++n) {
+      const int j = __ffs(m) - 1;
+      m &= m - 1u;
+      olist[e++] = (uint16_t)(ri | (k++ << 3) | ((kBulkNV * li + j) << 8));
     }
-    ++k;
+  }
+  __syncwarp();
+  for (int e = lane; e < total; e += 32) {
+    const uint32_t en = olist[e];
+    const int r = en & 7, k = (en >> 3) & 31, dim = (int)(en >> 8);
+    const float v = __half2float(
+        *reinterpret_cast<const __half*>(slot + bulk_slot_off(r, dim >> 3) + (dim & 7) * 2));
+    const bool hi = v > p.t_hi;
+    const float mq = fminf(rintf(__fdiv_rn(hi ? v - p.t_hi : -(v - p.t_lo), p.s_out)), p.m_max);
+    const int d = hi ? (int)mq : -(int)mq;
+    sbuf[r * kSlots + k] = (uint16_t)((uint32_t)dim | ((uint32_t)(uint8_t)(int8_t)d << 8));
   }
   __syncwarp();
   if (in && c.pos < a.max_tokens) {
     *reinterpret_cast<uint4*>(c.codes) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
     reinterpret_cast<uint2*>(c.meta)[li] = reinterpret_cast<const uint2*>(srow)[li];
   }
-  __syncwarp();  // the slot rows are rewritten by the next unit
+  __syncwarp();  // the slot rows and the list are rewritten by the next unit
 }
 
 __global__ void __launch_bounds__(kBulkWarps * 32) oaken_bulk_kernel(const QuantArgs a,
@@ -216,12 +270,12 @@ __global__ void __launch_bounds__(kBulkWarps * 32) oaken_bulk_kernel(const Quant
                                                                      int units_per_warp) {
   __shared__ __align__(16) uint8_t ring[kBulkWarps][kBulkDepth][kUnitBytes];
   __shared__ __align__(16) uint16_t sbuf[kBulkWarps][kUnitRows][kSlots];
+  __shared__ __align__(16) uint16_t olist[kBulkWarps][kOakList];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int li = lane % kBulkLanes, ri = lane / kBulkLanes;
   bulk_loop<OakDst>(a, units_per_row, n_units, units_per_warp, &ring[warp][0][0],
                     [&](const OakDst& c, const uint32_t (&roff)[kBulkNV / 8],
                         const uint8_t* slot) {
-                      oaken_work(a, li, ri, c, roff, slot, &sbuf[warp][0][0]);
+                      oaken_work(a, lane, c, roff, slot, &sbuf[warp][0][0], &olist[warp][0]);
                     });
 }
 
