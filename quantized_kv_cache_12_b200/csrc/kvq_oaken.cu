@@ -300,7 +300,7 @@ OakenParams make_oaken_params(float s_in, int z_in, float s_out, int outer_bits)
 
 cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s) {
   cudaError_t e;
-  if (2LL * a.kv_heads * a.n_new <= 512) {
+  if (a.n_new < kUnitRows) {
     // a few rows per sequence (the decode-step append): half a warp per row
     const long long rows = 2LL * a.batch * a.kv_heads * a.n_new;
     const long long blocks = (rows + 15) / 16;

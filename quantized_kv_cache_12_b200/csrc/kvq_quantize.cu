@@ -233,8 +233,9 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
     }
   }
   const int rows_per_seq = (2 - a.side0) * a.kv_heads * a.n_new;
-  if (rows_per_seq <= 512) {
-    // one pass over the sequence's rows when they fit in one CTA
+  if (a.n_new < kUnitRows || rows_per_seq <= 64) {
+    // a few tokens per sequence (the decode-step append): one CTA per
+    // sequence, one pass when its rows fit
     int threads = ((rows_per_seq * 16 + 63) / 64) * 64;
     if (threads > 1024) threads = 1024;
     quantize_append_kernel<BITS, G, BF><<<a.batch, threads, 0, s>>>(a);

@@ -133,7 +133,7 @@ def _sweep_rows(fmt):
                                         (8, 128, "sym8")])
 def test_bf16_scale_sweep_bulk_kernel(kvq, bits, G, fmt):
     rows = _sweep_rows(fmt)
-    n, H = rows.shape[0], 4   # 4 heads x 2 sides x n rows > 512: the bulk kernel
+    n, H = rows.shape[0], 4   # n >= 8 tokens per (sequence, head): the bulk kernel
     k = torch.stack([rows] * H).view(1, H, n, 128).to(DEV).contiguous()
     v = torch.stack([rows.flip(0)] * H).view(1, H, n, 128).to(DEV).contiguous()
     k[0, 1] = -k[0, 1]
@@ -145,8 +145,8 @@ def test_bf16_scale_sweep_bulk_kernel(kvq, bits, G, fmt):
     # the same rows, a few at a time, through the append kernel
     c2 = _alloc(kvq, 1, H, cap, bits, G, fmt)
     c2.seq_lens.zero_()
-    for i in range(0, n, 16):
-        m = min(16, n - i)
+    for i in range(0, n, 4):   # fewer than 8 tokens a call: the append kernel
+        m = min(4, n - i)
         kvq.kvq_quantize_append(c2, k[:, :, i:i + m].contiguous(), v[:, :, i:i + m].contiguous(),
                                 m, advance_seq_lens=True)
     assert torch.equal(c2.k_codes[:, :, :n], c.k_codes[:, :, :n])

@@ -165,7 +165,7 @@ def test_prefill_full_size_long_context_sampled(kvq):
         assert np.array_equal(_meta_bits(meta[0, h, t]), em)
 
 
-# ---- the bulk (prefill) kernel: more than 512 rows per sequence
+# ---- the bulk (prefill) kernel: eight or more tokens per sequence
 
 
 def _alloc_fmt(kvq, B, H, max_tokens, bits, G, fmt):
@@ -225,7 +225,7 @@ def test_bulk_kernel_scale_sweep_and_adversarial(kvq, bits, G, fmt):
             x = rng.standard_normal(128) * 2.0 ** e + off * 2.0 ** max(e, 0)
             rows.append(np.clip(x, -65504, 65504).astype(np.float16))
     rows = np.concatenate([np.stack(rows), _adversarial_rows()])
-    n = rows.shape[0]  # rows per head: 4 heads x 2 sides x n > 512 rows per sequence
+    n = rows.shape[0]  # tokens per (sequence, head): the bulk kernel
     H = 4
     k = torch.from_numpy(np.stack([rows] * H)).to(DEV).view(1, H, n, 128).contiguous()
     v = torch.from_numpy(np.stack([rows[::-1]] * H)).to(DEV).view(1, H, n, 128).contiguous()

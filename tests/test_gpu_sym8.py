@@ -44,7 +44,7 @@ def _adversarial(k, v):
     v[1, 0, 5] = -0.0
 
 
-@pytest.mark.parametrize("H,T", [(2, 41), (4, 77)])  # 164 rows: append kernel; 616: bulk
+@pytest.mark.parametrize("H,T", [(2, 7), (4, 77)])  # under 8 tokens: append kernel; 77: bulk
 @pytest.mark.parametrize("G", [32, 64, 128])
 def test_quantize_bit_exact(kvq, G, H, T):
     wl = workloads.WORKLOADS["long_gqa_int4"].scaled(batch=3, kv_heads=H, q_heads=H)
