@@ -93,6 +93,30 @@ def test_split_counts_do_not_change_results(kvq, hint):
     assert_close(out, ref, lse, lref, what=f"hint {hint}")
 
 
+@pytest.mark.parametrize("B,H,L", [(2, 2, 5000), (1, 1, 65536)])
+def test_many_partials_and_the_two_call_form(kvq, B, H, L):
+    """Plans of 40 and of 410 partials per query head (one sequence and one
+    KV head over 65536 tokens: the merge kernel's largest thread groups),
+    through the one-call attention and the two-call form (kvq_decode_partials
+    + kvq_decode_merge), against the oracle."""
+    wl = workloads.WORKLOADS["long_gqa_int4"].scaled(batch=B, kv_heads=H, q_heads=4 * H)
+    lens = [L] + [L - 777] * (B - 1)
+    out, lse, ref, lref = _case(kvq, wl, lens, workloads.round_up(L, 64))
+    assert_close(out, ref, lse, lref, what=f"attention B{B} H{H} L{L}")
+    k, v = workloads.kv_tokens(wl, L, DEV, batch=B)
+    q = workloads.queries(wl, DEV, batch=B)
+    c = kvq.QuantizedKVCache.allocate(B, H, 128, workloads.round_up(L, 64), 4, 64, DEV)
+    fill_cache(kvq, c, k, v, lens)
+    ws = kvq.alloc_workspace(c, 4 * H, 0, device=DEV)
+    o2 = torch.full((B, 4 * H, 128), float("nan"), device=DEV)
+    l2 = torch.full((B, 4 * H), float("nan"), device=DEV)
+    kvq.kvq_decode_partials(c, q, o2, l2, ws)
+    kvq.kvq_decode_merge(c, q, o2, l2, ws)
+    torch.cuda.synchronize()
+    assert kvq.workspace_error_word(ws) == 0
+    assert_close(o2, ref, l2, lref, what=f"two-call B{B} H{H} L{L}")
+
+
 def test_edge_lengths(kvq):
     """Empty sequence (out 0, lse -inf), one token, exact tile multiples, the
     full capacity, and a tail of one token past a tile."""
