@@ -665,6 +665,57 @@ cudaError_t launch_decode_segment(const DecodeArgs& a, const SegView& seg, cudaS
   return cudaErrorInvalidValue;
 }
 
+// The merge for up to kSmallParts partials: one thread per output dim
+// issues every load it needs at once -- all (m, l) pairs of its head (the
+// same for the head's threads) and its dim of every partial's o -- and
+// reduces in registers: a single round trip to L2, no barrier.
+constexpr int kSmallParts = 16;
+
+__global__ void __launch_bounds__(kHeadDim) decode_merge_small_kernel(const DecodeArgs a) {
+  grid_dependency_wait();
+  const long long bh = blockIdx.x;
+  const int d = threadIdx.x;
+  const int P = a.parts;
+  const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + bh * P;
+  const float* po = a.part_o + bh * P * kHeadDim + d;
+  float2 v[kSmallParts];
+  float x[kSmallParts];
+#pragma unroll
+  for (int p = 0; p < kSmallParts; ++p) {
+    v[p] = p < P ? ml[p] : make_float2(-INFINITY, 0.f);
+    x[p] = p < P ? po[(long long)p * kHeadDim] : 0.f;
+  }
+  float M = -INFINITY;
+#pragma unroll
+  for (int p = 0; p < kSmallParts; ++p)
+    if (v[p].y > 0.f) M = fmaxf(M, v[p].x);
+  float L = 0.f, O = 0.f;
+#pragma unroll
+  for (int p = 0; p < kSmallParts; ++p) {
+    // a partial with no tokens (l = 0, o = 0) weighs 0
+    const float w = (v[p].y > 0.f) ? exp2f(v[p].x - M) : 0.f;
+    L = fmaf(w, v[p].y, L);
+    O = fmaf(w, x[p], O);
+  }
+  a.out[bh * kHeadDim + d] = (L > 0.f) ? O / L : 0.f;
+  if (a.lse != nullptr && d == 0)
+    a.lse[bh] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+cudaError_t launch_merge_small(const DecodeArgs& a, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long long)a.batch * a.q_heads));
+  cfg.blockDim = dim3(kHeadDim);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_merge_small_kernel, a);
+}
+
 template <int PG>
 cudaError_t launch_merge_pg(const DecodeArgs& a, cudaStream_t s) {
   const size_t smem = ((size_t)a.parts + (PG > 1 ? PG * kHeadDim : 0)) * sizeof(float);
@@ -690,8 +741,8 @@ cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t s) {
   // more partials: more thread groups, so that each thread's chain of
   // dependent loads stays short
   if (a.parts >= 48) return launch_merge_pg<4>(a, s);
-  if (a.parts >= 16) return launch_merge_pg<2>(a, s);
-  return launch_merge_pg<1>(a, s);
+  if (a.parts > kSmallParts) return launch_merge_pg<2>(a, s);
+  return launch_merge_small(a, s);
 }
 
 }  // namespace kvq
