@@ -488,6 +488,24 @@ def cpu_baseline_mixed(wl, k, v, q, seconds: float, wlr):
 
 # ---------------------------------------------------------------- kvq arm
 
+def oaken_outlier_stats(x, params) -> dict:
+    """Outliers per token row of one plane of an Oaken workload's prompt:
+    values outside [T_lo, T_hi] (T_lo = -z_in s_in, T_hi = (15 - z_in) s_in,
+    exact for an fp16 s_in and an integer z_in), and the rows with more than
+    the 16 slots hold (those past the 16th reconstruct to their threshold)."""
+    s_in, z_in, _, _ = params
+    t_lo, t_hi = -z_in * s_in, (15 - z_in) * s_in
+    xf = x.float()
+    cnt = ((xf < t_lo) | (xf > t_hi)).sum(-1).flatten()
+    total = int(cnt.sum())
+    dropped = int((cnt - 16).clamp(min=0).sum())
+    return {"rows": int(cnt.numel()), "rows_over_16": int((cnt > 16).sum()),
+            "frac_rows_over_16": float((cnt > 16).float().mean()),
+            "mean_outliers_per_row": total / max(1, int(cnt.numel())),
+            "max_outliers_per_row": int(cnt.max()), "outliers_dropped": dropped,
+            "frac_outliers_dropped": dropped / max(1, total)}
+
+
 def max_over_ranks(x: float, device) -> float:
     """The largest of every rank's value (a job is as slow as its slowest
     rank); `device` is where the backend wants its tensors."""
@@ -522,6 +540,7 @@ def run_kvq(args, wl, rank, world, local_rank):
 
     # ---- resident inputs (untimed set-up)
     prefill = None  # set by the single-cache set-up below
+    outlier_stats = None  # Oaken codec: how often a row overflows its 16 slots
     chunk_timing = None  # set by the chunk-level mixed set-up below
     if wl.chunk_tokens:
         # chunk-level mixed precision: search, reorder, quantize the prompt
@@ -577,6 +596,9 @@ def run_kvq(args, wl, rank, world, local_rank):
         cache.seq_lens.zero_()
         kvq.kvq_quantize_append(cache, k, v, ctx, advance_seq_lens=True)
         base_lens = cache.seq_lens.clone()
+        if wl.fmt == "oaken":
+            outlier_stats = {"k": oaken_outlier_stats(k, oaken["k_oaken"]),
+                             "v": oaken_outlier_stats(v, oaken["v_oaken"])}
         # the prefill quantize (bulk quantize-on-write of the whole context),
         # timed on its own: HBM-bound, fp16 K/V read once, codes and (s, z)
         # written once
@@ -868,6 +890,7 @@ def run_kvq(args, wl, rank, world, local_rank):
                        **({"prefill_quantize": prefill["us"]} if prefill else {})},
         "gpu_launches": launches_per_step * args.steps,
         **({"prefill_quantize": {**prefill, "frac": prefill["gbs"] / peak}} if prefill else {}),
+        **({"oaken_outliers": outlier_stats} if outlier_stats else {}),
         **({"chunk_reorder": {**chunk_timing, "frac": chunk_timing["reorder_gbs"] / peak}}
            if chunk_timing else {}),
         "clocks": clocks,

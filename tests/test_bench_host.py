@@ -34,3 +34,17 @@ def test_kernel_hash_covers_every_decode_source():
     src = inspect.getsource(bench.kernel_source_hash)
     for f in decode_files:
         assert f'"{f}"' in src, f
+
+
+def test_oaken_outlier_stats():
+    """Rows with more outliers than the 16 slots: s_in = 1, z_in = 8 puts the
+    thresholds at -8 and 7; values equal to a threshold are inner."""
+    import torch
+    x = torch.zeros((1, 1, 3, 128), dtype=torch.float16)
+    x[0, 0, 0, :20] = 7.5          # 20 outliers above T_hi: 4 dropped
+    x[0, 0, 1, :3] = -9.0          # 3 below T_lo
+    x[0, 0, 1, 3:5] = 7.0          # on T_hi: inner
+    x[0, 0, 2, 0] = -8.0           # on T_lo: inner
+    st = bench.oaken_outlier_stats(x, (1.0, 8, 0.5, 5))
+    assert st["rows"] == 3 and st["rows_over_16"] == 1 and st["max_outliers_per_row"] == 20
+    assert st["outliers_dropped"] == 4 and abs(st["mean_outliers_per_row"] - 23 / 3) < 1e-12
