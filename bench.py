@@ -602,24 +602,28 @@ def run_kvq(args, wl, rank, world, local_rank):
         # the prefill quantize (bulk quantize-on-write of the whole context),
         # timed on its own: HBM-bound, fp16 K/V read once, codes and (s, z)
         # written once
-        pf_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        pf_reps = 3
+        # each call timed alone (the seq_lens reset between calls is not)
+        pf_reps = 5
+        pf_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(pf_reps)]
         torch.cuda.synchronize()
-        pf_ev[0].record()
-        for _ in range(pf_reps):
+        for e0, e1 in pf_ev:
             cache.seq_lens.zero_()
+            e0.record()
             kvq.kvq_quantize_append(cache, k, v, ctx, advance_seq_lens=True)
-        pf_ev[1].record()
+            e1.record()
         torch.cuda.synchronize()
-        pf_us = pf_ev[0].elapsed_time(pf_ev[1]) * 1e3 / pf_reps
+        pf_us = statistics.median(e0.elapsed_time(e1) * 1e3 for e0, e1 in pf_ev)
         pf_bytes = B * H * ctx * (2 * D * 2 + bytes_per_head_token(wl.bits, wl.group, D, kpc,
                                                                    wl.fmt))
         prefill = {"tokens": B * ctx, "us": pf_us, "bytes": pf_bytes,
                    "gbs": pf_bytes / (pf_us / 1e6) / 1e9,
-                   "kernel": ("oaken_quantize_kernel" if wl.fmt == "oaken"
+                   "kernel": ("oaken_bulk_kernel" if wl.fmt == "oaken" else
+                              "quantize_k_channels_kernel + quantize_bulk_kernel" if kpc
                               else "quantize_bulk_kernel"),
-                   "note": "fp16 K and V read + packed codes and (s, z) written, per launch "
-                           "(3 launches, each after a 4-byte seq_lens reset)"}
+                   "note": "fp16 K and V read + packed codes and (s, z) written, per "
+                           "kvq_quantize_append call (median of 5 calls, each timed alone "
+                           "after a 4-byte seq_lens reset)"}
         segs = [cache]
         seg_bits = [wl.bits]
         seg_lens = None

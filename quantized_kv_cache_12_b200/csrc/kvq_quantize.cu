@@ -150,11 +150,12 @@ __global__ void __launch_bounds__(kHeadDim) quantize_k_channels_kernel(const Qua
   float x[TB];
 #pragma unroll
   for (int t = 0; t < TB; ++t) x[t] = __half2float(xs[t][d]);
+  // the channel's extremes (-0 and +0 give the same scale and zero point)
   float mn = x[0], mx = x[0];
 #pragma unroll
   for (int t = 1; t < TB; ++t) {
-    mn = x[t] < mn ? x[t] : mn;
-    mx = x[t] > mx ? x[t] : mx;
+    mn = fminf(mn, x[t]);
+    mx = fmaxf(mx, x[t]);
   }
   constexpr int qmax_i = (1 << BITS) - 1;
   constexpr float qmax = float(qmax_i), kInvQmax = 1.0f / qmax;
@@ -172,18 +173,28 @@ __global__ void __launch_bounds__(kHeadDim) quantize_k_channels_kernel(const Qua
   // code = clamp(rint(x / s) + z, 0, qmax): (q + M) + z is M + the code, whose
   // low mantissa bits are the code, when the channel needs no clamp (|z| <=
   // 2048 and its top code, (q_max + M) + (z - M), <= qmax; see the per-token
-  // quantizer), else with the quotient clamped first
+  // quantizer), else with the quotient clamped first.  Tokens t and t + 16
+  // share one packed f32x2 operation.
   const float top = __fadd_rn(__fadd_rn(div_rn(mx, s, r), kMagic), zm);
+  const uint64_t r2 = f2_pack(r, r), nd2 = f2_pack(-s, -s);
+  const uint64_t m2 = f2_pack(kMagic, kMagic), z2 = f2_pack(z, z);
+  constexpr int HT = TB / 2;
   if (fabsf(zf) <= 2048.0f && top <= qmax) {
 #pragma unroll
-    for (int t = 0; t < TB; ++t)
-      cs[t][d] = (uint8_t)__float_as_uint(__fadd_rn(__fadd_rn(div_rn(x[t], s, r), kMagic), z));
+    for (int t = 0; t < HT; ++t) {
+      const float2 c = f2_unpack(f2_add(f2_add(div_rn2(f2_pack(x[t], x[t + HT]), nd2, r2), m2), z2));
+      cs[t][d] = (uint8_t)__float_as_uint(c.x);
+      cs[t + HT][d] = (uint8_t)__float_as_uint(c.y);
+    }
   } else {
     const float lo = -z, hi = __fadd_rn(qmax, -z);
 #pragma unroll
-    for (int t = 0; t < TB; ++t) {
-      const float q = fminf(fmaxf(div_rn(x[t], s, r), lo), hi);
-      cs[t][d] = (uint8_t)__float_as_uint(__fadd_rn(__fadd_rn(q, kMagic), z));
+    for (int t = 0; t < HT; ++t) {
+      const float2 q = f2_unpack(div_rn2(f2_pack(x[t], x[t + HT]), nd2, r2));
+      const uint64_t qc = f2_pack(fminf(fmaxf(q.x, lo), hi), fminf(fmaxf(q.y, lo), hi));
+      const float2 c = f2_unpack(f2_add(f2_add(qc, m2), z2));
+      cs[t][d] = (uint8_t)__float_as_uint(c.x);
+      cs[t + HT][d] = (uint8_t)__float_as_uint(c.y);
     }
   }
   const long long blk = (long long)bh * (a.max_tokens / TB) + pos0 / TB;
