@@ -103,11 +103,13 @@ kvq_status check_cache(const kvq_cache* c, bool allow16) {
 // unit + a fixed per-unit cost) / min(1, c/3), tokens per unit being rounded
 // up to the 32-token stage, with at least 128 tokens per unit.  The fixed
 // cost -- the start of a unit waits for its query rows and first copies,
-// its end merges the warps -- is about 300 tokens' worth of work.  Both
+// its end merges the warps -- is about 300 tokens' worth of work; more than
+// one split adds the merge kernel's launch, about 600 tokens' worth (it
+// decides only for tiny caches, where one split then avoids the launch).  The
 // constants were fitted to split-count sweeps on B200 (INT4, INT8, FP8,
 // per-channel K; 8 to 512 (sequence, head) pairs, 4k to 131k tokens).
 int choose_splits_uncached(long long pairs, long long len, int sms, int ctas) {
-  constexpr long long kOverhead = 300, kGran = 32, kMinTokens = 128;
+  constexpr long long kOverhead = 300, kMerge = 600, kGran = 32, kMinTokens = 128;
   constexpr double kSat = 3.0;
   const long long cap = (len + kMinTokens - 1) / kMinTokens;
   long long best_n = 1;
@@ -119,7 +121,7 @@ int choose_splits_uncached(long long pairs, long long len, int sms, int ctas) {
     const double c_full = (double)ctas, c_rest = (double)rest;
     double rounds = (double)full * c_full / (c_full < kSat ? c_full / kSat : 1.0);
     if (rest > 0) rounds += c_rest / (c_rest < kSat ? c_rest / kSat : 1.0);
-    const double cost = rounds * (double)(chunk + kOverhead);
+    const double cost = rounds * (double)(chunk + kOverhead) + (n > 1 ? (double)kMerge : 0.0);
     if (best_cost < 0 || cost < best_cost * (1.0 - 1e-9)) {
       best_cost = cost;
       best_n = n;

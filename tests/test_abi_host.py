@@ -437,7 +437,9 @@ def test_split_plan_per_workload(kvq):
     without a device), as partials per (sequence, query head).  The plan
     minimises the busiest SM's time: u = ceil(units / SMs) units in rounds of
     up to C (the format's CTAs per SM), a round of c < 3 units at c/3 of the
-    SM's rate, each unit (tokens rounded up to 32) + 300 tokens of fixed cost:
+    SM's rate, each unit (tokens rounded up to 32) + 300 tokens of fixed cost,
+    plus 600 for the merge kernel when there is more than one split (the
+    costs below leave it out: it is the same for every n > 1):
       Llama-3 GQA INT4 (256 pairs, L 8292, C 4): 4 splits, u = 7, rounds 4 + 3,
         7 x (2080 + 300) = 16660; 2 splits cost 4 x 4460 = 17840, 6 splits
         11 x 1708 = 18788, 5 splits (4 + 4 + a lone unit) 11 x 1964 = 21604.
@@ -456,6 +458,10 @@ def test_split_plan_per_workload(kvq):
     assert parts(1, 8, 32, 131392, 131328) == 55
     assert parts(16, 32, 32, 4224, 4196, bits=8, group=128) == 4
     assert parts(32, 8, 32, 8320, 8192, group=128, fmt=kvq.KVQ_FMT_OAKEN) == 5
+    # Tiny (1 pair, 256 tokens): one split, 3 x (256 + 300) = 1668 with the
+    # lone unit at a third of the SM's rate, against 3 x (128 + 300) + 600 =
+    # 1884 for two splits and their merge
+    assert parts(1, 1, 1, 256, 256) == 1
 
 
 def test_split_plan_follows_the_sm_count(tmp_path):
