@@ -123,107 +123,140 @@ __global__ void advance_seq_lens_kernel(int32_t* seq_lens, int batch, int n_new,
 }
 
 // Per-channel K (the KV-cache page's INT8 item: the Key quantized per
-// channel): one CTA per block of kChannelBlock new tokens of one (sequence,
-// KV head), thread d owning channel d.  The block's rows are staged in shared
-// memory; each channel's min, max, scale, zero point and codes follow the
-// same fp32 steps as the per-token groups (the IEEE quotient, round half to
-// even), then the codes are packed along the token rows.  A sequence whose
-// length is not a multiple of the block is skipped; blocks at or past
-// max_tokens (a multiple of 64) are dropped whole.
+// channel).  Work item: a block of kChannelBlock new tokens of one (sequence,
+// KV head), whose fp16 rows are one contiguous 8 KB run of the input.  Each
+// CTA (thread d owning channel d) takes every gridDim.x-th block and keeps
+// the next kChanDepth - 1 blocks in flight as cp.async copies into its ring.
+// Each channel's min, max, scale, zero point and codes follow the same fp32
+// steps as the per-token groups (the IEEE quotient, round half to even), then
+// the codes are packed along the token rows.  A sequence whose length is not
+// a multiple of the block is skipped; blocks at or past max_tokens (a
+// multiple of 64) are dropped whole.
+constexpr int kChanDepth = 3;
+
 template <int BITS>
 __global__ void __launch_bounds__(kHeadDim) quantize_k_channels_kernel(const QuantArgs a) {
   constexpr int D = kHeadDim, TB = kChannelBlock, RB = D * BITS / 8;
-  __shared__ __align__(16) __half xs[TB][D];
+  constexpr int CHUNKS = TB * D / 8 / kHeadDim;  // 16-byte copies per thread and block
+  __shared__ __align__(16) __half ring[kChanDepth][TB][D];
   __shared__ __align__(16) uint8_t cs[TB][D];
-  const int bh = blockIdx.y;
-  const int j = blockIdx.x;
-  const int b = bh / a.kv_heads;
-  const int base = a.seq_lens[b];
-  if (base % TB != 0) return;
-  const int pos0 = base + j * TB;
-  if (pos0 >= a.max_tokens) return;
-  const uint4* src = reinterpret_cast<const uint4*>(a.k_new + ((long long)bh * a.n_new + j * TB) * D);
-  for (int i = threadIdx.x; i < TB * D / 8; i += blockDim.x)
-    reinterpret_cast<uint4*>(&xs[0][0])[i] = src[i];
-  __syncthreads();
+  const int nblk = a.n_new / TB;
+  const long long total = (long long)a.batch * a.kv_heads * nblk;
   const int d = threadIdx.x;
-  float x[TB];
+  const uint32_t ring0 = (uint32_t)__cvta_generic_to_shared(&ring[0][0][0]);
+  // block k of this CTA (global index blockIdx.x + k * gridDim.x) into slot k % depth
+  auto issue = [&](long long k) {
+    const long long q = blockIdx.x + k * gridDim.x;
+    if (q < total) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.k_new) + q * (TB * D / 8);
+      const uint32_t slot = ring0 + (uint32_t)((k % kChanDepth) * (TB * D * 2));
 #pragma unroll
-  for (int t = 0; t < TB; ++t) x[t] = __half2float(xs[t][d]);
-  // the channel's extremes (-0 and +0 give the same scale and zero point)
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int t = 1; t < TB; ++t) {
-    mn = fminf(mn, x[t]);
-    mx = fmaxf(mx, x[t]);
-  }
-  constexpr int qmax_i = (1 << BITS) - 1;
-  constexpr float qmax = float(qmax_i), kInvQmax = 1.0f / qmax;
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  // x / d below: the correction step on RN(1/d), the IEEE quotient
-  const float s32 = fmaxf(div_rn(__fsub_rn(mx, mn), qmax, kInvQmax), 1e-5f);
-  const __half s16 = __float2half_ru(s32);
-  const float s = __half2float(s16);
-  const float r = __frcp_rn(s);
-  float zf = __fadd_rn(rintf(div_rn(-mn, s, r)), 0.0f);
-  zf = fminf(fmaxf(zf, -65504.0f), 65504.0f);
-  const __half z16 = __float2half_rn(zf);
-  const float z = __half2float(z16);
-  const float zm = z - kMagic;
-  // code = clamp(rint(x / s) + z, 0, qmax): (q + M) + z is M + the code, whose
-  // low mantissa bits are the code, when the channel needs no clamp (|z| <=
-  // 2048 and its top code, (q_max + M) + (z - M), <= qmax; see the per-token
-  // quantizer), else with the quotient clamped first.  Tokens t and t + 16
-  // share one packed f32x2 operation.
-  const float top = __fadd_rn(__fadd_rn(div_rn(mx, s, r), kMagic), zm);
-  const uint64_t r2 = f2_pack(r, r), nd2 = f2_pack(-s, -s);
-  const uint64_t m2 = f2_pack(kMagic, kMagic), z2 = f2_pack(z, z);
-  constexpr int HT = TB / 2;
-  if (fabsf(zf) <= 2048.0f && top <= qmax) {
-#pragma unroll
-    for (int t = 0; t < HT; ++t) {
-      const float2 c = f2_unpack(f2_add(f2_add(div_rn2(f2_pack(x[t], x[t + HT]), nd2, r2), m2), z2));
-      cs[t][d] = (uint8_t)__float_as_uint(c.x);
-      cs[t + HT][d] = (uint8_t)__float_as_uint(c.y);
+      for (int c = 0; c < CHUNKS; ++c)
+        cp_async16(slot + (c * kHeadDim + d) * 16, src + c * kHeadDim + d);
     }
-  } else {
-    const float lo = -z, hi = __fadd_rn(qmax, -z);
+    cp_async_commit();  // possibly empty: the wait count stays uniform
+  };
 #pragma unroll
-    for (int t = 0; t < HT; ++t) {
-      const float2 q = f2_unpack(div_rn2(f2_pack(x[t], x[t + HT]), nd2, r2));
-      const uint64_t qc = f2_pack(fminf(fmaxf(q.x, lo), hi), fminf(fmaxf(q.y, lo), hi));
-      const float2 c = f2_unpack(f2_add(f2_add(qc, m2), z2));
-      cs[t][d] = (uint8_t)__float_as_uint(c.x);
-      cs[t + HT][d] = (uint8_t)__float_as_uint(c.y);
-    }
-  }
-  const long long blk = (long long)bh * (a.max_tokens / TB) + pos0 / TB;
-  reinterpret_cast<__half2*>(a.k_meta)[blk * D + d] = __halves2half2(s16, z16);
-  __syncthreads();
-  // rows of codes: whole words read from the byte codes
-  for (int i = threadIdx.x; i < TB * RB / 4; i += blockDim.x) {
-    const int t = i / (RB / 4), w = i % (RB / 4);
-    uint32_t word;
-    if constexpr (BITS == 8) {
-      word = *reinterpret_cast<const uint32_t*>(&cs[t][4 * w]);
-    } else if constexpr (BITS == 4) {
-      const uint2 v = *reinterpret_cast<const uint2*>(&cs[t][8 * w]);
-      const uint32_t a0 = v.x | (v.x >> 4), a1 = v.y | (v.y >> 4);  // bytes 0, 2: code pairs
-      word = __byte_perm(a0, a1, 0x6420);
-    } else {
-      const uint4 v = *reinterpret_cast<const uint4*>(&cs[t][16 * w]);
-      const uint32_t q4[4] = {v.x, v.y, v.z, v.w};
-      uint32_t b[4];
+  for (int k = 0; k < kChanDepth - 1; ++k) issue(k);
+  for (long long k = 0;; ++k) {
+    const long long q = blockIdx.x + k * gridDim.x;
+    if (q >= total) break;
+    // the slot of block k - 1 was read before the previous barrier
+    issue(k + kChanDepth - 1);
+    cp_async_wait<kChanDepth - 1>();  // this thread's copies of block k have landed
+    __syncthreads();                  // ... and every thread's; cs is free
+    const int bh = (int)(q / nblk);
+    const int j = (int)(q - (long long)bh * nblk);
+    const int b = bh / a.kv_heads;
+    const int base = a.seq_lens[b];
+    const int pos0 = base + j * TB;
+    const bool skip = base % TB != 0 || pos0 >= a.max_tokens;  // uniform over the CTA
+    const __half (*xs)[D] = ring[k % kChanDepth];
+    if (!skip) {
+      float x[TB];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t c1 = q4[k] | (q4[k] >> 6);  // bytes 0, 2: code pairs
-        b[k] = c1 | (c1 >> 12);                    // byte 0: four codes
+      for (int t = 0; t < TB; ++t) x[t] = __half2float(xs[t][d]);
+      // the channel's extremes (-0 and +0 give the same scale and zero point)
+      float mn = x[0], mx = x[0];
+#pragma unroll
+      for (int t = 1; t < TB; ++t) {
+        mn = fminf(mn, x[t]);
+        mx = fmaxf(mx, x[t]);
       }
-      word = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+      constexpr int qmax_i = (1 << BITS) - 1;
+      constexpr float qmax = float(qmax_i), kInvQmax = 1.0f / qmax;
+      constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+      // x / d below: the correction step on RN(1/d), the IEEE quotient
+      const float s32 = fmaxf(div_rn(__fsub_rn(mx, mn), qmax, kInvQmax), 1e-5f);
+      const __half s16 = __float2half_ru(s32);
+      const float s = __half2float(s16);
+      const float r = __frcp_rn(s);
+      float zf = __fadd_rn(rintf(div_rn(-mn, s, r)), 0.0f);
+      zf = fminf(fmaxf(zf, -65504.0f), 65504.0f);
+      const __half z16 = __float2half_rn(zf);
+      const float z = __half2float(z16);
+      const float zm = z - kMagic;
+      // code = clamp(rint(x / s) + z, 0, qmax): (q + M) + z is M + the code, whose
+      // low mantissa bits are the code, when the channel needs no clamp (|z| <=
+      // 2048 and its top code, (q_max + M) + (z - M), <= qmax; see the per-token
+      // quantizer), else with the quotient clamped first.  Tokens t and t + 16
+      // share one packed f32x2 operation.
+      const float top = __fadd_rn(__fadd_rn(div_rn(mx, s, r), kMagic), zm);
+      const uint64_t r2 = f2_pack(r, r), nd2 = f2_pack(-s, -s);
+      const uint64_t m2 = f2_pack(kMagic, kMagic), z2 = f2_pack(z, z);
+      constexpr int HT = TB / 2;
+      if (fabsf(zf) <= 2048.0f && top <= qmax) {
+#pragma unroll
+        for (int t = 0; t < HT; ++t) {
+          const float2 c =
+              f2_unpack(f2_add(f2_add(div_rn2(f2_pack(x[t], x[t + HT]), nd2, r2), m2), z2));
+          cs[t][d] = (uint8_t)__float_as_uint(c.x);
+          cs[t + HT][d] = (uint8_t)__float_as_uint(c.y);
+        }
+      } else {
+        const float lo = -z, hi = __fadd_rn(qmax, -z);
+#pragma unroll
+        for (int t = 0; t < HT; ++t) {
+          const float2 qv = f2_unpack(div_rn2(f2_pack(x[t], x[t + HT]), nd2, r2));
+          const uint64_t qc = f2_pack(fminf(fmaxf(qv.x, lo), hi), fminf(fmaxf(qv.y, lo), hi));
+          const float2 c = f2_unpack(f2_add(f2_add(qc, m2), z2));
+          cs[t][d] = (uint8_t)__float_as_uint(c.x);
+          cs[t + HT][d] = (uint8_t)__float_as_uint(c.y);
+        }
+      }
+      const long long blk = (long long)bh * (a.max_tokens / TB) + pos0 / TB;
+      reinterpret_cast<__half2*>(a.k_meta)[blk * D + d] = __halves2half2(s16, z16);
     }
-    reinterpret_cast<uint32_t*>(a.k_codes + ((long long)bh * a.max_tokens + pos0 + t) * RB)[w] =
-        word;
+    __syncthreads();  // the block's codes are in cs
+    if (!skip) {
+      // rows of codes: whole words read from the byte codes
+      for (int i = threadIdx.x; i < TB * RB / 4; i += blockDim.x) {
+        const int t = i / (RB / 4), w = i % (RB / 4);
+        uint32_t word;
+        if constexpr (BITS == 8) {
+          word = *reinterpret_cast<const uint32_t*>(&cs[t][4 * w]);
+        } else if constexpr (BITS == 4) {
+          const uint2 v = *reinterpret_cast<const uint2*>(&cs[t][8 * w]);
+          const uint32_t a0 = v.x | (v.x >> 4), a1 = v.y | (v.y >> 4);  // bytes 0, 2: code pairs
+          word = __byte_perm(a0, a1, 0x6420);
+        } else {
+          const uint4 v = *reinterpret_cast<const uint4*>(&cs[t][16 * w]);
+          const uint32_t q4[4] = {v.x, v.y, v.z, v.w};
+          uint32_t c4[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t c1 = q4[m] | (q4[m] >> 6);  // bytes 0, 2: code pairs
+            c4[m] = c1 | (c1 >> 12);                   // byte 0: four codes
+          }
+          word = __byte_perm(__byte_perm(c4[0], c4[1], 0x0040), __byte_perm(c4[2], c4[3], 0x0040),
+                             0x5410);
+        }
+        reinterpret_cast<uint32_t*>(a.k_codes + ((long long)bh * a.max_tokens + pos0 + t) * RB)[w] =
+            word;
+      }
+    }
   }
+  cp_async_wait<0>();
 }
 
 template <int BITS, int G, bool BF>
@@ -232,10 +265,19 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
   if (a.k_channels) {
     // K: whole blocks, per channel; then the per-token kernels write V only
     if constexpr ((BITS == 2 || BITS == 4 || BITS == 8) && !BF) {
-      if (a.n_new % kChannelBlock != 0 || (long long)a.batch * a.kv_heads > 65535)
-        return cudaErrorInvalidValue;
-      const dim3 grid(a.n_new / kChannelBlock, a.batch * a.kv_heads);
-      quantize_k_channels_kernel<BITS><<<grid, kHeadDim, 0, s>>>(a);
+      if (a.n_new % kChannelBlock != 0) return cudaErrorInvalidValue;
+      static int ch_per_sm = 0;  // resident CTAs per SM of the channel kernel
+      if (ch_per_sm == 0) {
+        int r = 0;
+        const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &r, quantize_k_channels_kernel<BITS>, kHeadDim, 0);
+        if (e != cudaSuccess) return e;
+        ch_per_sm = r > 0 ? r : 1;
+      }
+      const long long blocks = (long long)a.batch * a.kv_heads * (a.n_new / kChannelBlock);
+      const long long slots = (long long)device_sm_count() * ch_per_sm;
+      const unsigned grid = (unsigned)(blocks < slots ? blocks : slots);
+      if (grid > 0) quantize_k_channels_kernel<BITS><<<grid, kHeadDim, 0, s>>>(a);
       const cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
       a.side0 = 1;

@@ -64,6 +64,29 @@ def test_quantize_channels_bit_exact(kvq, bits, G, H, T):
         assert (c.k_meta[b, :, :st // TB].view(torch.int16) == -1).all()
 
 
+@pytest.mark.parametrize("bits", [4, 2])
+def test_quantize_channels_many_blocks(kvq, bits):
+    """Thousands of 32-token blocks, several per CTA of the persistent channel
+    kernel (its copy ring runs over many blocks): sequence 1's last block runs
+    past max_tokens and is dropped, sequence 2 is off a block boundary and left
+    untouched."""
+    B, H, T, cap = 3, 8, 8192, 8192
+    wl = workloads.WORKLOADS["llama3_8b_gqa_int4"].scaled(batch=B, kv_heads=H, q_heads=H)
+    k, v = workloads.kv_tokens(wl, T, DEV)
+    c = _alloc(kvq, B, H, cap, bits, 64)
+    start = [0, 32, 7]
+    c.seq_lens.copy_(torch.tensor(start, dtype=torch.int32))
+    kvq.kvq_quantize_append(c, k, v, T, advance_seq_lens=True)
+    assert c.seq_lens.tolist() == [T, cap, 7]
+    kc, km = oracle.quantize_cache_channels(f16_bits(k), bits)
+    for b, st in enumerate(start[:2]):
+        n = min(T, cap - st)
+        assert np.array_equal(c.k_codes[b, :, st:st + n].cpu().numpy(), kc[b, :, :n])
+        assert np.array_equal(c.k_meta[b, :, st // TB:(st + n) // TB].cpu().numpy().view(np.uint16),
+                              km[b, :, :n // TB])
+    assert (c.k_codes[2] == 0xA5).all() and (c.k_meta[2].view(torch.int16) == -1).all()
+
+
 def _kpc_segment(k, v, bits, G):
     kc, km = oracle.quantize_cache_channels(f16_bits(k), bits)
     vc, vm = oracle.quantize_cache(f16_bits(v), G, bits)
