@@ -54,8 +54,8 @@ __device__ __forceinline__ float div_rn(float x, float d, float r) {
   return __fmaf_rn(e, r, q0);
 }
 
-// div_rn on two values at once: x2 = (x0, x1), nd2 = (-d, -d), r2 = (r, r)
-// (q0 * -d + x is the same fma as -q0 * d + x).
+// div_rn on two values at once, each with its own divisor: x2 = (x0, x1),
+// nd2 = (-d0, -d1), r2 = (r0, r1) (q0 * -d + x is the same fma as -q0 * d + x).
 __device__ __forceinline__ uint64_t div_rn2(uint64_t x2, uint64_t nd2, uint64_t r2) {
   const uint64_t q0 = f2_mul(x2, r2);
   const uint64_t e = f2_fma(q0, nd2, x2);

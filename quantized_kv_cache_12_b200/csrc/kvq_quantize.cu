@@ -124,136 +124,155 @@ __global__ void advance_seq_lens_kernel(int32_t* seq_lens, int batch, int n_new,
 
 // Per-channel K (the KV-cache page's INT8 item: the Key quantized per
 // channel).  Work item: a block of kChannelBlock new tokens of one (sequence,
-// KV head), whose fp16 rows are one contiguous 8 KB run of the input.  Each
-// CTA (thread d owning channel d) takes every gridDim.x-th block and keeps
-// the next kChanDepth - 1 blocks in flight as cp.async copies into its ring.
-// Each channel's min, max, scale, zero point and codes follow the same fp32
-// steps as the per-token groups (the IEEE quotient, round half to even), then
-// the codes are packed along the token rows.  A sequence whose length is not
-// a multiple of the block is skipped; blocks at or past max_tokens (a
-// multiple of 64) are dropped whole.
+// KV head), whose fp16 rows are one contiguous 8 KB run of the input and
+// whose code rows are one contiguous run of the cache.  Each CTA takes every
+// gridDim.x-th block and keeps the next kChanDepth - 1 blocks in flight as
+// cp.async copies into its ring; thread p owns channels 2p and 2p + 1, read
+// as fp16 pairs.  Each channel's min, max, scale, zero point and codes follow
+// the same fp32 steps as the per-token groups (the IEEE quotient, round half
+// to even), the two channels sharing packed f32x2 operations; the codes are
+// packed into the block's rows in shared memory and copied out whole.  A
+// sequence whose length is not a multiple of the block is skipped; blocks at
+// or past max_tokens (a multiple of 64) are dropped whole.
 constexpr int kChanDepth = 3;
+constexpr int kChanThreads = kHeadDim / 2;
+
+// Scale and zero point of one channel of a block from its extremes, and
+// whether its codes need no clamp (see the per-token quantizer): |z| <= 2048
+// and the top code (q_max + M) + (z - M) <= q_max.
+template <int BITS>
+__device__ __forceinline__ bool channel_params(float mn, float mx, __half& s16, __half& z16,
+                                               float& s, float& r, float& z) {
+  constexpr float qmax = float((1 << BITS) - 1), kInvQmax = 1.0f / qmax;
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const float s32 = fmaxf(div_rn(__fsub_rn(mx, mn), qmax, kInvQmax), 1e-5f);
+  s16 = __float2half_ru(s32);
+  s = __half2float(s16);
+  r = __frcp_rn(s);
+  float zf = __fadd_rn(rintf(div_rn(-mn, s, r)), 0.0f);
+  zf = fminf(fmaxf(zf, -65504.0f), 65504.0f);
+  z16 = __float2half_rn(zf);
+  z = __half2float(z16);
+  const float top = __fadd_rn(__fadd_rn(div_rn(mx, s, r), kMagic), z - kMagic);
+  return fabsf(zf) <= 2048.0f && top <= qmax;
+}
 
 template <int BITS>
-__global__ void __launch_bounds__(kHeadDim) quantize_k_channels_kernel(const QuantArgs a) {
+__global__ void __launch_bounds__(kChanThreads) quantize_k_channels_kernel(const QuantArgs a) {
   constexpr int D = kHeadDim, TB = kChannelBlock, RB = D * BITS / 8;
-  constexpr int CHUNKS = TB * D / 8 / kHeadDim;  // 16-byte copies per thread and block
+  constexpr int CHUNKS = TB * D * 2 / 16 / kChanThreads;  // 16-byte copies per thread and block
+  constexpr int OUT = TB * RB / 16 / kChanThreads;        // 16-byte code stores per thread
+  static_assert(OUT >= 1 && TB * RB == OUT * 16 * kChanThreads, "whole 16-byte code stores");
   __shared__ __align__(16) __half ring[kChanDepth][TB][D];
-  __shared__ __align__(16) uint8_t cs[TB][D];
+  __shared__ __align__(16) uint8_t cs[TB][RB];  // the block's packed code rows
   const int nblk = a.n_new / TB;
-  const long long total = (long long)a.batch * a.kv_heads * nblk;
-  const int d = threadIdx.x;
+  const int planes = a.batch * a.kv_heads;
+  const int p = threadIdx.x;
   const uint32_t ring0 = (uint32_t)__cvta_generic_to_shared(&ring[0][0][0]);
-  // block k of this CTA (global index blockIdx.x + k * gridDim.x) into slot k % depth
-  auto issue = [&](long long k) {
-    const long long q = blockIdx.x + k * gridDim.x;
-    if (q < total) {
-      const uint4* src = reinterpret_cast<const uint4*>(a.k_new) + q * (TB * D / 8);
-      const uint32_t slot = ring0 + (uint32_t)((k % kChanDepth) * (TB * D * 2));
+  // the copy cursor: block (bh, j) = blockIdx.x + k * gridDim.x, k = 0, 1, ...
+  // (stepped without dividing), and its ring slot
+  const int step_bh = (int)(gridDim.x / nblk), step_j = (int)(gridDim.x % nblk);
+  auto advance = [&](int& bh, int& j) {
+    j += step_j;
+    bh += step_bh;
+    if (j >= nblk) {
+      j -= nblk;
+      ++bh;
+    }
+  };
+  int ibh = (int)(blockIdx.x / nblk), ij = (int)(blockIdx.x % nblk), islot = 0;
+  auto issue = [&]() {
+    if (ibh < planes) {
+      const uint4* src =
+          reinterpret_cast<const uint4*>(a.k_new + ((long long)ibh * a.n_new + ij * TB) * D);
+      const uint32_t slot = ring0 + (uint32_t)(islot * (TB * D * 2));
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c)
-        cp_async16(slot + (c * kHeadDim + d) * 16, src + c * kHeadDim + d);
+        cp_async16(slot + (c * kChanThreads + p) * 16, src + c * kChanThreads + p);
     }
     cp_async_commit();  // possibly empty: the wait count stays uniform
+    advance(ibh, ij);
+    islot = islot + 1 == kChanDepth ? 0 : islot + 1;
   };
 #pragma unroll
-  for (int k = 0; k < kChanDepth - 1; ++k) issue(k);
-  for (long long k = 0;; ++k) {
-    const long long q = blockIdx.x + k * gridDim.x;
-    if (q >= total) break;
-    // the slot of block k - 1 was read before the previous barrier
-    issue(k + kChanDepth - 1);
-    cp_async_wait<kChanDepth - 1>();  // this thread's copies of block k have landed
+  for (int k = 0; k < kChanDepth - 1; ++k) issue();
+  // the work cursor
+  int bh = (int)(blockIdx.x / nblk), j = (int)(blockIdx.x % nblk), slot = 0;
+  for (; bh < planes; advance(bh, j)) {
+    issue();  // into the slot read before the previous barrier
+    cp_async_wait<kChanDepth - 1>();  // this thread's copies of the block have landed
     __syncthreads();                  // ... and every thread's; cs is free
-    const int bh = (int)(q / nblk);
-    const int j = (int)(q - (long long)bh * nblk);
+    const __half (*xs)[D] = ring[slot];
+    slot = slot + 1 == kChanDepth ? 0 : slot + 1;
     const int b = bh / a.kv_heads;
     const int base = a.seq_lens[b];
     const int pos0 = base + j * TB;
     const bool skip = base % TB != 0 || pos0 >= a.max_tokens;  // uniform over the CTA
-    const __half (*xs)[D] = ring[k % kChanDepth];
     if (!skip) {
-      float x[TB];
+      __half2 xv[TB];
 #pragma unroll
-      for (int t = 0; t < TB; ++t) x[t] = __half2float(xs[t][d]);
-      // the channel's extremes (-0 and +0 give the same scale and zero point)
-      float mn = x[0], mx = x[0];
+      for (int t = 0; t < TB; ++t) xv[t] = *reinterpret_cast<const __half2*>(&xs[t][2 * p]);
+      // the channels' extremes, a pairwise tree (exact; -0 and +0 give the
+      // same scale and zero point)
+      __half2 lo2[TB / 2], hi2[TB / 2];
 #pragma unroll
-      for (int t = 1; t < TB; ++t) {
-        mn = fminf(mn, x[t]);
-        mx = fmaxf(mx, x[t]);
+      for (int t = 0; t < TB / 2; ++t) {
+        lo2[t] = __hmin2(xv[2 * t], xv[2 * t + 1]);
+        hi2[t] = __hmax2(xv[2 * t], xv[2 * t + 1]);
       }
-      constexpr int qmax_i = (1 << BITS) - 1;
-      constexpr float qmax = float(qmax_i), kInvQmax = 1.0f / qmax;
-      constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-      // x / d below: the correction step on RN(1/d), the IEEE quotient
-      const float s32 = fmaxf(div_rn(__fsub_rn(mx, mn), qmax, kInvQmax), 1e-5f);
-      const __half s16 = __float2half_ru(s32);
-      const float s = __half2float(s16);
-      const float r = __frcp_rn(s);
-      float zf = __fadd_rn(rintf(div_rn(-mn, s, r)), 0.0f);
-      zf = fminf(fmaxf(zf, -65504.0f), 65504.0f);
-      const __half z16 = __float2half_rn(zf);
-      const float z = __half2float(z16);
-      const float zm = z - kMagic;
-      // code = clamp(rint(x / s) + z, 0, qmax): (q + M) + z is M + the code, whose
-      // low mantissa bits are the code, when the channel needs no clamp (|z| <=
-      // 2048 and its top code, (q_max + M) + (z - M), <= qmax; see the per-token
-      // quantizer), else with the quotient clamped first.  Tokens t and t + 16
-      // share one packed f32x2 operation.
-      const float top = __fadd_rn(__fadd_rn(div_rn(mx, s, r), kMagic), zm);
-      const uint64_t r2 = f2_pack(r, r), nd2 = f2_pack(-s, -s);
-      const uint64_t m2 = f2_pack(kMagic, kMagic), z2 = f2_pack(z, z);
-      constexpr int HT = TB / 2;
-      if (fabsf(zf) <= 2048.0f && top <= qmax) {
 #pragma unroll
-        for (int t = 0; t < HT; ++t) {
-          const float2 c =
-              f2_unpack(f2_add(f2_add(div_rn2(f2_pack(x[t], x[t + HT]), nd2, r2), m2), z2));
-          cs[t][d] = (uint8_t)__float_as_uint(c.x);
-          cs[t + HT][d] = (uint8_t)__float_as_uint(c.y);
-        }
-      } else {
-        const float lo = -z, hi = __fadd_rn(qmax, -z);
+      for (int w = TB / 4; w >= 1; w /= 2)
 #pragma unroll
-        for (int t = 0; t < HT; ++t) {
-          const float2 qv = f2_unpack(div_rn2(f2_pack(x[t], x[t + HT]), nd2, r2));
-          const uint64_t qc = f2_pack(fminf(fmaxf(qv.x, lo), hi), fminf(fmaxf(qv.y, lo), hi));
-          const float2 c = f2_unpack(f2_add(f2_add(qc, m2), z2));
-          cs[t][d] = (uint8_t)__float_as_uint(c.x);
-          cs[t + HT][d] = (uint8_t)__float_as_uint(c.y);
+        for (int t = 0; t < w; ++t) {
+          lo2[t] = __hmin2(lo2[t], lo2[t + w]);
+          hi2[t] = __hmax2(hi2[t], hi2[t + w]);
         }
-      }
+      __half s0h, z0h, s1h, z1h;
+      float s0, r0, z0, s1, r1, z1;
+      const bool ok0 = channel_params<BITS>(__low2float(lo2[0]), __low2float(hi2[0]), s0h, z0h,
+                                            s0, r0, z0);
+      const bool ok1 = channel_params<BITS>(__high2float(lo2[0]), __high2float(hi2[0]), s1h,
+                                            z1h, s1, r1, z1);
       const long long blk = (long long)bh * (a.max_tokens / TB) + pos0 / TB;
-      reinterpret_cast<__half2*>(a.k_meta)[blk * D + d] = __halves2half2(s16, z16);
-    }
-    __syncthreads();  // the block's codes are in cs
-    if (!skip) {
-      // rows of codes: whole words read from the byte codes
-      for (int i = threadIdx.x; i < TB * RB / 4; i += blockDim.x) {
-        const int t = i / (RB / 4), w = i % (RB / 4);
-        uint32_t word;
-        if constexpr (BITS == 8) {
-          word = *reinterpret_cast<const uint32_t*>(&cs[t][4 * w]);
-        } else if constexpr (BITS == 4) {
-          const uint2 v = *reinterpret_cast<const uint2*>(&cs[t][8 * w]);
-          const uint32_t a0 = v.x | (v.x >> 4), a1 = v.y | (v.y >> 4);  // bytes 0, 2: code pairs
-          word = __byte_perm(a0, a1, 0x6420);
-        } else {
-          const uint4 v = *reinterpret_cast<const uint4*>(&cs[t][16 * w]);
-          const uint32_t q4[4] = {v.x, v.y, v.z, v.w};
-          uint32_t c4[4];
+      reinterpret_cast<uint2*>(a.k_meta)[blk * (D / 2) + p] =
+          make_uint2(h2_as_u32(__halves2half2(s0h, z0h)), h2_as_u32(__halves2half2(s1h, z1h)));
+      // code = clamp(rint(x / s) + z, 0, qmax): (q + M) + z is M + the code,
+      // whose low mantissa bits are the code, when neither channel needs a
+      // clamp, else with the quotients clamped first
+      constexpr float qmax = float((1 << BITS) - 1), kMagic = 12582912.0f;
+      const uint64_t r2 = f2_pack(r0, r1), nd2 = f2_pack(-s0, -s1);
+      const uint64_t m2 = f2_pack(kMagic, kMagic), z2 = f2_pack(z0, z1);
+      const bool fast = ok0 && ok1;
+      const float lo0 = -z0, hi0 = __fadd_rn(qmax, -z0), lo1 = -z1, hi1 = __fadd_rn(qmax, -z1);
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint32_t c1 = q4[m] | (q4[m] >> 6);  // bytes 0, 2: code pairs
-            c4[m] = c1 | (c1 >> 12);                   // byte 0: four codes
-          }
-          word = __byte_perm(__byte_perm(c4[0], c4[1], 0x0040), __byte_perm(c4[2], c4[3], 0x0040),
-                             0x5410);
+      for (int t = 0; t < TB; ++t) {
+        const float2 xf = __half22float2(xv[t]);
+        uint64_t qv = div_rn2(f2_pack(xf.x, xf.y), nd2, r2);
+        if (!fast) {
+          const float2 u = f2_unpack(qv);
+          qv = f2_pack(fminf(fmaxf(u.x, lo0), hi0), fminf(fmaxf(u.y, lo1), hi1));
         }
-        reinterpret_cast<uint32_t*>(a.k_codes + ((long long)bh * a.max_tokens + pos0 + t) * RB)[w] =
-            word;
+        const float2 c = f2_unpack(f2_add(f2_add(qv, m2), z2));
+        const uint32_t c0 = __float_as_uint(c.x) & 0xFFu, c1 = __float_as_uint(c.y) & 0xFFu;
+        if constexpr (BITS == 8) {
+          *reinterpret_cast<uint16_t*>(&cs[t][2 * p]) = (uint16_t)(c0 | (c1 << 8));
+        } else if constexpr (BITS == 4) {
+          cs[t][p] = (uint8_t)(c0 | (c1 << 4));
+        } else {
+          // four 2-bit codes a byte: the odd thread's pair joins the even one's
+          const uint32_t nib = c0 | (c1 << 2);
+          const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
+          if ((p & 1) == 0) cs[t][p >> 1] = (uint8_t)(nib | (other << 4));
+        }
       }
+    }
+    __syncthreads();  // the block's code rows are in cs
+    if (!skip) {
+      uint4* dst = reinterpret_cast<uint4*>(a.k_codes + ((long long)bh * a.max_tokens + pos0) * RB);
+#pragma unroll
+      for (int c = 0; c < OUT; ++c)
+        dst[c * kChanThreads + p] =
+            reinterpret_cast<const uint4*>(&cs[0][0])[c * kChanThreads + p];
     }
   }
   cp_async_wait<0>();
@@ -270,14 +289,14 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
       if (ch_per_sm == 0) {
         int r = 0;
         const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &r, quantize_k_channels_kernel<BITS>, kHeadDim, 0);
+            &r, quantize_k_channels_kernel<BITS>, kChanThreads, 0);
         if (e != cudaSuccess) return e;
         ch_per_sm = r > 0 ? r : 1;
       }
       const long long blocks = (long long)a.batch * a.kv_heads * (a.n_new / kChannelBlock);
       const long long slots = (long long)device_sm_count() * ch_per_sm;
       const unsigned grid = (unsigned)(blocks < slots ? blocks : slots);
-      if (grid > 0) quantize_k_channels_kernel<BITS><<<grid, kHeadDim, 0, s>>>(a);
+      if (grid > 0) quantize_k_channels_kernel<BITS><<<grid, kChanThreads, 0, s>>>(a);
       const cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
       a.side0 = 1;
