@@ -113,6 +113,10 @@ __global__ void __launch_bounds__(kBulkWarps * 32) quantize_bulk_kernel(const Qu
                  [&](const Dst& c, const uint32_t (&roff)[kBulkNV / 8], const uint8_t* slot) {
                    bulk_work<BITS, G, BF>(a, li, c, roff, slot);
                  });
+  // launched as the per-channel K kernel's dependent (V rows only), this one
+  // starts on the SMs that kernel leaves and must not finish before it: the
+  // seq_lens update after it assumes both are done (a no-op otherwise)
+  grid_dependency_wait();
 }
 
 __global__ void advance_seq_lens_kernel(int32_t* seq_lens, int batch, int n_new,
@@ -165,6 +169,7 @@ __global__ void __launch_bounds__(kChanThreads) quantize_k_channels_kernel(const
   static_assert(OUT >= 1 && TB * RB == OUT * 16 * kChanThreads, "whole 16-byte code stores");
   __shared__ __align__(16) __half ring[kChanDepth][TB][D];
   __shared__ __align__(16) uint8_t cs[TB][RB];  // the block's packed code rows
+  grid_dependents_may_launch();  // the V kernel may fill the SMs this one leaves
   const int nblk = a.n_new / TB;
   const int planes = a.batch * a.kv_heads;
   const int p = threadIdx.x;
@@ -281,6 +286,7 @@ __global__ void __launch_bounds__(kChanThreads) quantize_k_channels_kernel(const
 template <int BITS, int G, bool BF>
 cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
   QuantArgs a = a_in;
+  bool after_k = false;  // the per-channel K kernel was launched just before
   if (a.k_channels) {
     // K: whole blocks, per channel; then the per-token kernels write V only
     if constexpr ((BITS == 2 || BITS == 4 || BITS == 8) && !BF) {
@@ -296,9 +302,12 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
       const long long blocks = (long long)a.batch * a.kv_heads * (a.n_new / kChannelBlock);
       const long long slots = (long long)device_sm_count() * ch_per_sm;
       const unsigned grid = (unsigned)(blocks < slots ? blocks : slots);
-      if (grid > 0) quantize_k_channels_kernel<BITS><<<grid, kChanThreads, 0, s>>>(a);
-      const cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
+      if (grid > 0) {
+        quantize_k_channels_kernel<BITS><<<grid, kChanThreads, 0, s>>>(a);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        after_k = true;
+      }
       a.side0 = 1;
     } else {
       return cudaErrorInvalidValue;
@@ -323,9 +332,27 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
   }
   BulkShape sh;
   if (!bulk_shape(a, per_sm, &sh)) return cudaErrorInvalidValue;
-  quantize_bulk_kernel<BITS, G, BF><<<sh.blocks, kBulkWarps * 32, 0, s>>>(
-      a, sh.units_per_row, sh.n_units, sh.per_warp);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (after_k) {
+    // V only, after the per-channel K kernel: a programmatic dependent, so
+    // its CTAs take the SMs that kernel's CTAs leave
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sh.blocks);
+    cfg.blockDim = dim3(kBulkWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, quantize_bulk_kernel<BITS, G, BF>, a, sh.units_per_row,
+                           sh.n_units, sh.per_warp);
+  } else {
+    quantize_bulk_kernel<BITS, G, BF><<<sh.blocks, kBulkWarps * 32, 0, s>>>(
+        a, sh.units_per_row, sh.n_units, sh.per_warp);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess || !a.advance) return e;
   advance_seq_lens_kernel<<<(a.batch + 127) / 128, 128, 0, s>>>(a.seq_lens, a.batch, a.n_new,
                                                                a.max_tokens, a.k_channels);
