@@ -202,4 +202,24 @@ inline bool bulk_shape(const QuantArgs& a, int ctas_per_sm, BulkShape* sh) {
   return true;
 }
 
+// Host side: launch `kernel` as a programmatic dependent of the kernel before
+// it on the stream.  It may be scheduled once that kernel's CTAs have all
+// signalled (grid_dependents_may_launch) or exited, so it must call
+// grid_dependency_wait() before it touches memory that kernel writes.
+template <class... KArgs, class... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                                    cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace kvq

@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(kBulkWarps * 32) oaken_bulk_kernel(const Quant
   __shared__ __align__(16) uint8_t ring[kBulkWarps][kBulkDepth][kUnitBytes];
   __shared__ __align__(16) uint16_t sbuf[kBulkWarps][kUnitRows][kSlots];
   __shared__ __align__(16) uint16_t olist[kBulkWarps][kOakList];
+  grid_dependents_may_launch();  // the seq_lens update may be scheduled
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   bulk_loop<OakDst>(a, units_per_row, n_units, units_per_warp, &ring[warp][0][0],
                     [&](const OakDst& c, const uint32_t (&roff)[kBulkNV / 8],
@@ -280,6 +281,7 @@ __global__ void __launch_bounds__(kBulkWarps * 32) oaken_bulk_kernel(const Quant
 }
 
 __global__ void oaken_advance_kernel(int32_t* seq_lens, int batch, int n_new, int max_tokens) {
+  grid_dependency_wait();  // the quantizer before it reads seq_lens
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < batch) seq_lens[b] = min(seq_lens[b] + n_new, max_tokens);
 }
@@ -322,9 +324,9 @@ cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s) {
   }
   e = cudaGetLastError();
   if (e != cudaSuccess || !a.advance) return e;
-  oaken_advance_kernel<<<(a.batch + 127) / 128, 128, 0, s>>>(a.seq_lens, a.batch, a.n_new,
-                                                             a.max_tokens);
-  return cudaGetLastError();
+  // a programmatic dependent: scheduled while the quantizer runs
+  return launch_dependent(oaken_advance_kernel, dim3((a.batch + 127) / 128), dim3(128), s,
+                          a.seq_lens, a.batch, a.n_new, a.max_tokens);
 }
 
 }  // namespace kvq

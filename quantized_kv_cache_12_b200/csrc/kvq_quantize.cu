@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(kBulkWarps * 32) quantize_bulk_kernel(const Qu
                                                                         int n_units,
                                                                         int units_per_warp) {
   __shared__ __align__(16) uint8_t ring[kBulkWarps][kBulkDepth][kUnitBytes];
+  grid_dependents_may_launch();  // the seq_lens update may be scheduled
   const int li = (threadIdx.x & 31) % kBulkLanes;
   using Dst = BulkDst<kHeadDim * code_bits(BITS) / 8, (kHeadDim / G) * 4>;
   bulk_loop<Dst>(a, units_per_row, n_units, units_per_warp, &ring[threadIdx.x >> 5][0][0],
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(kBulkWarps * 32) quantize_bulk_kernel(const Qu
 
 __global__ void advance_seq_lens_kernel(int32_t* seq_lens, int batch, int n_new,
                                         int max_tokens, int k_channels) {
+  grid_dependency_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < batch && !(k_channels && seq_lens[b] % kChannelBlock != 0))
     seq_lens[b] = min(seq_lens[b] + n_new, max_tokens);
@@ -336,27 +338,18 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
   if (after_k) {
     // V only, after the per-channel K kernel: a programmatic dependent, so
     // its CTAs take the SMs that kernel's CTAs leave
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(sh.blocks);
-    cfg.blockDim = dim3(kBulkWarps * 32);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, quantize_bulk_kernel<BITS, G, BF>, a, sh.units_per_row,
-                           sh.n_units, sh.per_warp);
+    e = launch_dependent(quantize_bulk_kernel<BITS, G, BF>, dim3(sh.blocks),
+                         dim3(kBulkWarps * 32), s, a, sh.units_per_row, sh.n_units, sh.per_warp);
   } else {
     quantize_bulk_kernel<BITS, G, BF><<<sh.blocks, kBulkWarps * 32, 0, s>>>(
         a, sh.units_per_row, sh.n_units, sh.per_warp);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess || !a.advance) return e;
-  advance_seq_lens_kernel<<<(a.batch + 127) / 128, 128, 0, s>>>(a.seq_lens, a.batch, a.n_new,
-                                                               a.max_tokens, a.k_channels);
-  return cudaGetLastError();
+  // a programmatic dependent: scheduled while the quantizer runs, it waits
+  // for it before moving seq_lens (which the quantizer reads)
+  return launch_dependent(advance_seq_lens_kernel, dim3((a.batch + 127) / 128), dim3(128), s,
+                          a.seq_lens, a.batch, a.n_new, a.max_tokens, a.k_channels);
 }
 
 }  // namespace
