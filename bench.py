@@ -864,15 +864,20 @@ def run_kvq(args, wl, rank, world, local_rank):
                 "segments": {f"bits{b}": int(ln.sum()) for b, ln in zip(seg_bits, seg_lens)}}
                if seg_lens is not None else {}),
             "launch": "each step replayed from one CUDA graph per episode position "
-                      "(split-K kernel, then the merge as a programmatic dependent); "
-                      "event-record nodes in the graph time the split-K launch",
+                      + ("(split-K kernel, then the merge as a programmatic dependent); "
+                         if parts > 1 else
+                         "(one split: the attention kernel writes the output, no merge); ")
+                      + "event-record nodes in the graph time the split-K launch",
             "l2": f"inputs larger than L2: {sum(kv_bytes) / args.steps / 1e6:.0f} MB of packed "
                   f"K/V read per step per GPU (L2 126 MB)",
             "step": ("kvq_decode_step: quantize-on-write of 1 token/seq inside the split-K "
-                     "decode attention kernel, then the LSE merge" if wl.append else
-                     "split-K decode attention over the FP16/INT4/INT2 segments + LSE merge"
+                     "decode attention kernel" + (", then the LSE merge" if parts > 1 else "")
+                     if wl.append else
+                     "split-K decode attention over the FP16/INT4/INT2 segments" +
+                     (" + LSE merge" if parts > 1 else "")
                      if wl.chunk_tokens else
-                     "split-K decode attention over the prefilled cache + LSE merge")}),
+                     "split-K decode attention over the prefilled cache" +
+                     (" + LSE merge" if parts > 1 else ""))}),
         "kv_read_gbs": sum(kv_bytes) / (ms / 1e3) / 1e9 * world,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
