@@ -249,16 +249,9 @@ __global__ void __launch_bounds__(kChanThreads) quantize_k_channels_kernel(const
       constexpr float qmax = float((1 << BITS) - 1), kMagic = 12582912.0f;
       const uint64_t r2 = f2_pack(r0, r1), nd2 = f2_pack(-s0, -s1);
       const uint64_t m2 = f2_pack(kMagic, kMagic), z2 = f2_pack(z0, z1);
-      const bool fast = ok0 && ok1;
       const float lo0 = -z0, hi0 = __fadd_rn(qmax, -z0), lo1 = -z1, hi1 = __fadd_rn(qmax, -z1);
-#pragma unroll
-      for (int t = 0; t < TB; ++t) {
-        const float2 xf = __half22float2(xv[t]);
-        uint64_t qv = div_rn2(f2_pack(xf.x, xf.y), nd2, r2);
-        if (!fast) {
-          const float2 u = f2_unpack(qv);
-          qv = f2_pack(fminf(fmaxf(u.x, lo0), hi0), fminf(fmaxf(u.y, lo1), hi1));
-        }
+      // the token's two codes into its code row
+      auto put = [&](int t, uint64_t qv) {
         const float2 c = f2_unpack(f2_add(f2_add(qv, m2), z2));
         const uint32_t c0 = __float_as_uint(c.x) & 0xFFu, c1 = __float_as_uint(c.y) & 0xFFu;
         if constexpr (BITS == 8) {
@@ -270,6 +263,23 @@ __global__ void __launch_bounds__(kChanThreads) quantize_k_channels_kernel(const
           const uint32_t nib = c0 | (c1 << 2);
           const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
           if ((p & 1) == 0) cs[t][p >> 1] = (uint8_t)(nib | (other << 4));
+        }
+      };
+      // two loops, so that the common case carries no clamp; the choice is
+      // the warp's (the clamp leaves in-range quotients as they are), which
+      // keeps the 2-bit path's shuffle convergent
+      if (__all_sync(0xffffffffu, ok0 && ok1)) {
+#pragma unroll
+        for (int t = 0; t < TB; ++t) {
+          const float2 xf = __half22float2(xv[t]);
+          put(t, div_rn2(f2_pack(xf.x, xf.y), nd2, r2));
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < TB; ++t) {
+          const float2 xf = __half22float2(xv[t]);
+          const float2 u = f2_unpack(div_rn2(f2_pack(xf.x, xf.y), nd2, r2));
+          put(t, f2_pack(fminf(fmaxf(u.x, lo0), hi0), fminf(fmaxf(u.y, lo1), hi1)));
         }
       }
     }

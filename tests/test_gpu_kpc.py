@@ -67,12 +67,16 @@ def test_quantize_channels_bit_exact(kvq, bits, G, H, T):
 @pytest.mark.parametrize("bits", [4, 2])
 def test_quantize_channels_many_blocks(kvq, bits):
     """Thousands of 32-token blocks, several per CTA of the persistent channel
-    kernel (its copy ring runs over many blocks): sequence 1's last block runs
-    past max_tokens and is dropped, sequence 2 is off a block boundary and left
-    untouched."""
+    kernel (its copy ring runs over many blocks), a few of them on the clamped
+    path: sequence 1's last block runs past max_tokens and is dropped,
+    sequence 2 is off a block boundary and left untouched."""
     B, H, T, cap = 3, 8, 8192, 8192
     wl = workloads.WORKLOADS["llama3_8b_gqa_int4"].scaled(batch=B, kv_heads=H, q_heads=H)
     k, v = workloads.kv_tokens(wl, T, DEV)
+    # blocks that take the clamped path: a constant channel (the scale floor
+    # puts |z| far past 2048) and a channel block spanning a huge range
+    k[1, 2, 64:96, 7] = 3.0
+    k[0, 5, 4096:4128, 100] = torch.linspace(-60000.0, 60000.0, 32)
     c = _alloc(kvq, B, H, cap, bits, 64)
     start = [0, 32, 7]
     c.seq_lens.copy_(torch.tensor(start, dtype=torch.int32))
