@@ -435,10 +435,10 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
       const __half* qfrow = qf_tab + qh * D + 32 * tig;
       const __half2* szr = reinterpret_cast<const __half2*>(sKm) + 32 * tig;  // (s, z) of its channels
       const bool lo_part = gid & 1;
-      // bias terms by pair position j: their query values carry 2^(EMAX - e_j)
-      float bpj[WP::kPairs];
-#pragma unroll
-      for (int j = 0; j < WP::kPairs; ++j) bpj[j] = 0.f;
+      // the chunk's zero points as A rows of the bias MMA: pair p holds
+      // (z_d0, z_d1) 2^(e_j - 24), exact in fp16 (z is an integer), the
+      // units of the codes
+      uint32_t zf[16];
 #pragma unroll
       for (int wb = 0; wb < 32 / KD; ++wb) {
         // this word block's query values and (s, z) pairs, in vector loads
@@ -461,24 +461,20 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
           const float r0 = fma_h(q0, __low2half(sz0), -__low2float(hi));
           const float r1 = fma_h(q1, __low2half(sz1), -__high2float(hi));
           const __half2 lo = __floats2half2_rn(r0, r1);
-          float b = bpj[j];
-          b = fma_h(__low2half(hi), __high2half(sz0), b);
-          b = fma_h(__high2half(hi), __high2half(sz1), b);
-          b = fma_h(__low2half(lo), __high2half(sz0), b);
-          bpj[j] = fma_h(__high2half(lo), __high2half(sz1), b);
           qb[p / 2][p % 2] = h2_as_u32(lo_part ? lo : hi);
+          zf[p] = h2_as_u32(
+              __hmul2(__highs2half2(sz0, sz1), __float2half2_rn(pow2f(WP::exp(j) - 24))));
         }
       }
-      // in the MMA's units, 2^(EMAX - 24) sum q s z: each term's query value
-      // already carries 2^(EMAX - e_j), so it takes 2^(e_j - 24); then the
-      // head's sum over its 128 channels (the four lanes of this gid), read
-      // from a lane holding the owned head (gid = 2 h)
-      float bp = 0.f;
+      // every row of the accumulator is sum_d z_d (q s)_d over the column's
+      // part, in the QK MMA's units: columns 2 tig (hi) and 2 tig + 1 (lo)
+      // of head tig mod g, the lane's own
+      float b_even[4] = {0.f, 0.f, 0.f, 0.f}, b_odd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < WP::kPairs; ++j) bp = fmaf(bpj[j], pow2f(WP::exp(j) - 24), bp);
-      bp += __shfl_xor_sync(0xffffffffu, bp, 1);
-      bp += __shfl_xor_sync(0xffffffffu, bp, 2);
-      kbias = __shfl_sync(0xffffffffu, bp, 8 * own_h[0]);
+      for (int ks = 0; ks < 8; ++ks)
+        mma_f16((ks & 1) ? b_odd : b_even, zf[2 * ks], zf[2 * ks], zf[2 * ks + 1], zf[2 * ks + 1],
+                qb[ks][0], qb[ks][1]);
+      kbias = (b_even[0] + b_odd[0]) + (b_even[1] + b_odd[1]);
     }
   };
 
