@@ -74,6 +74,7 @@ def _load():
         lib.kvqo_quantize_group_e5m2.argtypes = [P, i32, P, P]
         lib.kvqo_quantize_rows_e5m2.argtypes = [P, i64, i32, i32, P, P]
         lib.kvqo_quantize_block_channels.argtypes = [P, i32, i32, i32, P, P]
+        lib.kvqo_quantize_block_channels_in.argtypes = [P, i32, i32, i32, i32, P, P]
         lib.kvqo_dequantize_block_channels.argtypes = [P, P, i32, i32, i32, P]
         lib.kvqo_quantize_rows_sym8.argtypes = [P, i64, i32, i32, P, P]
         lib.kvqo_dequantize_rows_fmt.argtypes = [P, P, i64, i32, i32, i32, i32, P]
@@ -276,15 +277,18 @@ def quantize_group_sym8(x16):
 KPC_BLOCK = 32
 
 
-def quantize_block_channels(x16, bits: int):
-    """One block of token rows [T, D] (fp16 patterns) -> (codes [T, D*bits/8],
-    meta [D, 2] uint16 (s, z) per channel)."""
+def quantize_block_channels(x16, bits: int, in_dtype: str = "f16"):
+    """One block of token rows [T, D] (fp16 patterns, or bfloat16 ones with
+    in_dtype "bf16", read exactly into fp32 like the fp16 ones) ->
+    (codes [T, D*bits/8], meta [D, 2] uint16 (s, z) per channel)."""
+    assert in_dtype in ("f16", "bf16"), in_dtype
     lib = _load()
     x16 = _c(x16, np.uint16)
     T, D = x16.shape
     codes = np.zeros((T, D * bits // 8), np.uint8)
     meta = np.zeros((D, 2), np.uint16)
-    lib.kvqo_quantize_block_channels(_p(x16), T, D, bits, _p(codes), _p(meta))
+    lib.kvqo_quantize_block_channels_in(_p(x16), int(in_dtype == "bf16"), T, D, bits, _p(codes),
+                                        _p(meta))
     return codes, meta
 
 
@@ -299,9 +303,10 @@ def dequantize_block_channels(codes, meta, D: int, bits: int) -> np.ndarray:
     return out
 
 
-def quantize_cache_channels(x16, bits: int):
-    """x16 [..., T, D] with T a multiple of KPC_BLOCK -> codes [..., T, D*bits/8],
-    meta [..., T / KPC_BLOCK, D, 2]."""
+def quantize_cache_channels(x16, bits: int, in_dtype: str = "f16"):
+    """x16 [..., T, D] (fp16, or with in_dtype "bf16" bfloat16, patterns) with
+    T a multiple of KPC_BLOCK -> codes [..., T, D*bits/8], meta
+    [..., T / KPC_BLOCK, D, 2]."""
     x16 = _c(x16, np.uint16)
     lead, (T, D) = x16.shape[:-2], x16.shape[-2:]
     assert T % KPC_BLOCK == 0, T
@@ -310,7 +315,7 @@ def quantize_cache_channels(x16, bits: int):
     meta = np.zeros((flat.shape[0], T // KPC_BLOCK, D, 2), np.uint16)
     for i in range(flat.shape[0]):
         for blk in range(T // KPC_BLOCK):
-            c, m = quantize_block_channels(flat[i, blk], bits)
+            c, m = quantize_block_channels(flat[i, blk], bits, in_dtype)
             codes[i, blk * KPC_BLOCK:(blk + 1) * KPC_BLOCK] = c
             meta[i, blk] = m
     return (codes.reshape(*lead, T, D * bits // 8),

@@ -710,12 +710,13 @@ void kvqo_dequantize_rows(const uint8_t *codes, const uint16_t *meta,
 /* Per-channel K ([P2'] item 2: the Key quantized per channel; R16)         */
 /* ------------------------------------------------------------------------ */
 
-/* One block of T token rows x [T][D] (binary16) of one (sequence, KV head):
- * the T values of channel d form one group, quantized with the asymmetric
- * formula of R1-R5 (kvqo_quantize_group).  codes: [T][D*bits/8], packed
- * along each token row (R7); meta: [D][2], the (s, z) of each channel. */
-void kvqo_quantize_block_channels(const uint16_t *x, int T, int D, int bits, uint8_t *codes,
-                                  uint16_t *meta)
+/* One block of T token rows x [T][D] (binary16, or bfloat16 when in_bf16,
+ * R19) of one (sequence, KV head): the T values of channel d form one
+ * group, quantized with the asymmetric formula of R1-R5
+ * (kvqo_quantize_group_in).  codes: [T][D*bits/8], packed along each token
+ * row (R7); meta: [D][2], the (s, z) of each channel. */
+void kvqo_quantize_block_channels_in(const uint16_t *x, int in_bf16, int T, int D, int bits,
+                                     uint8_t *codes, uint16_t *meta)
 {
     const int64_t row_bytes = (int64_t)D * bits / 8;
     uint16_t *col = (uint16_t *)malloc((size_t)T * sizeof(uint16_t));
@@ -725,7 +726,7 @@ void kvqo_quantize_block_channels(const uint16_t *x, int T, int D, int bits, uin
         for (int t = 0; t < T; ++t)
             col[t] = x[(int64_t)t * D + d];
         uint16_t s16, z16;
-        kvqo_quantize_group(col, T, bits, tmp, &s16, &z16);
+        kvqo_quantize_group_in(col, in_bf16, T, bits, tmp, &s16, &z16);
         meta[d * 2 + 0] = s16;
         meta[d * 2 + 1] = z16;
         const int bitpos = d * bits;
@@ -734,6 +735,13 @@ void kvqo_quantize_block_channels(const uint16_t *x, int T, int D, int bits, uin
     }
     free(col);
     free(tmp);
+}
+
+/* The binary16 form of the above. */
+void kvqo_quantize_block_channels(const uint16_t *x, int T, int D, int bits, uint8_t *codes,
+                                  uint16_t *meta)
+{
+    kvqo_quantize_block_channels_in(x, 0, T, D, bits, codes, meta);
 }
 
 /* x_hat[t][d] = (c[t][d] - z_d) * s_d of one block, in fp64 (exact). */

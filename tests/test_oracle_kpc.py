@@ -88,3 +88,38 @@ def test_attention_over_a_per_channel_segment_matches_torch():
                 qq[None, :, None], torch.from_numpy(K)[None, None].expand(1, g, n, 128),
                 torch.from_numpy(V)[None, None].expand(1, g, n, 128), scale=128 ** -0.5)
             assert np.allclose(o[b, h * g:(h + 1) * g], ref[0, :, 0].numpy(), atol=1e-12)
+
+
+def test_bf16_block_with_the_worked_example_in_one_channel():
+    """bf16 input (reading R19) through the per-channel path: channel 9 of a
+    block holds the hand-worked bf16 INT4 group of tests/golden (values beyond
+    the fp16 range), four times over, so its min and max, and hence its
+    scale, zero point and codes, are the fixture's."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                                    "bf16_worked_example.json")))
+    pat = np.array([int(h, 16) for h in g["bf16_patterns"]], np.uint16)
+    rng = np.random.default_rng(25)
+    x = torch.from_numpy(rng.standard_normal((T, 128)).astype(np.float32))
+    xb = x.to(torch.bfloat16).contiguous().view(torch.int16).numpy().view(np.uint16).copy()
+    xb[:, 9] = np.tile(pat, T // len(pat))
+    codes, meta = oracle.quantize_block_channels(xb, 4, in_dtype="bf16")
+    assert _unpack(codes, 4, 128)[:, 9].tolist() == g["codes"] * (T // len(pat))
+    assert int(meta[9, 0]) == int(g["scale_f16"], 16)
+    assert int(meta[9, 1]) == int(g["zero_f16"], 16)
+
+
+def test_bf16_block_of_fp16_values_matches_the_fp16_path():
+    """A bf16 block whose values are all fp16 values gives exactly the codes
+    and (s, z) of its fp16 form (both widen to the same fp32 values)."""
+    rng = np.random.default_rng(26)
+    for bits in (2, 4, 8):
+        x = torch.from_numpy(_block(rng).astype(np.float32))
+        xb = x.to(torch.bfloat16).float()
+        assert torch.equal(xb.half().float(), xb)
+        b16 = xb.to(torch.bfloat16).contiguous().view(torch.int16).numpy().view(np.uint16)
+        f16 = xb.to(torch.float16).contiguous().view(torch.int16).numpy().view(np.uint16)
+        cb, mb = oracle.quantize_block_channels(b16, bits, in_dtype="bf16")
+        cf, mf = oracle.quantize_block_channels(f16, bits)
+        assert np.array_equal(cb, cf) and np.array_equal(mb, mf), bits
