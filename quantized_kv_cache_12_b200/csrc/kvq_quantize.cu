@@ -130,11 +130,13 @@ __global__ void advance_seq_lens_kernel(int32_t* seq_lens, int batch, int n_new,
 
 // Per-channel K (the KV-cache page's INT8 item: the Key quantized per
 // channel).  Work item: a block of kChannelBlock new tokens of one (sequence,
-// KV head), whose fp16 rows are one contiguous 8 KB run of the input and
+// KV head), whose fp16 (or, with BF, bf16) rows are one contiguous 8 KB run
+// of the input and
 // whose code rows are one contiguous run of the cache.  Each CTA takes every
 // gridDim.x-th block and keeps the next kChanDepth - 1 blocks in flight as
 // cp.async copies into its ring; thread p owns channels 2p and 2p + 1, read
-// as fp16 pairs.  Each channel's min, max, scale, zero point and codes follow
+// as 16-bit pairs (widened to fp32 exactly).  Each channel's min, max, scale,
+// zero point and codes follow
 // the same fp32 steps as the per-token groups (the IEEE quotient, round half
 // to even), the two channels sharing packed f32x2 operations; the codes are
 // packed into the block's rows in shared memory and copied out whole.  A
@@ -163,8 +165,9 @@ __device__ __forceinline__ bool channel_params(float mn, float mx, __half& s16, 
   return fabsf(zf) <= 2048.0f && top <= qmax;
 }
 
-template <int BITS>
+template <int BITS, bool BF>
 __global__ void __launch_bounds__(kChanThreads) quantize_k_channels_kernel(const QuantArgs a) {
+  using IP = InPair<BF>;
   constexpr int D = kHeadDim, TB = kChannelBlock, RB = D * BITS / 8;
   constexpr int CHUNKS = TB * D * 2 / 16 / kChanThreads;  // 16-byte copies per thread and block
   constexpr int OUT = TB * RB / 16 / kChanThreads;        // 16-byte code stores per thread
@@ -209,37 +212,36 @@ __global__ void __launch_bounds__(kChanThreads) quantize_k_channels_kernel(const
     issue();  // into the slot read before the previous barrier
     cp_async_wait<kChanDepth - 1>();  // this thread's copies of the block have landed
     __syncthreads();                  // ... and every thread's; cs is free
-    const __half (*xs)[D] = ring[slot];
+    const uint32_t* xs = reinterpret_cast<const uint32_t*>(&ring[slot][0][0]);  // [TB][D / 2]
     slot = slot + 1 == kChanDepth ? 0 : slot + 1;
     const int b = bh / a.kv_heads;
     const int base = a.seq_lens[b];
     const int pos0 = base + j * TB;
     const bool skip = base % TB != 0 || pos0 >= a.max_tokens;  // uniform over the CTA
     if (!skip) {
-      __half2 xv[TB];
+      uint32_t xv[TB];  // token t: the pair (channel 2p, channel 2p + 1)
 #pragma unroll
-      for (int t = 0; t < TB; ++t) xv[t] = *reinterpret_cast<const __half2*>(&xs[t][2 * p]);
+      for (int t = 0; t < TB; ++t) xv[t] = xs[t * (D / 2) + p];
       // the channels' extremes, a pairwise tree (exact; -0 and +0 give the
       // same scale and zero point)
-      __half2 lo2[TB / 2], hi2[TB / 2];
+      uint32_t lo2[TB / 2], hi2[TB / 2];
 #pragma unroll
       for (int t = 0; t < TB / 2; ++t) {
-        lo2[t] = __hmin2(xv[2 * t], xv[2 * t + 1]);
-        hi2[t] = __hmax2(xv[2 * t], xv[2 * t + 1]);
+        lo2[t] = IP::min2(xv[2 * t], xv[2 * t + 1]);
+        hi2[t] = IP::max2(xv[2 * t], xv[2 * t + 1]);
       }
 #pragma unroll
       for (int w = TB / 4; w >= 1; w /= 2)
 #pragma unroll
         for (int t = 0; t < w; ++t) {
-          lo2[t] = __hmin2(lo2[t], lo2[t + w]);
-          hi2[t] = __hmax2(hi2[t], hi2[t + w]);
+          lo2[t] = IP::min2(lo2[t], lo2[t + w]);
+          hi2[t] = IP::max2(hi2[t], hi2[t + w]);
         }
+      const float2 mn = IP::widen(lo2[0]), mx = IP::widen(hi2[0]);
       __half s0h, z0h, s1h, z1h;
       float s0, r0, z0, s1, r1, z1;
-      const bool ok0 = channel_params<BITS>(__low2float(lo2[0]), __low2float(hi2[0]), s0h, z0h,
-                                            s0, r0, z0);
-      const bool ok1 = channel_params<BITS>(__high2float(lo2[0]), __high2float(hi2[0]), s1h,
-                                            z1h, s1, r1, z1);
+      const bool ok0 = channel_params<BITS>(mn.x, mx.x, s0h, z0h, s0, r0, z0);
+      const bool ok1 = channel_params<BITS>(mn.y, mx.y, s1h, z1h, s1, r1, z1);
       const long long blk = (long long)bh * (a.max_tokens / TB) + pos0 / TB;
       reinterpret_cast<uint2*>(a.k_meta)[blk * (D / 2) + p] =
           make_uint2(h2_as_u32(__halves2half2(s0h, z0h)), h2_as_u32(__halves2half2(s1h, z1h)));
@@ -271,13 +273,13 @@ __global__ void __launch_bounds__(kChanThreads) quantize_k_channels_kernel(const
       if (__all_sync(0xffffffffu, ok0 && ok1)) {
 #pragma unroll
         for (int t = 0; t < TB; ++t) {
-          const float2 xf = __half22float2(xv[t]);
+          const float2 xf = IP::widen(xv[t]);
           put(t, div_rn2(f2_pack(xf.x, xf.y), nd2, r2));
         }
       } else {
 #pragma unroll
         for (int t = 0; t < TB; ++t) {
-          const float2 xf = __half22float2(xv[t]);
+          const float2 xf = IP::widen(xv[t]);
           const float2 u = f2_unpack(div_rn2(f2_pack(xf.x, xf.y), nd2, r2));
           put(t, f2_pack(fminf(fmaxf(u.x, lo0), hi0), fminf(fmaxf(u.y, lo1), hi1)));
         }
@@ -301,13 +303,13 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
   bool after_k = false;  // the per-channel K kernel was launched just before
   if (a.k_channels) {
     // K: whole blocks, per channel; then the per-token kernels write V only
-    if constexpr ((BITS == 2 || BITS == 4 || BITS == 8) && !BF) {
+    if constexpr (BITS == 2 || BITS == 4 || BITS == 8) {
       if (a.n_new % kChannelBlock != 0) return cudaErrorInvalidValue;
       static int ch_per_sm = 0;  // resident CTAs per SM of the channel kernel
       if (ch_per_sm == 0) {
         int r = 0;
         const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &r, quantize_k_channels_kernel<BITS>, kChanThreads, 0);
+            &r, quantize_k_channels_kernel<BITS, BF>, kChanThreads, 0);
         if (e != cudaSuccess) return e;
         ch_per_sm = r > 0 ? r : 1;
       }
@@ -315,7 +317,7 @@ cudaError_t launch_q(const QuantArgs& a_in, cudaStream_t s) {
       const long long slots = (long long)device_sm_count() * ch_per_sm;
       const unsigned grid = (unsigned)(blocks < slots ? blocks : slots);
       if (grid > 0) {
-        quantize_k_channels_kernel<BITS><<<grid, kChanThreads, 0, s>>>(a);
+        quantize_k_channels_kernel<BITS, BF><<<grid, kChanThreads, 0, s>>>(a);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         after_k = true;

@@ -136,9 +136,10 @@ def test_quantize_append_rejects_bad_arguments(kvq):
 
 
 def test_quantize_append_kv_dtype(kvq):
-    """kv_dtype is KVQ_F16 or KVQ_BF16; bf16 input is refused for per-channel
-    K and Oaken planes (token-grouped formats only); the binding passes the
-    tensors' dtype and refuses mixed or other dtypes before calling."""
+    """kv_dtype is KVQ_F16 or KVQ_BF16; bf16 input is refused for Oaken planes
+    only (a per-channel K plane takes it, and goes on to its block check); the
+    binding passes the tensors' dtype and refuses mixed or other dtypes before
+    calling."""
     import torch
     fake = ctypes.c_void_p(0x60000)
 
@@ -150,7 +151,7 @@ def test_quantize_append_kv_dtype(kvq):
     assert st(_fake_cache(kvq, bits=3), kvq.KVQ_BF16) == kvq.KVQ_ERR_UNSUPPORTED
     c = _fake_cache(kvq, bits=4)
     c.k.axis = kvq.KVQ_AXIS_CHANNEL
-    assert st(c, kvq.KVQ_BF16, n=32) == kvq.KVQ_ERR_UNSUPPORTED
+    assert st(c, kvq.KVQ_BF16, n=31) == kvq.KVQ_ERR_INVALID_ARG  # off a block boundary
     c = _fake_cache(kvq, bits=4, group=128)
     c.k.fmt = c.v.fmt = kvq.KVQ_FMT_OAKEN
     c.k.oaken = kvq.kvq_oaken(0.25, 8, 0.5, 5)

@@ -91,6 +91,47 @@ def test_quantize_channels_many_blocks(kvq, bits):
     assert (c.k_codes[2] == 0xA5).all() and (c.k_meta[2].view(torch.int16) == -1).all()
 
 
+@pytest.mark.parametrize("bits", [4, 2, 8])
+def test_quantize_channels_bf16_bit_exact(kvq, bits):
+    """bf16 K/V (reading R19) through the per-channel K kernel and the
+    per-token V kernel, against the oracle's bf16 path: thousands of blocks,
+    several per CTA, and (at 4 and 8 bits) one channel block holding the
+    hand-worked bf16 group of tests/golden (values beyond the fp16 range) four
+    times over."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                                    "bf16_worked_example.json")))
+    B, H, T, cap = 2, 8, 4096, 4096 + 64
+    wl = workloads.WORKLOADS["llama3_8b_gqa_int4"].scaled(batch=B, kv_heads=H, q_heads=H)
+    k, v = workloads.kv_tokens(wl, T, DEV, dtype=torch.bfloat16)
+    vals = torch.tensor(g["values"], dtype=torch.float32).to(torch.bfloat16)
+    if (max(g["values"]) - min(g["values"])) / ((1 << bits) - 1) <= 65504:
+        # planted where its scale fits fp16 (at 2 bits it does not, and the
+        # header leaves such a group's codes unspecified)
+        k[1, 3, 96:128, 9] = vals.repeat(TB // len(g["values"])).to(DEV)
+    c = _alloc(kvq, B, H, cap, bits, 64)
+    start = [0, 32]
+    c.seq_lens.copy_(torch.tensor(start, dtype=torch.int32))
+    kvq.kvq_quantize_append(c, k, v, T, advance_seq_lens=True)
+    assert c.seq_lens.tolist() == [T, T + 32]
+
+    def b16(t):
+        return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    kc, km = oracle.quantize_cache_channels(b16(k), bits, in_dtype="bf16")
+    vc, vm = oracle.quantize_cache(b16(v), 64, bits, in_dtype="bf16")
+    if bits == g["bits"]:  # the worked block's scale and zero point
+        assert int(km[1, 3, 3, 9, 0]) == int(g["scale_f16"], 16)
+        assert int(km[1, 3, 3, 9, 1]) == int(g["zero_f16"], 16)
+    for b, st in enumerate(start):
+        p = slice(st, st + T)
+        assert np.array_equal(c.k_codes[b, :, p].cpu().numpy(), kc[b]), b
+        assert np.array_equal(c.k_meta[b, :, st // TB:(st + T) // TB].cpu().numpy().view(np.uint16),
+                              km[b]), b
+        assert np.array_equal(c.v_codes[b, :, p].cpu().numpy(), vc[b]), b
+        assert np.array_equal(c.v_meta[b, :, p].cpu().numpy().view(np.uint16), vm[b]), b
+
+
 def _kpc_segment(k, v, bits, G):
     kc, km = oracle.quantize_cache_channels(f16_bits(k), bits)
     vc, vm = oracle.quantize_cache(f16_bits(v), G, bits)
