@@ -84,6 +84,8 @@ def _load():
         lib.kvqo_chunk_partition.argtypes = [P, i32, P, P]
         f32 = ctypes.c_float
         lib.kvqo_oaken_quantize_rows.argtypes = [P, i64, i32, f32, i32, f32, i32, P, P]
+        lib.kvqo_oaken_quantize_rows_in.argtypes = [P, i32, i64, i32, f32, i32, f32, i32, P,
+                                                    P]
         lib.kvqo_oaken_dequantize_rows.argtypes = [P, P, i64, i32, f32, i32, f32, P]
         lib.kvqo_kv_elements.argtypes = [u64, u64, u64, u64, u64]
         lib.kvqo_kv_elements.restype = u64
@@ -341,16 +343,20 @@ def dequantize_channels(codes, meta, L: int, D: int, bits: int) -> np.ndarray:
 OAKEN_SLOTS = 16
 
 
-def oaken_quantize_rows(x16, s_in: float, z_in: int, s_out: float, outer_bits: int):
-    """Token rows [N, D] (fp16 patterns) -> (codes [N, D/2] uint8, slots
-    [N, OAKEN_SLOTS] uint16) with the plane's offline parameters."""
+def oaken_quantize_rows(x16, s_in: float, z_in: int, s_out: float, outer_bits: int,
+                        in_dtype: str = "f16"):
+    """Token rows [N, D] (fp16 patterns, or bfloat16 ones with in_dtype "bf16",
+    read exactly into fp32) -> (codes [N, D/2] uint8, slots [N, OAKEN_SLOTS]
+    uint16) with the plane's offline parameters."""
+    assert in_dtype in ("f16", "bf16"), in_dtype
     lib = _load()
     x16 = _c(x16, np.uint16)
     N, D = x16.shape
     codes = np.zeros((N, D // 2), np.uint8)
     slots = np.zeros((N, OAKEN_SLOTS), np.uint16)
-    lib.kvqo_oaken_quantize_rows(_p(x16), N, D, float(s_in), int(z_in), float(s_out),
-                                 int(outer_bits), _p(codes), _p(slots))
+    lib.kvqo_oaken_quantize_rows_in(_p(x16), int(in_dtype == "bf16"), N, D, float(s_in),
+                                    int(z_in), float(s_out), int(outer_bits), _p(codes),
+                                    _p(slots))
     return codes, slots
 
 
@@ -366,12 +372,13 @@ def oaken_dequantize_rows(codes, slots, D: int, s_in: float, z_in: int, s_out: f
     return out
 
 
-def oaken_quantize_cache(x16, params):
-    """x16 [..., T, D] -> codes [..., T, D/2], slots [..., T, OAKEN_SLOTS];
-    params = (s_in, z_in, s_out, outer_bits)."""
+def oaken_quantize_cache(x16, params, in_dtype: str = "f16"):
+    """x16 [..., T, D] (fp16, or with in_dtype "bf16" bfloat16, patterns) ->
+    codes [..., T, D/2], slots [..., T, OAKEN_SLOTS]; params = (s_in, z_in,
+    s_out, outer_bits)."""
     x16 = _c(x16, np.uint16)
     lead, D = x16.shape[:-1], x16.shape[-1]
-    codes, slots = oaken_quantize_rows(x16.reshape(-1, D), *params)
+    codes, slots = oaken_quantize_rows(x16.reshape(-1, D), *params, in_dtype=in_dtype)
     return codes.reshape(*lead, D // 2), slots.reshape(*lead, OAKEN_SLOTS)
 
 

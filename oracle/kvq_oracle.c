@@ -574,8 +574,8 @@ void kvqo_quantize_rows_any(const uint16_t *x, int in_bf16, int64_t n_rows, int 
  * values to packed 4-bit codes (D / 2 bytes) and 16 outlier slots. */
 #define KVQO_OAKEN_SLOTS 16
 
-void kvqo_oaken_quantize_row(const uint16_t *x, int D, float s_in, int z_in, float s_out,
-                             int outer_bits, uint8_t *codes, uint16_t *slots)
+void kvqo_oaken_quantize_row_in(const uint16_t *x, int in_bf16, int D, float s_in, int z_in,
+                                float s_out, int outer_bits, uint8_t *codes, uint16_t *slots)
 {
     const float z = (float)z_in;
     const float t_lo = -z * s_in;
@@ -586,7 +586,7 @@ void kvqo_oaken_quantize_row(const uint16_t *x, int D, float s_in, int z_in, flo
     for (int i = 0; i < KVQO_OAKEN_SLOTS; ++i)
         slots[i] = 0;
     for (int j = 0; j < D; ++j) {
-        const float v = kvqo_f16_to_f32(x[j]);
+        const float v = kvqo_in(x, j, in_bf16); /* binary16 or bfloat16 (R19), exact */
         unsigned c;
         int outlier = 0, d = 0;
         if (v > t_hi) { /* outer zone, high side: shift by T_hi */
@@ -621,12 +621,25 @@ void kvqo_oaken_quantize_row(const uint16_t *x, int D, float s_in, int z_in, flo
     }
 }
 
+void kvqo_oaken_quantize_row(const uint16_t *x, int D, float s_in, int z_in, float s_out,
+                             int outer_bits, uint8_t *codes, uint16_t *slots)
+{
+    kvqo_oaken_quantize_row_in(x, 0, D, s_in, z_in, s_out, outer_bits, codes, slots);
+}
+
+void kvqo_oaken_quantize_rows_in(const uint16_t *x, int in_bf16, int64_t n_rows, int D,
+                                 float s_in, int z_in, float s_out, int outer_bits,
+                                 uint8_t *codes, uint16_t *slots)
+{
+    for (int64_t r = 0; r < n_rows; ++r)
+        kvqo_oaken_quantize_row_in(x + r * D, in_bf16, D, s_in, z_in, s_out, outer_bits,
+                                   codes + r * (D / 2), slots + r * KVQO_OAKEN_SLOTS);
+}
+
 void kvqo_oaken_quantize_rows(const uint16_t *x, int64_t n_rows, int D, float s_in, int z_in,
                               float s_out, int outer_bits, uint8_t *codes, uint16_t *slots)
 {
-    for (int64_t r = 0; r < n_rows; ++r)
-        kvqo_oaken_quantize_row(x + r * D, D, s_in, z_in, s_out, outer_bits,
-                                codes + r * (D / 2), slots + r * KVQO_OAKEN_SLOTS);
+    kvqo_oaken_quantize_rows_in(x, 0, n_rows, D, s_in, z_in, s_out, outer_bits, codes, slots);
 }
 
 /* x_hat = (c - z_in) * s_in + d * s_out in fp64 (R18); the dense part is the

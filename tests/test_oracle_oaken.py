@@ -140,3 +140,43 @@ def test_dense_sparse_equals_the_page_dequantization():
     so = float(np.float32(s_out))  # the plane's parameters are fp32
     expect = np.where(np.arange(16) < 8, t_hi + m * so, t_lo + m * so)
     assert np.array_equal(xh, expect)
+
+
+def test_bf16_worked_row():
+    """bf16 input (reading R19) through the Oaken encoder: the hand-worked row
+    of tests/golden/oaken_bf16_worked_example.json, with outliers beyond the
+    fp16 range on both sides (capped magnitudes), values on the thresholds
+    (inner), a zero-magnitude outlier and two halfway magnitudes."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                                    "oaken_bf16_worked_example.json")))
+    import torch
+    vals = torch.tensor(g["values"], dtype=torch.float32)
+    pat = np.array([int(h, 16) for h in g["bf16_patterns"]], np.uint16)
+    assert np.array_equal(vals.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16), pat)
+    codes, slots = oracle.oaken_quantize_rows(pat[None], g["s_in"], g["z_in"], g["s_out"],
+                                              g["outer_bits"], in_dtype="bf16")
+    assert [(int(codes[0, j // 2]) >> (4 * (j % 2))) & 15 for j in range(8)] == g["codes"]
+    want = [int(h, 16) for h in g["slots"]]
+    assert slots[0, :len(want)].tolist() == want
+    assert not slots[0, len(want):].any()
+
+
+def test_bf16_rows_of_fp16_values_match_the_fp16_path():
+    """bf16 rows whose values are all fp16 values (outliers included) give
+    exactly the fp16 path's codes and slots."""
+    import torch
+    gen = torch.Generator().manual_seed(31)
+    x = torch.randn((48, 128), generator=gen) * 2
+    x[:, 7] *= 40.0
+    x[:, 90] *= -25.0
+    x[3, :20] = torch.linspace(-60.0, 60.0, 20)
+    xb = x.to(torch.bfloat16).float()
+    assert torch.equal(xb.half().float(), xb)
+    b16 = xb.to(torch.bfloat16).contiguous().view(torch.int16).numpy().view(np.uint16)
+    f16 = xb.to(torch.float16).contiguous().view(torch.int16).numpy().view(np.uint16)
+    for params in ((0.25, 8, 0.5, 5), (0.125, 3, 0.05, 7), (0.5, 0, 2.0, 6)):
+        cb, sb = oracle.oaken_quantize_rows(b16, *params, in_dtype="bf16")
+        cf, sf = oracle.oaken_quantize_rows(f16, *params)
+        assert np.array_equal(cb, cf) and np.array_equal(sb, sf), params
