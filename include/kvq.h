@@ -222,11 +222,9 @@ uint64_t kvq_kv_elements(uint64_t layers, uint64_t kv_heads, uint64_t head_dim,
  *   kv_dtype:     KVQ_F16 or KVQ_BF16.  Values of either type are widened to
  *                 fp32 exactly and go through the same fp32 steps, so a bf16
  *                 row holding fp16-representable values gives the codes of
- *                 its fp16 form.  bf16 input is taken by every format but
- *                 the Oaken codec (asymmetric integer per token or, for K,
- *                 per channel; FP8 E4M3/E5M2; symmetric INT8); an Oaken
- *                 plane with bf16 input returns KVQ_ERR_UNSUPPORTED.  bf16
- *                 values reach
+ *                 its fp16 form.  Every format takes either (asymmetric
+ *                 integer per token or, for K, per channel; FP8 E4M3/E5M2;
+ *                 symmetric INT8; the Oaken codec).  bf16 values reach
  *                 beyond fp16: a group is encodable when its scale fits fp16
  *                 ((max - min) / (2^bits - 1), or |max| / 448, / 57344,
  *                 / 127, at most 65504) and its values are below 2^64 in

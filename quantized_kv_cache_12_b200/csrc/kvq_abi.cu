@@ -316,9 +316,6 @@ kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const 
   if (kv_dtype != KVQ_F16 && kv_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
   if (n_new < 1) return KVQ_ERR_INVALID_ARG;
   if (n_new > cache->max_tokens) return KVQ_ERR_CAPACITY;
-  // bf16 input: every format but the Oaken codec (whose encoder clamps to
-  // its thresholds in fp16)
-  if (kv_dtype == KVQ_BF16 && cache->k.fmt == KVQ_FMT_OAKEN) return KVQ_ERR_UNSUPPORTED;
   kvq::QuantArgs a;
   a.in_bf16 = kv_dtype == KVQ_BF16;
   a.k_new = static_cast<const __half*>(k_new);

@@ -25,6 +25,7 @@
 //     lanes per row, 32 dims a lane), dense codes branch-free, outliers in
 //     a compact per-lane loop.  HBM-bound: 256 B read and 96 B written per
 //     row.
+//   Both take fp16 or bf16 rows (BF), widened to fp32 exactly.
 //   The decode attention over these planes is the tokens-on-M kernel's
 //     (kvq_decode_tm.cu): the dense codes through the tensor cores like
 //     INT4 with the plane's one (s, z), the K slots as per-token score
@@ -47,6 +48,15 @@ constexpr int D = kHeadDim;
 constexpr int kSlots = KVQ_OAKEN_SLOTS;
 constexpr int kRowBytes = D / 2;         // 4-bit codes of one row
 constexpr int kSlotBytes = kSlots * 2;   // outlier slots of one row
+
+// A 16-bit input element (fp16, or bf16 with BF) widened to fp32, exactly.
+template <bool BF>
+__device__ __forceinline__ float in_f32(uint16_t h) {
+  if constexpr (BF)
+    return __uint_as_float((uint32_t)h << 16);
+  else
+    return __half2float(__ushort_as_half(h));
+}
 
 // One element: its 4-bit code, and its signed outlier magnitude (0 inside).
 __device__ __forceinline__ uint32_t oaken_code(float v, const OakenParams& p, int& d,
@@ -72,6 +82,7 @@ __device__ __forceinline__ uint32_t oaken_code(float v, const OakenParams& p, in
 }
 
 // Half a warp per row: lane li of the half owns dims 8 li .. 8 li + 7.
+template <bool BF>
 __global__ void __launch_bounds__(256) oaken_quantize_kernel(const QuantArgs a) {
   const int lane = threadIdx.x & 31;
   const int li = lane & 15;
@@ -96,13 +107,13 @@ __global__ void __launch_bounds__(256) oaken_quantize_kernel(const QuantArgs a) 
         reinterpret_cast<uint16_t*>((plane ? a.v_meta : a.k_meta) + dst_row * kSlotBytes);
 
     const uint4 raw = reinterpret_cast<const uint4*>(src)[li];
-    const __half* hv = reinterpret_cast<const __half*>(&raw);
+    const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw);
     uint32_t word = 0, flags = 0;
     int dv[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       bool o;
-      word |= oaken_code(__half2float(hv[e]), p, dv[e], o) << (4 * e);
+      word |= oaken_code(in_f32<BF>(hv[e]), p, dv[e], o) << (4 * e);
       flags |= (uint32_t)o << e;
     }
     reinterpret_cast<uint32_t*>(codes)[li] = word;
@@ -146,9 +157,10 @@ constexpr int kOakList = kUnitRows * kSlots;  // outliers a unit can keep
 
 struct OakUnitParams {
   float s_in, r_in, z, t_lo, t_hi, s_out, m_max;
-  uint32_t tl2, th2;  // fp16 pairs (tl, tl) and (th, th)
+  uint32_t tl2, th2;  // pairs (tl, tl) and (th, th) in the input's 16-bit type
 };
 
+template <bool BF>
 __device__ __forceinline__ OakUnitParams oaken_unit_params(const OakenParams& p) {
   OakUnitParams u;
   u.s_in = p.s_in;
@@ -158,12 +170,20 @@ __device__ __forceinline__ OakUnitParams oaken_unit_params(const OakenParams& p)
   u.t_hi = p.t_hi;
   u.s_out = p.s_out;
   u.m_max = p.m_max;
-  const __half tl = __float2half_ru(p.t_lo), th = __float2half_rd(p.t_hi);
-  u.tl2 = h2_as_u32(__halves2half2(tl, tl));
-  u.th2 = h2_as_u32(__halves2half2(th, th));
+  if constexpr (BF) {
+    const uint32_t tl = __bfloat16_as_ushort(__float2bfloat16_ru(p.t_lo));
+    const uint32_t th = __bfloat16_as_ushort(__float2bfloat16_rd(p.t_hi));
+    u.tl2 = tl | (tl << 16);
+    u.th2 = th | (th << 16);
+  } else {
+    const __half tl = __float2half_ru(p.t_lo), th = __float2half_rd(p.t_hi);
+    u.tl2 = h2_as_u32(__halves2half2(tl, tl));
+    u.th2 = h2_as_u32(__halves2half2(th, th));
+  }
   return u;
 }
 
+template <bool BF>
 __device__ __forceinline__ void oaken_work(const QuantArgs& a, int lane, const OakDst& c,
                                            const uint32_t (&roff)[kBulkNV / 8],
                                            const uint8_t* slot, uint16_t* sbuf,
@@ -172,7 +192,8 @@ __device__ __forceinline__ void oaken_work(const QuantArgs& a, int lane, const O
   const int li = lane % kBulkLanes, ri = lane / kBulkLanes;
   const bool in = c.p.t < a.n_new;
   // the unit's plane parameters in registers (one side per unit)
-  const OakUnitParams p = oaken_unit_params(c.p.side ? a.v_oaken : a.k_oaken);
+  const OakUnitParams p = oaken_unit_params<BF>(c.p.side ? a.v_oaken : a.k_oaken);
+  using IP = InPair<BF>;
   uint4 raw[kBulkNV / 8];
 #pragma unroll
   for (int k = 0; k < kBulkNV / 8; ++k)
@@ -184,10 +205,15 @@ __device__ __forceinline__ void oaken_work(const QuantArgs& a, int lane, const O
   uint32_t omask = 0;
 #pragma unroll
   for (int i = 0; i < kBulkNV / 2; ++i) {
-    const __half2 h = u32_as_h2(w[i]);
-    const __half2 cl = __hmin2(__hmax2(h, u32_as_h2(p.tl2)), u32_as_h2(p.th2));
-    omask |= __hne2_mask(cl, h) & (0x00010001u << i);
-    const float2 f = __half22float2(cl);
+    const uint32_t cl = IP::min2(IP::max2(w[i], p.tl2), p.th2);
+    uint32_t ne;
+    if constexpr (BF)
+      ne = __hne2_mask(*reinterpret_cast<const __nv_bfloat162*>(&cl),
+                       *reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    else
+      ne = __hne2_mask(u32_as_h2(cl), u32_as_h2(w[i]));
+    omask |= ne & (0x00010001u << i);
+    const float2 f = IP::widen(cl);
     x[2 * i] = f.x;
     x[2 * i + 1] = f.y;
   }
@@ -249,8 +275,8 @@ __device__ __forceinline__ void oaken_work(const QuantArgs& a, int lane, const O
   for (int e = lane; e < total; e += 32) {
     const uint32_t en = olist[e];
     const int r = en & 7, k = (en >> 3) & 31, dim = (int)(en >> 8);
-    const float v = __half2float(
-        *reinterpret_cast<const __half*>(slot + bulk_slot_off(r, dim >> 3) + (dim & 7) * 2));
+    const float v = in_f32<BF>(
+        *reinterpret_cast<const uint16_t*>(slot + bulk_slot_off(r, dim >> 3) + (dim & 7) * 2));
     const bool hi = v > p.t_hi;
     const float mq = fminf(rintf(__fdiv_rn(hi ? v - p.t_hi : -(v - p.t_lo), p.s_out)), p.m_max);
     const int d = hi ? (int)mq : -(int)mq;
@@ -264,6 +290,7 @@ __device__ __forceinline__ void oaken_work(const QuantArgs& a, int lane, const O
   __syncwarp();  // the slot rows and the list are rewritten by the next unit
 }
 
+template <bool BF>
 __global__ void __launch_bounds__(kBulkWarps * 32) oaken_bulk_kernel(const QuantArgs a,
                                                                      int units_per_row,
                                                                      int n_units,
@@ -276,7 +303,7 @@ __global__ void __launch_bounds__(kBulkWarps * 32) oaken_bulk_kernel(const Quant
   bulk_loop<OakDst>(a, units_per_row, n_units, units_per_warp, &ring[warp][0][0],
                     [&](const OakDst& c, const uint32_t (&roff)[kBulkNV / 8],
                         const uint8_t* slot) {
-                      oaken_work(a, lane, c, roff, slot, &sbuf[warp][0][0], &olist[warp][0]);
+                      oaken_work<BF>(a, lane, c, roff, slot, &sbuf[warp][0][0], &olist[warp][0]);
                     });
 }
 
@@ -300,7 +327,10 @@ OakenParams make_oaken_params(float s_in, int z_in, float s_out, int outer_bits)
   return p;
 }
 
-cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s) {
+namespace {
+
+template <bool BF>
+cudaError_t launch_oaken(const QuantArgs& a, cudaStream_t s) {
   cudaError_t e;
   if (a.n_new < kUnitRows) {
     // a few rows per sequence (the decode-step append): half a warp per row
@@ -308,25 +338,32 @@ cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s) {
     const long long blocks = (rows + 15) / 16;
     const long long cap = (long long)device_sm_count() * 8;
     const unsigned grid = (unsigned)(blocks < cap ? blocks : cap);
-    oaken_quantize_kernel<<<grid, 256, 0, s>>>(a);
+    oaken_quantize_kernel<BF><<<grid, 256, 0, s>>>(a);
   } else {
     static int per_sm = 0;  // resident CTAs per SM of the bulk kernel
     if (per_sm == 0) {
       int r = 0;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, oaken_bulk_kernel, kBulkWarps * 32, 0);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&r, oaken_bulk_kernel<BF>,
+                                                        kBulkWarps * 32, 0);
       if (e != cudaSuccess) return e;
       per_sm = r > 0 ? r : 1;
     }
     BulkShape sh;
     if (!bulk_shape(a, per_sm, &sh)) return cudaErrorInvalidValue;
-    oaken_bulk_kernel<<<sh.blocks, kBulkWarps * 32, 0, s>>>(a, sh.units_per_row, sh.n_units,
-                                                            sh.per_warp);
+    oaken_bulk_kernel<BF><<<sh.blocks, kBulkWarps * 32, 0, s>>>(a, sh.units_per_row, sh.n_units,
+                                                                sh.per_warp);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess || !a.advance) return e;
   // a programmatic dependent: scheduled while the quantizer runs
   return launch_dependent(oaken_advance_kernel, dim3((a.batch + 127) / 128), dim3(128), s,
                           a.seq_lens, a.batch, a.n_new, a.max_tokens);
+}
+
+}  // namespace
+
+cudaError_t launch_oaken_quantize(const QuantArgs& a, cudaStream_t s) {
+  return a.in_bf16 ? launch_oaken<true>(a, s) : launch_oaken<false>(a, s);
 }
 
 }  // namespace kvq

@@ -136,10 +136,10 @@ def test_quantize_append_rejects_bad_arguments(kvq):
 
 
 def test_quantize_append_kv_dtype(kvq):
-    """kv_dtype is KVQ_F16 or KVQ_BF16; bf16 input is refused for Oaken planes
-    only (a per-channel K plane takes it, and goes on to its block check); the
-    binding passes the tensors' dtype and refuses mixed or other dtypes before
-    calling."""
+    """kv_dtype is KVQ_F16 or KVQ_BF16, taken by every format (a per-channel K
+    plane goes on to its block check, an Oaken plane to its capacity check
+    exactly as with fp16); the binding passes the tensors' dtype and refuses
+    mixed or other dtypes before calling.  No call here reaches a launch."""
     import torch
     fake = ctypes.c_void_p(0x60000)
 
@@ -156,7 +156,8 @@ def test_quantize_append_kv_dtype(kvq):
     c.k.fmt = c.v.fmt = kvq.KVQ_FMT_OAKEN
     c.k.oaken = kvq.kvq_oaken(0.25, 8, 0.5, 5)
     c.v.oaken = kvq.kvq_oaken(0.125, 3, 0.05, 7)
-    assert st(c, kvq.KVQ_BF16) == kvq.KVQ_ERR_UNSUPPORTED
+    big = c.max_tokens + 1
+    assert st(c, kvq.KVQ_BF16, n=big) == st(c, kvq.KVQ_F16, n=big) == kvq.KVQ_ERR_CAPACITY
 
     class T:
         def __init__(self, dtype):

@@ -2,7 +2,7 @@
 实践" page, sections 3.1, 3.2.1, 3.2.2; the oracle's reading R18): codes and
 outlier slots written by kvq_quantize_append byte for byte equal to the
 oracle's (ragged starts, the capacity edge, thresholds, ties, rows with more
-outliers than slots); decode attention over them within the attention
+outliers than slots, bf16 rows); decode attention over them within the attention
 tolerance of the fp64 oracle (g = 1, 2, 4, 8; ragged, empty and one-token
 lengths; bf16 queries; several split counts; rising scores); the decode
 step (append, then attention); and the full-size workload in the
@@ -232,3 +232,40 @@ def test_full_size_sampled(kvq):
         lref[b, h * g:(h + 1) * g] = lr[0]
         mask[b, h * g:(h + 1) * g] = True
     assert_close(out, ref, lse, lref, mask=mask, what="llama3_8b_gqa_oaken")
+
+
+@pytest.mark.parametrize("n_new", [3, 160])
+def test_bf16_quantize_bit_exact(kvq, n_new):
+    """bf16 K/V (reading R19) through the append kernel (3 tokens) and the
+    bulk kernel (160), against the oracle's bf16 path: the workload's rows,
+    the hand-worked bf16 row of tests/golden (outliers beyond the fp16 range,
+    values on the thresholds, halfway magnitudes) and a row of values far
+    beyond fp16, byte for byte in codes and slots."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                                    "oaken_bf16_worked_example.json")))
+    params = (g["s_in"], g["z_in"], g["s_out"], g["outer_bits"])
+    B, H = 2, 4
+    wl = WL.scaled(batch=B, kv_heads=H, q_heads=H)
+    k, v = workloads.kv_tokens(wl, n_new, DEV, dtype=torch.bfloat16)
+    k[1, 2, 1, :8] = torch.tensor(g["values"], dtype=torch.float32).to(torch.bfloat16).to(DEV)
+    v[0, 1, 0] = (torch.randn(128, device=DEV) * 1e6).to(torch.bfloat16)
+    c = _alloc(kvq, B, H, 256, kp=params, vp=params)
+    start = [0, 37]
+    c.seq_lens.copy_(torch.tensor(start, dtype=torch.int32))
+    kvq.kvq_quantize_append(c, k, v, n_new, advance_seq_lens=True)
+    assert c.seq_lens.tolist() == [s + n_new for s in start]
+
+    def b16(t):
+        return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    kc, ks = oracle.oaken_quantize_cache(b16(k), params, in_dtype="bf16")
+    vc, vs = oracle.oaken_quantize_cache(b16(v), params, in_dtype="bf16")
+    assert ks[1, 2, 1, :5].tolist() == [int(h, 16) for h in g["slots"]]
+    for b, st in enumerate(start):
+        p = slice(st, st + n_new)
+        assert np.array_equal(c.k_codes[b, :, p].cpu().numpy(), kc[b]), b
+        assert np.array_equal(c.v_codes[b, :, p].cpu().numpy(), vc[b]), b
+        assert np.array_equal(c.k_meta[b, :, p].cpu().numpy().view(np.uint16), ks[b]), b
+        assert np.array_equal(c.v_meta[b, :, p].cpu().numpy().view(np.uint16), vs[b]), b
+        assert (c.k_codes[b, :, :st] == 0xA5).all() and (c.v_codes[b, :, st + n_new:] == 0x5A).all()
