@@ -41,6 +41,8 @@ FMT_NAME = {"fp8": "fp8 e4m3", "sym8": "symmetric int8", "e5m2": "fp8 e5m2",
 FMT_CODE = {"int": 0, "fp8": 1, "sym8": 2, "e5m2": 3, "oaken": 4}
 OAKEN_SLOTS = 16
 NOMINAL_HBM_GBS = 8000.0
+# one graph in this many carries the event nodes that time the split-K kernel
+INSTR_EVERY = 10
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -682,14 +684,17 @@ def run_kvq(args, wl, rank, world, local_rank):
     # ---- every episode position as one CUDA graph (reset at the start of an
     # episode, split-K partials, merge), so the timed loop is paced by the
     # device and the merge is a programmatic dependent of the split-K kernel
-    # inside the graph.  Event-record nodes inside each graph bracket the
-    # split-K launch; after the loop each pair holds the time of its graph's
-    # last replay (the last `episode` steps of the timed region).
+    # inside the graph.  In every INSTR_EVERY-th position's graph, event-record
+    # nodes bracket the split-K launch; after the loop each pair holds the
+    # time of its graph's last replay.  The other graphs carry no timing
+    # nodes, so most timed steps run as a caller's would.
     from cuda.bindings import runtime as cudart
 
-    split_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(episode)]
-    for e0, e1 in split_evs:  # create the events before the capture
+    # instrumented positions, the first timed step's among them
+    instr = [e for e in range(episode) if (e - args.warmup) % INSTR_EVERY == 0]
+    split_evs = {e: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for e in instr}
+    for e0, e1 in split_evs.values():  # create the events before the capture
         e0.record(stream)
         e1.record(stream)
     torch.cuda.synchronize()
@@ -711,16 +716,20 @@ def run_kvq(args, wl, rank, world, local_rank):
             g.capture_begin()
             if wl.append and e == 0:
                 reset_fn(e)
-            record_in_graph(split_evs[e][0], cap)
-            partials_fn(e)
-            # the end event hangs off the split-K node on a branch, so the
-            # merge still follows that node directly (programmatic edge)
-            fork.record(cap)
-            side.wait_event(fork)
-            record_in_graph(split_evs[e][1], side)
-            join.record(side)
-            merge_fn(e)
-            cap.wait_event(join)
+            if e in split_evs:
+                record_in_graph(split_evs[e][0], cap)
+                partials_fn(e)
+                # the end event hangs off the split-K node on a branch, so the
+                # merge still follows that node directly (programmatic edge)
+                fork.record(cap)
+                side.wait_event(fork)
+                record_in_graph(split_evs[e][1], side)
+                join.record(side)
+                merge_fn(e)
+                cap.wait_event(join)
+            else:
+                partials_fn(e)
+                merge_fn(e)
             g.capture_end()
             graphs.append(g)
     stream.wait_stream(cap)
@@ -769,8 +778,10 @@ def run_kvq(args, wl, rank, world, local_rank):
     h1 = time.time()
     ms = (sum(a.elapsed_time(b) for a, b in step_evs) if flush_l2
           else t_start.elapsed_time(t_end))
-    # the split-K time of each graph's last replay in the timed region
-    last_step = {(args.warmup + i) % episode: args.warmup + i for i in range(args.steps)}
+    # the split-K time of each instrumented graph's last replay in the timed
+    # region
+    last_step = {(args.warmup + i) % episode: args.warmup + i for i in range(args.steps)
+                 if (args.warmup + i) % episode in split_evs}
     split_us = {e: split_evs[e][0].elapsed_time(split_evs[e][1]) * 1e3 for e in last_step}
     assert kvq.workspace_error_word(ws) == 0, "device wait gave up (error word set)"
     if world > 1:
@@ -884,7 +895,8 @@ def run_kvq(args, wl, rank, world, local_rank):
                       + ("(split-K kernel, then the merge as a programmatic dependent); "
                          if parts > 1 else
                          "(one split: the attention kernel writes the output, no merge); ")
-                      + "event-record nodes in the graph time the split-K launch",
+                      + f"event-record nodes in one graph of every {INSTR_EVERY} time the split-K "
+                      "launch",
             "l2": (f"L2 flushed before every step ({sum(kv_bytes) / args.steps / 1e3:.0f} KB "
                    f"of packed K/V per step, L2 {l2_bytes / 1e6:.0f} MB): a write of twice the "
                    "L2 size outside each step's events; ms_per_step sums the steps' event times"
