@@ -299,9 +299,10 @@ kvq_status kvq_decode_workspace_bytes(const kvq_cache *segs, int32_t n_segs,
  * The call is one split-K kernel launch per segment, then one merge kernel
  * when the plan has more than one partial.
  * Supported: head_dim 128; g in 1..8; bits 2/4/8 with G 32/64/128, and bits
- * 16 with fp16 q; KVQ_FMT_OAKEN segments with g = 1, 2, 4 or 8 (their own
- * split-K kernel, the codes' dense part plus the outlier slots).  Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED,
- * KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA.
+ * 16 with fp16 q; KVQ_FMT_OAKEN segments with g = 1, 2, 4 or 8 (the dense
+ * codes through the tensor cores like INT4, plus the outlier slots).
+ * Errors: KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE,
+ * KVQ_ERR_CUDA.
  */
 kvq_status kvq_decode_attention(const kvq_cache *segs, int32_t n_segs,
                                 const void *q, kvq_dtype q_dtype,
