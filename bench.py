@@ -219,7 +219,8 @@ def segment_oracle_pairs(wl, k, v, q, pairs):
 def run_reference(args, wl):
     """The CPU oracle as it stands, on this host's cores (one thread per
     core): each step attends one (sequence, KV head) of the workload after
-    appending one token."""
+    appending one token (attention alone for a workload without an
+    append, as its GPU step)."""
     import numpy as np
     import torch
 
@@ -281,6 +282,10 @@ def run_reference(args, wl):
 
     def step(i):
         kc, km, vc, vm, qh, knew, vnew = prepared[i % len(prepared)]
+        if not wl.append:  # the step is the attention over the prefilled cache
+            oracle.attention_packed(qh, wl.q_dtype == "bf16", kc, km, wl.bits, vc, vm, wl.bits,
+                                    wl.group, L, 128 ** -0.5, wl.fmt)
+            return
         ck, mk = oracle.quantize_rows(knew, wl.group, wl.bits, wl.fmt)
         cv, mv = oracle.quantize_rows(vnew, wl.group, wl.bits, wl.fmt)
         kc2 = np.concatenate([kc, ck])
@@ -294,9 +299,10 @@ def run_reference(args, wl):
         step(i)
     el = run_steps_parallel(step, args.steps)
     value = args.steps / wl.kv_heads / el
-    sample = (f"each step: one (sequence, KV head) of {wl.name} at {L + 1} tokens "
-              f"(append 1 token + attention of {g} query heads); tokens/s = steps / kv_heads "
-              f"({wl.kv_heads}) / seconds")
+    what = (f"at {L + 1} tokens (append 1 token + attention of {g} query heads)" if wl.append
+            else f"at {L} tokens (attention of {g} query heads, no append)")
+    sample = (f"each step: one (sequence, KV head) of {wl.name} {what}; tokens/s = steps / "
+              f"kv_heads ({wl.kv_heads}) / seconds")
     print(json.dumps(reference_line(args, wl, value, el, sample)), flush=True)
 
 
@@ -393,7 +399,8 @@ def oracle_baseline(wl, jobs, seconds: float, what: str):
 
 def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
     """The oracle (C, fp64 attention) on a bounded sample of the same inputs:
-    (sequence, KV head) pairs, each one append + attention."""
+    (sequence, KV head) pairs, each one append + attention (kn, vn: the new
+    token's rows), or attention alone for a workload without an append."""
     import numpy as np
     import torch
 
@@ -418,6 +425,12 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
         kc, km = oracle.quantize_rows(kk, wl.group, wl.bits, wl.fmt)
         vc, vm = oracle.quantize_rows(vv, wl.group, wl.bits, wl.fmt)
         qh = q[b, h * g:(h + 1) * g].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        if kn is None:  # no append: attention over the prefilled tokens
+            def job(kc=kc, km=km, vc=vc, vm=vm, qh=qh):
+                oracle.attention_packed(qh, wl.q_dtype == "bf16", kc, km, wl.bits, vc, vm,
+                                        wl.bits, wl.group, L, 128 ** -0.5, fmt=wl.fmt)
+            jobs.append(job)
+            continue
         knew = kn[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
         vnew = vn[b, h].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
@@ -429,8 +442,9 @@ def cpu_baseline(wl, k, v, kn, vn, q, seconds: float):
                                     np.concatenate([vc, cv]), np.concatenate([vm, mv]),
                                     wl.bits, wl.group, L + 1, 128 ** -0.5, fmt=wl.fmt)
         jobs.append(job)
-    return oracle_baseline(wl, jobs, seconds,
-                           f"decode steps (append + attention) of {wl.name} at {L + 1} tokens")
+    what = (f"decode steps (append + attention) of {wl.name} at {L + 1} tokens" if kn is not None
+            else f"attentions of {wl.name} over {L} tokens")
+    return oracle_baseline(wl, jobs, seconds, what)
 
 
 def prepare_mixed_oracle(wl, k, v, q, wlr):
@@ -690,8 +704,10 @@ def run_kvq(args, wl, rank, world, local_rank):
     # nodes, so most timed steps run as a caller's would.
     from cuda.bindings import runtime as cudart
 
-    # instrumented positions, the first timed step's among them
-    instr = [e for e in range(episode) if (e - args.warmup) % INSTR_EVERY == 0]
+    # instrumented positions: those of timed steps 0, INSTR_EVERY, 2 INSTR_EVERY,
+    # ... within the first episode (the first timed step's always among them)
+    instr = sorted({(args.warmup + i) % episode
+                    for i in range(0, min(args.steps, episode), INSTR_EVERY)})
     split_evs = {e: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                  for e in instr}
     for e0, e1 in split_evs.values():  # create the events before the capture
