@@ -426,6 +426,10 @@ kvq_status decode_stages(const kvq_cache* segs, int32_t n_segs, const void* q,
     }
     v.part_base = base;
     base += plan.n_split[i];
+    // each segment its own work counters, so that the segments' kernels may
+    // run side by side: the later ones are programmatic dependents
+    v.ctr = 1 + 2 * i;
+    v.after_prev = i > 0;
     if ((stages & kPartials) && kvq::launch_decode_segment(a, v, s) != cudaSuccess)
       return KVQ_ERR_CUDA;
   }

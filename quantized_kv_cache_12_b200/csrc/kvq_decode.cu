@@ -110,7 +110,7 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   int* unit_sm = reinterpret_cast<int*>(smem + C::HDR_MISC);
   int* fail_sm = unit_sm + 1;
   int* qexp_sm = unit_sm + 8;  // [8] power-of-two shift of each staged query row
-  uint32_t* counters = a.err + 1;  // [0] next unit, [1] CTAs done
+  uint32_t* counters = a.err + seg.ctr;  // [0] next unit, [1] CTAs done
 
   const uint64_t policy = l2_evict_first_policy();
   // the stage ring (position and mbarrier phase) runs on across units
@@ -535,6 +535,7 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
   }  // unit loop
 
   if (t == 0) release_counters(counters);
+  grid_dependency_wait();  // after the previous segment's kernel (see decode_tm_kernel)
 }
 
 // Merge the partial (m, l, o) of every split and segment (log-sum-exp).
@@ -627,8 +628,8 @@ cudaError_t launch_split_g(const DecodeArgs& a, const SegView& seg, cudaStream_t
   const long long units = (long long)seg.n_split * a.kv_heads * a.batch;
   const long long slots = (long long)seg.sms * C::MIN_CTAS;  // one wave of persistent CTAs
   const unsigned grid = (unsigned)(units < slots ? units : slots);
-  decode_split_kernel<BITS, GE, GR><<<grid, kWarps * 32, C::SMEM, s>>>(P);
-  return cudaGetLastError();
+  return launch_segment_kernel(decode_split_kernel<BITS, GE, GR>, grid, kWarps * 32, C::SMEM, s,
+                               seg.after_prev != 0, P);
 }
 
 }  // namespace

@@ -225,7 +225,7 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   uint8_t* new_sm = smem + C::HDR_NEW;
   uint2* qf_sm = reinterpret_cast<uint2*>(smem + C::HDR_QF);     // [8 ks][32 lanes]
   uint8_t* stages = smem + C::HDR_BYTES + warp * C::STAGES * C::STAGE;
-  uint32_t* counters = a.err + 1;  // [0] next unit, [1] CTAs done
+  uint32_t* counters = a.err + seg.ctr;  // [0] next unit, [1] CTAs done
 
   // ---- per-lane constants
   // QK B column gid: head (gid / CPH) mod g, group gid mod NG; the lane's K
@@ -982,6 +982,9 @@ decode_tm_kernel(const __grid_constant__ SplitParams P) {
   }  // unit loop
 
   if (t == 0) release_counters(counters);
+  // after the previous segment's kernel (a no-op for a plain launch): the
+  // merge after the last segment then sees every segment done
+  grid_dependency_wait();
 }
 
 template <int BITS, int GE, int GR, bool KPC>
@@ -1003,8 +1006,8 @@ cudaError_t launch_tm(const DecodeArgs& a, const SegView& seg, cudaStream_t s) {
   const long long units = (long long)seg.n_split * a.kv_heads * a.batch;
   const long long slots = (long long)seg.sms * C::MIN_CTAS;  // one wave of persistent CTAs
   const unsigned grid = (unsigned)(units < slots ? units : slots);
-  decode_tm_kernel<BITS, GE, GR, KPC><<<grid, kWarps * 32, C::SMEM, s>>>(P);
-  return cudaGetLastError();
+  return launch_segment_kernel(decode_tm_kernel<BITS, GE, GR, KPC>, grid, kWarps * 32, C::SMEM, s,
+                               seg.after_prev != 0, P);
 }
 
 // Per-channel K (G is V's group size): the (bits, G, g) whose QK columns

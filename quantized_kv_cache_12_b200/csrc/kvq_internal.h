@@ -44,7 +44,36 @@ struct SegView {
   int32_t k_channels;    // K grouped per channel over kChannelBlock-token blocks
   int32_t sms;           // streaming multiprocessors of the device
   OakenParams k_oaken, v_oaken;  // bits == kOaken: the planes' parameters
+  // this segment's pair of work counters (next unit, CTAs done) in the
+  // workspace header: words ctr, ctr + 1 after the error word at word 0
+  int32_t ctr;
+  // launched as a programmatic dependent of the previous segment's kernel
+  // (several segments in one call): its CTAs may run beside that kernel's,
+  // and it waits for that kernel before it exits
+  int32_t after_prev;
 };
+
+// Launch a split-K decode kernel: a plain launch, or (after_prev) a
+// programmatic dependent of the kernel before it on the stream.
+template <class Kernel, class Params>
+inline cudaError_t launch_segment_kernel(Kernel kernel, unsigned grid, unsigned block, size_t smem,
+                                         cudaStream_t s, bool after_prev, const Params& p) {
+  if (!after_prev) {
+    kernel<<<grid, block, smem, s>>>(p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
 
 // warps of a decode CTA
 constexpr int kWarpsPerCta = 4;
