@@ -542,8 +542,10 @@ decode_split_kernel(const __grid_constant__ SplitParams P) {
 // One CTA of 128 x PG threads per (sequence, query head): all threads
 // reduce the max and the weights over the partials together; thread
 // (group j, dim d) then sums dim d over the partials j, j + PG, j + 2 PG, ...
-// with four independent sums (several loads in flight), and group 0 adds the
-// groups' sums.  It is launched as a programmatic dependent of the split-K
+// eight loads in flight at a time, and group 0 adds the groups' sums.  At
+// 512 threads of 32 registers a CTA still fits on an SM beside three CTAs
+// of the split kernel, so it can be resident before they end (a
+// 1024-thread CTA cannot, and measured slower).  It is launched as a programmatic dependent of the split-K
 // kernels: the launch overlaps their tail, and griddepcontrol.wait holds
 // every thread until they have completed and their stores are visible.
 template <int PG>
@@ -586,16 +588,20 @@ __global__ void __launch_bounds__(kHeadDim * PG) decode_merge_kernel(const Decod
   // every partial's o is finite (a split with no tokens stores 0), so a
   // weight of 0 contributes exactly nothing; the loads stay independent of
   // the weights
-  float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
-  int p = grp;
-  for (; p + 3 * PG < P; p += 4 * PG) {
-    O0 = fmaf(w_sm[p], po[(long long)p * kHeadDim + d], O0);
-    O1 = fmaf(w_sm[p + PG], po[(long long)(p + PG) * kHeadDim + d], O1);
-    O2 = fmaf(w_sm[p + 2 * PG], po[(long long)(p + 2 * PG) * kHeadDim + d], O2);
-    O3 = fmaf(w_sm[p + 3 * PG], po[(long long)(p + 3 * PG) * kHeadDim + d], O3);
+  // the thread's partials grp, grp + PG, ... eight at a time, all eight
+  // loads issued before the first is used
+  float O = 0.f;
+  for (int p0 = grp; p0 < P; p0 += 8 * PG) {
+    float v[8], wv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int p = p0 + j * PG;
+      v[j] = p < P ? po[(long long)p * kHeadDim + d] : 0.f;
+      wv[j] = p < P ? w_sm[p] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) O = fmaf(wv[j], v[j], O);
   }
-  for (; p < P; p += PG) O0 = fmaf(w_sm[p], po[(long long)p * kHeadDim + d], O0);
-  float O = (O0 + O1) + (O2 + O3);
   if constexpr (PG > 1) {
     float* osm = w_sm + P;
     osm[grp * kHeadDim + d] = O;
